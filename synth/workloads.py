@@ -1,0 +1,166 @@
+"""The five synthetic MoE-layer workloads and how their inputs are drawn.
+
+Shapes, distributions and routing parameters follow the workload list of the
+project (tiny, DeepSeek-V3.2-shaped decode, Kimi-K2-shaped prefill, Kimi-K3-
+shaped latent decode, skewed Kimi-K2 stress).  Every tensor comes from the
+counter-based generator in ``synth.h`` with its own tensor id, so any slice can
+be regenerated on either side.
+
+Recipe (seed 0 unless stated):
+  x    [N, d_r]  bf16  ~ N(0, 1)          tensor id 1 (rank r uses rows r*N .. r*N+N-1)
+  W    [E, d_r]  fp32  ~ N(0, 0.02)       tensor id 2
+  b    [E]       fp32  ~ U(-0.01, 0.01)   tensor id 3 (skewed workload: calibrated file)
+  w1   [E, F, d_e] bf16 ~ N(0, 0.02)      tensor id 4
+  w3   [E, F, d_e] bf16 ~ N(0, 0.02)      tensor id 5
+  w2   [E, d_e, F] bf16 ~ N(0, 0.02)      tensor id 6
+  x_e  [N, d_e]  bf16  ~ N(0, 1)          tensor id 7 (latent workload only; else x_e = x)
+"""
+from __future__ import annotations
+
+import os
+from dataclasses import dataclass, asdict
+
+import numpy as np
+
+TID_X, TID_W, TID_BIAS, TID_W1, TID_W3, TID_W2, TID_XE, TID_POP = 1, 2, 3, 4, 5, 6, 7, 8
+
+SIGMA_X = 1.0
+SIGMA_W = 0.02
+SIGMA_EXPERT = 0.02
+BIAS_LO, BIAS_HI = -0.01, 0.01
+
+_REPO = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+SKEW_BIAS_FILE = os.path.join(_REPO, "tests", "golden", "k2_skew_bias.txt")
+
+
+@dataclass(frozen=True)
+class Workload:
+    name: str
+    N: int
+    d_r: int
+    d_e: int
+    E: int
+    G: int
+    TG: int
+    K: int
+    F: int
+    act: str            # "silu" or "situ"
+    route_scale: float
+    beta: float = 1.0   # SiTU beta
+    lbeta: float = 0.0  # SiTU linear_beta; 0 means "not set"
+    norm: bool = True   # norm_topk_prob
+    latent: bool = False
+    skew: bool = False
+    seed: int = 0
+
+    @property
+    def S(self) -> int:
+        return self.N * self.K
+
+    def as_dict(self) -> dict:
+        return asdict(self)
+
+
+WORKLOADS = {
+    "tiny": Workload("tiny", N=64, d_r=256, d_e=256, E=16, G=4, TG=2, K=4, F=128,
+                     act="silu", route_scale=2.5),
+    "dsv32_decode": Workload("dsv32_decode", N=128, d_r=7168, d_e=7168, E=256, G=8, TG=4, K=8,
+                             F=2048, act="silu", route_scale=2.5),
+    "k2_prefill": Workload("k2_prefill", N=4096, d_r=7168, d_e=7168, E=384, G=1, TG=1, K=8,
+                           F=2048, act="silu", route_scale=2.827),
+    "k3_latent_decode": Workload("k3_latent_decode", N=64, d_r=7168, d_e=2048, E=896, G=1, TG=1,
+                                 K=8, F=3072, act="situ", route_scale=2.827, beta=4.0, lbeta=8.0,
+                                 latent=True),
+    "k2_skew": Workload("k2_skew", N=16384, d_r=7168, d_e=7168, E=384, G=1, TG=1, K=8, F=2048,
+                        act="silu", route_scale=2.827, skew=True),
+}
+
+
+def get_workload(name: str) -> Workload:
+    return WORKLOADS[name]
+
+
+def scaled(wl: Workload, **kw) -> Workload:
+    """A copy of a workload with some fields replaced (e.g. fewer tokens)."""
+    d = wl.as_dict()
+    d.update(kw)
+    return Workload(**d)
+
+
+# ------------------------------------------------------------------ host side
+def skew_bias() -> np.ndarray:
+    """Calibrated correction bias of the skewed workload (384 fp32 values)."""
+    vals = []
+    with open(SKEW_BIAS_FILE) as f:
+        for line in f:
+            line = line.strip()
+            if line and not line.startswith("#"):
+                vals.append(float.fromhex(line))
+    return np.asarray(vals, dtype=np.float32)
+
+
+def host_inputs(wl: Workload, rank: int = 0) -> dict:
+    """Router-side inputs and x_e on the host (expert weights: ``host_expert``)."""
+    from . import host_normal_bf16, host_normal_f32, host_uniform_f32
+    x = host_normal_bf16(wl.seed, TID_X, (wl.N, wl.d_r), SIGMA_X, start=rank * wl.N * wl.d_r)
+    W = host_normal_f32(wl.seed, TID_W, (wl.E, wl.d_r), SIGMA_W)
+    if wl.skew:
+        b = skew_bias()
+        assert b.shape == (wl.E,)
+    else:
+        b = host_uniform_f32(wl.seed, TID_BIAS, (wl.E,), BIAS_LO, BIAS_HI)
+    if wl.latent:
+        xe = host_normal_bf16(wl.seed, TID_XE, (wl.N, wl.d_e), SIGMA_X, start=rank * wl.N * wl.d_e)
+    else:
+        xe = x
+    return {"x": x, "W": W, "bias": b, "x_e": xe}
+
+
+def host_expert(wl: Workload, e: int):
+    """(w1 [F, d_e], w3 [F, d_e], w2 [d_e, F]) of expert e as bf16 bit patterns."""
+    from . import host_normal_bf16
+    n = wl.F * wl.d_e
+    w1 = host_normal_bf16(wl.seed, TID_W1, (wl.F, wl.d_e), SIGMA_EXPERT, start=e * n)
+    w3 = host_normal_bf16(wl.seed, TID_W3, (wl.F, wl.d_e), SIGMA_EXPERT, start=e * n)
+    w2 = host_normal_bf16(wl.seed, TID_W2, (wl.d_e, wl.F), SIGMA_EXPERT, start=e * n)
+    return w1, w3, w2
+
+
+def host_experts_all(wl: Workload):
+    """All experts stacked: w1, w3 [E, F, d_e], w2 [E, d_e, F] (small workloads only)."""
+    from . import host_normal_bf16
+    w1 = host_normal_bf16(wl.seed, TID_W1, (wl.E, wl.F, wl.d_e), SIGMA_EXPERT)
+    w3 = host_normal_bf16(wl.seed, TID_W3, (wl.E, wl.F, wl.d_e), SIGMA_EXPERT)
+    w2 = host_normal_bf16(wl.seed, TID_W2, (wl.E, wl.d_e, wl.F), SIGMA_EXPERT)
+    return w1, w3, w2
+
+
+# ---------------------------------------------------------------- device side
+def dev_inputs(wl: Workload, rank: int = 0, device="cuda", experts: bool = True) -> dict:
+    """All inputs as torch CUDA tensors, drawn by the device twin."""
+    import torch
+    from . import dev_normal_bf16, dev_normal_f32, dev_uniform_f32
+    bf, f32 = torch.bfloat16, torch.float32
+    x = dev_normal_bf16(torch.empty((wl.N, wl.d_r), dtype=bf, device=device), wl.seed, TID_X,
+                        SIGMA_X, start=rank * wl.N * wl.d_r)
+    W = dev_normal_f32(torch.empty((wl.E, wl.d_r), dtype=f32, device=device), wl.seed, TID_W,
+                       SIGMA_W)
+    if wl.skew:
+        b = torch.from_numpy(skew_bias()).to(device)
+    else:
+        b = dev_uniform_f32(torch.empty((wl.E,), dtype=f32, device=device), wl.seed, TID_BIAS,
+                            BIAS_LO, BIAS_HI)
+    if wl.latent:
+        xe = dev_normal_bf16(torch.empty((wl.N, wl.d_e), dtype=bf, device=device), wl.seed,
+                             TID_XE, SIGMA_X, start=rank * wl.N * wl.d_e)
+    else:
+        xe = x
+    out = {"x": x, "W": W, "bias": b, "x_e": xe}
+    if experts:
+        out["w1"] = dev_normal_bf16(torch.empty((wl.E, wl.F, wl.d_e), dtype=bf, device=device),
+                                    wl.seed, TID_W1, SIGMA_EXPERT)
+        out["w3"] = dev_normal_bf16(torch.empty((wl.E, wl.F, wl.d_e), dtype=bf, device=device),
+                                    wl.seed, TID_W3, SIGMA_EXPERT)
+        out["w2"] = dev_normal_bf16(torch.empty((wl.E, wl.d_e, wl.F), dtype=bf, device=device),
+                                    wl.seed, TID_W2, SIGMA_EXPERT)
+    return out
