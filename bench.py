@@ -1,0 +1,378 @@
+"""Benchmark of the routed MoE layer (route + dispatch + expert MLP + combine).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+One step = one moe_forward over one batch of the workload (default: the
+DeepSeek-V3.2-shaped decode batch, N=128 tokens, d=7168, 256 experts, top-8,
+d_ff=2048).  Inputs are seeded and synthetic, drawn on the device; the
+expert weights (22.5 GB) are larger than L2 and L2 is also flushed (256 MB
+write) between steps, outside the per-step events.  Under torchrun every rank
+runs its own batch (token rows rank*N .. rank*N+N-1) with the same weights:
+weak scaling with no collective on the data path; the step time is the max
+over ranks.  Rank 0 prints one JSON line.
+
+--impl reference times the CPU reference (oracle/) on the host cores on a
+bounded sample of the same workload; it is the slow reference arm, not a
+target.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "routed tokens/sec per MoE layer (route+dispatch+FFN+combine)"
+UNIT = "tokens/s"
+DEFAULT_WORKLOAD = "dsv32_decode"
+KERNELS_PER_STEP = 10  # gate_partial, select, hist, scan, scatter, gather, tiles, gate_up, down, combine
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=20)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    p.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    return p.parse_args()
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    """nvidia-smi sampling of SM clock and throttle reasons during a region."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        os.makedirs(os.path.join(ROOT, "gpurun_out"), exist_ok=True)
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_{os.getpid()}.csv")
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            time.sleep(0.2)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        if self.proc is None or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- our arm
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import moe_routing_expert_fp32_b200 as moe
+    import synth
+    from synth.workloads import WORKLOADS, dev_inputs
+
+    wl = WORKLOADS[args.workload]
+    torch.cuda.set_device(local_rank)
+    dev = dev_inputs(wl, rank=rank)
+    cfg = moe.RouteConfig(wl.E, wl.G, wl.TG, wl.K, wl.route_scale, wl.norm)
+    act = moe.ActConfig(wl.act, wl.beta, wl.lbeta)
+    x_e = dev["x_e"] if wl.latent else None
+    ws = moe.workspace(moe.workspace_size(wl.N, wl.d_r, wl.d_e, cfg, wl.F))
+    out = torch.empty((wl.N, wl.d_e), dtype=torch.bfloat16, device="cuda")
+    counts_probe = torch.empty((wl.N, wl.K), dtype=torch.int32, device="cuda")
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    names = ["after_route", "after_dispatch", "after_gate_up", "after_down", "after_combine"]
+
+    def step(events=None, idx=None):
+        moe.forward(dev["x"], dev["W"], dev["bias"], cfg, dev["w1"], dev["w3"], dev["w2"], act,
+                    x_e=x_e, ws=ws, out=out, topk_idx=idx, events=events)
+
+    torch.cuda.synchronize()
+    for _ in range(max(args.warmup, 3)):
+        flush.zero_()
+        step()
+    # per-step events: start + one per stage
+    ev = [{"start": torch.cuda.Event(enable_timing=True),
+           **{n: torch.cuda.Event(enable_timing=True) for n in names}} for _ in range(args.steps)]
+    for e in ev:  # create the CUDA events before handing their handles to the library
+        for v in e.values():
+            v.record()
+    torch.cuda.synchronize()
+
+    def barrier():
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+
+    with ClockSampler(local_rank) as clk:
+        barrier()
+        torch.cuda.synchronize()
+        t0 = time.perf_counter()
+        for i in range(args.steps):
+            flush.zero_()
+            ev[i]["start"].record()
+            step(events={n: ev[i][n] for n in names})
+        torch.cuda.synchronize()
+        barrier()
+        wall = time.perf_counter() - t0
+    step_ms = [e["start"].elapsed_time(e["after_combine"]) for e in ev]
+    stage_ms = {}
+    prev = "start"
+    for n in names:
+        stage_ms[n.replace("after_", "")] = statistics.mean(
+            e[prev].elapsed_time(e[n]) for e in ev)
+        prev = n
+    ms = statistics.mean(step_ms)
+
+    # routing statistics of the timed batch (for the algorithmic byte count)
+    step(idx=counts_probe)
+    torch.cuda.synchronize()
+    counts = np.bincount(counts_probe.cpu().numpy().ravel(), minlength=wl.E)
+    touched = int((counts > 0).sum())
+
+    # end to end through the public API from pinned host buffers
+    x_host = torch.empty((wl.N, wl.d_r), dtype=torch.bfloat16, pin_memory=True)
+    x_host.copy_(dev["x"].cpu())
+    xe_host = None
+    if wl.latent:
+        xe_host = torch.empty((wl.N, wl.d_e), dtype=torch.bfloat16, pin_memory=True)
+        xe_host.copy_(dev["x_e"].cpu())
+    out_host = torch.empty((wl.N, wl.d_e), dtype=torch.bfloat16, pin_memory=True)
+    x_dev = torch.empty_like(dev["x"])
+    xe_dev = torch.empty_like(dev["x_e"]) if wl.latent else None
+
+    def e2e_step():
+        x_dev.copy_(x_host, non_blocking=True)
+        if wl.latent:
+            xe_dev.copy_(xe_host, non_blocking=True)
+        moe.forward(x_dev, dev["W"], dev["bias"], cfg, dev["w1"], dev["w3"], dev["w2"], act,
+                    x_e=xe_dev, ws=ws, out=out)
+        out_host.copy_(out, non_blocking=True)
+
+    for _ in range(3):
+        flush.zero_()
+        e2e_step()
+    torch.cuda.synchronize()
+    e2e_ms = []
+    for _ in range(args.steps):
+        flush.zero_()
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record()
+        e2e_step()
+        e.record()
+        e.synchronize()
+        e2e_ms.append(s.elapsed_time(e))
+    h2d = wl.N * wl.d_r * 2 + (wl.N * wl.d_e * 2 if wl.latent else 0)
+    d2h = wl.N * wl.d_e * 2
+
+    # max over ranks
+    vals = torch.tensor([ms, statistics.mean(e2e_ms), stage_ms["gate_up"], wall],
+                        dtype=torch.float64, device="cuda")
+    if world > 1:
+        import torch.distributed as dist
+        dist.all_reduce(vals, op=dist.ReduceOp.MAX)
+    ms_max, e2e_max, gu_ms, wall_max = vals.tolist()
+
+    res = {
+        "ms": ms_max, "e2e_ms": e2e_max, "stage_ms": stage_ms, "gate_up_ms": gu_ms,
+        "touched": touched, "counts_max": int(counts.max()), "clocks": clk.summary(),
+        "h2d": h2d, "d2h": d2h, "wall_s": wall_max,
+    }
+    return wl, res
+
+
+def gate_up_bytes(wl, touched):
+    """Algorithmic HBM bytes of one w1/w3 launch: both weight matrices of every
+    touched expert, the gathered rows read, the h rows written."""
+    S = wl.N * wl.K
+    return touched * 2 * wl.F * wl.d_e * 2 + S * wl.d_e * 2 + S * wl.F * 2
+
+
+# ------------------------------------------------------------ oracle arm
+def oracle_sample(wl, n_experts=8):
+    """Time the CPU reference on a bounded sample of the workload.
+
+    Route, dispatch and combine run on the whole batch; the expert MLP runs on
+    the rows of the first `n_experts` experts that received rows and its time
+    is scaled by (all slots / sampled slots).  Returns tokens/s and details.
+    """
+    import oracle
+    import synth
+    from synth.workloads import host_inputs, host_expert
+
+    oracle.set_threads(os.cpu_count() or 1)
+    cores = oracle.max_threads()
+    inp = host_inputs(wl)
+    t = {}
+    t0 = time.perf_counter()
+    idx, w, _ = oracle.route(inp["x"], inp["W"], inp["bias"], wl.G, wl.TG, wl.K,
+                             wl.route_scale, wl.norm)
+    t["route"] = time.perf_counter() - t0
+    t0 = time.perf_counter()
+    counts, offsets, perm, pos = oracle.dispatch(idx, wl.E)
+    xs = oracle.gather(inp["x_e"], perm, wl.K)
+    t["dispatch"] = time.perf_counter() - t0
+    experts = [e for e in range(wl.E) if counts[e] > 0][:n_experts]
+    weights = {e: host_expert(wl, e) for e in experts}  # inputs, not timed
+    ys = np.zeros_like(xs)
+    t0 = time.perf_counter()
+    done = 0
+    for e in experts:
+        a, b = int(offsets[e]), int(offsets[e + 1])
+        ys[a:b] = oracle.expert_ffn(xs[a:b], *weights[e], wl.act, wl.beta, wl.lbeta)
+        done += b - a
+    t_ffn_sample = time.perf_counter() - t0
+    S = wl.N * wl.K
+    t["ffn"] = t_ffn_sample * S / max(done, 1)
+    t0 = time.perf_counter()
+    oracle.combine(ys, pos, w, wl.K)
+    t["combine"] = time.perf_counter() - t0
+    total = sum(t.values())
+    return {
+        "value": wl.N / total, "cores": cores, "seconds": t,
+        "sample": (f"route+dispatch+combine on all {wl.N} tokens; expert MLP on the {done} "
+                   f"rows of {len(experts)} experts, time scaled by {S}/{done} slots"),
+    }
+
+
+def run_reference(args, rank, world):
+    from synth.workloads import WORKLOADS
+    if rank != 0:
+        return
+    wl = WORKLOADS[args.workload]
+    for _ in range(args.warmup):
+        pass  # the reference has nothing to warm up; steps are timed below
+    vals = []
+    t_start = time.perf_counter()
+    res = None
+    for _ in range(args.steps):
+        res = oracle_sample(wl)
+        vals.append(res["value"])
+    wall = time.perf_counter() - t_start
+    v = statistics.mean(vals)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * wl.N / v,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": {"workload": wl.name, "N": wl.N, "d_r": wl.d_r,
+                                        "d_e": wl.d_e, "E": wl.E, "K": wl.K, "F": wl.F},
+        "cpu_baseline": {"value": v, "unit": UNIT, "cores": res["cores"], "kind": "oracle",
+                         "sample": res["sample"]},
+        "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "wall_s": wall,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    rank = int(os.environ.get("RANK", 0))
+    world = int(os.environ.get("WORLD_SIZE", 1))
+    local_rank = int(os.environ.get("LOCAL_RANK", 0))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+    import torch
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    wl, r = run_ours(args, rank, world, local_rank)
+    peaks = load_peaks()
+    achieved = gate_up_bytes(wl, r["touched"]) / (r["gate_up_ms"] * 1e-3) / 1e9
+    line = {
+        "metric": METRIC,
+        "value": world * wl.N / (r["ms"] * 1e-3),
+        "unit": UNIT,
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": max(args.warmup, 3),
+        "ms_per_step": r["ms"],
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": wl.name, "N": wl.N, "d_r": wl.d_r, "d_e": wl.d_e, "E": wl.E,
+                   "n_group": wl.G, "topk_group": wl.TG, "K": wl.K, "F": wl.F, "act": wl.act,
+                   "global_batch": world * wl.N, "parallelism": f"dp{world}",
+                   "l2": "expert weights > L2, plus a 256 MB write between steps outside the "
+                         "per-step events"},
+        "roofline": {"kernel": "expert w1/w3 (gate_up) grouped GEMM", "bound": "hbm",
+                     "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": achieved / peaks["hbm_gbs"], "traffic": None,
+                     "peak_source": peaks["source"], "touched_experts": r["touched"]},
+        "stages_ms": r["stage_ms"],
+        "e2e": {"value": world * wl.N / (r["e2e_ms"] * 1e-3), "unit": UNIT,
+                "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"]},
+        "gpu_launches": KERNELS_PER_STEP * args.steps,
+        "clocks": r["clocks"],
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cb = oracle_sample(wl)
+        line["cpu_baseline"] = {"value": cb["value"], "unit": UNIT, "cores": cb["cores"],
+                                "kind": "oracle", "sample": cb["sample"]}
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,218 @@
+/*
+ * moe.h -- C ABI of the B200 (sm_100a) inference MoE layer library, libmoe.so.
+ *
+ * The layer is the routed half of a DeepSeek-V3-style MoE block as the pages
+ * show it:
+ *   router   "Kimi K2 · Affinities", gate-forward excerpt (MoEGate.forward,
+ *            noaux_tc) and "DeepSeek-V3.2-Exp · Affinities", gate-forward
+ *            excerpt (Gate.forward): fp32 logits x.W^T, sigmoid, selection-only
+ *            correction bias, group score = sum of the group's top two, top
+ *            topk_group groups, top top_k experts, unbiased weights
+ *            renormalised and multiplied by the route scale;
+ *   dispatch "Kimi K3 · Add shared output", moe-forward excerpt (moe_infer):
+ *            per-expert counts, sort of the token slots by expert, row gather;
+ *   experts  "Kimi K3 · Gate features", expert excerpt (KimiBlockSparseMLP)
+ *            and situ excerpt (SituAndMul): w1/w3 projections, SiLU-and-mul or
+ *            SiTU, w2 projection;
+ *   combine  moe_infer again: unpermute, fp32 weighted sum over k, cast.
+ *
+ * Conventions shared by every entry point
+ *   - Tensor pointers are DEVICE pointers owned by the caller; the library
+ *     never allocates, frees or keeps them.  Row-major, densely packed.
+ *     bf16 tensors are passed as uint16_t bit patterns (moe_bf16).
+ *   - Scratch memory is passed in as (ws, ws_bytes), a device buffer of at
+ *     least the size the matching *_workspace_size function returns, 256-byte
+ *     aligned.  Its first 256 bytes hold the device status word.
+ *   - Every call enqueues its kernels on `stream` (a cudaStream_t, NULL = the
+ *     legacy default stream) and returns without synchronising.  No entry point
+ *     copies data to the host or waits for the GPU, so a sequence of calls can
+ *     be captured in a CUDA graph.
+ *   - Return value: MOE_OK or a negative moe_status.  Argument errors are found
+ *     on the host before anything is enqueued.  Errors found by the kernels
+ *     themselves (an expert index out of range, inconsistent offsets, a wait
+ *     that ran out) are recorded in the status word of the workspace; they are
+ *     sticky until moe_get_status() reads and clears them.
+ *   - N = 0 (no tokens) is a valid, empty call.
+ *   - Index tensors are int32 (the pages use int64).
+ *   - Stateless and thread-safe; device attributes are read once per device.
+ */
+#ifndef MOE_H
+#define MOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+typedef uint16_t moe_bf16;
+
+typedef enum moe_status {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = -1,    /* null pointer, negative size, inconsistent config */
+  MOE_ERR_UNSUPPORTED = -2,    /* shape outside the kernels' limits (see below)   */
+  MOE_ERR_ALIGNMENT = -3,      /* pointer not 16-byte aligned                      */
+  MOE_ERR_WORKSPACE = -4,      /* ws too small or not 256-byte aligned             */
+  MOE_ERR_CUDA = -5,           /* a CUDA call or launch failed                     */
+  MOE_ERR_DEVICE_TIMEOUT = -6, /* a kernel's bounded wait ran out (status word)    */
+  MOE_ERR_DEVICE_BOUNDS = -7,  /* a kernel met an index out of range (status word) */
+  MOE_ERR_NO_DEVICE = -8       /* no sm_100 device is current                      */
+} moe_status;
+
+/* Routing configuration ("Kimi K2 · Affinities", gate-init excerpt: the
+ * MoEGate fields; "DeepSeek-V3.2-Exp · Affinities", gate-init excerpt).
+ * Limits: 1 <= num_experts <= 1024; num_experts % n_group == 0;
+ * 1 <= n_group <= 32; if n_group > 1 each group holds >= 2 experts;
+ * 1 <= topk_group <= n_group; 1 <= top_k <= 16;
+ * top_k <= topk_group * num_experts / n_group. */
+typedef struct moe_route_cfg {
+  int num_experts;     /* E: n_routed_experts                                  */
+  int n_group;         /* G: groups of E/G consecutive experts                 */
+  int topk_group;      /* TG: groups kept per token                            */
+  int top_k;           /* K: experts per token (num_experts_per_tok)           */
+  int norm_topk_prob;  /* nonzero: renormalise the K weights when K > 1        */
+  float route_scale;   /* routed_scaling_factor / route_scale                  */
+} moe_route_cfg;
+
+/* Expert activation ("Kimi K3 · Gate features", situ excerpt).
+ * kind MOE_ACT_SILU: h = bf16(bf16(silu(g)) * u), silu(g) = g * sigmoid(g).
+ * kind MOE_ACT_SITU: h = bf16(beta*tanh(g/beta)*sigmoid(g) * u'),
+ *   u' = linear_beta*tanh(u/linear_beta) when linear_beta is set, else u;
+ *   evaluated in fp32.  beta == 0 or NaN means 1.0 (the page's "beta or 1.0");
+ *   linear_beta == 0 or NaN means "not set". */
+typedef enum moe_act_kind { MOE_ACT_SILU = 0, MOE_ACT_SITU = 1 } moe_act_kind;
+typedef struct moe_act_cfg {
+  int kind;
+  float beta;
+  float linear_beta;
+} moe_act_cfg;
+
+/* Expert-shape limits: d (hidden width of the experts) and F (d_ff) are
+ * multiples of 128; d_r (router width) is a multiple of 8; all bf16 row
+ * pointers 16-byte aligned. */
+
+/* ------------------------------------------------------------------ router */
+
+/* Scratch bytes needed by moe_route (and by moe_route_from_logits, which
+ * needs only the status word). */
+MOE_API size_t moe_route_workspace_size(int64_t N, int d_r, const moe_route_cfg* cfg);
+
+/* Router: for each of the N tokens,
+ *   L = fp32(x . W^T)                      ([N, d_r] bf16 x [E, d_r] fp32)
+ *   s = sigmoid(L) (fp32), c = s + bias    (bias only steers the choice)
+ *   if n_group > 1: group score = sum of the two largest c of the group; the
+ *     topk_group best groups are kept, the other experts get c = -inf
+ *   topk_idx = the top_k largest c, ordered by (c descending, index ascending)
+ *     -- ties go to the lowest expert index
+ *   topk_w[k] = s[topk_idx[k]]; if top_k > 1 and norm_topk_prob:
+ *     topk_w /= (sum_k topk_w + 1e-20), summed in k order; topk_w *= route_scale
+ * x: [N, d_r] bf16; W: [E, d_r] fp32; bias: [E] fp32 or NULL;
+ * topk_idx: [N, K] int32 out; topk_w: [N, K] fp32 out.
+ * The logits are accumulated in fp32 (the page's fp32 F.linear). */
+MOE_API int moe_route(const moe_bf16* x, int64_t N, int d_r, const float* W, const float* bias,
+                      const moe_route_cfg* cfg, int32_t* topk_idx, float* topk_w, void* ws,
+                      size_t ws_bytes, void* stream);
+
+/* Selection and weights only, from caller-supplied fp32 logits [N, E]: the
+ * same computation as moe_route after its gate GEMM.  Bit-exact: sigmoid is
+ * the fp32 rounding of 1/(1+exp(-L)) evaluated in double. */
+MOE_API int moe_route_from_logits(const float* logits, int64_t N, const float* bias,
+                                  const moe_route_cfg* cfg, int32_t* topk_idx, float* topk_w,
+                                  void* ws, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------- dispatch */
+
+MOE_API size_t moe_dispatch_workspace_size(int64_t N, int K, int E);
+
+/* moe_infer's dispatch with no host round trip:
+ *   counts[e]  = number of slots (t,k) with topk_idx[t,k] == e
+ *   offsets    = exclusive prefix sum of counts, offsets[E] = S = N*K
+ *   perm[j]    = slot t*K+k at sorted position j; the sort is STABLE: slots of
+ *                one expert keep ascending slot order
+ *   pos[slot]  = its sorted position (pos[perm[j]] == j)
+ *   xs[j, :]   = x_e[perm[j] / K, :]
+ * topk_idx: [N, K] int32; x_e: [N, d_e] bf16; counts [E], offsets [E+1],
+ * perm [S], pos [S] int32 out; xs [S, d_e] bf16 out.
+ * An expert index outside [0, E) is recorded as MOE_ERR_DEVICE_BOUNDS and its
+ * slot is left out of every output. */
+MOE_API int moe_dispatch(const int32_t* topk_idx, int64_t N, int K, int E, const moe_bf16* x_e,
+                         int d_e, int32_t* counts, int32_t* offsets, int32_t* perm, int32_t* pos,
+                         moe_bf16* xs, void* ws, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------- expert MLP */
+
+MOE_API size_t moe_expert_ffn_workspace_size(int64_t S, int d_e, int E, int F);
+
+/* Grouped expert MLP over the sorted rows: for every expert e, the rows
+ * offsets[e] .. offsets[e+1]-1 of xs go through
+ *   g = bf16(xs . w1[e]^T), u = bf16(xs . w3[e]^T)   (fp32 accumulation)
+ *   h = act(g, u) (see moe_act_cfg), y = bf16(h . w2[e]^T)
+ * xs: [S, d_e] bf16; offsets: [E+1] int32 (non-decreasing, offsets[0] = 0,
+ * offsets[E] = S); w1, w3: [E, F, d_e] bf16; w2: [E, d_e, F] bf16;
+ * y: [S, d_e] bf16 out.  Experts with no rows cost nothing. */
+MOE_API int moe_expert_ffn(const moe_bf16* xs, const int32_t* offsets, int E, int64_t S, int d_e,
+                           int F, const moe_bf16* w1, const moe_bf16* w3, const moe_bf16* w2,
+                           const moe_act_cfg* act, moe_bf16* y, void* ws, size_t ws_bytes,
+                           void* stream);
+
+/* ----------------------------------------------------------------- combine */
+
+MOE_API size_t moe_combine_workspace_size(void);
+
+/* Unpermute and combine:
+ *   out[t, :] = bf16( sum_{k=0..K-1} fp32(y[pos[t*K+k], :]) * topk_w[t, k] )
+ * with every product rounded to fp32 and the sum taken in k order in fp32.
+ * y: [S, d_e] bf16; pos: [S] int32; topk_w: [N, K] fp32; out: [N, d_e] bf16. */
+MOE_API int moe_combine(const moe_bf16* y, const int32_t* pos, const float* topk_w, int64_t N,
+                        int K, int d_e, moe_bf16* out, void* ws, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------ whole layer */
+
+MOE_API size_t moe_workspace_size(int64_t N, int d_r, int d_e, const moe_route_cfg* cfg, int F);
+
+/* Optional CUDA events recorded between the stages of moe_forward (each entry
+ * a cudaEvent_t or NULL): after routing, after dispatch, after the w1/w3
+ * kernel, after the w2 kernel, after the combine. */
+typedef struct moe_stage_events {
+  void* after_route;
+  void* after_dispatch;
+  void* after_gate_up;
+  void* after_down;
+  void* after_combine;
+} moe_stage_events;
+
+/* The routed MoE layer, moe_route -> moe_dispatch -> moe_expert_ffn ->
+ * moe_combine, on one stream with no host synchronisation.
+ * x_r: [N, d_r] bf16, the router's input.  x_e: [N, d_e] bf16, the experts'
+ * input, or NULL to use x_r (then d_e must equal d_r); a latent MoE routes on
+ * the full width and runs its experts on a narrower input.
+ * topk_idx_out [N, K] int32 and topk_w_out [N, K] fp32 may be NULL.
+ * events may be NULL. */
+MOE_API int moe_forward(const moe_bf16* x_r, const moe_bf16* x_e, int64_t N, int d_r, int d_e,
+                        const float* W, const float* bias, const moe_route_cfg* cfg,
+                        const moe_bf16* w1, const moe_bf16* w3, const moe_bf16* w2, int F,
+                        const moe_act_cfg* act, moe_bf16* out, int32_t* topk_idx_out,
+                        float* topk_w_out, void* ws, size_t ws_bytes, void* stream,
+                        const moe_stage_events* events);
+
+/* --------------------------------------------------------------- status */
+
+/* Reads (synchronising `stream`) and clears the device status word of a
+ * workspace.  Returns MOE_OK or the first device-side error recorded. */
+MOE_API int moe_get_status(void* ws, void* stream);
+
+/* Text for a moe_status code. */
+MOE_API const char* moe_strerror(int code);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_H */

@@ -1,0 +1,293 @@
+"""Python binding of libmoe.so, the B200 (sm_100a) inference MoE layer.
+
+Argument marshalling only: every step of the layer runs in the library's CUDA
+kernels.  Tensors are torch CUDA tensors (PyTorch provides device memory and
+streams); every call enqueues on ``torch.cuda.current_stream()`` and returns
+without synchronising.  The entry points and their semantics are those of
+``include/moe.h``.
+
+There is no fallback: if ``libmoe.so`` has not been built, importing the
+binding's functions raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libmoe.so")
+
+MOE_ACT_SILU, MOE_ACT_SITU = 0, 1
+_ERR = {
+    0: "ok", -1: "invalid argument", -2: "unsupported shape", -3: "misaligned pointer",
+    -4: "workspace too small or misaligned", -5: "CUDA call failed",
+    -6: "device wait timed out", -7: "device index out of range", -8: "no sm_100 device",
+}
+
+
+class MoeError(RuntimeError):
+    def __init__(self, fn: str, code: int):
+        super().__init__(f"{fn} failed: {code} ({_ERR.get(code, 'unknown')})")
+        self.code = code
+
+
+class _RouteCfg(ctypes.Structure):
+    _fields_ = [("num_experts", ctypes.c_int), ("n_group", ctypes.c_int),
+                ("topk_group", ctypes.c_int), ("top_k", ctypes.c_int),
+                ("norm_topk_prob", ctypes.c_int), ("route_scale", ctypes.c_float)]
+
+
+class _ActCfg(ctypes.Structure):
+    _fields_ = [("kind", ctypes.c_int), ("beta", ctypes.c_float),
+                ("linear_beta", ctypes.c_float)]
+
+
+class _StageEvents(ctypes.Structure):
+    _fields_ = [("after_route", ctypes.c_void_p), ("after_dispatch", ctypes.c_void_p),
+                ("after_gate_up", ctypes.c_void_p), ("after_down", ctypes.c_void_p),
+                ("after_combine", ctypes.c_void_p)]
+
+
+@dataclass(frozen=True)
+class RouteConfig:
+    num_experts: int
+    n_group: int
+    topk_group: int
+    top_k: int
+    route_scale: float
+    norm_topk_prob: bool = True
+
+    def _c(self) -> _RouteCfg:
+        return _RouteCfg(self.num_experts, self.n_group, self.topk_group, self.top_k,
+                         int(bool(self.norm_topk_prob)), self.route_scale)
+
+
+@dataclass(frozen=True)
+class ActConfig:
+    kind: str = "silu"        # "silu" or "situ"
+    beta: float = 1.0
+    linear_beta: float = 0.0  # 0 = not set
+
+    def _c(self) -> _ActCfg:
+        return _ActCfg({"silu": MOE_ACT_SILU, "situ": MOE_ACT_SITU}[self.kind], self.beta,
+                       self.linear_beta)
+
+
+_lib = None
+EXPORTS = ("moe_route_workspace_size", "moe_route", "moe_route_from_logits",
+           "moe_dispatch_workspace_size", "moe_dispatch", "moe_expert_ffn_workspace_size",
+           "moe_expert_ffn", "moe_combine_workspace_size", "moe_combine", "moe_workspace_size",
+           "moe_forward", "moe_get_status", "moe_strerror")
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded libmoe.so (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing: build it with "
+                          "`python -m moe_routing_expert_fp32_b200.build`")
+    L = ctypes.CDLL(LIB_PATH)
+    vp, i64, i32, sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t
+    rc, ac, ev = ctypes.POINTER(_RouteCfg), ctypes.POINTER(_ActCfg), ctypes.POINTER(_StageEvents)
+    sig = {
+        "moe_route_workspace_size": ([i64, i32, rc], sz),
+        "moe_route": ([vp, i64, i32, vp, vp, rc, vp, vp, vp, sz, vp], i32),
+        "moe_route_from_logits": ([vp, i64, vp, rc, vp, vp, vp, sz, vp], i32),
+        "moe_dispatch_workspace_size": ([i64, i32, i32], sz),
+        "moe_dispatch": ([vp, i64, i32, i32, vp, i32, vp, vp, vp, vp, vp, vp, sz, vp], i32),
+        "moe_expert_ffn_workspace_size": ([i64, i32, i32, i32], sz),
+        "moe_expert_ffn": ([vp, vp, i32, i64, i32, i32, vp, vp, vp, ac, vp, vp, sz, vp], i32),
+        "moe_combine_workspace_size": ([], sz),
+        "moe_combine": ([vp, vp, vp, i64, i32, i32, vp, vp, sz, vp], i32),
+        "moe_workspace_size": ([i64, i32, i32, rc, i32], sz),
+        "moe_forward": ([vp, vp, i64, i32, i32, vp, vp, rc, vp, vp, vp, i32, ac, vp, vp, vp, vp,
+                         sz, vp, ev], i32),
+        "moe_get_status": ([vp, vp], i32),
+        "moe_strerror": ([i32], ctypes.c_char_p),
+    }
+    for name, (args, res) in sig.items():
+        fn = getattr(L, name)
+        fn.argtypes = args
+        fn.restype = res
+    _lib = L
+    return L
+
+
+# ----------------------------------------------------------------- helpers
+def _torch():
+    import torch
+    return torch
+
+
+def _stream():
+    return ctypes.c_void_p(_torch().cuda.current_stream().cuda_stream)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _check(fn: str, code: int) -> None:
+    if code != 0:
+        raise MoeError(fn, code)
+
+
+def _need(t, dtype, shape=None, name="tensor"):
+    torch = _torch()
+    if not (t.is_cuda and t.is_contiguous() and t.dtype == dtype):
+        raise ValueError(f"{name} must be a contiguous CUDA {dtype} tensor")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+    return torch
+
+
+def workspace(nbytes: int, device=None):
+    """A 256-byte aligned device buffer of at least nbytes (torch allocations are)."""
+    torch = _torch()
+    return torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device or "cuda")
+
+
+def get_status(ws) -> int:
+    """Device status of the last call on this workspace (synchronises)."""
+    return int(lib().moe_get_status(_ptr(ws), _stream()))
+
+
+# --------------------------------------------------------------- entry points
+def route(x, W, bias, cfg: RouteConfig, ws=None):
+    torch = _torch()
+    N, d_r = x.shape
+    _need(x, torch.bfloat16, name="x")
+    _need(W, torch.float32, (cfg.num_experts, d_r), "W")
+    if bias is not None:
+        _need(bias, torch.float32, (cfg.num_experts,), "bias")
+    c = cfg._c()
+    need = lib().moe_route_workspace_size(N, d_r, ctypes.byref(c))
+    ws = workspace(need, x.device) if ws is None else ws
+    idx = torch.empty((N, cfg.top_k), dtype=torch.int32, device=x.device)
+    w = torch.empty((N, cfg.top_k), dtype=torch.float32, device=x.device)
+    _check("moe_route", lib().moe_route(_ptr(x), N, d_r, _ptr(W), _ptr(bias), ctypes.byref(c),
+                                        _ptr(idx), _ptr(w), _ptr(ws), ws.numel(), _stream()))
+    return idx, w
+
+
+def route_from_logits(logits, bias, cfg: RouteConfig, ws=None):
+    torch = _torch()
+    N, E = logits.shape
+    _need(logits, torch.float32, name="logits")
+    if E != cfg.num_experts:
+        raise ValueError("logits width != num_experts")
+    if bias is not None:
+        _need(bias, torch.float32, (E,), "bias")
+    ws = workspace(256, logits.device) if ws is None else ws
+    idx = torch.empty((N, cfg.top_k), dtype=torch.int32, device=logits.device)
+    w = torch.empty((N, cfg.top_k), dtype=torch.float32, device=logits.device)
+    c = cfg._c()
+    _check("moe_route_from_logits",
+           lib().moe_route_from_logits(_ptr(logits), N, _ptr(bias), ctypes.byref(c), _ptr(idx),
+                                       _ptr(w), _ptr(ws), ws.numel(), _stream()))
+    return idx, w
+
+
+def dispatch(topk_idx, x_e, num_experts: int, ws=None):
+    """(counts [E], offsets [E+1], perm [S], pos [S], xs [S, d_e])."""
+    torch = _torch()
+    N, K = topk_idx.shape
+    d_e = x_e.shape[1]
+    _need(topk_idx, torch.int32, name="topk_idx")
+    _need(x_e, torch.bfloat16, (N, d_e), "x_e")
+    E = num_experts
+    S = N * K
+    dev = x_e.device
+    need = lib().moe_dispatch_workspace_size(N, K, E)
+    ws = workspace(need, dev) if ws is None else ws
+    counts = torch.empty(E, dtype=torch.int32, device=dev)
+    offsets = torch.empty(E + 1, dtype=torch.int32, device=dev)
+    perm = torch.empty(S, dtype=torch.int32, device=dev)
+    pos = torch.empty(S, dtype=torch.int32, device=dev)
+    xs = torch.empty((S, d_e), dtype=torch.bfloat16, device=dev)
+    _check("moe_dispatch",
+           lib().moe_dispatch(_ptr(topk_idx), N, K, E, _ptr(x_e), d_e, _ptr(counts),
+                              _ptr(offsets), _ptr(perm), _ptr(pos), _ptr(xs), _ptr(ws),
+                              ws.numel(), _stream()))
+    return counts, offsets, perm, pos, xs
+
+
+def expert_ffn(xs, offsets, w1, w3, w2, act: ActConfig, ws=None, y=None):
+    torch = _torch()
+    S, d_e = xs.shape
+    E, F, _ = w1.shape
+    _need(xs, torch.bfloat16, name="xs")
+    _need(offsets, torch.int32, (E + 1,), "offsets")
+    _need(w1, torch.bfloat16, (E, F, d_e), "w1")
+    _need(w3, torch.bfloat16, (E, F, d_e), "w3")
+    _need(w2, torch.bfloat16, (E, d_e, F), "w2")
+    dev = xs.device
+    need = lib().moe_expert_ffn_workspace_size(S, d_e, E, F)
+    ws = workspace(need, dev) if ws is None else ws
+    y = torch.empty((S, d_e), dtype=torch.bfloat16, device=dev) if y is None else y
+    a = act._c()
+    _check("moe_expert_ffn",
+           lib().moe_expert_ffn(_ptr(xs), _ptr(offsets), E, S, d_e, F, _ptr(w1), _ptr(w3),
+                                _ptr(w2), ctypes.byref(a), _ptr(y), _ptr(ws), ws.numel(),
+                                _stream()))
+    return y
+
+
+def combine(y, pos, topk_w, ws=None):
+    torch = _torch()
+    N, K = topk_w.shape
+    d_e = y.shape[1]
+    _need(y, torch.bfloat16, (N * K, d_e), "y")
+    _need(pos, torch.int32, (N * K,), "pos")
+    _need(topk_w, torch.float32, name="topk_w")
+    ws = workspace(256, y.device) if ws is None else ws
+    out = torch.empty((N, d_e), dtype=torch.bfloat16, device=y.device)
+    _check("moe_combine", lib().moe_combine(_ptr(y), _ptr(pos), _ptr(topk_w), N, K, d_e,
+                                            _ptr(out), _ptr(ws), ws.numel(), _stream()))
+    return out
+
+
+def workspace_size(N: int, d_r: int, d_e: int, cfg: RouteConfig, F: int) -> int:
+    c = cfg._c()
+    return int(lib().moe_workspace_size(N, d_r, d_e, ctypes.byref(c), F))
+
+
+def forward(x_r, W, bias, cfg: RouteConfig, w1, w3, w2, act: ActConfig, x_e=None, ws=None,
+            out=None, topk_idx=None, topk_w=None, events=None):
+    """The routed MoE layer (moe_forward). Returns ``out`` [N, d_e] bf16.
+
+    ``events``: optional dict of torch.cuda.Event recorded between the stages
+    (keys after_route, after_dispatch, after_gate_up, after_down, after_combine).
+    """
+    torch = _torch()
+    N, d_r = x_r.shape
+    E, F, d_e = w1.shape
+    _need(x_r, torch.bfloat16, name="x_r")
+    if x_e is not None:
+        _need(x_e, torch.bfloat16, (N, d_e), "x_e")
+    elif d_e != d_r:
+        raise ValueError("x_e is required when the experts' width differs from the router's")
+    _need(W, torch.float32, (E, d_r), "W")
+    if bias is not None:
+        _need(bias, torch.float32, (E,), "bias")
+    dev = x_r.device
+    c = cfg._c()
+    a = act._c()
+    need = lib().moe_workspace_size(N, d_r, d_e, ctypes.byref(c), F)
+    ws = workspace(need, dev) if ws is None else ws
+    out = torch.empty((N, d_e), dtype=torch.bfloat16, device=dev) if out is None else out
+    evp = None
+    if events:
+        se = _StageEvents(*[ctypes.c_void_p(events[k].cuda_event) if k in events else None
+                            for k in ("after_route", "after_dispatch", "after_gate_up",
+                                      "after_down", "after_combine")])
+        evp = ctypes.byref(se)
+    _check("moe_forward",
+           lib().moe_forward(_ptr(x_r), _ptr(x_e), N, d_r, d_e, _ptr(W), _ptr(bias),
+                             ctypes.byref(c), _ptr(w1), _ptr(w3), _ptr(w2), F, ctypes.byref(a),
+                             _ptr(out), _ptr(topk_idx), _ptr(topk_w), _ptr(ws), ws.numel(),
+                             _stream(), evp))
+    return out

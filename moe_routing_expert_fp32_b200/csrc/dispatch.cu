@@ -1,0 +1,203 @@
+// dispatch.cu -- moe_infer's dispatch without a host round trip.
+//
+// Follows "Kimi K3 · Add shared output", moe-forward excerpt (moe_infer):
+// per-expert counts (cnts.scatter_ + sum), argsort of the flat slots, and
+// sorted_tokens = x[idxs // K].  The page copies the counts to the host
+// (.cpu()) to drive a Python loop over experts; here the counts, offsets and
+// the grouped GEMM's tile list stay on the device.
+//
+// The slot sort is a stable counting sort in three passes:
+//   k_hist    one warp per chunk of CH consecutive slots: per-chunk expert
+//             counts (warp-aggregated with __match_any_sync);
+//   k_scan    one block: counts[e], offsets (exclusive scan) and, per chunk,
+//             the first sorted position of each expert;
+//   k_scatter one warp per chunk again: slots ranked in slot order within the
+//             chunk -> pos[slot] and perm[pos].
+// Then k_gather copies every token row once from HBM and writes it to its K
+// sorted positions (token-major, so x_e is read once, not K times).
+#include "moe_internal.cuh"
+
+namespace moe {
+namespace {
+
+constexpr int kWarps = 4;
+
+__device__ __forceinline__ unsigned lanemask_lt() {
+  unsigned m;
+  asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
+  return m;
+}
+
+__global__ void __launch_bounds__(32 * kWarps) k_hist(const int32_t* __restrict__ idx, int64_t S,
+                                                      int E, int CH, int nchunks,
+                                                      int32_t* __restrict__ cc, DeviceStatus* st) {
+  extern __shared__ int32_t cnt_all[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int c = blockIdx.x * kWarps + warp;
+  if (c >= nchunks) return;
+  int32_t* cnt = cnt_all + warp * E;
+  for (int e = lane; e < E; e += 32) cnt[e] = 0;
+  __syncwarp();
+  const int64_t beg = (int64_t)c * CH;
+  const int64_t end = beg + CH < S ? beg + CH : S;
+  for (int64_t base = beg; base < end; base += 32) {
+    const int64_t slot = base + lane;
+    int e = -1;
+    if (slot < end) {
+      e = idx[slot];
+      if (e < 0 || e >= E) {
+        record_error(st, MOE_ERR_DEVICE_BOUNDS, 10);
+        e = -1;
+      }
+    }
+    const unsigned peers = __match_any_sync(0xffffffffu, e);
+    if (e >= 0 && lane == __ffs(peers) - 1) cnt[e] += __popc(peers);
+    __syncwarp();
+  }
+  int32_t* out = cc + (int64_t)c * E;
+  for (int e = lane; e < E; e += 32) out[e] = cnt[e];
+}
+
+// One block of 1024 threads; thread e owns expert e (E <= 1024).
+__global__ void __launch_bounds__(1024) k_scan(int32_t* __restrict__ cc, int nchunks, int E,
+                                               int32_t* __restrict__ counts,
+                                               int32_t* __restrict__ offsets) {
+  __shared__ int32_t warp_tot[32];
+  const int e = threadIdx.x;
+  const int lane = e & 31, warp = e >> 5;
+  int32_t tot = 0;
+  if (e < E)
+    for (int c = 0; c < nchunks; ++c) tot += cc[(int64_t)c * E + e];
+  // block exclusive scan of tot
+  int32_t v = tot;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int32_t o = __shfl_up_sync(0xffffffffu, v, off);
+    if (lane >= off) v += o;
+  }
+  if (lane == 31) warp_tot[warp] = v;
+  __syncthreads();
+  if (warp == 0) {
+    int32_t w = warp_tot[lane];
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int32_t o = __shfl_up_sync(0xffffffffu, w, off);
+      if (lane >= off) w += o;
+    }
+    warp_tot[lane] = w;
+  }
+  __syncthreads();
+  const int32_t excl = v - tot + (warp > 0 ? warp_tot[warp - 1] : 0);
+  if (e < E) {
+    counts[e] = tot;
+    offsets[e] = excl;
+    if (e == E - 1) offsets[E] = excl + tot;
+    int32_t run = excl;
+    for (int c = 0; c < nchunks; ++c) {
+      const int32_t n = cc[(int64_t)c * E + e];
+      cc[(int64_t)c * E + e] = run;
+      run += n;
+    }
+  }
+}
+
+__global__ void __launch_bounds__(32 * kWarps) k_scatter(const int32_t* __restrict__ idx,
+                                                         int64_t S, int E, int CH, int nchunks,
+                                                         const int32_t* __restrict__ cc,
+                                                         int32_t* __restrict__ perm,
+                                                         int32_t* __restrict__ pos) {
+  extern __shared__ int32_t base_all[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int c = blockIdx.x * kWarps + warp;
+  if (c >= nchunks) return;
+  int32_t* base = base_all + warp * E;
+  const int32_t* in = cc + (int64_t)c * E;
+  for (int e = lane; e < E; e += 32) base[e] = in[e];
+  __syncwarp();
+  const unsigned lt = lanemask_lt();
+  const int64_t beg = (int64_t)c * CH;
+  const int64_t end = beg + CH < S ? beg + CH : S;
+  for (int64_t b0 = beg; b0 < end; b0 += 32) {
+    const int64_t slot = b0 + lane;
+    int e = -1;
+    if (slot < end) {
+      e = idx[slot];
+      if (e < 0 || e >= E) e = -1;
+    }
+    const unsigned peers = __match_any_sync(0xffffffffu, e);
+    if (slot < end) {
+      if (e >= 0) {
+        const int32_t p = base[e] + __popc(peers & lt);
+        pos[slot] = p;
+        perm[p] = (int32_t)slot;
+      } else {
+        pos[slot] = -1;
+      }
+    }
+    __syncwarp();
+    if (e >= 0 && lane == __ffs(peers) - 1) base[e] += __popc(peers);
+    __syncwarp();
+  }
+}
+
+// One warp per token: read its row once (16-byte vectors), write it to the
+// K sorted positions pos[t*K + k].
+__global__ void __launch_bounds__(256) k_gather(const __nv_bfloat16* __restrict__ x, int64_t N,
+                                                int K, int d, const int32_t* __restrict__ pos,
+                                                __nv_bfloat16* __restrict__ xs) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nv = d / 8;
+  for (int64_t t = (int64_t)blockIdx.x * 8 + warp; t < N; t += (int64_t)gridDim.x * 8) {
+    const int my_p = lane < K ? pos[t * K + lane] : -1;
+    const uint4* src = reinterpret_cast<const uint4*>(x + t * d);
+    for (int v = lane; v < nv; v += 32) {
+      const uint4 val = src[v];
+      for (int k = 0; k < K; ++k) {
+        const int p = __shfl_sync(0xffffffffu, my_p, k);
+        if (p >= 0) reinterpret_cast<uint4*>(xs + (int64_t)p * d)[v] = val;
+      }
+    }
+  }
+}
+
+}  // namespace
+
+int dispatch_chunks(int64_t S) {
+  int64_t ch = S / 256;
+  if (ch < 64) ch = 64;
+  if (ch > 1024) ch = 1024;
+  ch = (ch + 31) / 32 * 32;
+  return (int)((S + ch - 1) / ch);
+}
+
+static int dispatch_chunk_len(int64_t S) {
+  int64_t ch = S / 256;
+  if (ch < 64) ch = 64;
+  if (ch > 1024) ch = 1024;
+  return (int)((ch + 31) / 32 * 32);
+}
+
+size_t dispatch_scratch_bytes(int64_t S, int E) {
+  return align_up(sizeof(int32_t) * (size_t)dispatch_chunks(S) * (size_t)E, 256);
+}
+
+cudaError_t launch_dispatch(const int32_t* idx, int64_t N, int K, int E, const __nv_bfloat16* x_e,
+                            int d_e, int32_t* counts, int32_t* offsets, int32_t* perm,
+                            int32_t* pos, __nv_bfloat16* xs, int32_t* scratch, DeviceStatus* st,
+                            cudaStream_t s) {
+  const int64_t S = N * K;
+  const int CH = dispatch_chunk_len(S);
+  const int nchunks = dispatch_chunks(S);
+  const size_t smem = sizeof(int32_t) * (size_t)E * kWarps;
+  const unsigned blocks = (unsigned)((nchunks + kWarps - 1) / kWarps);
+  k_hist<<<blocks, 32 * kWarps, smem, s>>>(idx, S, E, CH, nchunks, scratch, st);
+  k_scan<<<1, 1024, 0, s>>>(scratch, nchunks, E, counts, offsets);
+  k_scatter<<<blocks, 32 * kWarps, smem, s>>>(idx, S, E, CH, nchunks, scratch, perm, pos);
+  int64_t gb = (N + 7) / 8;
+  const int64_t cap = (int64_t)dev_info()->sm_count * 8;
+  if (gb > cap) gb = cap;
+  k_gather<<<(unsigned)gb, 256, 0, s>>>(x_e, N, K, d_e, pos, xs);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -1,0 +1,521 @@
+// expert_gemm.cu -- grouped expert MLP on the 5th-generation tensor cores.
+//
+// Follows "Kimi K3 · Gate features", expert excerpt (KimiBlockSparseMLP:
+// w1 = gate, w3 = up, w2 = down, all bias-free nn.Linear) and situ excerpt
+// (SituAndMul), and the per-expert loop of moe_infer ("Kimi K3 · Add shared
+// output", moe-forward excerpt), which is replaced by one persistent launch
+// over a device-built tile list.
+//
+// Design (sm_100a):
+//   * swap-AB: the MMA's M=128 side is a block of 128 weight rows, the N side
+//     is up to 128 token rows of one expert (N rounded up to 16).  Decode
+//     batches put 1-8 tokens on an expert, so the kernel is a weight stream;
+//     weight tiles fill the 128-lane accumulator whatever the token count.
+//   * TMA (cp.async.bulk.tensor, 128-byte swizzle) brings a 128x64 weight tile
+//     per operand (w1 and w3 share the token tile) and the token tile as 16-row
+//     boxes, into a 4-6 stage shared-memory ring guarded by mbarriers.
+//   * one elected thread issues tcgen05.mma (kind::f16, bf16 in, fp32 out)
+//     into TMEM; the 512 TMEM columns hold two accumulator buffers so the
+//     epilogue of one tile overlaps the MMAs of the next.
+//   * 4 epilogue warps read the accumulator with tcgen05.ld, apply the page's
+//     rounding points (g, u rounded to bf16; SiLU output rounded to bf16; h
+//     rounded to bf16) and store bf16 rows.
+//   * unit u -> (token tile, weight-row block) with the row block fastest, so
+//     CTAs that run at the same time share one token tile from L2 and stream
+//     disjoint weight rows.
+//   * every wait is bounded (2 s of %globaltimer); a wait that runs out
+//     records MOE_ERR_DEVICE_TIMEOUT, tells the other roles to stop, and the
+//     kernel frees its TMEM and returns.
+#include <cuda.h>
+#include <math.h>
+
+#include "moe_internal.cuh"
+
+namespace moe {
+namespace {
+
+constexpr int BM = 128;       // weight rows per tile (MMA M)
+constexpr int BK = 64;        // K elements per stage: one 128-byte swizzle row
+constexpr int NT = 128;       // token rows per tile (max MMA N)
+constexpr int UK = 16;        // K per tcgen05.mma for 16-bit inputs
+constexpr int kThreads = 192; // warp 0: TMA, warp 1: MMA + TMEM, warps 2-5: epilogue
+constexpr int kBoxRows = 16;  // token rows per TMA box
+constexpr uint64_t kTimeoutNs = 2000000000ull;
+
+enum Mode { kGateUp = 0, kDown = 1 };
+
+template <int MODE>
+struct Cfg {
+  static constexpr int kA = (MODE == kGateUp) ? 2 : 1;
+  static constexpr int kABytes = BM * BK * 2;
+  static constexpr int kBBytes = NT * BK * 2;
+  static constexpr int kStageBytes = kA * kABytes + kBBytes;
+  static constexpr int kStages = (MODE == kGateUp) ? 4 : 6;
+  static constexpr int kBufCols = 256;  // TMEM columns per accumulator buffer
+  static constexpr int kTmemCols = 512;
+  static constexpr size_t kSmem = (size_t)kStages * kStageBytes + 1024 + 256;
+};
+
+// ------------------------------------------------------------ PTX wrappers
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ uint64_t gtimer() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
+}
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
+               "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Waits for the phase of parity `parity` to complete; false if it did not
+// within kTimeoutNs or another role gave up first.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
+                                          volatile int* abort_flag) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = gtimer();
+  for (uint32_t i = 1;; ++i) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((i & 63) == 0) {
+      if (*abort_flag) return false;
+      if (gtimer() - t0 > kTimeoutNs) return false;
+    }
+  }
+}
+__device__ __forceinline__ void tma_load_2d(const CUtensorMap* map, uint64_t* bar, void* dst,
+                                            int c0, int c1) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1)
+      : "memory");
+}
+__device__ __forceinline__ void tma_load_3d(const CUtensorMap* map, uint64_t* bar, void* dst,
+                                            int c0, int c1, int c2) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                          uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate));
+}
+__device__ __forceinline__ void umma_commit(uint64_t* bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+          smem_u32(bar))
+      : "memory");
+}
+// 32 lanes x 16 consecutive fp32 columns; waits for the load before returning.
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float* v) {
+  uint32_t r[16];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+        "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr)
+      : "memory");
+#pragma unroll
+  for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// Shared-memory matrix descriptor: K-major operand, 128-byte swizzle, rows of
+// 128 bytes, 8-row groups 1024 bytes apart (tile base 1024-byte aligned).
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr & 0x3FFFFu) >> 4);  // start address
+  d |= (uint64_t)1 << 16;                     // leading byte offset (unused here)
+  d |= (uint64_t)(1024 >> 4) << 32;           // stride byte offset
+  d |= (uint64_t)1 << 46;                     // descriptor version
+  d |= (uint64_t)2 << 61;                     // 128-byte swizzle
+  return d;
+}
+// Instruction descriptor: bf16 x bf16 -> fp32, both K-major, M = 128.
+__device__ __forceinline__ uint32_t idesc_bf16(int n) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) |
+         ((uint32_t)(BM >> 4) << 24);
+}
+
+__device__ __forceinline__ float bf16r(float x) {
+  return __bfloat162float(__float2bfloat16_rn(x));
+}
+
+// SiLU-and-mul with the page's rounding points: g and u are bf16 Linear
+// outputs; silu(g) is evaluated in fp32 and rounded to bf16; the product of two
+// bf16 values is exact in fp32 and rounded to bf16 by the store.
+__device__ __forceinline__ float silu_mul(float g, float u) {
+  g = bf16r(g);
+  u = bf16r(u);
+  const float a = bf16r(__fdiv_rn(g, __fadd_rn(1.0f, expf(-g))));
+  return __fmul_rn(a, u);
+}
+// SiTU: beta*tanh(g/beta)*sigmoid(g) * (lbeta*tanh(u/lbeta) or u), in fp32.
+__device__ __forceinline__ float situ_mul(float g, float u, float beta, float lbeta, bool has_lb) {
+  g = bf16r(g);
+  u = bf16r(u);
+  const float t = __fmul_rn(beta, tanhf(__fdiv_rn(g, beta)));
+  const float sg = __fdiv_rn(1.0f, __fadd_rn(1.0f, expf(-g)));
+  const float up = has_lb ? __fmul_rn(lbeta, tanhf(__fdiv_rn(u, lbeta))) : u;
+  return __fmul_rn(__fmul_rn(t, sg), up);
+}
+
+struct Unit {
+  int e, row0, nrows, rb;
+};
+
+__device__ __forceinline__ Unit decode_unit(int64_t u, int RB, const int32_t* tile_start,
+                                            const int32_t* offsets, int E) {
+  Unit r;
+  const int tt = (int)(u / RB);
+  r.rb = (int)(u - (int64_t)tt * RB);
+  int lo = 0, hi = E - 1;
+  while (lo < hi) {  // largest e with tile_start[e] <= tt
+    const int mid = (lo + hi + 1) >> 1;
+    if (tile_start[mid] <= tt) lo = mid;
+    else hi = mid - 1;
+  }
+  r.e = lo;
+  r.row0 = offsets[lo] + (tt - tile_start[lo]) * NT;
+  const int rem = offsets[lo + 1] - r.row0;
+  r.nrows = rem < NT ? rem : NT;
+  return r;
+}
+
+template <int MODE>
+__global__ void __launch_bounds__(kThreads, 1)
+    k_expert_gemm(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA1,
+                  const __grid_constant__ CUtensorMap tmB, const int32_t* __restrict__ offsets,
+                  const int32_t* __restrict__ tile_start, int E, int M_rows, int Kdim,
+                  __nv_bfloat16* __restrict__ out, int act_kind, float beta, float lbeta,
+                  DeviceStatus* st) {
+  using C = Cfg<MODE>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kStages * C::kStageBytes);
+  uint64_t* empty = full + C::kStages;
+  uint64_t* tfull = empty + C::kStages;
+  uint64_t* tempty = tfull + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + 2);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int RB = M_rows / BM;
+  const int KB = Kdim / BK;
+  const int64_t total_units = (int64_t)tile_start[E] * RB;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tfull[b], 1);
+      mbar_init(&tempty[b], 128);
+    }
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(tmem_slot)),
+                 "r"(C::kTmemCols));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int64_t u = blockIdx.x; u < total_units && ok; u += gridDim.x) {
+        const Unit w = decode_unit(u, RB, tile_start, offsets, E);
+        const int nb = (w.nrows + kBoxRows - 1) / kBoxRows;
+        const uint32_t bytes = C::kA * C::kABytes + nb * kBoxRows * BK * 2;
+        for (int kb = 0; kb < KB; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag)) { ok = false; break; }
+          uint8_t* sA = smem + stage * C::kStageBytes;
+          uint8_t* sB = sA + C::kA * C::kABytes;
+          mbar_arrive_expect_tx(&full[stage], bytes);
+          tma_load_3d(&tmA0, &full[stage], sA, kb * BK, w.rb * BM, w.e);
+          if (MODE == kGateUp) tma_load_3d(&tmA1, &full[stage], sA + C::kABytes, kb * BK, w.rb * BM, w.e);
+          for (int i = 0; i < nb; ++i)
+            tma_load_2d(&tmB, &full[stage], sB + i * kBoxRows * BK * 2, kb * BK,
+                        w.row0 + i * kBoxRows);
+          if (++stage == C::kStages) { stage = 0; phase ^= 1; }
+        }
+      }
+      if (!ok) {
+        record_error(st, MOE_ERR_DEVICE_TIMEOUT, 100 + MODE);
+        *abort_flag = 1;
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int local = 0;
+      bool ok = true;
+      for (int64_t u = blockIdx.x; u < total_units && ok; u += gridDim.x, ++local) {
+        const Unit w = decode_unit(u, RB, tile_start, offsets, E);
+        const int n = ((w.nrows + 15) / 16) * 16;
+        const uint32_t idesc = idesc_bf16(n);
+        const int buf = local & 1;
+        const uint32_t tphase = (local >> 1) & 1;
+        if (!mbar_wait(&tempty[buf], tphase ^ 1, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t d0 = tmem_base + buf * C::kBufCols;
+        for (int kb = 0; kb < KB; ++kb) {
+          if (!mbar_wait(&full[stage], phase, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(smem + stage * C::kStageBytes);
+          const uint32_t b0 = a0 + C::kA * C::kABytes;
+#pragma unroll
+          for (int k = 0; k < BK / UK; ++k) {
+            const uint32_t acc = (kb | k) != 0;
+            umma_bf16(d0, sw128_desc(a0 + k * UK * 2), sw128_desc(b0 + k * UK * 2), idesc, acc);
+            if (MODE == kGateUp)
+              umma_bf16(d0 + NT, sw128_desc(a0 + C::kABytes + k * UK * 2),
+                        sw128_desc(b0 + k * UK * 2), idesc, acc);
+          }
+          umma_commit(&empty[stage]);
+          if (++stage == C::kStages) { stage = 0; phase ^= 1; }
+        }
+        if (ok) umma_commit(&tfull[buf]);
+      }
+      if (!ok) {
+        record_error(st, MOE_ERR_DEVICE_TIMEOUT, 110 + MODE);
+        *abort_flag = 1;
+      }
+    }
+  } else {
+    // ------------------------------------------------------ epilogue
+    const int quarter = warp & 3;  // TMEM lanes this warp may read
+    const int r_in = quarter * 32 + lane;
+    const bool has_lb = !(lbeta == 0.0f || lbeta != lbeta);
+    const float b_eff = (beta == 0.0f || beta != beta) ? 1.0f : beta;
+    int local = 0;
+    for (int64_t u = blockIdx.x; u < total_units; u += gridDim.x, ++local) {
+      const Unit w = decode_unit(u, RB, tile_start, offsets, E);
+      const int buf = local & 1;
+      const uint32_t tphase = (local >> 1) & 1;
+      if (!mbar_wait(&tfull[buf], tphase, abort_flag)) {
+        if (lane == 0) record_error(st, MOE_ERR_DEVICE_TIMEOUT, 120 + MODE);
+        *abort_flag = 1;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + buf * C::kBufCols;
+      const int m = w.rb * BM + r_in;
+      __nv_bfloat16* col = out + m;
+      for (int c0 = 0; c0 < w.nrows; c0 += 16) {
+        float v[16];
+        tmem_ld16(taddr + c0, v);
+        if (MODE == kGateUp) {
+          float uu[16];
+          tmem_ld16(taddr + NT + c0, uu);
+#pragma unroll
+          for (int j = 0; j < 16; ++j)
+            v[j] = act_kind == MOE_ACT_SITU ? situ_mul(v[j], uu[j], b_eff, lbeta, has_lb)
+                                            : silu_mul(v[j], uu[j]);
+        }
+        const int lim = w.nrows - c0 < 16 ? w.nrows - c0 : 16;
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+          if (j < lim) col[(int64_t)(w.row0 + c0 + j) * M_rows] = __float2bfloat16_rn(v[j]);
+      }
+      tc_fence_before();
+      mbar_arrive(&tempty[buf]);
+    }
+  }
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
+                 "r"(C::kTmemCols));
+  }
+}
+
+// Token tiles per expert and their prefix: tile_start[e] = sum_{e'<e}
+// ceil(n_e'/NT), tile_start[E] = total.  Inconsistent offsets are recorded
+// and give the expert no tile, so the GEMM never reads outside xs.
+__global__ void __launch_bounds__(1024) k_tiles(const int32_t* __restrict__ offsets, int E,
+                                                int64_t S, int32_t* __restrict__ tile_start,
+                                                DeviceStatus* st) {
+  __shared__ int32_t warp_tot[32];
+  const int e = threadIdx.x, lane = e & 31, warp = e >> 5;
+  int32_t n = 0;
+  if (e < E) {
+    const int32_t a = offsets[e], b = offsets[e + 1];
+    const bool bad = a < 0 || b < a || b > S || (e == 0 && a != 0) || (e == E - 1 && b != S);
+    if (bad) record_error(st, MOE_ERR_DEVICE_BOUNDS, 30);
+    else n = (b - a + NT - 1) / NT;
+  }
+  int32_t v = n;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int32_t o = __shfl_up_sync(0xffffffffu, v, off);
+    if (lane >= off) v += o;
+  }
+  if (lane == 31) warp_tot[warp] = v;
+  __syncthreads();
+  if (warp == 0) {
+    int32_t w = warp_tot[lane];
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int32_t o = __shfl_up_sync(0xffffffffu, w, off);
+      if (lane >= off) w += o;
+    }
+    warp_tot[lane] = w;
+  }
+  __syncthreads();
+  const int32_t excl = v - n + (warp > 0 ? warp_tot[warp - 1] : 0);
+  if (e < E) {
+    tile_start[e] = excl;
+    if (e == E - 1) tile_start[E] = excl + n;
+  }
+}
+
+// ------------------------------------------------------------ tensor maps
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static bool tried = false;
+  if (!tried) {
+    tried = true;
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// [batch, rows, cols] bf16, box cols=64 x rows=box_rows x 1
+bool make_map_3d(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, uint64_t batch,
+                 uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {cols, rows, batch};
+  cuuint64_t strides[2] = {cols * 2, cols * rows * 2};
+  cuuint32_t box[3] = {(cuuint32_t)BK, box_rows, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
+            es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool make_map_2d(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows,
+                 uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * 2};
+  cuuint32_t box[2] = {(cuuint32_t)BK, box_rows};
+  cuuint32_t es[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+            es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int MODE>
+cudaError_t launch_gemm(const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorMap& b,
+                        const int32_t* offsets, const int32_t* tile_start, int E, int M_rows,
+                        int Kdim, __nv_bfloat16* out, const moe_act_cfg& act, DeviceStatus* st,
+                        cudaStream_t s) {
+  using C = Cfg<MODE>;
+  static bool attr_set[64] = {false};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && !attr_set[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(k_expert_gemm<MODE>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)C::kSmem);
+    if (e != cudaSuccess) return e;
+    attr_set[dev] = true;
+  }
+  k_expert_gemm<MODE><<<dev_info()->sm_count, kThreads, C::kSmem, s>>>(
+      a0, a1, b, offsets, tile_start, E, M_rows, Kdim, out, act.kind, act.beta, act.linear_beta,
+      st);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+size_t expert_scratch_bytes(int64_t S, int E, int F) {
+  return align_up(sizeof(int32_t) * (size_t)(E + 1), 256) +
+         align_up(sizeof(__nv_bfloat16) * (size_t)S * (size_t)F, 256);
+}
+
+int expert_ffn_run(const __nv_bfloat16* xs, const int32_t* offsets, int E, int64_t S, int d_e,
+                   int F, const __nv_bfloat16* w1, const __nv_bfloat16* w3,
+                   const __nv_bfloat16* w2, const moe_act_cfg& act, __nv_bfloat16* y,
+                   void* scratch, DeviceStatus* st, cudaStream_t s, cudaEvent_t after_gate_up) {
+  int32_t* tile_start = static_cast<int32_t*>(scratch);
+  __nv_bfloat16* h = reinterpret_cast<__nv_bfloat16*>(
+      static_cast<uint8_t*>(scratch) + align_up(sizeof(int32_t) * (size_t)(E + 1), 256));
+  CUtensorMap mw1, mw3, mw2, mxs, mh;
+  if (!make_map_3d(&mw1, w1, d_e, F, E, BM) || !make_map_3d(&mw3, w3, d_e, F, E, BM) ||
+      !make_map_3d(&mw2, w2, F, d_e, E, BM) || !make_map_2d(&mxs, xs, d_e, S, kBoxRows) ||
+      !make_map_2d(&mh, h, F, S, kBoxRows))
+    return MOE_ERR_CUDA;
+  k_tiles<<<1, 1024, 0, s>>>(offsets, E, S, tile_start, st);
+  if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
+  if (launch_gemm<kGateUp>(mw1, mw3, mxs, offsets, tile_start, E, F, d_e, h, act, st, s) !=
+      cudaSuccess)
+    return MOE_ERR_CUDA;
+  if (after_gate_up && cudaEventRecord(after_gate_up, s) != cudaSuccess) return MOE_ERR_CUDA;
+  if (launch_gemm<kDown>(mw2, mw2, mh, offsets, tile_start, E, d_e, F, y, act, st, s) !=
+      cudaSuccess)
+    return MOE_ERR_CUDA;
+  return MOE_OK;
+}
+
+}  // namespace moe

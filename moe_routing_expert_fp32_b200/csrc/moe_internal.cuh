@@ -1,0 +1,72 @@
+// moe_internal.cuh -- definitions shared by the kernels of libmoe (not part of
+// the public ABI).  sm_100a only.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "moe.h"
+
+namespace moe {
+
+// ------------------------------------------------------------ status word
+// The first 256 bytes of every workspace; kernels record the first error.
+struct DeviceStatus {
+  int code;       // 0 or a negative moe_status
+  int detail;     // kernel-specific: where it happened
+};
+constexpr size_t kStatusBytes = 256;
+
+__device__ __forceinline__ void record_error(DeviceStatus* st, int code, int detail) {
+  if (st && atomicCAS(&st->code, 0, code) == 0) st->detail = detail;
+}
+
+// Bounded waits: ~2^28 polls is seconds on any healthy GPU; a wait that runs
+// out records MOE_ERR_DEVICE_TIMEOUT and gives up instead of hanging.
+constexpr uint32_t kSpinLimit = 1u << 28;
+
+inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+// --------------------------------------------------------- kernel launches
+// (all enqueue on `stream`, no synchronisation)
+
+// router.cu
+int route_splits(int64_t N, int E, int d_r);
+size_t route_partial_bytes(int64_t N, int E, int d_r);
+cudaError_t launch_gate_partial(const __nv_bfloat16* x, int64_t N, int d_r, const float* W, int E,
+                                int splits, float* part, cudaStream_t s);
+cudaError_t launch_select(const float* part, int splits, int64_t N, const float* bias,
+                          const moe_route_cfg& cfg, int32_t* idx, float* w, DeviceStatus* st,
+                          cudaStream_t s);
+
+// dispatch.cu
+int dispatch_chunks(int64_t S);
+size_t dispatch_scratch_bytes(int64_t S, int E);
+cudaError_t launch_dispatch(const int32_t* idx, int64_t N, int K, int E, const __nv_bfloat16* x_e,
+                            int d_e, int32_t* counts, int32_t* offsets, int32_t* perm,
+                            int32_t* pos, __nv_bfloat16* xs, int32_t* scratch, DeviceStatus* st,
+                            cudaStream_t s);
+
+// expert_gemm.cu
+size_t expert_scratch_bytes(int64_t S, int E, int F);
+int expert_ffn_run(const __nv_bfloat16* xs, const int32_t* offsets, int E, int64_t S, int d_e,
+                   int F, const __nv_bfloat16* w1, const __nv_bfloat16* w3,
+                   const __nv_bfloat16* w2, const moe_act_cfg& act, __nv_bfloat16* y,
+                   void* scratch, DeviceStatus* st, cudaStream_t s, cudaEvent_t after_gate_up);
+
+// combine.cu
+cudaError_t launch_combine(const __nv_bfloat16* y, const int32_t* pos, const float* w, int64_t N,
+                           int K, int d_e, int64_t S, __nv_bfloat16* out, DeviceStatus* st,
+                           cudaStream_t s);
+
+// device properties, read once per device
+struct DevInfo {
+  int sm_count;
+  int cc_major;
+  int cc_minor;
+  size_t smem_optin;
+};
+const DevInfo* dev_info();
+
+}  // namespace moe

@@ -1,0 +1,231 @@
+// router.cu -- the fp32 router of the MoE layer.
+//
+// Follows "Kimi K2 · Affinities", gate-forward excerpt (MoEGate.forward with
+// noaux_tc) and "DeepSeek-V3.2-Exp · Affinities", gate-forward excerpt
+// (Gate.forward):
+//   k_gate_partial : logits = x . W^T in fp32 (x upcast from bf16, W fp32),
+//                    split over d_r into `splits` partial sums so that decode
+//                    batches still fill the GPU; partials summed in split order.
+//   k_select       : one warp per token: sigmoid, + bias, group top-2 sums,
+//                    top-TG groups (others -> -inf), top-K experts by
+//                    (score desc, index asc), unbiased weights, renormalise
+//                    (sequential fp32 sum over k + 1e-20), route scale.
+// Every fp32 step of k_select is an explicit round-to-nearest intrinsic, so no
+// multiply-add is fused and the result is the IEEE result of the page's ops.
+#include <math.h>
+
+#include "moe_internal.cuh"
+
+namespace moe {
+namespace {
+
+constexpr int GT = 64;   // tokens per tile
+constexpr int GE = 64;   // experts per tile
+constexpr int GK = 32;   // k per smem stage
+constexpr float kNegInf = -INFINITY;
+
+__global__ void __launch_bounds__(256) k_gate_partial(const __nv_bfloat16* __restrict__ x,
+                                                      int64_t N, int d,
+                                                      const float* __restrict__ W, int E,
+                                                      int cps, float* __restrict__ part) {
+  __shared__ __align__(16) float xs[GK][GT];
+  __shared__ __align__(16) float wsm[GK][GE];
+  const int tid = threadIdx.x;
+  const int tx = tid & 15, ty = tid >> 4;
+  const int64_t t0 = (int64_t)blockIdx.y * GT;
+  const int e0 = blockIdx.x * GE;
+  const int nk = d / GK;
+  const int kc0 = blockIdx.z * cps;
+  const int kc1 = min(nk, kc0 + cps);
+  float acc[4][4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
+
+  for (int kc = kc0; kc < kc1; ++kc) {
+    const int k0 = kc * GK;
+    {  // x tile: 64 tokens x 32 k (bf16 -> fp32), one 16-byte load per thread
+      const int tok = tid >> 2, kk = (tid & 3) * 8;
+      uint4 v = make_uint4(0, 0, 0, 0);
+      if (t0 + tok < N) v = *reinterpret_cast<const uint4*>(x + (t0 + tok) * d + k0 + kk);
+      const __nv_bfloat16* h = reinterpret_cast<const __nv_bfloat16*>(&v);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) xs[kk + j][tok] = __bfloat162float(h[j]);
+    }
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {  // W tile: 64 experts x 32 k fp32
+      const int i = tid + 256 * r;
+      const int ex = i >> 3, kq = (i & 7) * 4;
+      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (e0 + ex < E) v = *reinterpret_cast<const float4*>(W + (int64_t)(e0 + ex) * d + k0 + kq);
+      wsm[kq + 0][ex] = v.x;
+      wsm[kq + 1][ex] = v.y;
+      wsm[kq + 2][ex] = v.z;
+      wsm[kq + 3][ex] = v.w;
+    }
+    __syncthreads();
+#pragma unroll 8
+    for (int k = 0; k < GK; ++k) {
+      const float4 a = *reinterpret_cast<const float4*>(&xs[k][ty * 4]);
+      const float4 b = *reinterpret_cast<const float4*>(&wsm[k][tx * 4]);
+      const float av[4] = {a.x, a.y, a.z, a.w};
+      const float bv[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
+    }
+    __syncthreads();
+  }
+  float* out = part + (int64_t)blockIdx.z * N * E;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int64_t t = t0 + ty * 4 + i;
+    if (t >= N) continue;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int e = e0 + tx * 4 + j;
+      if (e < E) out[t * E + e] = acc[i][j];
+    }
+  }
+}
+
+// "a ranks before b": larger value first, ties to the lower index.
+__device__ __forceinline__ bool ranks_before(float va, int ia, float vb, int ib) {
+  return va > vb || (va == vb && ia < ib);
+}
+
+__device__ __forceinline__ void warp_best(float& v, int& i) {
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+    const float ov = __shfl_xor_sync(0xffffffffu, v, off);
+    const int oi = __shfl_xor_sync(0xffffffffu, i, off);
+    if (ranks_before(ov, oi, v, i)) { v = ov; i = oi; }
+  }
+}
+
+constexpr int kSelWarps = 4;
+
+__global__ void __launch_bounds__(32 * kSelWarps) k_select(
+    const float* __restrict__ part, int splits, int64_t N, int E, const float* __restrict__ bias,
+    int G, int TG, int K, int norm, float route_scale, int32_t* __restrict__ idx_out,
+    float* __restrict__ w_out, DeviceStatus* st) {
+  extern __shared__ float sm[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  float* s_s = sm + warp * 2 * E;
+  float* s_c = s_s + E;
+  const int64_t split_stride = N * (int64_t)E;
+  for (int64_t t = (int64_t)blockIdx.x * kSelWarps + warp; t < N;
+       t += (int64_t)gridDim.x * kSelWarps) {
+    const float* p = part + t * E;
+    for (int e = lane; e < E; e += 32) {
+      float L = p[e];
+      for (int z = 1; z < splits; ++z) L = __fadd_rn(L, p[z * split_stride + e]);
+      // sigmoid: fp32 rounding of 1/(1+exp(-L)) evaluated in double
+      const float s = (float)(1.0 / (1.0 + exp(-(double)L)));
+      s_s[e] = s;
+      s_c[e] = bias ? __fadd_rn(s, bias[e]) : s;
+    }
+    __syncwarp();
+    if (G > 1) {
+      const int gsz = E / G;
+      float gs = kNegInf;
+      if (lane < G) {
+        float a = kNegInf, b = kNegInf;
+        for (int i = 0; i < gsz; ++i) {
+          const float v = s_c[lane * gsz + i];
+          if (v > a) { b = a; a = v; }
+          else if (v > b) { b = v; }
+        }
+        gs = __fadd_rn(a, b);
+      }
+      bool kept = false;
+      for (int r = 0; r < TG; ++r) {
+        float v = (lane < G && !kept) ? gs : kNegInf;
+        int i = (lane < G && !kept) ? lane : 0x7fffffff;
+        warp_best(v, i);
+        if (lane == i) kept = true;
+      }
+      const unsigned keptmask = __ballot_sync(0xffffffffu, kept);
+      for (int e = lane; e < E; e += 32)
+        if (!((keptmask >> (e / gsz)) & 1u)) s_c[e] = kNegInf;
+      __syncwarp();
+    }
+    unsigned chosen = 0;
+    int my_e = 0;
+    for (int k = 0; k < K; ++k) {
+      float bv = kNegInf;
+      int bi = 0x7fffffff;
+      for (int i = 0, e = lane; e < E; ++i, e += 32) {
+        if ((chosen >> i) & 1u) continue;
+        const float v = s_c[e];
+        if (ranks_before(v, e, bv, bi)) { bv = v; bi = e; }
+      }
+      warp_best(bv, bi);
+      if (bi == 0x7fffffff) {  // cannot happen for a validated config
+        record_error(st, MOE_ERR_DEVICE_BOUNDS, 1);
+        bi = 0;
+      }
+      if ((bi & 31) == lane) chosen |= 1u << (bi >> 5);
+      if (lane == k) my_e = bi;
+    }
+    float wk = (lane < K) ? s_s[my_e] : 0.f;
+    if (K > 1 && norm) {
+      float den = __shfl_sync(0xffffffffu, wk, 0);
+      for (int k = 1; k < K; ++k) den = __fadd_rn(den, __shfl_sync(0xffffffffu, wk, k));
+      den = __fadd_rn(den, 1e-20f);
+      wk = __fdiv_rn(wk, den);
+    }
+    wk = __fmul_rn(wk, route_scale);
+    if (lane < K) {
+      idx_out[t * K + lane] = my_e;
+      w_out[t * K + lane] = wk;
+    }
+    __syncwarp();
+  }
+}
+
+}  // namespace
+
+int route_splits(int64_t N, int E, int d_r) {
+  int64_t tiles = ((E + GE - 1) / GE) * ((N + GT - 1) / GT);
+  if (tiles < 1) tiles = 1;
+  const int nk = d_r / GK > 0 ? d_r / GK : 1;
+  int64_t want = (296 + tiles - 1) / tiles;
+  int64_t maxs = nk / 4 > 0 ? nk / 4 : 1;
+  if (want > maxs) want = maxs;
+  if (want > 64) want = 64;
+  if (want < 1) want = 1;
+  const int cps = (int)((nk + want - 1) / want);
+  return (nk + cps - 1) / cps;
+}
+
+size_t route_partial_bytes(int64_t N, int E, int d_r) {
+  return align_up(sizeof(float) * (size_t)route_splits(N, E, d_r) * (size_t)N * (size_t)E, 256);
+}
+
+cudaError_t launch_gate_partial(const __nv_bfloat16* x, int64_t N, int d_r, const float* W, int E,
+                                int splits, float* part, cudaStream_t s) {
+  const int nk = d_r / GK;
+  const int cps = (nk + splits - 1) / splits;
+  dim3 grid((E + GE - 1) / GE, (unsigned)((N + GT - 1) / GT), splits);
+  k_gate_partial<<<grid, 256, 0, s>>>(x, N, d_r, W, E, cps, part);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_select(const float* part, int splits, int64_t N, const float* bias,
+                          const moe_route_cfg& cfg, int32_t* idx, float* w, DeviceStatus* st,
+                          cudaStream_t s) {
+  const int E = cfg.num_experts;
+  const size_t smem = sizeof(float) * 2 * E * kSelWarps;
+  int64_t blocks = (N + kSelWarps - 1) / kSelWarps;
+  const int64_t cap = (int64_t)dev_info()->sm_count * 16;
+  if (blocks > cap) blocks = cap;
+  k_select<<<(unsigned)blocks, 32 * kSelWarps, smem, s>>>(
+      part, splits, N, E, bias, cfg.n_group, cfg.topk_group, cfg.top_k, cfg.norm_topk_prob,
+      cfg.route_scale, idx, w, st);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -1,0 +1,147 @@
+"""The C-ABI library loads without a GPU, exports every entry point its header
+declares, and rejects bad arguments on the host before touching CUDA."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "moe.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    from moe_routing_expert_fp32_b200 import build as b
+    b.build()
+    import moe_routing_expert_fp32_b200 as m
+    return m.lib()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    return re.findall(r"MOE_API\s+[\w\s\*]+?\b(moe_\w+)\s*\(", text)
+
+
+def test_header_declares_the_entry_points():
+    names = set(declared_functions())
+    for n in ("moe_route", "moe_dispatch", "moe_expert_ffn", "moe_combine", "moe_forward",
+              "moe_route_from_logits", "moe_workspace_size", "moe_get_status", "moe_strerror"):
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported(L):
+    for name in declared_functions():
+        assert hasattr(L, name), f"{name} declared in moe.h but not exported"
+
+
+def test_binding_names_match_the_header():
+    import moe_routing_expert_fp32_b200 as m
+    assert set(m.EXPORTS) <= set(declared_functions())
+
+
+def _cfg(m, E=16, G=4, TG=2, K=4, rs=2.5):
+    return m._RouteCfg(E, G, TG, K, 1, rs)
+
+
+@pytest.mark.parametrize("E,G,TG,K,code", [
+    (16, 4, 2, 4, -4),    # valid config; fails on the NULL workspace, not on the config
+    (16, 3, 2, 4, -1),    # E not divisible by G
+    (16, 4, 5, 4, -1),    # TG > G
+    (16, 4, 1, 5, -1),    # K > TG * E / G
+    (16, 16, 2, 2, -1),   # one expert per group with G > 1
+    (2048, 1, 1, 8, -2),  # E > 1024
+    (64, 64, 2, 2, -1),   # G > 32 is checked after E/G >= 2 ... E/G = 1 -> invalid
+    (16, 1, 1, 17, -1),   # K > E
+    (32, 1, 1, 17, -2),   # K > 16
+    (0, 1, 1, 1, -1),
+])
+def test_route_config_validation(L, E, G, TG, K, code):
+    import moe_routing_expert_fp32_b200 as m
+    c = _cfg(m, E, G, TG, K)
+    rc = L.moe_route(None, 4, 256, None, None, ctypes.byref(c), None, None, None, 0, None)
+    if code == -4:
+        assert rc == -1  # NULL tensors with N > 0 are caught first
+    else:
+        assert rc == code
+
+
+def test_route_rejects_before_cuda(L):
+    import moe_routing_expert_fp32_b200 as m
+    c = _cfg(m)
+    assert L.moe_route(None, -1, 256, None, None, ctypes.byref(c), None, None, None, 0, None) == -1
+    assert L.moe_route(None, 4, 100, None, None, ctypes.byref(c), None, None, None, 0, None) == -2
+    assert L.moe_route(None, 4, 256, None, None, None, None, None, None, 0, None) == -1
+    # N = 0 with a NULL workspace: workspace error, no CUDA call
+    assert L.moe_route(None, 0, 256, None, None, ctypes.byref(c), None, None, None, 0, None) == -4
+    c.route_scale = float("inf")
+    assert L.moe_route(None, 4, 256, None, None, ctypes.byref(c), None, None, None, 0, None) == -1
+
+
+def test_workspace_checks(L):
+    import moe_routing_expert_fp32_b200 as m
+    c = _cfg(m)
+    need = L.moe_route_workspace_size(64, 256, ctypes.byref(c))
+    assert need >= 256 + 64 * 16 * 4
+    buf = (ctypes.c_uint8 * (need + 512))()
+    base = ctypes.addressof(buf)
+    aligned = (base + 255) // 256 * 256
+    # too small
+    rc = L.moe_route(ctypes.c_void_p(16), 64, 256, ctypes.c_void_p(16), None, ctypes.byref(c),
+                     ctypes.c_void_p(16), ctypes.c_void_p(16), ctypes.c_void_p(aligned), need - 1,
+                     None)
+    assert rc == -4
+    # misaligned
+    rc = L.moe_route(ctypes.c_void_p(16), 64, 256, ctypes.c_void_p(16), None, ctypes.byref(c),
+                     ctypes.c_void_p(16), ctypes.c_void_p(16), ctypes.c_void_p(aligned + 16),
+                     need, None)
+    assert rc == -4
+    # misaligned tensor
+    rc = L.moe_route(ctypes.c_void_p(18), 64, 256, ctypes.c_void_p(16), None, ctypes.byref(c),
+                     ctypes.c_void_p(16), ctypes.c_void_p(16), ctypes.c_void_p(aligned), need,
+                     None)
+    assert rc == -3
+
+
+def test_expert_ffn_shape_limits(L):
+    import moe_routing_expert_fp32_b200 as m
+    a = m._ActCfg(0, 1.0, 0.0)
+    p = ctypes.c_void_p(256)
+    # d_e not a multiple of 128
+    assert L.moe_expert_ffn(p, p, 4, 16, 100, 128, p, p, p, ctypes.byref(a), p, p, 1 << 20,
+                            None) == -2
+    # F not a multiple of 128
+    assert L.moe_expert_ffn(p, p, 4, 16, 128, 96, p, p, p, ctypes.byref(a), p, p, 1 << 20,
+                            None) == -2
+    bad = m._ActCfg(7, 1.0, 0.0)
+    assert L.moe_expert_ffn(p, p, 4, 16, 128, 128, p, p, p, ctypes.byref(bad), p, p, 1 << 20,
+                            None) == -1
+    assert L.moe_expert_ffn(p, p, 4, 16, 128, 128, None, p, p, ctypes.byref(a), p, p, 1 << 20,
+                            None) == -1
+
+
+def test_dispatch_and_combine_validation(L):
+    p = ctypes.c_void_p(256)
+    assert L.moe_dispatch(p, 4, 0, 16, p, 256, p, p, p, p, p, p, 1 << 20, None) == -1
+    assert L.moe_dispatch(p, 4, 17, 16, p, 256, p, p, p, p, p, p, 1 << 20, None) == -2
+    assert L.moe_dispatch(p, 4, 4, 16, p, 250, p, p, p, p, p, p, 1 << 20, None) == -2
+    assert L.moe_combine(p, p, p, 4, 4, 250, p, p, 256, None) == -2
+    assert L.moe_combine(None, p, p, 4, 4, 256, p, p, 256, None) == -1
+
+
+def test_forward_validation(L):
+    import moe_routing_expert_fp32_b200 as m
+    c = _cfg(m)
+    a = m._ActCfg(0, 1.0, 0.0)
+    p = ctypes.c_void_p(256)
+    # x_e NULL but d_e != d_r
+    assert L.moe_forward(p, None, 4, 256, 128, p, None, ctypes.byref(c), p, p, p, 128,
+                         ctypes.byref(a), p, None, None, p, 1 << 30, None, None) == -1
+    sz = L.moe_workspace_size(64, 256, 256, ctypes.byref(c), 128)
+    assert sz > 64 * 4 * 256 * 2 * 2  # holds xs and y
+
+
+def test_strerror(L):
+    for code in range(-8, 1):
+        assert L.moe_strerror(code)
+    assert L.moe_strerror(-99) == b"unknown moe_status"

@@ -1,0 +1,347 @@
+"""Parity of every C-ABI entry point with the CPU reference, on the GPU.
+
+Both sides get the same seeded inputs (host twin -> reference, device twin or a
+copy of the host array -> CUDA library).  Bars:
+  * selection from supplied logits: indices and weights bit-exact;
+  * end-to-end routing: index sets equal for tokens whose biased-score margin
+    exceeds 1e-5, weights within 1e-5 relative;
+  * dispatch: counts, offsets, perm, pos exact; gathered rows bitwise;
+  * combine: bitwise;
+  * expert MLP and layer output: relative L2 <= 2e-2 in bf16.
+Full-size workloads are checked on sampled tokens / experts the reference can
+compute in seconds; the kernels always run at the full size.
+"""
+import numpy as np
+import pytest
+
+import oracle
+import synth
+from synth.workloads import WORKLOADS, host_inputs, host_expert, scaled
+from tests.gpu_util import (MARGIN, REL_L2_OUT, W_REL, dev_bf16, host_bf16, random_topk, rel_l2,
+                            ulp_diff)
+
+pytestmark = pytest.mark.gpu
+
+ALL = list(WORKLOADS)
+
+
+@pytest.fixture(scope="module")
+def moe():
+    import torch
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    import moe_routing_expert_fp32_b200 as m
+    m.lib()
+    oracle.set_threads(0)
+    return m
+
+
+def rcfg(m, wl):
+    return m.RouteConfig(wl.E, wl.G, wl.TG, wl.K, wl.route_scale, wl.norm)
+
+
+def acfg(m, wl):
+    return m.ActConfig(wl.act, wl.beta, wl.lbeta)
+
+
+# ------------------------------------------------------ selection from logits
+def _logits(wl, N, mode):
+    if mode == "normal":
+        return synth.host_normal_f32(11, 9, (N, wl.E), 1.7)
+    # exact ties: few distinct logits
+    raw = synth.host_raw(11, 9, N * wl.E).reshape(N, wl.E)
+    return (np.float32(-1.0) + np.float32(0.25) * (raw % 9).astype(np.float32)).astype(np.float32)
+
+
+@pytest.mark.parametrize("name", ALL)
+@pytest.mark.parametrize("mode", ["normal", "ties"])
+def test_route_from_logits_bit_exact(moe, name, mode):
+    import torch
+    wl = WORKLOADS[name]
+    N = wl.N
+    L = _logits(wl, N, mode)
+    b = host_inputs(scaled(wl, N=1))["bias"]
+    if mode == "ties":
+        b = np.round(b * 200).astype(np.float32) / np.float32(200)  # few distinct bias values
+    idx_r, w_r, _ = oracle.route_from_logits(L, b, wl.G, wl.TG, wl.K, wl.route_scale, wl.norm)
+    idx_g, w_g = moe.route_from_logits(torch.from_numpy(L).cuda(), torch.from_numpy(b).cuda(),
+                                       rcfg(moe, wl))
+    assert np.array_equal(idx_g.cpu().numpy(), idx_r)
+    assert np.array_equal(w_g.cpu().numpy().view(np.uint32), w_r.view(np.uint32))
+
+
+@pytest.mark.parametrize("E,G,TG,K,norm", [(16, 4, 2, 4, True), (8, 1, 1, 1, True),
+                                           (64, 8, 8, 16, True), (1024, 32, 3, 16, True),
+                                           (12, 3, 2, 6, False), (6, 1, 1, 6, True)])
+def test_route_from_logits_shapes(moe, E, G, TG, K, norm):
+    import torch
+    rng = np.random.default_rng(E * 100 + K)
+    N = 777
+    L = rng.choice(np.array([-0.5, 0.0, 0.5, 1.0], np.float32), size=(N, E))
+    L[: N // 2] = rng.standard_normal((N // 2, E)).astype(np.float32)
+    b = rng.choice(np.array([0.0, 0.01, -0.01], np.float32), size=E)
+    idx_r, w_r, _ = oracle.route_from_logits(L, b, G, TG, K, 2.0, norm)
+    cfg = moe.RouteConfig(E, G, TG, K, 2.0, norm)
+    idx_g, w_g = moe.route_from_logits(torch.from_numpy(L).cuda(), torch.from_numpy(b).cuda(), cfg)
+    assert np.array_equal(idx_g.cpu().numpy(), idx_r)
+    assert np.array_equal(w_g.cpu().numpy().view(np.uint32), w_r.view(np.uint32))
+    # no bias
+    idx_r, w_r, _ = oracle.route_from_logits(L, None, G, TG, K, 2.0, norm)
+    idx_g, w_g = moe.route_from_logits(torch.from_numpy(L).cuda(), None, cfg)
+    assert np.array_equal(idx_g.cpu().numpy(), idx_r)
+    assert np.array_equal(w_g.cpu().numpy().view(np.uint32), w_r.view(np.uint32))
+
+
+# ----------------------------------------------------------- routing end to end
+def _check_routing(idx_g, w_g, idx_r, w_r, margin):
+    ok = margin > MARGIN
+    assert ok.mean() > 0.5
+    for t in np.nonzero(ok)[0]:
+        assert set(idx_g[t].tolist()) == set(idx_r[t].tolist()), t
+        og = dict(zip(idx_g[t].tolist(), w_g[t].tolist()))
+        for e, wr in zip(idx_r[t].tolist(), w_r[t].tolist()):
+            assert abs(og[e] - wr) <= W_REL * abs(wr), (t, e, og[e], wr)
+    return int((~ok).sum())
+
+
+@pytest.mark.parametrize("name", ALL)
+def test_route_end_to_end(moe, name):
+    import torch
+    wl = WORKLOADS[name]
+    inp = host_inputs(wl)
+    x, W, b = inp["x"], inp["W"], inp["bias"]
+    idx_g, w_g = moe.route(dev_bf16(x), torch.from_numpy(W).cuda(), torch.from_numpy(b).cuda(),
+                           rcfg(moe, wl))
+    idx_g, w_g = idx_g.cpu().numpy(), w_g.cpu().numpy()
+    rows = np.arange(wl.N)
+    if wl.N > 1024:  # the reference routes a sample of the batch
+        rows = np.unique(np.concatenate([np.arange(256), np.arange(wl.N - 256, wl.N),
+                                         np.random.default_rng(0).choice(wl.N, 512, False)]))
+    idx_r, w_r, margin = oracle.route(np.ascontiguousarray(x[rows]), W, b, wl.G, wl.TG, wl.K,
+                                      wl.route_scale, wl.norm)
+    n_low = _check_routing(idx_g[rows], w_g[rows], idx_r, w_r, margin)
+    print(f"{name}: {len(rows)} tokens checked, {n_low} at or below the margin")
+
+
+# ------------------------------------------------------------------ dispatch
+def _dispatch_case(moe, N, K, E, d, idx):
+    import torch
+    x = synth.host_normal_bf16(3, 1, (N, d), 1.0)
+    c_g, o_g, p_g, q_g, xs_g = moe.dispatch(torch.from_numpy(idx).cuda(), dev_bf16(x), E)
+    c_r, o_r, p_r, q_r = oracle.dispatch(idx, E)
+    assert np.array_equal(c_g.cpu().numpy(), c_r)
+    assert np.array_equal(o_g.cpu().numpy(), o_r)
+    assert np.array_equal(p_g.cpu().numpy(), p_r)
+    assert np.array_equal(q_g.cpu().numpy(), q_r)
+    S = N * K
+    rows = np.arange(S) if S <= 4096 else np.unique(
+        np.concatenate([np.arange(1024), np.arange(S - 1024, S),
+                        np.random.default_rng(1).choice(S, 2048, False)]))
+    xs_rows = host_bf16(xs_g[torch.from_numpy(rows).cuda()])
+    assert np.array_equal(xs_rows, x[p_r[rows] // K])
+
+
+@pytest.mark.parametrize("name", ALL)
+def test_dispatch(moe, name):
+    wl = WORKLOADS[name]
+    rng = np.random.default_rng(21)
+    idx = random_topk(wl.N, wl.K, wl.E, rng, skew=1.2 if wl.skew else 0.0)
+    _dispatch_case(moe, wl.N, wl.K, wl.E, wl.d_e, idx)
+
+
+@pytest.mark.parametrize("N,K,E", [(1, 8, 384), (1000, 1, 16), (333, 3, 7), (5000, 16, 1024)])
+def test_dispatch_edge_shapes(moe, N, K, E):
+    rng = np.random.default_rng(N + K + E)
+    _dispatch_case(moe, N, K, E, 128, random_topk(N, K, E, rng, skew=1.5))
+
+
+def test_dispatch_all_slots_one_expert(moe):
+    N, K, E = 3000, 1, 64
+    _dispatch_case(moe, N, K, E, 256, np.full((N, K), 17, np.int32))
+
+
+def test_dispatch_out_of_range_index_is_reported_not_faulted(moe):
+    import torch
+    N, K, E, d = 64, 4, 16, 128
+    idx = random_topk(N, K, E, np.random.default_rng(5))
+    idx[3, 1] = E + 5
+    idx[40, 0] = -2
+    ws = moe.workspace(1 << 16)
+    c, o, p, q, xs = moe.dispatch(torch.from_numpy(idx).cuda(), dev_bf16(
+        synth.host_normal_bf16(0, 1, (N, d), 1.0)), E, ws=ws)
+    assert moe.get_status(ws) == -7
+    assert int(o[-1].item()) == N * K - 2
+    assert q[3 * K + 1].item() == -1 and q[40 * K].item() == -1
+
+
+# ---------------------------------------------------------------- combine
+@pytest.mark.parametrize("name", ALL)
+def test_combine_bitwise(moe, name):
+    import torch
+    wl = WORKLOADS[name]
+    N, K, d = wl.N, wl.K, wl.d_e
+    S = N * K
+    y = synth.host_normal_bf16(4, 10, (S, d), 0.05)
+    pos = np.random.default_rng(2).permutation(S).astype(np.int32)
+    w = synth.host_uniform_f32(4, 11, (N, K), 0.0, 0.7)
+    out_g = host_bf16(moe.combine(dev_bf16(y), torch.from_numpy(pos).cuda(),
+                                  torch.from_numpy(w).cuda()))
+    out_r = oracle.combine(y, pos, w, K)
+    assert np.array_equal(out_g, out_r)
+
+
+# ------------------------------------------------------------- expert MLP
+def _expert_case(moe, wl, counts, sample_experts, rows_per_expert=48, seed=5):
+    """Run moe_expert_ffn on all segments; check sampled experts' rows."""
+    import torch
+    E, F, d = wl.E, wl.F, wl.d_e
+    offsets = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
+    S = int(offsets[-1])
+    xs_d = synth.dev_normal_bf16(torch.empty((S, d), dtype=torch.bfloat16, device="cuda"),
+                                 seed, 12, 1.0)
+    dev = synth.workloads.dev_inputs(wl, experts=True)
+    y_d = moe.expert_ffn(xs_d, torch.from_numpy(offsets).cuda(), dev["w1"], dev["w3"], dev["w2"],
+                         acfg(moe, wl))
+    torch.cuda.synchronize()
+    worst = 0.0
+    for e in sample_experts:
+        a, b = int(offsets[e]), int(offsets[e + 1])
+        if b == a:
+            continue
+        n = b - a
+        if n <= rows_per_expert:
+            rows = np.arange(a, b)
+        else:  # first tile, a tile boundary, the ragged tail
+            cand = [a, a + 1, a + 127, a + 128, a + 129, b - 2, b - 1]
+            cand += list(np.random.default_rng(e).choice(np.arange(a, b), rows_per_expert - 7))
+            rows = np.unique(np.clip(cand, a, b - 1))
+        xs_rows = np.stack([synth.host_normal_bf16(seed, 12, (d,), 1.0, start=int(r) * d)
+                            for r in rows])
+        w1, w3, w2 = host_expert(wl, e)
+        y_r = oracle.expert_ffn(xs_rows, w1, w3, w2, wl.act, wl.beta, wl.lbeta)
+        y_g = host_bf16(y_d[torch.from_numpy(rows).cuda()])
+        err = rel_l2(y_g, y_r)
+        u = ulp_diff(y_g, y_r)
+        print(f"expert {e}: rows {len(rows)}/{n} rel_l2 {err:.2e} max_ulp {u.max()} "
+              f"frac>1ulp {(u > 1).mean():.2e}")
+        assert err <= REL_L2_OUT
+        worst = max(worst, err)
+    return worst
+
+
+@pytest.mark.parametrize("name", ALL)
+def test_expert_ffn(moe, name):
+    wl = WORKLOADS[name]
+    rng = np.random.default_rng(31)
+    idx = random_topk(wl.N, wl.K, wl.E, rng, skew=1.2 if wl.skew else 0.0)
+    counts = np.bincount(idx.ravel(), minlength=wl.E)
+    order = np.argsort(-counts, kind="stable")
+    nz = order[counts[order] > 0]
+    sample = sorted({int(nz[0]), int(nz[len(nz) // 2]), int(nz[-1])})
+    if wl.E <= 16:
+        sample = list(range(wl.E))
+    _expert_case(moe, wl, counts, sample)
+
+
+def test_expert_ffn_one_long_segment_and_empty_experts(moe):
+    """All rows on one expert: a segment many tiles long with a ragged tail."""
+    wl = scaled(WORKLOADS["tiny"], E=8)
+    counts = np.zeros(8, np.int64)
+    counts[5] = 1000
+    _expert_case(moe, wl, counts, [5], rows_per_expert=64)
+
+
+def test_expert_ffn_situ_shapes(moe):
+    wl = scaled(WORKLOADS["k3_latent_decode"], E=24, d_e=256, F=384, N=200)
+    counts = np.random.default_rng(3).integers(0, 140, 24)
+    counts[[2, 7]] = 0
+    _expert_case(moe, wl, counts, list(range(24)), rows_per_expert=200)
+
+
+# ------------------------------------------------------------ whole layer
+def _forward(moe, wl, dev):
+    import torch
+    N = wl.N
+    idx = torch.empty((N, wl.K), dtype=torch.int32, device="cuda")
+    w = torch.empty((N, wl.K), dtype=torch.float32, device="cuda")
+    out = moe.forward(dev["x"], dev["W"], dev["bias"], rcfg(moe, wl), dev["w1"], dev["w3"],
+                      dev["w2"], acfg(moe, wl), x_e=dev["x_e"] if wl.latent else None,
+                      topk_idx=idx, topk_w=w)
+    return host_bf16(out), idx.cpu().numpy(), w.cpu().numpy()
+
+
+@pytest.mark.parametrize("name", ALL)
+def test_forward_end_to_end(moe, name):
+    wl = WORKLOADS[name]
+    dev = synth.workloads.dev_inputs(wl)
+    out_g, idx_g, w_g = _forward(moe, wl, dev)
+    inp = host_inputs(wl)
+    n_tok = wl.N if wl.N <= 64 else 12
+    toks = np.arange(wl.N) if n_tok == wl.N else np.unique(
+        np.concatenate([[0, wl.N - 1], np.random.default_rng(7).choice(wl.N, n_tok - 2, False)]))
+    x = np.ascontiguousarray(inp["x"][toks])
+    xe = np.ascontiguousarray(inp["x_e"][toks])
+    idx_r, w_r, margin = oracle.route(x, inp["W"], inp["bias"], wl.G, wl.TG, wl.K,
+                                      wl.route_scale, wl.norm)
+    _check_routing(idx_g[toks], w_g[toks], idx_r, w_r, margin)
+    keep = margin > MARGIN
+    cache = {}
+    out_r = np.zeros((len(toks), wl.d_e), np.uint16)
+    for i in range(len(toks)):
+        ys = []
+        for k in range(wl.K):
+            e = int(idx_r[i, k])
+            if e not in cache:
+                cache[e] = host_expert(wl, e)
+            w1, w3, w2 = cache[e]
+            ys.append(oracle.expert_ffn(xe[i:i + 1], w1, w3, w2, wl.act, wl.beta, wl.lbeta)[0])
+        out_r[i] = oracle.combine(np.stack(ys), np.arange(wl.K, dtype=np.int32),
+                                  np.ascontiguousarray(w_r[i:i + 1]), wl.K)[0]
+    err = rel_l2(out_g[toks][keep], out_r[keep])
+    print(f"{name}: {keep.sum()}/{len(toks)} tokens, rel_l2 {err:.2e}")
+    assert err <= REL_L2_OUT
+
+
+def test_forward_tiny_matches_reference_moe_infer_exactly_where_routing_agrees(moe):
+    """At the tiny size the whole batch goes through the reference's sorted
+    moe_infer; compare every token with margin > 1e-5."""
+    wl = WORKLOADS["tiny"]
+    dev = synth.workloads.dev_inputs(wl)
+    out_g, idx_g, w_g = _forward(moe, wl, dev)
+    inp = host_inputs(wl)
+    from synth.workloads import host_experts_all
+    w1, w3, w2 = host_experts_all(wl)
+    idx_r, w_r, margin = oracle.route(inp["x"], inp["W"], inp["bias"], wl.G, wl.TG, wl.K,
+                                      wl.route_scale)
+    out_r = oracle.moe_infer(inp["x_e"], idx_r, w_r, w1, w3, w2, wl.act)
+    keep = margin > MARGIN
+    err = rel_l2(out_g[keep], out_r[keep])
+    u = ulp_diff(out_g[keep], out_r[keep])
+    print(f"tiny: rel_l2 {err:.2e}, max ulp {u.max()}, frac>1ulp {(u > 1).mean():.2e}")
+    assert err <= REL_L2_OUT
+
+
+def test_forward_deterministic_and_empty(moe):
+    import torch
+    wl = WORKLOADS["dsv32_decode"]
+    dev = synth.workloads.dev_inputs(wl)
+    a, _, _ = _forward(moe, wl, dev)
+    b, _, _ = _forward(moe, wl, dev)
+    assert np.array_equal(a, b)
+    # N = 0 is a valid empty call
+    x0 = torch.empty((0, wl.d_r), dtype=torch.bfloat16, device="cuda")
+    out = moe.forward(x0, dev["W"], dev["bias"], rcfg(moe, wl), dev["w1"], dev["w3"], dev["w2"],
+                      acfg(moe, wl))
+    assert out.shape == (0, wl.d_e)
+
+
+def test_forward_single_token(moe):
+    wl = scaled(WORKLOADS["k2_prefill"], N=1)
+    dev = synth.workloads.dev_inputs(wl)
+    out_g, idx_g, w_g = _forward(moe, wl, dev)
+    inp = host_inputs(wl)
+    idx_r, w_r, margin = oracle.route(inp["x"], inp["W"], inp["bias"], 1, 1, wl.K,
+                                      wl.route_scale)
+    assert set(idx_g[0]) == set(idx_r[0])
+    ys = [oracle.expert_ffn(inp["x_e"], *host_expert(wl, int(e)))[0] for e in idx_r[0]]
+    out_r = oracle.combine(np.stack(ys), np.arange(wl.K, dtype=np.int32), w_r, wl.K)
+    assert rel_l2(out_g, out_r) <= REL_L2_OUT
