@@ -45,7 +45,21 @@ def parse():
     p.add_argument("--workload", default=DEFAULT_WORKLOAD)
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--no-cpu-baseline", action="store_true")
+    # profiling cases: the same workload with fewer tokens / experts
+    p.add_argument("--tokens", type=int, default=None)
+    p.add_argument("--experts", type=int, default=None)
     return p.parse_args()
+
+
+def workload_of(args):
+    from synth.workloads import WORKLOADS, scaled
+    wl = WORKLOADS[args.workload]
+    kw = {}
+    if args.tokens:
+        kw["N"] = args.tokens
+    if args.experts:
+        kw["E"] = args.experts
+    return scaled(wl, **kw) if kw else wl
 
 
 def load_peaks():
@@ -116,14 +130,31 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
+# ------------------------------------------------------------ multi-rank
+def max_over_ranks(values, world, device="cpu"):
+    """Element-wise max of per-rank timings (the slowest rank sets the step)."""
+    if world <= 1:
+        return list(values)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor(values, dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def aggregate_throughput(tokens_per_rank, world, step_ms_max):
+    """Whole-job routed tokens/s: every rank's tokens over the slowest rank's time."""
+    return world * tokens_per_rank / (step_ms_max * 1e-3)
+
+
 # ---------------------------------------------------------------- our arm
 def run_ours(args, rank, world, local_rank):
     import torch
     import moe_routing_expert_fp32_b200 as moe
     import synth
-    from synth.workloads import WORKLOADS, dev_inputs
+    from synth.workloads import dev_inputs
 
-    wl = WORKLOADS[args.workload]
+    wl = workload_of(args)
     torch.cuda.set_device(local_rank)
     dev = dev_inputs(wl, rank=rank)
     cfg = moe.RouteConfig(wl.E, wl.G, wl.TG, wl.K, wl.route_scale, wl.norm)
@@ -217,13 +248,8 @@ def run_ours(args, rank, world, local_rank):
     h2d = wl.N * wl.d_r * 2 + (wl.N * wl.d_e * 2 if wl.latent else 0)
     d2h = wl.N * wl.d_e * 2
 
-    # max over ranks
-    vals = torch.tensor([ms, statistics.mean(e2e_ms), stage_ms["gate_up"], wall],
-                        dtype=torch.float64, device="cuda")
-    if world > 1:
-        import torch.distributed as dist
-        dist.all_reduce(vals, op=dist.ReduceOp.MAX)
-    ms_max, e2e_max, gu_ms, wall_max = vals.tolist()
+    ms_max, e2e_max, gu_ms, wall_max = max_over_ranks(
+        [ms, statistics.mean(e2e_ms), stage_ms["gate_up"], wall], world, "cuda")
 
     res = {
         "ms": ms_max, "e2e_ms": e2e_max, "stage_ms": stage_ms, "gate_up_ms": gu_ms,
@@ -231,6 +257,22 @@ def run_ours(args, rank, world, local_rank):
         "h2d": h2d, "d2h": d2h, "wall_s": wall_max,
     }
     return wl, res
+
+
+def gate_up_traffic(touched):
+    """DRAM bytes of one gate_up launch from the committed ncu capture of a
+    smaller case, scaled by touched experts; None once the kernel source has
+    changed since the capture."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", "expert_gemm_traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        rec = json.load(f)
+    with open(os.path.join(ROOT, rec["source"]), "rb") as f:
+        if hashlib.sha256(f.read()).hexdigest() != rec["source_sha256"]:
+            return None
+    return (rec["dram_bytes_read"] + rec["dram_bytes_write"]) * touched / rec["touched_experts"]
 
 
 def gate_up_bytes(wl, touched):
@@ -288,10 +330,9 @@ def oracle_sample(wl, n_experts=8):
 
 
 def run_reference(args, rank, world):
-    from synth.workloads import WORKLOADS
     if rank != 0:
         return
-    wl = WORKLOADS[args.workload]
+    wl = workload_of(args)
     for _ in range(args.warmup):
         pass  # the reference has nothing to warm up; steps are timed below
     vals = []
@@ -336,7 +377,7 @@ def main():
     achieved = gate_up_bytes(wl, r["touched"]) / (r["gate_up_ms"] * 1e-3) / 1e9
     line = {
         "metric": METRIC,
-        "value": world * wl.N / (r["ms"] * 1e-3),
+        "value": aggregate_throughput(wl.N, world, r["ms"]),
         "unit": UNIT,
         "n_gpus": world,
         "steps": args.steps,
@@ -354,10 +395,10 @@ def main():
                          "per-step events"},
         "roofline": {"kernel": "expert w1/w3 (gate_up) grouped GEMM", "bound": "hbm",
                      "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                     "frac": achieved / peaks["hbm_gbs"], "traffic": None,
+                     "frac": achieved / peaks["hbm_gbs"], "traffic": gate_up_traffic(r["touched"]),
                      "peak_source": peaks["source"], "touched_experts": r["touched"]},
         "stages_ms": r["stage_ms"],
-        "e2e": {"value": world * wl.N / (r["e2e_ms"] * 1e-3), "unit": UNIT,
+        "e2e": {"value": aggregate_throughput(wl.N, world, r["e2e_ms"]), "unit": UNIT,
                 "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"]},
         "gpu_launches": KERNELS_PER_STEP * args.steps,
         "clocks": r["clocks"],

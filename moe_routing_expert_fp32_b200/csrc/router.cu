@@ -5,7 +5,10 @@
 // (Gate.forward):
 //   k_gate_partial : logits = x . W^T in fp32 (x upcast from bf16, W fp32),
 //                    split over d_r into `splits` partial sums so that decode
-//                    batches still fill the GPU; partials summed in split order.
+//                    batches still fill the GPU.  FMA chains are 32 terms long;
+//                    the 32-term blocks are added with Kahan compensation and
+//                    the split partials in double, which keeps the logit error
+//                    near 1e-7 instead of the ~1e-5 of one 7168-term chain.
 //   k_select       : one warp per token: sigmoid, + bias, group top-2 sums,
 //                    top-TG groups (others -> -inf), top-K experts by
 //                    (score desc, index asc), unbiased weights, renormalise
@@ -37,11 +40,13 @@ __global__ void __launch_bounds__(256) k_gate_partial(const __nv_bfloat16* __res
   const int nk = d / GK;
   const int kc0 = blockIdx.z * cps;
   const int kc1 = min(nk, kc0 + cps);
-  float acc[4][4];
+  // Running sums with Kahan compensation; each 32-wide k block is first
+  // accumulated on its own, so no fp32 chain is longer than 32 terms.
+  float acc[4][4], comp[4][4];
 #pragma unroll
   for (int i = 0; i < 4; ++i)
 #pragma unroll
-    for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
+    for (int j = 0; j < 4; ++j) acc[i][j] = comp[i][j] = 0.f;
 
   for (int kc = kc0; kc < kc1; ++kc) {
     const int k0 = kc * GK;
@@ -65,6 +70,11 @@ __global__ void __launch_bounds__(256) k_gate_partial(const __nv_bfloat16* __res
       wsm[kq + 3][ex] = v.w;
     }
     __syncthreads();
+    float blk[4][4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) blk[i][j] = 0.f;
 #pragma unroll 8
     for (int k = 0; k < GK; ++k) {
       const float4 a = *reinterpret_cast<const float4*>(&xs[k][ty * 4]);
@@ -74,8 +84,17 @@ __global__ void __launch_bounds__(256) k_gate_partial(const __nv_bfloat16* __res
 #pragma unroll
       for (int i = 0; i < 4; ++i)
 #pragma unroll
-        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
+        for (int j = 0; j < 4; ++j) blk[i][j] = fmaf(av[i], bv[j], blk[i][j]);
     }
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float yv = __fsub_rn(blk[i][j], comp[i][j]);
+        const float tv = __fadd_rn(acc[i][j], yv);
+        comp[i][j] = __fsub_rn(__fsub_rn(tv, acc[i][j]), yv);
+        acc[i][j] = tv;
+      }
     __syncthreads();
   }
   float* out = part + (int64_t)blockIdx.z * N * E;
@@ -86,7 +105,7 @@ __global__ void __launch_bounds__(256) k_gate_partial(const __nv_bfloat16* __res
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       const int e = e0 + tx * 4 + j;
-      if (e < E) out[t * E + e] = acc[i][j];
+      if (e < E) out[t * E + e] = __fsub_rn(acc[i][j], comp[i][j]);
     }
   }
 }
@@ -121,7 +140,11 @@ __global__ void __launch_bounds__(32 * kSelWarps) k_select(
     const float* p = part + t * E;
     for (int e = lane; e < E; e += 32) {
       float L = p[e];
-      for (int z = 1; z < splits; ++z) L = __fadd_rn(L, p[z * split_stride + e]);
+      if (splits > 1) {  // split-K partials summed in double, rounded once
+        double Ld = (double)L;
+        for (int z = 1; z < splits; ++z) Ld += (double)p[z * split_stride + e];
+        L = (float)Ld;
+      }
       // sigmoid: fp32 rounding of 1/(1+exp(-L)) evaluated in double
       const float s = (float)(1.0 / (1.0 + exp(-(double)L)));
       s_s[e] = s;
