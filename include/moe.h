@@ -146,6 +146,36 @@ MOE_API int moe_dispatch(const int32_t* topk_idx, int64_t N, int K, int E, const
                          int d_e, int32_t* counts, int32_t* offsets, int32_t* perm, int32_t* pos,
                          moe_bf16* xs, void* ws, size_t ws_bytes, void* stream);
 
+/* Fixed size of the device array that moe_dispatch_static uses as scratch. */
+#define MOE_DISPATCH_STATIC_SCRATCH_BYTES (2u << 20)
+
+/* moe_dispatch for callers that cannot allocate device memory.
+ * The pages have no counterpart: this entry point exists for library users
+ * who have no way to provide the workspace that moe_dispatch takes, e.g. a
+ * plugin that its host framework hands only input and output tensors, a
+ * serving process whose device memory is fully reserved by another
+ * allocator, or a latency-critical loop that must not call cudaMalloc (it can
+ * synchronise the device).
+ * Arguments, outputs and results are those of moe_dispatch without (ws,
+ * ws_bytes); it enqueues the same kernels and allocates nothing (no
+ * cudaMalloc, cudaFree or allocating library routine).
+ * Scratch: a file-scope device array of MOE_DISPATCH_STATIC_SCRATCH_BYTES
+ * (2 MiB) inside libmoe.so, held by every GPU that loads the library until
+ * the process exits.  Calls whose per-chunk counts (4 * chunks * E bytes,
+ * chunks = ceil(N*K / clamp(N*K/256, 64, 1024) rounded up to 32)) exceed it
+ * return MOE_ERR_UNSUPPORTED; 131072 slots over 384 experts use 0.4 MiB.
+ * Set-up: the first call made on a device looks up the array's device
+ * address (cudaGetSymbolAddress) with that device current; make that first
+ * call before any stream capture.
+ * Every call shares the one array and overwrites it, so calls that can
+ * overlap on the GPU (different streams, or different host threads without
+ * ordering) race and corrupt each other's results; serialise them on one
+ * stream.  An expert index outside [0, E) is skipped as in moe_dispatch but
+ * is not reported (there is no status word). */
+MOE_API int moe_dispatch_static(const int32_t* topk_idx, int64_t N, int K, int E,
+                                const moe_bf16* x_e, int d_e, int32_t* counts, int32_t* offsets,
+                                int32_t* perm, int32_t* pos, moe_bf16* xs, void* stream);
+
 /* ------------------------------------------------------------- expert MLP */
 
 MOE_API size_t moe_expert_ffn_workspace_size(int64_t S, int d_e, int E, int F);

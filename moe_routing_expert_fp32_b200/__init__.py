@@ -78,7 +78,7 @@ _lib = None
 EXPORTS = ("moe_route_workspace_size", "moe_route", "moe_route_from_logits",
            "moe_dispatch_workspace_size", "moe_dispatch", "moe_expert_ffn_workspace_size",
            "moe_expert_ffn", "moe_combine_workspace_size", "moe_combine", "moe_workspace_size",
-           "moe_forward", "moe_get_status", "moe_strerror")
+           "moe_forward", "moe_get_status", "moe_strerror", "moe_dispatch_static")
 
 
 def lib() -> ctypes.CDLL:
@@ -106,6 +106,7 @@ def lib() -> ctypes.CDLL:
         "moe_forward": ([vp, vp, i64, i32, i32, vp, vp, rc, vp, vp, vp, i32, ac, vp, vp, vp, vp,
                          sz, vp, ev], i32),
         "moe_get_status": ([vp, vp], i32),
+        "moe_dispatch_static": ([vp, i64, i32, i32, vp, i32, vp, vp, vp, vp, vp, vp], i32),
         "moe_strerror": ([i32], ctypes.c_char_p),
     }
     for name, (args, res) in sig.items():
@@ -212,6 +213,31 @@ def dispatch(topk_idx, x_e, num_experts: int, ws=None):
            lib().moe_dispatch(_ptr(topk_idx), N, K, E, _ptr(x_e), d_e, _ptr(counts),
                               _ptr(offsets), _ptr(perm), _ptr(pos), _ptr(xs), _ptr(ws),
                               ws.numel(), _stream()))
+    return counts, offsets, perm, pos, xs
+
+
+def dispatch_static(topk_idx, x_e, num_experts: int):
+    """moe_dispatch without a workspace, for callers that cannot allocate device
+    memory: the scratch is a fixed 2 MiB array inside libmoe.so (see
+    moe_dispatch_static in include/moe.h for its limit and sharing rules).
+    This Python wrapper still allocates its outputs with torch; a caller that
+    cannot allocate passes its own buffers to the C entry point."""
+    torch = _torch()
+    N, K = topk_idx.shape
+    d_e = x_e.shape[1]
+    _need(topk_idx, torch.int32, name="topk_idx")
+    _need(x_e, torch.bfloat16, (N, d_e), "x_e")
+    E = num_experts
+    S = N * K
+    dev = x_e.device
+    counts = torch.empty(E, dtype=torch.int32, device=dev)
+    offsets = torch.empty(E + 1, dtype=torch.int32, device=dev)
+    perm = torch.empty(S, dtype=torch.int32, device=dev)
+    pos = torch.empty(S, dtype=torch.int32, device=dev)
+    xs = torch.empty((S, d_e), dtype=torch.bfloat16, device=dev)
+    _check("moe_dispatch_static",
+           lib().moe_dispatch_static(_ptr(topk_idx), N, K, E, _ptr(x_e), d_e, _ptr(counts),
+                                     _ptr(offsets), _ptr(perm), _ptr(pos), _ptr(xs), _stream()))
     return counts, offsets, perm, pos, xs
 
 
