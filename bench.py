@@ -34,7 +34,17 @@ if ROOT not in sys.path:
 METRIC = "routed tokens/sec per MoE layer (route+dispatch+FFN+combine)"
 UNIT = "tokens/s"
 DEFAULT_WORKLOAD = "dsv32_decode"
-KERNELS_PER_STEP = 10  # gate_partial, select, hist, scan, scatter, gather, tiles, gate_up, down, combine
+# gate_partial, [reduce_partials,] select, hist, scan, scatter, gather, tiles, gate_up, down,
+# combine; the reduce runs when the gate GEMM is split over d_r (decode batches)
+KERNELS_PER_STEP = 10
+
+
+def kernels_per_step(wl):
+    tiles = ((wl.E + 63) // 64) * ((wl.N + 63) // 64)
+    nk = wl.d_r // 32
+    want = max(1, min((296 + tiles - 1) // tiles, max(nk // 4, 1), 64))
+    cps = (nk + want - 1) // want
+    return KERNELS_PER_STEP + (1 if (nk + cps - 1) // cps > 1 else 0)
 
 
 def parse():
@@ -400,7 +410,7 @@ def main():
         "stages_ms": r["stage_ms"],
         "e2e": {"value": aggregate_throughput(wl.N, world, r["e2e_ms"]), "unit": UNIT,
                 "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"]},
-        "gpu_launches": KERNELS_PER_STEP * args.steps,
+        "gpu_launches": kernels_per_step(wl) * args.steps,
         "clocks": r["clocks"],
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -140,22 +140,25 @@ __global__ void __launch_bounds__(32 * kWarps) k_scatter(const int32_t* __restri
   }
 }
 
-// One warp per token: read its row once (16-byte vectors), write it to the
-// K sorted positions pos[t*K + k].
+// One warp per (token, chunk of 256 columns): each lane reads one 16-byte
+// vector of the token's row once and writes it to the K sorted positions
+// pos[t*K + k] (token-major, so x_e is read once, not K times).
 __global__ void __launch_bounds__(256) k_gather(const __nv_bfloat16* __restrict__ x, int64_t N,
                                                 int K, int d, const int32_t* __restrict__ pos,
                                                 __nv_bfloat16* __restrict__ xs) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nv = d / 8;
-  for (int64_t t = (int64_t)blockIdx.x * 8 + warp; t < N; t += (int64_t)gridDim.x * 8) {
+  const int nch = (nv + 31) / 32;
+  const int64_t items = N * nch;
+  for (int64_t it = (int64_t)blockIdx.x * 8 + warp; it < items; it += (int64_t)gridDim.x * 8) {
+    const int64_t t = it / nch;
+    const int v = (int)(it - t * nch) * 32 + lane;
     const int my_p = lane < K ? pos[t * K + lane] : -1;
-    const uint4* src = reinterpret_cast<const uint4*>(x + t * d);
-    for (int v = lane; v < nv; v += 32) {
-      const uint4 val = src[v];
-      for (int k = 0; k < K; ++k) {
-        const int p = __shfl_sync(0xffffffffu, my_p, k);
-        if (p >= 0) reinterpret_cast<uint4*>(xs + (int64_t)p * d)[v] = val;
-      }
+    uint4 val = make_uint4(0, 0, 0, 0);
+    if (v < nv) val = reinterpret_cast<const uint4*>(x + t * d)[v];
+    for (int k = 0; k < K; ++k) {
+      const int p = __shfl_sync(0xffffffffu, my_p, k);
+      if (p >= 0 && v < nv) reinterpret_cast<uint4*>(xs + (int64_t)p * d)[v] = val;
     }
   }
 }
@@ -193,8 +196,8 @@ cudaError_t launch_dispatch(const int32_t* idx, int64_t N, int K, int E, const _
   k_hist<<<blocks, 32 * kWarps, smem, s>>>(idx, S, E, CH, nchunks, scratch, st);
   k_scan<<<1, 1024, 0, s>>>(scratch, nchunks, E, counts, offsets);
   k_scatter<<<blocks, 32 * kWarps, smem, s>>>(idx, S, E, CH, nchunks, scratch, perm, pos);
-  int64_t gb = (N + 7) / 8;
-  const int64_t cap = (int64_t)dev_info()->sm_count * 8;
+  int64_t gb = (N * ((d_e / 8 + 31) / 32) + 7) / 8;
+  const int64_t cap = (int64_t)dev_info()->sm_count * 16;
   if (gb > cap) gb = cap;
   k_gather<<<(unsigned)gb, 256, 0, s>>>(x_e, N, K, d_e, pos, xs);
   return cudaGetLastError();

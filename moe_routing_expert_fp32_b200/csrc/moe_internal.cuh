@@ -36,6 +36,9 @@ int route_splits(int64_t N, int E, int d_r);
 size_t route_partial_bytes(int64_t N, int E, int d_r);
 cudaError_t launch_gate_partial(const __nv_bfloat16* x, int64_t N, int d_r, const float* W, int E,
                                 int splits, float* part, cudaStream_t s);
+float* route_logits_of(float* part, int64_t N, int E, int splits);
+cudaError_t launch_reduce_partials(const float* part, int splits, int64_t N, int E,
+                                   float* logits, cudaStream_t s);
 cudaError_t launch_select(const float* part, int splits, int64_t N, const float* bias,
                           const moe_route_cfg& cfg, int32_t* idx, float* w, DeviceStatus* st,
                           cudaStream_t s);

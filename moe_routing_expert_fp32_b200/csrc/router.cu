@@ -110,6 +110,25 @@ __global__ void __launch_bounds__(256) k_gate_partial(const __nv_bfloat16* __res
   }
 }
 
+// Split-K partials -> logits, one thread per (token, expert): the <= 64 fp32
+// partials are summed in double (two interleaved chains; exact unless their
+// exponents span more than ~29 bits) and rounded once to fp32.
+__global__ void __launch_bounds__(256) k_reduce_partials(const float* __restrict__ part,
+                                                         int splits, int64_t NE,
+                                                         float* __restrict__ logits) {
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < NE;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    double a0 = 0.0, a1 = 0.0;
+    int z = 0;
+    for (; z + 1 < splits; z += 2) {  // two independent chains, joined in order below
+      a0 += (double)part[(int64_t)z * NE + i];
+      a1 += (double)part[(int64_t)(z + 1) * NE + i];
+    }
+    if (z < splits) a0 += (double)part[(int64_t)z * NE + i];
+    logits[i] = (float)(a0 + a1);
+  }
+}
+
 // "a ranks before b": larger value first, ties to the lower index.
 __device__ __forceinline__ bool ranks_before(float va, int ia, float vb, int ib) {
   return va > vb || (va == vb && ia < ib);
@@ -225,7 +244,26 @@ int route_splits(int64_t N, int E, int d_r) {
 }
 
 size_t route_partial_bytes(int64_t N, int E, int d_r) {
-  return align_up(sizeof(float) * (size_t)route_splits(N, E, d_r) * (size_t)N * (size_t)E, 256);
+  const int splits = route_splits(N, E, d_r);
+  const size_t ne = (size_t)N * (size_t)E;
+  return align_up(sizeof(float) * (size_t)splits * ne, 256) +
+         (splits > 1 ? align_up(sizeof(float) * ne, 256) : 0);
+}
+
+float* route_logits_of(float* part, int64_t N, int E, int splits) {
+  if (splits <= 1) return part;
+  return reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(part) +
+                                  align_up(sizeof(float) * (size_t)splits * N * E, 256));
+}
+
+cudaError_t launch_reduce_partials(const float* part, int splits, int64_t N, int E,
+                                   float* logits, cudaStream_t s) {
+  const int64_t ne = N * (int64_t)E;
+  int64_t blocks = (ne + 255) / 256;
+  const int64_t cap = (int64_t)dev_info()->sm_count * 16;
+  if (blocks > cap) blocks = cap;
+  k_reduce_partials<<<(unsigned)blocks, 256, 0, s>>>(part, splits, ne, logits);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_gate_partial(const __nv_bfloat16* x, int64_t N, int d_r, const float* W, int E,
