@@ -4,28 +4,35 @@
 // w1 = gate, w3 = up, w2 = down, all bias-free nn.Linear) and situ excerpt
 // (SituAndMul), and the per-expert loop of moe_infer ("Kimi K3 · Add shared
 // output", moe-forward excerpt), which is replaced by one persistent launch
-// over a device-built tile list.
+// over a device-built tile list per projection.
 //
 // Design (sm_100a):
-//   * swap-AB: the MMA's M=128 side is a block of 128 weight rows, the N side
-//     is up to 128 token rows of one expert (N rounded up to 16).  Decode
-//     batches put 1-8 tokens on an expert, so the kernel is a weight stream;
-//     weight tiles fill the 128-lane accumulator whatever the token count.
-//   * TMA (cp.async.bulk.tensor, 128-byte swizzle) brings a 128x64 weight tile
-//     per operand (w1 and w3 share the token tile) and the token tile as 16-row
-//     boxes, into a 4-6 stage shared-memory ring guarded by mbarriers.
-//   * one elected thread issues tcgen05.mma (kind::f16, bf16 in, fp32 out)
-//     into TMEM; the 512 TMEM columns hold two accumulator buffers so the
-//     epilogue of one tile overlaps the MMAs of the next.
-//   * 4 epilogue warps read the accumulator with tcgen05.ld, apply the page's
-//     rounding points (g, u rounded to bf16; SiLU output rounded to bf16; h
-//     rounded to bf16) and store bf16 rows.
-//   * unit u -> (token tile, weight-row block) with the row block fastest, so
-//     CTAs that run at the same time share one token tile from L2 and stream
-//     disjoint weight rows.
-//   * every wait is bounded (2 s of %globaltimer); a wait that runs out
-//     records MOE_ERR_DEVICE_TIMEOUT, tells the other roles to stop, and the
-//     kernel frees its TMEM and returns.
+//   * swap-AB: the MMA's M = 128 side is weight rows, the N side is up to NTMAX
+//     token rows of one expert (N rounded up to 16).  Decode batches put 1-8
+//     rows on an expert, so the kernel is a weight stream whatever the count.
+//   * gate_up unit = 64 rows of d_ff: its 128-row A tile is w1 rows f0..f0+63
+//     over w3 rows f0..f0+63 (two 64-row TMA boxes), so one MMA per k-step
+//     yields g (TMEM lanes 0-63) and u (lanes 64-127); the epilogue warps that
+//     hold g and u of the same 32 rows swap half of each 16-column chunk
+//     through shared memory, so all four warps apply the activation.
+//   * down unit = 128 rows of d.
+//   * TMA (cp.async.bulk.tensor, 128-byte swizzle) fills a STAGES-deep ring of
+//     (A 128x64, B NTMAX x64) bf16 tiles guarded by mbarriers; one elected
+//     thread issues tcgen05.mma kind::f16 (bf16 in, fp32 accumulate) into
+//     TMEM; two accumulator buffers let the epilogue of one unit overlap the
+//     MMAs of the next; 4 epilogue warps drain TMEM with tcgen05.ld.
+//   * three variants by average rows per expert: decode (NTMAX 32, 10 stages:
+//     ~160 KB of weights in flight per SM, weights loaded with an L2
+//     evict-first hint since each is read once), mid (NTMAX 128, two A blocks
+//     and accumulators per unit, 4 stages) and large (NTMAX 256, 4 stages:
+//     128x256x16 MMAs).
+//   * the page's rounding points: g, u rounded to bf16; SiLU output rounded to
+//     bf16 before the product; SiTU evaluated in fp32; h and y rounded to bf16.
+//   * unit u -> (token tile, weight-row block), row block fastest: CTAs that
+//     run together share one token tile from L2 and stream disjoint weights.
+//   * every wait is bounded (2 s of %globaltimer); a wait that runs out records
+//     MOE_ERR_DEVICE_TIMEOUT, tells the other roles to stop, frees TMEM and the
+//     kernel returns.
 #include <cuda.h>
 #include <math.h>
 
@@ -34,26 +41,31 @@
 namespace moe {
 namespace {
 
-constexpr int BM = 128;       // weight rows per tile (MMA M)
-constexpr int BK = 64;        // K elements per stage: one 128-byte swizzle row
-constexpr int NT = 128;       // token rows per tile (max MMA N)
-constexpr int UK = 16;        // K per tcgen05.mma for 16-bit inputs
-constexpr int kThreads = 192; // warp 0: TMA, warp 1: MMA + TMEM, warps 2-5: epilogue
-constexpr int kBoxRows = 16;  // token rows per TMA box
+constexpr int BM = 128;        // A rows per tile (MMA M)
+constexpr int BK = 64;         // K elements per stage: one 128-byte swizzle row
+constexpr int UK = 16;         // K per tcgen05.mma for 16-bit inputs
+constexpr int kThreads = 192;  // warp 0: TMA, warp 1: MMA + TMEM, warps 2-5: epilogue
+constexpr int kBoxRows = 16;   // token rows per small TMA box
+constexpr int kBigBoxRows = 64;  // token rows per large TMA box (prefill variant)
+constexpr int kGateUpRows = 64;  // d_ff rows per gate_up unit (w1 + w3 = 128 A rows)
+constexpr int kXchgBytes = 8192;  // gate_up epilogue exchange: 2 pairs x 2 bufs x 2 x 32x8 fp32
 constexpr uint64_t kTimeoutNs = 2000000000ull;
 
 enum Mode { kGateUp = 0, kDown = 1 };
 
-template <int MODE>
+// UM = A blocks (of 128 rows) per unit, each with its own accumulator.
+template <int NTMAX, int STAGES, int UM>
 struct Cfg {
-  static constexpr int kA = (MODE == kGateUp) ? 2 : 1;
-  static constexpr int kABytes = BM * BK * 2;
-  static constexpr int kBBytes = NT * BK * 2;
-  static constexpr int kStageBytes = kA * kABytes + kBBytes;
-  static constexpr int kStages = (MODE == kGateUp) ? 4 : 6;
-  static constexpr int kBufCols = 256;  // TMEM columns per accumulator buffer
-  static constexpr int kTmemCols = 512;
-  static constexpr size_t kSmem = (size_t)kStages * kStageBytes + 1024 + 256;
+  static constexpr int kABlockBytes = BM * BK * 2;
+  static constexpr int kABytes = UM * kABlockBytes;
+  static constexpr int kBBytes = NTMAX * BK * 2;
+  static constexpr int kStageBytes = kABytes + kBBytes;
+  static constexpr int kBufCols = UM * NTMAX;  // TMEM columns per accumulator buffer
+  static constexpr int kTmemCols = (2 * kBufCols < 32) ? 32 : 2 * kBufCols;
+  static constexpr size_t kSmem = (size_t)STAGES * kStageBytes + 1024 + 256 + kXchgBytes;
+  static_assert(kStageBytes % 1024 == 0, "stages must keep 1024-byte alignment");
+  static_assert((kTmemCols & (kTmemCols - 1)) == 0 && kTmemCols <= 512, "TMEM columns");
+  static_assert(kSmem <= 227 * 1024, "shared memory");
 };
 
 // ------------------------------------------------------------ PTX wrappers
@@ -117,6 +129,21 @@ __device__ __forceinline__ void tma_load_3d(const CUtensorMap* map, uint64_t* ba
       "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2)
       : "memory");
 }
+__device__ __forceinline__ uint64_t l2_evict_first_policy() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+__device__ __forceinline__ void tma_load_3d_hint(const CUtensorMap* map, uint64_t* bar, void* dst,
+                                                 int c0, int c1, int c2, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%3, %4, %5}], [%2], %6;" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2),
+      "l"(policy)
+      : "memory");
+}
+
 __device__ __forceinline__ void tc_fence_before() {
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
 }
@@ -197,7 +224,7 @@ struct Unit {
   int e, row0, nrows, rb;
 };
 
-__device__ __forceinline__ Unit decode_unit(int64_t u, int RB, const int32_t* tile_start,
+__device__ __forceinline__ Unit decode_unit(int64_t u, int RB, int nt, const int32_t* tile_start,
                                             const int32_t* offsets, int E) {
   Unit r;
   const int tt = (int)(u / RB);
@@ -209,37 +236,43 @@ __device__ __forceinline__ Unit decode_unit(int64_t u, int RB, const int32_t* ti
     else hi = mid - 1;
   }
   r.e = lo;
-  r.row0 = offsets[lo] + (tt - tile_start[lo]) * NT;
+  r.row0 = offsets[lo] + (tt - tile_start[lo]) * nt;
   const int rem = offsets[lo + 1] - r.row0;
-  r.nrows = rem < NT ? rem : NT;
+  r.nrows = rem < nt ? rem : nt;
   return r;
 }
 
-template <int MODE>
+template <int MODE, int NTMAX, int STAGES, int UM>
 __global__ void __launch_bounds__(kThreads, 1)
     k_expert_gemm(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA1,
-                  const __grid_constant__ CUtensorMap tmB, const int32_t* __restrict__ offsets,
+                  const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmB64,
+                  const int32_t* __restrict__ offsets,
                   const int32_t* __restrict__ tile_start, int E, int M_rows, int Kdim,
                   __nv_bfloat16* __restrict__ out, int act_kind, float beta, float lbeta,
                   DeviceStatus* st) {
-  using C = Cfg<MODE>;
+  using C = Cfg<NTMAX, STAGES, UM>;
+  constexpr bool kDecode = NTMAX <= 32;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kStages * C::kStageBytes);
-  uint64_t* empty = full + C::kStages;
-  uint64_t* tfull = empty + C::kStages;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * C::kStageBytes);
+  uint64_t* empty = full + STAGES;
+  uint64_t* tfull = empty + STAGES;
   uint64_t* tempty = tfull + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  float* xchg = reinterpret_cast<float*>(smem + STAGES * C::kStageBytes + 256);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int RB = M_rows / BM;
+  // rows of the output per A block: 64 d_ff rows (gate_up) or 128 d rows (down)
+  const int blk_rows = (MODE == kGateUp) ? kGateUpRows : BM;
+  const int unit_rows = UM * blk_rows;
+  const int RB = (M_rows + unit_rows - 1) / unit_rows;
   const int KB = Kdim / BK;
   const int64_t total_units = (int64_t)tile_start[E] * RB;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < C::kStages; ++s) {
+    for (int s = 0; s < STAGES; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
@@ -264,24 +297,46 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) {
     // ------------------------------------------------------ TMA producer
     if (lane == 0) {
+      const uint64_t wpol = kDecode ? l2_evict_first_policy() : 0;
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
       for (int64_t u = blockIdx.x; u < total_units && ok; u += gridDim.x) {
-        const Unit w = decode_unit(u, RB, tile_start, offsets, E);
-        const int nb = (w.nrows + kBoxRows - 1) / kBoxRows;
-        const uint32_t bytes = C::kA * C::kABytes + nb * kBoxRows * BK * 2;
+        const Unit w = decode_unit(u, RB, NTMAX, tile_start, offsets, E);
+        // token rows: 16-row boxes for short tiles, 64-row boxes otherwise
+        const bool big = !kDecode && w.nrows > 2 * kBoxRows;
+        const int brows = big ? kBigBoxRows : kBoxRows;
+        const int nb = (w.nrows + brows - 1) / brows;
+        const uint32_t bytes = C::kABytes + nb * brows * BK * 2;
+        const int r0 = w.rb * unit_rows;
         for (int kb = 0; kb < KB; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag)) { ok = false; break; }
           uint8_t* sA = smem + stage * C::kStageBytes;
-          uint8_t* sB = sA + C::kA * C::kABytes;
+          uint8_t* sB = sA + C::kABytes;
           mbar_arrive_expect_tx(&full[stage], bytes);
-          tma_load_3d(&tmA0, &full[stage], sA, kb * BK, w.rb * BM, w.e);
-          if (MODE == kGateUp) tma_load_3d(&tmA1, &full[stage], sA + C::kABytes, kb * BK, w.rb * BM, w.e);
+#pragma unroll
+          for (int a = 0; a < UM; ++a) {
+            uint8_t* dA = sA + a * C::kABlockBytes;
+            const int ra = r0 + a * blk_rows;
+            if (MODE == kGateUp) {
+              // w1 rows ra..ra+63 over w3 rows ra..ra+63
+              void* d3 = dA + kGateUpRows * BK * 2;
+              if (kDecode) {
+                tma_load_3d_hint(&tmA0, &full[stage], dA, kb * BK, ra, w.e, wpol);
+                tma_load_3d_hint(&tmA1, &full[stage], d3, kb * BK, ra, w.e, wpol);
+              } else {
+                tma_load_3d(&tmA0, &full[stage], dA, kb * BK, ra, w.e);
+                tma_load_3d(&tmA1, &full[stage], d3, kb * BK, ra, w.e);
+              }
+            } else {
+              if (kDecode) tma_load_3d_hint(&tmA0, &full[stage], dA, kb * BK, ra, w.e, wpol);
+              else tma_load_3d(&tmA0, &full[stage], dA, kb * BK, ra, w.e);
+            }
+          }
           for (int i = 0; i < nb; ++i)
-            tma_load_2d(&tmB, &full[stage], sB + i * kBoxRows * BK * 2, kb * BK,
-                        w.row0 + i * kBoxRows);
-          if (++stage == C::kStages) { stage = 0; phase ^= 1; }
+            tma_load_2d(big ? &tmB64 : &tmB, &full[stage], sB + i * brows * BK * 2, kb * BK,
+                        w.row0 + i * brows);
+          if (++stage == STAGES) { stage = 0; phase ^= 1; }
         }
       }
       if (!ok) {
@@ -297,7 +352,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       int local = 0;
       bool ok = true;
       for (int64_t u = blockIdx.x; u < total_units && ok; u += gridDim.x, ++local) {
-        const Unit w = decode_unit(u, RB, tile_start, offsets, E);
+        const Unit w = decode_unit(u, RB, NTMAX, tile_start, offsets, E);
         const int n = ((w.nrows + 15) / 16) * 16;
         const uint32_t idesc = idesc_bf16(n);
         const int buf = local & 1;
@@ -309,17 +364,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!mbar_wait(&full[stage], phase, abort_flag)) { ok = false; break; }
           tc_fence_after();
           const uint32_t a0 = smem_u32(smem + stage * C::kStageBytes);
-          const uint32_t b0 = a0 + C::kA * C::kABytes;
+          const uint32_t b0 = a0 + C::kABytes;
 #pragma unroll
-          for (int k = 0; k < BK / UK; ++k) {
-            const uint32_t acc = (kb | k) != 0;
-            umma_bf16(d0, sw128_desc(a0 + k * UK * 2), sw128_desc(b0 + k * UK * 2), idesc, acc);
-            if (MODE == kGateUp)
-              umma_bf16(d0 + NT, sw128_desc(a0 + C::kABytes + k * UK * 2),
-                        sw128_desc(b0 + k * UK * 2), idesc, acc);
-          }
+          for (int k = 0; k < BK / UK; ++k)
+#pragma unroll
+            for (int a = 0; a < UM; ++a)
+              umma_bf16(d0 + a * NTMAX, sw128_desc(a0 + a * C::kABlockBytes + k * UK * 2),
+                        sw128_desc(b0 + k * UK * 2), idesc, (kb | k) != 0);
           umma_commit(&empty[stage]);
-          if (++stage == C::kStages) { stage = 0; phase ^= 1; }
+          if (++stage == STAGES) { stage = 0; phase ^= 1; }
         }
         if (ok) umma_commit(&tfull[buf]);
       }
@@ -330,13 +383,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ------------------------------------------------------ epilogue
-    const int quarter = warp & 3;  // TMEM lanes this warp may read
-    const int r_in = quarter * 32 + lane;
+    const int quarter = warp & 3;  // TMEM lanes 32*quarter .. +31 belong to this warp
     const bool has_lb = !(lbeta == 0.0f || lbeta != lbeta);
     const float b_eff = (beta == 0.0f || beta != beta) ? 1.0f : beta;
     int local = 0;
+    uint32_t xbuf = 0;  // exchange buffer parity (gate_up)
     for (int64_t u = blockIdx.x; u < total_units; u += gridDim.x, ++local) {
-      const Unit w = decode_unit(u, RB, tile_start, offsets, E);
+      const Unit w = decode_unit(u, RB, NTMAX, tile_start, offsets, E);
       const int buf = local & 1;
       const uint32_t tphase = (local >> 1) & 1;
       if (!mbar_wait(&tfull[buf], tphase, abort_flag)) {
@@ -345,25 +398,59 @@ __global__ void __launch_bounds__(kThreads, 1)
         break;
       }
       tc_fence_after();
-      const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + buf * C::kBufCols;
-      const int m = w.rb * BM + r_in;
-      __nv_bfloat16* col = out + m;
-      for (int c0 = 0; c0 < w.nrows; c0 += 16) {
-        float v[16];
-        tmem_ld16(taddr + c0, v);
-        if (MODE == kGateUp) {
-          float uu[16];
-          tmem_ld16(taddr + NT + c0, uu);
+      for (int a = 0; a < UM; ++a) {
+      const uint32_t taddr =
+          tmem_base + ((uint32_t)(quarter * 32) << 16) + buf * C::kBufCols + a * NTMAX;
+      const int r0 = w.rb * unit_rows + a * blk_rows;
+      if (MODE == kGateUp) {
+        // quarters 0/1 hold g of rows 0-31 / 32-63, quarters 2/3 hold u of the
+        // same rows; pair p = quarter & 1.  Per 16-column chunk the g warp keeps
+        // columns 0-7 and hands g of columns 8-15 to the u warp, which keeps
+        // columns 8-15 and hands u of columns 0-7 back.
+        const int pair = quarter & 1;
+        const bool is_g = quarter < 2;
+        const int f = r0 + pair * 32 + lane;
+        __nv_bfloat16* col = out + f;
+        const bool live = f < M_rows;
+        for (int c0 = 0; c0 < w.nrows; c0 += 16, ++xbuf) {
+          float v[16];
+          tmem_ld16(taddr + c0, v);
+          float* xg = xchg + ((pair * 2 + (xbuf & 1)) * 2 + 0) * 256;  // g cols 8-15
+          float* xu = xchg + ((pair * 2 + (xbuf & 1)) * 2 + 1) * 256;  // u cols 0-7
+          float4* mine = reinterpret_cast<float4*>((is_g ? xg : xu) + lane * 8);
+          const float* give = is_g ? v + 8 : v;
+          mine[0] = make_float4(give[0], give[1], give[2], give[3]);
+          mine[1] = make_float4(give[4], give[5], give[6], give[7]);
+          asm volatile("bar.sync %0, 64;" ::"r"(1 + pair) : "memory");
+          const float4* theirs = reinterpret_cast<const float4*>((is_g ? xu : xg) + lane * 8);
+          const float4 t0 = theirs[0], t1 = theirs[1];
+          const float other[8] = {t0.x, t0.y, t0.z, t0.w, t1.x, t1.y, t1.z, t1.w};
+          const int cbase = c0 + (is_g ? 0 : 8);
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const float g = is_g ? v[j] : other[j];
+            const float uu = is_g ? other[j] : v[8 + j];
+            const float h = act_kind == MOE_ACT_SITU ? situ_mul(g, uu, b_eff, lbeta, has_lb)
+                                                     : silu_mul(g, uu);
+            if (live && cbase + j < w.nrows)
+              col[(int64_t)(w.row0 + cbase + j) * M_rows] = __float2bfloat16_rn(h);
+          }
+        }
+      } else {
+        const int m = r0 + quarter * 32 + lane;
+        __nv_bfloat16* col = out + m;
+        const int lim_m = m < M_rows ? 16 : 0;
+        for (int c0 = 0; c0 < w.nrows; c0 += 16) {
+          float v[16];
+          tmem_ld16(taddr + c0, v);
+          int lim = w.nrows - c0 < 16 ? w.nrows - c0 : 16;
+          lim = lim < lim_m ? lim : lim_m;
 #pragma unroll
           for (int j = 0; j < 16; ++j)
-            v[j] = act_kind == MOE_ACT_SITU ? situ_mul(v[j], uu[j], b_eff, lbeta, has_lb)
-                                            : silu_mul(v[j], uu[j]);
+            if (j < lim) col[(int64_t)(w.row0 + c0 + j) * M_rows] = __float2bfloat16_rn(v[j]);
         }
-        const int lim = w.nrows - c0 < 16 ? w.nrows - c0 : 16;
-#pragma unroll
-        for (int j = 0; j < 16; ++j)
-          if (j < lim) col[(int64_t)(w.row0 + c0 + j) * M_rows] = __float2bfloat16_rn(v[j]);
       }
+      }  // accumulators
       tc_fence_before();
       mbar_arrive(&tempty[buf]);
     }
@@ -378,10 +465,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // Token tiles per expert and their prefix: tile_start[e] = sum_{e'<e}
-// ceil(n_e'/NT), tile_start[E] = total.  Inconsistent offsets are recorded
+// ceil(n_e'/nt), tile_start[E] = total.  Inconsistent offsets are recorded
 // and give the expert no tile, so the GEMM never reads outside xs.
 __global__ void __launch_bounds__(1024) k_tiles(const int32_t* __restrict__ offsets, int E,
-                                                int64_t S, int32_t* __restrict__ tile_start,
+                                                int64_t S, int nt, int32_t* __restrict__ tile_start,
                                                 DeviceStatus* st) {
   __shared__ int32_t warp_tot[32];
   const int e = threadIdx.x, lane = e & 31, warp = e >> 5;
@@ -390,7 +477,7 @@ __global__ void __launch_bounds__(1024) k_tiles(const int32_t* __restrict__ offs
     const int32_t a = offsets[e], b = offsets[e + 1];
     const bool bad = a < 0 || b < a || b > S || (e == 0 && a != 0) || (e == E - 1 && b != S);
     if (bad) record_error(st, MOE_ERR_DEVICE_BOUNDS, 30);
-    else n = (b - a + NT - 1) / NT;
+    else n = (b - a + nt - 1) / nt;
   }
   int32_t v = n;
 #pragma unroll
@@ -465,26 +552,61 @@ bool make_map_2d(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int MODE>
+template <int MODE, int NTMAX, int STAGES, int UM>
 cudaError_t launch_gemm(const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorMap& b,
-                        const int32_t* offsets, const int32_t* tile_start, int E, int M_rows,
+                        const CUtensorMap& b64, const int32_t* offsets, const int32_t* tile_start, int E, int M_rows,
                         int Kdim, __nv_bfloat16* out, const moe_act_cfg& act, DeviceStatus* st,
                         cudaStream_t s) {
-  using C = Cfg<MODE>;
+  using C = Cfg<NTMAX, STAGES, UM>;
   static bool attr_set[64] = {false};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 64 && !attr_set[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(k_expert_gemm<MODE>,
+    cudaError_t e = cudaFuncSetAttribute(k_expert_gemm<MODE, NTMAX, STAGES, UM>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)C::kSmem);
     if (e != cudaSuccess) return e;
     attr_set[dev] = true;
   }
-  k_expert_gemm<MODE><<<dev_info()->sm_count, kThreads, C::kSmem, s>>>(
-      a0, a1, b, offsets, tile_start, E, M_rows, Kdim, out, act.kind, act.beta, act.linear_beta,
-      st);
+  k_expert_gemm<MODE, NTMAX, STAGES, UM><<<dev_info()->sm_count, kThreads, C::kSmem, s>>>(
+      a0, a1, b, b64, offsets, tile_start, E, M_rows, Kdim, out, act.kind, act.beta,
+      act.linear_beta, st);
   return cudaGetLastError();
+}
+
+// Variant choice from shapes only (no host round trip), by the average rows
+// per expert S / E: decode (<= 16: weight stream, deep ring of small stages),
+// mid (<= 128: weight-bound; two 128-row A blocks per unit halve the token
+// tile traffic per weight byte), large (tensor-bound: 128x256 MMAs).
+constexpr int kNtDecode = 32, kStagesDecode = 10, kUmDecode = 1;
+constexpr int kNtMid = 128, kStagesMid = 4, kUmMid = 2;
+constexpr int kNtLarge = 256, kStagesLarge = 4, kUmLarge = 1;
+
+enum Variant { kVarDecode = 0, kVarMid = 1, kVarLarge = 2 };
+
+Variant pick_variant(int64_t S, int E) {
+  if (S <= 16 * (int64_t)E) return kVarDecode;
+  if (S <= 128 * (int64_t)E) return kVarMid;
+  return kVarLarge;
+}
+
+template <int MODE>
+cudaError_t launch_variant(Variant v, const CUtensorMap& a0, const CUtensorMap& a1,
+                           const CUtensorMap& b, const CUtensorMap& b64, const int32_t* offsets,
+                           const int32_t* tile_start, int E, int M_rows, int Kdim,
+                           __nv_bfloat16* out, const moe_act_cfg& act, DeviceStatus* st,
+                           cudaStream_t s) {
+  switch (v) {
+    case kVarDecode:
+      return launch_gemm<MODE, kNtDecode, kStagesDecode, kUmDecode>(a0, a1, b, b64, offsets, tile_start, E,
+                                                         M_rows, Kdim, out, act, st, s);
+    case kVarMid:
+      return launch_gemm<MODE, kNtMid, kStagesMid, kUmMid>(a0, a1, b, b64, offsets, tile_start, E, M_rows,
+                                                   Kdim, out, act, st, s);
+    default:
+      return launch_gemm<MODE, kNtLarge, kStagesLarge, kUmLarge>(a0, a1, b, b64, offsets, tile_start, E,
+                                                       M_rows, Kdim, out, act, st, s);
+  }
 }
 
 }  // namespace
@@ -501,21 +623,23 @@ int expert_ffn_run(const __nv_bfloat16* xs, const int32_t* offsets, int E, int64
   int32_t* tile_start = static_cast<int32_t*>(scratch);
   __nv_bfloat16* h = reinterpret_cast<__nv_bfloat16*>(
       static_cast<uint8_t*>(scratch) + align_up(sizeof(int32_t) * (size_t)(E + 1), 256));
-  CUtensorMap mw1, mw3, mw2, mxs, mh;
-  if (!make_map_3d(&mw1, w1, d_e, F, E, BM) || !make_map_3d(&mw3, w3, d_e, F, E, BM) ||
-      !make_map_3d(&mw2, w2, F, d_e, E, BM) || !make_map_2d(&mxs, xs, d_e, S, kBoxRows) ||
-      !make_map_2d(&mh, h, F, S, kBoxRows))
+  CUtensorMap mw1, mw3, mw2, mxs, mh, mxs64, mh64;
+  if (!make_map_3d(&mw1, w1, d_e, F, E, kGateUpRows) ||
+      !make_map_3d(&mw3, w3, d_e, F, E, kGateUpRows) || !make_map_3d(&mw2, w2, F, d_e, E, BM) ||
+      !make_map_2d(&mxs, xs, d_e, S, kBoxRows) || !make_map_2d(&mh, h, F, S, kBoxRows) ||
+      !make_map_2d(&mxs64, xs, d_e, S, kBigBoxRows) || !make_map_2d(&mh64, h, F, S, kBigBoxRows))
     return MOE_ERR_CUDA;
-  k_tiles<<<1, 1024, 0, s>>>(offsets, E, S, tile_start, st);
+  const Variant var = pick_variant(S, E);
+  const int nt = var == kVarDecode ? kNtDecode : (var == kVarMid ? kNtMid : kNtLarge);
+  k_tiles<<<1, 1024, 0, s>>>(offsets, E, S, nt, tile_start, st);
   if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
-  if (launch_gemm<kGateUp>(mw1, mw3, mxs, offsets, tile_start, E, F, d_e, h, act, st, s) !=
-      cudaSuccess)
-    return MOE_ERR_CUDA;
+  cudaError_t rc = launch_variant<kGateUp>(var, mw1, mw3, mxs, mxs64, offsets, tile_start, E, F,
+                                           d_e, h, act, st, s);
+  if (rc != cudaSuccess) return MOE_ERR_CUDA;
   if (after_gate_up && cudaEventRecord(after_gate_up, s) != cudaSuccess) return MOE_ERR_CUDA;
-  if (launch_gemm<kDown>(mw2, mw2, mh, offsets, tile_start, E, d_e, F, y, act, st, s) !=
-      cudaSuccess)
-    return MOE_ERR_CUDA;
-  return MOE_OK;
+  rc = launch_variant<kDown>(var, mw2, mw2, mh, mh64, offsets, tile_start, E, d_e, F, y, act, st,
+                             s);
+  return rc == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
 }  // namespace moe

@@ -345,3 +345,20 @@ def test_forward_single_token(moe):
     ys = [oracle.expert_ffn(inp["x_e"], *host_expert(wl, int(e)))[0] for e in idx_r[0]]
     out_r = oracle.combine(np.stack(ys), np.arange(wl.K, dtype=np.int32), w_r, wl.K)
     assert rel_l2(out_g, out_r) <= REL_L2_OUT
+
+
+@pytest.mark.parametrize("counts", [[1500, 700, 37, 0, 1763], [900, 5, 300, 800, 2000]])
+def test_expert_ffn_large_tiles_ragged(moe, counts):
+    """> 128 rows per expert on average selects the 256-row tile variant; the
+    segments end mid-tile, below 32 rows and on a 64-row box boundary."""
+    wl = scaled(WORKLOADS["tiny"], E=5, d_e=256, F=384)
+    _expert_case(moe, wl, np.array(counts), list(range(5)), rows_per_expert=96)
+
+
+@pytest.mark.parametrize("act", ["silu", "situ"])
+def test_expert_ffn_mid_tiles(moe, act):
+    """17..128 rows per expert on average selects the 128-row tile variant."""
+    wl = scaled(WORKLOADS["k3_latent_decode"], E=12, d_e=384, F=256, act=act)
+    counts = np.random.default_rng(9).integers(20, 200, 12)
+    counts[4] = 0
+    _expert_case(moe, wl, counts, list(range(12)), rows_per_expert=64)
