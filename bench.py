@@ -58,6 +58,7 @@ def parse():
     # profiling cases: the same workload with fewer tokens / experts
     p.add_argument("--tokens", type=int, default=None)
     p.add_argument("--experts", type=int, default=None)
+    p.add_argument("--ffn", type=int, default=None)
     return p.parse_args()
 
 
@@ -69,6 +70,8 @@ def workload_of(args):
         kw["N"] = args.tokens
     if args.experts:
         kw["E"] = args.experts
+    if args.ffn:
+        kw["F"] = args.ffn
     return scaled(wl, **kw) if kw else wl
 
 

@@ -84,13 +84,9 @@ int route_impl(const __nv_bfloat16* x, int64_t N, int d_r, const float* W, const
                const moe_route_cfg& cfg, int32_t* idx, float* w, uint8_t* scratch,
                DeviceStatus* st, cudaStream_t s) {
   const int E = cfg.num_experts;
-  const int splits = route_splits(N, E, d_r);
-  float* part = reinterpret_cast<float*>(scratch);
-  float* logits = route_logits_of(part, N, E, splits);
-  if (launch_gate_partial(x, N, d_r, W, E, splits, part, s) != cudaSuccess) return MOE_ERR_CUDA;
-  if (splits > 1 && launch_reduce_partials(part, splits, N, E, logits, s) != cudaSuccess)
+  if (launch_gate(x, N, d_r, W, E, scratch, s) != cudaSuccess) return MOE_ERR_CUDA;
+  if (launch_select(route_logits_of(scratch), 1, N, bias, cfg, idx, w, st, s) != cudaSuccess)
     return MOE_ERR_CUDA;
-  if (launch_select(logits, 1, N, bias, cfg, idx, w, st, s) != cudaSuccess) return MOE_ERR_CUDA;
   return MOE_OK;
 }
 

@@ -34,11 +34,10 @@ inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 // router.cu
 int route_splits(int64_t N, int E, int d_r);
 size_t route_partial_bytes(int64_t N, int E, int d_r);
-cudaError_t launch_gate_partial(const __nv_bfloat16* x, int64_t N, int d_r, const float* W, int E,
-                                int splits, float* part, cudaStream_t s);
-float* route_logits_of(float* part, int64_t N, int E, int splits);
-cudaError_t launch_reduce_partials(const float* part, int splits, int64_t N, int E,
-                                   float* logits, cudaStream_t s);
+// gate GEMM into the router scratch; the fp32 logits [N, E] are at its start
+cudaError_t launch_gate(const __nv_bfloat16* x, int64_t N, int d_r, const float* W, int E,
+                        void* scratch, cudaStream_t s);
+float* route_logits_of(void* scratch);
 cudaError_t launch_select(const float* part, int splits, int64_t N, const float* bias,
                           const moe_route_cfg& cfg, int32_t* idx, float* w, DeviceStatus* st,
                           cudaStream_t s);

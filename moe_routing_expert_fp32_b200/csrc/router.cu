@@ -3,12 +3,12 @@
 // Follows "Kimi K2 · Affinities", gate-forward excerpt (MoEGate.forward with
 // noaux_tc) and "DeepSeek-V3.2-Exp · Affinities", gate-forward excerpt
 // (Gate.forward):
-//   k_gate_partial : logits = x . W^T in fp32 (x upcast from bf16, W fp32),
-//                    split over d_r into `splits` partial sums so that decode
-//                    batches still fill the GPU.  FMA chains are 32 terms long;
-//                    the 32-term blocks are added with Kahan compensation and
-//                    the split partials in double, which keeps the logit error
-//                    near 1e-7 instead of the ~1e-5 of one 7168-term chain.
+//   k_gate_partial : logits = x . W^T in fp32 (x upcast from bf16, W fp32);
+//                    decode batches split d_r over several CTAs (partials in
+//                    double, summed by k_reduce_partials).  FMA chains are 32
+//                    terms long and the 32-term blocks are added in double,
+//                    which keeps the logit error near 1e-7 instead of the
+//                    ~1e-5 of one 7168-term fp32 chain.
 //   k_select       : one warp per token: sigmoid, + bias, group top-2 sums,
 //                    top-TG groups (others -> -inf), top-K experts by
 //                    (score desc, index asc), unbiased weights, renormalise
@@ -22,110 +22,128 @@
 namespace moe {
 namespace {
 
-constexpr int GT = 64;   // tokens per tile
-constexpr int GE = 64;   // experts per tile
-constexpr int GK = 32;   // k per smem stage
+constexpr int GT = 64;    // tokens per tile
+constexpr int GE = 64;    // experts per tile
+constexpr int GK = 32;    // k per chunk = length of every fp32 FMA chain
+constexpr int GEP = GE + 2;  // padded row of the transposed W tile (8-byte aligned)
 constexpr float kNegInf = -INFINITY;
 
-__global__ void __launch_bounds__(256) k_gate_partial(const __nv_bfloat16* __restrict__ x,
-                                                      int64_t N, int d,
-                                                      const float* __restrict__ W, int E,
-                                                      int cps, float* __restrict__ part) {
-  __shared__ __align__(16) float xs[GK][GT];
-  __shared__ __align__(16) float wsm[GK][GE];
+// logits (or split-K partials) of a 64-token x 64-expert tile.  Thread
+// (tx = lane, ty = warp) owns tokens ty*8..ty*8+7 and experts tx*2, tx*2+1;
+// the token values are warp-uniform (broadcast loads).  Each 32-wide k chunk
+// is accumulated in fp32 (FMA) and then added to a double accumulator, so no
+// fp32 rounding chain is longer than 32 terms.  Chunks are staged global ->
+// registers -> shared memory one chunk ahead (double buffer).
+__global__ void __launch_bounds__(256, 2) k_gate_partial(const __nv_bfloat16* __restrict__ x,
+                                                         int64_t N, int d,
+                                                         const float* __restrict__ W, int E,
+                                                         int cps, int splits,
+                                                         float* __restrict__ logits,
+                                                         double* __restrict__ part) {
+  __shared__ __align__(16) float xs[2][GK][GT];
+  __shared__ __align__(16) float wsm[2][GK][GEP];
   const int tid = threadIdx.x;
-  const int tx = tid & 15, ty = tid >> 4;
+  const int tx = tid & 31, ty = tid >> 5;
   const int64_t t0 = (int64_t)blockIdx.y * GT;
   const int e0 = blockIdx.x * GE;
   const int nk = d / GK;
   const int kc0 = blockIdx.z * cps;
   const int kc1 = min(nk, kc0 + cps);
-  // Running sums with Kahan compensation; each 32-wide k block is first
-  // accumulated on its own, so no fp32 chain is longer than 32 terms.
-  float acc[4][4], comp[4][4];
-#pragma unroll
-  for (int i = 0; i < 4; ++i)
-#pragma unroll
-    for (int j = 0; j < 4; ++j) acc[i][j] = comp[i][j] = 0.f;
 
-  for (int kc = kc0; kc < kc1; ++kc) {
+  // global -> register staging of one chunk: x 64 tokens x 32 k (one 16-byte
+  // vector per thread), W 64 experts x 32 k (two float4 per thread)
+  const int xtok = tid >> 2, xkk = (tid & 3) * 8;
+  uint4 xr = make_uint4(0, 0, 0, 0);
+  float4 wr[2];
+  auto load_chunk = [&](int kc) {
     const int k0 = kc * GK;
-    {  // x tile: 64 tokens x 32 k (bf16 -> fp32), one 16-byte load per thread
-      const int tok = tid >> 2, kk = (tid & 3) * 8;
-      uint4 v = make_uint4(0, 0, 0, 0);
-      if (t0 + tok < N) v = *reinterpret_cast<const uint4*>(x + (t0 + tok) * d + k0 + kk);
-      const __nv_bfloat16* h = reinterpret_cast<const __nv_bfloat16*>(&v);
+    xr = make_uint4(0, 0, 0, 0);
+    if (t0 + xtok < N) xr = *reinterpret_cast<const uint4*>(x + (t0 + xtok) * d + k0 + xkk);
 #pragma unroll
-      for (int j = 0; j < 8; ++j) xs[kk + j][tok] = __bfloat162float(h[j]);
-    }
-#pragma unroll
-    for (int r = 0; r < 2; ++r) {  // W tile: 64 experts x 32 k fp32
+    for (int r = 0; r < 2; ++r) {
       const int i = tid + 256 * r;
       const int ex = i >> 3, kq = (i & 7) * 4;
-      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (e0 + ex < E) v = *reinterpret_cast<const float4*>(W + (int64_t)(e0 + ex) * d + k0 + kq);
-      wsm[kq + 0][ex] = v.x;
-      wsm[kq + 1][ex] = v.y;
-      wsm[kq + 2][ex] = v.z;
-      wsm[kq + 3][ex] = v.w;
+      wr[r] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (e0 + ex < E)
+        wr[r] = *reinterpret_cast<const float4*>(W + (int64_t)(e0 + ex) * d + k0 + kq);
     }
-    __syncthreads();
-    float blk[4][4];
+  };
+  auto store_chunk = [&](int b) {
+    const __nv_bfloat16* h = reinterpret_cast<const __nv_bfloat16*>(&xr);
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
+    for (int j = 0; j < 8; ++j) xs[b][xkk + j][xtok] = __bfloat162float(h[j]);
 #pragma unroll
-      for (int j = 0; j < 4; ++j) blk[i][j] = 0.f;
+    for (int r = 0; r < 2; ++r) {
+      const int i = tid + 256 * r;
+      const int ex = i >> 3, kq = (i & 7) * 4;
+      wsm[b][kq + 0][ex] = wr[r].x;
+      wsm[b][kq + 1][ex] = wr[r].y;
+      wsm[b][kq + 2][ex] = wr[r].z;
+      wsm[b][kq + 3][ex] = wr[r].w;
+    }
+  };
+
+  double acc[8][2];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) acc[i][0] = acc[i][1] = 0.0;
+
+  int buf = 0;
+  if (kc0 < kc1) {
+    load_chunk(kc0);
+    store_chunk(0);
+  }
+  __syncthreads();
+  for (int kc = kc0; kc < kc1; ++kc) {
+    const bool more = kc + 1 < kc1;
+    if (more) load_chunk(kc + 1);
+    float blk[8][2];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) blk[i][0] = blk[i][1] = 0.f;
 #pragma unroll 8
     for (int k = 0; k < GK; ++k) {
-      const float4 a = *reinterpret_cast<const float4*>(&xs[k][ty * 4]);
-      const float4 b = *reinterpret_cast<const float4*>(&wsm[k][tx * 4]);
-      const float av[4] = {a.x, a.y, a.z, a.w};
-      const float bv[4] = {b.x, b.y, b.z, b.w};
+      const float4 a0 = *reinterpret_cast<const float4*>(&xs[buf][k][ty * 8]);
+      const float4 a1 = *reinterpret_cast<const float4*>(&xs[buf][k][ty * 8 + 4]);
+      const float2 b = *reinterpret_cast<const float2*>(&wsm[buf][k][tx * 2]);
+      const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
 #pragma unroll
-      for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) blk[i][j] = fmaf(av[i], bv[j], blk[i][j]);
+      for (int i = 0; i < 8; ++i) {
+        blk[i][0] = fmaf(av[i], b.x, blk[i][0]);
+        blk[i][1] = fmaf(av[i], b.y, blk[i][1]);
+      }
     }
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const float yv = __fsub_rn(blk[i][j], comp[i][j]);
-        const float tv = __fadd_rn(acc[i][j], yv);
-        comp[i][j] = __fsub_rn(__fsub_rn(tv, acc[i][j]), yv);
-        acc[i][j] = tv;
-      }
+    for (int i = 0; i < 8; ++i) {
+      acc[i][0] += (double)blk[i][0];
+      acc[i][1] += (double)blk[i][1];
+    }
+    if (more) store_chunk(buf ^ 1);
     __syncthreads();
+    buf ^= 1;
   }
-  float* out = part + (int64_t)blockIdx.z * N * E;
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int64_t t = t0 + ty * 4 + i;
+  for (int i = 0; i < 8; ++i) {
+    const int64_t t = t0 + ty * 8 + i;
     if (t >= N) continue;
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int e = e0 + tx * 4 + j;
-      if (e < E) out[t * E + e] = __fsub_rn(acc[i][j], comp[i][j]);
+    for (int j = 0; j < 2; ++j) {
+      const int e = e0 + tx * 2 + j;
+      if (e >= E) continue;
+      if (splits == 1) logits[t * E + e] = (float)acc[i][j];
+      else part[((int64_t)blockIdx.z * N + t) * E + e] = acc[i][j];
     }
   }
 }
 
-// Split-K partials -> logits, one thread per (token, expert): the <= 64 fp32
-// partials are summed in double (two interleaved chains; exact unless their
-// exponents span more than ~29 bits) and rounded once to fp32.
-__global__ void __launch_bounds__(256) k_reduce_partials(const float* __restrict__ part,
+// Split-K partials (double) -> logits, one thread per (token, expert): summed
+// in split order in double and rounded once to fp32.
+__global__ void __launch_bounds__(256) k_reduce_partials(const double* __restrict__ part,
                                                          int splits, int64_t NE,
                                                          float* __restrict__ logits) {
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < NE;
        i += (int64_t)gridDim.x * blockDim.x) {
-    double a0 = 0.0, a1 = 0.0;
-    int z = 0;
-    for (; z + 1 < splits; z += 2) {  // two independent chains, joined in order below
-      a0 += (double)part[(int64_t)z * NE + i];
-      a1 += (double)part[(int64_t)(z + 1) * NE + i];
-    }
-    if (z < splits) a0 += (double)part[(int64_t)z * NE + i];
-    logits[i] = (float)(a0 + a1);
+    double a = 0.0;
+    for (int z = 0; z < splits; ++z) a += part[(int64_t)z * NE + i];
+    logits[i] = (float)a;
   }
 }
 
@@ -234,44 +252,46 @@ int route_splits(int64_t N, int E, int d_r) {
   int64_t tiles = ((E + GE - 1) / GE) * ((N + GT - 1) / GT);
   if (tiles < 1) tiles = 1;
   const int nk = d_r / GK > 0 ? d_r / GK : 1;
-  int64_t want = (296 + tiles - 1) / tiles;
-  int64_t maxs = nk / 4 > 0 ? nk / 4 : 1;
+  int64_t want = (296 + tiles - 1) / tiles;  // about two CTAs per SM
+  int64_t maxs = nk / 4 > 0 ? nk / 4 : 1;    // at least 4 chunks per split
   if (want > maxs) want = maxs;
-  if (want > 64) want = 64;
+  if (want > 32) want = 32;
   if (want < 1) want = 1;
   const int cps = (int)((nk + want - 1) / want);
   return (nk + cps - 1) / cps;
 }
 
+// Router scratch: [logits N x E fp32][partials splits x N x E double, if split]
 size_t route_partial_bytes(int64_t N, int E, int d_r) {
   const int splits = route_splits(N, E, d_r);
   const size_t ne = (size_t)N * (size_t)E;
-  return align_up(sizeof(float) * (size_t)splits * ne, 256) +
-         (splits > 1 ? align_up(sizeof(float) * ne, 256) : 0);
+  return align_up(sizeof(float) * ne, 256) +
+         (splits > 1 ? align_up(sizeof(double) * (size_t)splits * ne, 256) : 0);
 }
 
-float* route_logits_of(float* part, int64_t N, int E, int splits) {
-  if (splits <= 1) return part;
-  return reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(part) +
-                                  align_up(sizeof(float) * (size_t)splits * N * E, 256));
+float* route_logits_of(void* scratch) { return static_cast<float*>(scratch); }
+
+static double* route_part_of(void* scratch, int64_t N, int E) {
+  return reinterpret_cast<double*>(static_cast<uint8_t*>(scratch) +
+                                   align_up(sizeof(float) * (size_t)N * (size_t)E, 256));
 }
 
-cudaError_t launch_reduce_partials(const float* part, int splits, int64_t N, int E,
-                                   float* logits, cudaStream_t s) {
-  const int64_t ne = N * (int64_t)E;
-  int64_t blocks = (ne + 255) / 256;
-  const int64_t cap = (int64_t)dev_info()->sm_count * 16;
-  if (blocks > cap) blocks = cap;
-  k_reduce_partials<<<(unsigned)blocks, 256, 0, s>>>(part, splits, ne, logits);
-  return cudaGetLastError();
-}
-
-cudaError_t launch_gate_partial(const __nv_bfloat16* x, int64_t N, int d_r, const float* W, int E,
-                                int splits, float* part, cudaStream_t s) {
+cudaError_t launch_gate(const __nv_bfloat16* x, int64_t N, int d_r, const float* W, int E,
+                        void* scratch, cudaStream_t s) {
+  const int splits = route_splits(N, E, d_r);
   const int nk = d_r / GK;
   const int cps = (nk + splits - 1) / splits;
+  float* logits = route_logits_of(scratch);
+  double* part = route_part_of(scratch, N, E);
   dim3 grid((E + GE - 1) / GE, (unsigned)((N + GT - 1) / GT), splits);
-  k_gate_partial<<<grid, 256, 0, s>>>(x, N, d_r, W, E, cps, part);
+  k_gate_partial<<<grid, 256, 0, s>>>(x, N, d_r, W, E, cps, splits, logits, part);
+  if (splits > 1) {
+    const int64_t ne = N * (int64_t)E;
+    int64_t blocks = (ne + 255) / 256;
+    const int64_t cap = (int64_t)dev_info()->sm_count * 16;
+    if (blocks > cap) blocks = cap;
+    k_reduce_partials<<<(unsigned)blocks, 256, 0, s>>>(part, splits, ne, logits);
+  }
   return cudaGetLastError();
 }
 
