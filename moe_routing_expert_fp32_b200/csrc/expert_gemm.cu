@@ -24,8 +24,8 @@
 //   * three variants by average rows per expert: decode (NTMAX 32, 10 stages:
 //     ~160 KB of weights in flight per SM, weights loaded with an L2
 //     evict-first hint since each is read once), mid (NTMAX 128, two A blocks
-//     and accumulators per unit, 4 stages) and large (NTMAX 256, 4 stages:
-//     128x256x16 MMAs).
+//     and accumulators per unit, 4 stages) and large (a CTA pair running
+//     256x256x16 cta_group::2 MMAs, 6 stages; see k_expert_gemm_pair).
 //   * the page's rounding points: g, u rounded to bf16; SiLU output rounded to
 //     bf16 before the product; SiTU evaluated in fp32; h and y rounded to bf16.
 //   * unit u -> (token tile, weight-row block), row block fastest: CTAs that
@@ -464,6 +464,300 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
+// ------------------------------------------------------------ CTA-pair variant
+// Large variant on a CTA pair (cluster of 2, tcgen05 cta_group::2): one MMA is
+// M = 256 weight rows (128 per CTA, each from its own shared memory) x N = up
+// to 256 token rows (N/2 rows held by each CTA), accumulating into each CTA's
+// own TMEM (its 128 rows x N).  Each CTA therefore fetches half of the token
+// tile it multiplies with, which halves the operand bytes per FLOP that every
+// SM pulls from L2.  No TMA multicast: each CTA loads its own operands.
+// Protocol:
+//   full[s]   (even CTA only) one arrive.expect_tx by the even CTA's producer
+//             for both CTAs' bytes; both CTAs' TMA loads credit it;
+//   empty[s]  (both CTAs) the MMA commit is multicast to both;
+//   tfull[b]  (both CTAs) the MMA commit is multicast to both;
+//   tempty[b] (even CTA) 256 arrivals: the epilogue threads of both CTAs.
+// Cluster barriers after set-up and before freeing TMEM; every mbarrier wait
+// is bounded as in the single-CTA kernel.
+constexpr uint32_t kPeerBitMask = 0xFEFFFFFFu;  // clears the pair-rank bit of a cluster address
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::
+                   : "memory");
+}
+__device__ __forceinline__ uint32_t peer_addr(uint32_t local, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(local), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
+               : "memory");
+}
+__device__ __forceinline__ void tma_load_2d_pair(const CUtensorMap* map, uint64_t* bar, void* dst,
+                                                 int c0, int c1) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar) & kPeerBitMask), "r"(c0), "r"(c1)
+      : "memory");
+}
+__device__ __forceinline__ void tma_load_3d_pair(const CUtensorMap* map, uint64_t* bar, void* dst,
+                                                 int c0, int c1, int c2) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar) & kPeerBitMask), "r"(c0), "r"(c1),
+      "r"(c2)
+      : "memory");
+}
+__device__ __forceinline__ void umma_bf16_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                               uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate));
+}
+__device__ __forceinline__ void umma_commit_pair(uint64_t* bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
+      " [%0], %1;" ::"r"(smem_u32(bar)),
+      "h"((uint16_t)0x3)
+      : "memory");
+}
+__device__ __forceinline__ uint32_t idesc_bf16_m256(int n) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) |
+         ((uint32_t)(256 >> 4) << 24);
+}
+
+constexpr int kPairNt = 256;     // token rows per tile (N, split 128 + 128)
+constexpr int kPairStages = 6;   // (A 16 KB + B half 16 KB) per stage
+
+struct PairCfg {
+  static constexpr int kABytes = BM * BK * 2;
+  static constexpr int kBBytes = (kPairNt / 2) * BK * 2;
+  static constexpr int kStageBytes = kABytes + kBBytes;
+  static constexpr int kBufCols = kPairNt;
+  static constexpr int kTmemCols = 2 * kPairNt;
+  static constexpr size_t kSmem = (size_t)kPairStages * kStageBytes + 1024 + 256 + kXchgBytes;
+  static_assert(kSmem <= 227 * 1024, "shared memory");
+};
+
+template <int MODE>
+__global__ void __launch_bounds__(kThreads, 1)
+    k_expert_gemm_pair(const __grid_constant__ CUtensorMap tmA0,
+                       const __grid_constant__ CUtensorMap tmA1,
+                       const __grid_constant__ CUtensorMap tmB,
+                       const __grid_constant__ CUtensorMap tmB64,
+                       const int32_t* __restrict__ offsets, const int32_t* __restrict__ tile_start,
+                       int E, int M_rows, int Kdim, __nv_bfloat16* __restrict__ out, int act_kind,
+                       float beta, float lbeta, DeviceStatus* st) {
+  using C = PairCfg;
+  constexpr int STAGES = kPairStages;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * C::kStageBytes);
+  uint64_t* empty = full + STAGES;
+  uint64_t* tfull = empty + STAGES;
+  uint64_t* tempty = tfull + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + 2);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  float* xchg = reinterpret_cast<float*>(smem + STAGES * C::kStageBytes + 256);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_rank();  // 0: issues the MMAs for the pair
+  const bool leader = rank == 0;
+  const int pair_id = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+  // rows of the output per CTA: 64 d_ff rows (gate_up) or 128 d rows (down)
+  const int blk_rows = (MODE == kGateUp) ? kGateUpRows : BM;
+  const int unit_rows = 2 * blk_rows;
+  const int RB = (M_rows + unit_rows - 1) / unit_rows;
+  const int KB = Kdim / BK;
+  const int64_t total_units = (int64_t)tile_start[E] * RB;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tfull[b], 1);
+      mbar_init(&tempty[b], 256);
+    }
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(tmem_slot)),
+                 "r"(C::kTmemCols));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;");
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync_all();  // both CTAs' barriers exist before any remote arrive / credit
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------ TMA producer (both CTAs)
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int64_t u = pair_id; u < total_units && ok; u += npairs) {
+        const Unit w = decode_unit(u, RB, kPairNt, tile_start, offsets, E);
+        const int n = ((w.nrows + 15) / 16) * 16;
+        const int half = n / 2;  // token rows this CTA contributes
+        const bool big = half > 2 * kBoxRows;
+        const int brows = big ? kBigBoxRows : kBoxRows;
+        const int nb = (half + brows - 1) / brows;
+        const uint32_t cta_bytes = C::kABytes + nb * brows * BK * 2;
+        const int ra = w.rb * unit_rows + rank * blk_rows;
+        const int tb = w.row0 + rank * half;
+        for (int kb = 0; kb < KB; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag)) { ok = false; break; }
+          uint8_t* sA = smem + stage * C::kStageBytes;
+          uint8_t* sB = sA + C::kABytes;
+          if (leader) mbar_arrive_expect_tx(&full[stage], 2 * cta_bytes);
+          if (MODE == kGateUp) {
+            tma_load_3d_pair(&tmA0, &full[stage], sA, kb * BK, ra, w.e);
+            tma_load_3d_pair(&tmA1, &full[stage], sA + kGateUpRows * BK * 2, kb * BK, ra, w.e);
+          } else {
+            tma_load_3d_pair(&tmA0, &full[stage], sA, kb * BK, ra, w.e);
+          }
+          for (int i = 0; i < nb; ++i)
+            tma_load_2d_pair(big ? &tmB64 : &tmB, &full[stage], sB + i * brows * BK * 2, kb * BK,
+                             tb + i * brows);
+          if (++stage == STAGES) { stage = 0; phase ^= 1; }
+        }
+      }
+      if (!ok) {
+        record_error(st, MOE_ERR_DEVICE_TIMEOUT, 200 + MODE);
+        *abort_flag = 1;
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------ MMA issuer (even CTA)
+    if (lane == 0 && leader) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int local = 0;
+      bool ok = true;
+      for (int64_t u = pair_id; u < total_units && ok; u += npairs, ++local) {
+        const Unit w = decode_unit(u, RB, kPairNt, tile_start, offsets, E);
+        const int n = ((w.nrows + 15) / 16) * 16;
+        const uint32_t idesc = idesc_bf16_m256(n);
+        const int buf = local & 1;
+        const uint32_t tphase = (local >> 1) & 1;
+        if (!mbar_wait(&tempty[buf], tphase ^ 1, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t d0 = tmem_base + buf * C::kBufCols;
+        for (int kb = 0; kb < KB; ++kb) {
+          if (!mbar_wait(&full[stage], phase, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(smem + stage * C::kStageBytes);
+          const uint32_t b0 = a0 + C::kABytes;
+#pragma unroll
+          for (int k = 0; k < BK / UK; ++k)
+            umma_bf16_pair(d0, sw128_desc(a0 + k * UK * 2), sw128_desc(b0 + k * UK * 2), idesc,
+                           (kb | k) != 0);
+          umma_commit_pair(&empty[stage]);
+          if (++stage == STAGES) { stage = 0; phase ^= 1; }
+        }
+        if (ok) umma_commit_pair(&tfull[buf]);
+      }
+      if (!ok) {
+        record_error(st, MOE_ERR_DEVICE_TIMEOUT, 210 + MODE);
+        *abort_flag = 1;
+      }
+    }
+  } else {
+    // ------------------------------------------------------ epilogue (both CTAs)
+    const int quarter = warp & 3;
+    const bool has_lb = !(lbeta == 0.0f || lbeta != lbeta);
+    const float b_eff = (beta == 0.0f || beta != beta) ? 1.0f : beta;
+    const uint32_t tempty_leader0 = peer_addr(smem_u32(&tempty[0]), 0);
+    int local = 0;
+    uint32_t xbuf = 0;
+    for (int64_t u = pair_id; u < total_units; u += npairs, ++local) {
+      const Unit w = decode_unit(u, RB, kPairNt, tile_start, offsets, E);
+      const int buf = local & 1;
+      const uint32_t tphase = (local >> 1) & 1;
+      if (!mbar_wait(&tfull[buf], tphase, abort_flag)) {
+        if (lane == 0) record_error(st, MOE_ERR_DEVICE_TIMEOUT, 220 + MODE);
+        *abort_flag = 1;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + buf * C::kBufCols;
+      const int r0 = w.rb * unit_rows + rank * blk_rows;
+      if (MODE == kGateUp) {
+        const int pair = quarter & 1;
+        const bool is_g = quarter < 2;
+        const int f = r0 + pair * 32 + lane;
+        __nv_bfloat16* col = out + f;
+        const bool live = f < M_rows;
+        for (int c0 = 0; c0 < w.nrows; c0 += 16, ++xbuf) {
+          float v[16];
+          tmem_ld16(taddr + c0, v);
+          float* xg = xchg + ((pair * 2 + (xbuf & 1)) * 2 + 0) * 256;
+          float* xu = xchg + ((pair * 2 + (xbuf & 1)) * 2 + 1) * 256;
+          float4* mine = reinterpret_cast<float4*>((is_g ? xg : xu) + lane * 8);
+          const float* give = is_g ? v + 8 : v;
+          mine[0] = make_float4(give[0], give[1], give[2], give[3]);
+          mine[1] = make_float4(give[4], give[5], give[6], give[7]);
+          asm volatile("bar.sync %0, 64;" ::"r"(1 + pair) : "memory");
+          const float4* theirs = reinterpret_cast<const float4*>((is_g ? xu : xg) + lane * 8);
+          const float4 t0 = theirs[0], t1 = theirs[1];
+          const float other[8] = {t0.x, t0.y, t0.z, t0.w, t1.x, t1.y, t1.z, t1.w};
+          const int cbase = c0 + (is_g ? 0 : 8);
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const float g = is_g ? v[j] : other[j];
+            const float uu = is_g ? other[j] : v[8 + j];
+            const float h = act_kind == MOE_ACT_SITU ? situ_mul(g, uu, b_eff, lbeta, has_lb)
+                                                     : silu_mul(g, uu);
+            if (live && cbase + j < w.nrows)
+              col[(int64_t)(w.row0 + cbase + j) * M_rows] = __float2bfloat16_rn(h);
+          }
+        }
+      } else {
+        const int m = r0 + quarter * 32 + lane;
+        __nv_bfloat16* col = out + m;
+        const int lim_m = m < M_rows ? 16 : 0;
+        for (int c0 = 0; c0 < w.nrows; c0 += 16) {
+          float v[16];
+          tmem_ld16(taddr + c0, v);
+          int lim = w.nrows - c0 < 16 ? w.nrows - c0 : 16;
+          lim = lim < lim_m ? lim : lim_m;
+#pragma unroll
+          for (int j = 0; j < 16; ++j)
+            if (j < lim) col[(int64_t)(w.row0 + c0 + j) * M_rows] = __float2bfloat16_rn(v[j]);
+        }
+      }
+      tc_fence_before();
+      // release the buffer to the even CTA's MMA issuer
+      mbar_arrive_remote(tempty_leader0 + buf * (uint32_t)sizeof(uint64_t));
+    }
+  }
+  __syncthreads();
+  cluster_sync_all();  // no MMA of the pair is still writing either CTA's TMEM
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
+                 "r"(C::kTmemCols));
+  }
+}
+
 // Token tiles per expert and their prefix: tile_start[e] = sum_{e'<e}
 // ceil(n_e'/nt), tile_start[E] = total.  Inconsistent offsets are recorded
 // and give the expert no tile, so the GEMM never reads outside xs.
@@ -574,13 +868,54 @@ cudaError_t launch_gemm(const CUtensorMap& a0, const CUtensorMap& a1, const CUte
   return cudaGetLastError();
 }
 
+// Launches the CTA-pair kernel on as many pairs as can be resident at once.
+template <int MODE>
+cudaError_t launch_gemm_pair(const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorMap& b,
+                             const CUtensorMap& b64, const int32_t* offsets,
+                             const int32_t* tile_start, int E, int M_rows, int Kdim,
+                             __nv_bfloat16* out, const moe_act_cfg& act, DeviceStatus* st,
+                             cudaStream_t s) {
+  using C = PairCfg;
+  static bool attr_set[64] = {false};
+  static int grid_of[64] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = C::kSmem;
+  cfg.stream = s;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (dev < 64 && !attr_set[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(k_expert_gemm_pair<MODE>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)C::kSmem);
+    if (e != cudaSuccess) return e;
+    int pairs = 0;
+    cfg.gridDim = dim3(dev_info()->sm_count & ~1, 1, 1);
+    e = cudaOccupancyMaxActiveClusters(&pairs, k_expert_gemm_pair<MODE>, &cfg);
+    if (e != cudaSuccess || pairs < 1) pairs = dev_info()->sm_count / 2;
+    if (pairs > dev_info()->sm_count / 2) pairs = dev_info()->sm_count / 2;
+    grid_of[dev] = 2 * pairs;
+    attr_set[dev] = true;
+  }
+  cfg.gridDim = dim3(grid_of[dev < 64 ? dev : 0], 1, 1);
+  return cudaLaunchKernelEx(&cfg, k_expert_gemm_pair<MODE>, a0, a1, b, b64, offsets, tile_start,
+                            E, M_rows, Kdim, out, (int)act.kind, act.beta, act.linear_beta, st);
+}
+
 // Variant choice from shapes only (no host round trip), by the average rows
 // per expert S / E: decode (<= 16: weight stream, deep ring of small stages),
 // mid (<= 128: weight-bound; two 128-row A blocks per unit halve the token
-// tile traffic per weight byte), large (tensor-bound: 128x256 MMAs).
+// tile traffic per weight byte), large (tensor-bound: the CTA-pair kernel,
+// 256x256 MMAs).
 constexpr int kNtDecode = 32, kStagesDecode = 10, kUmDecode = 1;
 constexpr int kNtMid = 128, kStagesMid = 4, kUmMid = 2;
-constexpr int kNtLarge = 256, kStagesLarge = 4, kUmLarge = 1;
 
 enum Variant { kVarDecode = 0, kVarMid = 1, kVarLarge = 2 };
 
@@ -604,8 +939,8 @@ cudaError_t launch_variant(Variant v, const CUtensorMap& a0, const CUtensorMap& 
       return launch_gemm<MODE, kNtMid, kStagesMid, kUmMid>(a0, a1, b, b64, offsets, tile_start, E, M_rows,
                                                    Kdim, out, act, st, s);
     default:
-      return launch_gemm<MODE, kNtLarge, kStagesLarge, kUmLarge>(a0, a1, b, b64, offsets, tile_start, E,
-                                                       M_rows, Kdim, out, act, st, s);
+      return launch_gemm_pair<MODE>(a0, a1, b, b64, offsets, tile_start, E, M_rows, Kdim, out,
+                                    act, st, s);
   }
 }
 
@@ -630,7 +965,7 @@ int expert_ffn_run(const __nv_bfloat16* xs, const int32_t* offsets, int E, int64
       !make_map_2d(&mxs64, xs, d_e, S, kBigBoxRows) || !make_map_2d(&mh64, h, F, S, kBigBoxRows))
     return MOE_ERR_CUDA;
   const Variant var = pick_variant(S, E);
-  const int nt = var == kVarDecode ? kNtDecode : (var == kVarMid ? kNtMid : kNtLarge);
+  const int nt = var == kVarDecode ? kNtDecode : (var == kVarMid ? kNtMid : kPairNt);
   k_tiles<<<1, 1024, 0, s>>>(offsets, E, S, nt, tile_start, st);
   if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
   cudaError_t rc = launch_variant<kGateUp>(var, mw1, mw3, mxs, mxs64, offsets, tile_start, E, F,
