@@ -187,12 +187,6 @@ def run_ours(args, rank, world, local_rank):
     for _ in range(max(args.warmup, 3)):
         flush.zero_()
         step()
-    # per-step events: start + one per stage
-    ev = [{"start": torch.cuda.Event(enable_timing=True),
-           **{n: torch.cuda.Event(enable_timing=True) for n in names}} for _ in range(args.steps)]
-    for e in ev:  # create the CUDA events before handing their handles to the library
-        for v in e.values():
-            v.record()
     torch.cuda.synchronize()
 
     def barrier():
@@ -200,25 +194,43 @@ def run_ours(args, rank, world, local_rank):
             import torch.distributed as dist
             dist.barrier()
 
+    # timed region: K steps, one start/end event pair around each moe_forward
+    ev0 = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
     with ClockSampler(local_rank) as clk:
         barrier()
         torch.cuda.synchronize()
         t0 = time.perf_counter()
         for i in range(args.steps):
             flush.zero_()
-            ev[i]["start"].record()
-            step(events={n: ev[i][n] for n in names})
+            ev0[i][0].record()
+            step()
+            ev0[i][1].record()
         torch.cuda.synchronize()
         barrier()
         wall = time.perf_counter() - t0
-    step_ms = [e["start"].elapsed_time(e["after_combine"]) for e in ev]
+    ms = statistics.mean(a.elapsed_time(b) for a, b in ev0)
+
+    # breakdown pass: the same steps with an event after every stage (events
+    # between the two expert kernels hold back the second one's early start,
+    # so this pass is used for the per-stage times only)
+    ev = [{"start": torch.cuda.Event(enable_timing=True),
+           **{n: torch.cuda.Event(enable_timing=True) for n in names}} for _ in range(args.steps)]
+    for e in ev:  # create the CUDA events before handing their handles to the library
+        for v in e.values():
+            v.record()
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        flush.zero_()
+        ev[i]["start"].record()
+        step(events={n: ev[i][n] for n in names})
+    torch.cuda.synchronize()
     stage_ms = {}
     prev = "start"
     for n in names:
         stage_ms[n.replace("after_", "")] = statistics.mean(
             e[prev].elapsed_time(e[n]) for e in ev)
         prev = n
-    ms = statistics.mean(step_ms)
 
     # routing statistics of the timed batch (for the algorithmic byte count)
     step(idx=counts_probe)

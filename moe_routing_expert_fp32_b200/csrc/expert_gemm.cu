@@ -53,12 +53,15 @@ constexpr uint64_t kTimeoutNs = 2000000000ull;
 
 enum Mode { kGateUp = 0, kDown = 1 };
 
-// UM = A blocks (of 128 rows) per unit, each with its own accumulator.
-template <int NTMAX, int STAGES, int UM>
+// UM = A blocks (of 128 rows) per unit, each with its own accumulator;
+// KSUB = 64-column sub-tiles per stage (a stage covers 64*KSUB of K, so each
+// weight row is read KSUB*128 contiguous bytes at a time).
+template <int NTMAX, int STAGES, int UM, int KSUB>
 struct Cfg {
   static constexpr int kABlockBytes = BM * BK * 2;
-  static constexpr int kABytes = UM * kABlockBytes;
-  static constexpr int kBBytes = NTMAX * BK * 2;
+  static constexpr int kABytes = UM * KSUB * kABlockBytes;
+  static constexpr int kBSubBytes = NTMAX * BK * 2;
+  static constexpr int kBBytes = KSUB * kBSubBytes;
   static constexpr int kStageBytes = kABytes + kBBytes;
   static constexpr int kBufCols = UM * NTMAX;  // TMEM columns per accumulator buffer
   static constexpr int kTmemCols = (2 * kBufCols < 32) ? 32 : 2 * kBufCols;
@@ -142,6 +145,15 @@ __device__ __forceinline__ void tma_load_3d_hint(const CUtensorMap* map, uint64_
       "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2),
       "l"(policy)
       : "memory");
+}
+
+// Programmatic dependent launch: the dependent kernel waits here until the
+// preceding kernel's memory is visible; a primary lets dependents launch.
+__device__ __forceinline__ void grid_dep_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+__device__ __forceinline__ void grid_dep_launch() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
 __device__ __forceinline__ void tc_fence_before() {
@@ -242,15 +254,16 @@ __device__ __forceinline__ Unit decode_unit(int64_t u, int RB, int nt, const int
   return r;
 }
 
-template <int MODE, int NTMAX, int STAGES, int UM>
+template <int MODE, int NTMAX, int STAGES, int UM, int KSUB>
 __global__ void __launch_bounds__(kThreads, 1)
     k_expert_gemm(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA1,
                   const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmB64,
                   const int32_t* __restrict__ offsets,
                   const int32_t* __restrict__ tile_start, int E, int M_rows, int Kdim,
                   __nv_bfloat16* __restrict__ out, int act_kind, float beta, float lbeta,
-                  DeviceStatus* st) {
-  using C = Cfg<NTMAX, STAGES, UM>;
+                  DeviceStatus* st, int pdl) {
+  using C = Cfg<NTMAX, STAGES, UM, KSUB>;
+  constexpr int KS = BK * KSUB;  // K columns per stage
   constexpr bool kDecode = NTMAX <= 32;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -268,7 +281,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int blk_rows = (MODE == kGateUp) ? kGateUpRows : BM;
   const int unit_rows = UM * blk_rows;
   const int RB = (M_rows + unit_rows - 1) / unit_rows;
-  const int KB = Kdim / BK;
+  const int KB = Kdim / KS;
   const int64_t total_units = (int64_t)tile_start[E] * RB;
 
   if (threadIdx.x == 0) {
@@ -301,44 +314,82 @@ __global__ void __launch_bounds__(kThreads, 1)
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
+      // With programmatic dependent launch the token rows (written by the
+      // preceding kernel) may be read only after grid_dep_wait(); the weight
+      // tiles of the first ring of stages are fetched before it.
+      bool dep_pending = pdl != 0;
       for (int64_t u = blockIdx.x; u < total_units && ok; u += gridDim.x) {
         const Unit w = decode_unit(u, RB, NTMAX, tile_start, offsets, E);
         // token rows: 16-row boxes for short tiles, 64-row boxes otherwise
         const bool big = !kDecode && w.nrows > 2 * kBoxRows;
         const int brows = big ? kBigBoxRows : kBoxRows;
         const int nb = (w.nrows + brows - 1) / brows;
-        const uint32_t bytes = C::kABytes + nb * brows * BK * 2;
+        const uint32_t bytes = C::kABytes + KSUB * nb * brows * BK * 2;
         const int r0 = w.rb * unit_rows;
-        for (int kb = 0; kb < KB; ++kb) {
-          if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag)) { ok = false; break; }
-          uint8_t* sA = smem + stage * C::kStageBytes;
-          uint8_t* sB = sA + C::kABytes;
-          mbar_arrive_expect_tx(&full[stage], bytes);
+        auto load_a = [&](int kb, uint8_t* sA) {
 #pragma unroll
-          for (int a = 0; a < UM; ++a) {
-            uint8_t* dA = sA + a * C::kABlockBytes;
-            const int ra = r0 + a * blk_rows;
-            if (MODE == kGateUp) {
-              // w1 rows ra..ra+63 over w3 rows ra..ra+63
-              void* d3 = dA + kGateUpRows * BK * 2;
-              if (kDecode) {
-                tma_load_3d_hint(&tmA0, &full[stage], dA, kb * BK, ra, w.e, wpol);
-                tma_load_3d_hint(&tmA1, &full[stage], d3, kb * BK, ra, w.e, wpol);
+          for (int sub = 0; sub < KSUB; ++sub) {
+            const int kc = kb * KS + sub * BK;
+#pragma unroll
+            for (int a = 0; a < UM; ++a) {
+              uint8_t* dA = sA + (a * KSUB + sub) * C::kABlockBytes;
+              const int ra = r0 + a * blk_rows;
+              if (MODE == kGateUp) {
+                // w1 rows ra..ra+63 over w3 rows ra..ra+63
+                void* d3 = dA + kGateUpRows * BK * 2;
+                if (kDecode) {
+                  tma_load_3d_hint(&tmA0, &full[stage], dA, kc, ra, w.e, wpol);
+                  tma_load_3d_hint(&tmA1, &full[stage], d3, kc, ra, w.e, wpol);
+                } else {
+                  tma_load_3d(&tmA0, &full[stage], dA, kc, ra, w.e);
+                  tma_load_3d(&tmA1, &full[stage], d3, kc, ra, w.e);
+                }
               } else {
-                tma_load_3d(&tmA0, &full[stage], dA, kb * BK, ra, w.e);
-                tma_load_3d(&tmA1, &full[stage], d3, kb * BK, ra, w.e);
+                if (kDecode) tma_load_3d_hint(&tmA0, &full[stage], dA, kc, ra, w.e, wpol);
+                else tma_load_3d(&tmA0, &full[stage], dA, kc, ra, w.e);
               }
-            } else {
-              if (kDecode) tma_load_3d_hint(&tmA0, &full[stage], dA, kb * BK, ra, w.e, wpol);
-              else tma_load_3d(&tmA0, &full[stage], dA, kb * BK, ra, w.e);
             }
           }
-          for (int i = 0; i < nb; ++i)
-            tma_load_2d(big ? &tmB64 : &tmB, &full[stage], sB + i * brows * BK * 2, kb * BK,
-                        w.row0 + i * brows);
+        };
+        auto load_b = [&](int kb, uint8_t* sB, int st_idx) {
+#pragma unroll
+          for (int sub = 0; sub < KSUB; ++sub)
+            for (int i = 0; i < nb; ++i)
+              tma_load_2d(big ? &tmB64 : &tmB, &full[st_idx],
+                          sB + sub * C::kBSubBytes + i * brows * BK * 2, kb * KS + sub * BK,
+                          w.row0 + i * brows);
+        };
+        int kb = 0;
+        if (dep_pending) {
+          // weights of up to STAGES k-blocks first, then wait, then their tokens
+          const int pre = KB < STAGES ? KB : STAGES;
+          for (; kb < pre; ++kb) {
+            if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag)) { ok = false; break; }
+            mbar_arrive_expect_tx(&full[stage], bytes);
+            load_a(kb, smem + stage * C::kStageBytes);
+            if (++stage == STAGES) { stage = 0; phase ^= 1; }
+          }
+          grid_dep_wait();
+          dep_pending = false;
+          int st_idx = 0;  // the first unit started at stage 0
+          for (int j = 0; j < kb; ++j) {
+            load_b(j, smem + st_idx * C::kStageBytes + C::kABytes, st_idx);
+            if (++st_idx == STAGES) st_idx = 0;
+          }
+          if (!ok) break;
+        }
+        for (; kb < KB; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag)) { ok = false; break; }
+          uint8_t* sA = smem + stage * C::kStageBytes;
+          mbar_arrive_expect_tx(&full[stage], bytes);
+          load_a(kb, sA);
+          load_b(kb, sA + C::kABytes, stage);
           if (++stage == STAGES) { stage = 0; phase ^= 1; }
         }
       }
+      if (dep_pending) grid_dep_wait();
+      // every load of this CTA is issued: let the dependent kernel launch
+      grid_dep_launch();
       if (!ok) {
         record_error(st, MOE_ERR_DEVICE_TIMEOUT, 100 + MODE);
         *abort_flag = 1;
@@ -366,11 +417,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t a0 = smem_u32(smem + stage * C::kStageBytes);
           const uint32_t b0 = a0 + C::kABytes;
 #pragma unroll
-          for (int k = 0; k < BK / UK; ++k)
+          for (int sub = 0; sub < KSUB; ++sub)
 #pragma unroll
-            for (int a = 0; a < UM; ++a)
-              umma_bf16(d0 + a * NTMAX, sw128_desc(a0 + a * C::kABlockBytes + k * UK * 2),
-                        sw128_desc(b0 + k * UK * 2), idesc, (kb | k) != 0);
+            for (int k = 0; k < BK / UK; ++k)
+#pragma unroll
+              for (int a = 0; a < UM; ++a)
+                umma_bf16(d0 + a * NTMAX,
+                          sw128_desc(a0 + (a * KSUB + sub) * C::kABlockBytes + k * UK * 2),
+                          sw128_desc(b0 + sub * C::kBSubBytes + k * UK * 2), idesc,
+                          (kb | sub | k) != 0);
           umma_commit(&empty[stage]);
           if (++stage == STAGES) { stage = 0; phase ^= 1; }
         }
@@ -557,7 +612,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                        const __grid_constant__ CUtensorMap tmB64,
                        const int32_t* __restrict__ offsets, const int32_t* __restrict__ tile_start,
                        int E, int M_rows, int Kdim, __nv_bfloat16* __restrict__ out, int act_kind,
-                       float beta, float lbeta, DeviceStatus* st) {
+                       float beta, float lbeta, DeviceStatus* st, int pdl) {
   using C = PairCfg;
   constexpr int STAGES = kPairStages;
   extern __shared__ uint8_t smem_raw[];
@@ -612,6 +667,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
+      bool dep_pending = pdl != 0;  // see the single-CTA kernel
       for (int64_t u = pair_id; u < total_units && ok; u += npairs) {
         const Unit w = decode_unit(u, RB, kPairNt, tile_start, offsets, E);
         const int n = ((w.nrows + 15) / 16) * 16;
@@ -622,23 +678,45 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t cta_bytes = C::kABytes + nb * brows * BK * 2;
         const int ra = w.rb * unit_rows + rank * blk_rows;
         const int tb = w.row0 + rank * half;
-        for (int kb = 0; kb < KB; ++kb) {
+        auto load_a = [&](int kb, uint8_t* sA, int st_idx) {
+          if (MODE == kGateUp) {
+            tma_load_3d_pair(&tmA0, &full[st_idx], sA, kb * BK, ra, w.e);
+            tma_load_3d_pair(&tmA1, &full[st_idx], sA + kGateUpRows * BK * 2, kb * BK, ra, w.e);
+          } else {
+            tma_load_3d_pair(&tmA0, &full[st_idx], sA, kb * BK, ra, w.e);
+          }
+        };
+        auto load_b = [&](int kb, uint8_t* sB, int st_idx) {
+          for (int i = 0; i < nb; ++i)
+            tma_load_2d_pair(big ? &tmB64 : &tmB, &full[st_idx], sB + i * brows * BK * 2, kb * BK,
+                             tb + i * brows);
+        };
+        int kb = 0;
+        if (dep_pending) {
+          const int pre = KB < STAGES ? KB : STAGES;
+          for (; kb < pre; ++kb) {
+            if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag)) { ok = false; break; }
+            if (leader) mbar_arrive_expect_tx(&full[stage], 2 * cta_bytes);
+            load_a(kb, smem + stage * C::kStageBytes, stage);
+            if (++stage == STAGES) { stage = 0; phase ^= 1; }
+          }
+          grid_dep_wait();
+          dep_pending = false;
+          for (int j = 0; j < kb; ++j)
+            load_b(j, smem + j * C::kStageBytes + C::kABytes, j);
+          if (!ok) break;
+        }
+        for (; kb < KB; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag)) { ok = false; break; }
           uint8_t* sA = smem + stage * C::kStageBytes;
-          uint8_t* sB = sA + C::kABytes;
           if (leader) mbar_arrive_expect_tx(&full[stage], 2 * cta_bytes);
-          if (MODE == kGateUp) {
-            tma_load_3d_pair(&tmA0, &full[stage], sA, kb * BK, ra, w.e);
-            tma_load_3d_pair(&tmA1, &full[stage], sA + kGateUpRows * BK * 2, kb * BK, ra, w.e);
-          } else {
-            tma_load_3d_pair(&tmA0, &full[stage], sA, kb * BK, ra, w.e);
-          }
-          for (int i = 0; i < nb; ++i)
-            tma_load_2d_pair(big ? &tmB64 : &tmB, &full[stage], sB + i * brows * BK * 2, kb * BK,
-                             tb + i * brows);
+          load_a(kb, sA, stage);
+          load_b(kb, sA + C::kABytes, stage);
           if (++stage == STAGES) { stage = 0; phase ^= 1; }
         }
       }
+      if (dep_pending) grid_dep_wait();
+      grid_dep_launch();
       if (!ok) {
         record_error(st, MOE_ERR_DEVICE_TIMEOUT, 200 + MODE);
         *abort_flag = 1;
@@ -846,26 +924,38 @@ bool make_map_2d(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int MODE, int NTMAX, int STAGES, int UM>
+template <int MODE, int NTMAX, int STAGES, int UM, int KSUB>
 cudaError_t launch_gemm(const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorMap& b,
-                        const CUtensorMap& b64, const int32_t* offsets, const int32_t* tile_start, int E, int M_rows,
-                        int Kdim, __nv_bfloat16* out, const moe_act_cfg& act, DeviceStatus* st,
-                        cudaStream_t s) {
-  using C = Cfg<NTMAX, STAGES, UM>;
+                        const CUtensorMap& b64, const int32_t* offsets, const int32_t* tile_start,
+                        int E, int M_rows, int Kdim, __nv_bfloat16* out, const moe_act_cfg& act,
+                        DeviceStatus* st, cudaStream_t s) {
+  using C = Cfg<NTMAX, STAGES, UM, KSUB>;
   static bool attr_set[64] = {false};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 64 && !attr_set[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(k_expert_gemm<MODE, NTMAX, STAGES, UM>,
+    cudaError_t e = cudaFuncSetAttribute(k_expert_gemm<MODE, NTMAX, STAGES, UM, KSUB>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)C::kSmem);
     if (e != cudaSuccess) return e;
     attr_set[dev] = true;
   }
-  k_expert_gemm<MODE, NTMAX, STAGES, UM><<<dev_info()->sm_count, kThreads, C::kSmem, s>>>(
-      a0, a1, b, b64, offsets, tile_start, E, M_rows, Kdim, out, act.kind, act.beta,
-      act.linear_beta, st);
-  return cudaGetLastError();
+  // The down projection is launched as a programmatic dependent of the gate_up
+  // kernel: its CTAs start as gate_up CTAs retire and prefetch w2 tiles.
+  const int pdl = MODE == kDown ? 1 : 0;
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.gridDim = dim3(dev_info()->sm_count, 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = C::kSmem;
+  cfg.stream = s;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, k_expert_gemm<MODE, NTMAX, STAGES, UM, KSUB>, a0, a1, b, b64,
+                            offsets, tile_start, E, M_rows, Kdim, out, (int)act.kind, act.beta,
+                            act.linear_beta, st, pdl);
 }
 
 // Launches the CTA-pair kernel on as many pairs as can be resident at once.
@@ -881,16 +971,19 @@ cudaError_t launch_gemm_pair(const CUtensorMap& a0, const CUtensorMap& a1, const
   int dev = 0;
   cudaGetDevice(&dev);
   cudaLaunchConfig_t cfg = {};
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 2;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.blockDim = dim3(kThreads, 1, 1);
   cfg.dynamicSmemBytes = C::kSmem;
   cfg.stream = s;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
+  const int pdl = MODE == kDown ? 1 : 0;
   if (dev < 64 && !attr_set[dev]) {
     cudaError_t e = cudaFuncSetAttribute(k_expert_gemm_pair<MODE>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -905,8 +998,10 @@ cudaError_t launch_gemm_pair(const CUtensorMap& a0, const CUtensorMap& a1, const
     attr_set[dev] = true;
   }
   cfg.gridDim = dim3(grid_of[dev < 64 ? dev : 0], 1, 1);
+  cfg.numAttrs = pdl ? 2 : 1;
   return cudaLaunchKernelEx(&cfg, k_expert_gemm_pair<MODE>, a0, a1, b, b64, offsets, tile_start,
-                            E, M_rows, Kdim, out, (int)act.kind, act.beta, act.linear_beta, st);
+                            E, M_rows, Kdim, out, (int)act.kind, act.beta, act.linear_beta, st,
+                            pdl);
 }
 
 // Variant choice from shapes only (no host round trip), by the average rows
@@ -914,8 +1009,8 @@ cudaError_t launch_gemm_pair(const CUtensorMap& a0, const CUtensorMap& a1, const
 // mid (<= 128: weight-bound; two 128-row A blocks per unit halve the token
 // tile traffic per weight byte), large (tensor-bound: the CTA-pair kernel,
 // 256x256 MMAs).
-constexpr int kNtDecode = 32, kStagesDecode = 10, kUmDecode = 1;
-constexpr int kNtMid = 128, kStagesMid = 4, kUmMid = 2;
+constexpr int kNtDecode = 32, kStagesDecode = 5, kUmDecode = 1, kKsubDecode = 2;
+constexpr int kNtMid = 128, kStagesMid = 4, kUmMid = 2, kKsubMid = 1;
 
 enum Variant { kVarDecode = 0, kVarMid = 1, kVarLarge = 2 };
 
@@ -933,10 +1028,10 @@ cudaError_t launch_variant(Variant v, const CUtensorMap& a0, const CUtensorMap& 
                            cudaStream_t s) {
   switch (v) {
     case kVarDecode:
-      return launch_gemm<MODE, kNtDecode, kStagesDecode, kUmDecode>(a0, a1, b, b64, offsets, tile_start, E,
+      return launch_gemm<MODE, kNtDecode, kStagesDecode, kUmDecode, kKsubDecode>(a0, a1, b, b64, offsets, tile_start, E,
                                                          M_rows, Kdim, out, act, st, s);
     case kVarMid:
-      return launch_gemm<MODE, kNtMid, kStagesMid, kUmMid>(a0, a1, b, b64, offsets, tile_start, E, M_rows,
+      return launch_gemm<MODE, kNtMid, kStagesMid, kUmMid, kKsubMid>(a0, a1, b, b64, offsets, tile_start, E, M_rows,
                                                    Kdim, out, act, st, s);
     default:
       return launch_gemm_pair<MODE>(a0, a1, b, b64, offsets, tile_start, E, M_rows, Kdim, out,
