@@ -94,9 +94,9 @@ typedef struct moe_act_cfg {
   float linear_beta;
 } moe_act_cfg;
 
-/* Expert-shape limits: d (hidden width of the experts) and F (d_ff) are
- * multiples of 128; d_r (router width) is a multiple of 8; all bf16 row
- * pointers 16-byte aligned. */
+/* Shape limits: d (hidden width of the experts) and F (d_ff) are multiples
+ * of 128; d_r (router width) is a multiple of 32; all bf16 row pointers
+ * 16-byte aligned. */
 
 /* ------------------------------------------------------------------ router */
 
@@ -115,10 +115,21 @@ MOE_API size_t moe_route_workspace_size(int64_t N, int d_r, const moe_route_cfg*
  *     topk_w /= (sum_k topk_w + 1e-20), summed in k order; topk_w *= route_scale
  * x: [N, d_r] bf16; W: [E, d_r] fp32; bias: [E] fp32 or NULL;
  * topk_idx: [N, K] int32 out; topk_w: [N, K] fp32 out.
- * The logits are accumulated in fp32 (the page's fp32 F.linear). */
+ * The logits are fp32-accurate (the page's fp32 F.linear; see moe_gate_logits). */
 MOE_API int moe_route(const moe_bf16* x, int64_t N, int d_r, const float* W, const float* bias,
                       const moe_route_cfg* cfg, int32_t* topk_idx, float* topk_w, void* ws,
                       size_t ws_bytes, void* stream);
+
+/* The router's gate GEMM alone ("Kimi K2 · Affinities", gate-forward: the
+ * F.linear of the fp32-upcast hidden states with the fp32 weight):
+ * logits[t, e] = fp32(sum_j x[t, j] * W[e, j]), x: [N, d_r] bf16, W: [E, d_r]
+ * fp32, logits: [N, E] fp32 out.  Same kernels as moe_route: fp32 FMA chains
+ * of 32 terms added in double for small batches; for batches that fill the
+ * GPU, exact int8 tensor-core products of 7-bit digits of x and W (error
+ * below ~2e-8 for unit-scale logits).  Scratch: moe_gate_logits_workspace_size. */
+MOE_API size_t moe_gate_logits_workspace_size(int64_t N, int d_r, int E);
+MOE_API int moe_gate_logits(const moe_bf16* x, int64_t N, int d_r, const float* W, int E,
+                            float* logits, void* ws, size_t ws_bytes, void* stream);
 
 /* Selection and weights only, from caller-supplied fp32 logits [N, E]: the
  * same computation as moe_route after its gate GEMM.  Bit-exact: sigmoid is

@@ -76,6 +76,7 @@ class ActConfig:
 
 _lib = None
 EXPORTS = ("moe_route_workspace_size", "moe_route", "moe_route_from_logits",
+           "moe_gate_logits_workspace_size", "moe_gate_logits",
            "moe_dispatch_workspace_size", "moe_dispatch", "moe_expert_ffn_workspace_size",
            "moe_expert_ffn", "moe_combine_workspace_size", "moe_combine", "moe_workspace_size",
            "moe_forward", "moe_get_status", "moe_strerror", "moe_dispatch_static")
@@ -96,6 +97,8 @@ def lib() -> ctypes.CDLL:
         "moe_route_workspace_size": ([i64, i32, rc], sz),
         "moe_route": ([vp, i64, i32, vp, vp, rc, vp, vp, vp, sz, vp], i32),
         "moe_route_from_logits": ([vp, i64, vp, rc, vp, vp, vp, sz, vp], i32),
+        "moe_gate_logits_workspace_size": ([i64, i32, i32], sz),
+        "moe_gate_logits": ([vp, i64, i32, vp, i32, vp, vp, sz, vp], i32),
         "moe_dispatch_workspace_size": ([i64, i32, i32], sz),
         "moe_dispatch": ([vp, i64, i32, i32, vp, i32, vp, vp, vp, vp, vp, vp, sz, vp], i32),
         "moe_expert_ffn_workspace_size": ([i64, i32, i32, i32], sz),
@@ -172,6 +175,21 @@ def route(x, W, bias, cfg: RouteConfig, ws=None):
     _check("moe_route", lib().moe_route(_ptr(x), N, d_r, _ptr(W), _ptr(bias), ctypes.byref(c),
                                         _ptr(idx), _ptr(w), _ptr(ws), ws.numel(), _stream()))
     return idx, w
+
+
+def gate_logits(x, W, ws=None):
+    """fp32 logits [N, E] of the router's gate GEMM (moe_gate_logits)."""
+    torch = _torch()
+    N, d_r = x.shape
+    E = W.shape[0]
+    _need(x, torch.bfloat16, name="x")
+    _need(W, torch.float32, (E, d_r), "W")
+    need = lib().moe_gate_logits_workspace_size(N, d_r, E)
+    ws = workspace(need, x.device) if ws is None else ws
+    out = torch.empty((N, E), dtype=torch.float32, device=x.device)
+    _check("moe_gate_logits", lib().moe_gate_logits(_ptr(x), N, d_r, _ptr(W), E, _ptr(out),
+                                                    _ptr(ws), ws.numel(), _stream()))
+    return out
 
 
 def route_from_logits(logits, bias, cfg: RouteConfig, ws=None):

@@ -84,7 +84,7 @@ int route_impl(const __nv_bfloat16* x, int64_t N, int d_r, const float* W, const
                const moe_route_cfg& cfg, int32_t* idx, float* w, uint8_t* scratch,
                DeviceStatus* st, cudaStream_t s) {
   const int E = cfg.num_experts;
-  if (launch_gate(x, N, d_r, W, E, scratch, s) != cudaSuccess) return MOE_ERR_CUDA;
+  if (launch_gate(x, N, d_r, W, E, scratch, st, s) != cudaSuccess) return MOE_ERR_CUDA;
   if (launch_select(route_logits_of(scratch), 1, N, bias, cfg, idx, w, st, s) != cudaSuccess)
     return MOE_ERR_CUDA;
   return MOE_OK;
@@ -143,6 +143,34 @@ int moe_route(const moe_bf16* x, int64_t N, int d_r, const float* W, const float
   if (N == 0) return MOE_OK;
   return route_impl(reinterpret_cast<const __nv_bfloat16*>(x), N, d_r, W, bias, *cfg, topk_idx,
                     topk_w, body_of(ws), status_of(ws), s);
+}
+
+size_t moe_gate_logits_workspace_size(int64_t N, int d_r, int E) {
+  if (N < 0 || d_r <= 0 || E <= 0) return 0;
+  return kStatusBytes + route_body(N, d_r, E);
+}
+
+int moe_gate_logits(const moe_bf16* x, int64_t N, int d_r, const float* W, int E, float* logits,
+                    void* ws, size_t ws_bytes, void* stream) {
+  if (N < 0 || d_r <= 0 || E < 1) return MOE_ERR_INVALID_ARG;
+  if (E > 1024) return MOE_ERR_UNSUPPORTED;
+  if (d_r % 32 != 0) return MOE_ERR_UNSUPPORTED;
+  if (N > 0 && (!x || !W || !logits)) return MOE_ERR_INVALID_ARG;
+  if (N > 0 && (!aligned16(x) || !aligned16(W))) return MOE_ERR_ALIGNMENT;
+  int rc;
+  if ((rc = check_ws(ws, ws_bytes, moe_gate_logits_workspace_size(N, d_r, E)))) return rc;
+  if ((rc = check_device())) return rc;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if ((rc = reset_status(ws, s))) return rc;
+  if (N == 0) return MOE_OK;
+  uint8_t* scratch = body_of(ws);
+  if (launch_gate(reinterpret_cast<const __nv_bfloat16*>(x), N, d_r, W, E, scratch, status_of(ws),
+                  s) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  return cudaMemcpyAsync(logits, route_logits_of(scratch), sizeof(float) * (size_t)N * E,
+                         cudaMemcpyDeviceToDevice, s) == cudaSuccess
+             ? MOE_OK
+             : MOE_ERR_CUDA;
 }
 
 int moe_route_from_logits(const float* logits, int64_t N, const float* bias,

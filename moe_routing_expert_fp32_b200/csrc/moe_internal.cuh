@@ -36,7 +36,14 @@ int route_splits(int64_t N, int E, int d_r);
 size_t route_partial_bytes(int64_t N, int E, int d_r);
 // gate GEMM into the router scratch; the fp32 logits [N, E] are at its start
 cudaError_t launch_gate(const __nv_bfloat16* x, int64_t N, int d_r, const float* W, int E,
-                        void* scratch, cudaStream_t s);
+                        void* scratch, DeviceStatus* st, cudaStream_t s);
+
+// router_i8.cu: the same GEMM on the int8 tensor cores (exact digit products),
+// used when the batch fills enough 128x96 tiles
+bool gate_i8_applies(int64_t N, int E, int d_r);
+size_t gate_i8_scratch_bytes(int64_t N, int E, int d_r);
+cudaError_t launch_gate_i8(const __nv_bfloat16* x, int64_t N, int d_r, const float* W, int E,
+                           void* scratch, DeviceStatus* st, cudaStream_t s);
 float* route_logits_of(void* scratch);
 cudaError_t launch_select(const float* part, int splits, int64_t N, const float* bias,
                           const moe_route_cfg& cfg, int32_t* idx, float* w, DeviceStatus* st,

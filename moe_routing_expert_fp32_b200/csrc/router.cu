@@ -3,7 +3,9 @@
 // Follows "Kimi K2 · Affinities", gate-forward excerpt (MoEGate.forward with
 // noaux_tc) and "DeepSeek-V3.2-Exp · Affinities", gate-forward excerpt
 // (Gate.forward):
-//   k_gate_partial : logits = x . W^T in fp32 (x upcast from bf16, W fp32);
+//   k_gate_partial : logits = x . W^T in fp32 (x upcast from bf16, W fp32) for
+//                    batches too small to fill the GPU with int8 tensor-core
+//                    tiles (router_i8.cu takes the others);
 //                    decode batches split d_r over several CTAs (partials in
 //                    double, summed by k_reduce_partials).  FMA chains are 32
 //                    terms long and the 32-term blocks are added in double,
@@ -263,6 +265,7 @@ int route_splits(int64_t N, int E, int d_r) {
 
 // Router scratch: [logits N x E fp32][partials splits x N x E double, if split]
 size_t route_partial_bytes(int64_t N, int E, int d_r) {
+  if (gate_i8_applies(N, E, d_r)) return gate_i8_scratch_bytes(N, E, d_r);
   const int splits = route_splits(N, E, d_r);
   const size_t ne = (size_t)N * (size_t)E;
   return align_up(sizeof(float) * ne, 256) +
@@ -277,7 +280,8 @@ static double* route_part_of(void* scratch, int64_t N, int E) {
 }
 
 cudaError_t launch_gate(const __nv_bfloat16* x, int64_t N, int d_r, const float* W, int E,
-                        void* scratch, cudaStream_t s) {
+                        void* scratch, DeviceStatus* st, cudaStream_t s) {
+  if (gate_i8_applies(N, E, d_r)) return launch_gate_i8(x, N, d_r, W, E, scratch, st, s);
   const int splits = route_splits(N, E, d_r);
   const int nk = d_r / GK;
   const int cps = (nk + splits - 1) / splits;

@@ -1,0 +1,434 @@
+// router_i8.cu -- the router's fp32 gate GEMM on the int8 tensor cores, for
+// batches large enough to fill the GPU.
+//
+// "Kimi K2 · Affinities", gate-forward excerpt: logits = F.linear of the fp32
+// hidden states with the fp32 gate weight.  Tensor-core fp32 accumulation
+// is not accurate enough for that (routing weights must agree to 1e-5), but
+// integer accumulation is exact, so the product is split into exact int8
+// pieces (a slicing scheme in the manner of Ozaki's error-free splitting):
+//   * every row (a token's x, an expert's W) gets a power-of-two scale 2^sig
+//     with |v| < 2^sig, and v / 2^sig is cut into PS = 4 signed 7-bit digits:
+//     v = 2^sig * sum_p a_p 2^(-7(p+1)) + r,   |r| < 2^(sig-28)
+//     (bf16 x is always exact in 4 digits when its exponent range is < 20);
+//   * x . w = 2^(sig_t + sig_e - 14) * sum_s 2^(-7s) S_s,
+//     S_s = sum_{i+k=s} (x digits i) . (w digits k), an exact int32 dot product
+//     over d (|S_s| < 4 * 127^2 * d < 2^31 for d <= 32768);
+//   * pairs with i + k > 4 are dropped; with the digit truncation the logit
+//     error stays below ~2e-8 for unit-variance x and 0.02-scale W, far below
+//     one fp32 ulp of a logit of size 1.
+// k_slice_* cut the rows; k_gate_i8 runs the 13 int8 products per k-block
+// with tcgen05.mma kind::i8 into five int32 TMEM accumulators (one per s) and
+// recombines them in double in its epilogue, rounding once to fp32.
+#include <cuda.h>
+#include <math.h>
+
+#include "moe_internal.cuh"
+
+namespace moe {
+namespace {
+
+constexpr int PS = 4;            // digits per operand
+constexpr int SMAX = 4;          // keep digit pairs with i + k <= SMAX
+constexpr int NACC = SMAX + 1;   // accumulators, one per i + k
+constexpr int IM = 128;          // experts per tile (MMA M)
+constexpr int INT = 96;          // tokens per tile (MMA N)
+constexpr int IKB = 64;          // K bytes per stage (64-byte swizzle rows)
+constexpr int IUK = 32;          // K per tcgen05.mma kind::i8
+constexpr int ISTAGES = 3;
+constexpr int kThreadsI8 = 192;
+constexpr uint64_t kTimeoutNsI8 = 2000000000ull;
+
+constexpr int kAStageBytes = PS * IM * IKB;   // 32 KB
+constexpr int kBStageBytes = PS * INT * IKB;  // 24 KB
+constexpr int kStageBytesI8 = kAStageBytes + kBStageBytes;
+constexpr size_t kSmemI8 = (size_t)ISTAGES * kStageBytesI8 + 1024 + 256;
+static_assert(kSmemI8 <= 227 * 1024, "shared memory");
+static_assert(NACC * INT <= 512, "TMEM columns");
+
+// ------------------------------------------------------------------ slicing
+// Row scale: sig with max|v| < 2^sig (frexp exponent of the row maximum).
+__device__ __forceinline__ int row_sig(float m) {
+  int e = 0;
+  frexp((double)m, &e);
+  return m > 0.f ? e : 0;
+}
+
+__device__ __forceinline__ void digits4(float v, int sig, int8_t* d) {
+  double r = ldexp((double)v, -sig);  // exact, |r| < 1
+#pragma unroll
+  for (int p = 0; p < PS; ++p) {
+    r *= 128.0;
+    const double a = trunc(r);
+    d[p] = (int8_t)a;
+    r -= a;
+  }
+}
+
+template <typename T>
+__device__ __forceinline__ float4 load4(const T* p);
+template <>
+__device__ __forceinline__ float4 load4<float>(const float* p) {
+  return *reinterpret_cast<const float4*>(p);
+}
+template <>
+__device__ __forceinline__ float4 load4<__nv_bfloat16>(const __nv_bfloat16* p) {
+  const uint2 raw = *reinterpret_cast<const uint2*>(p);
+  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&raw);
+  const float2 a = __bfloat1622float2(h[0]), b = __bfloat1622float2(h[1]);
+  return make_float4(a.x, a.y, b.x, b.y);
+}
+
+// One block per row: row maximum -> scale, then 4 digits of every element,
+// 4 elements per thread per step (d % 4 == 0).  out: [PS][rows][d] int8.
+template <typename T>
+__global__ void __launch_bounds__(256) k_slice_rows(const T* __restrict__ v, int64_t rows, int d,
+                                                    int8_t* __restrict__ out,
+                                                    int* __restrict__ sig_out) {
+  __shared__ float wmax[8];
+  const int64_t row = blockIdx.x;
+  const T* src = v + row * d;
+  float m = 0.f;
+  for (int j = threadIdx.x * 4; j < d; j += blockDim.x * 4) {
+    const float4 q = load4<T>(src + j);
+    m = fmaxf(m, fmaxf(fmaxf(fabsf(q.x), fabsf(q.y)), fmaxf(fabsf(q.z), fabsf(q.w))));
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+  if ((threadIdx.x & 31) == 0) wmax[threadIdx.x >> 5] = m;
+  __syncthreads();
+  m = 0.f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) m = fmaxf(m, wmax[i]);
+  const int sig = row_sig(m);
+  if (threadIdx.x == 0) sig_out[row] = sig;
+  const int64_t plane = rows * (int64_t)d;
+  for (int j = threadIdx.x * 4; j < d; j += blockDim.x * 4) {
+    const float4 q = load4<T>(src + j);
+    int8_t a[4][PS];
+    digits4(q.x, sig, a[0]);
+    digits4(q.y, sig, a[1]);
+    digits4(q.z, sig, a[2]);
+    digits4(q.w, sig, a[3]);
+#pragma unroll
+    for (int p = 0; p < PS; ++p) {
+      const uint32_t packed = (uint32_t)(uint8_t)a[0][p] | ((uint32_t)(uint8_t)a[1][p] << 8) |
+                              ((uint32_t)(uint8_t)a[2][p] << 16) |
+                              ((uint32_t)(uint8_t)a[3][p] << 24);
+      *reinterpret_cast<uint32_t*>(out + p * plane + row * d + j) = packed;
+    }
+  }
+}
+
+// -------------------------------------------------------------- PTX helpers
+__device__ __forceinline__ uint32_t su32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ uint64_t gtime() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+__device__ __forceinline__ void bar_init(uint64_t* b, uint32_t n) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(su32(b)), "r"(n));
+}
+__device__ __forceinline__ void bar_expect(uint64_t* b, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(su32(b)), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ bool bar_try(uint64_t* b, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(su32(b)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ bool bar_wait(uint64_t* b, uint32_t parity, volatile int* abort_flag) {
+  if (bar_try(b, parity)) return true;
+  const uint64_t t0 = gtime();
+  for (uint32_t i = 1;; ++i) {
+    if (bar_try(b, parity)) return true;
+    if ((i & 63) == 0) {
+      if (*abort_flag) return false;
+      if (gtime() - t0 > kTimeoutNsI8) return false;
+    }
+  }
+}
+__device__ __forceinline__ void tma3(const CUtensorMap* map, uint64_t* b, void* dst, int c0, int c1,
+                                     int c2) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(su32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(su32(b)), "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
+}
+__device__ __forceinline__ void fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void umma_i8(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc,
+                                        uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(d),
+      "l"(a), "l"(b), "r"(idesc), "r"(acc));
+}
+__device__ __forceinline__ void commit(uint64_t* b) {
+  asm volatile(
+      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(su32(b))
+      : "memory");
+}
+__device__ __forceinline__ void tld16(uint32_t taddr, int32_t* v) {
+  uint32_t r[16];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+        "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr)
+      : "memory");
+#pragma unroll
+  for (int i = 0; i < 16; ++i) v[i] = (int32_t)r[i];
+}
+// K-major operand in 64-byte swizzle: rows of 64 bytes, 8-row groups 512 B apart.
+__device__ __forceinline__ uint64_t sw64_desc(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr & 0x3FFFFu) >> 4);
+  d |= (uint64_t)1 << 16;
+  d |= (uint64_t)(512 >> 4) << 32;
+  d |= (uint64_t)1 << 46;
+  d |= (uint64_t)4 << 61;
+  return d;
+}
+// s8 x s8 -> s32, both K-major, M = 128.
+__device__ __forceinline__ uint32_t idesc_i8(int n) {
+  return (2u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) |
+         ((uint32_t)(IM >> 4) << 24);
+}
+
+// One 128-expert x 96-token tile per CTA.  Warp 0: TMA producer; warp 1: MMA
+// issuer and TMEM owner; warps 2-5: epilogue.
+__global__ void __launch_bounds__(kThreadsI8, 1)
+    k_gate_i8(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
+              const int* __restrict__ sig_w, const int* __restrict__ sig_x, int64_t N, int E,
+              int d, float* __restrict__ logits, DeviceStatus* st) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + ISTAGES * kStageBytesI8);
+  uint64_t* empty = full + ISTAGES;
+  uint64_t* tfull = empty + ISTAGES;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tfull + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int e0 = blockIdx.x * IM;
+  const int64_t t0 = (int64_t)blockIdx.y * INT;
+  const int KB = d / IKB;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < ISTAGES; ++s) {
+      bar_init(&full[s], 1);
+      bar_init(&empty[s], 1);
+    }
+    bar_init(tfull, 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     su32(tmem_slot)),
+                 "r"(512));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  fence_before();
+  __syncthreads();
+  fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      for (int kb = 0; kb < KB; ++kb) {
+        if (!bar_wait(&empty[stage], phase ^ 1, abort_flag)) {
+          record_error(st, MOE_ERR_DEVICE_TIMEOUT, 300);
+          *abort_flag = 1;
+          break;
+        }
+        uint8_t* sA = smem + stage * kStageBytesI8;
+        uint8_t* sB = sA + kAStageBytes;
+        bar_expect(&full[stage], kStageBytesI8);
+#pragma unroll
+        for (int p = 0; p < PS; ++p) {
+          tma3(&tmW, &full[stage], sA + p * IM * IKB, kb * IKB, e0, p);
+          tma3(&tmX, &full[stage], sB + p * INT * IKB, kb * IKB, (int)t0, p);
+        }
+        if (++stage == ISTAGES) { stage = 0; phase ^= 1; }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t idesc = idesc_i8(INT);
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int kb = 0; kb < KB; ++kb) {
+        if (!bar_wait(&full[stage], phase, abort_flag)) { ok = false; break; }
+        fence_after();
+        const uint32_t a0 = su32(smem + stage * kStageBytesI8);
+        const uint32_t b0 = a0 + kAStageBytes;
+        // digit pairs (i of x, k of W), grouped by s = i + k
+#pragma unroll
+        for (int s = 0; s <= SMAX; ++s) {
+          bool first = kb == 0;
+#pragma unroll
+          for (int i = 0; i < PS; ++i) {
+            const int k = s - i;
+            if (k < 0 || k >= PS) continue;
+#pragma unroll
+            for (int h = 0; h < IKB / IUK; ++h) {
+              umma_i8(tmem + s * INT, sw64_desc(a0 + k * IM * IKB + h * IUK),
+                      sw64_desc(b0 + i * INT * IKB + h * IUK), idesc, first ? 0u : 1u);
+              first = false;
+            }
+          }
+        }
+        commit(&empty[stage]);
+        if (++stage == ISTAGES) { stage = 0; phase ^= 1; }
+      }
+      if (ok) commit(tfull);
+      else {
+        record_error(st, MOE_ERR_DEVICE_TIMEOUT, 310);
+        *abort_flag = 1;
+      }
+    }
+  } else {
+    const int quarter = warp & 3;
+    const int e = e0 + quarter * 32 + lane;
+    if (bar_wait(tfull, 0, abort_flag)) {
+      fence_after();
+      const uint32_t taddr = tmem + ((uint32_t)(quarter * 32) << 16);
+      const int sw = e < E ? sig_w[e] : 0;
+      for (int c0 = 0; c0 < INT; c0 += 16) {
+        int32_t acc[NACC][16];
+#pragma unroll
+        for (int s = 0; s < NACC; ++s) tld16(taddr + s * INT + c0, acc[s]);
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          const int64_t t = t0 + c0 + j;
+          if (t >= N || e >= E) continue;
+          double v = 0.0;
+#pragma unroll
+          for (int s = NACC - 1; s >= 0; --s) v = v * 0x1p-7 + (double)acc[s][j];
+          logits[t * E + e] = (float)ldexp(v, sig_x[t] + sw - 14);
+        }
+      }
+    } else {
+      if (lane == 0) record_error(st, MOE_ERR_DEVICE_TIMEOUT, 320);
+      *abort_flag = 1;
+    }
+  }
+  fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(512));
+  }
+}
+
+typedef CUresult (*EncodeTiledFnI8)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                    const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                    const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                    CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFnI8 encode_i8() {
+  static EncodeTiledFnI8 fn = nullptr;
+  static bool tried = false;
+  if (!tried) {
+    tried = true;
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFnI8>(p);
+  }
+  return fn;
+}
+
+// [planes][rows][d] int8, box 64 bytes x box_rows x 1, 64-byte swizzle
+bool map_planes(CUtensorMap* m, const void* base, uint64_t d, uint64_t rows, uint32_t box_rows) {
+  EncodeTiledFnI8 fn = encode_i8();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {d, rows, (cuuint64_t)PS};
+  cuuint64_t strides[2] = {d, d * rows};
+  cuuint32_t box[3] = {(cuuint32_t)IKB, box_rows, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+struct I8Layout {
+  size_t logits, wd, ws, xd, xs, total;
+};
+
+I8Layout i8_layout(int64_t N, int E, int d) {
+  I8Layout L{};
+  size_t o = 0;
+  L.logits = o; o += align_up(sizeof(float) * (size_t)N * E, 256);
+  L.wd = o; o += align_up((size_t)PS * E * d, 256);
+  L.ws = o; o += align_up(sizeof(int) * (size_t)E, 256);
+  L.xd = o; o += align_up((size_t)PS * N * d, 256);
+  L.xs = o; o += align_up(sizeof(int) * (size_t)N, 256);
+  L.total = o;
+  return L;
+}
+
+}  // namespace
+
+bool gate_i8_applies(int64_t N, int E, int d_r) {
+  const int64_t tiles = ((E + IM - 1) / IM) * ((N + INT - 1) / INT);
+  return tiles >= 24 && d_r % IKB == 0 && d_r <= 32768;
+}
+
+size_t gate_i8_scratch_bytes(int64_t N, int E, int d_r) { return i8_layout(N, E, d_r).total; }
+
+cudaError_t launch_gate_i8(const __nv_bfloat16* x, int64_t N, int d_r, const float* W, int E,
+                           void* scratch, DeviceStatus* st, cudaStream_t s) {
+  const I8Layout L = i8_layout(N, E, d_r);
+  uint8_t* base = static_cast<uint8_t*>(scratch);
+  float* logits = reinterpret_cast<float*>(base + L.logits);
+  int8_t* wd = reinterpret_cast<int8_t*>(base + L.wd);
+  int* wsig = reinterpret_cast<int*>(base + L.ws);
+  int8_t* xd = reinterpret_cast<int8_t*>(base + L.xd);
+  int* xsig = reinterpret_cast<int*>(base + L.xs);
+  k_slice_rows<float><<<E, 256, 0, s>>>(W, E, d_r, wd, wsig);
+  k_slice_rows<__nv_bfloat16><<<(unsigned)N, 256, 0, s>>>(x, N, d_r, xd, xsig);
+  CUtensorMap mw, mx;
+  if (!map_planes(&mw, wd, d_r, E, IM) || !map_planes(&mx, xd, d_r, N, INT))
+    return cudaErrorInvalidValue;
+  static bool attr_set[64] = {false};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && !attr_set[dev]) {
+    cudaError_t e =
+        cudaFuncSetAttribute(k_gate_i8, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemI8);
+    if (e != cudaSuccess) return e;
+    attr_set[dev] = true;
+  }
+  dim3 grid((E + IM - 1) / IM, (unsigned)((N + INT - 1) / INT), 1);
+  k_gate_i8<<<grid, kThreadsI8, kSmemI8, s>>>(mw, mx, wsig, xsig, N, E, d_r, logits, st);
+  return cudaGetLastError();
+}
+
+}  // namespace moe
