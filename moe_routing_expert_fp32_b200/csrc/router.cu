@@ -177,6 +177,7 @@ __global__ void __launch_bounds__(32 * kSelWarps) k_select(
   for (int64_t t = (int64_t)blockIdx.x * kSelWarps + warp; t < N;
        t += (int64_t)gridDim.x * kSelWarps) {
     const float* p = part + t * E;
+    // the token's logits first, all loads in flight together
     for (int e = lane; e < E; e += 32) {
       float L = p[e];
       if (splits > 1) {  // split-K partials summed in double, rounded once
@@ -184,8 +185,12 @@ __global__ void __launch_bounds__(32 * kSelWarps) k_select(
         for (int z = 1; z < splits; ++z) Ld += (double)p[z * split_stride + e];
         L = (float)Ld;
       }
+      s_s[e] = L;
+    }
+    __syncwarp();
+    for (int e = lane; e < E; e += 32) {
       // sigmoid: fp32 rounding of 1/(1+exp(-L)) evaluated in double
-      const float s = (float)(1.0 / (1.0 + exp(-(double)L)));
+      const float s = (float)(1.0 / (1.0 + exp(-(double)s_s[e])));
       s_s[e] = s;
       s_c[e] = bias ? __fadd_rn(s, bias[e]) : s;
     }

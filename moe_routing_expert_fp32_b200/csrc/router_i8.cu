@@ -7,7 +7,8 @@
 // integer accumulation is exact, so the product is split into exact int8
 // pieces (a slicing scheme in the manner of Ozaki's error-free splitting):
 //   * every row (a token's x, an expert's W) gets a power-of-two scale 2^sig
-//     with |v| < 2^sig, and v / 2^sig is cut into PS = 4 signed 7-bit digits:
+//     with |v| < 2^sig, and v / 2^sig is cut into PS = 4 signed 7-bit digits
+//     (read off the float's bits; finite inputs):
 //     v = 2^sig * sum_p a_p 2^(-7(p+1)) + r,   |r| < 2^(sig-28)
 //     (bf16 x is always exact in 4 digits when its exponent range is < 20);
 //   * x . w = 2^(sig_t + sig_e - 14) * sum_s 2^(-7s) S_s,
@@ -53,68 +54,96 @@ __device__ __forceinline__ int row_sig(float m) {
   return m > 0.f ? e : 0;
 }
 
-__device__ __forceinline__ void digits4(float v, int sig, int8_t* d) {
-  double r = ldexp((double)v, -sig);  // exact, |r| < 1
+// The 4 digits of v / 2^sig, read off the float's bits: |v| = M * 2^(Ebits-150)
+// (M the 24-bit significand), so X = floor(|v| * 2^(28-sig)) is M shifted by
+// Ebits - 122 - sig, and digit p is bits 21-7p .. 27-7p of X, with v's sign.
+// This equals the truncation v/2^sig -> 128 r -> trunc -> ... done exactly.
+__device__ __forceinline__ uint32_t fixed28(uint32_t bits, int sig) {
+  const int eb = (int)((bits >> 23) & 0xFFu);
+  const uint32_t mant = bits & 0x7FFFFFu;
+  const uint32_t M = eb ? (mant | 0x800000u) : mant;
+  const int sh = (eb ? eb : 1) - 122 - sig;
+  if (sh >= 0) return M << sh;  // sh <= 4 because |v| < 2^sig
+  return sh > -32 ? M >> (-sh) : 0u;
+}
+__device__ __forceinline__ void digits4(uint32_t bits, int sig, int8_t* d) {
+  const uint32_t X = fixed28(bits, sig);
+  const bool neg = (bits >> 31) != 0;
 #pragma unroll
   for (int p = 0; p < PS; ++p) {
-    r *= 128.0;
-    const double a = trunc(r);
-    d[p] = (int8_t)a;
-    r -= a;
+    const int a = (int)((X >> (7 * (PS - 1 - p))) & 0x7Fu);
+    d[p] = (int8_t)(neg ? -a : a);
   }
 }
 
 template <typename T>
-__device__ __forceinline__ float4 load4(const T* p);
+struct Vec;  // 16-byte loads: 4 fp32 or 8 bf16 per thread
 template <>
-__device__ __forceinline__ float4 load4<float>(const float* p) {
-  return *reinterpret_cast<const float4*>(p);
-}
+struct Vec<float> {
+  static constexpr int n = 4;
+  __device__ static void bits(const float* p, uint32_t* b) {
+    const uint4 r = *reinterpret_cast<const uint4*>(p);
+    b[0] = r.x; b[1] = r.y; b[2] = r.z; b[3] = r.w;
+  }
+};
 template <>
-__device__ __forceinline__ float4 load4<__nv_bfloat16>(const __nv_bfloat16* p) {
-  const uint2 raw = *reinterpret_cast<const uint2*>(p);
-  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&raw);
-  const float2 a = __bfloat1622float2(h[0]), b = __bfloat1622float2(h[1]);
-  return make_float4(a.x, a.y, b.x, b.y);
-}
+struct Vec<__nv_bfloat16> {
+  static constexpr int n = 8;
+  __device__ static void bits(const __nv_bfloat16* p, uint32_t* b) {
+    const uint4 r = *reinterpret_cast<const uint4*>(p);
+    const uint32_t w[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      b[2 * i] = w[i] << 16;
+      b[2 * i + 1] = w[i] & 0xFFFF0000u;
+    }
+  }
+};
 
-// One block per row: row maximum -> scale, then 4 digits of every element,
-// 4 elements per thread per step (d % 4 == 0).  out: [PS][rows][d] int8.
+// One block per row: row maximum -> scale, then the 4 digits of every element
+// (n elements per thread per step; d % 8 == 0).  out: [PS][rows][d] int8.
 template <typename T>
 __global__ void __launch_bounds__(256) k_slice_rows(const T* __restrict__ v, int64_t rows, int d,
                                                     int8_t* __restrict__ out,
                                                     int* __restrict__ sig_out) {
+  constexpr int VN = Vec<T>::n;
   __shared__ float wmax[8];
   const int64_t row = blockIdx.x;
   const T* src = v + row * d;
-  float m = 0.f;
-  for (int j = threadIdx.x * 4; j < d; j += blockDim.x * 4) {
-    const float4 q = load4<T>(src + j);
-    m = fmaxf(m, fmaxf(fmaxf(fabsf(q.x), fabsf(q.y)), fmaxf(fabsf(q.z), fabsf(q.w))));
+  uint32_t mx = 0;
+  for (int j = threadIdx.x * VN; j < d; j += blockDim.x * VN) {
+    uint32_t b[VN];
+    Vec<T>::bits(src + j, b);
+#pragma unroll
+    for (int i = 0; i < VN; ++i) mx = max(mx, b[i] & 0x7FFFFFFFu);  // |v| ordered as integers
   }
 #pragma unroll
-  for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
-  if ((threadIdx.x & 31) == 0) wmax[threadIdx.x >> 5] = m;
+  for (int off = 16; off > 0; off >>= 1) mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+  if ((threadIdx.x & 31) == 0) wmax[threadIdx.x >> 5] = __uint_as_float(mx);
   __syncthreads();
-  m = 0.f;
+  float m = 0.f;
 #pragma unroll
   for (int i = 0; i < 8; ++i) m = fmaxf(m, wmax[i]);
   const int sig = row_sig(m);
   if (threadIdx.x == 0) sig_out[row] = sig;
   const int64_t plane = rows * (int64_t)d;
-  for (int j = threadIdx.x * 4; j < d; j += blockDim.x * 4) {
-    const float4 q = load4<T>(src + j);
-    int8_t a[4][PS];
-    digits4(q.x, sig, a[0]);
-    digits4(q.y, sig, a[1]);
-    digits4(q.z, sig, a[2]);
-    digits4(q.w, sig, a[3]);
+  for (int j = threadIdx.x * VN; j < d; j += blockDim.x * VN) {
+    uint32_t b[VN];
+    Vec<T>::bits(src + j, b);
+    int8_t a[VN][PS];
+#pragma unroll
+    for (int i = 0; i < VN; ++i) digits4(b[i], sig, a[i]);
 #pragma unroll
     for (int p = 0; p < PS; ++p) {
-      const uint32_t packed = (uint32_t)(uint8_t)a[0][p] | ((uint32_t)(uint8_t)a[1][p] << 8) |
-                              ((uint32_t)(uint8_t)a[2][p] << 16) |
-                              ((uint32_t)(uint8_t)a[3][p] << 24);
-      *reinterpret_cast<uint32_t*>(out + p * plane + row * d + j) = packed;
+      uint32_t w[VN / 4];
+#pragma unroll
+      for (int q = 0; q < VN / 4; ++q)
+        w[q] = (uint32_t)(uint8_t)a[4 * q][p] | ((uint32_t)(uint8_t)a[4 * q + 1][p] << 8) |
+               ((uint32_t)(uint8_t)a[4 * q + 2][p] << 16) |
+               ((uint32_t)(uint8_t)a[4 * q + 3][p] << 24);
+      int8_t* dst = out + p * plane + row * d + j;
+      if (VN == 8) *reinterpret_cast<uint2*>(dst) = make_uint2(w[0], w[VN / 4 - 1]);
+      else *reinterpret_cast<uint32_t*>(dst) = w[0];
     }
   }
 }
@@ -398,7 +427,7 @@ I8Layout i8_layout(int64_t N, int E, int d) {
 
 bool gate_i8_applies(int64_t N, int E, int d_r) {
   const int64_t tiles = ((E + IM - 1) / IM) * ((N + INT - 1) / INT);
-  return tiles >= 24 && d_r % IKB == 0 && d_r <= 32768;
+  return tiles >= 24 && d_r % IKB == 0 && d_r <= 32768;  // d_r % 64 also serves the slicers
 }
 
 size_t gate_i8_scratch_bytes(int64_t N, int E, int d_r) { return i8_layout(N, E, d_r).total; }
