@@ -14,6 +14,8 @@ import numpy as np
 from .build import build as _build
 
 ACT_SILU, ACT_SITU = 0, 1
+SCORE_SIGMOID, SCORE_SOFTMAX = 0, 1
+GROUP_TOP2_SUM, GROUP_MAX = 0, 1
 _lib = None
 
 
@@ -30,6 +32,10 @@ def lib() -> ctypes.CDLL:
             "oracle_group_scores": ([vp, i64, i32, i32, vp], None),
             "oracle_route_from_logits": ([vp, i64, i32, vp, i32, i32, i32, i32, f32, vp, vp, vp],
                                          None),
+            "oracle_route_from_logits_ex": ([vp, i64, i32, vp, i32, i32, i32, i32, f32, i32, i32,
+                                             vp, vp, vp], None),
+            "oracle_group_scores_ex": ([vp, i64, i32, i32, i32, vp], None),
+            "oracle_choice_scores_ex": ([vp, i64, i32, vp, i32, i32, i32, i32, vp], None),
             "oracle_choice_scores": ([vp, i64, i32, vp, i32, i32, vp], None),
             "oracle_dispatch": ([vp, i64, i32, i32, vp, vp, vp, vp], None),
             "oracle_gather": ([vp, i32, vp, i64, i32, vp], None),
@@ -90,15 +96,16 @@ def sigmoid(L: float) -> float:
     return float(lib().oracle_sigmoid(float(L)))
 
 
-def group_scores(c: np.ndarray, G: int) -> np.ndarray:
+def group_scores(c: np.ndarray, G: int, mode: int = GROUP_TOP2_SUM) -> np.ndarray:
     c = _c(c, np.float32)
     N, E = c.shape
     out = np.empty((N, G), dtype=np.float32)
-    lib().oracle_group_scores(_p(c), N, E, G, _p(out))
+    lib().oracle_group_scores_ex(_p(c), N, E, G, int(mode), _p(out))
     return out
 
 
-def route_from_logits(logits, bias, G, TG, K, route_scale, norm=True):
+def route_from_logits(logits, bias, G, TG, K, route_scale, norm=True, score=SCORE_SIGMOID,
+                      group=GROUP_TOP2_SUM):
     """(idx int32 [N,K], w fp32 [N,K], margin float64 [N])."""
     logits = _c(logits, np.float32)
     N, E = logits.shape
@@ -106,22 +113,24 @@ def route_from_logits(logits, bias, G, TG, K, route_scale, norm=True):
     idx = np.empty((N, K), dtype=np.int32)
     w = np.empty((N, K), dtype=np.float32)
     margin = np.empty((N,), dtype=np.float64)
-    lib().oracle_route_from_logits(_p(logits), N, E, _p(b), G, TG, K, int(bool(norm)),
-                                   float(route_scale), _p(idx), _p(w), _p(margin))
+    lib().oracle_route_from_logits_ex(_p(logits), N, E, _p(b), G, TG, K, int(bool(norm)),
+                                      float(route_scale), int(score), int(group), _p(idx), _p(w),
+                                      _p(margin))
     return idx, w, margin
 
 
-def choice_scores(logits, bias, G, TG) -> np.ndarray:
+def choice_scores(logits, bias, G, TG, score=SCORE_SIGMOID, group=GROUP_TOP2_SUM) -> np.ndarray:
     logits = _c(logits, np.float32)
     N, E = logits.shape
     b = None if bias is None else _c(bias, np.float32)
     out = np.empty((N, E), dtype=np.float32)
-    lib().oracle_choice_scores(_p(logits), N, E, _p(b), G, TG, _p(out))
+    lib().oracle_choice_scores_ex(_p(logits), N, E, _p(b), G, TG, int(score), int(group), _p(out))
     return out
 
 
-def route(x, W, bias, G, TG, K, route_scale, norm=True):
-    return route_from_logits(gate_logits(x, W), bias, G, TG, K, route_scale, norm)
+def route(x, W, bias, G, TG, K, route_scale, norm=True, score=SCORE_SIGMOID,
+          group=GROUP_TOP2_SUM):
+    return route_from_logits(gate_logits(x, W), bias, G, TG, K, route_scale, norm, score, group)
 
 
 # --------------------------------------------------------------- moe_infer

@@ -11,8 +11,9 @@
  * and bf16 x fp32 products are exact in double) and rounded once to the dtype
  * the page's tensor has at that point:
  *
- *   gate logits, sigmoid, biased choice score, group top-2 score, group and
- *   expert top-k, unbiased weights, renormalisation, route scale
+ *   gate logits, sigmoid (or softmax), biased choice score, group top-2 score
+ *   (or group maximum), group and expert top-k, unbiased weights,
+ *   renormalisation, route scale
  *       -- "Kimi K2 · Affinities", gate-forward excerpt (MoEGate.forward,
  *          noaux_tc) and "DeepSeek-V3.2-Exp · Affinities", gate-forward
  *          excerpt (Gate.forward)
@@ -148,10 +149,48 @@ static float group_top2(const float* c, int gsz) {
   return c[i1] + c[i2];
 }
 
-void oracle_group_scores(const float* c, int64_t N, int E, int G, float* gs) {
+/* Group score when the group has no top-2 sum: its largest choice score
+ * ("DeepSeek-V3.2-Exp · Affinities", gate-forward: scores.amax(dim=-1), the
+ * form that page uses when there is no correction bias). */
+static float group_max(const float* c, int gsz) {
+  float m = c[0];
+  for (int i = 1; i < gsz; ++i)
+    if (c[i] > m) m = c[i];
+  return m;
+}
+
+enum { ORACLE_GROUP_TOP2_SUM = 0, ORACLE_GROUP_MAX = 1 };
+enum { ORACLE_SCORE_SIGMOID = 0, ORACLE_SCORE_SOFTMAX = 1 };
+
+static float group_score(const float* c, int gsz, int mode) {
+  return mode == ORACLE_GROUP_MAX ? group_max(c, gsz) : group_top2(c, gsz);
+}
+
+void oracle_group_scores_ex(const float* c, int64_t N, int E, int G, int mode, float* gs) {
   const int gsz = E / G;
   for (int64_t t = 0; t < N; ++t)
-    for (int g = 0; g < G; ++g) gs[t * G + g] = group_top2(c + t * (int64_t)E + g * gsz, gsz);
+    for (int g = 0; g < G; ++g) gs[t * G + g] = group_score(c + t * (int64_t)E + g * gsz, gsz, mode);
+}
+
+void oracle_group_scores(const float* c, int64_t N, int E, int G, float* gs) {
+  oracle_group_scores_ex(c, N, E, G, ORACLE_GROUP_TOP2_SUM, gs);
+}
+
+/* Affinity scores of one token: sigmoid of each logit (both router pages), or
+ * the softmax over all experts ("DeepSeek-V3.2-Exp · Affinities",
+ * gate-forward: scores.softmax(dim=-1)), evaluated in double with the row
+ * maximum subtracted, each rounded once to fp32. */
+static void token_scores(const float* L, int E, int score_func, float* s) {
+  if (score_func == ORACLE_SCORE_SOFTMAX) {
+    double m = (double)L[0];
+    for (int e = 1; e < E; ++e)
+      if ((double)L[e] > m) m = (double)L[e];
+    double sum = 0.0;
+    for (int e = 0; e < E; ++e) sum += exp((double)L[e] - m);
+    for (int e = 0; e < E; ++e) s[e] = (float)(exp((double)L[e] - m) / sum);
+  } else {
+    for (int e = 0; e < E; ++e) s[e] = oracle_sigmoid(L[e]);
+  }
 }
 
 /* Selection and weights for one token, from its logits.
@@ -162,16 +201,15 @@ void oracle_group_scores(const float* c, int64_t N, int E, int G, float* gs) {
  * margin (optional) = min(gs_(TG) - gs_(TG+1), c_(K) - c_(K+1)) in double,
  * +inf where a boundary does not exist. */
 static void route_token(const float* L, int E, const float* bias, int G, int TG, int K,
-                        int norm, float route_scale, int32_t* idx, float* w, double* margin,
-                        float* s, float* c, float* gs, unsigned char* used) {
-  for (int e = 0; e < E; ++e) {
-    s[e] = oracle_sigmoid(L[e]);
-    c[e] = bias ? s[e] + bias[e] : s[e];
-  }
+                        int norm, float route_scale, int score_func, int group_mode,
+                        int32_t* idx, float* w, double* margin, float* s, float* c, float* gs,
+                        unsigned char* used) {
+  token_scores(L, E, score_func, s);
+  for (int e = 0; e < E; ++e) c[e] = bias ? s[e] + bias[e] : s[e];
   double m_g = INFINITY, m_e = INFINITY;
   if (G > 1) {
     const int gsz = E / G;
-    for (int g = 0; g < G; ++g) gs[g] = group_top2(c + g * gsz, gsz);
+    for (int g = 0; g < G; ++g) gs[g] = group_score(c + g * gsz, gsz, group_mode);
     /* top-TG groups by (gs desc, g asc) */
     memset(used, 0, (size_t)G);
     float last_kept = 0.0f;
@@ -220,9 +258,10 @@ static void route_token(const float* L, int E, const float* bias, int G, int TG,
   if (margin) *margin = m_g < m_e ? m_g : m_e;
 }
 
-void oracle_route_from_logits(const float* logits, int64_t N, int E, const float* bias, int G,
-                              int TG, int K, int norm, float route_scale, int32_t* idx,
-                              float* w, double* margin) {
+void oracle_route_from_logits_ex(const float* logits, int64_t N, int E, const float* bias,
+                                 int G, int TG, int K, int norm, float route_scale,
+                                 int score_func, int group_mode, int32_t* idx, float* w,
+                                 double* margin) {
 #pragma omp parallel
   {
     float* s = (float*)malloc(sizeof(float) * (size_t)E);
@@ -231,27 +270,33 @@ void oracle_route_from_logits(const float* logits, int64_t N, int E, const float
     unsigned char* used = (unsigned char*)malloc((size_t)(E > G ? E : G));
 #pragma omp for schedule(static)
     for (int64_t t = 0; t < N; ++t)
-      route_token(logits + t * (int64_t)E, E, bias, G, TG, K, norm, route_scale,
-                  idx + t * (int64_t)K, w + t * (int64_t)K, margin ? margin + t : NULL, s, c,
-                  gs, used);
+      route_token(logits + t * (int64_t)E, E, bias, G, TG, K, norm, route_scale, score_func,
+                  group_mode, idx + t * (int64_t)K, w + t * (int64_t)K,
+                  margin ? margin + t : NULL, s, c, gs, used);
     free(s); free(c); free(gs); free(used);
   }
 }
 
+void oracle_route_from_logits(const float* logits, int64_t N, int E, const float* bias, int G,
+                              int TG, int K, int norm, float route_scale, int32_t* idx,
+                              float* w, double* margin) {
+  oracle_route_from_logits_ex(logits, N, E, bias, G, TG, K, norm, route_scale,
+                              ORACLE_SCORE_SIGMOID, ORACLE_GROUP_TOP2_SUM, idx, w, margin);
+}
+
 /* Biased choice scores with the non-kept groups masked to -inf (for tests). */
-void oracle_choice_scores(const float* logits, int64_t N, int E, const float* bias, int G,
-                          int TG, float* c_out) {
+void oracle_choice_scores_ex(const float* logits, int64_t N, int E, const float* bias, int G,
+                             int TG, int score_func, int group_mode, float* c_out) {
   float* gs = (float*)malloc(sizeof(float) * (size_t)(G > 0 ? G : 1));
   unsigned char* used = (unsigned char*)malloc((size_t)(G > 0 ? G : 1));
+  float* sc = (float*)malloc(sizeof(float) * (size_t)E);
   for (int64_t t = 0; t < N; ++t) {
     float* c = c_out + t * (int64_t)E;
-    for (int e = 0; e < E; ++e) {
-      float s = oracle_sigmoid(logits[t * (int64_t)E + e]);
-      c[e] = bias ? s + bias[e] : s;
-    }
+    token_scores(logits + t * (int64_t)E, E, score_func, sc);
+    for (int e = 0; e < E; ++e) c[e] = bias ? sc[e] + bias[e] : sc[e];
     if (G > 1) {
       const int gsz = E / G;
-      for (int g = 0; g < G; ++g) gs[g] = group_top2(c + g * gsz, gsz);
+      for (int g = 0; g < G; ++g) gs[g] = group_score(c + g * gsz, gsz, group_mode);
       memset(used, 0, (size_t)G);
       for (int r = 0; r < TG; ++r) {
         int best = -1;
@@ -264,7 +309,13 @@ void oracle_choice_scores(const float* logits, int64_t N, int E, const float* bi
           for (int i = 0; i < gsz; ++i) c[g * gsz + i] = -INFINITY;
     }
   }
-  free(gs); free(used);
+  free(gs); free(used); free(sc);
+}
+
+void oracle_choice_scores(const float* logits, int64_t N, int E, const float* bias, int G,
+                          int TG, float* c_out) {
+  oracle_choice_scores_ex(logits, N, E, bias, G, TG, ORACLE_SCORE_SIGMOID,
+                          ORACLE_GROUP_TOP2_SUM, c_out);
 }
 
 /* ------------------------------------------------------------- moe_infer */
