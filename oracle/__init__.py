@@ -46,6 +46,9 @@ def lib() -> ctypes.CDLL:
                                   vp, vp], None),
             "oracle_moe_dense": ([vp, i64, i32, vp, vp, i32, i32, vp, vp, vp, i32, f32, f32, vp],
                                  None),
+            "oracle_linear": ([vp, i64, i32, vp, i32, vp], None),
+            "oracle_add": ([vp, vp, i64, vp], None),
+            "oracle_rms_norm": ([vp, i64, i32, vp, f32, vp], None),
             "oracle_bf16_round_double": ([ctypes.c_double], ctypes.c_uint16),
             "oracle_bf16_round_float": ([f32], ctypes.c_uint16),
         }
@@ -210,6 +213,59 @@ def moe_dense(x_e, idx, w, w1, w3, w2, act="silu", beta=1.0, lbeta=0.0) -> np.nd
     lib().oracle_moe_dense(_p(x_e), N, d, _p(idx), _p(w), K, F, _p(w1), _p(w3), _p(w2),
                            act_code(act), float(beta), float(lbeta), _p(out))
     return out
+
+
+# ----------------------------------------------------- the block around it
+def linear(x, W) -> np.ndarray:
+    """Bias-free bf16 Linear: bf16(x . W^T), x [M, K], W [N_out, K]."""
+    x = _c(x, np.uint16)
+    W = _c(W, np.uint16)
+    M, K = x.shape
+    Nout = W.shape[0]
+    assert W.shape[1] == K
+    y = np.empty((M, Nout), dtype=np.uint16)
+    if M:
+        lib().oracle_linear(_p(x), M, K, _p(W), Nout, _p(y))
+    return y
+
+
+def add(a, b) -> np.ndarray:
+    a = _c(a, np.uint16)
+    b = _c(b, np.uint16)
+    assert a.shape == b.shape
+    out = np.empty_like(a)
+    lib().oracle_add(_p(a), _p(b), a.size, _p(out))
+    return out
+
+
+def rms_norm(x, w, eps: float) -> np.ndarray:
+    x = _c(x, np.uint16)
+    w = _c(w, np.uint16)
+    N, d = x.shape
+    assert w.shape == (d,)
+    out = np.empty_like(x)
+    if N:
+        lib().oracle_rms_norm(_p(x), N, d, _p(w), float(eps), _p(out))
+    return out
+
+
+def block_forward(x, W, bias, G, TG, K, route_scale, w1, w3, w2, act="silu", beta=1.0,
+                  lbeta=0.0, norm=True, down_proj=None, norm_w=None, eps=1e-6, up_proj=None,
+                  shared=None, score=SCORE_SIGMOID, group=GROUP_TOP2_SUM):
+    """KimiSparseMoeBlock.forward ("Kimi K3 · Add shared output", moe-forward):
+    gate on the full-width x; optional routed_expert_down_proj; moe_infer;
+    optional routed_expert_norm and routed_expert_up_proj; plus the shared
+    experts (w1, w3, w2) on x.  Returns (out, idx, w, margin)."""
+    idx, w, margin = route(x, W, bias, G, TG, K, route_scale, norm, score, group)
+    xe = linear(x, down_proj) if down_proj is not None else _c(x, np.uint16)
+    y = moe_infer(xe, idx, w, w1, w3, w2, act, beta, lbeta)
+    if down_proj is not None:
+        if norm_w is not None:
+            y = rms_norm(y, norm_w, eps)
+        y = linear(y, up_proj)
+    if shared is not None:
+        y = add(y, expert_ffn(x, *shared, act=act, beta=beta, lbeta=lbeta))
+    return y, idx, w, margin
 
 
 def bf16_round_double(v: float) -> int:

@@ -22,6 +22,9 @@
  *   expert MLP, SiLU-and-mul, SiTU
  *       -- "Kimi K3 · Gate features", expert excerpt (KimiBlockSparseMLP) and
  *          situ excerpt (SituAndMul, _get_situ_activation_params)
+ *   latent down/up projections, routed-expert norm, shared-expert add
+ *       -- "Kimi K3 · Add shared output", moe-forward excerpt
+ *          (KimiSparseMoeBlock.forward)
  *
  * Readings where the pages are silent or disagree (each also listed in the
  * design notes):
@@ -32,7 +35,10 @@
  *     (value descending, index ascending) order;
  *   - sums over k (weight normaliser, combine) run sequentially k = 0..K-1;
  *   - the slot sort is stable (slots of one expert keep ascending slot order);
- *   - the sigmoid is the fp32 rounding of 1/(1+exp(-L)) evaluated in double.
+ *   - the sigmoid is the fp32 rounding of 1/(1+exp(-L)) evaluated in double;
+ *   - the routed-expert norm is an RMSNorm (see oracle_rms_norm); the latent
+ *     projections are bias-free; the shared experts are one gated MLP of the
+ *     experts' kind on the full width (oracle_expert_ffn on every token).
  *
  * Build: gcc -O2 -ffp-contract=off -fno-fast-math -fopenmp (no x87: x86-64 SSE
  * arithmetic, so every float operation below is one IEEE fp32 operation).
@@ -468,6 +474,58 @@ void oracle_moe_dense(const bf16_t* x, int64_t N, int d, const int32_t* idx, con
   }
   free(yk);
   free(posk);
+}
+
+/* ------------------------------------------------- the block around moe_infer */
+
+/* Bias-free bf16 nn.Linear: y[m,n] = bf16( sum_k x[m,k] * W[n,k] ), the sum in
+ * double and rounded once.  routed_expert_down_proj and routed_expert_up_proj
+ * of the latent block ("Kimi K3 · Add shared output", moe-forward excerpt,
+ * KimiSparseMoeBlock.forward); their bias-free form is a reading, the same as
+ * the experts' own Linear layers ("Kimi K3 · Gate features", expert excerpt). */
+void oracle_linear(const bf16_t* x, int64_t M, int K, const bf16_t* W, int Nout, bf16_t* y) {
+#pragma omp parallel for schedule(dynamic, 1)
+  for (int64_t m = 0; m < M; ++m) {
+    const bf16_t* xr = x + m * (int64_t)K;
+    for (int n = 0; n < Nout; ++n) {
+      const bf16_t* wr = W + (int64_t)n * K;
+      double acc = 0.0;
+      for (int k = 0; k < K; ++k) acc += (double)bf16_value(xr[k]) * (double)bf16_value(wr[k]);
+      y[m * (int64_t)Nout + n] = bf16_round_d(acc);
+    }
+  }
+}
+
+/* out = bf16( a + b ) elementwise for bf16 a, b: the exact sum rounded once
+ * (the block's final y + shared_experts(identity)). */
+void oracle_add(const bf16_t* a, const bf16_t* b, int64_t n, bf16_t* out) {
+#pragma omp parallel for schedule(static)
+  for (int64_t i = 0; i < n; ++i)
+    out[i] = bf16_round_d((double)bf16_value(a[i]) + (double)bf16_value(b[i]));
+}
+
+/* routed_expert_norm of the latent block, whose kind the pages do not show;
+ * read as the RMSNorm the model family uses elsewhere (DeepseekV3RMSNorm in
+ * "Kimi K2 · Masked scores", transformer excerpt): per row,
+ *   r = 1 / sqrt( mean_i y_i^2 + eps )          (double)
+ *   n_i = bf16( y_i * r )                         (normalised, cast back)
+ *   out_i = bf16( w_i * n_i )                     (bf16 weight times bf16) */
+void oracle_rms_norm(const bf16_t* x, int64_t N, int d, const bf16_t* w, float eps,
+                     bf16_t* out) {
+#pragma omp parallel for schedule(static)
+  for (int64_t t = 0; t < N; ++t) {
+    const bf16_t* xr = x + t * (int64_t)d;
+    double ss = 0.0;
+    for (int i = 0; i < d; ++i) {
+      const double v = (double)bf16_value(xr[i]);
+      ss += v * v;
+    }
+    const double r = 1.0 / sqrt(ss / (double)d + (double)eps);
+    for (int i = 0; i < d; ++i) {
+      const double nv = (double)bf16_value(bf16_round_d((double)bf16_value(xr[i]) * r));
+      out[t * (int64_t)d + i] = bf16_round_d((double)bf16_value(w[i]) * nv);
+    }
+  }
 }
 
 /* Rounding helpers, exported so that tests can pin them. */

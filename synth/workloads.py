@@ -14,6 +14,12 @@ Recipe (seed 0 unless stated):
   w3   [E, F, d_e] bf16 ~ N(0, 0.02)      tensor id 5
   w2   [E, d_e, F] bf16 ~ N(0, 0.02)      tensor id 6
   x_e  [N, d_e]  bf16  ~ N(0, 1)          tensor id 7 (latent workload only; else x_e = x)
+
+The whole-block workload (routed layer inside KimiSparseMoeBlock) adds:
+  down_proj [d_e, d_r] bf16 ~ N(0, 0.02)          tensor id 9
+  norm_w    [d_e]      bf16 = bf16(U(0.5, 1.5))   tensor id 10
+  up_proj   [d_r, d_e] bf16 ~ N(0, 0.02)          tensor id 11
+  shared w1, w3 [F_sh, d_r], w2 [d_r, F_sh] bf16 ~ N(0, 0.02)   tensor ids 12, 13, 14
 """
 from __future__ import annotations
 
@@ -23,6 +29,8 @@ from dataclasses import dataclass, asdict
 import numpy as np
 
 TID_X, TID_W, TID_BIAS, TID_W1, TID_W3, TID_W2, TID_XE, TID_POP = 1, 2, 3, 4, 5, 6, 7, 8
+TID_DOWN, TID_NORM, TID_UP, TID_SW1, TID_SW3, TID_SW2 = 9, 10, 11, 12, 13, 14
+NORM_LO, NORM_HI = 0.5, 1.5
 
 SIGMA_X = 1.0
 SIGMA_W = 0.02
@@ -52,6 +60,8 @@ class Workload:
     latent: bool = False
     skew: bool = False
     seed: int = 0
+    F_shared: int = 0       # whole-block workloads: shared experts' hidden width
+    norm_eps: float = 1e-6  # whole-block workloads: routed_expert_norm epsilon
 
     @property
     def S(self) -> int:
@@ -85,6 +95,18 @@ def scaled(wl: Workload, **kw) -> Workload:
     d = wl.as_dict()
     d.update(kw)
     return Workload(**d)
+
+
+# The whole KimiSparseMoeBlock at the Kimi-K3 latent decode shape: x_e is the
+# down projection of x (not a tensor of its own), then RMSNorm, up projection
+# and one shared expert of width 3072 on the full 7168 width.
+BLOCKS = {
+    "k3_block_decode": scaled(WORKLOADS["k3_latent_decode"], name="k3_block_decode",
+                              F_shared=3072),
+    "tiny_block": Workload("tiny_block", N=64, d_r=256, d_e=128, E=16, G=4, TG=2, K=4, F=128,
+                           act="situ", route_scale=2.5, beta=4.0, lbeta=8.0, latent=True,
+                           F_shared=256),
+}
 
 
 # ------------------------------------------------------------------ host side
@@ -163,4 +185,50 @@ def dev_inputs(wl: Workload, rank: int = 0, device="cuda", experts: bool = True)
                                     wl.seed, TID_W3, SIGMA_EXPERT)
         out["w2"] = dev_normal_bf16(torch.empty((wl.E, wl.d_e, wl.F), dtype=bf, device=device),
                                     wl.seed, TID_W2, SIGMA_EXPERT)
+    return out
+
+
+# ------------------------------------------------------- the block around it
+def _bf16_bits_rne(a: np.ndarray) -> np.ndarray:
+    u = np.ascontiguousarray(a, dtype=np.float32).view(np.uint32).astype(np.uint64)
+    return ((u + 0x7FFF + ((u >> 16) & 1)) >> 16).astype(np.uint16)
+
+
+def host_block(wl: Workload) -> dict:
+    """Block weights on the host as bf16 bit patterns (down/up/norm absent
+    unless latent, shared absent unless F_shared)."""
+    from . import host_normal_bf16, host_uniform_f32
+    out = {"down_proj": None, "norm_w": None, "up_proj": None, "shared": None}
+    if wl.latent:
+        out["down_proj"] = host_normal_bf16(wl.seed, TID_DOWN, (wl.d_e, wl.d_r), SIGMA_EXPERT)
+        out["norm_w"] = _bf16_bits_rne(host_uniform_f32(wl.seed, TID_NORM, (wl.d_e,), NORM_LO,
+                                                        NORM_HI))
+        out["up_proj"] = host_normal_bf16(wl.seed, TID_UP, (wl.d_r, wl.d_e), SIGMA_EXPERT)
+    if wl.F_shared:
+        out["shared"] = (
+            host_normal_bf16(wl.seed, TID_SW1, (wl.F_shared, wl.d_r), SIGMA_EXPERT),
+            host_normal_bf16(wl.seed, TID_SW3, (wl.F_shared, wl.d_r), SIGMA_EXPERT),
+            host_normal_bf16(wl.seed, TID_SW2, (wl.d_r, wl.F_shared), SIGMA_EXPERT))
+    return out
+
+
+def dev_block(wl: Workload, device="cuda") -> dict:
+    """The same block weights drawn by the device twin (torch CUDA tensors)."""
+    import torch
+    from . import dev_normal_bf16, dev_uniform_f32
+    bf = torch.bfloat16
+    out = {"down_proj": None, "norm_w": None, "up_proj": None, "shared": None}
+
+    def nrm(tid, shape):
+        return dev_normal_bf16(torch.empty(shape, dtype=bf, device=device), wl.seed, tid,
+                               SIGMA_EXPERT)
+    if wl.latent:
+        out["down_proj"] = nrm(TID_DOWN, (wl.d_e, wl.d_r))
+        u = dev_uniform_f32(torch.empty((wl.d_e,), dtype=torch.float32, device=device), wl.seed,
+                            TID_NORM, NORM_LO, NORM_HI)
+        out["norm_w"] = u.to(bf)  # round to nearest even, as the host twin
+        out["up_proj"] = nrm(TID_UP, (wl.d_r, wl.d_e))
+    if wl.F_shared:
+        out["shared"] = (nrm(TID_SW1, (wl.F_shared, wl.d_r)), nrm(TID_SW3, (wl.F_shared, wl.d_r)),
+                         nrm(TID_SW2, (wl.d_r, wl.F_shared)))
     return out
