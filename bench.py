@@ -34,17 +34,26 @@ if ROOT not in sys.path:
 METRIC = "routed tokens/sec per MoE layer (route+dispatch+FFN+combine)"
 UNIT = "tokens/s"
 DEFAULT_WORKLOAD = "dsv32_decode"
-# gate_partial, [reduce_partials,] select, hist, scan, scatter, gather, tiles, gate_up, down,
-# combine; the reduce runs when the gate GEMM is split over d_r (decode batches)
-KERNELS_PER_STEP = 10
+# select, hist, scan, scatter, gather, tiles, gate_up, down, combine, plus the gate GEMM:
+# gate_partial [+ reduce_partials when split over d_r] for decode batches, or
+# slice(W) + slice(x) + gate_i8 once the batch fills 24 tiles of 128 x 96
+KERNELS_AFTER_GATE = 9
+
+
+def gate_kernels(wl):
+    """Launches of the router's gate GEMM (mirrors the library's choice)."""
+    if ((wl.E + 127) // 128) * ((wl.N + 95) // 96) >= 24 and wl.d_r % 64 == 0 \
+            and wl.d_r <= 32768:
+        return 3
+    tiles = max(1, ((wl.E + 63) // 64) * ((wl.N + 63) // 64))
+    nk = max(1, wl.d_r // 32)
+    want = max(1, min((296 + tiles - 1) // tiles, max(nk // 4, 1), 32))
+    cps = (nk + want - 1) // want
+    return 1 + (1 if (nk + cps - 1) // cps > 1 else 0)
 
 
 def kernels_per_step(wl):
-    tiles = ((wl.E + 63) // 64) * ((wl.N + 63) // 64)
-    nk = wl.d_r // 32
-    want = max(1, min((296 + tiles - 1) // tiles, max(nk // 4, 1), 64))
-    cps = (nk + want - 1) // want
-    return KERNELS_PER_STEP + (1 if (nk + cps - 1) // cps > 1 else 0)
+    return gate_kernels(wl) + KERNELS_AFTER_GATE
 
 
 def parse():
@@ -63,8 +72,8 @@ def parse():
 
 
 def workload_of(args):
-    from synth.workloads import WORKLOADS, scaled
-    wl = WORKLOADS[args.workload]
+    from synth.workloads import BLOCKS, WORKLOADS, scaled
+    wl = WORKLOADS[args.workload] if args.workload in WORKLOADS else BLOCKS[args.workload]
     kw = {}
     if args.tokens:
         kw["N"] = args.tokens
@@ -284,6 +293,149 @@ def run_ours(args, rank, world, local_rank):
     return wl, res
 
 
+# ------------------------------------------------------ whole-block arm
+BLOCK_METRIC = "tokens/sec per MoE block (route+shared experts+latent projections+routed experts)"
+
+
+def block_kernels(wl):
+    """The routed layer's launches plus the dense tile list, the shared
+    experts' two GEMMs and the two latent projections (the RMSNorm is fused
+    into the combine)."""
+    return kernels_per_step(wl) + 1 + (2 if wl.F_shared else 0) + (2 if wl.latent else 0)
+
+
+def block_bytes(wl, touched):
+    """Algorithmic HBM bytes of one block step: every weight byte read once
+    (gate fp32; projections, norm, shared and touched routed experts bf16) and
+    the activations each stage must write and read back."""
+    N, S = wl.N, wl.N * wl.K
+    w = wl.E * wl.d_r * 4 + touched * 3 * wl.F * wl.d_e * 2
+    if wl.latent:
+        w += 2 * wl.d_e * wl.d_r * 2 + wl.d_e * 2
+    if wl.F_shared:
+        w += 3 * wl.F_shared * wl.d_r * 2
+    act = N * wl.d_r * 2 + N * wl.d_r * 2                # x read, out written
+    act += 2 * (S * wl.d_e * 2) + 2 * (S * wl.F * 2) + 2 * (S * wl.d_e * 2)  # xs, h, y
+    if wl.latent:
+        act += 2 * N * wl.d_e * 2 * 2                     # x_e and the combined rows
+    if wl.F_shared:
+        act += 2 * N * wl.F_shared * 2 + 2 * N * wl.d_r * 2  # shared h and output
+    return w + act
+
+
+def run_block(args, rank, world, local_rank):
+    import torch
+    import moe_routing_expert_fp32_b200 as moe
+    from synth.workloads import dev_block, dev_inputs
+
+    wl = workload_of(args)
+    torch.cuda.set_device(local_rank)
+    dev = dev_inputs(wl, rank=rank)
+    blk = dev_block(wl)
+    sh = blk["shared"] or (None, None, None)
+    W = moe.BlockWeights(gate_weight=dev["W"], gate_bias=dev["bias"], w1=dev["w1"], w3=dev["w3"],
+                         w2=dev["w2"], down_proj=blk["down_proj"], norm_weight=blk["norm_w"],
+                         up_proj=blk["up_proj"], shared_w1=sh[0], shared_w3=sh[1],
+                         shared_w2=sh[2])
+    cfg = moe.RouteConfig(wl.E, wl.G, wl.TG, wl.K, wl.route_scale, wl.norm)
+    act = moe.ActConfig(wl.act, wl.beta, wl.lbeta)
+    out = torch.empty((wl.N, wl.d_r), dtype=torch.bfloat16, device="cuda")
+    idx = torch.empty((wl.N, wl.K), dtype=torch.int32, device="cuda")
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    ws = [None]
+
+    def step(x=None):
+        o = moe.block_forward(dev["x"] if x is None else x, W, cfg, act, norm_eps=wl.norm_eps,
+                              ws=ws[0], out=out, topk_idx=idx)
+        return o
+
+    # first call sizes the workspace; keep it
+    import ctypes
+    dims = moe._BlockDims(wl.d_r, wl.d_e, wl.F, wl.F_shared, wl.norm_eps)
+    wc, c = W._c(), cfg._c()
+    ws[0] = moe.workspace(moe.lib().moe_block_workspace_size(wl.N, ctypes.byref(dims),
+                                                             ctypes.byref(wc), ctypes.byref(c)))
+    torch.cuda.synchronize()
+    for _ in range(max(args.warmup, 3)):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+
+    def barrier():
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+
+    ev0 = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    with ClockSampler(local_rank) as clk:
+        barrier()
+        torch.cuda.synchronize()
+        t0 = time.perf_counter()
+        for i in range(args.steps):
+            flush.zero_()
+            ev0[i][0].record()
+            step()
+            ev0[i][1].record()
+        torch.cuda.synchronize()
+        barrier()
+        wall = time.perf_counter() - t0
+    ms = statistics.mean(a.elapsed_time(b) for a, b in ev0)
+    counts = np.bincount(idx.cpu().numpy().ravel(), minlength=wl.E)
+    touched = int((counts > 0).sum())
+
+    x_host = torch.empty((wl.N, wl.d_r), dtype=torch.bfloat16, pin_memory=True)
+    x_host.copy_(dev["x"].cpu())
+    out_host = torch.empty((wl.N, wl.d_r), dtype=torch.bfloat16, pin_memory=True)
+    x_dev = torch.empty_like(dev["x"])
+
+    def e2e_step():
+        x_dev.copy_(x_host, non_blocking=True)
+        step(x_dev)
+        out_host.copy_(out, non_blocking=True)
+
+    for _ in range(3):
+        flush.zero_()
+        e2e_step()
+    torch.cuda.synchronize()
+    e2e_ms = []
+    for _ in range(args.steps):
+        flush.zero_()
+        s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s0.record()
+        e2e_step()
+        s1.record()
+        s1.synchronize()
+        e2e_ms.append(s0.elapsed_time(s1))
+    ms_max, e2e_max, wall_max = max_over_ranks([ms, statistics.mean(e2e_ms), wall], world, "cuda")
+    return wl, {"ms": ms_max, "e2e_ms": e2e_max, "touched": touched, "clocks": clk.summary(),
+                "h2d": wl.N * wl.d_r * 2, "d2h": wl.N * wl.d_r * 2, "wall_s": wall_max}
+
+
+def block_line(args, wl, r, world):
+    peaks = load_peaks()
+    achieved = block_bytes(wl, r["touched"]) / (r["ms"] * 1e-3) / 1e9
+    return {
+        "metric": BLOCK_METRIC, "value": aggregate_throughput(wl.N, world, r["ms"]),
+        "unit": UNIT, "n_gpus": world, "steps": args.steps, "warmup": max(args.warmup, 3),
+        "ms_per_step": r["ms"], "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": wl.name, "N": wl.N, "d_r": wl.d_r, "d_e": wl.d_e, "E": wl.E,
+                   "K": wl.K, "F": wl.F, "F_shared": wl.F_shared, "act": wl.act,
+                   "global_batch": world * wl.N, "parallelism": f"dp{world}",
+                   "l2": "weights > L2, plus a 256 MB write between steps outside the "
+                         "per-step events"},
+        "roofline": {"kernel": "whole block step (HBM-bound weight stream)", "bound": "hbm",
+                     "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": achieved / peaks["hbm_gbs"], "traffic": None,
+                     "peak_source": peaks["source"], "touched_experts": r["touched"]},
+        "e2e": {"value": aggregate_throughput(wl.N, world, r["e2e_ms"]), "unit": UNIT,
+                "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"]},
+        "gpu_launches": block_kernels(wl) * args.steps,
+        "clocks": r["clocks"],
+    }
+
+
 def gate_up_traffic(touched):
     """DRAM bytes of one gate_up launch from the committed ncu capture of a
     smaller case, scaled by touched experts; None once the kernel source has
@@ -397,6 +549,17 @@ def main():
         torch.cuda.set_device(local_rank)
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local_rank))
+    from synth.workloads import BLOCKS
+    if args.workload in BLOCKS:
+        wl, r = run_block(args, rank, world, local_rank)
+        line = block_line(args, wl, r, world)
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+            dist.destroy_process_group()
+        if rank == 0:
+            print(json.dumps(line), flush=True)
+        return
     wl, r = run_ours(args, rank, world, local_rank)
     peaks = load_peaks()
     achieved = gate_up_bytes(wl, r["touched"]) / (r["gate_up_ms"] * 1e-3) / 1e9

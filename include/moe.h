@@ -79,7 +79,21 @@ typedef struct moe_route_cfg {
   int top_k;           /* K: experts per token (num_experts_per_tok)           */
   int norm_topk_prob;  /* nonzero: renormalise the K weights when K > 1        */
   float route_scale;   /* routed_scaling_factor / route_scale                  */
+  int score_func;      /* MOE_SCORE_SIGMOID (0, default) or MOE_SCORE_SOFTMAX   */
+  int group_score;     /* MOE_GROUP_TOP2_SUM (0, default) or MOE_GROUP_MAX      */
 } moe_route_cfg;
+
+/* Scoring variants ("DeepSeek-V3.2-Exp · Affinities", gate-forward):
+ *   MOE_SCORE_SOFTMAX: s = softmax over all E logits (fp32 rounding of
+ *     exp(L_e - max) / sum_j exp(L_j - max), evaluated in double with the sum
+ *     taken in expert order) in place of the sigmoid; that page renormalises
+ *     only sigmoid scores, so softmax routing in its form sets
+ *     norm_topk_prob = 0;
+ *   MOE_GROUP_MAX: group score = the group's largest choice score (the page's
+ *     amax, used there when the gate has no correction bias) in place of the
+ *     sum of its two largest. */
+enum { MOE_SCORE_SIGMOID = 0, MOE_SCORE_SOFTMAX = 1 };
+enum { MOE_GROUP_TOP2_SUM = 0, MOE_GROUP_MAX = 1 };
 
 /* Expert activation ("Kimi K3 · Gate features", situ excerpt).
  * kind MOE_ACT_SILU: h = bf16(bf16(silu(g)) * u), silu(g) = g * sigmoid(g).
@@ -242,6 +256,77 @@ MOE_API int moe_forward(const moe_bf16* x_r, const moe_bf16* x_e, int64_t N, int
                         const moe_act_cfg* act, moe_bf16* out, int32_t* topk_idx_out,
                         float* topk_w_out, void* ws, size_t ws_bytes, void* stream,
                         const moe_stage_events* events);
+
+/* ------------------------------------------------ the block around the layer
+ *
+ * KimiSparseMoeBlock.forward ("Kimi K3 · Add shared output", moe-forward
+ * excerpt): the gate scores the full-width input x; a latent block projects x
+ * down (routed_expert_down_proj) before moe_infer, then normalises
+ * (routed_expert_norm) and projects up (routed_expert_up_proj); the shared
+ * experts' output on x is added last.  Readings where the pages are silent:
+ * both projections are bias-free Linear layers; routed_expert_norm is an
+ * RMSNorm with a bf16 weight (moe_rms_norm); the shared experts are one gated
+ * MLP of the routed experts' kind and activation on the full width, of hidden
+ * width F_shared (the sum over shared experts). */
+
+/* Bias-free bf16 Linear, y[m, n] = bf16( sum_k x[m, k] * W[n, k] ) with fp32
+ * tensor-core accumulation, and with a residual y = bf16( bf16(sum) +
+ * residual[m, n] ).  x [M, K], W [N_out, K] (nn.Linear layout), residual and
+ * y [M, N_out]: bf16, row-major, device memory, 16-byte aligned.  K and N_out
+ * multiples of 128.  y may be the residual buffer; it must not overlap x or
+ * W.  Workspace: moe_linear_workspace_size() bytes. */
+MOE_API size_t moe_linear_workspace_size(void);
+MOE_API int moe_linear(const moe_bf16* x, int64_t M, int K, const moe_bf16* W, int N_out,
+                       const moe_bf16* residual, moe_bf16* y, void* ws, size_t ws_bytes,
+                       void* stream);
+
+/* RMSNorm of each row of x [N, d] (the reading of routed_expert_norm):
+ *   r = 1 / sqrt(mean(x^2) + eps)   (double)
+ *   out = bf16( weight * bf16(x * r) )
+ * weight [d] bf16; d a multiple of 8, at most 8192; eps finite and >= 0.
+ * out may equal x.  No workspace, no device-side failure. */
+MOE_API int moe_rms_norm(const moe_bf16* x, int64_t N, int d, const moe_bf16* weight, float eps,
+                         moe_bf16* out, void* stream);
+
+typedef struct moe_block_dims {
+  int d_r;          /* hidden size (router input, block output)              */
+  int d_e;          /* routed experts' width: d_r, or the latent width        */
+  int F;            /* routed experts' hidden width (moe_intermediate_size)   */
+  int F_shared;     /* shared experts' hidden width, 0 = no shared experts    */
+  float norm_eps;   /* routed_expert_norm epsilon                             */
+} moe_block_dims;
+
+/* Device pointers, 16-byte aligned.  NULL marks an absent part. */
+typedef struct moe_block_weights {
+  const float* gate_weight;     /* [E, d_r] fp32                                  */
+  const float* gate_bias;       /* [E] fp32 correction bias, or NULL              */
+  const moe_bf16* down_proj;    /* [d_e, d_r]; NULL: not latent (d_e == d_r)      */
+  const moe_bf16* norm_weight;  /* [d_e]; NULL: no routed_expert_norm (latent only)*/
+  const moe_bf16* up_proj;      /* [d_r, d_e]; given exactly when down_proj is    */
+  const moe_bf16* w1;           /* routed experts [E, F, d_e]                     */
+  const moe_bf16* w3;           /* [E, F, d_e]                                    */
+  const moe_bf16* w2;           /* [E, d_e, F]                                    */
+  const moe_bf16* shared_w1;    /* [F_shared, d_r], or NULL with the two below    */
+  const moe_bf16* shared_w3;    /* [F_shared, d_r]                                */
+  const moe_bf16* shared_w2;    /* [d_r, F_shared]                                */
+} moe_block_weights;
+
+/* Workspace bytes for moe_block_forward (0 if the arguments are invalid). */
+MOE_API size_t moe_block_workspace_size(int64_t N, const moe_block_dims* dims,
+                                        const moe_block_weights* weights,
+                                        const moe_route_cfg* cfg);
+
+/* out [N, d_r] bf16 = the block on x [N, d_r] bf16, on one stream with no host
+ * synchronisation: route -> shared experts -> down_proj -> dispatch -> expert
+ * MLP -> combine (+ RMSNorm) -> up_proj (+ shared output); without a latent
+ * projection the combine adds the shared output.  d_r, d_e, F, F_shared
+ * multiples of 128; d_e <= 8192; the routed layer's limits apply.
+ * topk_idx_out / topk_w_out as in moe_forward.  act applies to the routed and
+ * the shared experts. */
+MOE_API int moe_block_forward(const moe_bf16* x, int64_t N, const moe_block_dims* dims,
+                              const moe_block_weights* weights, const moe_route_cfg* cfg,
+                              const moe_act_cfg* act, moe_bf16* out, int32_t* topk_idx_out,
+                              float* topk_w_out, void* ws, size_t ws_bytes, void* stream);
 
 /* --------------------------------------------------------------- status */
 

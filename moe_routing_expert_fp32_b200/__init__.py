@@ -35,7 +35,8 @@ class MoeError(RuntimeError):
 class _RouteCfg(ctypes.Structure):
     _fields_ = [("num_experts", ctypes.c_int), ("n_group", ctypes.c_int),
                 ("topk_group", ctypes.c_int), ("top_k", ctypes.c_int),
-                ("norm_topk_prob", ctypes.c_int), ("route_scale", ctypes.c_float)]
+                ("norm_topk_prob", ctypes.c_int), ("route_scale", ctypes.c_float),
+                ("score_func", ctypes.c_int), ("group_score", ctypes.c_int)]
 
 
 class _ActCfg(ctypes.Structure):
@@ -57,10 +58,50 @@ class RouteConfig:
     top_k: int
     route_scale: float
     norm_topk_prob: bool = True
+    score_func: str = "sigmoid"   # or "softmax"
+    group_score: str = "top2_sum"  # or "max"
 
     def _c(self) -> _RouteCfg:
         return _RouteCfg(self.num_experts, self.n_group, self.topk_group, self.top_k,
-                         int(bool(self.norm_topk_prob)), self.route_scale)
+                         int(bool(self.norm_topk_prob)), self.route_scale,
+                         {"sigmoid": 0, "softmax": 1}[self.score_func],
+                         {"top2_sum": 0, "max": 1}[self.group_score])
+
+
+class _BlockDims(ctypes.Structure):
+    _fields_ = [("d_r", ctypes.c_int), ("d_e", ctypes.c_int), ("F", ctypes.c_int),
+                ("F_shared", ctypes.c_int), ("norm_eps", ctypes.c_float)]
+
+
+class _BlockWeights(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in (
+        "gate_weight", "gate_bias", "down_proj", "norm_weight", "up_proj", "w1", "w3", "w2",
+        "shared_w1", "shared_w3", "shared_w2")]
+
+
+@dataclass
+class BlockWeights:
+    """Device tensors of one MoE block (None marks an absent part).
+
+    gate_weight [E, d_r] fp32, gate_bias [E] fp32; down_proj [d_e, d_r],
+    norm_weight [d_e], up_proj [d_r, d_e]; routed w1, w3 [E, F, d_e], w2
+    [E, d_e, F]; shared_w1, shared_w3 [F_sh, d_r], shared_w2 [d_r, F_sh]; bf16.
+    """
+    gate_weight: object
+    w1: object
+    w3: object
+    w2: object
+    gate_bias: object = None
+    down_proj: object = None
+    norm_weight: object = None
+    up_proj: object = None
+    shared_w1: object = None
+    shared_w3: object = None
+    shared_w2: object = None
+
+    def _c(self) -> _BlockWeights:
+        return _BlockWeights(*[None if getattr(self, n) is None else getattr(self, n).data_ptr()
+                               for n, _ in _BlockWeights._fields_])
 
 
 @dataclass(frozen=True)
@@ -79,7 +120,9 @@ EXPORTS = ("moe_route_workspace_size", "moe_route", "moe_route_from_logits",
            "moe_gate_logits_workspace_size", "moe_gate_logits",
            "moe_dispatch_workspace_size", "moe_dispatch", "moe_expert_ffn_workspace_size",
            "moe_expert_ffn", "moe_combine_workspace_size", "moe_combine", "moe_workspace_size",
-           "moe_forward", "moe_get_status", "moe_strerror", "moe_dispatch_static")
+           "moe_forward", "moe_get_status", "moe_strerror", "moe_dispatch_static",
+           "moe_linear_workspace_size", "moe_linear", "moe_rms_norm", "moe_block_workspace_size",
+           "moe_block_forward")
 
 
 def lib() -> ctypes.CDLL:
@@ -93,6 +136,7 @@ def lib() -> ctypes.CDLL:
     L = ctypes.CDLL(LIB_PATH)
     vp, i64, i32, sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t
     rc, ac, ev = ctypes.POINTER(_RouteCfg), ctypes.POINTER(_ActCfg), ctypes.POINTER(_StageEvents)
+    bd, bw = ctypes.POINTER(_BlockDims), ctypes.POINTER(_BlockWeights)
     sig = {
         "moe_route_workspace_size": ([i64, i32, rc], sz),
         "moe_route": ([vp, i64, i32, vp, vp, rc, vp, vp, vp, sz, vp], i32),
@@ -111,6 +155,11 @@ def lib() -> ctypes.CDLL:
         "moe_get_status": ([vp, vp], i32),
         "moe_dispatch_static": ([vp, i64, i32, i32, vp, i32, vp, vp, vp, vp, vp, vp], i32),
         "moe_strerror": ([i32], ctypes.c_char_p),
+        "moe_linear_workspace_size": ([], sz),
+        "moe_linear": ([vp, i64, i32, vp, i32, vp, vp, vp, sz, vp], i32),
+        "moe_rms_norm": ([vp, i64, i32, vp, ctypes.c_float, vp, vp], i32),
+        "moe_block_workspace_size": ([i64, bd, bw, rc], sz),
+        "moe_block_forward": ([vp, i64, bd, bw, rc, ac, vp, vp, vp, vp, sz, vp], i32),
     }
     for name, (args, res) in sig.items():
         fn = getattr(L, name)
@@ -334,4 +383,60 @@ def forward(x_r, W, bias, cfg: RouteConfig, w1, w3, w2, act: ActConfig, x_e=None
                              ctypes.byref(c), _ptr(w1), _ptr(w3), _ptr(w2), F, ctypes.byref(a),
                              _ptr(out), _ptr(topk_idx), _ptr(topk_w), _ptr(ws), ws.numel(),
                              _stream(), evp))
+    return out
+
+
+# ------------------------------------------------------- the block around it
+def linear(x, W, residual=None, out=None, ws=None):
+    """bf16(x . W^T) (+ residual) through moe_linear; x [M, K], W [N_out, K]."""
+    torch = _torch()
+    M, K = x.shape
+    N_out = W.shape[0]
+    _need(x, torch.bfloat16, name="x")
+    _need(W, torch.bfloat16, (N_out, K), "W")
+    if residual is not None:
+        _need(residual, torch.bfloat16, (M, N_out), "residual")
+    ws = workspace(lib().moe_linear_workspace_size(), x.device) if ws is None else ws
+    out = torch.empty((M, N_out), dtype=torch.bfloat16, device=x.device) if out is None else out
+    _check("moe_linear", lib().moe_linear(_ptr(x), M, K, _ptr(W), N_out, _ptr(residual),
+                                          _ptr(out), _ptr(ws), ws.numel(), _stream()))
+    return out
+
+
+def rms_norm(x, weight, eps, out=None):
+    torch = _torch()
+    N, d = x.shape
+    _need(x, torch.bfloat16, name="x")
+    _need(weight, torch.bfloat16, (d,), "weight")
+    out = torch.empty_like(x) if out is None else out
+    _check("moe_rms_norm", lib().moe_rms_norm(_ptr(x), N, d, _ptr(weight), float(eps), _ptr(out),
+                                              _stream()))
+    return out
+
+
+def block_forward(x, weights: BlockWeights, cfg: RouteConfig, act: ActConfig, norm_eps=1e-6,
+                  ws=None, out=None, topk_idx=None, topk_w=None):
+    """KimiSparseMoeBlock.forward (moe_block_forward). Returns ``out`` [N, d_r] bf16."""
+    torch = _torch()
+    N, d_r = x.shape
+    E, F, d_e = weights.w1.shape
+    _need(x, torch.bfloat16, name="x")
+    _need(weights.gate_weight, torch.float32, (E, d_r), "gate_weight")
+    if weights.down_proj is not None:
+        _need(weights.down_proj, torch.bfloat16, (d_e, d_r), "down_proj")
+        _need(weights.up_proj, torch.bfloat16, (d_r, d_e), "up_proj")
+    F_sh = 0 if weights.shared_w1 is None else weights.shared_w1.shape[0]
+    dims = _BlockDims(d_r, d_e, F, F_sh, float(norm_eps))
+    wc = weights._c()
+    c = cfg._c()
+    a = act._c()
+    need = lib().moe_block_workspace_size(N, ctypes.byref(dims), ctypes.byref(wc), ctypes.byref(c))
+    if need == 0:
+        raise MoeError("moe_block_workspace_size", -1)
+    ws = workspace(need, x.device) if ws is None else ws
+    out = torch.empty((N, d_r), dtype=torch.bfloat16, device=x.device) if out is None else out
+    _check("moe_block_forward",
+           lib().moe_block_forward(_ptr(x), N, ctypes.byref(dims), ctypes.byref(wc),
+                                   ctypes.byref(c), ctypes.byref(a), _ptr(out), _ptr(topk_idx),
+                                   _ptr(topk_w), _ptr(ws), ws.numel(), _stream()))
     return out

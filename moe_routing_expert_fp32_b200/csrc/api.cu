@@ -53,6 +53,10 @@ int check_route_cfg(const moe_route_cfg* c) {
   if (G > 1 && E / G < 2) return MOE_ERR_INVALID_ARG;
   if ((int64_t)K > (int64_t)TG * (E / G)) return MOE_ERR_INVALID_ARG;
   if (!isfinite(c->route_scale)) return MOE_ERR_INVALID_ARG;
+  if (c->score_func != MOE_SCORE_SIGMOID && c->score_func != MOE_SCORE_SOFTMAX)
+    return MOE_ERR_INVALID_ARG;
+  if (c->group_score != MOE_GROUP_TOP2_SUM && c->group_score != MOE_GROUP_MAX)
+    return MOE_ERR_INVALID_ARG;
   if (E > 1024 || G > 32 || K > 16) return MOE_ERR_UNSUPPORTED;
   return MOE_OK;
 }
@@ -382,6 +386,188 @@ int moe_forward(const moe_bf16* x_r, const moe_bf16* x_e, int64_t N, int d_r, in
     return MOE_ERR_CUDA;
   if (events && !rec(events->after_combine)) return MOE_ERR_CUDA;
   return MOE_OK;
+}
+
+// ------------------------------------------------------------ dense layers
+size_t moe_linear_workspace_size(void) { return kStatusBytes + kDenseTilesBytes; }
+
+int moe_linear(const moe_bf16* x, int64_t M, int K, const moe_bf16* W, int N_out,
+               const moe_bf16* residual, moe_bf16* y, void* ws, size_t ws_bytes, void* stream) {
+  if (M < 0 || K <= 0 || N_out <= 0) return MOE_ERR_INVALID_ARG;
+  if (K % 128 != 0 || N_out % 128 != 0 || M > INT32_MAX) return MOE_ERR_UNSUPPORTED;
+  if (!W) return MOE_ERR_INVALID_ARG;
+  if (M > 0 && (!x || !y)) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(W)) return MOE_ERR_ALIGNMENT;
+  if (M > 0 && (!aligned16(x) || !aligned16(y) || (residual && !aligned16(residual))))
+    return MOE_ERR_ALIGNMENT;
+  int rc;
+  if ((rc = check_ws(ws, ws_bytes, moe_linear_workspace_size()))) return rc;
+  if ((rc = check_device())) return rc;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if ((rc = reset_status(ws, s))) return rc;
+  if (M == 0) return MOE_OK;
+  int32_t* tiles = reinterpret_cast<int32_t*>(body_of(ws));
+  if (launch_dense_tiles(M, tiles, s) != cudaSuccess) return MOE_ERR_CUDA;
+  return linear_run(reinterpret_cast<const __nv_bfloat16*>(x), M, K,
+                    reinterpret_cast<const __nv_bfloat16*>(W), N_out,
+                    reinterpret_cast<const __nv_bfloat16*>(residual),
+                    reinterpret_cast<__nv_bfloat16*>(y), tiles, status_of(ws), s,
+                    /*pdl_ok=*/false);  // the tile list was written by the kernel just before
+}
+
+int moe_rms_norm(const moe_bf16* x, int64_t N, int d, const moe_bf16* weight, float eps,
+                 moe_bf16* out, void* stream) {
+  if (N < 0 || d <= 0 || !(eps >= 0.0f) || !isfinite(eps)) return MOE_ERR_INVALID_ARG;
+  if (d % 8 != 0 || d > 8192) return MOE_ERR_UNSUPPORTED;
+  if (!weight) return MOE_ERR_INVALID_ARG;
+  if (N > 0 && (!x || !out)) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(weight) || (N > 0 && (!aligned16(x) || !aligned16(out))))
+    return MOE_ERR_ALIGNMENT;
+  int rc;
+  if ((rc = check_device())) return rc;
+  if (N == 0) return MOE_OK;
+  return launch_rms_norm(reinterpret_cast<const __nv_bfloat16*>(x), N, d,
+                         reinterpret_cast<const __nv_bfloat16*>(weight), eps,
+                         reinterpret_cast<__nv_bfloat16*>(out),
+                         static_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? MOE_OK
+             : MOE_ERR_CUDA;
+}
+
+// ------------------------------------------------------------ whole block
+namespace {
+struct BlockLayout {
+  ForwardLayout fwd;     // the routed layer's regions (status word at 0)
+  size_t tiles, xe, yc, sh, hsh, total;
+};
+
+BlockLayout block_layout(int64_t N, const moe_block_dims& d, const moe_route_cfg& c,
+                         bool latent, bool shared) {
+  BlockLayout L{};
+  L.fwd = forward_layout(N, d.d_r, d.d_e, c.num_experts, c.top_k, d.F);
+  size_t o = L.fwd.total;
+  L.tiles = o; o += kDenseTilesBytes;
+  const size_t ne = sizeof(__nv_bfloat16) * (size_t)N * (size_t)d.d_e;
+  if (latent) {
+    L.xe = o; o += align_up(ne, 256);
+    L.yc = o; o += align_up(ne, 256);
+  }
+  if (shared) {
+    L.sh = o; o += align_up(sizeof(__nv_bfloat16) * (size_t)N * (size_t)d.d_r, 256);
+    L.hsh = o; o += align_up(sizeof(__nv_bfloat16) * (size_t)N * (size_t)d.F_shared, 256);
+  }
+  L.total = o;
+  return L;
+}
+
+int check_block(int64_t N, const moe_block_dims* d, const moe_block_weights* wt,
+                const moe_route_cfg* cfg, bool* latent, bool* shared) {
+  if (!d || !wt) return MOE_ERR_INVALID_ARG;
+  int rc = check_route_cfg(cfg);
+  if (rc) return rc;
+  if (N < 0 || d->d_r <= 0 || d->d_e <= 0 || d->F <= 0 || d->F_shared < 0)
+    return MOE_ERR_INVALID_ARG;
+  if (!(d->norm_eps >= 0.0f) || !isfinite(d->norm_eps)) return MOE_ERR_INVALID_ARG;
+  *latent = wt->down_proj != nullptr;
+  *shared = wt->shared_w1 != nullptr;
+  if ((wt->up_proj != nullptr) != *latent) return MOE_ERR_INVALID_ARG;
+  if (!*latent && (d->d_e != d->d_r || wt->norm_weight)) return MOE_ERR_INVALID_ARG;
+  if ((wt->shared_w3 != nullptr) != *shared || (wt->shared_w2 != nullptr) != *shared ||
+      (d->F_shared > 0) != *shared)
+    return MOE_ERR_INVALID_ARG;
+  if (!wt->gate_weight || !wt->w1 || !wt->w3 || !wt->w2) return MOE_ERR_INVALID_ARG;
+  if ((rc = check_expert_shape(N * (int64_t)cfg->top_k, d->d_e, cfg->num_experts, d->F)))
+    return rc;
+  if (d->d_r % 128 != 0 || d->F_shared % 128 != 0 || d->d_e > 8192 || N > INT32_MAX)
+    return MOE_ERR_UNSUPPORTED;
+  const void* ptrs[] = {wt->gate_weight, wt->down_proj, wt->norm_weight, wt->up_proj, wt->w1,
+                        wt->w3, wt->w2, wt->shared_w1, wt->shared_w3, wt->shared_w2};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return MOE_ERR_ALIGNMENT;
+  return MOE_OK;
+}
+}  // namespace
+
+size_t moe_block_workspace_size(int64_t N, const moe_block_dims* dims,
+                                const moe_block_weights* weights, const moe_route_cfg* cfg) {
+  bool latent = false, shared = false;
+  if (check_block(N, dims, weights, cfg, &latent, &shared) != MOE_OK) return 0;
+  return block_layout(N, *dims, *cfg, latent, shared).total;
+}
+
+int moe_block_forward(const moe_bf16* x, int64_t N, const moe_block_dims* dims,
+                      const moe_block_weights* wt, const moe_route_cfg* cfg,
+                      const moe_act_cfg* act, moe_bf16* out, int32_t* topk_idx_out,
+                      float* topk_w_out, void* ws, size_t ws_bytes, void* stream) {
+  bool latent = false, shared = false;
+  int rc = check_block(N, dims, wt, cfg, &latent, &shared);
+  if (rc) return rc;
+  if ((rc = check_act(act))) return rc;
+  if (N > 0 && (!x || !out)) return MOE_ERR_INVALID_ARG;
+  if (N > 0 && (!aligned16(x) || !aligned16(out))) return MOE_ERR_ALIGNMENT;
+  const BlockLayout L = block_layout(N, *dims, *cfg, latent, shared);
+  if ((rc = check_ws(ws, ws_bytes, L.total))) return rc;
+  if ((rc = check_device())) return rc;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if ((rc = reset_status(ws, s))) return rc;
+  if (N == 0) return MOE_OK;
+  const int d_r = dims->d_r, d_e = dims->d_e, E = cfg->num_experts, K = cfg->top_k;
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  DeviceStatus* st = status_of(ws);
+  auto bf = [&](size_t off) { return reinterpret_cast<__nv_bfloat16*>(base + off); };
+  auto cbf = [](const moe_bf16* p) { return reinterpret_cast<const __nv_bfloat16*>(p); };
+  const ForwardLayout& F = L.fwd;
+  uint8_t* stage = base + F.stage;
+  int32_t* idx = topk_idx_out ? topk_idx_out : reinterpret_cast<int32_t*>(base + F.idx);
+  float* w = topk_w_out ? topk_w_out : reinterpret_cast<float*>(base + F.w);
+  int32_t* offsets = reinterpret_cast<int32_t*>(base + F.offsets);
+  int32_t* pos = reinterpret_cast<int32_t*>(base + F.pos);
+  int32_t* tiles = reinterpret_cast<int32_t*>(base + L.tiles);
+  const __nv_bfloat16* xr = cbf(x);
+  __nv_bfloat16* sh = shared ? bf(L.sh) : nullptr;
+  __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(out);
+
+  if (launch_dense_tiles(N, tiles, s) != cudaSuccess) return MOE_ERR_CUDA;
+  // gate on the full-width input
+  if ((rc = route_impl(xr, N, d_r, wt->gate_weight, wt->gate_bias, *cfg, idx, w, stage, st, s)))
+    return rc;
+  // shared experts on the full-width input (their output is the residual of
+  // the last step)
+  if (shared && (rc = shared_ffn_run(xr, N, d_r, dims->F_shared, cbf(wt->shared_w1),
+                                     cbf(wt->shared_w3), cbf(wt->shared_w2), *act, nullptr, sh,
+                                     bf(L.hsh), tiles, st, s)))
+    return rc;
+  // routed_expert_down_proj
+  const __nv_bfloat16* xe = xr;
+  if (latent) {
+    // (the tile list was written before the router's kernels: a programmatic
+    // dependent launch is safe here and below)
+    if ((rc = linear_run(xr, N, d_r, cbf(wt->down_proj), d_e, nullptr, bf(L.xe), tiles, st, s,
+                         true)))
+      return rc;
+    xe = bf(L.xe);
+  }
+  // moe_infer
+  if (launch_dispatch(idx, N, K, E, xe, d_e, reinterpret_cast<int32_t*>(base + F.counts), offsets,
+                      reinterpret_cast<int32_t*>(base + F.perm), pos, bf(F.xs),
+                      reinterpret_cast<int32_t*>(stage), st, s) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  if ((rc = expert_ffn_run(bf(F.xs), offsets, E, N * K, d_e, dims->F, cbf(wt->w1), cbf(wt->w3),
+                           cbf(wt->w2), *act, bf(F.y), stage, st, s, nullptr)))
+    return rc;
+  if (!latent)
+    return launch_combine(bf(F.y), pos, w, N, K, d_e, N * K, o, st, s, sh) == cudaSuccess
+               ? MOE_OK
+               : MOE_ERR_CUDA;
+  // routed_expert_norm (fused with the combine) and routed_expert_up_proj,
+  // whose epilogue adds the shared experts' output
+  cudaError_t e = wt->norm_weight
+                      ? launch_combine_rms_norm(bf(F.y), pos, w, N, K, d_e, N * K,
+                                                cbf(wt->norm_weight), dims->norm_eps, bf(L.yc),
+                                                st, s)
+                      : launch_combine(bf(F.y), pos, w, N, K, d_e, N * K, bf(L.yc), st, s);
+  if (e != cudaSuccess) return MOE_ERR_CUDA;
+  return linear_run(bf(L.yc), N, d_e, cbf(wt->up_proj), d_r, sh, o, tiles, st, s, true);
 }
 
 }  // extern "C"

@@ -213,6 +213,16 @@ __device__ __forceinline__ float bf16r(float x) {
   return __bfloat162float(__float2bfloat16_rn(x));
 }
 
+// Down-projection output element (row, m): bf16 of the accumulator, or with a
+// residual bf16( bf16(acc) + res ) -- the Linear output is a bf16 tensor
+// before the add, and the add of two bf16 values is rounded once.
+__device__ __forceinline__ __nv_bfloat16 down_out(float acc, const __nv_bfloat16* res, int row,
+                                                  int M_rows, int m) {
+  if (!res) return __float2bfloat16_rn(acc);
+  return __float2bfloat16_rn(
+      __fadd_rn(bf16r(acc), __bfloat162float(res[(int64_t)row * M_rows + m])));
+}
+
 // SiLU-and-mul with the page's rounding points: g and u are bf16 Linear
 // outputs; silu(g) is evaluated in fp32 and rounded to bf16; the product of two
 // bf16 values is exact in fp32 and rounded to bf16 by the store.
@@ -260,8 +270,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                   const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmB64,
                   const int32_t* __restrict__ offsets,
                   const int32_t* __restrict__ tile_start, int E, int M_rows, int Kdim,
-                  __nv_bfloat16* __restrict__ out, int act_kind, float beta, float lbeta,
-                  DeviceStatus* st, int pdl) {
+                  __nv_bfloat16* __restrict__ out, const __nv_bfloat16* __restrict__ res,
+                  int act_kind, float beta, float lbeta, DeviceStatus* st, int pdl) {
   using C = Cfg<NTMAX, STAGES, UM, KSUB>;
   constexpr int KS = BK * KSUB;  // K columns per stage
   constexpr bool kDecode = NTMAX <= 32;
@@ -502,7 +512,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           lim = lim < lim_m ? lim : lim_m;
 #pragma unroll
           for (int j = 0; j < 16; ++j)
-            if (j < lim) col[(int64_t)(w.row0 + c0 + j) * M_rows] = __float2bfloat16_rn(v[j]);
+            if (j < lim) col[(int64_t)(w.row0 + c0 + j) * M_rows] = down_out(v[j], res, w.row0 + c0 + j, M_rows, m);
         }
       }
       }  // accumulators
@@ -611,8 +621,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                        const __grid_constant__ CUtensorMap tmB,
                        const __grid_constant__ CUtensorMap tmB64,
                        const int32_t* __restrict__ offsets, const int32_t* __restrict__ tile_start,
-                       int E, int M_rows, int Kdim, __nv_bfloat16* __restrict__ out, int act_kind,
-                       float beta, float lbeta, DeviceStatus* st, int pdl) {
+                       int E, int M_rows, int Kdim, __nv_bfloat16* __restrict__ out,
+                       const __nv_bfloat16* __restrict__ res, int act_kind, float beta,
+                       float lbeta, DeviceStatus* st, int pdl) {
   using C = PairCfg;
   constexpr int STAGES = kPairStages;
   extern __shared__ uint8_t smem_raw[];
@@ -818,7 +829,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           lim = lim < lim_m ? lim : lim_m;
 #pragma unroll
           for (int j = 0; j < 16; ++j)
-            if (j < lim) col[(int64_t)(w.row0 + c0 + j) * M_rows] = __float2bfloat16_rn(v[j]);
+            if (j < lim) col[(int64_t)(w.row0 + c0 + j) * M_rows] = down_out(v[j], res, w.row0 + c0 + j, M_rows, m);
         }
       }
       tc_fence_before();
@@ -927,8 +938,9 @@ bool make_map_2d(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows,
 template <int MODE, int NTMAX, int STAGES, int UM, int KSUB>
 cudaError_t launch_gemm(const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorMap& b,
                         const CUtensorMap& b64, const int32_t* offsets, const int32_t* tile_start,
-                        int E, int M_rows, int Kdim, __nv_bfloat16* out, const moe_act_cfg& act,
-                        DeviceStatus* st, cudaStream_t s) {
+                        int E, int M_rows, int Kdim, __nv_bfloat16* out,
+                        const __nv_bfloat16* res, const moe_act_cfg& act, DeviceStatus* st,
+                        cudaStream_t s, bool pdl_ok) {
   using C = Cfg<NTMAX, STAGES, UM, KSUB>;
   static bool attr_set[64] = {false};
   int dev = 0;
@@ -940,9 +952,12 @@ cudaError_t launch_gemm(const CUtensorMap& a0, const CUtensorMap& a1, const CUte
     if (e != cudaSuccess) return e;
     attr_set[dev] = true;
   }
-  // The down projection is launched as a programmatic dependent of the gate_up
-  // kernel: its CTAs start as gate_up CTAs retire and prefetch w2 tiles.
-  const int pdl = MODE == kDown ? 1 : 0;
+  // The down projection is launched as a programmatic dependent of the kernel
+  // before it (the gate_up kernel in the expert MLP): its CTAs start as those
+  // CTAs retire and prefetch weight tiles.  Every role reads the tile list
+  // before griddepcontrol.wait, so the caller allows this only when the list
+  // was complete before the preceding kernel started.
+  const int pdl = (MODE == kDown && pdl_ok) ? 1 : 0;
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -954,8 +969,8 @@ cudaError_t launch_gemm(const CUtensorMap& a0, const CUtensorMap& a1, const CUte
   cfg.attrs = attr;
   cfg.numAttrs = pdl ? 1 : 0;
   return cudaLaunchKernelEx(&cfg, k_expert_gemm<MODE, NTMAX, STAGES, UM, KSUB>, a0, a1, b, b64,
-                            offsets, tile_start, E, M_rows, Kdim, out, (int)act.kind, act.beta,
-                            act.linear_beta, st, pdl);
+                            offsets, tile_start, E, M_rows, Kdim, out, res, (int)act.kind,
+                            act.beta, act.linear_beta, st, pdl);
 }
 
 // Launches the CTA-pair kernel on as many pairs as can be resident at once.
@@ -963,8 +978,9 @@ template <int MODE>
 cudaError_t launch_gemm_pair(const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorMap& b,
                              const CUtensorMap& b64, const int32_t* offsets,
                              const int32_t* tile_start, int E, int M_rows, int Kdim,
-                             __nv_bfloat16* out, const moe_act_cfg& act, DeviceStatus* st,
-                             cudaStream_t s) {
+                             __nv_bfloat16* out, const __nv_bfloat16* res,
+                             const moe_act_cfg& act, DeviceStatus* st, cudaStream_t s,
+                             bool pdl_ok) {
   using C = PairCfg;
   static bool attr_set[64] = {false};
   static int grid_of[64] = {0};
@@ -983,7 +999,7 @@ cudaError_t launch_gemm_pair(const CUtensorMap& a0, const CUtensorMap& a1, const
   cfg.stream = s;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  const int pdl = MODE == kDown ? 1 : 0;
+  const int pdl = (MODE == kDown && pdl_ok) ? 1 : 0;
   if (dev < 64 && !attr_set[dev]) {
     cudaError_t e = cudaFuncSetAttribute(k_expert_gemm_pair<MODE>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -1000,8 +1016,8 @@ cudaError_t launch_gemm_pair(const CUtensorMap& a0, const CUtensorMap& a1, const
   cfg.gridDim = dim3(grid_of[dev < 64 ? dev : 0], 1, 1);
   cfg.numAttrs = pdl ? 2 : 1;
   return cudaLaunchKernelEx(&cfg, k_expert_gemm_pair<MODE>, a0, a1, b, b64, offsets, tile_start,
-                            E, M_rows, Kdim, out, (int)act.kind, act.beta, act.linear_beta, st,
-                            pdl);
+                            E, M_rows, Kdim, out, res, (int)act.kind, act.beta, act.linear_beta,
+                            st, pdl);
 }
 
 // Variant choice from shapes only (no host round trip), by the average rows
@@ -1024,18 +1040,18 @@ template <int MODE>
 cudaError_t launch_variant(Variant v, const CUtensorMap& a0, const CUtensorMap& a1,
                            const CUtensorMap& b, const CUtensorMap& b64, const int32_t* offsets,
                            const int32_t* tile_start, int E, int M_rows, int Kdim,
-                           __nv_bfloat16* out, const moe_act_cfg& act, DeviceStatus* st,
-                           cudaStream_t s) {
+                           __nv_bfloat16* out, const __nv_bfloat16* res, const moe_act_cfg& act,
+                           DeviceStatus* st, cudaStream_t s, bool pdl_ok = true) {
   switch (v) {
     case kVarDecode:
-      return launch_gemm<MODE, kNtDecode, kStagesDecode, kUmDecode, kKsubDecode>(a0, a1, b, b64, offsets, tile_start, E,
-                                                         M_rows, Kdim, out, act, st, s);
+      return launch_gemm<MODE, kNtDecode, kStagesDecode, kUmDecode, kKsubDecode>(
+          a0, a1, b, b64, offsets, tile_start, E, M_rows, Kdim, out, res, act, st, s, pdl_ok);
     case kVarMid:
-      return launch_gemm<MODE, kNtMid, kStagesMid, kUmMid, kKsubMid>(a0, a1, b, b64, offsets, tile_start, E, M_rows,
-                                                   Kdim, out, act, st, s);
+      return launch_gemm<MODE, kNtMid, kStagesMid, kUmMid, kKsubMid>(
+          a0, a1, b, b64, offsets, tile_start, E, M_rows, Kdim, out, res, act, st, s, pdl_ok);
     default:
       return launch_gemm_pair<MODE>(a0, a1, b, b64, offsets, tile_start, E, M_rows, Kdim, out,
-                                    act, st, s);
+                                    res, act, st, s, pdl_ok);
   }
 }
 
@@ -1049,7 +1065,8 @@ size_t expert_scratch_bytes(int64_t S, int E, int F) {
 int expert_ffn_run(const __nv_bfloat16* xs, const int32_t* offsets, int E, int64_t S, int d_e,
                    int F, const __nv_bfloat16* w1, const __nv_bfloat16* w3,
                    const __nv_bfloat16* w2, const moe_act_cfg& act, __nv_bfloat16* y,
-                   void* scratch, DeviceStatus* st, cudaStream_t s, cudaEvent_t after_gate_up) {
+                   void* scratch, DeviceStatus* st, cudaStream_t s, cudaEvent_t after_gate_up,
+                   const __nv_bfloat16* residual) {
   int32_t* tile_start = static_cast<int32_t*>(scratch);
   __nv_bfloat16* h = reinterpret_cast<__nv_bfloat16*>(
       static_cast<uint8_t*>(scratch) + align_up(sizeof(int32_t) * (size_t)(E + 1), 256));
@@ -1064,12 +1081,75 @@ int expert_ffn_run(const __nv_bfloat16* xs, const int32_t* offsets, int E, int64
   k_tiles<<<1, 1024, 0, s>>>(offsets, E, S, nt, tile_start, st);
   if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
   cudaError_t rc = launch_variant<kGateUp>(var, mw1, mw3, mxs, mxs64, offsets, tile_start, E, F,
-                                           d_e, h, act, st, s);
+                                           d_e, h, nullptr, act, st, s);
   if (rc != cudaSuccess) return MOE_ERR_CUDA;
   if (after_gate_up && cudaEventRecord(after_gate_up, s) != cudaSuccess) return MOE_ERR_CUDA;
-  rc = launch_variant<kDown>(var, mw2, mw2, mh, mh64, offsets, tile_start, E, d_e, F, y, act, st,
-                             s);
+  rc = launch_variant<kDown>(var, mw2, mw2, mh, mh64, offsets, tile_start, E, d_e, F, y, residual,
+                             act, st, s);
   return rc == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+// ------------------------------------------------------------ dense layers
+// A dense bias-free Linear (or a shared-expert MLP) is the grouped GEMM with
+// one expert whose segment is every row: offsets = {0, M}, one tile list.
+__global__ void k_dense_tiles(int64_t M, int32_t* __restrict__ tiles) {
+  if (threadIdx.x == 0) {
+    tiles[0] = 0;  // offsets
+    tiles[1] = (int32_t)M;
+    tiles[2] = 0;  // tile_start for each variant's token tile
+    tiles[3] = (int32_t)((M + kNtDecode - 1) / kNtDecode);
+    tiles[4] = 0;
+    tiles[5] = (int32_t)((M + kNtMid - 1) / kNtMid);
+    tiles[6] = 0;
+    tiles[7] = (int32_t)((M + kPairNt - 1) / kPairNt);
+  }
+}
+
+namespace {
+const int32_t* dense_tile_start(const int32_t* tiles, Variant v) {
+  return tiles + 2 + 2 * (int)v;
+}
+}  // namespace
+
+cudaError_t launch_dense_tiles(int64_t M, int32_t* tiles, cudaStream_t s) {
+  k_dense_tiles<<<1, 32, 0, s>>>(M, tiles);
+  return cudaGetLastError();
+}
+
+int linear_run(const __nv_bfloat16* x, int64_t M, int K, const __nv_bfloat16* W, int Nout,
+               const __nv_bfloat16* residual, __nv_bfloat16* y, const int32_t* tiles,
+               DeviceStatus* st, cudaStream_t s, bool pdl_ok) {
+  CUtensorMap mw, mx, mx64;
+  if (!make_map_3d(&mw, W, K, Nout, 1, BM) || !make_map_2d(&mx, x, K, M, kBoxRows) ||
+      !make_map_2d(&mx64, x, K, M, kBigBoxRows))
+    return MOE_ERR_CUDA;
+  const Variant var = pick_variant(M, 1);
+  const moe_act_cfg none = {MOE_ACT_SILU, 1.0f, 0.0f};
+  return launch_variant<kDown>(var, mw, mw, mx, mx64, tiles, dense_tile_start(tiles, var), 1, Nout,
+                               K, y, residual, none, st, s, pdl_ok) == cudaSuccess
+             ? MOE_OK
+             : MOE_ERR_CUDA;
+}
+
+int shared_ffn_run(const __nv_bfloat16* x, int64_t M, int d, int F, const __nv_bfloat16* w1,
+                   const __nv_bfloat16* w3, const __nv_bfloat16* w2, const moe_act_cfg& act,
+                   const __nv_bfloat16* residual, __nv_bfloat16* y, __nv_bfloat16* h,
+                   const int32_t* tiles, DeviceStatus* st, cudaStream_t s) {
+  CUtensorMap mw1, mw3, mw2, mx, mh, mx64, mh64;
+  if (!make_map_3d(&mw1, w1, d, F, 1, kGateUpRows) || !make_map_3d(&mw3, w3, d, F, 1, kGateUpRows) ||
+      !make_map_3d(&mw2, w2, F, d, 1, BM) || !make_map_2d(&mx, x, d, M, kBoxRows) ||
+      !make_map_2d(&mh, h, F, M, kBoxRows) || !make_map_2d(&mx64, x, d, M, kBigBoxRows) ||
+      !make_map_2d(&mh64, h, F, M, kBigBoxRows))
+    return MOE_ERR_CUDA;
+  const Variant var = pick_variant(M, 1);
+  const int32_t* ts = dense_tile_start(tiles, var);
+  if (launch_variant<kGateUp>(var, mw1, mw3, mx, mx64, tiles, ts, 1, F, d, h, nullptr, act, st,
+                              s) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  return launch_variant<kDown>(var, mw2, mw2, mh, mh64, tiles, ts, 1, d, F, y, residual, act, st,
+                               s) == cudaSuccess
+             ? MOE_OK
+             : MOE_ERR_CUDA;
 }
 
 }  // namespace moe

@@ -59,15 +59,42 @@ cudaError_t launch_dispatch(const int32_t* idx, int64_t N, int K, int E, const _
 
 // expert_gemm.cu
 size_t expert_scratch_bytes(int64_t S, int E, int F);
+// residual (optional, [S, d_e] bf16): y = bf16(bf16(x.w2^T) + residual)
 int expert_ffn_run(const __nv_bfloat16* xs, const int32_t* offsets, int E, int64_t S, int d_e,
                    int F, const __nv_bfloat16* w1, const __nv_bfloat16* w3,
                    const __nv_bfloat16* w2, const moe_act_cfg& act, __nv_bfloat16* y,
-                   void* scratch, DeviceStatus* st, cudaStream_t s, cudaEvent_t after_gate_up);
+                   void* scratch, DeviceStatus* st, cudaStream_t s, cudaEvent_t after_gate_up,
+                   const __nv_bfloat16* residual = nullptr);
+// Dense layers on the same kernels (one expert, every row): `tiles` is 8 int32
+// of device memory written by launch_dense_tiles(M) before use.
+constexpr size_t kDenseTilesBytes = 256;
+cudaError_t launch_dense_tiles(int64_t M, int32_t* tiles, cudaStream_t s);
+// y [M, Nout] = bf16(x [M, K] . W [Nout, K]^T) (+ residual [M, Nout]).
+// pdl_ok: the kernel may start as a programmatic dependent of the preceding
+// kernel; allowed only if `tiles` was written before that kernel started.
+int linear_run(const __nv_bfloat16* x, int64_t M, int K, const __nv_bfloat16* W, int Nout,
+               const __nv_bfloat16* residual, __nv_bfloat16* y, const int32_t* tiles,
+               DeviceStatus* st, cudaStream_t s, bool pdl_ok);
+// the gated MLP of one expert on every row of x [M, d]; h: [M, F] bf16 scratch
+// (its down kernel is a programmatic dependent of its gate_up kernel)
+int shared_ffn_run(const __nv_bfloat16* x, int64_t M, int d, int F, const __nv_bfloat16* w1,
+                   const __nv_bfloat16* w3, const __nv_bfloat16* w2, const moe_act_cfg& act,
+                   const __nv_bfloat16* residual, __nv_bfloat16* y, __nv_bfloat16* h,
+                   const int32_t* tiles, DeviceStatus* st, cudaStream_t s);
 
 // combine.cu
+// residual (optional, [N, d_e]): out = bf16(bf16(sum) + residual)
 cudaError_t launch_combine(const __nv_bfloat16* y, const int32_t* pos, const float* w, int64_t N,
                            int K, int d_e, int64_t S, __nv_bfloat16* out, DeviceStatus* st,
-                           cudaStream_t s);
+                           cudaStream_t s, const __nv_bfloat16* residual = nullptr);
+// combine followed by the RMSNorm of each combined row (one warp per token)
+cudaError_t launch_combine_rms_norm(const __nv_bfloat16* y, const int32_t* pos, const float* w,
+                                    int64_t N, int K, int d_e, int64_t S,
+                                    const __nv_bfloat16* norm_w, float eps,
+                                    __nv_bfloat16* out, DeviceStatus* st, cudaStream_t s);
+// out [N, d] = RMSNorm(x) with a bf16 weight
+cudaError_t launch_rms_norm(const __nv_bfloat16* x, int64_t N, int d, const __nv_bfloat16* w,
+                            float eps, __nv_bfloat16* out, cudaStream_t s);
 
 // device properties, read once per device
 struct DevInfo {

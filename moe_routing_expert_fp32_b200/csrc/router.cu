@@ -11,7 +11,8 @@
 //                    terms long and the 32-term blocks are added in double,
 //                    which keeps the logit error near 1e-7 instead of the
 //                    ~1e-5 of one 7168-term fp32 chain.
-//   k_select       : one warp per token: sigmoid, + bias, group top-2 sums,
+//   k_select       : one warp per token: sigmoid (or softmax), + bias, group
+//                    top-2 sums (or group maxima),
 //                    top-TG groups (others -> -inf), top-K experts by
 //                    (score desc, index asc), unbiased weights, renormalise
 //                    (sequential fp32 sum over k + 1e-20), route scale.
@@ -167,12 +168,14 @@ constexpr int kSelWarps = 4;
 
 __global__ void __launch_bounds__(32 * kSelWarps) k_select(
     const float* __restrict__ part, int splits, int64_t N, int E, const float* __restrict__ bias,
-    int G, int TG, int K, int norm, float route_scale, int32_t* __restrict__ idx_out,
-    float* __restrict__ w_out, DeviceStatus* st) {
+    int G, int TG, int K, int norm, float route_scale, int score_func, int group_mode,
+    int32_t* __restrict__ idx_out, float* __restrict__ w_out, DeviceStatus* st) {
   extern __shared__ float sm[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   float* s_s = sm + warp * 2 * E;
   float* s_c = s_s + E;
+  // softmax only: E doubles per warp after the float arrays
+  double* s_x = reinterpret_cast<double*>(sm + kSelWarps * 2 * E) + warp * E;
   const int64_t split_stride = N * (int64_t)E;
   for (int64_t t = (int64_t)blockIdx.x * kSelWarps + warp; t < N;
        t += (int64_t)gridDim.x * kSelWarps) {
@@ -188,11 +191,31 @@ __global__ void __launch_bounds__(32 * kSelWarps) k_select(
       s_s[e] = L;
     }
     __syncwarp();
-    for (int e = lane; e < E; e += 32) {
-      // sigmoid: fp32 rounding of 1/(1+exp(-L)) evaluated in double
-      const float s = (float)(1.0 / (1.0 + exp(-(double)s_s[e])));
-      s_s[e] = s;
-      s_c[e] = bias ? __fadd_rn(s, bias[e]) : s;
+    if (score_func == MOE_SCORE_SOFTMAX) {
+      // softmax over the E logits: exp(L - max) in double, summed in expert
+      // order by one lane, quotient rounded once to fp32
+      float mx = -INFINITY;
+      for (int e = lane; e < E; e += 32) mx = fmaxf(mx, s_s[e]);
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+      for (int e = lane; e < E; e += 32) s_x[e] = exp((double)s_s[e] - (double)mx);
+      __syncwarp();
+      double sum = 0.0;
+      if (lane == 0)
+        for (int e = 0; e < E; ++e) sum += s_x[e];
+      sum = __shfl_sync(0xffffffffu, sum, 0);
+      for (int e = lane; e < E; e += 32) {
+        const float s = (float)(s_x[e] / sum);
+        s_s[e] = s;
+        s_c[e] = bias ? __fadd_rn(s, bias[e]) : s;
+      }
+    } else {
+      for (int e = lane; e < E; e += 32) {
+        // sigmoid: fp32 rounding of 1/(1+exp(-L)) evaluated in double
+        const float s = (float)(1.0 / (1.0 + exp(-(double)s_s[e])));
+        s_s[e] = s;
+        s_c[e] = bias ? __fadd_rn(s, bias[e]) : s;
+      }
     }
     __syncwarp();
     if (G > 1) {
@@ -205,7 +228,7 @@ __global__ void __launch_bounds__(32 * kSelWarps) k_select(
           if (v > a) { b = a; a = v; }
           else if (v > b) { b = v; }
         }
-        gs = __fadd_rn(a, b);
+        gs = group_mode == MOE_GROUP_MAX ? a : __fadd_rn(a, b);
       }
       bool kept = false;
       for (int r = 0; r < TG; ++r) {
@@ -308,13 +331,25 @@ cudaError_t launch_select(const float* part, int splits, int64_t N, const float*
                           const moe_route_cfg& cfg, int32_t* idx, float* w, DeviceStatus* st,
                           cudaStream_t s) {
   const int E = cfg.num_experts;
-  const size_t smem = sizeof(float) * 2 * E * kSelWarps;
+  const bool softmax = cfg.score_func == MOE_SCORE_SOFTMAX;
+  const size_t smem = sizeof(float) * 2 * E * kSelWarps + (softmax ? sizeof(double) * E * kSelWarps : 0);
+  if (softmax && smem > 48 * 1024) {
+    static bool attr_set[64] = {false};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 64 && !attr_set[dev]) {
+      const cudaError_t e =
+          cudaFuncSetAttribute(k_select, cudaFuncAttributeMaxDynamicSharedMemorySize, 64 * 1024);
+      if (e != cudaSuccess) return e;
+      attr_set[dev] = true;
+    }
+  }
   int64_t blocks = (N + kSelWarps - 1) / kSelWarps;
   const int64_t cap = (int64_t)dev_info()->sm_count * 16;
   if (blocks > cap) blocks = cap;
   k_select<<<(unsigned)blocks, 32 * kSelWarps, smem, s>>>(
       part, splits, N, E, bias, cfg.n_group, cfg.topk_group, cfg.top_k, cfg.norm_topk_prob,
-      cfg.route_scale, idx, w, st);
+      cfg.route_scale, cfg.score_func, cfg.group_score, idx, w, st);
   return cudaGetLastError();
 }
 

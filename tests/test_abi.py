@@ -78,6 +78,27 @@ def test_route_rejects_before_cuda(L):
     assert L.moe_route(None, 4, 256, None, None, ctypes.byref(c), None, None, None, 0, None) == -1
 
 
+@pytest.mark.parametrize("field,value,code", [
+    ("score_func", 1, -4), ("group_score", 1, -4),    # valid variants: NULL workspace next
+    ("score_func", 2, -1), ("score_func", -1, -1), ("group_score", 2, -1),
+])
+def test_route_variant_validation(L, field, value, code):
+    import moe_routing_expert_fp32_b200 as m
+    c = _cfg(m)
+    setattr(c, field, value)
+    assert L.moe_route(None, 0, 256, None, None, ctypes.byref(c), None, None, None, 0, None) == code
+    assert L.moe_route_from_logits(None, 0, None, ctypes.byref(c), None, None, None, 0,
+                                   None) == code
+
+
+def test_route_config_binding_defaults():
+    import moe_routing_expert_fp32_b200 as m
+    c = m.RouteConfig(16, 4, 2, 4, 2.5)._c()
+    assert (c.score_func, c.group_score, c.norm_topk_prob) == (0, 0, 1)
+    c = m.RouteConfig(16, 4, 2, 4, 2.5, False, score_func="softmax", group_score="max")._c()
+    assert (c.score_func, c.group_score, c.norm_topk_prob) == (1, 1, 0)
+
+
 def test_workspace_checks(L):
     import moe_routing_expert_fp32_b200 as m
     c = _cfg(m)
@@ -145,3 +166,67 @@ def test_strerror(L):
     for code in range(-8, 1):
         assert L.moe_strerror(code)
     assert L.moe_strerror(-99) == b"unknown moe_status"
+
+
+def _block_args(m, d_r=256, d_e=128, F=128, F_sh=256, latent=True, shared=True, norm=True):
+    dims = m._BlockDims(d_r, d_e, F, F_sh if shared else 0, 1e-6)
+    p = ctypes.c_void_p(256)  # never dereferenced: validation only
+    w = m._BlockWeights(p, None, p if latent else None, p if (latent and norm) else None,
+                        p if latent else None, p, p, p, p if shared else None,
+                        p if shared else None, p if shared else None)
+    return dims, w
+
+
+@pytest.mark.parametrize("kw,ok", [
+    ({}, True),
+    ({"shared": False}, True),
+    ({"norm": False}, True),
+    ({"latent": False, "d_e": 256, "norm": False}, True),
+    ({"latent": False, "d_e": 128, "norm": False}, False),   # d_e != d_r without projections
+    ({"d_r": 200}, False),                                    # d_r not a multiple of 128
+    ({"F_sh": 100}, False),
+    ({"d_e": 16384, "d_r": 16384}, False),                    # latent width above 8192
+])
+def test_block_workspace_validation(L, kw, ok):
+    import moe_routing_expert_fp32_b200 as m
+    dims, w = _block_args(m, **kw)
+    c = _cfg(m)
+    need = L.moe_block_workspace_size(64, ctypes.byref(dims), ctypes.byref(w), ctypes.byref(c))
+    assert (need > 0) == ok
+
+
+def test_block_rejects_inconsistent_parts(L):
+    import moe_routing_expert_fp32_b200 as m
+    c = _cfg(m)
+    a = m._ActCfg(0, 1.0, 0.0)
+    dims, w = _block_args(m)
+    w.up_proj = None                       # down_proj without up_proj
+    assert L.moe_block_forward(None, 0, ctypes.byref(dims), ctypes.byref(w), ctypes.byref(c),
+                               ctypes.byref(a), None, None, None, None, 0, None) == -1
+    dims, w = _block_args(m)
+    w.shared_w2 = None                     # a partial shared expert
+    assert L.moe_block_forward(None, 0, ctypes.byref(dims), ctypes.byref(w), ctypes.byref(c),
+                               ctypes.byref(a), None, None, None, None, 0, None) == -1
+    dims, w = _block_args(m)
+    dims.norm_eps = float("nan")
+    assert L.moe_block_forward(None, 0, ctypes.byref(dims), ctypes.byref(w), ctypes.byref(c),
+                               ctypes.byref(a), None, None, None, None, 0, None) == -1
+    dims, w = _block_args(m)               # valid: fails on the NULL workspace only
+    assert L.moe_block_forward(None, 0, ctypes.byref(dims), ctypes.byref(w), ctypes.byref(c),
+                               ctypes.byref(a), None, None, None, None, 0, None) == -4
+
+
+def test_linear_and_norm_validation(L):
+    assert L.moe_linear_workspace_size() >= 256
+    # K and N_out must be multiples of 128
+    assert L.moe_linear(None, 0, 100, ctypes.c_void_p(256), 128, None, None, None, 0, None) == -2
+    assert L.moe_linear(None, 0, 128, None, 128, None, None, None, 0, None) == -1
+    assert L.moe_linear(None, 0, 128, ctypes.c_void_p(258), 128, None, None, None, 0, None) == -3
+    assert L.moe_linear(None, 0, 128, ctypes.c_void_p(256), 128, None, None, None, 0, None) == -4
+    # RMSNorm: negative or NaN eps, widths
+    w = ctypes.c_void_p(256)
+    assert L.moe_rms_norm(None, 0, 128, w, -1.0, None, None) == -1
+    assert L.moe_rms_norm(None, 0, 128, w, float("nan"), None, None) == -1
+    assert L.moe_rms_norm(None, 0, 100, w, 1e-6, None, None) == -2
+    assert L.moe_rms_norm(None, 0, 16384, w, 1e-6, None, None) == -2
+    assert L.moe_rms_norm(None, 4, 128, w, 1e-6, None, None) == -1

@@ -91,6 +91,36 @@ def test_route_from_logits_shapes(moe, E, G, TG, K, norm):
     assert np.array_equal(w_g.cpu().numpy().view(np.uint32), w_r.view(np.uint32))
 
 
+_SCORE = {"sigmoid": oracle.SCORE_SIGMOID, "softmax": oracle.SCORE_SOFTMAX}
+_GROUP = {"top2_sum": oracle.GROUP_TOP2_SUM, "max": oracle.GROUP_MAX}
+
+
+@pytest.mark.parametrize("score,group", [("softmax", "top2_sum"), ("sigmoid", "max"),
+                                         ("softmax", "max")])
+@pytest.mark.parametrize("E,G,TG,K,norm", [(256, 8, 4, 8, False), (256, 8, 4, 8, True),
+                                           (1024, 32, 3, 16, True), (896, 1, 1, 8, True),
+                                           (16, 4, 2, 4, False), (6, 1, 1, 6, True)])
+def test_route_variants_bit_exact(moe, score, group, E, G, TG, K, norm):
+    """Softmax scoring and group-max scores: indices and weights bit-exact from
+    the same logits, with and without bias, ties included."""
+    import torch
+    rng = np.random.default_rng(E * 1000 + K + 7 * len(score + group))
+    N = 777
+    L = rng.choice(np.array([-0.5, 0.0, 0.5, 1.0], np.float32), size=(N, E))
+    L[: N // 2] = (rng.standard_normal((N // 2, E)) * 2).astype(np.float32)
+    L[: 8] += np.float32(300.0)  # large logits: softmax must subtract the row maximum
+    b = rng.choice(np.array([0.0, 0.001, -0.001], np.float32), size=E)
+    cfg = moe.RouteConfig(E, G, TG, K, 2.0, norm, score_func=score, group_score=group)
+    for bias in (b, None):
+        idx_r, w_r, _ = oracle.route_from_logits(L, bias, G, TG, K, 2.0, norm, score=_SCORE[score],
+                                                 group=_GROUP[group])
+        idx_g, w_g = moe.route_from_logits(torch.from_numpy(L).cuda(),
+                                           None if bias is None else torch.from_numpy(bias).cuda(),
+                                           cfg)
+        assert np.array_equal(idx_g.cpu().numpy(), idx_r)
+        assert np.array_equal(w_g.cpu().numpy().view(np.uint32), w_r.view(np.uint32))
+
+
 # ----------------------------------------------------------- routing end to end
 def _check_routing(idx_g, w_g, idx_r, w_r, margin):
     ok = margin > MARGIN
@@ -120,6 +150,22 @@ def test_route_end_to_end(moe, name):
                                       wl.route_scale, wl.norm)
     n_low = _check_routing(idx_g[rows], w_g[rows], idx_r, w_r, margin)
     print(f"{name}: {len(rows)} tokens checked, {n_low} at or below the margin")
+
+
+@pytest.mark.parametrize("score,group", [("softmax", "max"), ("sigmoid", "max")])
+def test_route_variants_end_to_end(moe, score, group):
+    """The gate GEMM followed by a variant selection, at the 256-expert decode shape."""
+    import torch
+    wl = WORKLOADS["dsv32_decode"]
+    inp = host_inputs(wl)
+    x, W = inp["x"], inp["W"]
+    cfg = moe.RouteConfig(wl.E, wl.G, wl.TG, wl.K, wl.route_scale, score == "sigmoid",
+                          score_func=score, group_score=group)
+    idx_g, w_g = moe.route(dev_bf16(x), torch.from_numpy(W).cuda(), None, cfg)
+    idx_r, w_r, margin = oracle.route(x, W, None, wl.G, wl.TG, wl.K, wl.route_scale,
+                                      score == "sigmoid", score=_SCORE[score], group=_GROUP[group])
+    n_low = _check_routing(idx_g.cpu().numpy(), w_g.cpu().numpy(), idx_r, w_r, margin)
+    print(f"{score}/{group}: {wl.N} tokens checked, {n_low} at or below the margin")
 
 
 # ------------------------------------------------------------------ dispatch
