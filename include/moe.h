@@ -228,6 +228,42 @@ MOE_API size_t moe_combine_workspace_size(void);
 MOE_API int moe_combine(const moe_bf16* y, const int32_t* pos, const float* topk_w, int64_t N,
                         int K, int d_e, moe_bf16* out, void* ws, size_t ws_bytes, void* stream);
 
+/* moe_expert_ffn with the gather inside the w1/w3 kernel: row j of segment
+ * e is x_e[perm[j] / K] (perm and offsets as moe_dispatch writes them), read
+ * by tile::gather4 TMA loads, so no S x d_e copy of the tokens is made.
+ * x_e [N, d_e] bf16.  Decode and mid-size batches only (S <= 128 * E, else
+ * MOE_ERR_UNSUPPORTED).  It saves the copy's memory, not time: on a B200 the
+ * separate token-major gather plus tiled loads is faster (the layer,
+ * moe_forward, uses that).  Workspace as moe_expert_ffn. */
+MOE_API int moe_expert_ffn_gathered(const moe_bf16* x_e, int64_t N, int K, const int32_t* perm,
+                                    const int32_t* offsets, int E, int d_e, int F,
+                                    const moe_bf16* w1, const moe_bf16* w3, const moe_bf16* w2,
+                                    const moe_act_cfg* act, moe_bf16* y, void* ws,
+                                    size_t ws_bytes, void* stream);
+
+/* ------------------------------------------- expert parallelism, receive side
+ *
+ * With the experts split over P ranks (rank q holds experts q*E_local ..
+ * q*E_local + E_local - 1, "Kimi K3 · Add shared output", moe-forward excerpt:
+ * self.experts[i + self.ep_rank * self.experts_per_rank]), a rank's rows
+ * sorted by moe_dispatch are already grouped by destination rank, so one
+ * all-to-all sends each rank its slice; the rows a rank receives arrive
+ * grouped by source rank and, within a source, sorted by local expert.
+ * moe_ep_expert_ffn runs the local experts' MLP on them in that order:
+ *   xr [R, d_e] bf16       the received rows, R = sum of recv_counts;
+ *   recv_counts [P, E_local] int32 (device): rows source p sent for local
+ *                          expert e, the segment (p, e) of xr;
+ *   w1, w3 [E_local, F, d_e], w2 [E_local, d_e, F]: this rank's experts;
+ *   y [R, d_e] bf16        the outputs, in xr's order (to be sent back).
+ * P * E_local <= 1024.  Counts that do not add up to R are reported in the
+ * status word (MOE_ERR_DEVICE_BOUNDS) and no row is read out of range.
+ * Workspace: moe_ep_expert_ffn_workspace_size(R, d_e, P, E_local, F). */
+MOE_API size_t moe_ep_expert_ffn_workspace_size(int64_t R, int d_e, int P, int E_local, int F);
+MOE_API int moe_ep_expert_ffn(const moe_bf16* xr, int64_t R, const int32_t* recv_counts, int P,
+                              int E_local, int d_e, int F, const moe_bf16* w1,
+                              const moe_bf16* w3, const moe_bf16* w2, const moe_act_cfg* act,
+                              moe_bf16* y, void* ws, size_t ws_bytes, void* stream);
+
 /* ------------------------------------------------------------ whole layer */
 
 MOE_API size_t moe_workspace_size(int64_t N, int d_r, int d_e, const moe_route_cfg* cfg, int F);
@@ -274,11 +310,23 @@ MOE_API int moe_forward(const moe_bf16* x_r, const moe_bf16* x_e, int64_t N, int
  * residual[m, n] ).  x [M, K], W [N_out, K] (nn.Linear layout), residual and
  * y [M, N_out]: bf16, row-major, device memory, 16-byte aligned.  K and N_out
  * multiples of 128.  y may be the residual buffer; it must not overlap x or
- * W.  Workspace: moe_linear_workspace_size() bytes. */
-MOE_API size_t moe_linear_workspace_size(void);
+ * W.  Workspace: moe_linear_workspace_size(M, K, N_out) bytes (it holds the
+ * split-K partial sums of small M; 0 for invalid shapes). */
+MOE_API size_t moe_linear_workspace_size(int64_t M, int K, int N_out);
 MOE_API int moe_linear(const moe_bf16* x, int64_t M, int K, const moe_bf16* W, int N_out,
                        const moe_bf16* residual, moe_bf16* y, void* ws, size_t ws_bytes,
                        void* stream);
+
+/* The shared experts alone: one gated MLP (the routed experts' kind) on every
+ * row, y = bf16( h . w2^T ) with h = act(bf16(x . w1^T), bf16(x . w3^T)), and
+ * with a residual y = bf16( bf16(...) + residual ).  x and residual/y
+ * [M, d], w1 and w3 [F, d], w2 [d, F], bf16; d and F multiples of 128.
+ * Workspace: moe_shared_experts_workspace_size(M, d, F) bytes. */
+MOE_API size_t moe_shared_experts_workspace_size(int64_t M, int d, int F);
+MOE_API int moe_shared_experts(const moe_bf16* x, int64_t M, int d, int F, const moe_bf16* w1,
+                               const moe_bf16* w3, const moe_bf16* w2, const moe_act_cfg* act,
+                               const moe_bf16* residual, moe_bf16* y, void* ws,
+                               size_t ws_bytes, void* stream);
 
 /* RMSNorm of each row of x [N, d] (the reading of routed_expert_norm):
  *   r = 1 / sqrt(mean(x^2) + eps)   (double)

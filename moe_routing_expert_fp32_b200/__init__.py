@@ -122,7 +122,8 @@ EXPORTS = ("moe_route_workspace_size", "moe_route", "moe_route_from_logits",
            "moe_expert_ffn", "moe_combine_workspace_size", "moe_combine", "moe_workspace_size",
            "moe_forward", "moe_get_status", "moe_strerror", "moe_dispatch_static",
            "moe_linear_workspace_size", "moe_linear", "moe_rms_norm", "moe_block_workspace_size",
-           "moe_block_forward")
+           "moe_block_forward", "moe_shared_experts_workspace_size", "moe_shared_experts",
+           "moe_ep_expert_ffn_workspace_size", "moe_ep_expert_ffn", "moe_expert_ffn_gathered")
 
 
 def lib() -> ctypes.CDLL:
@@ -155,9 +156,16 @@ def lib() -> ctypes.CDLL:
         "moe_get_status": ([vp, vp], i32),
         "moe_dispatch_static": ([vp, i64, i32, i32, vp, i32, vp, vp, vp, vp, vp, vp], i32),
         "moe_strerror": ([i32], ctypes.c_char_p),
-        "moe_linear_workspace_size": ([], sz),
+        "moe_linear_workspace_size": ([i64, i32, i32], sz),
         "moe_linear": ([vp, i64, i32, vp, i32, vp, vp, vp, sz, vp], i32),
         "moe_rms_norm": ([vp, i64, i32, vp, ctypes.c_float, vp, vp], i32),
+        "moe_shared_experts_workspace_size": ([i64, i32, i32], sz),
+        "moe_ep_expert_ffn_workspace_size": ([i64, i32, i32, i32, i32], sz),
+        "moe_expert_ffn_gathered": ([vp, i64, i32, vp, vp, i32, i32, i32, vp, vp, vp, ac, vp, vp,
+                                     sz, vp], i32),
+        "moe_ep_expert_ffn": ([vp, i64, vp, i32, i32, i32, i32, vp, vp, vp, ac, vp, vp, sz, vp],
+                              i32),
+        "moe_shared_experts": ([vp, i64, i32, i32, vp, vp, vp, ac, vp, vp, vp, sz, vp], i32),
         "moe_block_workspace_size": ([i64, bd, bw, rc], sz),
         "moe_block_forward": ([vp, i64, bd, bw, rc, ac, vp, vp, vp, vp, sz, vp], i32),
     }
@@ -396,10 +404,83 @@ def linear(x, W, residual=None, out=None, ws=None):
     _need(W, torch.bfloat16, (N_out, K), "W")
     if residual is not None:
         _need(residual, torch.bfloat16, (M, N_out), "residual")
-    ws = workspace(lib().moe_linear_workspace_size(), x.device) if ws is None else ws
+    need = lib().moe_linear_workspace_size(M, K, N_out)
+    if need == 0:
+        raise MoeError("moe_linear_workspace_size", -1)
+    ws = workspace(need, x.device) if ws is None else ws
     out = torch.empty((M, N_out), dtype=torch.bfloat16, device=x.device) if out is None else out
     _check("moe_linear", lib().moe_linear(_ptr(x), M, K, _ptr(W), N_out, _ptr(residual),
                                           _ptr(out), _ptr(ws), ws.numel(), _stream()))
+    return out
+
+
+def expert_ffn_gathered(x_e, K, perm, offsets, w1, w3, w2, act: ActConfig, ws=None, y=None):
+    """moe_expert_ffn_gathered: the expert MLP on the rows x_e[perm // K]
+    without a gathered copy (decode and mid-size batches)."""
+    torch = _torch()
+    N, d_e = x_e.shape
+    E, F, _ = w1.shape
+    S = N * K
+    _need(x_e, torch.bfloat16, name="x_e")
+    _need(perm, torch.int32, (S,), "perm")
+    _need(offsets, torch.int32, (E + 1,), "offsets")
+    need = lib().moe_expert_ffn_workspace_size(S, d_e, E, F)
+    ws = workspace(need, x_e.device) if ws is None else ws
+    y = torch.empty((S, d_e), dtype=torch.bfloat16, device=x_e.device) if y is None else y
+    a = act._c()
+    _check("moe_expert_ffn_gathered",
+           lib().moe_expert_ffn_gathered(_ptr(x_e), N, K, _ptr(perm), _ptr(offsets), E, d_e, F,
+                                         _ptr(w1), _ptr(w3), _ptr(w2), ctypes.byref(a), _ptr(y),
+                                         _ptr(ws), ws.numel(), _stream()))
+    return y
+
+
+def ep_expert_ffn(xr, recv_counts, w1, w3, w2, act: ActConfig, y=None, ws=None):
+    """The local experts on rows received from P ranks (moe_ep_expert_ffn):
+    xr [R, d_e] grouped by source rank, then local expert; recv_counts
+    [P, E_local] int32 on the device; w1, w3 [E_local, F, d_e], w2
+    [E_local, d_e, F]."""
+    torch = _torch()
+    R, d_e = xr.shape
+    P, E_local = recv_counts.shape
+    F = w1.shape[1]
+    _need(xr, torch.bfloat16, name="xr")
+    _need(recv_counts, torch.int32, (P, E_local), "recv_counts")
+    _need(w1, torch.bfloat16, (E_local, F, d_e), "w1")
+    _need(w3, torch.bfloat16, (E_local, F, d_e), "w3")
+    _need(w2, torch.bfloat16, (E_local, d_e, F), "w2")
+    need = lib().moe_ep_expert_ffn_workspace_size(R, d_e, P, E_local, F)
+    ws = workspace(need, xr.device) if ws is None else ws
+    y = torch.empty((R, d_e), dtype=torch.bfloat16, device=xr.device) if y is None else y
+    a = act._c()
+    _check("moe_ep_expert_ffn",
+           lib().moe_ep_expert_ffn(_ptr(xr), R, _ptr(recv_counts), P, E_local, d_e, F, _ptr(w1),
+                                   _ptr(w3), _ptr(w2), ctypes.byref(a), _ptr(y), _ptr(ws),
+                                   ws.numel(), _stream()))
+    return y
+
+
+def shared_experts(x, w1, w3, w2, act: ActConfig, residual=None, out=None, ws=None):
+    """The shared experts' gated MLP on every row (moe_shared_experts)."""
+    torch = _torch()
+    M, d = x.shape
+    F = w1.shape[0]
+    _need(x, torch.bfloat16, name="x")
+    _need(w1, torch.bfloat16, (F, d), "w1")
+    _need(w3, torch.bfloat16, (F, d), "w3")
+    _need(w2, torch.bfloat16, (d, F), "w2")
+    if residual is not None:
+        _need(residual, torch.bfloat16, (M, d), "residual")
+    need = lib().moe_shared_experts_workspace_size(M, d, F)
+    if need == 0:
+        raise MoeError("moe_shared_experts_workspace_size", -1)
+    ws = workspace(need, x.device) if ws is None else ws
+    out = torch.empty((M, d), dtype=torch.bfloat16, device=x.device) if out is None else out
+    a = act._c()
+    _check("moe_shared_experts",
+           lib().moe_shared_experts(_ptr(x), M, d, F, _ptr(w1), _ptr(w3), _ptr(w2),
+                                    ctypes.byref(a), _ptr(residual), _ptr(out), _ptr(ws),
+                                    ws.numel(), _stream()))
     return out
 
 

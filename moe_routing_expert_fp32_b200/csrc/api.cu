@@ -264,6 +264,76 @@ int moe_expert_ffn(const moe_bf16* xs, const int32_t* offsets, int E, int64_t S,
                         nullptr);
 }
 
+// The expert MLP reading its token rows straight from x_e through perm (the
+// gather inside the w1/w3 kernel): no S x d_e copy of the tokens.
+int moe_expert_ffn_gathered(const moe_bf16* x_e, int64_t N, int K, const int32_t* perm,
+                            const int32_t* offsets, int E, int d_e, int F, const moe_bf16* w1,
+                            const moe_bf16* w3, const moe_bf16* w2, const moe_act_cfg* act,
+                            moe_bf16* y, void* ws, size_t ws_bytes, void* stream) {
+  if (N < 0 || K < 1) return MOE_ERR_INVALID_ARG;
+  const int64_t S = N * (int64_t)K;
+  int rc = check_expert_shape(S, d_e, E, F);
+  if (rc) return rc;
+  if ((rc = check_act(act))) return rc;
+  if (!expert_gather_fusable(S, E)) return MOE_ERR_UNSUPPORTED;
+  if (!offsets || !w1 || !w3 || !w2) return MOE_ERR_INVALID_ARG;
+  if (S > 0 && (!x_e || !perm || !y)) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(w1) || !aligned16(w3) || !aligned16(w2)) return MOE_ERR_ALIGNMENT;
+  if (S > 0 && (!aligned16(x_e) || !aligned16(y))) return MOE_ERR_ALIGNMENT;
+  if ((rc = check_ws(ws, ws_bytes, moe_expert_ffn_workspace_size(S, d_e, E, F)))) return rc;
+  if ((rc = check_device())) return rc;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if ((rc = reset_status(ws, s))) return rc;
+  if (S == 0) return MOE_OK;
+  const GatherSrc g{reinterpret_cast<const __nv_bfloat16*>(x_e), perm, N, K};
+  return expert_ffn_run(nullptr, offsets, E, S, d_e, F, reinterpret_cast<const __nv_bfloat16*>(w1),
+                        reinterpret_cast<const __nv_bfloat16*>(w3),
+                        reinterpret_cast<const __nv_bfloat16*>(w2), *act,
+                        reinterpret_cast<__nv_bfloat16*>(y), body_of(ws), status_of(ws), s,
+                        nullptr, nullptr, &g);
+}
+
+// ------------------------------------------------ expert parallel receive side
+size_t moe_ep_expert_ffn_workspace_size(int64_t R, int d_e, int P, int E_local, int F) {
+  if (R < 0 || d_e <= 0 || P < 1 || E_local < 1 || F <= 0) return 0;
+  const int n = P * E_local;
+  return kStatusBytes + align_up(sizeof(int32_t) * (size_t)(n + 1), 256) +
+         expert_scratch_bytes(R, n, F);
+}
+
+int moe_ep_expert_ffn(const moe_bf16* xr, int64_t R, const int32_t* recv_counts, int P,
+                      int E_local, int d_e, int F, const moe_bf16* w1, const moe_bf16* w3,
+                      const moe_bf16* w2, const moe_act_cfg* act, moe_bf16* y, void* ws,
+                      size_t ws_bytes, void* stream) {
+  if (P < 1 || E_local < 1 || !recv_counts) return MOE_ERR_INVALID_ARG;
+  if ((int64_t)P * E_local > 1024) return MOE_ERR_UNSUPPORTED;
+  const int n = P * E_local;
+  int rc = check_expert_shape(R, d_e, n, F);
+  if (rc) return rc;
+  if ((rc = check_act(act))) return rc;
+  if (!w1 || !w3 || !w2) return MOE_ERR_INVALID_ARG;
+  if (R > 0 && (!xr || !y)) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(w1) || !aligned16(w3) || !aligned16(w2)) return MOE_ERR_ALIGNMENT;
+  if (R > 0 && (!aligned16(xr) || !aligned16(y))) return MOE_ERR_ALIGNMENT;
+  if ((rc = check_ws(ws, ws_bytes, moe_ep_expert_ffn_workspace_size(R, d_e, P, E_local, F))))
+    return rc;
+  if ((rc = check_device())) return rc;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if ((rc = reset_status(ws, s))) return rc;
+  if (R == 0) return MOE_OK;
+  uint8_t* body = body_of(ws);
+  int32_t* offsets = reinterpret_cast<int32_t*>(body);
+  uint8_t* scratch = body + align_up(sizeof(int32_t) * (size_t)(n + 1), 256);
+  if (launch_counts_offsets(recv_counts, n, offsets, status_of(ws), s) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  return expert_ffn_run(reinterpret_cast<const __nv_bfloat16*>(xr), offsets, n, R, d_e, F,
+                        reinterpret_cast<const __nv_bfloat16*>(w1),
+                        reinterpret_cast<const __nv_bfloat16*>(w3),
+                        reinterpret_cast<const __nv_bfloat16*>(w2), *act,
+                        reinterpret_cast<__nv_bfloat16*>(y), scratch, status_of(ws), s, nullptr,
+                        nullptr, nullptr, E_local);
+}
+
 // ----------------------------------------------------------------- combine
 size_t moe_combine_workspace_size(void) { return kStatusBytes; }
 
@@ -389,7 +459,10 @@ int moe_forward(const moe_bf16* x_r, const moe_bf16* x_e, int64_t N, int d_r, in
 }
 
 // ------------------------------------------------------------ dense layers
-size_t moe_linear_workspace_size(void) { return kStatusBytes + kDenseTilesBytes; }
+size_t moe_linear_workspace_size(int64_t M, int K, int N_out) {
+  if (M < 0 || K <= 0 || N_out <= 0 || K % 128 != 0 || N_out % 128 != 0) return 0;
+  return kStatusBytes + kDenseTilesBytes + dense_part_bytes(M, K, N_out, false);
+}
 
 int moe_linear(const moe_bf16* x, int64_t M, int K, const moe_bf16* W, int N_out,
                const moe_bf16* residual, moe_bf16* y, void* ws, size_t ws_bytes, void* stream) {
@@ -401,18 +474,62 @@ int moe_linear(const moe_bf16* x, int64_t M, int K, const moe_bf16* W, int N_out
   if (M > 0 && (!aligned16(x) || !aligned16(y) || (residual && !aligned16(residual))))
     return MOE_ERR_ALIGNMENT;
   int rc;
-  if ((rc = check_ws(ws, ws_bytes, moe_linear_workspace_size()))) return rc;
+  if ((rc = check_ws(ws, ws_bytes, moe_linear_workspace_size(M, K, N_out)))) return rc;
   if ((rc = check_device())) return rc;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if ((rc = reset_status(ws, s))) return rc;
   if (M == 0) return MOE_OK;
   int32_t* tiles = reinterpret_cast<int32_t*>(body_of(ws));
+  float* part = dense_part_bytes(M, K, N_out, false)
+                    ? reinterpret_cast<float*>(body_of(ws) + kDenseTilesBytes)
+                    : nullptr;
   if (launch_dense_tiles(M, tiles, s) != cudaSuccess) return MOE_ERR_CUDA;
   return linear_run(reinterpret_cast<const __nv_bfloat16*>(x), M, K,
                     reinterpret_cast<const __nv_bfloat16*>(W), N_out,
                     reinterpret_cast<const __nv_bfloat16*>(residual),
                     reinterpret_cast<__nv_bfloat16*>(y), tiles, status_of(ws), s,
-                    /*pdl_ok=*/false);  // the tile list was written by the kernel just before
+                    /*pdl_ok=*/false, part);  // the tile list was written just before
+}
+
+size_t moe_shared_experts_workspace_size(int64_t M, int d, int F) {
+  if (M < 0 || d <= 0 || F <= 0 || d % 128 != 0 || F % 128 != 0) return 0;
+  const size_t p1 = dense_part_bytes(M, d, F, true), p2 = dense_part_bytes(M, F, d, false);
+  return kStatusBytes + kDenseTilesBytes +
+         align_up(sizeof(__nv_bfloat16) * (size_t)M * (size_t)F, 256) + (p1 > p2 ? p1 : p2);
+}
+
+int moe_shared_experts(const moe_bf16* x, int64_t M, int d, int F, const moe_bf16* w1,
+                       const moe_bf16* w3, const moe_bf16* w2, const moe_act_cfg* act,
+                       const moe_bf16* residual, moe_bf16* y, void* ws, size_t ws_bytes,
+                       void* stream) {
+  if (M < 0 || d <= 0 || F <= 0) return MOE_ERR_INVALID_ARG;
+  if (d % 128 != 0 || F % 128 != 0 || M > INT32_MAX) return MOE_ERR_UNSUPPORTED;
+  int rc;
+  if ((rc = check_act(act))) return rc;
+  if (!w1 || !w3 || !w2) return MOE_ERR_INVALID_ARG;
+  if (M > 0 && (!x || !y)) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(w1) || !aligned16(w3) || !aligned16(w2)) return MOE_ERR_ALIGNMENT;
+  if (M > 0 && (!aligned16(x) || !aligned16(y) || (residual && !aligned16(residual))))
+    return MOE_ERR_ALIGNMENT;
+  if ((rc = check_ws(ws, ws_bytes, moe_shared_experts_workspace_size(M, d, F)))) return rc;
+  if ((rc = check_device())) return rc;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if ((rc = reset_status(ws, s))) return rc;
+  if (M == 0) return MOE_OK;
+  uint8_t* body = body_of(ws);
+  int32_t* tiles = reinterpret_cast<int32_t*>(body);
+  __nv_bfloat16* h = reinterpret_cast<__nv_bfloat16*>(body + kDenseTilesBytes);
+  const size_t hb = align_up(sizeof(__nv_bfloat16) * (size_t)M * (size_t)F, 256);
+  float* part = reinterpret_cast<float*>(body + kDenseTilesBytes + hb);
+  const size_t p1 = dense_part_bytes(M, d, F, true), p2 = dense_part_bytes(M, F, d, false);
+  if (launch_dense_tiles(M, tiles, s) != cudaSuccess) return MOE_ERR_CUDA;
+  return shared_ffn_run(reinterpret_cast<const __nv_bfloat16*>(x), M, d, F,
+                        reinterpret_cast<const __nv_bfloat16*>(w1),
+                        reinterpret_cast<const __nv_bfloat16*>(w3),
+                        reinterpret_cast<const __nv_bfloat16*>(w2), *act,
+                        reinterpret_cast<const __nv_bfloat16*>(residual),
+                        reinterpret_cast<__nv_bfloat16*>(y), h, tiles, status_of(ws), s,
+                        (p1 || p2) ? part : nullptr);
 }
 
 int moe_rms_norm(const moe_bf16* x, int64_t N, int d, const moe_bf16* weight, float eps,
@@ -438,7 +555,7 @@ int moe_rms_norm(const moe_bf16* x, int64_t N, int d, const moe_bf16* weight, fl
 namespace {
 struct BlockLayout {
   ForwardLayout fwd;     // the routed layer's regions (status word at 0)
-  size_t tiles, xe, yc, sh, hsh, total;
+  size_t tiles, xe, yc, sh, hsh, part, part_bytes, total;
 };
 
 BlockLayout block_layout(int64_t N, const moe_block_dims& d, const moe_route_cfg& c,
@@ -452,10 +569,20 @@ BlockLayout block_layout(int64_t N, const moe_block_dims& d, const moe_route_cfg
     L.xe = o; o += align_up(ne, 256);
     L.yc = o; o += align_up(ne, 256);
   }
+  size_t pb = 0;
+  auto upd = [&](size_t b) { pb = b > pb ? b : pb; };
+  if (latent) {
+    upd(dense_part_bytes(N, d.d_r, d.d_e, false));
+    upd(dense_part_bytes(N, d.d_e, d.d_r, false));
+  }
   if (shared) {
     L.sh = o; o += align_up(sizeof(__nv_bfloat16) * (size_t)N * (size_t)d.d_r, 256);
     L.hsh = o; o += align_up(sizeof(__nv_bfloat16) * (size_t)N * (size_t)d.F_shared, 256);
+    upd(dense_part_bytes(N, d.d_r, d.F_shared, true));
+    upd(dense_part_bytes(N, d.F_shared, d.d_r, false));
   }
+  L.part = o; o += pb;
+  L.part_bytes = pb;
   L.total = o;
   return L;
 }
@@ -526,6 +653,7 @@ int moe_block_forward(const moe_bf16* x, int64_t N, const moe_block_dims* dims,
   const __nv_bfloat16* xr = cbf(x);
   __nv_bfloat16* sh = shared ? bf(L.sh) : nullptr;
   __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(out);
+  float* part = L.part_bytes ? reinterpret_cast<float*>(base + L.part) : nullptr;
 
   if (launch_dense_tiles(N, tiles, s) != cudaSuccess) return MOE_ERR_CUDA;
   // gate on the full-width input
@@ -535,7 +663,7 @@ int moe_block_forward(const moe_bf16* x, int64_t N, const moe_block_dims* dims,
   // the last step)
   if (shared && (rc = shared_ffn_run(xr, N, d_r, dims->F_shared, cbf(wt->shared_w1),
                                      cbf(wt->shared_w3), cbf(wt->shared_w2), *act, nullptr, sh,
-                                     bf(L.hsh), tiles, st, s)))
+                                     bf(L.hsh), tiles, st, s, part)))
     return rc;
   // routed_expert_down_proj
   const __nv_bfloat16* xe = xr;
@@ -543,7 +671,7 @@ int moe_block_forward(const moe_bf16* x, int64_t N, const moe_block_dims* dims,
     // (the tile list was written before the router's kernels: a programmatic
     // dependent launch is safe here and below)
     if ((rc = linear_run(xr, N, d_r, cbf(wt->down_proj), d_e, nullptr, bf(L.xe), tiles, st, s,
-                         true)))
+                         true, part)))
       return rc;
     xe = bf(L.xe);
   }
@@ -567,7 +695,7 @@ int moe_block_forward(const moe_bf16* x, int64_t N, const moe_block_dims* dims,
                                                 st, s)
                       : launch_combine(bf(F.y), pos, w, N, K, d_e, N * K, bf(L.yc), st, s);
   if (e != cudaSuccess) return MOE_ERR_CUDA;
-  return linear_run(bf(L.yc), N, d_e, cbf(wt->up_proj), d_r, sh, o, tiles, st, s, true);
+  return linear_run(bf(L.yc), N, d_e, cbf(wt->up_proj), d_r, sh, o, tiles, st, s, true, part);
 }
 
 }  // extern "C"

@@ -14,7 +14,8 @@
 //   k_scatter one warp per chunk again: slots ranked in slot order within the
 //             chunk -> pos[slot] and perm[pos].
 // Then k_gather copies every token row once from HBM and writes it to its K
-// sorted positions (token-major, so x_e is read once, not K times).
+// sorted positions (token-major, so x_e is read once, not K times).  Without
+// xs (the expert MLP gathering its rows itself) k_gather is skipped.
 #include "moe_internal.cuh"
 
 namespace moe {
@@ -163,7 +164,50 @@ __global__ void __launch_bounds__(256) k_gather(const __nv_bfloat16* __restrict_
   }
 }
 
+// offsets[i] = sum_{j<i} counts[j] for i <= n (n <= 1024), one block.
+__global__ void __launch_bounds__(1024) k_counts_offsets(const int32_t* __restrict__ counts, int n,
+                                                         int32_t* __restrict__ offsets,
+                                                         DeviceStatus* st) {
+  __shared__ int32_t warp_tot[32];
+  const int i = threadIdx.x, lane = i & 31, warp = i >> 5;
+  int32_t c = 0;
+  if (i < n) {
+    c = counts[i];
+    if (c < 0) {
+      record_error(st, MOE_ERR_DEVICE_BOUNDS, 12);
+      c = 0;
+    }
+  }
+  int32_t v = c;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int32_t o = __shfl_up_sync(0xffffffffu, v, off);
+    if (lane >= off) v += o;
+  }
+  if (lane == 31) warp_tot[warp] = v;
+  __syncthreads();
+  if (warp == 0) {
+    int32_t w = warp_tot[lane];
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int32_t o = __shfl_up_sync(0xffffffffu, w, off);
+      if (lane >= off) w += o;
+    }
+    warp_tot[lane] = w;
+  }
+  __syncthreads();
+  const int32_t excl = v - c + (warp > 0 ? warp_tot[warp - 1] : 0);
+  if (i < n) offsets[i] = excl;
+  if (i == n - 1) offsets[n] = excl + c;
+}
+
 }  // namespace
+
+cudaError_t launch_counts_offsets(const int32_t* counts, int n, int32_t* offsets,
+                                  DeviceStatus* st, cudaStream_t s) {
+  k_counts_offsets<<<1, 1024, 0, s>>>(counts, n, offsets, st);
+  return cudaGetLastError();
+}
 
 int dispatch_chunks(int64_t S) {
   int64_t ch = S / 256;
@@ -196,6 +240,7 @@ cudaError_t launch_dispatch(const int32_t* idx, int64_t N, int K, int E, const _
   k_hist<<<blocks, 32 * kWarps, smem, s>>>(idx, S, E, CH, nchunks, scratch, st);
   k_scan<<<1, 1024, 0, s>>>(scratch, nchunks, E, counts, offsets);
   k_scatter<<<blocks, 32 * kWarps, smem, s>>>(idx, S, E, CH, nchunks, scratch, perm, pos);
+  if (!xs) return cudaGetLastError();
   int64_t gb = (N * ((d_e / 8 + 31) / 32) + 7) / 8;
   const int64_t cap = (int64_t)dev_info()->sm_count * 16;
   if (gb > cap) gb = cap;

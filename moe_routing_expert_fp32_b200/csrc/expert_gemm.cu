@@ -21,8 +21,16 @@
 //     thread issues tcgen05.mma kind::f16 (bf16 in, fp32 accumulate) into
 //     TMEM; two accumulator buffers let the epilogue of one unit overlap the
 //     MMAs of the next; 4 epilogue warps drain TMEM with tcgen05.ld.
-//   * three variants by average rows per expert: decode (NTMAX 32, 10 stages:
-//     ~160 KB of weights in flight per SM, weights loaded with an L2
+//   * decode and mid variants can gather their token rows themselves: row i of
+//     a tile is x_e[perm[row0 + i] / K], fetched with tile::gather4 TMA loads
+//     (4 rows of 64 columns each, the same 128-byte swizzle), so no gathered
+//     copy xs of the tokens is needed (a memory saving: 32 small loads per
+//     128-row tile make it slower than a separate gather plus tiled loads);
+//   * dense layers (one expert, every row) split K over units when the row
+//     blocks alone would leave SMs idle, and k_splitk_reduce finishes them;
+//   * three variants by average rows per expert: decode (NTMAX 32, 5 stages
+//     of two 64-column sub-tiles: ~160 KB of weights in flight per SM, so each
+//     weight row is read 256 contiguous bytes at a time, loaded with an L2
 //     evict-first hint since each is read once), mid (NTMAX 128, two A blocks
 //     and accumulators per unit, 4 stages) and large (a CTA pair running
 //     256x256x16 cta_group::2 MMAs, 6 stages; see k_expert_gemm_pair).
@@ -147,6 +155,18 @@ __device__ __forceinline__ void tma_load_3d_hint(const CUtensorMap* map, uint64_
       : "memory");
 }
 
+// Four rows r0..r3 (any order, any rows) of a 2-D map whose box is 64 columns
+// x 1 row, written to dst as consecutive 128-byte rows with the map's swizzle.
+__device__ __forceinline__ void tma_gather4(const CUtensorMap* map, uint64_t* bar, void* dst,
+                                            int c0, int r0, int r1, int r2, int r3) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(r0), "r"(r1),
+      "r"(r2), "r"(r3)
+      : "memory");
+}
+
 // Programmatic dependent launch: the dependent kernel waits here until the
 // preceding kernel's memory is visible; a primary lets dependents launch.
 __device__ __forceinline__ void grid_dep_wait() {
@@ -242,12 +262,15 @@ __device__ __forceinline__ float situ_mul(float g, float u, float beta, float lb
   return __fmul_rn(__fmul_rn(t, sg), up);
 }
 
+// e: the weight index of the unit's segment.  Segment s (rows offsets[s] ..
+// offsets[s+1]) uses weights s % emod: emod = E for the layer, E_local for
+// rows received from several ranks, grouped by (source rank, local expert).
 struct Unit {
   int e, row0, nrows, rb;
 };
 
 __device__ __forceinline__ Unit decode_unit(int64_t u, int RB, int nt, const int32_t* tile_start,
-                                            const int32_t* offsets, int E) {
+                                            const int32_t* offsets, int E, int emod) {
   Unit r;
   const int tt = (int)(u / RB);
   r.rb = (int)(u - (int64_t)tt * RB);
@@ -257,7 +280,7 @@ __device__ __forceinline__ Unit decode_unit(int64_t u, int RB, int nt, const int
     if (tile_start[mid] <= tt) lo = mid;
     else hi = mid - 1;
   }
-  r.e = lo;
+  r.e = lo % emod;
   r.row0 = offsets[lo] + (tt - tile_start[lo]) * nt;
   const int rem = offsets[lo + 1] - r.row0;
   r.nrows = rem < nt ? rem : nt;
@@ -271,7 +294,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                   const int32_t* __restrict__ offsets,
                   const int32_t* __restrict__ tile_start, int E, int M_rows, int Kdim,
                   __nv_bfloat16* __restrict__ out, const __nv_bfloat16* __restrict__ res,
-                  int act_kind, float beta, float lbeta, DeviceStatus* st, int pdl) {
+                  int act_kind, float beta, float lbeta, DeviceStatus* st, int pdl,
+                  const int32_t* __restrict__ gperm, int gk, int gn, int ksplit,
+                  float* __restrict__ part, int emod) {
   using C = Cfg<NTMAX, STAGES, UM, KSUB>;
   constexpr int KS = BK * KSUB;  // K columns per stage
   constexpr bool kDecode = NTMAX <= 32;
@@ -292,7 +317,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int unit_rows = UM * blk_rows;
   const int RB = (M_rows + unit_rows - 1) / unit_rows;
   const int KB = Kdim / KS;
-  const int64_t total_units = (int64_t)tile_start[E] * RB;
+  // split-K (dense layers with few units): unit u covers k-blocks
+  // [ks*KB/ksplit, (ks+1)*KB/ksplit) of (token tile, row block) u / ksplit,
+  // and its epilogue writes fp32 partial sums to `part` for k_splitk_reduce
+  const int64_t total_units = (int64_t)tile_start[E] * RB * ksplit;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -317,9 +345,84 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
+  bool gathered = false;
+  if constexpr (MODE == kGateUp) {
+    if (warp == 0 && gperm != nullptr) {
+      // ---------------------------------------- TMA producer, gathered rows
+      // Row i of a unit's token tile is x_e[perm[row0 + i] / K] (sorted slot
+      // -> token): the warp reads the tile's token ids, lane 0 fetches the
+      // rows 4 at a time with tile::gather4 loads of tmB (box 64 x 1, same
+      // swizzle as a tiled box).  Rows past the segment up to the next
+      // multiple of 16 repeat its last row; their accumulator columns are
+      // never stored.
+      __shared__ int32_t tok_s[NTMAX];
+      gathered = true;
+      const uint64_t wpol = kDecode ? l2_evict_first_policy() : 0;
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int64_t u = blockIdx.x; u < total_units && ok; u += gridDim.x) {
+        const Unit w = decode_unit(u / ksplit, RB, NTMAX, tile_start, offsets, E, emod);
+        const int ks = (int)(u % ksplit);
+        const int kb0 = (int)((int64_t)ks * KB / ksplit), kb1 = (int)((int64_t)(ks + 1) * KB / ksplit);
+        const int rows = (w.nrows + 15) & ~15;
+        __syncwarp();
+        for (int i = lane; i < rows; i += 32) {
+          int32_t t = gperm[w.row0 + (i < w.nrows ? i : w.nrows - 1)] / gk;
+          if (t < 0 || t >= gn) {  // a slot outside the batch: recorded, row 0 read
+            record_error(st, MOE_ERR_DEVICE_BOUNDS, 31);
+            t = 0;
+          }
+          tok_s[i] = t;
+        }
+        __syncwarp();
+        if (lane == 0) {
+          const uint32_t bytes = C::kABytes + KSUB * rows * BK * 2;
+          const int r0 = w.rb * unit_rows;
+          for (int kb = kb0; kb < kb1; ++kb) {
+            if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag)) { ok = false; break; }
+            uint8_t* sA = smem + stage * C::kStageBytes;
+            uint8_t* sB = sA + C::kABytes;
+            mbar_arrive_expect_tx(&full[stage], bytes);
+#pragma unroll
+            for (int sub = 0; sub < KSUB; ++sub) {
+              const int kc = kb * KS + sub * BK;
+#pragma unroll
+              for (int a = 0; a < UM; ++a) {
+                uint8_t* dA = sA + (a * KSUB + sub) * C::kABlockBytes;
+                const int ra = r0 + a * blk_rows;
+                void* d3 = dA + kGateUpRows * BK * 2;
+                if (kDecode) {
+                  tma_load_3d_hint(&tmA0, &full[stage], dA, kc, ra, w.e, wpol);
+                  tma_load_3d_hint(&tmA1, &full[stage], d3, kc, ra, w.e, wpol);
+                } else {
+                  tma_load_3d(&tmA0, &full[stage], dA, kc, ra, w.e);
+                  tma_load_3d(&tmA1, &full[stage], d3, kc, ra, w.e);
+                }
+              }
+              for (int g = 0; g < rows; g += 4)
+                tma_gather4(&tmB, &full[stage], sB + sub * C::kBSubBytes + g * BK * 2, kc,
+                            tok_s[g], tok_s[g + 1], tok_s[g + 2], tok_s[g + 3]);
+            }
+            if (++stage == STAGES) { stage = 0; phase ^= 1; }
+          }
+        }
+        ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+      }
+      if (lane == 0) {
+        grid_dep_launch();
+        if (!ok) {
+          record_error(st, MOE_ERR_DEVICE_TIMEOUT, 105);
+          *abort_flag = 1;
+        }
+      }
+    }
+  }
   if (warp == 0) {
     // ------------------------------------------------------ TMA producer
-    if (lane == 0) {
+    // (warp 0 is the producer in both forms; with gathered rows it ran above,
+    // and it must not fall through to the MMA or epilogue roles)
+    if (lane == 0 && !gathered) {
       const uint64_t wpol = kDecode ? l2_evict_first_policy() : 0;
       int stage = 0;
       uint32_t phase = 0;
@@ -329,7 +432,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       // tiles of the first ring of stages are fetched before it.
       bool dep_pending = pdl != 0;
       for (int64_t u = blockIdx.x; u < total_units && ok; u += gridDim.x) {
-        const Unit w = decode_unit(u, RB, NTMAX, tile_start, offsets, E);
+        const Unit w = decode_unit(u / ksplit, RB, NTMAX, tile_start, offsets, E, emod);
+        const int ks = (int)(u % ksplit);
+        const int kb0 = (int)((int64_t)ks * KB / ksplit), kb1 = (int)((int64_t)(ks + 1) * KB / ksplit);
         // token rows: 16-row boxes for short tiles, 64-row boxes otherwise
         const bool big = !kDecode && w.nrows > 2 * kBoxRows;
         const int brows = big ? kBigBoxRows : kBoxRows;
@@ -369,10 +474,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                           sB + sub * C::kBSubBytes + i * brows * BK * 2, kb * KS + sub * BK,
                           w.row0 + i * brows);
         };
-        int kb = 0;
+        int kb = kb0;
         if (dep_pending) {
           // weights of up to STAGES k-blocks first, then wait, then their tokens
-          const int pre = KB < STAGES ? KB : STAGES;
+          const int pre = kb0 + (kb1 - kb0 < STAGES ? kb1 - kb0 : STAGES);
           for (; kb < pre; ++kb) {
             if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag)) { ok = false; break; }
             mbar_arrive_expect_tx(&full[stage], bytes);
@@ -382,13 +487,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           grid_dep_wait();
           dep_pending = false;
           int st_idx = 0;  // the first unit started at stage 0
-          for (int j = 0; j < kb; ++j) {
+          for (int j = kb0; j < kb; ++j) {
             load_b(j, smem + st_idx * C::kStageBytes + C::kABytes, st_idx);
             if (++st_idx == STAGES) st_idx = 0;
           }
           if (!ok) break;
         }
-        for (; kb < KB; ++kb) {
+        for (; kb < kb1; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag)) { ok = false; break; }
           uint8_t* sA = smem + stage * C::kStageBytes;
           mbar_arrive_expect_tx(&full[stage], bytes);
@@ -413,7 +518,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       int local = 0;
       bool ok = true;
       for (int64_t u = blockIdx.x; u < total_units && ok; u += gridDim.x, ++local) {
-        const Unit w = decode_unit(u, RB, NTMAX, tile_start, offsets, E);
+        const Unit w = decode_unit(u / ksplit, RB, NTMAX, tile_start, offsets, E, emod);
+        const int ks = (int)(u % ksplit);
+        const int kb0 = (int)((int64_t)ks * KB / ksplit), kb1 = (int)((int64_t)(ks + 1) * KB / ksplit);
         const int n = ((w.nrows + 15) / 16) * 16;
         const uint32_t idesc = idesc_bf16(n);
         const int buf = local & 1;
@@ -421,7 +528,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!mbar_wait(&tempty[buf], tphase ^ 1, abort_flag)) { ok = false; break; }
         tc_fence_after();
         const uint32_t d0 = tmem_base + buf * C::kBufCols;
-        for (int kb = 0; kb < KB; ++kb) {
+        for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait(&full[stage], phase, abort_flag)) { ok = false; break; }
           tc_fence_after();
           const uint32_t a0 = smem_u32(smem + stage * C::kStageBytes);
@@ -435,7 +542,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 umma_bf16(d0 + a * NTMAX,
                           sw128_desc(a0 + (a * KSUB + sub) * C::kABlockBytes + k * UK * 2),
                           sw128_desc(b0 + sub * C::kBSubBytes + k * UK * 2), idesc,
-                          (kb | sub | k) != 0);
+                          (kb != kb0 || sub != 0 || k != 0));
           umma_commit(&empty[stage]);
           if (++stage == STAGES) { stage = 0; phase ^= 1; }
         }
@@ -454,7 +561,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     int local = 0;
     uint32_t xbuf = 0;  // exchange buffer parity (gate_up)
     for (int64_t u = blockIdx.x; u < total_units; u += gridDim.x, ++local) {
-      const Unit w = decode_unit(u, RB, NTMAX, tile_start, offsets, E);
+      const Unit w = decode_unit(u / ksplit, RB, NTMAX, tile_start, offsets, E, emod);
+      const int ks = (int)(u % ksplit);
       const int buf = local & 1;
       const uint32_t tphase = (local >> 1) & 1;
       if (!mbar_wait(&tfull[buf], tphase, abort_flag)) {
@@ -467,7 +575,32 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t taddr =
           tmem_base + ((uint32_t)(quarter * 32) << 16) + buf * C::kBufCols + a * NTMAX;
       const int r0 = w.rb * unit_rows + a * blk_rows;
-      if (MODE == kGateUp) {
+      if (part) {
+        // fp32 partial sums: down -> part[ks][row][m]; gate_up -> g at
+        // part[ks][row][f], u at part[ks][row][F + f]
+        const int64_t S_rows = offsets[E];
+        int m, ld, moff;
+        if (MODE == kGateUp) {
+          m = r0 + (quarter & 1) * 32 + lane;
+          ld = 2 * M_rows;
+          moff = quarter < 2 ? 0 : M_rows;
+        } else {
+          m = r0 + quarter * 32 + lane;
+          ld = M_rows;
+          moff = 0;
+        }
+        float* pcol = part + (int64_t)ks * S_rows * ld + moff + m;
+        const int lim_m = m < M_rows ? 16 : 0;
+        for (int c0 = 0; c0 < w.nrows; c0 += 16) {
+          float v[16];
+          tmem_ld16(taddr + c0, v);
+          int lim = w.nrows - c0 < 16 ? w.nrows - c0 : 16;
+          lim = lim < lim_m ? lim : lim_m;
+#pragma unroll
+          for (int j = 0; j < 16; ++j)
+            if (j < lim) pcol[(int64_t)(w.row0 + c0 + j) * ld] = v[j];
+        }
+      } else if (MODE == kGateUp) {
         // quarters 0/1 hold g of rows 0-31 / 32-63, quarters 2/3 hold u of the
         // same rows; pair p = quarter & 1.  Per 16-column chunk the g warp keeps
         // columns 0-7 and hands g of columns 8-15 to the u warp, which keeps
@@ -623,7 +756,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                        const int32_t* __restrict__ offsets, const int32_t* __restrict__ tile_start,
                        int E, int M_rows, int Kdim, __nv_bfloat16* __restrict__ out,
                        const __nv_bfloat16* __restrict__ res, int act_kind, float beta,
-                       float lbeta, DeviceStatus* st, int pdl) {
+                       float lbeta, DeviceStatus* st, int pdl, int emod) {
   using C = PairCfg;
   constexpr int STAGES = kPairStages;
   extern __shared__ uint8_t smem_raw[];
@@ -680,7 +813,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       bool dep_pending = pdl != 0;  // see the single-CTA kernel
       for (int64_t u = pair_id; u < total_units && ok; u += npairs) {
-        const Unit w = decode_unit(u, RB, kPairNt, tile_start, offsets, E);
+        const Unit w = decode_unit(u, RB, kPairNt, tile_start, offsets, E, emod);
         const int n = ((w.nrows + 15) / 16) * 16;
         const int half = n / 2;  // token rows this CTA contributes
         const bool big = half > 2 * kBoxRows;
@@ -741,7 +874,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       int local = 0;
       bool ok = true;
       for (int64_t u = pair_id; u < total_units && ok; u += npairs, ++local) {
-        const Unit w = decode_unit(u, RB, kPairNt, tile_start, offsets, E);
+        const Unit w = decode_unit(u, RB, kPairNt, tile_start, offsets, E, emod);
         const int n = ((w.nrows + 15) / 16) * 16;
         const uint32_t idesc = idesc_bf16_m256(n);
         const int buf = local & 1;
@@ -777,7 +910,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     int local = 0;
     uint32_t xbuf = 0;
     for (int64_t u = pair_id; u < total_units; u += npairs, ++local) {
-      const Unit w = decode_unit(u, RB, kPairNt, tile_start, offsets, E);
+      const Unit w = decode_unit(u, RB, kPairNt, tile_start, offsets, E, emod);
       const int buf = local & 1;
       const uint32_t tphase = (local >> 1) & 1;
       if (!mbar_wait(&tfull[buf], tphase, abort_flag)) {
@@ -940,7 +1073,9 @@ cudaError_t launch_gemm(const CUtensorMap& a0, const CUtensorMap& a1, const CUte
                         const CUtensorMap& b64, const int32_t* offsets, const int32_t* tile_start,
                         int E, int M_rows, int Kdim, __nv_bfloat16* out,
                         const __nv_bfloat16* res, const moe_act_cfg& act, DeviceStatus* st,
-                        cudaStream_t s, bool pdl_ok) {
+                        cudaStream_t s, bool pdl_ok, const int32_t* gperm = nullptr,
+                        int gk = 1, int gn = 0, int ksplit = 1, float* part = nullptr,
+                        int emod = 0) {
   using C = Cfg<NTMAX, STAGES, UM, KSUB>;
   static bool attr_set[64] = {false};
   int dev = 0;
@@ -970,7 +1105,8 @@ cudaError_t launch_gemm(const CUtensorMap& a0, const CUtensorMap& a1, const CUte
   cfg.numAttrs = pdl ? 1 : 0;
   return cudaLaunchKernelEx(&cfg, k_expert_gemm<MODE, NTMAX, STAGES, UM, KSUB>, a0, a1, b, b64,
                             offsets, tile_start, E, M_rows, Kdim, out, res, (int)act.kind,
-                            act.beta, act.linear_beta, st, pdl);
+                            act.beta, act.linear_beta, st, pdl, gperm, gk, gn, ksplit, part,
+                            emod > 0 ? emod : E);
 }
 
 // Launches the CTA-pair kernel on as many pairs as can be resident at once.
@@ -980,7 +1116,7 @@ cudaError_t launch_gemm_pair(const CUtensorMap& a0, const CUtensorMap& a1, const
                              const int32_t* tile_start, int E, int M_rows, int Kdim,
                              __nv_bfloat16* out, const __nv_bfloat16* res,
                              const moe_act_cfg& act, DeviceStatus* st, cudaStream_t s,
-                             bool pdl_ok) {
+                             bool pdl_ok, int emod = 0) {
   using C = PairCfg;
   static bool attr_set[64] = {false};
   static int grid_of[64] = {0};
@@ -1017,7 +1153,7 @@ cudaError_t launch_gemm_pair(const CUtensorMap& a0, const CUtensorMap& a1, const
   cfg.numAttrs = pdl ? 2 : 1;
   return cudaLaunchKernelEx(&cfg, k_expert_gemm_pair<MODE>, a0, a1, b, b64, offsets, tile_start,
                             E, M_rows, Kdim, out, res, (int)act.kind, act.beta, act.linear_beta,
-                            st, pdl);
+                            st, pdl, emod > 0 ? emod : E);
 }
 
 // Variant choice from shapes only (no host round trip), by the average rows
@@ -1041,17 +1177,20 @@ cudaError_t launch_variant(Variant v, const CUtensorMap& a0, const CUtensorMap& 
                            const CUtensorMap& b, const CUtensorMap& b64, const int32_t* offsets,
                            const int32_t* tile_start, int E, int M_rows, int Kdim,
                            __nv_bfloat16* out, const __nv_bfloat16* res, const moe_act_cfg& act,
-                           DeviceStatus* st, cudaStream_t s, bool pdl_ok = true) {
+                           DeviceStatus* st, cudaStream_t s, bool pdl_ok = true,
+                           int emod = 0) {
   switch (v) {
     case kVarDecode:
       return launch_gemm<MODE, kNtDecode, kStagesDecode, kUmDecode, kKsubDecode>(
-          a0, a1, b, b64, offsets, tile_start, E, M_rows, Kdim, out, res, act, st, s, pdl_ok);
+          a0, a1, b, b64, offsets, tile_start, E, M_rows, Kdim, out, res, act, st, s, pdl_ok,
+          nullptr, 1, 0, 1, nullptr, emod);
     case kVarMid:
       return launch_gemm<MODE, kNtMid, kStagesMid, kUmMid, kKsubMid>(
-          a0, a1, b, b64, offsets, tile_start, E, M_rows, Kdim, out, res, act, st, s, pdl_ok);
+          a0, a1, b, b64, offsets, tile_start, E, M_rows, Kdim, out, res, act, st, s, pdl_ok,
+          nullptr, 1, 0, 1, nullptr, emod);
     default:
       return launch_gemm_pair<MODE>(a0, a1, b, b64, offsets, tile_start, E, M_rows, Kdim, out,
-                                    res, act, st, s, pdl_ok);
+                                    res, act, st, s, pdl_ok, emod);
   }
 }
 
@@ -1062,36 +1201,173 @@ size_t expert_scratch_bytes(int64_t S, int E, int F) {
          align_up(sizeof(__nv_bfloat16) * (size_t)S * (size_t)F, 256);
 }
 
+bool expert_gather_fusable(int64_t S, int E) { return pick_variant(S, E) != kVarLarge; }
+
 int expert_ffn_run(const __nv_bfloat16* xs, const int32_t* offsets, int E, int64_t S, int d_e,
                    int F, const __nv_bfloat16* w1, const __nv_bfloat16* w3,
                    const __nv_bfloat16* w2, const moe_act_cfg& act, __nv_bfloat16* y,
                    void* scratch, DeviceStatus* st, cudaStream_t s, cudaEvent_t after_gate_up,
-                   const __nv_bfloat16* residual) {
+                   const __nv_bfloat16* residual, const GatherSrc* gather, int n_weights) {
+  // segments s use weights s % n_weights (n_weights = E for the layer)
+  const int emod = n_weights > 0 ? n_weights : E;
   int32_t* tile_start = static_cast<int32_t*>(scratch);
   __nv_bfloat16* h = reinterpret_cast<__nv_bfloat16*>(
       static_cast<uint8_t*>(scratch) + align_up(sizeof(int32_t) * (size_t)(E + 1), 256));
   CUtensorMap mw1, mw3, mw2, mxs, mh, mxs64, mh64;
-  if (!make_map_3d(&mw1, w1, d_e, F, E, kGateUpRows) ||
-      !make_map_3d(&mw3, w3, d_e, F, E, kGateUpRows) || !make_map_3d(&mw2, w2, F, d_e, E, BM) ||
-      !make_map_2d(&mxs, xs, d_e, S, kBoxRows) || !make_map_2d(&mh, h, F, S, kBoxRows) ||
-      !make_map_2d(&mxs64, xs, d_e, S, kBigBoxRows) || !make_map_2d(&mh64, h, F, S, kBigBoxRows))
+  if (!make_map_3d(&mw1, w1, d_e, F, emod, kGateUpRows) ||
+      !make_map_3d(&mw3, w3, d_e, F, emod, kGateUpRows) ||
+      !make_map_3d(&mw2, w2, F, d_e, emod, BM) || !make_map_2d(&mh, h, F, S, kBoxRows) ||
+      !make_map_2d(&mh64, h, F, S, kBigBoxRows))
+    return MOE_ERR_CUDA;
+  if (!gather && (!make_map_2d(&mxs, xs, d_e, S, kBoxRows) ||
+                  !make_map_2d(&mxs64, xs, d_e, S, kBigBoxRows)))
     return MOE_ERR_CUDA;
   const Variant var = pick_variant(S, E);
   const int nt = var == kVarDecode ? kNtDecode : (var == kVarMid ? kNtMid : kPairNt);
   k_tiles<<<1, 1024, 0, s>>>(offsets, E, S, nt, tile_start, st);
   if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
-  cudaError_t rc = launch_variant<kGateUp>(var, mw1, mw3, mxs, mxs64, offsets, tile_start, E, F,
-                                           d_e, h, nullptr, act, st, s);
+  cudaError_t rc;
+  if (gather) {
+    // token rows straight from x_e (no xs): decode and mid variants only
+    if (var == kVarLarge) return MOE_ERR_INVALID_ARG;
+    CUtensorMap mxg;
+    if (!make_map_2d(&mxg, gather->x_e, d_e, gather->N, 1)) return MOE_ERR_CUDA;
+    rc = var == kVarDecode
+             ? launch_gemm<kGateUp, kNtDecode, kStagesDecode, kUmDecode, kKsubDecode>(
+                   mw1, mw3, mxg, mxg, offsets, tile_start, E, F, d_e, h, nullptr, act, st, s,
+                   false, gather->perm, gather->K, (int)gather->N, 1, nullptr, emod)
+             : launch_gemm<kGateUp, kNtMid, kStagesMid, kUmMid, kKsubMid>(
+                   mw1, mw3, mxg, mxg, offsets, tile_start, E, F, d_e, h, nullptr, act, st, s,
+                   false, gather->perm, gather->K, (int)gather->N, 1, nullptr, emod);
+  } else {
+    rc = launch_variant<kGateUp>(var, mw1, mw3, mxs, mxs64, offsets, tile_start, E, F, d_e, h,
+                                 nullptr, act, st, s, true, emod);
+  }
   if (rc != cudaSuccess) return MOE_ERR_CUDA;
   if (after_gate_up && cudaEventRecord(after_gate_up, s) != cudaSuccess) return MOE_ERR_CUDA;
   rc = launch_variant<kDown>(var, mw2, mw2, mh, mh64, offsets, tile_start, E, d_e, F, y, residual,
-                             act, st, s);
+                             act, st, s, true, emod);
   return rc == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
 // ------------------------------------------------------------ dense layers
 // A dense bias-free Linear (or a shared-expert MLP) is the grouped GEMM with
 // one expert whose segment is every row: offsets = {0, M}, one tile list.
+// At decode sizes that is only a few units of 128-256 weight rows, so the
+// weight stream is split over K as well (split-K): each unit writes fp32
+// partial sums and k_splitk_reduce adds them in split order, then applies
+// the bf16 rounding, the residual or the activation exactly as the GEMM's own
+// epilogue does.
+namespace {
+template <int MODE>
+__global__ void __launch_bounds__(256) k_splitk_reduce(const float* __restrict__ part, int ksplit,
+                                                       int64_t M, int cols,
+                                                       const __nv_bfloat16* __restrict__ res,
+                                                       __nv_bfloat16* __restrict__ out,
+                                                       int act_kind, float beta, float lbeta) {
+  const bool has_lb = !(lbeta == 0.0f || lbeta != lbeta);
+  const float b_eff = (beta == 0.0f || beta != beta) ? 1.0f : beta;
+  const int64_t ld = MODE == kGateUp ? 2 * (int64_t)cols : cols;
+  const int64_t n4 = M * cols / 4;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n4;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t t = (i * 4) / cols;
+    const int m = (int)(i * 4 - t * cols);
+    float a[4] = {0.f, 0.f, 0.f, 0.f}, g[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int ks = 0; ks < ksplit; ++ks) {
+      const float* row = part + ((int64_t)ks * M + t) * ld;
+      const float4 v = *reinterpret_cast<const float4*>(row + m);
+      if (ks == 0) { a[0] = v.x; a[1] = v.y; a[2] = v.z; a[3] = v.w; }
+      else {
+        a[0] = __fadd_rn(a[0], v.x); a[1] = __fadd_rn(a[1], v.y);
+        a[2] = __fadd_rn(a[2], v.z); a[3] = __fadd_rn(a[3], v.w);
+      }
+      if (MODE == kGateUp) {
+        const float4 u = *reinterpret_cast<const float4*>(row + cols + m);
+        if (ks == 0) { g[0] = u.x; g[1] = u.y; g[2] = u.z; g[3] = u.w; }
+        else {
+          g[0] = __fadd_rn(g[0], u.x); g[1] = __fadd_rn(g[1], u.y);
+          g[2] = __fadd_rn(g[2], u.z); g[3] = __fadd_rn(g[3], u.w);
+        }
+      }
+    }
+    __nv_bfloat16 o[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      if (MODE == kGateUp) {
+        // a = the w1 (gate) sum, g = the w3 (up) sum
+        const float h = act_kind == MOE_ACT_SITU ? situ_mul(a[j], g[j], b_eff, lbeta, has_lb)
+                                                 : silu_mul(a[j], g[j]);
+        o[j] = __float2bfloat16_rn(h);
+      } else {
+        o[j] = down_out(a[j], res, (int)t, cols, m + j);
+      }
+    }
+    __nv_bfloat16* dst = out + t * cols + m;
+    *reinterpret_cast<__nv_bfloat162*>(dst) = __halves2bfloat162(o[0], o[1]);
+    *reinterpret_cast<__nv_bfloat162*>(dst + 2) = __halves2bfloat162(o[2], o[3]);
+  }
+}
+
+// Split factor of a dense layer (one expert, M rows): enough units for the
+// 148 SMs of a B200, at least two k-blocks per split; 1 when the layer already
+// fills the GPU.  A function of the shapes only, so workspace sizes can be
+// computed before a device is chosen.
+constexpr int kSplitTargetUnits = 148;
+int dense_ksplit(Variant v, int mode, int64_t M, int M_rows, int Kdim) {
+  if (v == kVarLarge || M <= 0 || M_rows <= 0) return 1;
+  const int nt = v == kVarDecode ? kNtDecode : kNtMid;
+  const int um = v == kVarDecode ? kUmDecode : kUmMid;
+  const int ks = BK * (v == kVarDecode ? kKsubDecode : kKsubMid);
+  const int unit_rows = um * (mode == kGateUp ? kGateUpRows : BM);
+  const int64_t units = ((M + nt - 1) / nt) * ((M_rows + unit_rows - 1) / unit_rows);
+  const int sms = kSplitTargetUnits;
+  if (units * 2 >= sms) return 1;
+  int k = (int)((sms + units - 1) / units);
+  const int kb = Kdim / ks;
+  if (k > kb / 2) k = kb / 2;
+  if (k > 32) k = 32;
+  return k < 1 ? 1 : k;
+}
+
+template <int MODE>
+cudaError_t launch_dense(Variant var, const CUtensorMap& a0, const CUtensorMap& a1,
+                         const CUtensorMap& b, const CUtensorMap& b64, const int32_t* tiles,
+                         int64_t M, int M_rows, int Kdim, __nv_bfloat16* out,
+                         const __nv_bfloat16* res, const moe_act_cfg& act, DeviceStatus* st,
+                         cudaStream_t s, bool pdl_ok, float* part) {
+  const int32_t* ts = tiles + 2 + 2 * (int)var;
+  const int ksplit = part ? dense_ksplit(var, MODE, M, M_rows, Kdim) : 1;
+  if (ksplit <= 1)
+    return launch_variant<MODE>(var, a0, a1, b, b64, tiles, ts, 1, M_rows, Kdim, out, res, act,
+                                st, s, pdl_ok);
+  cudaError_t e =
+      var == kVarDecode
+          ? launch_gemm<MODE, kNtDecode, kStagesDecode, kUmDecode, kKsubDecode>(
+                a0, a1, b, b64, tiles, ts, 1, M_rows, Kdim, out, res, act, st, s, pdl_ok,
+                nullptr, 1, 0, ksplit, part)
+          : launch_gemm<MODE, kNtMid, kStagesMid, kUmMid, kKsubMid>(
+                a0, a1, b, b64, tiles, ts, 1, M_rows, Kdim, out, res, act, st, s, pdl_ok,
+                nullptr, 1, 0, ksplit, part);
+  if (e != cudaSuccess) return e;
+  const int64_t n4 = M * M_rows / 4;
+  int64_t blocks = (n4 + 255) / 256;
+  const int64_t cap = (int64_t)dev_info()->sm_count * 8;
+  if (blocks > cap) blocks = cap;
+  k_splitk_reduce<MODE><<<(unsigned)blocks, 256, 0, s>>>(part, ksplit, M, M_rows, res, out,
+                                                         (int)act.kind, act.beta,
+                                                         act.linear_beta);
+  return cudaGetLastError();
+}
+}  // namespace
+
+size_t dense_part_bytes(int64_t M, int K, int Nout, bool gate_up) {
+  const Variant v = pick_variant(M, 1);
+  const int k = dense_ksplit(v, gate_up ? kGateUp : kDown, M, Nout, K);
+  if (k <= 1) return 0;
+  return align_up(sizeof(float) * (size_t)k * (size_t)M * (size_t)Nout * (gate_up ? 2 : 1), 256);
+}
+
 __global__ void k_dense_tiles(int64_t M, int32_t* __restrict__ tiles) {
   if (threadIdx.x == 0) {
     tiles[0] = 0;  // offsets
@@ -1105,12 +1381,6 @@ __global__ void k_dense_tiles(int64_t M, int32_t* __restrict__ tiles) {
   }
 }
 
-namespace {
-const int32_t* dense_tile_start(const int32_t* tiles, Variant v) {
-  return tiles + 2 + 2 * (int)v;
-}
-}  // namespace
-
 cudaError_t launch_dense_tiles(int64_t M, int32_t* tiles, cudaStream_t s) {
   k_dense_tiles<<<1, 32, 0, s>>>(M, tiles);
   return cudaGetLastError();
@@ -1118,15 +1388,15 @@ cudaError_t launch_dense_tiles(int64_t M, int32_t* tiles, cudaStream_t s) {
 
 int linear_run(const __nv_bfloat16* x, int64_t M, int K, const __nv_bfloat16* W, int Nout,
                const __nv_bfloat16* residual, __nv_bfloat16* y, const int32_t* tiles,
-               DeviceStatus* st, cudaStream_t s, bool pdl_ok) {
+               DeviceStatus* st, cudaStream_t s, bool pdl_ok, float* part) {
   CUtensorMap mw, mx, mx64;
   if (!make_map_3d(&mw, W, K, Nout, 1, BM) || !make_map_2d(&mx, x, K, M, kBoxRows) ||
       !make_map_2d(&mx64, x, K, M, kBigBoxRows))
     return MOE_ERR_CUDA;
   const Variant var = pick_variant(M, 1);
   const moe_act_cfg none = {MOE_ACT_SILU, 1.0f, 0.0f};
-  return launch_variant<kDown>(var, mw, mw, mx, mx64, tiles, dense_tile_start(tiles, var), 1, Nout,
-                               K, y, residual, none, st, s, pdl_ok) == cudaSuccess
+  return launch_dense<kDown>(var, mw, mw, mx, mx64, tiles, M, Nout, K, y, residual, none, st, s,
+                             pdl_ok, part) == cudaSuccess
              ? MOE_OK
              : MOE_ERR_CUDA;
 }
@@ -1134,7 +1404,7 @@ int linear_run(const __nv_bfloat16* x, int64_t M, int K, const __nv_bfloat16* W,
 int shared_ffn_run(const __nv_bfloat16* x, int64_t M, int d, int F, const __nv_bfloat16* w1,
                    const __nv_bfloat16* w3, const __nv_bfloat16* w2, const moe_act_cfg& act,
                    const __nv_bfloat16* residual, __nv_bfloat16* y, __nv_bfloat16* h,
-                   const int32_t* tiles, DeviceStatus* st, cudaStream_t s) {
+                   const int32_t* tiles, DeviceStatus* st, cudaStream_t s, float* part) {
   CUtensorMap mw1, mw3, mw2, mx, mh, mx64, mh64;
   if (!make_map_3d(&mw1, w1, d, F, 1, kGateUpRows) || !make_map_3d(&mw3, w3, d, F, 1, kGateUpRows) ||
       !make_map_3d(&mw2, w2, F, d, 1, BM) || !make_map_2d(&mx, x, d, M, kBoxRows) ||
@@ -1142,12 +1412,11 @@ int shared_ffn_run(const __nv_bfloat16* x, int64_t M, int d, int F, const __nv_b
       !make_map_2d(&mh64, h, F, M, kBigBoxRows))
     return MOE_ERR_CUDA;
   const Variant var = pick_variant(M, 1);
-  const int32_t* ts = dense_tile_start(tiles, var);
-  if (launch_variant<kGateUp>(var, mw1, mw3, mx, mx64, tiles, ts, 1, F, d, h, nullptr, act, st,
-                              s) != cudaSuccess)
+  if (launch_dense<kGateUp>(var, mw1, mw3, mx, mx64, tiles, M, F, d, h, nullptr, act, st, s,
+                            false, part) != cudaSuccess)
     return MOE_ERR_CUDA;
-  return launch_variant<kDown>(var, mw2, mw2, mh, mh64, tiles, ts, 1, d, F, y, residual, act, st,
-                               s) == cudaSuccess
+  return launch_dense<kDown>(var, mw2, mw2, mh, mh64, tiles, M, d, F, y, residual, act, st, s,
+                             true, part) == cudaSuccess
              ? MOE_OK
              : MOE_ERR_CUDA;
 }

@@ -52,35 +52,62 @@ cudaError_t launch_select(const float* part, int splits, int64_t N, const float*
 // dispatch.cu
 int dispatch_chunks(int64_t S);
 size_t dispatch_scratch_bytes(int64_t S, int E);
+// xs == nullptr: counts, offsets, perm and pos only (no gather)
 cudaError_t launch_dispatch(const int32_t* idx, int64_t N, int K, int E, const __nv_bfloat16* x_e,
                             int d_e, int32_t* counts, int32_t* offsets, int32_t* perm,
                             int32_t* pos, __nv_bfloat16* xs, int32_t* scratch, DeviceStatus* st,
                             cudaStream_t s);
 
+// offsets [n+1] = exclusive prefix of counts [n] (n <= 1024)
+cudaError_t launch_counts_offsets(const int32_t* counts, int n, int32_t* offsets,
+                                  DeviceStatus* st, cudaStream_t s);
+
 // expert_gemm.cu
 size_t expert_scratch_bytes(int64_t S, int E, int F);
-// residual (optional, [S, d_e] bf16): y = bf16(bf16(x.w2^T) + residual)
+// Token rows gathered inside the w1/w3 kernel instead of read from xs: sorted
+// row j is x_e[perm[j] / K], x_e [N, d_e].
+struct GatherSrc {
+  const __nv_bfloat16* x_e;
+  const int32_t* perm;
+  int64_t N;
+  int K;
+};
+// whether the variant chosen for (S, E) gathers inside the kernel (the CTA-pair
+// variant reads a gathered xs)
+bool expert_gather_fusable(int64_t S, int E);
+// residual (optional, [S, d_e] bf16): y = bf16(bf16(x.w2^T) + residual);
+// gather (optional): xs is not read, the rows come from gather->x_e;
+// n_weights: E segments (offsets[E+1]) use weights s % n_weights of the
+// stacked w1/w3/w2 ([n_weights, ...]); 0 means n_weights = E
 int expert_ffn_run(const __nv_bfloat16* xs, const int32_t* offsets, int E, int64_t S, int d_e,
                    int F, const __nv_bfloat16* w1, const __nv_bfloat16* w3,
                    const __nv_bfloat16* w2, const moe_act_cfg& act, __nv_bfloat16* y,
                    void* scratch, DeviceStatus* st, cudaStream_t s, cudaEvent_t after_gate_up,
-                   const __nv_bfloat16* residual = nullptr);
+                   const __nv_bfloat16* residual = nullptr, const GatherSrc* gather = nullptr,
+                   int n_weights = 0);
 // Dense layers on the same kernels (one expert, every row): `tiles` is 8 int32
 // of device memory written by launch_dense_tiles(M) before use.
 constexpr size_t kDenseTilesBytes = 256;
 cudaError_t launch_dense_tiles(int64_t M, int32_t* tiles, cudaStream_t s);
+// fp32 split-K partials a dense layer of M rows needs (0: it runs unsplit);
+// gate_up: the w1/w3 GEMM of an MLP of hidden width Nout
+size_t dense_part_bytes(int64_t M, int K, int Nout, bool gate_up);
 // y [M, Nout] = bf16(x [M, K] . W [Nout, K]^T) (+ residual [M, Nout]).
 // pdl_ok: the kernel may start as a programmatic dependent of the preceding
 // kernel; allowed only if `tiles` was written before that kernel started.
+// part: dense_part_bytes(M, K, Nout, false) bytes of scratch, or nullptr
+// (no split).
 int linear_run(const __nv_bfloat16* x, int64_t M, int K, const __nv_bfloat16* W, int Nout,
                const __nv_bfloat16* residual, __nv_bfloat16* y, const int32_t* tiles,
-               DeviceStatus* st, cudaStream_t s, bool pdl_ok);
-// the gated MLP of one expert on every row of x [M, d]; h: [M, F] bf16 scratch
-// (its down kernel is a programmatic dependent of its gate_up kernel)
+               DeviceStatus* st, cudaStream_t s, bool pdl_ok, float* part);
+// the gated MLP of one expert on every row of x [M, d]; h: [M, F] bf16 scratch;
+// part: max(dense_part_bytes(M, d, F, true), dense_part_bytes(M, F, d, false))
+// bytes, or nullptr.  Its down kernel is a programmatic dependent of the
+// kernel before it.
 int shared_ffn_run(const __nv_bfloat16* x, int64_t M, int d, int F, const __nv_bfloat16* w1,
                    const __nv_bfloat16* w3, const __nv_bfloat16* w2, const moe_act_cfg& act,
                    const __nv_bfloat16* residual, __nv_bfloat16* y, __nv_bfloat16* h,
-                   const int32_t* tiles, DeviceStatus* st, cudaStream_t s);
+                   const int32_t* tiles, DeviceStatus* st, cudaStream_t s, float* part);
 
 // combine.cu
 // residual (optional, [N, d_e]): out = bf16(bf16(sum) + residual)

@@ -217,7 +217,9 @@ def test_block_rejects_inconsistent_parts(L):
 
 
 def test_linear_and_norm_validation(L):
-    assert L.moe_linear_workspace_size() >= 256
+    assert L.moe_linear_workspace_size(64, 7168, 2048) > 512       # split-K partials
+    assert L.moe_linear_workspace_size(4096, 7168, 2048) == 512    # fills the GPU: no split
+    assert L.moe_linear_workspace_size(64, 100, 2048) == 0
     # K and N_out must be multiples of 128
     assert L.moe_linear(None, 0, 100, ctypes.c_void_p(256), 128, None, None, None, 0, None) == -2
     assert L.moe_linear(None, 0, 128, None, 128, None, None, None, 0, None) == -1
@@ -230,3 +232,21 @@ def test_linear_and_norm_validation(L):
     assert L.moe_rms_norm(None, 0, 100, w, 1e-6, None, None) == -2
     assert L.moe_rms_norm(None, 0, 16384, w, 1e-6, None, None) == -2
     assert L.moe_rms_norm(None, 4, 128, w, 1e-6, None, None) == -1
+
+
+def test_ep_expert_ffn_validation(L):
+    import moe_routing_expert_fp32_b200 as m
+    a = m._ActCfg(0, 1.0, 0.0)
+    p = ctypes.c_void_p(256)
+    assert L.moe_ep_expert_ffn_workspace_size(100, 256, 2, 8, 128) > 256
+    assert L.moe_ep_expert_ffn_workspace_size(100, 256, 0, 8, 128) == 0
+    # P * E_local above 1024
+    assert L.moe_ep_expert_ffn(None, 0, p, 64, 32, 256, 128, p, p, p, ctypes.byref(a), None, None,
+                               0, None) == -2
+    # missing counts, bad widths, NULL workspace
+    assert L.moe_ep_expert_ffn(None, 0, None, 2, 8, 256, 128, p, p, p, ctypes.byref(a), None, None,
+                               0, None) == -1
+    assert L.moe_ep_expert_ffn(None, 0, p, 2, 8, 200, 128, p, p, p, ctypes.byref(a), None, None,
+                               0, None) == -2
+    assert L.moe_ep_expert_ffn(None, 0, p, 2, 8, 256, 128, p, p, p, ctypes.byref(a), None, None,
+                               0, None) == -4

@@ -1,0 +1,109 @@
+"""The expert-parallel exchange on CPU (gloo, world sizes 2 and 3).
+
+`exchange_forward` (the product's exchange logic: counts all-to-all, rows
+all-to-all-v, local experts on the received segments, the reverse
+all-to-all-v, combine) runs here with the four compute steps taken by the CPU
+reference, so the collectives and the bookkeeping are checked without a GPU.
+Every rank's output must equal, bit for bit, the reference moe_infer of its
+own tokens with all experts on one rank (the expert MLP and the combine are
+row-wise, so only a wrong exchange can change a result).
+"""
+import os
+import socket
+
+import numpy as np
+import pytest
+import torch.multiprocessing as mp
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    p = s.getsockname()[1]
+    s.close()
+    return p
+
+
+def _case(rank, E):
+    """Rank-dependent token batches (uneven sizes) and shared weights."""
+    rng = np.random.default_rng(100 + rank)
+    N = 10 + 7 * rank
+    d, F, K = 32, 16, 3
+    x = (rng.standard_normal((N, d)).astype(np.float32).view(np.uint32) >> 16).astype(np.uint16)
+    wr = np.random.default_rng(7)
+    W = (wr.standard_normal((E, d)) * 0.2).astype(np.float32)
+    b = wr.uniform(-0.01, 0.01, E).astype(np.float32)
+
+    def bf(shape):
+        return ((wr.standard_normal(shape) * 0.1).astype(np.float32).view(np.uint32)
+                >> 16).astype(np.uint16)
+    return x, W, b, bf((E, F, d)), bf((E, F, d)), bf((E, d, F)), K
+
+
+def _worker(rank, world, port, E, q):
+    import datetime
+    import torch
+    import torch.distributed as dist
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        import oracle
+        from moe_routing_expert_fp32_b200.ep import Steps, exchange_forward
+        x, W, b, w1, w3, w2, K = _case(rank, E)
+        E_local = E // world
+        lo = rank * E_local
+
+        def route(xr):
+            idx, w, _ = oracle.route(xr.numpy().view(np.uint16), W, b, 1, 1, K, 1.5)
+            return torch.from_numpy(idx), torch.from_numpy(w)
+
+        def dispatch(idx, xe):
+            counts, _, perm, pos = oracle.dispatch(idx.numpy(), E)
+            xs = oracle.gather(xe.numpy().view(np.uint16), perm, K)
+            return (torch.from_numpy(counts), torch.from_numpy(pos),
+                    torch.from_numpy(xs.view(np.int16)))
+
+        def experts(xr, recv_counts):
+            rows = xr.numpy().view(np.uint16)
+            y = np.zeros_like(rows)
+            o = 0
+            rc = recv_counts.numpy()
+            for p in range(rc.shape[0]):
+                for e in range(rc.shape[1]):
+                    n = int(rc[p, e])
+                    if n:
+                        y[o:o + n] = oracle.expert_ffn(rows[o:o + n], w1[lo + e], w3[lo + e],
+                                                       w2[lo + e], "silu")
+                    o += n
+            assert o == rows.shape[0]
+            return torch.from_numpy(y.view(np.int16))
+
+        def combine(y, pos, w):
+            return torch.from_numpy(oracle.combine(y.numpy().view(np.uint16), pos.numpy(),
+                                                   w.numpy(), K))
+
+        xt = torch.from_numpy(x.view(np.int16))
+        out, idx, w = exchange_forward(xt, xt, Steps(route, dispatch, experts, combine), E)
+        ref = oracle.moe_infer(x, idx.numpy(), w.numpy(), w1, w3, w2, "silu")
+        q.put((rank, bool(np.array_equal(out.numpy(), ref)), int(idx.numel())))
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world,E", [(2, 8), (3, 12)])
+def test_exchange_forward_equals_one_rank(world, E):
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker, args=(r, world, port, E, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    res = [q.get(timeout=120) for _ in range(world)]
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    assert sorted(r[0] for r in res) == list(range(world))
+    assert all(r[1] for r in res), res

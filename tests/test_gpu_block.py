@@ -42,7 +42,7 @@ def _rand_bf16(rng, shape, scale=1.0):
 # ------------------------------------------------------------------- linear
 @pytest.mark.parametrize("M,K,N_out", [(1, 7168, 2048), (7, 256, 128), (64, 7168, 2048),
                                        (64, 2048, 7168), (100, 512, 384), (300, 1024, 256),
-                                       (1000, 256, 640)])
+                                       (1000, 256, 640), (16, 7168, 2048), (128, 2048, 7168)])
 def test_linear(moe, M, K, N_out):
     rng = np.random.default_rng(M * 7 + K + N_out)
     x = _rand_bf16(rng, (M, K))
@@ -211,7 +211,30 @@ def test_block_equals_its_entry_points_bitwise(moe):
     y = moe.forward(dev["x"], dev["W"], dev["bias"], cfg, dev["w1"], dev["w3"], dev["w2"], act,
                     x_e=x_e)
     y = moe.rms_norm(y, blk["norm_w"], wl.norm_eps)
-    offs = torch.tensor([0, wl.N], dtype=torch.int32, device="cuda")
-    sh = moe.expert_ffn(dev["x"], offs, *[t.unsqueeze(0) for t in blk["shared"]], act)
+    sh = moe.shared_experts(dev["x"], *blk["shared"], act)
     out_p = moe.linear(y, blk["up_proj"], residual=sh)
     assert torch.equal(out_b.view(torch.int16), out_p.view(torch.int16))
+
+
+@pytest.mark.parametrize("M,d,F,act", [(64, 7168, 3072, "situ"), (1, 7168, 3072, "silu"),
+                                       (100, 512, 256, "silu"), (600, 256, 384, "situ")])
+def test_shared_experts(moe, M, d, F, act):
+    """The shared experts' MLP (split over K at small M) against the reference
+    expert MLP, with and without a residual."""
+    rng = np.random.default_rng(M + d + F)
+    x = _rand_bf16(rng, (M, d))
+    w1, w3 = _rand_bf16(rng, (F, d), 0.02), _rand_bf16(rng, (F, d), 0.02)
+    w2 = _rand_bf16(rng, (d, F), 0.02)
+    res = _rand_bf16(rng, (M, d))
+    a = moe.ActConfig(act, 4.0, 8.0) if act == "situ" else moe.ActConfig("silu")
+    y_g = host_bf16(moe.shared_experts(dev_bf16(x), dev_bf16(w1), dev_bf16(w3), dev_bf16(w2), a))
+    rows = np.arange(M) if M <= 100 else np.array([0, 1, 255, 256, M - 1])
+    y_r = oracle.expert_ffn(np.ascontiguousarray(x[rows]), w1, w3, w2, a.kind, a.beta,
+                            a.linear_beta)
+    err = rel_l2(y_g[rows], y_r)
+    print(f"M={M} d={d} F={F}: rel_l2 {err:.2e}")
+    assert err <= REL_L2_OUT
+    z_g = host_bf16(moe.shared_experts(dev_bf16(x), dev_bf16(w1), dev_bf16(w3), dev_bf16(w2), a,
+                                       residual=dev_bf16(res)))
+    assert np.array_equal(z_g, oracle.add(y_g, res))
+

@@ -408,3 +408,22 @@ def test_expert_ffn_mid_tiles(moe, act):
     counts = np.random.default_rng(9).integers(20, 200, 12)
     counts[4] = 0
     _expert_case(moe, wl, counts, list(range(12)), rows_per_expert=64)
+
+
+@pytest.mark.parametrize("name,N,E", [("dsv32_decode", 128, 256), ("tiny", 64, 16),
+                                      ("k2_prefill", 1024, 96), ("k3_latent_decode", 64, 896),
+                                      ("k2_prefill", 5, 384)])
+def test_expert_ffn_gathered_equals_the_separate_gather(moe, name, N, E):
+    """moe_expert_ffn_gathered (rows gathered inside the w1/w3 kernel by
+    tile::gather4) equals moe_expert_ffn on moe_dispatch's gathered copy, bit
+    for bit: the MMAs see the same rows in the same order."""
+    import torch
+    wl = scaled(WORKLOADS[name], N=N, E=E)
+    dev = synth.workloads.dev_inputs(wl)
+    act = acfg(moe, wl)
+    x_e = dev["x_e"] if wl.latent else dev["x"]
+    idx, w = moe.route(dev["x"], dev["W"], dev["bias"], rcfg(moe, wl))
+    counts, offsets, perm, pos, xs = moe.dispatch(idx, x_e, wl.E)
+    y_sep = moe.expert_ffn(xs, offsets, dev["w1"], dev["w3"], dev["w2"], act)
+    y_g = moe.expert_ffn_gathered(x_e, wl.K, perm, offsets, dev["w1"], dev["w3"], dev["w2"], act)
+    assert torch.equal(y_g.view(torch.int16), y_sep.view(torch.int16))
