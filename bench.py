@@ -9,7 +9,14 @@ expert weights (22.5 GB) are larger than L2 and L2 is also flushed (256 MB
 write) between steps, outside the per-step events.  Under torchrun every rank
 runs its own batch (token rows rank*N .. rank*N+N-1) with the same weights:
 weak scaling with no collective on the data path; the step time is the max
-over ranks.  Rank 0 prints one JSON line.
+over ranks.  Rank 0 prints one JSON line.  `--workload k3_block_decode` (or
+tiny_block) times the whole MoE block instead (moe_block_forward: gate,
+shared experts, latent projections and norm around the routed layer).
+
+The `e2e` figure is the same step through the public API from pinned host
+memory, each step uploading its tokens and downloading its output; the
+copies of neighbouring steps overlap on two copy streams (double-buffered),
+and the timed region spans the first upload to the last download.
 
 --impl reference times the CPU reference (oracle/) on the host cores on a
 bounded sample of the same workload; it is the slow reference arm, not a
@@ -68,7 +75,15 @@ def parse():
     p.add_argument("--tokens", type=int, default=None)
     p.add_argument("--experts", type=int, default=None)
     p.add_argument("--ffn", type=int, default=None)
+    # router variants ("DeepSeek-V3.2-Exp · Affinities", gate-forward)
+    p.add_argument("--score-func", default="sigmoid", choices=["sigmoid", "softmax"])
+    p.add_argument("--group-score", default="top2_sum", choices=["top2_sum", "max"])
     return p.parse_args()
+
+
+def route_cfg(moe, wl, args):
+    return moe.RouteConfig(wl.E, wl.G, wl.TG, wl.K, wl.route_scale, wl.norm,
+                           score_func=args.score_func, group_score=args.group_score)
 
 
 def workload_of(args):
@@ -169,6 +184,55 @@ def aggregate_throughput(tokens_per_rank, world, step_ms_max):
     return world * tokens_per_rank / (step_ms_max * 1e-3)
 
 
+def e2e_pipelined(torch, steps, hosts, run, out_like):
+    """Milliseconds per step end to end through the public API from pinned
+    host memory.  Every step uploads its inputs (`hosts`) and downloads its
+    output; the upload of step i runs on one copy stream while step i-1
+    computes and its download on another while step i+1 computes (two device
+    buffers each), the way a serving loop would run.  The timed region spans
+    the first upload to the last download, so every copy is inside it."""
+    comp = torch.cuda.current_stream()
+    up, down = torch.cuda.Stream(), torch.cuda.Stream()
+    devs = [[torch.empty(h.shape, dtype=h.dtype, device="cuda") for h in hosts] for _ in range(2)]
+    outs = [torch.empty_like(out_like) for _ in range(2)]
+    outs_h = [torch.empty(tuple(out_like.shape), dtype=out_like.dtype, pin_memory=True)
+              for _ in range(2)]
+    uploaded = [torch.cuda.Event() for _ in range(2)]
+    computed = [torch.cuda.Event() for _ in range(2)]
+    downloaded = [torch.cuda.Event() for _ in range(2)]
+
+    def one(i):
+        b = i & 1
+        with torch.cuda.stream(up):
+            if i >= 2:
+                up.wait_event(computed[b])  # the step that read buffer b is done
+            for d, h in zip(devs[b], hosts):
+                d.copy_(h, non_blocking=True)
+            uploaded[b].record(up)
+        comp.wait_event(uploaded[b])
+        if i >= 2:
+            comp.wait_event(downloaded[b])  # output buffer b has been read back
+        run(devs[b], outs[b])
+        computed[b].record(comp)
+        with torch.cuda.stream(down):
+            down.wait_event(computed[b])
+            outs_h[b].copy_(outs[b], non_blocking=True)
+            downloaded[b].record(down)
+
+    for i in range(3):
+        one(i)
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(comp)
+    up.wait_stream(comp)
+    for i in range(steps):
+        one(i)
+    comp.wait_stream(down)
+    t1.record(comp)
+    t1.synchronize()
+    return t0.elapsed_time(t1) / steps
+
+
 # ---------------------------------------------------------------- our arm
 def run_ours(args, rank, world, local_rank):
     import torch
@@ -179,7 +243,7 @@ def run_ours(args, rank, world, local_rank):
     wl = workload_of(args)
     torch.cuda.set_device(local_rank)
     dev = dev_inputs(wl, rank=rank)
-    cfg = moe.RouteConfig(wl.E, wl.G, wl.TG, wl.K, wl.route_scale, wl.norm)
+    cfg = route_cfg(moe, wl, args)
     act = moe.ActConfig(wl.act, wl.beta, wl.lbeta)
     x_e = dev["x_e"] if wl.latent else None
     ws = moe.workspace(moe.workspace_size(wl.N, wl.d_r, wl.d_e, cfg, wl.F))
@@ -218,7 +282,8 @@ def run_ours(args, rank, world, local_rank):
         torch.cuda.synchronize()
         barrier()
         wall = time.perf_counter() - t0
-    ms = statistics.mean(a.elapsed_time(b) for a, b in ev0)
+    per_step = [a.elapsed_time(b) for a, b in ev0]
+    ms = statistics.mean(per_step)
 
     # breakdown pass: the same steps with an event after every stage (events
     # between the two expert kernels hold back the second one's early start,
@@ -247,38 +312,19 @@ def run_ours(args, rank, world, local_rank):
     counts = np.bincount(counts_probe.cpu().numpy().ravel(), minlength=wl.E)
     touched = int((counts > 0).sum())
 
-    # end to end through the public API from pinned host buffers
-    x_host = torch.empty((wl.N, wl.d_r), dtype=torch.bfloat16, pin_memory=True)
-    x_host.copy_(dev["x"].cpu())
-    xe_host = None
+    # end to end through the public API from pinned host buffers (weights
+    # larger than L2; copies of neighbouring steps overlapped)
+    hosts = [torch.empty((wl.N, wl.d_r), dtype=torch.bfloat16, pin_memory=True)]
+    hosts[0].copy_(dev["x"].cpu())
     if wl.latent:
-        xe_host = torch.empty((wl.N, wl.d_e), dtype=torch.bfloat16, pin_memory=True)
-        xe_host.copy_(dev["x_e"].cpu())
-    out_host = torch.empty((wl.N, wl.d_e), dtype=torch.bfloat16, pin_memory=True)
-    x_dev = torch.empty_like(dev["x"])
-    xe_dev = torch.empty_like(dev["x_e"]) if wl.latent else None
+        hosts.append(torch.empty((wl.N, wl.d_e), dtype=torch.bfloat16, pin_memory=True))
+        hosts[1].copy_(dev["x_e"].cpu())
 
-    def e2e_step():
-        x_dev.copy_(x_host, non_blocking=True)
-        if wl.latent:
-            xe_dev.copy_(xe_host, non_blocking=True)
-        moe.forward(x_dev, dev["W"], dev["bias"], cfg, dev["w1"], dev["w3"], dev["w2"], act,
-                    x_e=xe_dev, ws=ws, out=out)
-        out_host.copy_(out, non_blocking=True)
+    def e2e_run(xs_dev, o):
+        moe.forward(xs_dev[0], dev["W"], dev["bias"], cfg, dev["w1"], dev["w3"], dev["w2"], act,
+                    x_e=xs_dev[1] if wl.latent else None, ws=ws, out=o)
 
-    for _ in range(3):
-        flush.zero_()
-        e2e_step()
-    torch.cuda.synchronize()
-    e2e_ms = []
-    for _ in range(args.steps):
-        flush.zero_()
-        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        s.record()
-        e2e_step()
-        e.record()
-        e.synchronize()
-        e2e_ms.append(s.elapsed_time(e))
+    e2e_ms = [e2e_pipelined(torch, args.steps, hosts, e2e_run, out)]
     h2d = wl.N * wl.d_r * 2 + (wl.N * wl.d_e * 2 if wl.latent else 0)
     d2h = wl.N * wl.d_e * 2
 
@@ -287,6 +333,7 @@ def run_ours(args, rank, world, local_rank):
 
     res = {
         "ms": ms_max, "e2e_ms": e2e_max, "stage_ms": stage_ms, "gate_up_ms": gu_ms,
+        "step_ms": [min(per_step), statistics.median(per_step), max(per_step)],
         "touched": touched, "counts_max": int(counts.max()), "clocks": clk.summary(),
         "h2d": h2d, "d2h": d2h, "wall_s": wall_max,
     }
@@ -337,7 +384,7 @@ def run_block(args, rank, world, local_rank):
                          w2=dev["w2"], down_proj=blk["down_proj"], norm_weight=blk["norm_w"],
                          up_proj=blk["up_proj"], shared_w1=sh[0], shared_w3=sh[1],
                          shared_w2=sh[2])
-    cfg = moe.RouteConfig(wl.E, wl.G, wl.TG, wl.K, wl.route_scale, wl.norm)
+    cfg = route_cfg(moe, wl, args)
     act = moe.ActConfig(wl.act, wl.beta, wl.lbeta)
     out = torch.empty((wl.N, wl.d_r), dtype=torch.bfloat16, device="cuda")
     idx = torch.empty((wl.N, wl.K), dtype=torch.int32, device="cuda")
@@ -384,29 +431,13 @@ def run_block(args, rank, world, local_rank):
     counts = np.bincount(idx.cpu().numpy().ravel(), minlength=wl.E)
     touched = int((counts > 0).sum())
 
-    x_host = torch.empty((wl.N, wl.d_r), dtype=torch.bfloat16, pin_memory=True)
-    x_host.copy_(dev["x"].cpu())
-    out_host = torch.empty((wl.N, wl.d_r), dtype=torch.bfloat16, pin_memory=True)
-    x_dev = torch.empty_like(dev["x"])
+    hosts = [torch.empty((wl.N, wl.d_r), dtype=torch.bfloat16, pin_memory=True)]
+    hosts[0].copy_(dev["x"].cpu())
 
-    def e2e_step():
-        x_dev.copy_(x_host, non_blocking=True)
-        step(x_dev)
-        out_host.copy_(out, non_blocking=True)
+    def e2e_run(xs_dev, o):
+        moe.block_forward(xs_dev[0], W, cfg, act, norm_eps=wl.norm_eps, ws=ws[0], out=o)
 
-    for _ in range(3):
-        flush.zero_()
-        e2e_step()
-    torch.cuda.synchronize()
-    e2e_ms = []
-    for _ in range(args.steps):
-        flush.zero_()
-        s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        s0.record()
-        e2e_step()
-        s1.record()
-        s1.synchronize()
-        e2e_ms.append(s0.elapsed_time(s1))
+    e2e_ms = [e2e_pipelined(torch, args.steps, hosts, e2e_run, out)]
     ms_max, e2e_max, wall_max = max_over_ranks([ms, statistics.mean(e2e_ms), wall], world, "cuda")
     return wl, {"ms": ms_max, "e2e_ms": e2e_max, "touched": touched, "clocks": clk.summary(),
                 "h2d": wl.N * wl.d_r * 2, "d2h": wl.N * wl.d_r * 2, "wall_s": wall_max}
@@ -422,6 +453,7 @@ def block_line(args, wl, r, world):
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": wl.name, "N": wl.N, "d_r": wl.d_r, "d_e": wl.d_e, "E": wl.E,
                    "K": wl.K, "F": wl.F, "F_shared": wl.F_shared, "act": wl.act,
+                   "router": f"{args.score_func}/{args.group_score}",
                    "global_batch": world * wl.N, "parallelism": f"dp{world}",
                    "l2": "weights > L2, plus a 256 MB write between steps outside the "
                          "per-step events"},
@@ -506,6 +538,36 @@ def oracle_sample(wl, n_experts=8):
     }
 
 
+def oracle_sample_block(wl, n_experts=8, n_tokens=4):
+    """The CPU reference on a bounded sample of a whole-block step: the routed
+    layer as oracle_sample; the latent projections and the norm on all
+    tokens; the shared experts on `n_tokens` tokens, scaled to all."""
+    import oracle
+    from synth.workloads import host_block, host_inputs
+
+    r = oracle_sample(wl, n_experts)
+    hb = host_block(wl)
+    x = host_inputs(wl)["x"]
+    t = dict(r["seconds"])
+    if wl.latent:
+        t0 = time.perf_counter()
+        xe = oracle.linear(x, hb["down_proj"])
+        y = oracle.rms_norm(xe, hb["norm_w"], wl.norm_eps)  # a stand-in row block of the width
+        oracle.linear(y, hb["up_proj"])
+        t["projections_norm"] = time.perf_counter() - t0
+    if wl.F_shared:
+        n = min(n_tokens, wl.N)
+        t0 = time.perf_counter()
+        oracle.expert_ffn(np.ascontiguousarray(x[:n]), *hb["shared"], wl.act, wl.beta, wl.lbeta)
+        t["shared"] = (time.perf_counter() - t0) * wl.N / n
+    total = sum(t.values())
+    return {"value": wl.N / total, "cores": r["cores"], "seconds": t,
+            "sample": r["sample"] + (f"; down/up projections and norm on all {wl.N} tokens"
+                                     if wl.latent else "") +
+                      (f"; shared experts on {min(n_tokens, wl.N)} tokens, time scaled to "
+                       f"{wl.N}" if wl.F_shared else "")}
+
+
 def run_reference(args, rank, world):
     if rank != 0:
         return
@@ -515,13 +577,16 @@ def run_reference(args, rank, world):
     vals = []
     t_start = time.perf_counter()
     res = None
+    from synth.workloads import BLOCKS
+    block = args.workload in BLOCKS
     for _ in range(args.steps):
-        res = oracle_sample(wl)
+        res = oracle_sample_block(wl) if block else oracle_sample(wl)
         vals.append(res["value"])
     wall = time.perf_counter() - t_start
     v = statistics.mean(vals)
     line = {
-        "impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": args.gpus,
+        "impl": "reference", "metric": BLOCK_METRIC if block else METRIC, "value": v,
+        "unit": UNIT, "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * wl.N / v,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic", "config": {"workload": wl.name, "N": wl.N, "d_r": wl.d_r,
@@ -553,6 +618,10 @@ def main():
     if args.workload in BLOCKS:
         wl, r = run_block(args, rank, world, local_rank)
         line = block_line(args, wl, r, world)
+        if rank == 0 and world == 1 and not args.no_cpu_baseline:
+            cb = oracle_sample_block(wl)
+            line["cpu_baseline"] = {"value": cb["value"], "unit": UNIT, "cores": cb["cores"],
+                                    "kind": "oracle", "sample": cb["sample"]}
         if world > 1:
             import torch.distributed as dist
             dist.barrier()
@@ -578,6 +647,7 @@ def main():
         "data": "synthetic",
         "config": {"workload": wl.name, "N": wl.N, "d_r": wl.d_r, "d_e": wl.d_e, "E": wl.E,
                    "n_group": wl.G, "topk_group": wl.TG, "K": wl.K, "F": wl.F, "act": wl.act,
+                   "router": f"{args.score_func}/{args.group_score}",
                    "global_batch": world * wl.N, "parallelism": f"dp{world}",
                    "l2": "expert weights > L2, plus a 256 MB write between steps outside the "
                          "per-step events"},
@@ -586,6 +656,7 @@ def main():
                      "frac": achieved / peaks["hbm_gbs"], "traffic": gate_up_traffic(r["touched"]),
                      "peak_source": peaks["source"], "touched_experts": r["touched"]},
         "stages_ms": r["stage_ms"],
+        "step_ms_min_median_max": r["step_ms"],
         "e2e": {"value": aggregate_throughput(wl.N, world, r["e2e_ms"]), "unit": UNIT,
                 "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"]},
         "gpu_launches": kernels_per_step(wl) * args.steps,
