@@ -492,7 +492,7 @@ def gate_up_bytes(wl, touched):
 
 
 # ------------------------------------------------------------ oracle arm
-def oracle_sample(wl, n_experts=8):
+def oracle_sample(wl, n_experts=8, router=("sigmoid", "top2_sum")):
     """Time the CPU reference on a bounded sample of the workload.
 
     Route, dispatch and combine run on the whole batch; the expert MLP runs on
@@ -509,7 +509,11 @@ def oracle_sample(wl, n_experts=8):
     t = {}
     t0 = time.perf_counter()
     idx, w, _ = oracle.route(inp["x"], inp["W"], inp["bias"], wl.G, wl.TG, wl.K,
-                             wl.route_scale, wl.norm)
+                             wl.route_scale, wl.norm,
+                             score={"sigmoid": oracle.SCORE_SIGMOID,
+                                    "softmax": oracle.SCORE_SOFTMAX}[router[0]],
+                             group={"top2_sum": oracle.GROUP_TOP2_SUM,
+                                    "max": oracle.GROUP_MAX}[router[1]])
     t["route"] = time.perf_counter() - t0
     t0 = time.perf_counter()
     counts, offsets, perm, pos = oracle.dispatch(idx, wl.E)
@@ -538,14 +542,14 @@ def oracle_sample(wl, n_experts=8):
     }
 
 
-def oracle_sample_block(wl, n_experts=8, n_tokens=4):
+def oracle_sample_block(wl, n_experts=8, n_tokens=4, router=("sigmoid", "top2_sum")):
     """The CPU reference on a bounded sample of a whole-block step: the routed
     layer as oracle_sample; the latent projections and the norm on all
     tokens; the shared experts on `n_tokens` tokens, scaled to all."""
     import oracle
     from synth.workloads import host_block, host_inputs
 
-    r = oracle_sample(wl, n_experts)
+    r = oracle_sample(wl, n_experts, router)
     hb = host_block(wl)
     x = host_inputs(wl)["x"]
     t = dict(r["seconds"])
@@ -580,7 +584,8 @@ def run_reference(args, rank, world):
     from synth.workloads import BLOCKS
     block = args.workload in BLOCKS
     for _ in range(args.steps):
-        res = oracle_sample_block(wl) if block else oracle_sample(wl)
+        rt = (args.score_func, args.group_score)
+        res = oracle_sample_block(wl, router=rt) if block else oracle_sample(wl, router=rt)
         vals.append(res["value"])
     wall = time.perf_counter() - t_start
     v = statistics.mean(vals)
@@ -590,7 +595,8 @@ def run_reference(args, rank, world):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * wl.N / v,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic", "config": {"workload": wl.name, "N": wl.N, "d_r": wl.d_r,
-                                        "d_e": wl.d_e, "E": wl.E, "K": wl.K, "F": wl.F},
+                                        "d_e": wl.d_e, "E": wl.E, "K": wl.K, "F": wl.F,
+                                        "router": f"{args.score_func}/{args.group_score}"},
         "cpu_baseline": {"value": v, "unit": UNIT, "cores": res["cores"], "kind": "oracle",
                          "sample": res["sample"]},
         "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -619,7 +625,7 @@ def main():
         wl, r = run_block(args, rank, world, local_rank)
         line = block_line(args, wl, r, world)
         if rank == 0 and world == 1 and not args.no_cpu_baseline:
-            cb = oracle_sample_block(wl)
+            cb = oracle_sample_block(wl, router=(args.score_func, args.group_score))
             line["cpu_baseline"] = {"value": cb["value"], "unit": UNIT, "cores": cb["cores"],
                                     "kind": "oracle", "sample": cb["sample"]}
         if world > 1:
@@ -663,7 +669,7 @@ def main():
         "clocks": r["clocks"],
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cb = oracle_sample(wl)
+        cb = oracle_sample(wl, router=(args.score_func, args.group_score))
         line["cpu_baseline"] = {"value": cb["value"], "unit": UNIT, "cores": cb["cores"],
                                 "kind": "oracle", "sample": cb["sample"]}
     if world > 1:
