@@ -22,6 +22,8 @@ __global__ void __launch_bounds__(32 * kWarps) k_combine(const __nv_bfloat16* __
                                                          __nv_bfloat16* __restrict__ out,
                                                          const __nv_bfloat16* __restrict__ res,
                                                          DeviceStatus* st) {
+  pdl_wait();
+  pdl_trigger();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nv = d / 8;
   const int nch = (nv + 31) / 32;
@@ -129,6 +131,8 @@ __global__ void __launch_bounds__(32 * kWarps) k_rms_norm(const __nv_bfloat16* _
                                                           const __nv_bfloat16* __restrict__ w,
                                                           float eps,
                                                           __nv_bfloat16* __restrict__ out) {
+  pdl_wait();
+  pdl_trigger();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nv = d / 8;
   for (int64_t t = (int64_t)blockIdx.x * kWarps + warp; t < N; t += (int64_t)gridDim.x * kWarps) {
@@ -160,6 +164,8 @@ __global__ void __launch_bounds__(32 * kWarps) k_combine_rms_norm(
     const float* __restrict__ w, int64_t N, int K, int d, int64_t S,
     const __nv_bfloat16* __restrict__ norm_w, float eps, __nv_bfloat16* __restrict__ out,
     DeviceStatus* st) {
+  pdl_wait();
+  pdl_trigger();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nv = d / 8;
   for (int64_t t = (int64_t)blockIdx.x * kWarps + warp; t < N; t += (int64_t)gridDim.x * kWarps) {
@@ -233,8 +239,8 @@ cudaError_t launch_combine(const __nv_bfloat16* y, const int32_t* pos, const flo
   int64_t blocks = (items + kWarps - 1) / kWarps;
   const int64_t cap = (int64_t)dev_info()->sm_count * 16;
   if (blocks > cap) blocks = cap;
-  k_combine<<<(unsigned)blocks, 32 * kWarps, 0, s>>>(y, pos, w, N, K, d_e, S, out, residual, st);
-  return cudaGetLastError();
+  return launch_pdl(k_combine, dim3((unsigned)blocks), dim3(32 * kWarps), 0, s, y, pos, w, N, K,
+                    d_e, S, out, residual, st);
 }
 
 // d <= 256 * NV columns; the smallest register footprint that holds the row
@@ -242,17 +248,19 @@ cudaError_t launch_combine(const __nv_bfloat16* y, const int32_t* pos, const flo
   do {                                                                          \
     const int nvl = (d + 255) / 256;                                            \
     const unsigned g = (unsigned)row_blocks(N);                                 \
-    if (nvl <= 4) KERNEL<4><<<g, 32 * kWarps, 0, s>>>(__VA_ARGS__);             \
-    else if (nvl <= 8) KERNEL<8><<<g, 32 * kWarps, 0, s>>>(__VA_ARGS__);        \
-    else if (nvl <= 16) KERNEL<16><<<g, 32 * kWarps, 0, s>>>(__VA_ARGS__);      \
-    else KERNEL<kMaxNormVecs><<<g, 32 * kWarps, 0, s>>>(__VA_ARGS__);           \
+    if (nvl <= 4) e = launch_pdl(KERNEL<4>, dim3(g), dim3(32 * kWarps), 0, s, __VA_ARGS__);  \
+    else if (nvl <= 8) e = launch_pdl(KERNEL<8>, dim3(g), dim3(32 * kWarps), 0, s, __VA_ARGS__); \
+    else if (nvl <= 16)                                                          \
+      e = launch_pdl(KERNEL<16>, dim3(g), dim3(32 * kWarps), 0, s, __VA_ARGS__);  \
+    else e = launch_pdl(KERNEL<kMaxNormVecs>, dim3(g), dim3(32 * kWarps), 0, s, __VA_ARGS__); \
   } while (0)
 
 cudaError_t launch_rms_norm(const __nv_bfloat16* x, int64_t N, int d, const __nv_bfloat16* w,
                             float eps, __nv_bfloat16* out, cudaStream_t s) {
   if (d > kMaxNormVecs * 256) return cudaErrorInvalidValue;
+  cudaError_t e;
   MOE_NORM_DISPATCH(k_rms_norm, x, N, d, w, eps, out);
-  return cudaGetLastError();
+  return e;
 }
 
 cudaError_t launch_combine_rms_norm(const __nv_bfloat16* y, const int32_t* pos, const float* w,
@@ -261,8 +269,9 @@ cudaError_t launch_combine_rms_norm(const __nv_bfloat16* y, const int32_t* pos, 
                                     __nv_bfloat16* out, DeviceStatus* st, cudaStream_t s) {
   const int d = d_e;
   if (d > kMaxNormVecs * 256) return cudaErrorInvalidValue;
+  cudaError_t e;
   MOE_NORM_DISPATCH(k_combine_rms_norm, y, pos, w, N, K, d, S, norm_w, eps, out, st);
-  return cudaGetLastError();
+  return e;
 }
 
 }  // namespace moe

@@ -32,6 +32,8 @@ __device__ __forceinline__ unsigned lanemask_lt() {
 __global__ void __launch_bounds__(32 * kWarps) k_hist(const int32_t* __restrict__ idx, int64_t S,
                                                       int E, int CH, int nchunks,
                                                       int32_t* __restrict__ cc, DeviceStatus* st) {
+  pdl_wait();
+  pdl_trigger();
   extern __shared__ int32_t cnt_all[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int c = blockIdx.x * kWarps + warp;
@@ -63,6 +65,8 @@ __global__ void __launch_bounds__(32 * kWarps) k_hist(const int32_t* __restrict_
 __global__ void __launch_bounds__(1024) k_scan(int32_t* __restrict__ cc, int nchunks, int E,
                                                int32_t* __restrict__ counts,
                                                int32_t* __restrict__ offsets) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ int32_t warp_tot[32];
   const int e = threadIdx.x;
   const int lane = e & 31, warp = e >> 5;
@@ -107,6 +111,8 @@ __global__ void __launch_bounds__(32 * kWarps) k_scatter(const int32_t* __restri
                                                          const int32_t* __restrict__ cc,
                                                          int32_t* __restrict__ perm,
                                                          int32_t* __restrict__ pos) {
+  pdl_wait();
+  pdl_trigger();
   extern __shared__ int32_t base_all[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int c = blockIdx.x * kWarps + warp;
@@ -147,6 +153,8 @@ __global__ void __launch_bounds__(32 * kWarps) k_scatter(const int32_t* __restri
 __global__ void __launch_bounds__(256) k_gather(const __nv_bfloat16* __restrict__ x, int64_t N,
                                                 int K, int d, const int32_t* __restrict__ pos,
                                                 __nv_bfloat16* __restrict__ xs) {
+  pdl_wait();
+  pdl_trigger();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nv = d / 8;
   const int nch = (nv + 31) / 32;
@@ -168,6 +176,8 @@ __global__ void __launch_bounds__(256) k_gather(const __nv_bfloat16* __restrict_
 __global__ void __launch_bounds__(1024) k_counts_offsets(const int32_t* __restrict__ counts, int n,
                                                          int32_t* __restrict__ offsets,
                                                          DeviceStatus* st) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ int32_t warp_tot[32];
   const int i = threadIdx.x, lane = i & 31, warp = i >> 5;
   int32_t c = 0;
@@ -205,8 +215,7 @@ __global__ void __launch_bounds__(1024) k_counts_offsets(const int32_t* __restri
 
 cudaError_t launch_counts_offsets(const int32_t* counts, int n, int32_t* offsets,
                                   DeviceStatus* st, cudaStream_t s) {
-  k_counts_offsets<<<1, 1024, 0, s>>>(counts, n, offsets, st);
-  return cudaGetLastError();
+  return launch_pdl(k_counts_offsets, dim3(1), dim3(1024), 0, s, counts, n, offsets, st);
 }
 
 int dispatch_chunks(int64_t S) {
@@ -237,15 +246,19 @@ cudaError_t launch_dispatch(const int32_t* idx, int64_t N, int K, int E, const _
   const int nchunks = dispatch_chunks(S);
   const size_t smem = sizeof(int32_t) * (size_t)E * kWarps;
   const unsigned blocks = (unsigned)((nchunks + kWarps - 1) / kWarps);
-  k_hist<<<blocks, 32 * kWarps, smem, s>>>(idx, S, E, CH, nchunks, scratch, st);
-  k_scan<<<1, 1024, 0, s>>>(scratch, nchunks, E, counts, offsets);
-  k_scatter<<<blocks, 32 * kWarps, smem, s>>>(idx, S, E, CH, nchunks, scratch, perm, pos);
-  if (!xs) return cudaGetLastError();
+  cudaError_t e;
+  if ((e = launch_pdl(k_hist, dim3(blocks), dim3(32 * kWarps), smem, s, idx, S, E, CH, nchunks,
+                      scratch, st)) != cudaSuccess ||
+      (e = launch_pdl(k_scan, dim3(1), dim3(1024), 0, s, scratch, nchunks, E, counts,
+                      offsets)) != cudaSuccess ||
+      (e = launch_pdl(k_scatter, dim3(blocks), dim3(32 * kWarps), smem, s, idx, S, E, CH,
+                      nchunks, scratch, perm, pos)) != cudaSuccess)
+    return e;
+  if (!xs) return cudaSuccess;
   int64_t gb = (N * ((d_e / 8 + 31) / 32) + 7) / 8;
   const int64_t cap = (int64_t)dev_info()->sm_count * 16;
   if (gb > cap) gb = cap;
-  k_gather<<<(unsigned)gb, 256, 0, s>>>(x_e, N, K, d_e, pos, xs);
-  return cudaGetLastError();
+  return launch_pdl(k_gather, dim3((unsigned)gb), dim3(256), 0, s, x_e, N, K, d_e, pos, xs);
 }
 
 }  // namespace moe

@@ -986,6 +986,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 __global__ void __launch_bounds__(1024) k_tiles(const int32_t* __restrict__ offsets, int E,
                                                 int64_t S, int nt, int32_t* __restrict__ tile_start,
                                                 DeviceStatus* st) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ int32_t warp_tot[32];
   const int e = threadIdx.x, lane = e & 31, warp = e >> 5;
   int32_t n = 0;
@@ -1224,8 +1226,9 @@ int expert_ffn_run(const __nv_bfloat16* xs, const int32_t* offsets, int E, int64
     return MOE_ERR_CUDA;
   const Variant var = pick_variant(S, E);
   const int nt = var == kVarDecode ? kNtDecode : (var == kVarMid ? kNtMid : kPairNt);
-  k_tiles<<<1, 1024, 0, s>>>(offsets, E, S, nt, tile_start, st);
-  if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
+  if (launch_pdl(k_tiles, dim3(1), dim3(1024), 0, s, offsets, E, S, nt, tile_start, st) !=
+      cudaSuccess)
+    return MOE_ERR_CUDA;
   cudaError_t rc;
   if (gather) {
     // token rows straight from x_e (no xs): decode and mid variants only
@@ -1265,6 +1268,8 @@ __global__ void __launch_bounds__(256) k_splitk_reduce(const float* __restrict__
                                                        const __nv_bfloat16* __restrict__ res,
                                                        __nv_bfloat16* __restrict__ out,
                                                        int act_kind, float beta, float lbeta) {
+  pdl_wait();
+  pdl_trigger();
   const bool has_lb = !(lbeta == 0.0f || lbeta != lbeta);
   const float b_eff = (beta == 0.0f || beta != beta) ? 1.0f : beta;
   const int64_t ld = MODE == kGateUp ? 2 * (int64_t)cols : cols;
@@ -1354,10 +1359,9 @@ cudaError_t launch_dense(Variant var, const CUtensorMap& a0, const CUtensorMap& 
   int64_t blocks = (n4 + 255) / 256;
   const int64_t cap = (int64_t)dev_info()->sm_count * 8;
   if (blocks > cap) blocks = cap;
-  k_splitk_reduce<MODE><<<(unsigned)blocks, 256, 0, s>>>(part, ksplit, M, M_rows, res, out,
-                                                         (int)act.kind, act.beta,
-                                                         act.linear_beta);
-  return cudaGetLastError();
+  return launch_pdl(k_splitk_reduce<MODE>, dim3((unsigned)blocks), dim3(256), 0, s,
+                    (const float*)part, ksplit, M, M_rows, res, out, (int)act.kind, act.beta,
+                    act.linear_beta);
 }
 }  // namespace
 
@@ -1369,6 +1373,8 @@ size_t dense_part_bytes(int64_t M, int K, int Nout, bool gate_up) {
 }
 
 __global__ void k_dense_tiles(int64_t M, int32_t* __restrict__ tiles) {
+  pdl_wait();
+  pdl_trigger();
   if (threadIdx.x == 0) {
     tiles[0] = 0;  // offsets
     tiles[1] = (int32_t)M;
@@ -1382,8 +1388,7 @@ __global__ void k_dense_tiles(int64_t M, int32_t* __restrict__ tiles) {
 }
 
 cudaError_t launch_dense_tiles(int64_t M, int32_t* tiles, cudaStream_t s) {
-  k_dense_tiles<<<1, 32, 0, s>>>(M, tiles);
-  return cudaGetLastError();
+  return launch_pdl(k_dense_tiles, dim3(1), dim3(32), 0, s, M, tiles);
 }
 
 int linear_run(const __nv_bfloat16* x, int64_t M, int K, const __nv_bfloat16* W, int Nout,

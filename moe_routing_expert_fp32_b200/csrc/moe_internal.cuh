@@ -28,6 +28,35 @@ constexpr uint32_t kSpinLimit = 1u << 28;
 
 inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
+// ------------------------------------------- programmatic dependent launch
+// The short kernels of the layer are launched as programmatic dependents of
+// the kernel before them on the stream (launch_pdl): their CTAs may be
+// scheduled while that kernel is still running, which hides the launch
+// latency between back-to-back small kernels.  Each such kernel starts with
+// pdl_wait() (no read or write of memory the predecessor touches before it),
+// then pdl_trigger() so that its own dependent can be scheduled in turn.
+// Launched without the attribute, both instructions return at once.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t s, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
 // --------------------------------------------------------- kernel launches
 // (all enqueue on `stream`, no synchronisation)
 

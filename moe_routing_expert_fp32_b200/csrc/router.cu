@@ -43,6 +43,8 @@ __global__ void __launch_bounds__(256, 2) k_gate_partial(const __nv_bfloat16* __
                                                          int cps, int splits,
                                                          float* __restrict__ logits,
                                                          double* __restrict__ part) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ __align__(16) float xs[2][GK][GT];
   __shared__ __align__(16) float wsm[2][GK][GEP];
   const int tid = threadIdx.x;
@@ -142,6 +144,8 @@ __global__ void __launch_bounds__(256, 2) k_gate_partial(const __nv_bfloat16* __
 __global__ void __launch_bounds__(256) k_reduce_partials(const double* __restrict__ part,
                                                          int splits, int64_t NE,
                                                          float* __restrict__ logits) {
+  pdl_wait();
+  pdl_trigger();
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < NE;
        i += (int64_t)gridDim.x * blockDim.x) {
     double a = 0.0;
@@ -170,6 +174,8 @@ __global__ void __launch_bounds__(32 * kSelWarps) k_select(
     const float* __restrict__ part, int splits, int64_t N, int E, const float* __restrict__ bias,
     int G, int TG, int K, int norm, float route_scale, int score_func, int group_mode,
     int32_t* __restrict__ idx_out, float* __restrict__ w_out, DeviceStatus* st) {
+  pdl_wait();
+  pdl_trigger();
   extern __shared__ float sm[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   float* s_s = sm + warp * 2 * E;
@@ -316,13 +322,17 @@ cudaError_t launch_gate(const __nv_bfloat16* x, int64_t N, int d_r, const float*
   float* logits = route_logits_of(scratch);
   double* part = route_part_of(scratch, N, E);
   dim3 grid((E + GE - 1) / GE, (unsigned)((N + GT - 1) / GT), splits);
-  k_gate_partial<<<grid, 256, 0, s>>>(x, N, d_r, W, E, cps, splits, logits, part);
+  cudaError_t e = launch_pdl(k_gate_partial, grid, dim3(256), 0, s, x, N, d_r, W, E, cps, splits,
+                             logits, part);
+  if (e != cudaSuccess) return e;
   if (splits > 1) {
     const int64_t ne = N * (int64_t)E;
     int64_t blocks = (ne + 255) / 256;
     const int64_t cap = (int64_t)dev_info()->sm_count * 16;
     if (blocks > cap) blocks = cap;
-    k_reduce_partials<<<(unsigned)blocks, 256, 0, s>>>(part, splits, ne, logits);
+    e = launch_pdl(k_reduce_partials, dim3((unsigned)blocks), dim3(256), 0, s,
+                   (const double*)part, splits, ne, logits);
+    if (e != cudaSuccess) return e;
   }
   return cudaGetLastError();
 }
@@ -347,9 +357,11 @@ cudaError_t launch_select(const float* part, int splits, int64_t N, const float*
   int64_t blocks = (N + kSelWarps - 1) / kSelWarps;
   const int64_t cap = (int64_t)dev_info()->sm_count * 16;
   if (blocks > cap) blocks = cap;
-  k_select<<<(unsigned)blocks, 32 * kSelWarps, smem, s>>>(
-      part, splits, N, E, bias, cfg.n_group, cfg.topk_group, cfg.top_k, cfg.norm_topk_prob,
-      cfg.route_scale, cfg.score_func, cfg.group_score, idx, w, st);
+  const cudaError_t e = launch_pdl(
+      k_select, dim3((unsigned)blocks), dim3(32 * kSelWarps), smem, s, part, splits, N, E, bias,
+      cfg.n_group, cfg.topk_group, cfg.top_k, cfg.norm_topk_prob, cfg.route_scale,
+      cfg.score_func, cfg.group_score, idx, w, st);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

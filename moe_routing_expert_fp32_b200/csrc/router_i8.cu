@@ -106,6 +106,8 @@ template <typename T>
 __global__ void __launch_bounds__(256) k_slice_rows(const T* __restrict__ v, int64_t rows, int d,
                                                     int8_t* __restrict__ out,
                                                     int* __restrict__ sig_out) {
+  pdl_wait();
+  pdl_trigger();
   constexpr int VN = Vec<T>::n;
   __shared__ float wmax[8];
   const int64_t row = blockIdx.x;
