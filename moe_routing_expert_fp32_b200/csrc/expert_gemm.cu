@@ -20,7 +20,10 @@
 //     (A 128x64, B NTMAX x64) bf16 tiles guarded by mbarriers; one elected
 //     thread issues tcgen05.mma kind::f16 (bf16 in, fp32 accumulate) into
 //     TMEM; two accumulator buffers let the epilogue of one unit overlap the
-//     MMAs of the next; 4 epilogue warps drain TMEM with tcgen05.ld.
+//     MMAs of the next; 4 epilogue warps drain TMEM with tcgen05.ld and
+//     write bf16 rows with 16-byte stores (an 8 x 8 / 8 x 16 shuffle
+//     transpose per 8-lane group turns one feature per lane into 8
+//     consecutive features per token);
 //   * decode and mid variants can gather their token rows themselves: row i of
 //     a tile is x_e[perm[row0 + i] / K], fetched with tile::gather4 TMA loads
 //     (4 rows of 64 columns each, the same 128-byte swizzle), so no gathered
@@ -265,6 +268,83 @@ __device__ __forceinline__ float situ_mul(float g, float u, float beta, float lb
 // e: the weight index of the unit's segment.  Segment s (rows offsets[s] ..
 // offsets[s+1]) uses weights s % emod: emod = E for the layer, E_local for
 // rows received from several ranks, grouped by (source rank, local expert).
+
+// Stores one 16-token chunk of a down-projection accumulator (lane l holds
+// feature m = m8 + (l & 7) of its 8-lane group, v[j] = token c0 + j) as
+// out[token][feature] with 16-byte stores: the 8 x 16 block of each 8-lane
+// group is transposed by shuffles so that lane i holds tokens 2i and 2i+1 of
+// the group's 8 features.  Every lane of the warp must call it.
+__device__ __forceinline__ void store_down_t8(const float* v, __nv_bfloat16* out, int64_t tok0,
+                                              int ntok, int M_rows, int m8, bool live, int lane) {
+  uint32_t a[8];
+#pragma unroll
+  for (int t = 0; t < 8; ++t) {
+    const __nv_bfloat162 h = __floats2bfloat162_rn(v[2 * t], v[2 * t + 1]);
+    a[t] = *reinterpret_cast<const uint32_t*>(&h);
+  }
+  const int i = lane & 7;
+#pragma unroll
+  for (int s = 1; s < 8; s <<= 1) {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      if ((j & s) == 0) {
+        const bool upper = (i & s) != 0;
+        const uint32_t send = upper ? a[j] : a[j | s];
+        const uint32_t recv = __shfl_xor_sync(0xffffffffu, send, s);
+        if (upper) a[j] = recv;
+        else a[j | s] = recv;
+      }
+    }
+  }
+  // a[j] = feature m8 + j, tokens (2i, 2i+1)
+  uint4 lo, hi;
+  lo.x = __byte_perm(a[0], a[1], 0x5410); hi.x = __byte_perm(a[0], a[1], 0x7632);
+  lo.y = __byte_perm(a[2], a[3], 0x5410); hi.y = __byte_perm(a[2], a[3], 0x7632);
+  lo.z = __byte_perm(a[4], a[5], 0x5410); hi.z = __byte_perm(a[4], a[5], 0x7632);
+  lo.w = __byte_perm(a[6], a[7], 0x5410); hi.w = __byte_perm(a[6], a[7], 0x7632);
+  if (live) {
+    if (2 * i < ntok) *reinterpret_cast<uint4*>(out + (tok0 + 2 * i) * M_rows + m8) = lo;
+    if (2 * i + 1 < ntok) *reinterpret_cast<uint4*>(out + (tok0 + 2 * i + 1) * M_rows + m8) = hi;
+  }
+}
+
+
+// The gate_up epilogue's 8 h values of one feature (lane l: feature f8 +
+// (l & 7), tokens tok0 .. tok0 + 7) stored as out[token][feature] with one
+// 16-byte store per lane: the 8 x 8 block of each 8-lane group is
+// transposed by shuffles so that lane i holds token tok0 + i of the group's
+// 8 features.  Every lane of the warp must call it.
+__device__ __forceinline__ void store_h_t8(const float* h, __nv_bfloat16* out, int64_t tok0,
+                                           int ntok, int M_rows, int f8, bool live, int lane) {
+  uint32_t a[8];
+#pragma unroll
+  for (int t = 0; t < 8; ++t) {
+    const __nv_bfloat16 b = __float2bfloat16_rn(h[t]);
+    a[t] = (uint32_t)(*reinterpret_cast<const uint16_t*>(&b));
+  }
+  const int i = lane & 7;
+#pragma unroll
+  for (int s = 1; s < 8; s <<= 1) {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      if ((j & s) == 0) {
+        const bool upper = (i & s) != 0;
+        const uint32_t send = upper ? a[j] : a[j | s];
+        const uint32_t recv = __shfl_xor_sync(0xffffffffu, send, s);
+        if (upper) a[j] = recv;
+        else a[j | s] = recv;
+      }
+    }
+  }
+  // a[j] = feature f8 + j at token tok0 + i
+  uint4 o;
+  o.x = a[0] | (a[1] << 16);
+  o.y = a[2] | (a[3] << 16);
+  o.z = a[4] | (a[5] << 16);
+  o.w = a[6] | (a[7] << 16);
+  if (live && i < ntok) *reinterpret_cast<uint4*>(out + (tok0 + i) * M_rows + f8) = o;
+}
+
 struct Unit {
   int e, row0, nrows, rb;
 };
@@ -608,7 +688,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int pair = quarter & 1;
         const bool is_g = quarter < 2;
         const int f = r0 + pair * 32 + lane;
-        __nv_bfloat16* col = out + f;
         const bool live = f < M_rows;
         for (int c0 = 0; c0 < w.nrows; c0 += 16, ++xbuf) {
           float v[16];
@@ -624,15 +703,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           const float4 t0 = theirs[0], t1 = theirs[1];
           const float other[8] = {t0.x, t0.y, t0.z, t0.w, t1.x, t1.y, t1.z, t1.w};
           const int cbase = c0 + (is_g ? 0 : 8);
+          float hv[8];
 #pragma unroll
           for (int j = 0; j < 8; ++j) {
             const float g = is_g ? v[j] : other[j];
             const float uu = is_g ? other[j] : v[8 + j];
-            const float h = act_kind == MOE_ACT_SITU ? situ_mul(g, uu, b_eff, lbeta, has_lb)
-                                                     : silu_mul(g, uu);
-            if (live && cbase + j < w.nrows)
-              col[(int64_t)(w.row0 + cbase + j) * M_rows] = __float2bfloat16_rn(h);
+            hv[j] = act_kind == MOE_ACT_SITU ? situ_mul(g, uu, b_eff, lbeta, has_lb)
+                                             : silu_mul(g, uu);
           }
+          store_h_t8(hv, out, w.row0 + cbase, w.nrows - cbase, M_rows, f & ~7, live, lane);
         }
       } else {
         const int m = r0 + quarter * 32 + lane;
@@ -642,6 +721,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           float v[16];
           tmem_ld16(taddr + c0, v);
           int lim = w.nrows - c0 < 16 ? w.nrows - c0 : 16;
+          if (!res) {
+            store_down_t8(v, out, w.row0 + c0, lim, M_rows, m & ~7, lim_m != 0, lane);
+            continue;
+          }
           lim = lim < lim_m ? lim : lim_m;
 #pragma unroll
           for (int j = 0; j < 16; ++j)
@@ -925,7 +1008,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int pair = quarter & 1;
         const bool is_g = quarter < 2;
         const int f = r0 + pair * 32 + lane;
-        __nv_bfloat16* col = out + f;
         const bool live = f < M_rows;
         for (int c0 = 0; c0 < w.nrows; c0 += 16, ++xbuf) {
           float v[16];
@@ -941,15 +1023,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           const float4 t0 = theirs[0], t1 = theirs[1];
           const float other[8] = {t0.x, t0.y, t0.z, t0.w, t1.x, t1.y, t1.z, t1.w};
           const int cbase = c0 + (is_g ? 0 : 8);
+          float hv[8];
 #pragma unroll
           for (int j = 0; j < 8; ++j) {
             const float g = is_g ? v[j] : other[j];
             const float uu = is_g ? other[j] : v[8 + j];
-            const float h = act_kind == MOE_ACT_SITU ? situ_mul(g, uu, b_eff, lbeta, has_lb)
-                                                     : silu_mul(g, uu);
-            if (live && cbase + j < w.nrows)
-              col[(int64_t)(w.row0 + cbase + j) * M_rows] = __float2bfloat16_rn(h);
+            hv[j] = act_kind == MOE_ACT_SITU ? situ_mul(g, uu, b_eff, lbeta, has_lb)
+                                             : silu_mul(g, uu);
           }
+          store_h_t8(hv, out, w.row0 + cbase, w.nrows - cbase, M_rows, f & ~7, live, lane);
         }
       } else {
         const int m = r0 + quarter * 32 + lane;
@@ -959,6 +1041,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           float v[16];
           tmem_ld16(taddr + c0, v);
           int lim = w.nrows - c0 < 16 ? w.nrows - c0 : 16;
+          if (!res) {
+            store_down_t8(v, out, w.row0 + c0, lim, M_rows, m & ~7, lim_m != 0, lane);
+            continue;
+          }
           lim = lim < lim_m ? lim : lim_m;
 #pragma unroll
           for (int j = 0; j < 16; ++j)
@@ -1029,17 +1115,15 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
 EncodeTiledFn encode_fn() {
-  static EncodeTiledFn fn = nullptr;
-  static bool tried = false;
-  if (!tried) {
-    tried = true;
+  static const EncodeTiledFn fn = [] {  // looked up once (thread-safe static)
     void* p = nullptr;
     cudaDriverEntryPointQueryResult q;
     if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
             cudaSuccess &&
         q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(p);
-  }
+      return reinterpret_cast<EncodeTiledFn>(p);
+    return static_cast<EncodeTiledFn>(nullptr);
+  }();
   return fn;
 }
 
@@ -1079,16 +1163,13 @@ cudaError_t launch_gemm(const CUtensorMap& a0, const CUtensorMap& a1, const CUte
                         int gk = 1, int gn = 0, int ksplit = 1, float* part = nullptr,
                         int emod = 0) {
   using C = Cfg<NTMAX, STAGES, UM, KSUB>;
-  static bool attr_set[64] = {false};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev < 64 && !attr_set[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(k_expert_gemm<MODE, NTMAX, STAGES, UM, KSUB>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)C::kSmem);
-    if (e != cudaSuccess) return e;
-    attr_set[dev] = true;
-  }
+  static std::once_flag once[kMaxDevices];
+  static cudaError_t set_up[kMaxDevices];
+  const cudaError_t e0 = once_per_device(once, set_up, [](int) {
+    return cudaFuncSetAttribute(k_expert_gemm<MODE, NTMAX, STAGES, UM, KSUB>,
+                                cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::kSmem);
+  });
+  if (e0 != cudaSuccess) return e0;
   // The down projection is launched as a programmatic dependent of the kernel
   // before it (the gate_up kernel in the expert MLP): its CTAs start as those
   // CTAs retire and prefetch weight tiles.  Every role reads the tile list
@@ -1120,10 +1201,9 @@ cudaError_t launch_gemm_pair(const CUtensorMap& a0, const CUtensorMap& a1, const
                              const moe_act_cfg& act, DeviceStatus* st, cudaStream_t s,
                              bool pdl_ok, int emod = 0) {
   using C = PairCfg;
-  static bool attr_set[64] = {false};
-  static int grid_of[64] = {0};
-  int dev = 0;
-  cudaGetDevice(&dev);
+  static std::once_flag once[kMaxDevices];
+  static cudaError_t set_up[kMaxDevices];
+  static int grid_of[kMaxDevices] = {0};
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -1138,20 +1218,25 @@ cudaError_t launch_gemm_pair(const CUtensorMap& a0, const CUtensorMap& a1, const
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   const int pdl = (MODE == kDown && pdl_ok) ? 1 : 0;
-  if (dev < 64 && !attr_set[dev]) {
+  // kernel attribute and the number of resident pairs, once per device
+  const cudaError_t e0 = once_per_device(once, set_up, [&](int dev) {
     cudaError_t e = cudaFuncSetAttribute(k_expert_gemm_pair<MODE>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)C::kSmem);
     if (e != cudaSuccess) return e;
     int pairs = 0;
-    cfg.gridDim = dim3(dev_info()->sm_count & ~1, 1, 1);
-    e = cudaOccupancyMaxActiveClusters(&pairs, k_expert_gemm_pair<MODE>, &cfg);
+    cudaLaunchConfig_t q = cfg;
+    q.gridDim = dim3(dev_info()->sm_count & ~1, 1, 1);
+    e = cudaOccupancyMaxActiveClusters(&pairs, k_expert_gemm_pair<MODE>, &q);
     if (e != cudaSuccess || pairs < 1) pairs = dev_info()->sm_count / 2;
     if (pairs > dev_info()->sm_count / 2) pairs = dev_info()->sm_count / 2;
     grid_of[dev] = 2 * pairs;
-    attr_set[dev] = true;
-  }
-  cfg.gridDim = dim3(grid_of[dev < 64 ? dev : 0], 1, 1);
+    return cudaSuccess;
+  });
+  if (e0 != cudaSuccess) return e0;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  cfg.gridDim = dim3(grid_of[dev], 1, 1);
   cfg.numAttrs = pdl ? 2 : 1;
   return cudaLaunchKernelEx(&cfg, k_expert_gemm_pair<MODE>, a0, a1, b, b64, offsets, tile_start,
                             E, M_rows, Kdim, out, res, (int)act.kind, act.beta, act.linear_beta,

@@ -6,6 +6,8 @@
 #include <cuda_bf16.h>
 #include <stdint.h>
 
+#include <mutex>
+
 #include "moe.h"
 
 namespace moe {
@@ -27,6 +29,19 @@ __device__ __forceinline__ void record_error(DeviceStatus* st, int code, int det
 constexpr uint32_t kSpinLimit = 1u << 28;
 
 inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+// ------------------------------------------------- per-device set-up
+// Runs init() once per device, however many host threads call at once, and
+// returns its result to every caller (kernel attributes, launch grids).
+constexpr int kMaxDevices = 64;
+template <typename F>
+cudaError_t once_per_device(std::once_flag* flags, cudaError_t* results, F&& init) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
+    return cudaErrorInvalidDevice;
+  std::call_once(flags[dev], [&] { results[dev] = init(dev); });
+  return results[dev];
+}
 
 // ------------------------------------------- programmatic dependent launch
 // The short kernels of the layer are launched as programmatic dependents of

@@ -344,15 +344,13 @@ cudaError_t launch_select(const float* part, int splits, int64_t N, const float*
   const bool softmax = cfg.score_func == MOE_SCORE_SOFTMAX;
   const size_t smem = sizeof(float) * 2 * E * kSelWarps + (softmax ? sizeof(double) * E * kSelWarps : 0);
   if (softmax && smem > 48 * 1024) {
-    static bool attr_set[64] = {false};
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (dev < 64 && !attr_set[dev]) {
-      const cudaError_t e =
-          cudaFuncSetAttribute(k_select, cudaFuncAttributeMaxDynamicSharedMemorySize, 64 * 1024);
-      if (e != cudaSuccess) return e;
-      attr_set[dev] = true;
-    }
+    static std::once_flag once[kMaxDevices];
+    static cudaError_t set_up[kMaxDevices];
+    const cudaError_t e0 = once_per_device(once, set_up, [](int) {
+      return cudaFuncSetAttribute(k_select, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  64 * 1024);
+    });
+    if (e0 != cudaSuccess) return e0;
   }
   int64_t blocks = (N + kSelWarps - 1) / kSelWarps;
   const int64_t cap = (int64_t)dev_info()->sm_count * 16;

@@ -382,17 +382,15 @@ typedef CUresult (*EncodeTiledFnI8)(CUtensorMap*, CUtensorMapDataType, cuuint32_
                                     CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
 EncodeTiledFnI8 encode_i8() {
-  static EncodeTiledFnI8 fn = nullptr;
-  static bool tried = false;
-  if (!tried) {
-    tried = true;
+  static const EncodeTiledFnI8 fn = [] {  // looked up once (thread-safe static)
     void* p = nullptr;
     cudaDriverEntryPointQueryResult q;
     if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
             cudaSuccess &&
         q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFnI8>(p);
-  }
+      return reinterpret_cast<EncodeTiledFnI8>(p);
+    return static_cast<EncodeTiledFnI8>(nullptr);
+  }();
   return fn;
 }
 
@@ -448,15 +446,13 @@ cudaError_t launch_gate_i8(const __nv_bfloat16* x, int64_t N, int d_r, const flo
   CUtensorMap mw, mx;
   if (!map_planes(&mw, wd, d_r, E, IM) || !map_planes(&mx, xd, d_r, N, INT))
     return cudaErrorInvalidValue;
-  static bool attr_set[64] = {false};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev < 64 && !attr_set[dev]) {
-    cudaError_t e =
-        cudaFuncSetAttribute(k_gate_i8, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemI8);
-    if (e != cudaSuccess) return e;
-    attr_set[dev] = true;
-  }
+  static std::once_flag once[kMaxDevices];
+  static cudaError_t set_up[kMaxDevices];
+  const cudaError_t e0 = once_per_device(once, set_up, [](int) {
+    return cudaFuncSetAttribute(k_gate_i8, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)kSmemI8);
+  });
+  if (e0 != cudaSuccess) return e0;
   dim3 grid((E + IM - 1) / IM, (unsigned)((N + INT - 1) / INT), 1);
   k_gate_i8<<<grid, kThreadsI8, kSmemI8, s>>>(mw, mx, wsig, xsig, N, E, d_r, logits, st);
   return cudaGetLastError();
