@@ -344,11 +344,34 @@ def run_ours(args, rank, world, local_rank):
 BLOCK_METRIC = "tokens/sec per MoE block (route+shared experts+latent projections+routed experts)"
 
 
+def dense_split(M, M_rows, K, gate_up):
+    """Whether a dense layer of M rows runs split over K (then a reduce kernel
+    follows its GEMM); mirrors the library's choice, a function of shapes."""
+    if M > 128 * 1:  # CTA-pair variant: never split
+        return False
+    decode = M <= 16
+    nt, um, ks = (32, 1, 128) if decode else (128, 2, 64)
+    unit_rows = um * (64 if gate_up else 128)
+    units = ((M + nt - 1) // nt) * ((M_rows + unit_rows - 1) // unit_rows)
+    if units * 2 >= 148:
+        return False
+    k = min((148 + units - 1) // units, (K // ks) // 2, 32)
+    return k > 1
+
+
 def block_kernels(wl):
     """The routed layer's launches plus the dense tile list, the shared
-    experts' two GEMMs and the two latent projections (the RMSNorm is fused
-    into the combine)."""
-    return kernels_per_step(wl) + 1 + (2 if wl.F_shared else 0) + (2 if wl.latent else 0)
+    experts' two GEMMs and the two latent projections, each followed by a
+    reduce kernel when it runs split over K (the RMSNorm is fused into the
+    combine)."""
+    n = kernels_per_step(wl) + 1
+    N = wl.N
+    if wl.F_shared:
+        n += 2 + dense_split(N, wl.F_shared, wl.d_r, True) + dense_split(N, wl.d_r, wl.F_shared,
+                                                                          False)
+    if wl.latent:
+        n += 2 + dense_split(N, wl.d_e, wl.d_r, False) + dense_split(N, wl.d_r, wl.d_e, False)
+    return n
 
 
 def block_bytes(wl, touched):
