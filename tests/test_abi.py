@@ -250,3 +250,14 @@ def test_ep_expert_ffn_validation(L):
                                0, None) == -2
     assert L.moe_ep_expert_ffn(None, 0, p, 2, 8, 256, 128, p, p, p, ctypes.byref(a), None, None,
                                0, None) == -4
+
+
+def test_bench_split_mirror_matches_the_library(L):
+    """bench.py counts a reduce kernel after every dense layer the library
+    splits over K; its mirror of that choice must agree with the library's
+    own workspace (split partials present <=> split)."""
+    import bench
+    for M in (1, 7, 16, 17, 64, 100, 128, 129, 300):
+        for K, N_out in ((7168, 2048), (2048, 7168), (256, 128), (128, 256), (3072, 7168)):
+            split = L.moe_linear_workspace_size(M, K, N_out) > 512
+            assert bench.dense_split(M, N_out, K, False) == split, (M, K, N_out)
