@@ -9,19 +9,23 @@
 // The slot sort is a stable counting sort in three passes:
 //   k_hist    one warp per chunk of CH consecutive slots: per-chunk expert
 //             counts (warp-aggregated with __match_any_sync);
-//   k_scan    one block: counts[e], offsets (exclusive scan) and, per chunk,
-//             the first sorted position of each expert;
-//   k_scatter one warp per chunk again: slots ranked in slot order within the
-//             chunk -> pos[slot] and perm[pos].
+//   k_scan    one block per 32 experts: counts[e] and, per chunk, the number
+//             of expert-e slots in the chunks before it;
+//   k_scatter one warp per chunk again: every block takes the exclusive scan
+//             of counts (block 0 stores it as offsets), then the slots are
+//             ranked in slot order within the chunk -> pos[slot], perm[pos].
 // Then k_gather copies every token row once from HBM and writes it to its K
 // sorted positions (token-major, so x_e is read once, not K times).  Without
 // xs (the expert MLP gathering its rows itself) k_gather is skipped.
+// The chunk passes load kIdxBatch slot indices per lane before using any, so
+// a warp has that many loads in flight instead of one.
 #include "moe_internal.cuh"
 
 namespace moe {
 namespace {
 
 constexpr int kWarps = 4;
+constexpr int kIdxBatch = 8;
 
 __device__ __forceinline__ unsigned lanemask_lt() {
   unsigned m;
@@ -43,62 +47,75 @@ __global__ void __launch_bounds__(32 * kWarps) k_hist(const int32_t* __restrict_
   __syncwarp();
   const int64_t beg = (int64_t)c * CH;
   const int64_t end = beg + CH < S ? beg + CH : S;
-  for (int64_t base = beg; base < end; base += 32) {
-    const int64_t slot = base + lane;
-    int e = -1;
-    if (slot < end) {
-      e = idx[slot];
-      if (e < 0 || e >= E) {
+  for (int64_t b0 = beg; b0 < end; b0 += 32 * kIdxBatch) {
+    int ev[kIdxBatch];
+#pragma unroll
+    for (int i = 0; i < kIdxBatch; ++i) {
+      const int64_t slot = b0 + 32 * i + lane;
+      ev[i] = slot < end ? idx[slot] : -1;
+    }
+#pragma unroll
+    for (int i = 0; i < kIdxBatch; ++i) {
+      int e = ev[i];
+      if (b0 + 32 * i + lane < end && (e < 0 || e >= E)) {
         record_error(st, MOE_ERR_DEVICE_BOUNDS, 10);
         e = -1;
       }
+      const unsigned peers = __match_any_sync(0xffffffffu, e);
+      if (e >= 0 && lane == __ffs(peers) - 1) cnt[e] += __popc(peers);
+      __syncwarp();
     }
-    const unsigned peers = __match_any_sync(0xffffffffu, e);
-    if (e >= 0 && lane == __ffs(peers) - 1) cnt[e] += __popc(peers);
-    __syncwarp();
   }
   int32_t* out = cc + (int64_t)c * E;
   for (int e = lane; e < E; e += 32) out[e] = cnt[e];
 }
 
-// One block of 1024 threads; thread e owns expert e (E <= 1024).
+// One block per 32 experts, 32 warps: lane l owns expert 32*blockIdx.x + l,
+// warp w the chunks [w*per, (w+1)*per).  cc[c][e] becomes the number of
+// expert-e slots in chunks 0..c-1; counts[e] the total.
+constexpr int kScanHeld = 8;  // chunks per warp kept in registers (per <= 8)
+
 __global__ void __launch_bounds__(1024) k_scan(int32_t* __restrict__ cc, int nchunks, int E,
-                                               int32_t* __restrict__ counts,
-                                               int32_t* __restrict__ offsets) {
+                                               int32_t* __restrict__ counts) {
   pdl_wait();
   pdl_trigger();
-  __shared__ int32_t warp_tot[32];
-  const int e = threadIdx.x;
-  const int lane = e & 31, warp = e >> 5;
-  int32_t tot = 0;
-  if (e < E)
-    for (int c = 0; c < nchunks; ++c) tot += cc[(int64_t)c * E + e];
-  // block exclusive scan of tot
-  int32_t v = tot;
+  __shared__ int32_t part[32][33];
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  const int e = blockIdx.x * 32 + lane;
+  const int per = (nchunks + 31) / 32;
+  const int c0 = w * per;
+  const int c1 = c0 + per < nchunks ? c0 + per : nchunks;
+  const bool live = e < E;
+  int32_t held[kScanHeld];
+  int32_t sum = 0;
+  if (per <= kScanHeld) {
 #pragma unroll
-  for (int off = 1; off < 32; off <<= 1) {
-    const int32_t o = __shfl_up_sync(0xffffffffu, v, off);
-    if (lane >= off) v += o;
-  }
-  if (lane == 31) warp_tot[warp] = v;
-  __syncthreads();
-  if (warp == 0) {
-    int32_t w = warp_tot[lane];
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-      const int32_t o = __shfl_up_sync(0xffffffffu, w, off);
-      if (lane >= off) w += o;
+    for (int i = 0; i < kScanHeld; ++i) {
+      held[i] = (live && c0 + i < c1) ? cc[(int64_t)(c0 + i) * E + e] : 0;
+      sum += held[i];
     }
-    warp_tot[lane] = w;
+  } else if (live) {
+    for (int c = c0; c < c1; ++c) sum += cc[(int64_t)c * E + e];
   }
+  part[w][lane] = sum;
   __syncthreads();
-  const int32_t excl = v - tot + (warp > 0 ? warp_tot[warp - 1] : 0);
-  if (e < E) {
+  int32_t run = 0;
+  for (int i = 0; i < w; ++i) run += part[i][lane];
+  if (w == 0 && live) {
+    int32_t tot = 0;
+    for (int i = 0; i < 32; ++i) tot += part[i][lane];
     counts[e] = tot;
-    offsets[e] = excl;
-    if (e == E - 1) offsets[E] = excl + tot;
-    int32_t run = excl;
-    for (int c = 0; c < nchunks; ++c) {
+  }
+  if (!live) return;
+  if (per <= kScanHeld) {
+#pragma unroll
+    for (int i = 0; i < kScanHeld; ++i)
+      if (c0 + i < c1) {
+        cc[(int64_t)(c0 + i) * E + e] = run;
+        run += held[i];
+      }
+  } else {
+    for (int c = c0; c < c1; ++c) {
       const int32_t n = cc[(int64_t)c * E + e];
       cc[(int64_t)c * E + e] = run;
       run += n;
@@ -109,47 +126,93 @@ __global__ void __launch_bounds__(1024) k_scan(int32_t* __restrict__ cc, int nch
 __global__ void __launch_bounds__(32 * kWarps) k_scatter(const int32_t* __restrict__ idx,
                                                          int64_t S, int E, int CH, int nchunks,
                                                          const int32_t* __restrict__ cc,
+                                                         const int32_t* __restrict__ counts,
+                                                         int32_t* __restrict__ offsets,
                                                          int32_t* __restrict__ perm,
                                                          int32_t* __restrict__ pos) {
   pdl_wait();
   pdl_trigger();
-  extern __shared__ int32_t base_all[];
+  extern __shared__ int32_t sm_all[];  // [E] expert offsets, then kWarps x [E] chunk bases
+  __shared__ int32_t warp_tot[kWarps];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  int32_t* off = sm_all;
+  // exclusive scan of counts: thread i owns experts i*per .. i*per+per-1
+  const int per = (E + 32 * kWarps - 1) / (32 * kWarps);
+  const int e0 = threadIdx.x * per;
+  int32_t mine = 0;
+  for (int j = 0; j < per; ++j)
+    if (e0 + j < E) mine += counts[e0 + j];
+  int32_t v = mine;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int32_t u = __shfl_up_sync(0xffffffffu, v, o);
+    if (lane >= o) v += u;
+  }
+  if (lane == 31) warp_tot[warp] = v;
+  __syncthreads();
+  int32_t run = v - mine;
+  for (int i = 0; i < warp; ++i) run += warp_tot[i];
+  for (int j = 0; j < per; ++j) {
+    const int e = e0 + j;
+    if (e < E) {
+      off[e] = run;
+      if (blockIdx.x == 0) offsets[e] = run;
+      run += counts[e];
+    }
+  }
+  if (blockIdx.x == 0 && threadIdx.x == 32 * kWarps - 1) offsets[E] = run;
+  __syncthreads();
   const int c = blockIdx.x * kWarps + warp;
   if (c >= nchunks) return;
-  int32_t* base = base_all + warp * E;
+  int32_t* base = sm_all + (1 + warp) * E;
   const int32_t* in = cc + (int64_t)c * E;
-  for (int e = lane; e < E; e += 32) base[e] = in[e];
+  for (int e = lane; e < E; e += 32) base[e] = off[e] + in[e];
   __syncwarp();
   const unsigned lt = lanemask_lt();
   const int64_t beg = (int64_t)c * CH;
   const int64_t end = beg + CH < S ? beg + CH : S;
-  for (int64_t b0 = beg; b0 < end; b0 += 32) {
-    const int64_t slot = b0 + lane;
-    int e = -1;
-    if (slot < end) {
-      e = idx[slot];
-      if (e < 0 || e >= E) e = -1;
+  for (int64_t b0 = beg; b0 < end; b0 += 32 * kIdxBatch) {
+    int ev[kIdxBatch];
+#pragma unroll
+    for (int i = 0; i < kIdxBatch; ++i) {
+      const int64_t slot = b0 + 32 * i + lane;
+      ev[i] = slot < end ? idx[slot] : -1;
     }
-    const unsigned peers = __match_any_sync(0xffffffffu, e);
-    if (slot < end) {
-      if (e >= 0) {
-        const int32_t p = base[e] + __popc(peers & lt);
-        pos[slot] = p;
-        perm[p] = (int32_t)slot;
-      } else {
-        pos[slot] = -1;
+#pragma unroll
+    for (int i = 0; i < kIdxBatch; ++i) {
+      const int64_t slot = b0 + 32 * i + lane;
+      const int e = (ev[i] < 0 || ev[i] >= E) ? -1 : ev[i];
+      const unsigned peers = __match_any_sync(0xffffffffu, e);
+      if (slot < end) {
+        if (e >= 0) {
+          const int32_t p = base[e] + __popc(peers & lt);
+          pos[slot] = p;
+          perm[p] = (int32_t)slot;
+        } else {
+          pos[slot] = -1;
+        }
       }
+      __syncwarp();
+      if (e >= 0 && lane == __ffs(peers) - 1) base[e] += __popc(peers);
+      __syncwarp();
     }
-    __syncwarp();
-    if (e >= 0 && lane == __ffs(peers) - 1) base[e] += __popc(peers);
-    __syncwarp();
   }
 }
 
 // One warp per (token, chunk of 256 columns): each lane reads one 16-byte
 // vector of the token's row once and writes it to the K sorted positions
-// pos[t*K + k] (token-major, so x_e is read once, not K times).
+// pos[t*K + k] (token-major, so x_e is read once, not K times).  The next
+// item's row and positions are loaded before this item's K stores issue.
+__device__ __forceinline__ void gather_load(const __nv_bfloat16* __restrict__ x, int K, int d,
+                                            int nv, int nch, int lane, int64_t it,
+                                            const int32_t* __restrict__ pos, uint4& val,
+                                            int& my_p) {
+  const int64_t t = it / nch;
+  const int v = (int)(it - t * nch) * 32 + lane;
+  my_p = lane < K ? pos[t * K + lane] : -1;
+  val = v < nv ? reinterpret_cast<const uint4*>(x + t * d)[v] : make_uint4(0, 0, 0, 0);
+}
+
 __global__ void __launch_bounds__(256) k_gather(const __nv_bfloat16* __restrict__ x, int64_t N,
                                                 int K, int d, const int32_t* __restrict__ pos,
                                                 __nv_bfloat16* __restrict__ xs) {
@@ -159,16 +222,24 @@ __global__ void __launch_bounds__(256) k_gather(const __nv_bfloat16* __restrict_
   const int nv = d / 8;
   const int nch = (nv + 31) / 32;
   const int64_t items = N * nch;
-  for (int64_t it = (int64_t)blockIdx.x * 8 + warp; it < items; it += (int64_t)gridDim.x * 8) {
+  const int64_t stride = (int64_t)gridDim.x * 8;
+  int64_t it = (int64_t)blockIdx.x * 8 + warp;
+  if (it >= items) return;
+  uint4 val;
+  int my_p;
+  gather_load(x, K, d, nv, nch, lane, it, pos, val, my_p);
+  for (; it < items; it += stride) {
+    uint4 nval = make_uint4(0, 0, 0, 0);
+    int n_p = -1;
+    if (it + stride < items) gather_load(x, K, d, nv, nch, lane, it + stride, pos, nval, n_p);
     const int64_t t = it / nch;
     const int v = (int)(it - t * nch) * 32 + lane;
-    const int my_p = lane < K ? pos[t * K + lane] : -1;
-    uint4 val = make_uint4(0, 0, 0, 0);
-    if (v < nv) val = reinterpret_cast<const uint4*>(x + t * d)[v];
     for (int k = 0; k < K; ++k) {
       const int p = __shfl_sync(0xffffffffu, my_p, k);
       if (p >= 0 && v < nv) reinterpret_cast<uint4*>(xs + (int64_t)p * d)[v] = val;
     }
+    val = nval;
+    my_p = n_p;
   }
 }
 
@@ -249,10 +320,10 @@ cudaError_t launch_dispatch(const int32_t* idx, int64_t N, int K, int E, const _
   cudaError_t e;
   if ((e = launch_pdl(k_hist, dim3(blocks), dim3(32 * kWarps), smem, s, idx, S, E, CH, nchunks,
                       scratch, st)) != cudaSuccess ||
-      (e = launch_pdl(k_scan, dim3(1), dim3(1024), 0, s, scratch, nchunks, E, counts,
-                      offsets)) != cudaSuccess ||
-      (e = launch_pdl(k_scatter, dim3(blocks), dim3(32 * kWarps), smem, s, idx, S, E, CH,
-                      nchunks, scratch, perm, pos)) != cudaSuccess)
+      (e = launch_pdl(k_scan, dim3((unsigned)((E + 31) / 32)), dim3(1024), 0, s, scratch,
+                      nchunks, E, counts)) != cudaSuccess ||
+      (e = launch_pdl(k_scatter, dim3(blocks), dim3(32 * kWarps), smem + sizeof(int32_t) * E, s,
+                      idx, S, E, CH, nchunks, scratch, counts, offsets, perm, pos)) != cudaSuccess)
     return e;
   if (!xs) return cudaSuccess;
   int64_t gb = (N * ((d_e / 8 + 31) / 32) + 7) / 8;

@@ -218,7 +218,8 @@ __global__ void __launch_bounds__(32 * kSelWarps) k_select(
     } else {
       for (int e = lane; e < E; e += 32) {
         // sigmoid: fp32 rounding of 1/(1+exp(-L)) evaluated in double
-        const float s = (float)(1.0 / (1.0 + exp(-(double)s_s[e])));
+        // (__drcp_rn is the correctly rounded reciprocal, i.e. IEEE 1.0 / v)
+        const float s = (float)__drcp_rn(1.0 + exp(-(double)s_s[e]));
         s_s[e] = s;
         s_c[e] = bias ? __fadd_rn(s, bias[e]) : s;
       }

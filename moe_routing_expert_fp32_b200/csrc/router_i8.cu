@@ -81,16 +81,14 @@ struct Vec;  // 16-byte loads: 4 fp32 or 8 bf16 per thread
 template <>
 struct Vec<float> {
   static constexpr int n = 4;
-  __device__ static void bits(const float* p, uint32_t* b) {
-    const uint4 r = *reinterpret_cast<const uint4*>(p);
+  __device__ static void bits(const uint4 r, uint32_t* b) {
     b[0] = r.x; b[1] = r.y; b[2] = r.z; b[3] = r.w;
   }
 };
 template <>
 struct Vec<__nv_bfloat16> {
   static constexpr int n = 8;
-  __device__ static void bits(const __nv_bfloat16* p, uint32_t* b) {
-    const uint4 r = *reinterpret_cast<const uint4*>(p);
+  __device__ static void bits(const uint4 r, uint32_t* b) {
     const uint32_t w[4] = {r.x, r.y, r.z, r.w};
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
@@ -100,54 +98,156 @@ struct Vec<__nv_bfloat16> {
   }
 };
 
-// One block per row: row maximum -> scale, then the 4 digits of every element
-// (n elements per thread per step; d % 8 == 0).  out: [PS][rows][d] int8.
+constexpr int kSliceThreads = 256;
+
+// The largest |v| of one 16-byte vector, as an integer (|v| bits order like |v|).
 template <typename T>
-__global__ void __launch_bounds__(256) k_slice_rows(const T* __restrict__ v, int64_t rows, int d,
-                                                    int8_t* __restrict__ out,
-                                                    int* __restrict__ sig_out) {
+__device__ __forceinline__ uint32_t vec_absmax(const uint4 r) {
+  uint32_t b[Vec<T>::n];
+  Vec<T>::bits(r, b);
+  uint32_t mx = 0;
+#pragma unroll
+  for (int i = 0; i < Vec<T>::n; ++i) mx = max(mx, b[i] & 0x7FFFFFFFu);
+  return mx;
+}
+
+// The PS digit planes of one vector of n elements starting at column j.
+template <typename T>
+__device__ __forceinline__ void store_digits(const uint4 r, int sig, int8_t* __restrict__ out,
+                                             int64_t plane, int64_t row, int d, int j) {
+  constexpr int VN = Vec<T>::n;
+  uint32_t b[VN];
+  Vec<T>::bits(r, b);
+  int8_t a[VN][PS];
+#pragma unroll
+  for (int i = 0; i < VN; ++i) digits4(b[i], sig, a[i]);
+#pragma unroll
+  for (int p = 0; p < PS; ++p) {
+    uint32_t w[VN / 4];
+#pragma unroll
+    for (int q = 0; q < VN / 4; ++q)
+      w[q] = (uint32_t)(uint8_t)a[4 * q][p] | ((uint32_t)(uint8_t)a[4 * q + 1][p] << 8) |
+             ((uint32_t)(uint8_t)a[4 * q + 2][p] << 16) |
+             ((uint32_t)(uint8_t)a[4 * q + 3][p] << 24);
+    int8_t* dst = out + p * plane + row * d + j;
+    if (VN == 8) *reinterpret_cast<uint2*>(dst) = make_uint2(w[0], w[VN / 4 - 1]);
+    else *reinterpret_cast<uint32_t*>(dst) = w[0];
+  }
+}
+
+// bf16 rows, four elements at a time.  A bf16 value has an 8-bit significand
+// M, so X = M shifted by t = Ebits - 106 - sig (the float form's shift + 16).
+// spread_bf16 puts digit p of X in byte 3-p; a 4 x 4 byte transpose turns four
+// such words into one word per digit plane, and negative elements are negated
+// bytewise: -a == (0x80 - a) ^ 0x80 for 0 <= a <= 127, so no byte borrows.
+__device__ __forceinline__ uint32_t spread_bf16(uint32_t h, int sig) {
+  const int eb = (int)((h >> 7) & 0xFFu);
+  const uint32_t M = (h & 0x7Fu) | (eb ? 0x80u : 0u);
+  const int t = (eb ? eb : 1) - 106 - sig;  // t <= 20 because |v| < 2^sig
+  const uint32_t X = t >= 0 ? M << t : (t > -8 ? M >> -t : 0u);
+  return (X & 0x7Fu) | ((X << 1) & 0x7F00u) | ((X << 2) & 0x7F0000u) | ((X << 3) & 0x7F000000u);
+}
+
+// Byte i = 0xFF where element i of {a.lo, a.hi, b.lo, b.hi} is negative
+// (prmt selectors with the sign-replicate bit, on bytes 1, 3, 5 and 7).
+__device__ __forceinline__ uint32_t sign_bytes(uint32_t a, uint32_t b) {
+  uint32_t m;
+  asm("prmt.b32 %0, %1, %2, 0xFDB9;" : "=r"(m) : "r"(a), "r"(b));
+  return m;
+}
+
+// The four digit-plane words of elements {a.lo, a.hi, b.lo, b.hi}.
+__device__ __forceinline__ void planes4_bf16(uint32_t a, uint32_t b, int sig, uint32_t* P) {
+  const uint32_t y0 = spread_bf16(a & 0xFFFFu, sig), y1 = spread_bf16(a >> 16, sig);
+  const uint32_t y2 = spread_bf16(b & 0xFFFFu, sig), y3 = spread_bf16(b >> 16, sig);
+  const uint32_t lo01 = __byte_perm(y0, y1, 0x5140), hi01 = __byte_perm(y0, y1, 0x7362);
+  const uint32_t lo23 = __byte_perm(y2, y3, 0x5140), hi23 = __byte_perm(y2, y3, 0x7362);
+  const uint32_t m = sign_bytes(a, b);
+  const uint32_t q[PS] = {__byte_perm(hi01, hi23, 0x7632), __byte_perm(hi01, hi23, 0x5410),
+                          __byte_perm(lo01, lo23, 0x7632), __byte_perm(lo01, lo23, 0x5410)};
+#pragma unroll
+  for (int p = 0; p < PS; ++p) {
+    const uint32_t neg = (0x80808080u - q[p]) ^ 0x80808080u;
+    P[p] = (neg & m) | (q[p] & ~m);
+  }
+}
+
+template <>
+__device__ __forceinline__ void store_digits<__nv_bfloat16>(const uint4 r, int sig,
+                                                            int8_t* __restrict__ out,
+                                                            int64_t plane, int64_t row, int d,
+                                                            int j) {
+  uint32_t P0[PS], P1[PS];
+  planes4_bf16(r.x, r.y, sig, P0);
+  planes4_bf16(r.z, r.w, sig, P1);
+#pragma unroll
+  for (int p = 0; p < PS; ++p)
+    *reinterpret_cast<uint2*>(out + p * plane + row * d + j) = make_uint2(P0[p], P1[p]);
+}
+
+// One block per row: row maximum -> scale, then the 4 digits of every element
+// (d % 8 == 0).  out: [PS][rows][d] int8.  With R > 0 (rows of at most
+// R * 256 vectors) every thread keeps its R vectors in registers, so the row
+// is read once with all of its loads in flight together; R == 0 reads the
+// row twice (any d).
+template <typename T, int R>
+__global__ void __launch_bounds__(kSliceThreads) k_slice_rows(const T* __restrict__ v,
+                                                              int64_t rows, int d,
+                                                              int8_t* __restrict__ out,
+                                                              int* __restrict__ sig_out) {
   pdl_wait();
   pdl_trigger();
   constexpr int VN = Vec<T>::n;
-  __shared__ float wmax[8];
+  constexpr int kStep = kSliceThreads * VN;
+  __shared__ uint32_t wmax[kSliceThreads / 32];
   const int64_t row = blockIdx.x;
   const T* src = v + row * d;
+  uint4 held[R > 0 ? R : 1];
   uint32_t mx = 0;
-  for (int j = threadIdx.x * VN; j < d; j += blockDim.x * VN) {
-    uint32_t b[VN];
-    Vec<T>::bits(src + j, b);
+  if constexpr (R > 0) {
 #pragma unroll
-    for (int i = 0; i < VN; ++i) mx = max(mx, b[i] & 0x7FFFFFFFu);  // |v| ordered as integers
+    for (int r = 0; r < R; ++r) {
+      const int j = r * kStep + threadIdx.x * VN;
+      held[r] = j < d ? *reinterpret_cast<const uint4*>(src + j) : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int r = 0; r < R; ++r) mx = max(mx, vec_absmax<T>(held[r]));
+  } else {
+    for (int j = threadIdx.x * VN; j < d; j += kStep)
+      mx = max(mx, vec_absmax<T>(*reinterpret_cast<const uint4*>(src + j)));
   }
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-  if ((threadIdx.x & 31) == 0) wmax[threadIdx.x >> 5] = __uint_as_float(mx);
+  if ((threadIdx.x & 31) == 0) wmax[threadIdx.x >> 5] = mx;
   __syncthreads();
-  float m = 0.f;
+  uint32_t m = 0;
 #pragma unroll
-  for (int i = 0; i < 8; ++i) m = fmaxf(m, wmax[i]);
-  const int sig = row_sig(m);
+  for (int i = 0; i < kSliceThreads / 32; ++i) m = max(m, wmax[i]);
+  const int sig = row_sig(__uint_as_float(m));
   if (threadIdx.x == 0) sig_out[row] = sig;
   const int64_t plane = rows * (int64_t)d;
-  for (int j = threadIdx.x * VN; j < d; j += blockDim.x * VN) {
-    uint32_t b[VN];
-    Vec<T>::bits(src + j, b);
-    int8_t a[VN][PS];
+  if constexpr (R > 0) {
 #pragma unroll
-    for (int i = 0; i < VN; ++i) digits4(b[i], sig, a[i]);
-#pragma unroll
-    for (int p = 0; p < PS; ++p) {
-      uint32_t w[VN / 4];
-#pragma unroll
-      for (int q = 0; q < VN / 4; ++q)
-        w[q] = (uint32_t)(uint8_t)a[4 * q][p] | ((uint32_t)(uint8_t)a[4 * q + 1][p] << 8) |
-               ((uint32_t)(uint8_t)a[4 * q + 2][p] << 16) |
-               ((uint32_t)(uint8_t)a[4 * q + 3][p] << 24);
-      int8_t* dst = out + p * plane + row * d + j;
-      if (VN == 8) *reinterpret_cast<uint2*>(dst) = make_uint2(w[0], w[VN / 4 - 1]);
-      else *reinterpret_cast<uint32_t*>(dst) = w[0];
+    for (int r = 0; r < R; ++r) {
+      const int j = r * kStep + threadIdx.x * VN;
+      if (j < d) store_digits<T>(held[r], sig, out, plane, row, d, j);
     }
+  } else {
+    for (int j = threadIdx.x * VN; j < d; j += kStep)
+      store_digits<T>(*reinterpret_cast<const uint4*>(src + j), sig, out, plane, row, d, j);
   }
+}
+
+// Launch with the smallest register tile that holds a row.
+template <typename T>
+void launch_slice_rows(const T* v, int64_t rows, int d, int8_t* out, int* sig, cudaStream_t s) {
+  const int steps = (d + kSliceThreads * Vec<T>::n - 1) / (kSliceThreads * Vec<T>::n);
+  const dim3 g((unsigned)rows), b(kSliceThreads);
+  if (steps <= 1) k_slice_rows<T, 1><<<g, b, 0, s>>>(v, rows, d, out, sig);
+  else if (steps <= 2) k_slice_rows<T, 2><<<g, b, 0, s>>>(v, rows, d, out, sig);
+  else if (steps <= 4) k_slice_rows<T, 4><<<g, b, 0, s>>>(v, rows, d, out, sig);
+  else if (steps <= 8) k_slice_rows<T, 8><<<g, b, 0, s>>>(v, rows, d, out, sig);
+  else k_slice_rows<T, 0><<<g, b, 0, s>>>(v, rows, d, out, sig);
 }
 
 // -------------------------------------------------------------- PTX helpers
@@ -441,8 +541,8 @@ cudaError_t launch_gate_i8(const __nv_bfloat16* x, int64_t N, int d_r, const flo
   int* wsig = reinterpret_cast<int*>(base + L.ws);
   int8_t* xd = reinterpret_cast<int8_t*>(base + L.xd);
   int* xsig = reinterpret_cast<int*>(base + L.xs);
-  k_slice_rows<float><<<E, 256, 0, s>>>(W, E, d_r, wd, wsig);
-  k_slice_rows<__nv_bfloat16><<<(unsigned)N, 256, 0, s>>>(x, N, d_r, xd, xsig);
+  launch_slice_rows(W, E, d_r, wd, wsig, s);
+  launch_slice_rows(x, N, d_r, xd, xsig, s);
   CUtensorMap mw, mx;
   if (!map_planes(&mw, wd, d_r, E, IM) || !map_planes(&mx, xd, d_r, N, INT))
     return cudaErrorInvalidValue;

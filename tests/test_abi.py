@@ -261,3 +261,26 @@ def test_bench_split_mirror_matches_the_library(L):
         for K, N_out in ((7168, 2048), (2048, 7168), (256, 128), (128, 256), (3072, 7168)):
             split = L.moe_linear_workspace_size(M, K, N_out) > 512
             assert bench.dense_split(M, N_out, K, False) == split, (M, K, N_out)
+
+
+def _dispatch_chunks(S):
+    """Chunk count of the stable sort as moe_dispatch_static's comment in
+    include/moe.h states it: chunk length clamp(S/256, 64, 1024) rounded up
+    to a multiple of 32."""
+    ch = min(max(S // 256, 64), 1024)
+    ch = (ch + 31) // 32 * 32
+    return (S + ch - 1) // ch
+
+
+@pytest.mark.parametrize("N,K,E", [(1, 1, 1), (64, 4, 16), (128, 8, 256), (4096, 8, 384),
+                                   (16384, 8, 384), (100000, 6, 1024), (3, 16, 1000)])
+def test_dispatch_workspace_follows_the_documented_chunking(L, N, K, E):
+    """The workspace holds the 256-byte status word and 4 * chunks * E bytes
+    of per-chunk counts (256-byte aligned); the static entry point's 2 MiB
+    limit is stated in the same terms."""
+    counts = 4 * _dispatch_chunks(N * K) * E
+    assert L.moe_dispatch_workspace_size(N, K, E) == 256 + (counts + 255) // 256 * 256
+    if counts > (2 << 20):
+        # rejected on the host, before any device work (the pointers are fake)
+        p = ctypes.c_void_p(256)
+        assert L.moe_dispatch_static(p, N, K, E, p, 128, p, p, p, p, p, None) == -2
