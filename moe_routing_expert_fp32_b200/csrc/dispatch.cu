@@ -136,6 +136,13 @@ __global__ void __launch_bounds__(32 * kWarps) k_scatter(const int32_t* __restri
   __shared__ int32_t warp_tot[kWarps];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   int32_t* off = sm_all;
+  const int c = blockIdx.x * kWarps + warp;
+  int32_t* base = sm_all + (1 + warp) * E;
+  // this chunk's counts first: their loads overlap the scan below
+  if (c < nchunks) {
+    const int32_t* in = cc + (int64_t)c * E;
+    for (int e = lane; e < E; e += 32) base[e] = in[e];
+  }
   // exclusive scan of counts: thread i owns experts i*per .. i*per+per-1
   const int per = (E + 32 * kWarps - 1) / (32 * kWarps);
   const int e0 = threadIdx.x * per;
@@ -162,11 +169,8 @@ __global__ void __launch_bounds__(32 * kWarps) k_scatter(const int32_t* __restri
   }
   if (blockIdx.x == 0 && threadIdx.x == 32 * kWarps - 1) offsets[E] = run;
   __syncthreads();
-  const int c = blockIdx.x * kWarps + warp;
   if (c >= nchunks) return;
-  int32_t* base = sm_all + (1 + warp) * E;
-  const int32_t* in = cc + (int64_t)c * E;
-  for (int e = lane; e < E; e += 32) base[e] = off[e] + in[e];
+  for (int e = lane; e < E; e += 32) base[e] += off[e];
   __syncwarp();
   const unsigned lt = lanemask_lt();
   const int64_t beg = (int64_t)c * CH;

@@ -284,3 +284,25 @@ def test_dispatch_workspace_follows_the_documented_chunking(L, N, K, E):
         # rejected on the host, before any device work (the pointers are fake)
         p = ctypes.c_void_p(256)
         assert L.moe_dispatch_static(p, N, K, E, p, 128, p, p, p, p, p, None) == -2
+
+
+def test_bench_roofline_picks_the_binding_peak():
+    """The bench's w1/w3 roofline object is HBM-bound for the decode and
+    prefill workloads and tensor-bound for the skewed one, with achieved /
+    peak computed against the matching measured figure."""
+    import bench
+    from synth.workloads import WORKLOADS
+    peaks = {"hbm_gbs": 6546.9, "bf16_tflops": 1676.5, "bf16_tflops_sustained": 1374.1,
+             "source": "measured"}
+    dec = bench.gate_up_roofline(WORKLOADS["dsv32_decode"], 252, 2.17, peaks)
+    assert dec["bound"] == "hbm" and dec["unit"] == "GB/s"
+    assert abs(dec["achieved"] - 14.82e9 / 2.17e-3 / 1e9) / dec["achieved"] < 0.01
+    assert abs(dec["frac"] - dec["achieved"] / 6546.9) < 1e-12
+    pre = bench.gate_up_roofline(WORKLOADS["k2_prefill"], 384, 3.5, peaks)
+    assert pre["bound"] == "hbm"
+    skew = WORKLOADS["k2_skew"]
+    sk = bench.gate_up_roofline(skew, 364, 8.8, peaks)
+    assert sk["bound"] == "tensor" and sk["unit"] == "TFLOP/s" and sk["traffic"] is None
+    flops = 4 * skew.N * skew.K * skew.F * skew.d_e
+    assert abs(sk["achieved"] - flops / 8.8e-3 / 1e12) < 1e-9
+    assert abs(sk["frac"] - sk["achieved"] / 1374.1) < 1e-12
