@@ -100,7 +100,8 @@ struct Vec<__nv_bfloat16> {
 
 constexpr int kSliceThreads = 256;
 
-// The largest |v| of one 16-byte vector, as an integer (|v| bits order like |v|).
+// The largest |v| of one 16-byte vector, as the bits of an fp32 (|v| bits
+// order like |v|).
 template <typename T>
 __device__ __forceinline__ uint32_t vec_absmax(const uint4 r) {
   uint32_t b[Vec<T>::n];
@@ -110,17 +111,41 @@ __device__ __forceinline__ uint32_t vec_absmax(const uint4 r) {
   for (int i = 0; i < Vec<T>::n; ++i) mx = max(mx, b[i] & 0x7FFFFFFFu);
   return mx;
 }
+// bf16: the magnitudes of each pair maxed as bf16x2 (exact), then the pair.
+template <>
+__device__ __forceinline__ uint32_t vec_absmax<__nv_bfloat16>(const uint4 r) {
+  const uint32_t w[4] = {r.x & 0x7FFF7FFFu, r.y & 0x7FFF7FFFu, r.z & 0x7FFF7FFFu,
+                         r.w & 0x7FFF7FFFu};
+  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(w);
+  const __nv_bfloat162 m2 = __hmax2(__hmax2(h[0], h[1]), __hmax2(h[2], h[3]));
+  const uint32_t mb = *reinterpret_cast<const uint32_t*>(&m2);
+  return max(mb << 16, mb & 0xFFFF0000u);
+}
+
+// A row's scale: sig (max|v| < 2^sig) and 2^(28 - sig) as the product s1 * s2
+// of two normal floats (28 - sig reaches 160 for the smallest bf16 rows).
+struct RowScale {
+  int sig;
+  float s1, s2;
+};
+__device__ __forceinline__ RowScale row_scale(int sig) {
+  const int k = 28 - sig;
+  const int k1 = k < 127 ? k : 127;
+  return {sig, __uint_as_float((uint32_t)(k1 + 127) << 23),
+          __uint_as_float((uint32_t)(k - k1 + 127) << 23)};
+}
 
 // The PS digit planes of one vector of n elements starting at column j.
 template <typename T>
-__device__ __forceinline__ void store_digits(const uint4 r, int sig, int8_t* __restrict__ out,
-                                             int64_t plane, int64_t row, int d, int j) {
+__device__ __forceinline__ void store_digits(const uint4 r, const RowScale& sc,
+                                             int8_t* __restrict__ out, int64_t plane,
+                                             int64_t row, int d, int j) {
   constexpr int VN = Vec<T>::n;
   uint32_t b[VN];
   Vec<T>::bits(r, b);
   int8_t a[VN][PS];
 #pragma unroll
-  for (int i = 0; i < VN; ++i) digits4(b[i], sig, a[i]);
+  for (int i = 0; i < VN; ++i) digits4(b[i], sc.sig, a[i]);
 #pragma unroll
   for (int p = 0; p < PS; ++p) {
     uint32_t w[VN / 4];
@@ -135,16 +160,16 @@ __device__ __forceinline__ void store_digits(const uint4 r, int sig, int8_t* __r
   }
 }
 
-// bf16 rows, four elements at a time.  A bf16 value has an 8-bit significand
-// M, so X = M shifted by t = Ebits - 106 - sig (the float form's shift + 16).
-// spread_bf16 puts digit p of X in byte 3-p; a 4 x 4 byte transpose turns four
-// such words into one word per digit plane, and negative elements are negated
-// bytewise: -a == (0x80 - a) ^ 0x80 for 0 <= a <= 127, so no byte borrows.
-__device__ __forceinline__ uint32_t spread_bf16(uint32_t h, int sig) {
-  const int eb = (int)((h >> 7) & 0xFFu);
-  const uint32_t M = (h & 0x7Fu) | (eb ? 0x80u : 0u);
-  const int t = (eb ? eb : 1) - 106 - sig;  // t <= 20 because |v| < 2^sig
-  const uint32_t X = t >= 0 ? M << t : (t > -8 ? M >> -t : 0u);
+// bf16 rows, four elements at a time.  X = floor(|v| * 2^(28 - sig)) in
+// floating point: the products are power-of-two scalings, exact unless one
+// falls below 2^-126 (then X is 0 either way), the result is below 2^28
+// because |v| < 2^sig, and the conversion truncates.  spread_bf16 puts digit
+// p of X in byte 3-p; a 4 x 4 byte transpose turns four such words into one
+// word per digit plane, and negative elements are negated bytewise:
+// -a == (0x80 - a) ^ 0x80 for 0 <= a <= 127, so no byte borrows.
+__device__ __forceinline__ uint32_t spread_bf16(uint32_t abs_bits, const RowScale& sc) {
+  const float v = __uint_as_float(abs_bits);  // |v| as fp32
+  const uint32_t X = __float2uint_rz(__fmul_rn(__fmul_rn(v, sc.s1), sc.s2));
   return (X & 0x7Fu) | ((X << 1) & 0x7F00u) | ((X << 2) & 0x7F0000u) | ((X << 3) & 0x7F000000u);
 }
 
@@ -157,9 +182,10 @@ __device__ __forceinline__ uint32_t sign_bytes(uint32_t a, uint32_t b) {
 }
 
 // The four digit-plane words of elements {a.lo, a.hi, b.lo, b.hi}.
-__device__ __forceinline__ void planes4_bf16(uint32_t a, uint32_t b, int sig, uint32_t* P) {
-  const uint32_t y0 = spread_bf16(a & 0xFFFFu, sig), y1 = spread_bf16(a >> 16, sig);
-  const uint32_t y2 = spread_bf16(b & 0xFFFFu, sig), y3 = spread_bf16(b >> 16, sig);
+__device__ __forceinline__ void planes4_bf16(uint32_t a, uint32_t b, const RowScale& sc,
+                                             uint32_t* P) {
+  const uint32_t y0 = spread_bf16((a & 0x7FFFu) << 16, sc), y1 = spread_bf16(a & 0x7FFF0000u, sc);
+  const uint32_t y2 = spread_bf16((b & 0x7FFFu) << 16, sc), y3 = spread_bf16(b & 0x7FFF0000u, sc);
   const uint32_t lo01 = __byte_perm(y0, y1, 0x5140), hi01 = __byte_perm(y0, y1, 0x7362);
   const uint32_t lo23 = __byte_perm(y2, y3, 0x5140), hi23 = __byte_perm(y2, y3, 0x7362);
   const uint32_t m = sign_bytes(a, b);
@@ -173,13 +199,13 @@ __device__ __forceinline__ void planes4_bf16(uint32_t a, uint32_t b, int sig, ui
 }
 
 template <>
-__device__ __forceinline__ void store_digits<__nv_bfloat16>(const uint4 r, int sig,
+__device__ __forceinline__ void store_digits<__nv_bfloat16>(const uint4 r, const RowScale& sc,
                                                             int8_t* __restrict__ out,
                                                             int64_t plane, int64_t row, int d,
                                                             int j) {
   uint32_t P0[PS], P1[PS];
-  planes4_bf16(r.x, r.y, sig, P0);
-  planes4_bf16(r.z, r.w, sig, P1);
+  planes4_bf16(r.x, r.y, sc, P0);
+  planes4_bf16(r.z, r.w, sc, P1);
 #pragma unroll
   for (int p = 0; p < PS; ++p)
     *reinterpret_cast<uint2*>(out + p * plane + row * d + j) = make_uint2(P0[p], P1[p]);
@@ -225,16 +251,17 @@ __global__ void __launch_bounds__(kSliceThreads) k_slice_rows(const T* __restric
   for (int i = 0; i < kSliceThreads / 32; ++i) m = max(m, wmax[i]);
   const int sig = row_sig(__uint_as_float(m));
   if (threadIdx.x == 0) sig_out[row] = sig;
+  const RowScale sc = row_scale(sig);
   const int64_t plane = rows * (int64_t)d;
   if constexpr (R > 0) {
 #pragma unroll
     for (int r = 0; r < R; ++r) {
       const int j = r * kStep + threadIdx.x * VN;
-      if (j < d) store_digits<T>(held[r], sig, out, plane, row, d, j);
+      if (j < d) store_digits<T>(held[r], sc, out, plane, row, d, j);
     }
   } else {
     for (int j = threadIdx.x * VN; j < d; j += kStep)
-      store_digits<T>(*reinterpret_cast<const uint4*>(src + j), sig, out, plane, row, d, j);
+      store_digits<T>(*reinterpret_cast<const uint4*>(src + j), sc, out, plane, row, d, j);
   }
 }
 
