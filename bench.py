@@ -30,6 +30,7 @@ import os
 import statistics
 import subprocess
 import sys
+import tempfile
 import time
 
 import numpy as np
@@ -123,10 +124,17 @@ class ClockSampler:
         self.index = index
         self.proc = None
         self.path = None
+        # raw samples go to a temporary file unless MOE_BENCH_CLOCKS_DIR names
+        # a folder to keep them in
+        self.keep_dir = os.environ.get("MOE_BENCH_CLOCKS_DIR")
 
     def __enter__(self):
-        os.makedirs(os.path.join(ROOT, "gpurun_out"), exist_ok=True)
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_{os.getpid()}.csv")
+        if self.keep_dir:
+            os.makedirs(self.keep_dir, exist_ok=True)
+            self.path = os.path.join(self.keep_dir, f"clocks_{os.getpid()}.csv")
+        else:
+            fd, self.path = tempfile.mkstemp(prefix="moe_clocks_", suffix=".csv")
+            os.close(fd)
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
@@ -148,6 +156,8 @@ class ClockSampler:
 
     def summary(self):
         if self.proc is None or not os.path.exists(self.path):
+            if not self.keep_dir and self.path and os.path.exists(self.path):
+                os.remove(self.path)
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
         sm, mx, reasons = [], None, set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
@@ -163,6 +173,8 @@ class ClockSampler:
             for n, v in zip(names, parts[5:9]):
                 if v.lower() == "active":
                     reasons.add(n)
+        if not self.keep_dir:
+            os.remove(self.path)
         return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
                 "reasons": sorted(reasons), "samples": len(sm)}
 
