@@ -89,7 +89,7 @@ int route_impl(const __nv_bfloat16* x, int64_t N, int d_r, const float* W, const
                DeviceStatus* st, cudaStream_t s) {
   const int E = cfg.num_experts;
   if (launch_gate(x, N, d_r, W, E, scratch, st, s) != cudaSuccess) return MOE_ERR_CUDA;
-  if (launch_select(route_logits_of(scratch), 1, N, bias, cfg, idx, w, st, s) != cudaSuccess)
+  if (launch_select(route_logits_of(scratch), N, bias, cfg, idx, w, st, s) != cudaSuccess)
     return MOE_ERR_CUDA;
   return MOE_OK;
 }
@@ -189,7 +189,7 @@ int moe_route_from_logits(const float* logits, int64_t N, const float* bias,
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if ((rc = reset_status(ws, s))) return rc;
   if (N == 0) return MOE_OK;
-  return launch_select(logits, 1, N, bias, *cfg, topk_idx, topk_w, status_of(ws), s) ==
+  return launch_select(logits, N, bias, *cfg, topk_idx, topk_w, status_of(ws), s) ==
                  cudaSuccess
              ? MOE_OK
              : MOE_ERR_CUDA;

@@ -89,7 +89,7 @@ size_t gate_i8_scratch_bytes(int64_t N, int E, int d_r);
 cudaError_t launch_gate_i8(const __nv_bfloat16* x, int64_t N, int d_r, const float* W, int E,
                            void* scratch, DeviceStatus* st, cudaStream_t s);
 float* route_logits_of(void* scratch);
-cudaError_t launch_select(const float* part, int splits, int64_t N, const float* bias,
+cudaError_t launch_select(const float* logits, int64_t N, const float* bias,
                           const moe_route_cfg& cfg, int32_t* idx, float* w, DeviceStatus* st,
                           cudaStream_t s);
 

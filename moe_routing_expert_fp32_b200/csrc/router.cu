@@ -171,7 +171,7 @@ __device__ __forceinline__ void warp_best(float& v, int& i) {
 constexpr int kSelWarps = 4;
 
 __global__ void __launch_bounds__(32 * kSelWarps) k_select(
-    const float* __restrict__ part, int splits, int64_t N, int E, const float* __restrict__ bias,
+    const float* __restrict__ logits, int64_t N, int E, const float* __restrict__ bias,
     int G, int TG, int K, int norm, float route_scale, int score_func, int group_mode,
     int32_t* __restrict__ idx_out, float* __restrict__ w_out, DeviceStatus* st) {
   pdl_wait();
@@ -182,20 +182,11 @@ __global__ void __launch_bounds__(32 * kSelWarps) k_select(
   float* s_c = s_s + E;
   // softmax only: E doubles per warp after the float arrays
   double* s_x = reinterpret_cast<double*>(sm + kSelWarps * 2 * E) + warp * E;
-  const int64_t split_stride = N * (int64_t)E;
   for (int64_t t = (int64_t)blockIdx.x * kSelWarps + warp; t < N;
        t += (int64_t)gridDim.x * kSelWarps) {
-    const float* p = part + t * E;
+    const float* p = logits + t * E;
     // the token's logits first, all loads in flight together
-    for (int e = lane; e < E; e += 32) {
-      float L = p[e];
-      if (splits > 1) {  // split-K partials summed in double, rounded once
-        double Ld = (double)L;
-        for (int z = 1; z < splits; ++z) Ld += (double)p[z * split_stride + e];
-        L = (float)Ld;
-      }
-      s_s[e] = L;
-    }
+    for (int e = lane; e < E; e += 32) s_s[e] = p[e];
     __syncwarp();
     if (score_func == MOE_SCORE_SOFTMAX) {
       // softmax over the E logits: exp(L - max) in double, summed in expert
@@ -338,7 +329,7 @@ cudaError_t launch_gate(const __nv_bfloat16* x, int64_t N, int d_r, const float*
   return cudaGetLastError();
 }
 
-cudaError_t launch_select(const float* part, int splits, int64_t N, const float* bias,
+cudaError_t launch_select(const float* logits, int64_t N, const float* bias,
                           const moe_route_cfg& cfg, int32_t* idx, float* w, DeviceStatus* st,
                           cudaStream_t s) {
   const int E = cfg.num_experts;
@@ -357,7 +348,7 @@ cudaError_t launch_select(const float* part, int splits, int64_t N, const float*
   const int64_t cap = (int64_t)dev_info()->sm_count * 16;
   if (blocks > cap) blocks = cap;
   const cudaError_t e = launch_pdl(
-      k_select, dim3((unsigned)blocks), dim3(32 * kSelWarps), smem, s, part, splits, N, E, bias,
+      k_select, dim3((unsigned)blocks), dim3(32 * kSelWarps), smem, s, logits, N, E, bias,
       cfg.n_group, cfg.topk_group, cfg.top_k, cfg.norm_topk_prob, cfg.route_scale,
       cfg.score_func, cfg.group_score, idx, w, st);
   if (e != cudaSuccess) return e;
