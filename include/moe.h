@@ -165,6 +165,9 @@ MOE_API size_t moe_dispatch_workspace_size(int64_t N, int K, int E);
  *   xs[j, :]   = x_e[perm[j] / K, :]
  * topk_idx: [N, K] int32; x_e: [N, d_e] bf16; counts [E], offsets [E+1],
  * perm [S], pos [S] int32 out; xs [S, d_e] bf16 out.
+ * xs may be NULL: then only counts, offsets, perm and pos are written and
+ * x_e is not read (it may be NULL too), for callers that move the rows
+ * themselves (moe_expert_ffn_gathered, moe_ep_dispatch_rows).
  * An expert index outside [0, E) is recorded as MOE_ERR_DEVICE_BOUNDS and its
  * slot is left out of every output. */
 MOE_API int moe_dispatch(const int32_t* topk_idx, int64_t N, int K, int E, const moe_bf16* x_e,
@@ -263,6 +266,59 @@ MOE_API int moe_ep_expert_ffn(const moe_bf16* xr, int64_t R, const int32_t* recv
                               int E_local, int d_e, int F, const moe_bf16* w1,
                               const moe_bf16* w3, const moe_bf16* w2, const moe_act_cfg* act,
                               moe_bf16* y, void* ws, size_t ws_bytes, void* stream);
+
+/* ----------------------------------------- expert parallelism over peer memory
+ *
+ * The same exchange without a collective library: the sending rank's kernel
+ * stores each token row straight into the receiving rank's row buffer, and
+ * the combine loads the expert outputs straight from the rank that computed
+ * them, through device addresses of the peers' buffers (NVLink peer mappings
+ * on a multi-GPU node; any device addresses the GPU can reach).
+ *
+ * Rank q holds experts q*E_local .. q*E_local + E_local - 1, E_local = E / P.
+ * On the sending rank, sorted position j (0 <= j < S, moe_dispatch's pos and
+ * offsets) belongs to the rank q with offsets[q*E_local] <= j <
+ * offsets[(q+1)*E_local], and its row in rank q's buffer is
+ *   first_row[q] + j - offsets[q*E_local].
+ * The caller sizes the buffers and chooses first_row so that the senders'
+ * segments do not overlap; with first_row[q] = the rows that ranks 0 .. p-1
+ * send to q (p this rank), rank q's buffer holds its received rows grouped by
+ * source rank and sorted by local expert, the layout moe_ep_expert_ffn takes.
+ * Ordering between ranks (all rows stored before a rank's experts read them,
+ * all outputs written before the senders' combines load them) is the
+ * caller's: a barrier across the ranks between the steps. */
+#define MOE_MAX_PEERS 64
+
+typedef struct moe_peer_rows {
+  int num_ranks;                    /* P, 1 .. MOE_MAX_PEERS; E % P == 0           */
+  void* rows[MOE_MAX_PEERS];        /* rank q's [capacity[q], d_e] bf16 buffer, as  */
+                                    /* a device address of this GPU (16-B aligned)  */
+  int64_t first_row[MOE_MAX_PEERS]; /* this rank's first row in rank q's buffer     */
+  int64_t capacity[MOE_MAX_PEERS];  /* rows in rank q's buffer                      */
+} moe_peer_rows;
+
+/* Send side: for every slot s = t*K + k with pos[s] = j >= 0, rank q's row
+ * first_row[q] + j - offsets[q*E_local] becomes x_e[t, :] (each token row is
+ * read from HBM once and stored K times).  x_e [N, d_e] bf16; pos [S],
+ * offsets [E+1] int32 as moe_dispatch writes them.  A row outside
+ * [0, capacity[q]) is not stored and is recorded as MOE_ERR_DEVICE_BOUNDS.
+ * Workspace: moe_combine_workspace_size() bytes (the status word). */
+MOE_API int moe_ep_dispatch_rows(const moe_bf16* x_e, int64_t N, int K, int d_e,
+                                 const int32_t* pos, const int32_t* offsets, int E,
+                                 const moe_peer_rows* peers, void* ws, size_t ws_bytes,
+                                 void* stream);
+
+/* Return side, fused with the combine: moe_combine where the row of slot s is
+ * loaded from rank q's buffer at first_row[q] + pos[s] - offsets[q*E_local]
+ * (peers->rows now name the buffers of expert outputs, laid out as the rows
+ * were sent).  Same arithmetic as moe_combine: products rounded to fp32,
+ * summed in k order, one rounding to bf16.  out [N, d_e] bf16; topk_w [N, K]
+ * fp32.  Rows out of range are skipped and recorded as
+ * MOE_ERR_DEVICE_BOUNDS.  Workspace: moe_combine_workspace_size() bytes. */
+MOE_API int moe_ep_combine_rows(const moe_peer_rows* peers, const int32_t* pos,
+                                const int32_t* offsets, int E, const float* topk_w, int64_t N,
+                                int K, int d_e, moe_bf16* out, void* ws, size_t ws_bytes,
+                                void* stream);
 
 /* ------------------------------------------------------------ whole layer */
 

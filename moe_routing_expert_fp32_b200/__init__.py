@@ -73,6 +73,32 @@ class _BlockDims(ctypes.Structure):
                 ("F_shared", ctypes.c_int), ("norm_eps", ctypes.c_float)]
 
 
+MOE_MAX_PEERS = 64
+
+
+class _PeerRows(ctypes.Structure):
+    _fields_ = [("num_ranks", ctypes.c_int), ("rows", ctypes.c_void_p * MOE_MAX_PEERS),
+                ("first_row", ctypes.c_int64 * MOE_MAX_PEERS),
+                ("capacity", ctypes.c_int64 * MOE_MAX_PEERS)]
+
+
+def peer_rows(rows, first_row, capacity) -> _PeerRows:
+    """The moe_peer_rows table: rows[q] is rank q's row buffer as a device
+    address of this GPU (an int, or a tensor on this GPU), first_row[q] this
+    rank's first row in it, capacity[q] its rows."""
+    P = len(rows)
+    if not (1 <= P <= MOE_MAX_PEERS and len(first_row) == P and len(capacity) == P):
+        raise ValueError("peer_rows: 1..64 ranks, one first_row and capacity per rank")
+    t = _PeerRows()
+    t.num_ranks = P
+    for q in range(P):
+        r = rows[q]
+        t.rows[q] = r if isinstance(r, int) else (None if r is None else r.data_ptr())
+        t.first_row[q] = int(first_row[q])
+        t.capacity[q] = int(capacity[q])
+    return t
+
+
 class _BlockWeights(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in (
         "gate_weight", "gate_bias", "down_proj", "norm_weight", "up_proj", "w1", "w3", "w2",
@@ -123,7 +149,8 @@ EXPORTS = ("moe_route_workspace_size", "moe_route", "moe_route_from_logits",
            "moe_forward", "moe_get_status", "moe_strerror", "moe_dispatch_static",
            "moe_linear_workspace_size", "moe_linear", "moe_rms_norm", "moe_block_workspace_size",
            "moe_block_forward", "moe_shared_experts_workspace_size", "moe_shared_experts",
-           "moe_ep_expert_ffn_workspace_size", "moe_ep_expert_ffn", "moe_expert_ffn_gathered")
+           "moe_ep_expert_ffn_workspace_size", "moe_ep_expert_ffn", "moe_expert_ffn_gathered",
+           "moe_ep_dispatch_rows", "moe_ep_combine_rows")
 
 
 def lib() -> ctypes.CDLL:
@@ -138,6 +165,7 @@ def lib() -> ctypes.CDLL:
     vp, i64, i32, sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t
     rc, ac, ev = ctypes.POINTER(_RouteCfg), ctypes.POINTER(_ActCfg), ctypes.POINTER(_StageEvents)
     bd, bw = ctypes.POINTER(_BlockDims), ctypes.POINTER(_BlockWeights)
+    pr = ctypes.POINTER(_PeerRows)
     sig = {
         "moe_route_workspace_size": ([i64, i32, rc], sz),
         "moe_route": ([vp, i64, i32, vp, vp, rc, vp, vp, vp, sz, vp], i32),
@@ -168,6 +196,8 @@ def lib() -> ctypes.CDLL:
         "moe_shared_experts": ([vp, i64, i32, i32, vp, vp, vp, ac, vp, vp, vp, sz, vp], i32),
         "moe_block_workspace_size": ([i64, bd, bw, rc], sz),
         "moe_block_forward": ([vp, i64, bd, bw, rc, ac, vp, vp, vp, vp, sz, vp], i32),
+        "moe_ep_dispatch_rows": ([vp, i64, i32, i32, vp, vp, i32, pr, vp, sz, vp], i32),
+        "moe_ep_combine_rows": ([pr, vp, vp, i32, vp, i64, i32, i32, vp, vp, sz, vp], i32),
     }
     for name, (args, res) in sig.items():
         fn = getattr(L, name)
@@ -267,8 +297,9 @@ def route_from_logits(logits, bias, cfg: RouteConfig, ws=None):
     return idx, w
 
 
-def dispatch(topk_idx, x_e, num_experts: int, ws=None):
-    """(counts [E], offsets [E+1], perm [S], pos [S], xs [S, d_e])."""
+def dispatch(topk_idx, x_e, num_experts: int, ws=None, gather=True):
+    """(counts [E], offsets [E+1], perm [S], pos [S], xs [S, d_e]); with
+    gather=False the rows are not copied and xs is None."""
     torch = _torch()
     N, K = topk_idx.shape
     d_e = x_e.shape[1]
@@ -283,7 +314,7 @@ def dispatch(topk_idx, x_e, num_experts: int, ws=None):
     offsets = torch.empty(E + 1, dtype=torch.int32, device=dev)
     perm = torch.empty(S, dtype=torch.int32, device=dev)
     pos = torch.empty(S, dtype=torch.int32, device=dev)
-    xs = torch.empty((S, d_e), dtype=torch.bfloat16, device=dev)
+    xs = torch.empty((S, d_e), dtype=torch.bfloat16, device=dev) if gather else None
     _check("moe_dispatch",
            lib().moe_dispatch(_ptr(topk_idx), N, K, E, _ptr(x_e), d_e, _ptr(counts),
                               _ptr(offsets), _ptr(perm), _ptr(pos), _ptr(xs), _ptr(ws),
@@ -458,6 +489,39 @@ def ep_expert_ffn(xr, recv_counts, w1, w3, w2, act: ActConfig, y=None, ws=None):
                                    _ptr(w3), _ptr(w2), ctypes.byref(a), _ptr(y), _ptr(ws),
                                    ws.numel(), _stream()))
     return y
+
+
+def ep_dispatch_rows(x_e, pos, offsets, num_experts: int, peers: _PeerRows, K: int, ws=None):
+    """Store every token row of x_e [N, d_e] into the receiving ranks' buffers
+    (moe_ep_dispatch_rows); pos [N*K], offsets [E+1] from dispatch()."""
+    torch = _torch()
+    N, d_e = x_e.shape
+    _need(x_e, torch.bfloat16, name="x_e")
+    _need(pos, torch.int32, (N * K,), "pos")
+    _need(offsets, torch.int32, (num_experts + 1,), "offsets")
+    ws = workspace(256, x_e.device) if ws is None else ws
+    _check("moe_ep_dispatch_rows",
+           lib().moe_ep_dispatch_rows(_ptr(x_e), N, K, d_e, _ptr(pos), _ptr(offsets), num_experts,
+                                      ctypes.byref(peers), _ptr(ws), ws.numel(), _stream()))
+
+
+def ep_combine_rows(peers: _PeerRows, pos, offsets, num_experts: int, topk_w, d_e: int, out=None,
+                    ws=None):
+    """The weighted combine with each slot's output loaded from the rank that
+    computed it (moe_ep_combine_rows); returns out [N, d_e] bf16."""
+    torch = _torch()
+    N, K = topk_w.shape
+    _need(topk_w, torch.float32, name="topk_w")
+    _need(pos, torch.int32, (N * K,), "pos")
+    _need(offsets, torch.int32, (num_experts + 1,), "offsets")
+    dev = topk_w.device
+    ws = workspace(256, dev) if ws is None else ws
+    out = torch.empty((N, d_e), dtype=torch.bfloat16, device=dev) if out is None else out
+    _check("moe_ep_combine_rows",
+           lib().moe_ep_combine_rows(ctypes.byref(peers), _ptr(pos), _ptr(offsets), num_experts,
+                                     _ptr(topk_w), N, K, d_e, _ptr(out), _ptr(ws), ws.numel(),
+                                     _stream()))
+    return out
 
 
 def shared_experts(x, w1, w3, w2, act: ActConfig, residual=None, out=None, ws=None):

@@ -209,8 +209,9 @@ int moe_dispatch(const int32_t* topk_idx, int64_t N, int K, int E, const moe_bf1
   if (d_e % 8 != 0) return MOE_ERR_UNSUPPORTED;
   if (N * (int64_t)K > INT32_MAX) return MOE_ERR_UNSUPPORTED;
   if (!counts || !offsets) return MOE_ERR_INVALID_ARG;
-  if (N > 0 && (!topk_idx || !x_e || !perm || !pos || !xs)) return MOE_ERR_INVALID_ARG;
-  if (N > 0 && (!aligned16(x_e) || !aligned16(xs))) return MOE_ERR_ALIGNMENT;
+  // xs == NULL: the sort only, x_e is not read
+  if (N > 0 && (!topk_idx || !perm || !pos || (xs && !x_e))) return MOE_ERR_INVALID_ARG;
+  if (N > 0 && xs && (!aligned16(x_e) || !aligned16(xs))) return MOE_ERR_ALIGNMENT;
   int rc;
   if ((rc = check_ws(ws, ws_bytes, moe_dispatch_workspace_size(N, K, E)))) return rc;
   if ((rc = check_device())) return rc;
@@ -352,6 +353,81 @@ int moe_combine(const moe_bf16* y, const int32_t* pos, const float* topk_w, int6
   if (N == 0) return MOE_OK;
   return launch_combine(reinterpret_cast<const __nv_bfloat16*>(y), pos, topk_w, N, K, d_e,
                         N * K, reinterpret_cast<__nv_bfloat16*>(out), status_of(ws), s) ==
+                 cudaSuccess
+             ? MOE_OK
+             : MOE_ERR_CUDA;
+}
+
+// ------------------------------------- expert parallelism over peer memory
+namespace {
+int peer_table(const moe_peer_rows* peers, int E, PeerTable* pt) {
+  if (!peers) return MOE_ERR_INVALID_ARG;
+  const int P = peers->num_ranks;
+  if (P < 1 || P > MOE_MAX_PEERS) return MOE_ERR_UNSUPPORTED;
+  if (E % P != 0) return MOE_ERR_INVALID_ARG;
+  pt->P = P;
+  pt->E_local = E / P;
+  for (int q = 0; q < MOE_MAX_PEERS; ++q) {
+    pt->rows[q] = nullptr;
+    pt->first[q] = 0;
+    pt->cap[q] = 0;
+    if (q >= P) continue;
+    if (peers->first_row[q] < 0 || peers->capacity[q] < 0) return MOE_ERR_INVALID_ARG;
+    if (peers->capacity[q] > 0 && !peers->rows[q]) return MOE_ERR_INVALID_ARG;
+    if (peers->rows[q] && !aligned16(peers->rows[q])) return MOE_ERR_ALIGNMENT;
+    pt->rows[q] = static_cast<__nv_bfloat16*>(peers->rows[q]);
+    pt->first[q] = peers->first_row[q];
+    pt->cap[q] = peers->capacity[q];
+  }
+  return MOE_OK;
+}
+
+int check_ep_rows(int64_t N, int K, int d_e, int E, const int32_t* pos, const int32_t* offsets) {
+  if (N < 0 || K < 1 || E < 1 || d_e <= 0) return MOE_ERR_INVALID_ARG;
+  if (K > 16 || E > 1024) return MOE_ERR_UNSUPPORTED;
+  if (d_e % 8 != 0) return MOE_ERR_UNSUPPORTED;
+  if (N * (int64_t)K > INT32_MAX) return MOE_ERR_UNSUPPORTED;
+  if (N > 0 && (!pos || !offsets)) return MOE_ERR_INVALID_ARG;
+  return MOE_OK;
+}
+}  // namespace
+
+int moe_ep_dispatch_rows(const moe_bf16* x_e, int64_t N, int K, int d_e, const int32_t* pos,
+                         const int32_t* offsets, int E, const moe_peer_rows* peers, void* ws,
+                         size_t ws_bytes, void* stream) {
+  int rc;
+  if ((rc = check_ep_rows(N, K, d_e, E, pos, offsets))) return rc;
+  if (N > 0 && !x_e) return MOE_ERR_INVALID_ARG;
+  if (N > 0 && !aligned16(x_e)) return MOE_ERR_ALIGNMENT;
+  PeerTable pt;
+  if ((rc = peer_table(peers, E, &pt))) return rc;
+  if ((rc = check_ws(ws, ws_bytes, kStatusBytes))) return rc;
+  if ((rc = check_device())) return rc;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if ((rc = reset_status(ws, s))) return rc;
+  if (N == 0) return MOE_OK;
+  return launch_ep_dispatch_rows(reinterpret_cast<const __nv_bfloat16*>(x_e), N, K, d_e, pos,
+                                 offsets, N * K, pt, status_of(ws), s) == cudaSuccess
+             ? MOE_OK
+             : MOE_ERR_CUDA;
+}
+
+int moe_ep_combine_rows(const moe_peer_rows* peers, const int32_t* pos, const int32_t* offsets,
+                        int E, const float* topk_w, int64_t N, int K, int d_e, moe_bf16* out,
+                        void* ws, size_t ws_bytes, void* stream) {
+  int rc;
+  if ((rc = check_ep_rows(N, K, d_e, E, pos, offsets))) return rc;
+  if (N > 0 && (!topk_w || !out)) return MOE_ERR_INVALID_ARG;
+  if (N > 0 && !aligned16(out)) return MOE_ERR_ALIGNMENT;
+  PeerTable pt;
+  if ((rc = peer_table(peers, E, &pt))) return rc;
+  if ((rc = check_ws(ws, ws_bytes, kStatusBytes))) return rc;
+  if ((rc = check_device())) return rc;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if ((rc = reset_status(ws, s))) return rc;
+  if (N == 0) return MOE_OK;
+  return launch_ep_combine_rows(pt, pos, offsets, N * K, topk_w, N, K, d_e,
+                                reinterpret_cast<__nv_bfloat16*>(out), status_of(ws), s) ==
                  cudaSuccess
              ? MOE_OK
              : MOE_ERR_CUDA;

@@ -167,6 +167,23 @@ cudaError_t launch_combine_rms_norm(const __nv_bfloat16* y, const int32_t* pos, 
 cudaError_t launch_rms_norm(const __nv_bfloat16* x, int64_t N, int d, const __nv_bfloat16* w,
                             float eps, __nv_bfloat16* out, cudaStream_t s);
 
+// ep_rows.cu: the expert-parallel exchange over peer memory (moe_ep_dispatch_rows,
+// moe_ep_combine_rows).  Passed by value as a __grid_constant__ kernel argument.
+struct PeerTable {
+  int P;        // ranks
+  int E_local;  // experts per rank
+  __nv_bfloat16* rows[MOE_MAX_PEERS];
+  int64_t first[MOE_MAX_PEERS];
+  int64_t cap[MOE_MAX_PEERS];
+};
+cudaError_t launch_ep_dispatch_rows(const __nv_bfloat16* x, int64_t N, int K, int d,
+                                    const int32_t* pos, const int32_t* offsets, int64_t S,
+                                    const PeerTable& pt, DeviceStatus* st, cudaStream_t s);
+cudaError_t launch_ep_combine_rows(const PeerTable& pt, const int32_t* pos,
+                                   const int32_t* offsets, int64_t S, const float* w, int64_t N,
+                                   int K, int d, __nv_bfloat16* out, DeviceStatus* st,
+                                   cudaStream_t s);
+
 // device properties, read once per device
 struct DevInfo {
   int sm_count;

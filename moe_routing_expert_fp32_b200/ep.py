@@ -16,6 +16,12 @@ One step on every rank:
   4. send the outputs back (the reverse all-to-all-v) into the slots the rows
      came from, and combine them with the routing weights (moe_combine).
 
+`ep_forward_p2p` is the same step without a collective moving the rows: the
+send kernel (moe_ep_dispatch_rows) stores each token row straight into the
+receiving ranks' buffers through peer addresses of a symmetric-memory
+allocation, and the combine (moe_ep_combine_rows) loads the outputs straight
+from the ranks that computed them; `p2p_plan` places every rank's rows.
+
 The collectives are torch.distributed all-to-alls (NCCL over NVLink on GPUs);
 their split sizes need the counts on the host, the one synchronisation of the
 step (the page's tokens_per_expert.cpu()).  Rows travel as int32 views of
@@ -92,3 +98,85 @@ def ep_forward(x_r, W, bias, cfg, w1_local, w3_local, w2_local, act, x_e=None, g
         combine=lambda y, pos, w: combine(y, pos, w),
     )
     return exchange_forward(x_r, x_e, steps, cfg.num_experts, group)
+
+
+def p2p_plan(all_counts, rank: int, P: int):
+    """Where this rank's rows go and what it receives, from every rank's
+    per-expert counts all_counts [P, E] (host integers, identical on all ranks):
+
+      first_row[q]  this rank's first row in rank q's buffer: the rows ranks
+                    0 .. rank-1 send to q, so q receives its rows grouped by
+                    source rank and, within a source, sorted by local expert;
+      recv_counts   [P, E_local] int32: the rows each source sends to this
+                    rank's experts (the segments moe_ep_expert_ffn runs);
+      recv_rows     the rows this rank receives.
+    """
+    import numpy as np
+
+    c = np.asarray(all_counts, dtype=np.int64)
+    if c.ndim != 2 or c.shape[0] != P or c.shape[1] % P != 0:
+        raise ValueError(f"counts of shape {c.shape} do not split over {P} ranks")
+    E_local = c.shape[1] // P
+    rows_to = c.reshape(P, P, E_local).sum(axis=2)  # [source rank, destination rank]
+    first_row = [int(rows_to[:rank, q].sum()) for q in range(P)]
+    recv_counts = np.ascontiguousarray(c[:, rank * E_local:(rank + 1) * E_local], dtype=np.int32)
+    return first_row, recv_counts, int(rows_to[:, rank].sum())
+
+
+def ep_forward_p2p(x_r, W, bias, cfg, w1_local, w3_local, w2_local, act, x_e=None, group=None):
+    """The routed layer with this rank's experts, the rows moved through peer
+    memory by this library's kernels.  One step on every rank:
+
+      1. route and sort its slots (moe_route, moe_dispatch without the copy);
+      2. all-gather the per-expert counts (the step's one host
+         synchronisation) and place the rows with p2p_plan;
+      3. moe_ep_dispatch_rows stores its rows into the receiving ranks' halves
+         of a symmetric-memory buffer (same size on every rank: the largest
+         receive count); barrier;
+      4. the local experts run on the received rows and write their outputs
+         to the other half; barrier;
+      5. moe_ep_combine_rows loads each slot's output from the rank that
+         computed it and combines; barrier (no rank frees the buffer while a
+         peer still reads it).
+
+    The barriers are a stream synchronisation and a process-group barrier.
+    Returns (out [N, d_e] bf16, topk_idx, topk_w)."""
+    import torch
+    import torch.distributed as dist
+    import torch.distributed._symmetric_memory as symm
+
+    from . import dispatch, ep_combine_rows, ep_dispatch_rows, ep_expert_ffn, peer_rows, route
+
+    group = group or dist.group.WORLD
+    P = dist.get_world_size(group)
+    rank = dist.get_rank(group)
+    E = cfg.num_experts
+    if E % P != 0:
+        raise ValueError(f"{E} experts do not split over {P} ranks")
+    x_e = x_r if x_e is None else x_e
+    d_e = x_e.shape[1]
+    idx, w = route(x_r, W, bias, cfg)
+    counts, offsets, _, pos, _ = dispatch(idx, x_e, E, gather=False)
+    gathered = torch.empty((P, E), dtype=torch.int32, device=counts.device)
+    dist.all_gather_into_tensor(gathered, counts, group=group)
+    all_counts = gathered.cpu().numpy()
+    first_row, recv_counts, R = p2p_plan(all_counts, rank, P)
+    cap = max(1, max(p2p_plan(all_counts, q, P)[2] for q in range(P)))
+    buf = symm.empty(2 * cap, d_e, dtype=torch.bfloat16, device=x_e.device)
+    handle = symm.rendezvous(buf, group)
+    offset = buf.data_ptr() - handle.buffer_ptrs[rank]
+    xr_at = [handle.buffer_ptrs[q] + offset for q in range(P)]
+    y_at = [a + cap * d_e * buf.element_size() for a in xr_at]
+
+    def barrier():
+        torch.cuda.current_stream().synchronize()
+        dist.barrier(group=group)
+
+    ep_dispatch_rows(x_e, pos, offsets, E, peer_rows(xr_at, first_row, [cap] * P), cfg.top_k)
+    barrier()
+    rc = torch.from_numpy(recv_counts).to(x_e.device)
+    ep_expert_ffn(buf[:R], rc, w1_local, w3_local, w2_local, act, y=buf[cap:cap + R])
+    barrier()
+    out = ep_combine_rows(peer_rows(y_at, first_row, [cap] * P), pos, offsets, E, w, d_e)
+    barrier()
+    return out, idx, w

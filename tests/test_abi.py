@@ -306,3 +306,57 @@ def test_bench_roofline_picks_the_binding_peak():
     flops = 4 * skew.N * skew.K * skew.F * skew.d_e
     assert abs(sk["achieved"] - flops / 8.8e-3 / 1e12) < 1e-9
     assert abs(sk["frac"] - sk["achieved"] / 1374.1) < 1e-12
+
+
+def test_ep_rows_validation(L):
+    """moe_ep_dispatch_rows / moe_ep_combine_rows reject bad arguments on the
+    host, before any device work (the pointers here are fake)."""
+    import moe_routing_expert_fp32_b200 as m
+    p = ctypes.c_void_p(256)
+    ws = ctypes.c_void_p(1 << 20)
+
+    def table(P, rows=256, cap=10, first=0):
+        return m.peer_rows([rows] * P, [first] * P, [cap] * P)
+
+    def disp(t, E=8, K=2, d=128, x=p, pos=p, offs=p, w=ws, wb=256):
+        return L.moe_ep_dispatch_rows(x, 4, K, d, pos, offs, E, ctypes.byref(t), w, wb, None)
+
+    def comb(t, E=8, K=2, d=128, out=p, tw=p, w=ws, wb=256):
+        return L.moe_ep_combine_rows(ctypes.byref(t), p, p, E, tw, 4, K, d, out, w, wb, None)
+
+    for f in (disp, comb):
+        assert f(table(3)) == -1                    # 8 experts do not split over 3 ranks
+        t = table(2)
+        t.num_ranks = 0
+        assert f(t) == -2                           # no ranks
+        t.num_ranks = 65
+        assert f(t) == -2                           # more than MOE_MAX_PEERS
+        assert f(table(2, rows=None)) == -1         # capacity without a buffer
+        assert f(table(2, rows=264)) == -3          # buffer not 16-byte aligned
+        assert f(table(2, cap=-1)) == -1
+        assert f(table(2, first=-1)) == -1
+        assert f(table(2), K=17) == -2
+        assert f(table(2), d=100) == -2
+        assert f(table(2), w=None) == -4            # no workspace
+        assert f(table(2), wb=8) == -4              # workspace too small
+    assert disp(table(2), x=None) == -1
+    assert disp(table(2), x=ctypes.c_void_p(264)) == -3
+    assert disp(table(2), pos=None) == -1
+    assert comb(table(2), out=None) == -1
+    assert comb(table(2), tw=None) == -1
+    with pytest.raises(ValueError):
+        m.peer_rows([], [], [])
+    with pytest.raises(ValueError):
+        m.peer_rows([256] * 65, [0] * 65, [1] * 65)
+
+
+def test_dispatch_without_the_copy_needs_no_rows(L):
+    """moe_dispatch with xs NULL sorts only, so x_e may be NULL too; with xs
+    given, x_e is required (host checks, fake pointers rejected before any
+    device work)."""
+    p = ctypes.c_void_p(256)
+    # xs given without x_e: rejected on the host
+    assert L.moe_dispatch(p, 4, 2, 8, None, 128, p, p, p, p, p, p, 1 << 20, None) == -1
+    # an unaligned x_e matters only when the rows are copied
+    assert L.moe_dispatch(p, 4, 2, 8, ctypes.c_void_p(264), 128, p, p, p, p, p, p, 1 << 20,
+                          None) == -3

@@ -107,3 +107,39 @@ def test_exchange_forward_equals_one_rank(world, E):
         assert p.exitcode == 0
     assert sorted(r[0] for r in res) == list(range(world))
     assert all(r[1] for r in res), res
+
+
+@pytest.mark.parametrize("P,E_local", [(1, 4), (2, 3), (4, 2), (8, 16)])
+def test_p2p_plan_places_rows_as_the_all_to_all_would(P, E_local):
+    """Brute force: lay out every destination rank's buffer as the all-to-all
+    delivers it (sources in rank order, each source's rows sorted by expert)
+    and check that p2p_plan puts each source's rows exactly there."""
+    from moe_routing_expert_fp32_b200.ep import p2p_plan
+    rng = np.random.default_rng(P * 100 + E_local)
+    E = P * E_local
+    counts = rng.integers(0, 7, size=(P, E))
+    counts[0, :] = 0                      # a rank that sends nothing
+    buffers = [[] for _ in range(P)]      # rank q's rows: (source, expert, i)
+    for p in range(P):
+        for q in range(P):
+            for e in range(q * E_local, (q + 1) * E_local):
+                buffers[q] += [(p, e, i) for i in range(counts[p, e])]
+    for rank in range(P):
+        first_row, recv_counts, recv_rows = p2p_plan(counts, rank, P)
+        assert recv_rows == len(buffers[rank])
+        assert recv_counts.dtype == np.int32 and recv_counts.shape == (P, E_local)
+        assert (recv_counts == counts[:, rank * E_local:(rank + 1) * E_local]).all()
+        for q in range(P):
+            # the sender's sorted positions for q's experts start at
+            # offsets[q*E_local]; position j lands at first_row[q] + j - that
+            sent = [(rank, e, i) for e in range(q * E_local, (q + 1) * E_local)
+                    for i in range(counts[rank, e])]
+            assert buffers[q][first_row[q]:first_row[q] + len(sent)] == sent
+
+
+def test_p2p_plan_rejects_counts_that_do_not_split():
+    from moe_routing_expert_fp32_b200.ep import p2p_plan
+    with pytest.raises(ValueError):
+        p2p_plan(np.zeros((2, 5), dtype=np.int64), 0, 2)
+    with pytest.raises(ValueError):
+        p2p_plan(np.zeros((3, 6), dtype=np.int64), 0, 2)
