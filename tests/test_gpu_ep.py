@@ -109,10 +109,11 @@ def test_ep_peer_rows_emulated(moe, name, P, N):
         d = synth.workloads.dev_inputs(wl, rank=p, experts=False)
         x_e = d["x_e"] if wl.latent else d["x"]
         idx, w = moe.route(d["x"], W, b, cfg)
-        counts, offs, _, pos, xs_none = moe.dispatch(idx, x_e, wl.E, gather=False)
+        counts, offs, perm, pos, xs_none = moe.dispatch(idx, x_e, wl.E, gather=False)
         assert xs_none is None
-        _, _, _, pos2, xs = moe.dispatch(idx, x_e, wl.E)
-        assert torch.equal(pos, pos2)
+        counts2, offs2, perm2, pos2, xs = moe.dispatch(idx, x_e, wl.E)
+        for a, b2 in ((counts, counts2), (offs, offs2), (perm, perm2), (pos, pos2)):
+            assert torch.equal(a, b2)
         ref = moe.forward(d["x"], W, b, cfg, w1, w3, w2, act, x_e=d["x_e"] if wl.latent else None)
         ranks.append(dict(x_e=x_e, w=w, counts=counts, offs=offs, pos=pos, xs=xs, ref=ref))
     all_counts = torch.stack([r["counts"] for r in ranks]).cpu().numpy()
