@@ -194,7 +194,10 @@ def test_dispatch(moe, name):
     _dispatch_case(moe, wl.N, wl.K, wl.E, wl.d_e, idx)
 
 
-@pytest.mark.parametrize("N,K,E", [(1, 8, 384), (1000, 1, 16), (333, 3, 7), (5000, 16, 1024)])
+# (40000, 8, 64): 320 000 slots make 313 chunks of 1024, more than the 256
+# that the scan keeps in registers, so its looping form runs
+@pytest.mark.parametrize("N,K,E", [(1, 8, 384), (1000, 1, 16), (333, 3, 7), (5000, 16, 1024),
+                                   (40000, 8, 64)])
 def test_dispatch_edge_shapes(moe, N, K, E):
     rng = np.random.default_rng(N + K + E)
     _dispatch_case(moe, N, K, E, 128, random_topk(N, K, E, rng, skew=1.5))
