@@ -123,22 +123,74 @@ def p2p_plan(all_counts, rank: int, P: int):
     return first_row, recv_counts, int(rows_to[:, rank].sum())
 
 
-def ep_forward_p2p(x_r, W, bias, cfg, w1_local, w3_local, w2_local, act, x_e=None, group=None):
-    """The routed layer with this rank's experts, the rows moved through peer
-    memory by this library's kernels.  One step on every rank:
+@dataclass
+class P2PSteps:
+    """The steps of the exchange through peer memory (`exchange_forward_p2p`).
 
-      1. route and sort its slots (moe_route, moe_dispatch without the copy);
+    route(x_r) -> (idx [N, K] int32, w [N, K] fp32)
+    dispatch(idx, x_e) -> (counts [E] int32, offsets [E+1] int32, pos [S] int32)
+    buffers(cap, d_e, like) -> (xr, y, xr_at, y_at): this rank's receive and
+        output buffers of `cap` rows and every rank's, as the send and combine
+        steps address them (the same `cap` on every rank)
+    send_rows(x_e, pos, offsets, xr_at, first_row, cap): store each slot's row
+        into its rank's receive buffer
+    experts(xr [R, d_e], recv_counts [P, E_local] int32, y [R, d_e]): the
+        local experts on the received rows, outputs into y
+    combine_rows(y_at, first_row, cap, pos, offsets, w) -> out [N, d_e]
+    barrier(): every rank's previous step has finished
+    """
+    route: Callable
+    dispatch: Callable
+    buffers: Callable
+    send_rows: Callable
+    experts: Callable
+    combine_rows: Callable
+    barrier: Callable
+
+
+def exchange_forward_p2p(x_r, x_e, steps: P2PSteps, num_experts: int, group=None):
+    """One expert-parallel step through peer memory on this rank:
+
+      1. route and sort its slots;
       2. all-gather the per-expert counts (the step's one host
          synchronisation) and place the rows with p2p_plan;
-      3. moe_ep_dispatch_rows stores its rows into the receiving ranks' halves
-         of a symmetric-memory buffer (same size on every rank: the largest
-         receive count); barrier;
-      4. the local experts run on the received rows and write their outputs
-         to the other half; barrier;
-      5. moe_ep_combine_rows loads each slot's output from the rank that
-         computed it and combines; barrier (no rank frees the buffer while a
-         peer still reads it).
+      3. store its rows into the receiving ranks' buffers; barrier;
+      4. run the local experts on the received rows; barrier;
+      5. combine, loading each slot's output from the rank that computed it;
+         barrier (no rank reuses its buffers while a peer still reads them).
 
+    Returns (out, topk_idx, topk_w)."""
+    import torch
+    import torch.distributed as dist
+
+    P = dist.get_world_size(group)
+    rank = dist.get_rank(group)
+    if num_experts % P != 0:
+        raise ValueError(f"{num_experts} experts do not split over {P} ranks")
+    idx, w = steps.route(x_r)
+    counts, offsets, pos = steps.dispatch(idx, x_e)
+    got = [torch.empty_like(counts) for _ in range(P)]
+    dist.all_gather(got, counts.contiguous(), group=group)
+    all_counts = torch.stack(got).cpu().numpy()
+    first_row, recv_counts, R = p2p_plan(all_counts, rank, P)
+    cap = max(1, max(p2p_plan(all_counts, q, P)[2] for q in range(P)))
+    xr, y, xr_at, y_at = steps.buffers(cap, x_e.shape[1], x_e)
+    steps.send_rows(x_e, pos, offsets, xr_at, first_row, cap)
+    steps.barrier()
+    steps.experts(xr[:R], recv_counts, y[:R])
+    steps.barrier()
+    out = steps.combine_rows(y_at, first_row, cap, pos, offsets, w)
+    steps.barrier()
+    return out, idx, w
+
+
+def ep_forward_p2p(x_r, W, bias, cfg, w1_local, w3_local, w2_local, act, x_e=None, group=None):
+    """The routed layer with this rank's experts (w1_local, w3_local
+    [E_local, F, d_e], w2_local [E_local, d_e, F]), the rows moved through
+    peer memory by this library's kernels: moe_ep_dispatch_rows stores them
+    into the receiving ranks' halves of a torch symmetric-memory buffer (the
+    same size on every rank: the largest receive count), the experts write
+    their outputs to the other half, and moe_ep_combine_rows loads them back.
     The barriers are a stream synchronisation and a process-group barrier.
     Returns (out [N, d_e] bf16, topk_idx, topk_w)."""
     import torch
@@ -151,32 +203,38 @@ def ep_forward_p2p(x_r, W, bias, cfg, w1_local, w3_local, w2_local, act, x_e=Non
     P = dist.get_world_size(group)
     rank = dist.get_rank(group)
     E = cfg.num_experts
-    if E % P != 0:
-        raise ValueError(f"{E} experts do not split over {P} ranks")
     x_e = x_r if x_e is None else x_e
-    d_e = x_e.shape[1]
-    idx, w = route(x_r, W, bias, cfg)
-    counts, offsets, _, pos, _ = dispatch(idx, x_e, E, gather=False)
-    gathered = torch.empty((P, E), dtype=torch.int32, device=counts.device)
-    dist.all_gather_into_tensor(gathered, counts, group=group)
-    all_counts = gathered.cpu().numpy()
-    first_row, recv_counts, R = p2p_plan(all_counts, rank, P)
-    cap = max(1, max(p2p_plan(all_counts, q, P)[2] for q in range(P)))
-    buf = symm.empty(2 * cap, d_e, dtype=torch.bfloat16, device=x_e.device)
-    handle = symm.rendezvous(buf, group)
-    offset = buf.data_ptr() - handle.buffer_ptrs[rank]
-    xr_at = [handle.buffer_ptrs[q] + offset for q in range(P)]
-    y_at = [a + cap * d_e * buf.element_size() for a in xr_at]
+    held = []  # the symmetric buffer lives until the step returns
 
-    def barrier():
+    def _dispatch(idx, xe):
+        counts, offsets, _, pos, _ = dispatch(idx, xe, E, gather=False)
+        return counts, offsets, pos
+
+    def _buffers(cap, d_e, like):
+        buf = symm.empty(2 * cap, d_e, dtype=torch.bfloat16, device=like.device)
+        handle = symm.rendezvous(buf, group)
+        held.append((buf, handle))
+        offset = buf.data_ptr() - handle.buffer_ptrs[rank]
+        xr_at = [handle.buffer_ptrs[q] + offset for q in range(P)]
+        y_at = [a + cap * d_e * buf.element_size() for a in xr_at]
+        return buf[:cap], buf[cap:], xr_at, y_at
+
+    def _send(xe, pos, offsets, xr_at, first_row, cap):
+        ep_dispatch_rows(xe, pos, offsets, E, peer_rows(xr_at, first_row, [cap] * P), cfg.top_k)
+
+    def _experts(xr, recv_counts, y):
+        rc = torch.from_numpy(recv_counts).to(xr.device)
+        ep_expert_ffn(xr, rc, w1_local, w3_local, w2_local, act, y=y)
+
+    def _combine(y_at, first_row, cap, pos, offsets, w):
+        return ep_combine_rows(peer_rows(y_at, first_row, [cap] * P), pos, offsets, E, w,
+                               x_e.shape[1])
+
+    def _barrier():
         torch.cuda.current_stream().synchronize()
         dist.barrier(group=group)
 
-    ep_dispatch_rows(x_e, pos, offsets, E, peer_rows(xr_at, first_row, [cap] * P), cfg.top_k)
-    barrier()
-    rc = torch.from_numpy(recv_counts).to(x_e.device)
-    ep_expert_ffn(buf[:R], rc, w1_local, w3_local, w2_local, act, y=buf[cap:cap + R])
-    barrier()
-    out = ep_combine_rows(peer_rows(y_at, first_row, [cap] * P), pos, offsets, E, w, d_e)
-    barrier()
-    return out, idx, w
+    steps = P2PSteps(route=lambda xr: route(xr, W, bias, cfg), dispatch=_dispatch,
+                     buffers=_buffers, send_rows=_send, experts=_experts,
+                     combine_rows=_combine, barrier=_barrier)
+    return exchange_forward_p2p(x_r, x_e, steps, E, group)

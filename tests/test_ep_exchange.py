@@ -143,3 +143,102 @@ def test_p2p_plan_rejects_counts_that_do_not_split():
         p2p_plan(np.zeros((2, 5), dtype=np.int64), 0, 2)
     with pytest.raises(ValueError):
         p2p_plan(np.zeros((3, 6), dtype=np.int64), 0, 2)
+
+
+def _p2p_worker(rank, world, port, E, q, xr_bufs, y_bufs):
+    """exchange_forward_p2p with the compute steps taken by the CPU reference
+    and every rank's row buffers in shared memory, so a rank's send step
+    writes straight into the other ranks' buffers and its combine reads from
+    them, as the peer-memory kernels do on GPUs."""
+    import datetime
+    import torch
+    import torch.distributed as dist
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        import oracle
+        from moe_routing_expert_fp32_b200.ep import P2PSteps, exchange_forward_p2p
+        x, W, b, w1, w3, w2, K = _case(rank, E)
+        E_local = E // world
+        lo = rank * E_local
+        d = x.shape[1]
+
+        def route(xr):
+            idx, w, _ = oracle.route(xr.numpy().view(np.uint16), W, b, 1, 1, K, 1.5)
+            return torch.from_numpy(idx), torch.from_numpy(w)
+
+        def dispatch(idx, xe):
+            counts, offsets, _, pos = oracle.dispatch(idx.numpy(), E)
+            return torch.from_numpy(counts), torch.from_numpy(offsets), torch.from_numpy(pos)
+
+        def buffers(cap, d_e, like):
+            assert d_e == d and cap <= xr_bufs[0].shape[0]
+            return xr_bufs[rank], y_bufs[rank], xr_bufs, y_bufs
+
+        def owner(offs, j):
+            return next(r for r in range(world) if j < offs[(r + 1) * E_local])
+
+        def send_rows(xe, pos, offsets, xr_at, first_row, cap):
+            offs = offsets.numpy()
+            for s, j in enumerate(pos.numpy()):
+                if j < 0:
+                    continue
+                r = owner(offs, j)
+                row = first_row[r] + j - offs[r * E_local]
+                assert row < cap
+                xr_at[r][row] = xe[s // K]
+
+        def experts(xr, recv_counts, y):
+            rows = xr.numpy().view(np.uint16)
+            out = y.numpy().view(np.uint16)
+            o = 0
+            for p in range(recv_counts.shape[0]):
+                for e in range(recv_counts.shape[1]):
+                    n = int(recv_counts[p, e])
+                    if n:
+                        out[o:o + n] = oracle.expert_ffn(rows[o:o + n], w1[lo + e], w3[lo + e],
+                                                         w2[lo + e], "silu")
+                    o += n
+            assert o == rows.shape[0]
+
+        def combine_rows(y_at, first_row, cap, pos, offsets, w):
+            offs = offsets.numpy()
+            home = np.zeros((pos.numel(), d), np.uint16)  # outputs in sorted order
+            for r in range(world):
+                a, z = offs[r * E_local], offs[(r + 1) * E_local]
+                f = first_row[r]
+                home[a:z] = y_at[r][f:f + (z - a)].numpy().view(np.uint16)
+            return torch.from_numpy(oracle.combine(home, pos.numpy(), w.numpy(), K))
+
+        steps = P2PSteps(route, dispatch, buffers, send_rows, experts, combine_rows,
+                         lambda: dist.barrier())
+        xt = torch.from_numpy(x.view(np.int16))
+        out, idx, w = exchange_forward_p2p(xt, xt, steps, E)
+        ref = oracle.moe_infer(x, idx.numpy(), w.numpy(), w1, w3, w2, "silu")
+        q.put((rank, bool(np.array_equal(out.numpy(), ref)), int(idx.numel())))
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world,E", [(2, 8), (3, 12)])
+def test_exchange_forward_p2p_equals_one_rank(world, E):
+    import torch
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    cap = 256  # more rows than any rank receives here (all ranks: 81 or 153 slots)
+    xr_bufs = [torch.zeros((cap, 32), dtype=torch.int16).share_memory_() for _ in range(world)]
+    y_bufs = [torch.zeros((cap, 32), dtype=torch.int16).share_memory_() for _ in range(world)]
+    procs = [ctx.Process(target=_p2p_worker, args=(r, world, port, E, q, xr_bufs, y_bufs))
+             for r in range(world)]
+    for p in procs:
+        p.start()
+    res = [q.get(timeout=120) for _ in range(world)]
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    assert sorted(r[0] for r in res) == list(range(world))
+    assert all(r[1] for r in res), res
