@@ -64,7 +64,7 @@ def moe():
 
 @pytest.mark.parametrize("N,d,E", [(64, 256, 16), (128, 7168, 256), (64, 7168, 896),
                                    (4096, 7168, 384), (3000, 512, 100), (2000, 1024, 1024),
-                                   (2304, 9216, 128)])
+                                   (2304, 9216, 128), (2304, 16448, 128)])
 def test_gate_logits_match_reference(moe, N, d, E):
     x = synth.host_normal_bf16(5, 1, (N, d), 1.0)
     W = synth.host_normal_f32(5, 2, (E, d), 0.02)
