@@ -286,7 +286,13 @@ MOE_API int moe_ep_expert_ffn(const moe_bf16* xr, int64_t R, const int32_t* recv
  * source rank and sorted by local expert, the layout moe_ep_expert_ffn takes.
  * Ordering between ranks (all rows stored before a rank's experts read them,
  * all outputs written before the senders' combines load them) is the
- * caller's: a barrier across the ranks between the steps. */
+ * caller's: a barrier across the ranks between the steps.
+ * Host checks of both calls: MOE_ERR_INVALID_ARG for E % P != 0, a negative
+ * first_row or capacity, a NULL buffer with capacity > 0 or a NULL tensor
+ * pointer; MOE_ERR_UNSUPPORTED for P outside 1 .. MOE_MAX_PEERS, K > 16,
+ * E > 1024 or d_e % 8 != 0; MOE_ERR_ALIGNMENT for a buffer, x_e or out not
+ * 16-byte aligned; MOE_ERR_WORKSPACE for a missing or short workspace.
+ * N = 0 is a successful no-op. */
 #define MOE_MAX_PEERS 64
 
 typedef struct moe_peer_rows {
