@@ -20,7 +20,9 @@ One step on every rank:
 send kernel (moe_ep_dispatch_rows) stores each token row straight into the
 receiving ranks' buffers through peer addresses of a symmetric-memory
 allocation, and the combine (moe_ep_combine_rows) loads the outputs straight
-from the ranks that computed them; `p2p_plan` places every rank's rows.
+from the ranks that computed them; `p2p_plan` places every rank's rows and
+`exchange_forward_p2p` holds that step's logic, its compute and memory steps
+passed in as callables (`P2PSteps`).
 
 The collectives are torch.distributed all-to-alls (NCCL over NVLink on GPUs);
 their split sizes need the counts on the host, the one synchronisation of the
