@@ -360,3 +360,34 @@ def test_dispatch_without_the_copy_needs_no_rows(L):
     # an unaligned x_e matters only when the rows are copied
     assert L.moe_dispatch(p, 4, 2, 8, ctypes.c_void_p(264), 128, p, p, p, p, p, p, 1 << 20,
                           None) == -3
+
+
+def _a256(n):
+    return (n + 255) // 256 * 256
+
+
+@pytest.mark.parametrize("N,E,d", [(64, 16, 256), (128, 256, 7168), (64, 896, 7168),
+                                   (4096, 384, 7168), (16384, 384, 7168), (2303, 128, 9216),
+                                   (2304, 128, 9216), (3000, 100, 512), (5, 8, 96)])
+def test_bench_gate_mirror_matches_the_library(L, N, E, d):
+    """bench.py counts the router's gate launches from its own mirror of the
+    library's choice (int8 tiles: 3 launches; fp32 tiles: 1, or 2 when split
+    over d_r).  The library's route workspace shows which layout it chose:
+    the int8 path holds the digit planes and row scales, the fp32 path the
+    logits and, when split, the double partials."""
+    import bench
+    import moe_routing_expert_fp32_b200 as m
+    from synth.workloads import WORKLOADS, scaled
+    cfg = m.RouteConfig(E, 1, 1, min(8, E), 1.0, True)
+    ws = L.moe_route_workspace_size(N, d, ctypes.byref(cfg._c()))
+    i8 = _a256(4 * N * E) + _a256(4 * E * d) + _a256(4 * E) + _a256(4 * N * d) + _a256(4 * N)
+    wl = scaled(WORKLOADS["tiny"], N=N, E=E, d_r=d, G=1, TG=1)
+    n = bench.gate_kernels(wl)
+    if n == 3:
+        assert ws == 256 + i8
+    else:
+        logits = _a256(4 * N * E)
+        rest = ws - 256 - logits
+        assert (rest > 0) == (n == 2), (ws, n)
+        if n == 2:
+            assert rest % (8 * N * E) < 256  # splits x N x E doubles, 256-aligned
