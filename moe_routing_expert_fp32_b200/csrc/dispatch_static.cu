@@ -13,8 +13,11 @@
 // The array is a file-scope __device__ variable, so every GPU that loads this
 // library holds MOE_DISPATCH_STATIC_SCRATCH_BYTES of it until the process
 // exits.  In host code `g_dispatch_scratch` names a host-side stand-in, not a
-// device address; the device address is looked up once per device with
-// cudaGetSymbolAddress (with that device current) and passed to the kernels.
+// device address; the device address is looked up with cudaGetSymbolAddress
+// once per device context (the first call made with that context current,
+// normally the device's primary context) and passed to the kernels.
+#include <cuda.h>
+
 #include <mutex>
 
 #include "moe_internal.cuh"
@@ -24,22 +27,51 @@ namespace {
 
 __device__ __align__(256) uint8_t g_dispatch_scratch[MOE_DISPATCH_STATIC_SCRATCH_BYTES];
 
-// Device address of g_dispatch_scratch on the current device, looked up on
-// the first call made with that device current; nullptr if the lookup failed.
-uint8_t* static_scratch_ptr() {
-  static std::mutex mu;
-  static uint8_t* ptr[64] = {nullptr};
-  static bool tried[64] = {false};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
-  std::lock_guard<std::mutex> lock(mu);
-  if (!tried[dev]) {
-    tried[dev] = true;
+// The driver context current on this thread, or nullptr (none current, or
+// the driver entry point is unavailable).  The symbol's device address is
+// valid only in the context it was looked up in, so the cache below is keyed
+// by context rather than by device number: a caller that switches between a
+// device's primary context and a context of its own gets each one's address.
+void* current_context() {
+  typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+  static const CtxGetCurrentFn fn = [] {
     void* p = nullptr;
-    const cudaError_t rc = cudaGetSymbolAddress(&p, g_dispatch_scratch);
-    if (rc == cudaSuccess) ptr[dev] = static_cast<uint8_t*>(p);
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      return reinterpret_cast<CtxGetCurrentFn>(p);
+    return static_cast<CtxGetCurrentFn>(nullptr);
+  }();
+  CUcontext c = nullptr;
+  if (!fn || fn(&c) != CUDA_SUCCESS) return nullptr;
+  return c;
+}
+
+// Device address of g_dispatch_scratch in the current context.  The lookup
+// runs on the first call made with a context current and is cached only when
+// it succeeds; a failed lookup (for instance a first call made during stream
+// capture) clears its error and returns nullptr, so a later call can retry.
+uint8_t* static_scratch_ptr() {
+  struct Entry {
+    void* ctx;
+    uint8_t* ptr;
+  };
+  static std::mutex mu;
+  static Entry cache[kMaxDevices];
+  static int n_cached = 0;
+  std::lock_guard<std::mutex> lock(mu);
+  void* ctx = current_context();
+  if (ctx)
+    for (int i = 0; i < n_cached; ++i)
+      if (cache[i].ctx == ctx) return cache[i].ptr;
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_dispatch_scratch) != cudaSuccess || !p) {
+    (void)cudaGetLastError();  // leave no pending error behind
+    return nullptr;
   }
-  return ptr[dev];
+  ctx = current_context();  // the lookup makes the primary context current if none was
+  if (ctx && n_cached < kMaxDevices) cache[n_cached++] = Entry{ctx, static_cast<uint8_t*>(p)};
+  return static_cast<uint8_t*>(p);
 }
 
 }  // namespace
@@ -56,9 +88,10 @@ extern "C" int moe_dispatch_static(const int32_t* topk_idx, int64_t N, int K, in
   if (d_e % 8 != 0) return MOE_ERR_UNSUPPORTED;
   if (N * (int64_t)K > INT32_MAX) return MOE_ERR_UNSUPPORTED;
   if (!counts || !offsets) return MOE_ERR_INVALID_ARG;
-  if (N > 0 && (!topk_idx || !x_e || !perm || !pos || !xs)) return MOE_ERR_INVALID_ARG;
-  if (N > 0 && ((reinterpret_cast<uintptr_t>(x_e) & 15u) ||
-                (reinterpret_cast<uintptr_t>(xs) & 15u)))
+  // xs == NULL: the sort only, x_e is not read (as in moe_dispatch)
+  if (N > 0 && (!topk_idx || !perm || !pos || (xs && !x_e))) return MOE_ERR_INVALID_ARG;
+  if (N > 0 && xs && ((reinterpret_cast<uintptr_t>(x_e) & 15u) ||
+                      (reinterpret_cast<uintptr_t>(xs) & 15u)))
     return MOE_ERR_ALIGNMENT;
   // The per-chunk counts of this call must fit in the fixed array.
   if (dispatch_scratch_bytes(N * K, E) > MOE_DISPATCH_STATIC_SCRATCH_BYTES)

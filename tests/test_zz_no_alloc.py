@@ -83,3 +83,26 @@ def test_static_dispatch_rejects_sizes_beyond_its_array():
     idx = torch.from_numpy(random_topk(50, 2, 7, np.random.default_rng(1))).cuda()
     x = dev_bf16(synth.host_normal_bf16(2, 1, (50, 128), 1.0))
     _same(torch, moe.dispatch_static(idx, x, 7), moe.dispatch(idx, x, 7))
+
+
+def test_static_dispatch_sort_only_matches_dispatch():
+    """xs = NULL: only counts, offsets, perm and pos, as moe_dispatch gives them
+    with gather=False; x_e is not read, so a NULL x_e is accepted too."""
+    import torch
+    import moe_routing_expert_fp32_b200 as moe
+    L = moe.lib()
+    vp = lambda t: ctypes.c_void_p(t.data_ptr())  # noqa: E731
+    for i, (N, K, E) in enumerate([(128, 8, 256), (4096, 8, 384), (1, 1, 3)]):
+        idx = torch.from_numpy(random_topk(N, K, E, np.random.default_rng(70 + i),
+                                           1.2 if N > 1000 else 0.0)).cuda()
+        x = dev_bf16(synth.host_normal_bf16(4, 1, (N, 128), 1.0))
+        ref = moe.dispatch(idx, x, E, gather=False)[:4]
+        got = moe.dispatch_static(idx, x, E, gather=False)
+        assert got[4] is None
+        _same(torch, got[:4], ref)
+        c, o, p, q = (torch.empty_like(t) for t in ref)
+        rc = L.moe_dispatch_static(vp(idx), N, K, E, None, 128, vp(c), vp(o), vp(p), vp(q), None,
+                                   ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+        assert rc == 0
+        torch.cuda.synchronize()
+        _same(torch, (c, o, p, q), ref)
