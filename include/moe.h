@@ -192,9 +192,14 @@ MOE_API int moe_dispatch(const int32_t* topk_idx, int64_t N, int K, int E, const
  * the process exits.  Calls whose per-chunk counts (4 * chunks * E bytes,
  * chunks = ceil(N*K / clamp(N*K/256, 64, 1024) rounded up to 32)) exceed it
  * return MOE_ERR_UNSUPPORTED; 131072 slots over 384 experts use 0.4 MiB.
- * Set-up: the first call made on a device looks up the array's device
- * address (cudaGetSymbolAddress) with that device current; make that first
- * call before any stream capture.
+ * Set-up: the first call made with a given CUDA context current (normally
+ * the device's primary context) looks up the array's device address in that
+ * context (cudaGetSymbolAddress) and caches it for that context; make that
+ * first call before any stream capture.  A lookup that fails is not cached:
+ * the call returns MOE_ERR_CUDA, leaves no pending CUDA error, and a later
+ * call tries again.
+ * xs may be NULL exactly as in moe_dispatch: then only counts, offsets, perm
+ * and pos are written and x_e is not read.
  * Every call shares the one array and overwrites it, so calls that can
  * overlap on the GPU (different streams, or different host threads without
  * ordering) race and corrupt each other's results; serialise them on one
@@ -446,6 +451,13 @@ MOE_API int moe_get_status(void* ws, void* stream);
 
 /* Text for a moe_status code. */
 MOE_API const char* moe_strerror(int code);
+
+/* Kernels this library has launched in this process so far, over all devices
+ * and host threads (the launches the CUDA runtime accepted).  A caller that
+ * accounts for GPU work reads it before and after a region: the difference is
+ * the number of libmoe kernels that region enqueued.  Not part of the pages'
+ * method: bookkeeping for measurement. */
+MOE_API uint64_t moe_launch_count(void);
 
 #ifdef __cplusplus
 }

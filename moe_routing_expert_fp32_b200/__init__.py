@@ -150,7 +150,7 @@ EXPORTS = ("moe_route_workspace_size", "moe_route", "moe_route_from_logits",
            "moe_linear_workspace_size", "moe_linear", "moe_rms_norm", "moe_block_workspace_size",
            "moe_block_forward", "moe_shared_experts_workspace_size", "moe_shared_experts",
            "moe_ep_expert_ffn_workspace_size", "moe_ep_expert_ffn", "moe_expert_ffn_gathered",
-           "moe_ep_dispatch_rows", "moe_ep_combine_rows")
+           "moe_ep_dispatch_rows", "moe_ep_combine_rows", "moe_launch_count")
 
 
 def lib() -> ctypes.CDLL:
@@ -198,6 +198,7 @@ def lib() -> ctypes.CDLL:
         "moe_block_forward": ([vp, i64, bd, bw, rc, ac, vp, vp, vp, vp, sz, vp], i32),
         "moe_ep_dispatch_rows": ([vp, i64, i32, i32, vp, vp, i32, pr, vp, sz, vp], i32),
         "moe_ep_combine_rows": ([pr, vp, vp, i32, vp, i64, i32, i32, vp, vp, sz, vp], i32),
+        "moe_launch_count": ([], ctypes.c_uint64),
     }
     for name, (args, res) in sig.items():
         fn = getattr(L, name)
@@ -205,6 +206,11 @@ def lib() -> ctypes.CDLL:
         fn.restype = res
     _lib = L
     return L
+
+
+def launch_count() -> int:
+    """Kernels libmoe has launched in this process so far (moe_launch_count)."""
+    return int(lib().moe_launch_count())
 
 
 # ----------------------------------------------------------------- helpers
@@ -322,12 +328,13 @@ def dispatch(topk_idx, x_e, num_experts: int, ws=None, gather=True):
     return counts, offsets, perm, pos, xs
 
 
-def dispatch_static(topk_idx, x_e, num_experts: int):
+def dispatch_static(topk_idx, x_e, num_experts: int, gather=True):
     """moe_dispatch without a workspace, for callers that cannot allocate device
     memory: the scratch is a fixed 2 MiB array inside libmoe.so (see
     moe_dispatch_static in include/moe.h for its limit and sharing rules).
     This Python wrapper still allocates its outputs with torch; a caller that
-    cannot allocate passes its own buffers to the C entry point."""
+    cannot allocate passes its own buffers to the C entry point.  With
+    gather=False the rows are not copied and xs is None."""
     torch = _torch()
     N, K = topk_idx.shape
     d_e = x_e.shape[1]
@@ -340,7 +347,7 @@ def dispatch_static(topk_idx, x_e, num_experts: int):
     offsets = torch.empty(E + 1, dtype=torch.int32, device=dev)
     perm = torch.empty(S, dtype=torch.int32, device=dev)
     pos = torch.empty(S, dtype=torch.int32, device=dev)
-    xs = torch.empty((S, d_e), dtype=torch.bfloat16, device=dev)
+    xs = torch.empty((S, d_e), dtype=torch.bfloat16, device=dev) if gather else None
     _check("moe_dispatch_static",
            lib().moe_dispatch_static(_ptr(topk_idx), N, K, E, _ptr(x_e), d_e, _ptr(counts),
                                      _ptr(offsets), _ptr(perm), _ptr(pos), _ptr(xs), _stream()))

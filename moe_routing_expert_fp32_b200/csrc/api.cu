@@ -3,11 +3,18 @@
 // kernels of router.cu, dispatch.cu, expert_gemm.cu and combine.cu.
 #include <math.h>
 
+#include <atomic>
 #include <mutex>
 
 #include "moe_internal.cuh"
 
 namespace moe {
+
+namespace {
+std::atomic<uint64_t> g_launches{0};
+}  // namespace
+
+void count_launches(int n) { g_launches.fetch_add((uint64_t)n, std::memory_order_relaxed); }
 
 const DevInfo* dev_info() {
   static std::mutex mu;
@@ -112,6 +119,8 @@ const char* moe_strerror(int code) {
     default: return "unknown moe_status";
   }
 }
+
+uint64_t moe_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 
 int moe_get_status(void* ws, void* stream) {
   if (!ws) return MOE_ERR_INVALID_ARG;

@@ -1186,10 +1186,10 @@ cudaError_t launch_gemm(const CUtensorMap& a0, const CUtensorMap& a1, const CUte
   cfg.stream = s;
   cfg.attrs = attr;
   cfg.numAttrs = pdl ? 1 : 0;
-  return cudaLaunchKernelEx(&cfg, k_expert_gemm<MODE, NTMAX, STAGES, UM, KSUB>, a0, a1, b, b64,
+  return counted(cudaLaunchKernelEx(&cfg, k_expert_gemm<MODE, NTMAX, STAGES, UM, KSUB>, a0, a1, b, b64,
                             offsets, tile_start, E, M_rows, Kdim, out, res, (int)act.kind,
                             act.beta, act.linear_beta, st, pdl, gperm, gk, gn, ksplit, part,
-                            emod > 0 ? emod : E);
+                            emod > 0 ? emod : E));
 }
 
 // Launches the CTA-pair kernel on as many pairs as can be resident at once.
@@ -1238,9 +1238,9 @@ cudaError_t launch_gemm_pair(const CUtensorMap& a0, const CUtensorMap& a1, const
   cudaGetDevice(&dev);
   cfg.gridDim = dim3(grid_of[dev], 1, 1);
   cfg.numAttrs = pdl ? 2 : 1;
-  return cudaLaunchKernelEx(&cfg, k_expert_gemm_pair<MODE>, a0, a1, b, b64, offsets, tile_start,
+  return counted(cudaLaunchKernelEx(&cfg, k_expert_gemm_pair<MODE>, a0, a1, b, b64, offsets, tile_start,
                             E, M_rows, Kdim, out, res, (int)act.kind, act.beta, act.linear_beta,
-                            st, pdl, emod > 0 ? emod : E);
+                            st, pdl, emod > 0 ? emod : E));
 }
 
 // Variant choice from shapes only (no host round trip), by the average rows

@@ -56,6 +56,15 @@ __device__ __forceinline__ void pdl_trigger() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
+// Every kernel launch of the library is counted (moe_launch_count): the
+// launch sites pass their result through counted(), which adds n launches
+// when the launch was accepted.
+void count_launches(int n);
+inline cudaError_t counted(cudaError_t e, int n = 1) {
+  if (e == cudaSuccess) count_launches(n);
+  return e;
+}
+
 template <typename... KArgs, typename... Args>
 cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
                        cudaStream_t s, Args... args) {
@@ -69,7 +78,7 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+  return counted(cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...));
 }
 
 // --------------------------------------------------------- kernel launches

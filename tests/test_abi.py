@@ -252,15 +252,12 @@ def test_ep_expert_ffn_validation(L):
                                0, None) == -4
 
 
-def test_bench_split_mirror_matches_the_library(L):
-    """bench.py counts a reduce kernel after every dense layer the library
-    splits over K; its mirror of that choice must agree with the library's
-    own workspace (split partials present <=> split)."""
-    import bench
-    for M in (1, 7, 16, 17, 64, 100, 128, 129, 300):
-        for K, N_out in ((7168, 2048), (2048, 7168), (256, 128), (128, 256), (3072, 7168)):
-            split = L.moe_linear_workspace_size(M, K, N_out) > 512
-            assert bench.dense_split(M, N_out, K, False) == split, (M, K, N_out)
+def test_launch_count_is_exported_and_starts_without_gpu_work(L):
+    """moe_launch_count is the library's own tally of accepted kernel launches;
+    calls rejected on the host add nothing to it."""
+    before = L.moe_launch_count()
+    assert L.moe_combine(None, None, None, 4, 0, 128, None, None, 0, None) == -1  # K = 0
+    assert L.moe_launch_count() == before
 
 
 def _dispatch_chunks(S):
@@ -362,32 +359,3 @@ def test_dispatch_without_the_copy_needs_no_rows(L):
                           None) == -3
 
 
-def _a256(n):
-    return (n + 255) // 256 * 256
-
-
-@pytest.mark.parametrize("N,E,d", [(64, 16, 256), (128, 256, 7168), (64, 896, 7168),
-                                   (4096, 384, 7168), (16384, 384, 7168), (2303, 128, 9216),
-                                   (2304, 128, 9216), (3000, 100, 512), (5, 8, 96)])
-def test_bench_gate_mirror_matches_the_library(L, N, E, d):
-    """bench.py counts the router's gate launches from its own mirror of the
-    library's choice (int8 tiles: 3 launches; fp32 tiles: 1, or 2 when split
-    over d_r).  The library's route workspace shows which layout it chose:
-    the int8 path holds the digit planes and row scales, the fp32 path the
-    logits and, when split, the double partials."""
-    import bench
-    import moe_routing_expert_fp32_b200 as m
-    from synth.workloads import WORKLOADS, scaled
-    cfg = m.RouteConfig(E, 1, 1, min(8, E), 1.0, True)
-    ws = L.moe_route_workspace_size(N, d, ctypes.byref(cfg._c()))
-    i8 = _a256(4 * N * E) + _a256(4 * E * d) + _a256(4 * E) + _a256(4 * N * d) + _a256(4 * N)
-    wl = scaled(WORKLOADS["tiny"], N=N, E=E, d_r=d, G=1, TG=1)
-    n = bench.gate_kernels(wl)
-    if n == 3:
-        assert ws == 256 + i8
-    else:
-        logits = _a256(4 * N * E)
-        rest = ws - 256 - logits
-        assert (rest > 0) == (n == 2), (ws, n)
-        if n == 2:
-            assert rest % (8 * N * E) < 256  # splits x N x E doubles, 256-aligned

@@ -1,0 +1,50 @@
+"""moe_launch_count counts the kernels the library actually launched: one per
+combine, four per dispatch that copies rows (histogram, scan, scatter,
+gather), three per sort-only dispatch, and the same number for every
+repetition of one moe_forward."""
+import numpy as np
+import pytest
+
+import synth
+from tests.gpu_util import dev_bf16, random_topk
+
+pytestmark = pytest.mark.gpu
+
+
+def test_launch_count_per_entry_point():
+    import torch
+    import moe_routing_expert_fp32_b200 as moe
+    N, K, E, d = 300, 4, 40, 256
+    idx = torch.from_numpy(random_topk(N, K, E, np.random.default_rng(5))).cuda()
+    x = dev_bf16(synth.host_normal_bf16(3, 1, (N, d), 1.0))
+    moe.dispatch(idx, x, E)  # first call: kernel attributes set up
+    n0 = moe.launch_count()
+    counts, offsets, perm, pos, xs = moe.dispatch(idx, x, E)
+    n1 = moe.launch_count()
+    moe.dispatch(idx, x, E, gather=False)
+    n2 = moe.launch_count()
+    w = torch.rand((N, K), dtype=torch.float32, device="cuda")
+    moe.combine(xs, pos, w)
+    n3 = moe.launch_count()
+    torch.cuda.synchronize()
+    assert (n1 - n0, n2 - n1, n3 - n2) == (4, 3, 1)
+
+
+def test_launch_count_of_forward_is_stable():
+    import torch
+    import moe_routing_expert_fp32_b200 as moe
+    from synth.workloads import WORKLOADS, dev_inputs
+    wl = WORKLOADS["tiny"]
+    dev = dev_inputs(wl)
+    cfg = moe.RouteConfig(wl.E, wl.G, wl.TG, wl.K, wl.route_scale, wl.norm)
+    act = moe.ActConfig(wl.act, wl.beta, wl.lbeta)
+    ws = moe.workspace(moe.workspace_size(wl.N, wl.d_r, wl.d_e, cfg, wl.F))
+    deltas = []
+    for _ in range(3):
+        n0 = moe.launch_count()
+        moe.forward(dev["x"], dev["W"], dev["bias"], cfg, dev["w1"], dev["w3"], dev["w2"], act,
+                    ws=ws)
+        deltas.append(moe.launch_count() - n0)
+    torch.cuda.synchronize()
+    # route (gate GEMM + selection), dispatch (4), tile list, two expert GEMMs, combine
+    assert deltas[0] == deltas[1] == deltas[2] and 10 <= deltas[0] <= 13
