@@ -2,16 +2,24 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
 
-One step = one moe_forward over one batch of the workload (default: the
-DeepSeek-V3.2-shaped decode batch, N=128 tokens, d=7168, 256 experts, top-8,
-d_ff=2048).  Inputs are seeded and synthetic, drawn on the device; the
-expert weights (22.5 GB) are larger than L2 and L2 is also flushed (256 MB
-write) between steps, outside the per-step events.  Under torchrun every rank
-runs its own batch (token rows rank*N .. rank*N+N-1) with the same weights:
-weak scaling with no collective on the data path; the step time is the max
-over ranks.  Rank 0 prints one JSON line.  `--workload k3_block_decode` (or
-tiny_block) times the whole MoE block instead (moe_block_forward: gate,
-shared experts, latent projections and norm around the routed layer).
+One step = one moe_forward over one batch of the workload.  The default is the
+largest single-GPU workload, the skewed Kimi-K2-shaped batch: N=16384 tokens,
+d=7168, 384 experts, top-8, d_ff=2048, a correction bias calibrated so that
+expert popularity follows Zipf(1.2) with 20 experts receiving no token (the
+other workloads are selected with --workload).  Inputs are seeded and
+synthetic, drawn on the device; the expert weights (33.8 GB) are larger than
+L2 and L2 is also flushed (256 MB write) between steps, outside the per-step
+events.  Under torchrun every rank runs its own batch (token rows rank*N ..
+rank*N+N-1) with the same weights: weak scaling with no collective on the
+data path; the step time is the max over ranks.  Rank 0 prints one JSON line.
+`--workload k3_block_decode` (or tiny_block) times the whole MoE block instead
+(moe_block_forward: gate, shared experts, latent projections and norm around
+the routed layer).
+
+`value` is tokens over the mean of the K per-step CUDA-event times (the
+median is reported beside it); `stages_ms` comes from a second pass of K
+steps with an event after every stage.  `gpu_launches` is the library's own
+count of the kernels it launched in the timed region (moe_launch_count).
 
 The `e2e` figure is the same step through the public API from pinned host
 memory, each step uploading its tokens and downloading its output; the
@@ -19,8 +27,8 @@ copies of neighbouring steps overlap on two copy streams (double-buffered),
 and the timed region spans the first upload to the last download.
 
 --impl reference times the CPU reference (oracle/) on the host cores on a
-bounded sample of the same workload; it is the slow reference arm, not a
-target.
+bounded sample of the same workload (its line says which sample and that the
+figure is extrapolated from it); it is the slow reference arm, not a target.
 """
 from __future__ import annotations
 
@@ -41,27 +49,10 @@ if ROOT not in sys.path:
 
 METRIC = "routed tokens/sec per MoE layer (route+dispatch+FFN+combine)"
 UNIT = "tokens/s"
-DEFAULT_WORKLOAD = "dsv32_decode"
-# select, hist, scan, scatter, gather, tiles, gate_up, down, combine, plus the gate GEMM:
-# gate_partial [+ reduce_partials when split over d_r] for decode batches, or
-# slice(W) + slice(x) + gate_i8 once the batch fills 24 tiles of 128 x 96
-KERNELS_AFTER_GATE = 9
-
-
-def gate_kernels(wl):
-    """Launches of the router's gate GEMM (mirrors the library's choice)."""
-    if ((wl.E + 127) // 128) * ((wl.N + 95) // 96) >= 24 and wl.d_r % 64 == 0 \
-            and wl.d_r <= 32768:
-        return 3
-    tiles = max(1, ((wl.E + 63) // 64) * ((wl.N + 63) // 64))
-    nk = max(1, wl.d_r // 32)
-    want = max(1, min((296 + tiles - 1) // tiles, max(nk // 4, 1), 32))
-    cps = (nk + want - 1) // want
-    return 1 + (1 if (nk + cps - 1) // cps > 1 else 0)
-
-
-def kernels_per_step(wl):
-    return gate_kernels(wl) + KERNELS_AFTER_GATE
+DEFAULT_WORKLOAD = "k2_skew"
+# nominal B200 figures, reported beside the measured peaks for context
+NOMINAL_HBM_GBS = 7700.0
+NOMINAL_BF16_TFLOPS = 2250.0
 
 
 def parse():
@@ -285,6 +276,7 @@ def run_ours(args, rank, world, local_rank):
     with ClockSampler(local_rank) as clk:
         barrier()
         torch.cuda.synchronize()
+        n0 = moe.launch_count()
         t0 = time.perf_counter()
         for i in range(args.steps):
             flush.zero_()
@@ -294,6 +286,7 @@ def run_ours(args, rank, world, local_rank):
         torch.cuda.synchronize()
         barrier()
         wall = time.perf_counter() - t0
+        launches = moe.launch_count() - n0
     per_step = [a.elapsed_time(b) for a, b in ev0]
     ms = statistics.mean(per_step)
 
@@ -343,47 +336,20 @@ def run_ours(args, rank, world, local_rank):
     ms_max, e2e_max, gu_ms, wall_max = max_over_ranks(
         [ms, statistics.mean(e2e_ms), stage_ms["gate_up"], wall], world, "cuda")
 
+    srt = np.sort(counts)[::-1]
+    top10 = float(srt[: max(1, wl.E // 10)].sum() / max(1, counts.sum()))
     res = {
         "ms": ms_max, "e2e_ms": e2e_max, "stage_ms": stage_ms, "gate_up_ms": gu_ms,
         "step_ms": [min(per_step), statistics.median(per_step), max(per_step)],
-        "touched": touched, "counts_max": int(counts.max()), "clocks": clk.summary(),
-        "h2d": h2d, "d2h": d2h, "wall_s": wall_max,
+        "touched": touched, "counts_max": int(counts.max()), "top10_share": top10,
+        "clocks": clk.summary(), "h2d": h2d, "d2h": d2h, "wall_s": wall_max,
+        "launches": launches,
     }
     return wl, res
 
 
 # ------------------------------------------------------ whole-block arm
 BLOCK_METRIC = "tokens/sec per MoE block (route+shared experts+latent projections+routed experts)"
-
-
-def dense_split(M, M_rows, K, gate_up):
-    """Whether a dense layer of M rows runs split over K (then a reduce kernel
-    follows its GEMM); mirrors the library's choice, a function of shapes."""
-    if M > 128 * 1:  # CTA-pair variant: never split
-        return False
-    decode = M <= 16
-    nt, um, ks = (32, 1, 128) if decode else (128, 2, 64)
-    unit_rows = um * (64 if gate_up else 128)
-    units = ((M + nt - 1) // nt) * ((M_rows + unit_rows - 1) // unit_rows)
-    if units * 2 >= 148:
-        return False
-    k = min((148 + units - 1) // units, (K // ks) // 2, 32)
-    return k > 1
-
-
-def block_kernels(wl):
-    """The routed layer's launches plus the dense tile list, the shared
-    experts' two GEMMs and the two latent projections, each followed by a
-    reduce kernel when it runs split over K (the RMSNorm is fused into the
-    combine)."""
-    n = kernels_per_step(wl) + 1
-    N = wl.N
-    if wl.F_shared:
-        n += 2 + dense_split(N, wl.F_shared, wl.d_r, True) + dense_split(N, wl.d_r, wl.F_shared,
-                                                                          False)
-    if wl.latent:
-        n += 2 + dense_split(N, wl.d_e, wl.d_r, False) + dense_split(N, wl.d_r, wl.d_e, False)
-    return n
 
 
 def block_bytes(wl, touched):
@@ -453,6 +419,7 @@ def run_block(args, rank, world, local_rank):
     with ClockSampler(local_rank) as clk:
         barrier()
         torch.cuda.synchronize()
+        n0 = moe.launch_count()
         t0 = time.perf_counter()
         for i in range(args.steps):
             flush.zero_()
@@ -462,7 +429,9 @@ def run_block(args, rank, world, local_rank):
         torch.cuda.synchronize()
         barrier()
         wall = time.perf_counter() - t0
-    ms = statistics.mean(a.elapsed_time(b) for a, b in ev0)
+        launches = moe.launch_count() - n0
+    per_step = [a.elapsed_time(b) for a, b in ev0]
+    ms = statistics.mean(per_step)
     counts = np.bincount(idx.cpu().numpy().ravel(), minlength=wl.E)
     touched = int((counts > 0).sum())
 
@@ -475,7 +444,9 @@ def run_block(args, rank, world, local_rank):
     e2e_ms = [e2e_pipelined(torch, args.steps, hosts, e2e_run, out)]
     ms_max, e2e_max, wall_max = max_over_ranks([ms, statistics.mean(e2e_ms), wall], world, "cuda")
     return wl, {"ms": ms_max, "e2e_ms": e2e_max, "touched": touched, "clocks": clk.summary(),
-                "h2d": wl.N * wl.d_r * 2, "d2h": wl.N * wl.d_r * 2, "wall_s": wall_max}
+                "h2d": wl.N * wl.d_r * 2, "d2h": wl.N * wl.d_r * 2, "wall_s": wall_max,
+                "launches": launches,
+                "step_ms": [min(per_step), statistics.median(per_step), max(per_step)]}
 
 
 def block_line(args, wl, r, world):
@@ -495,10 +466,14 @@ def block_line(args, wl, r, world):
         "roofline": {"kernel": "whole block step (HBM-bound weight stream)", "bound": "hbm",
                      "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                      "frac": achieved / peaks["hbm_gbs"], "traffic": None,
-                     "peak_source": peaks["source"], "touched_experts": r["touched"]},
+                     "peak_source": peaks["source"], "touched_experts": r["touched"],
+                     "peak_nominal": NOMINAL_HBM_GBS,
+                     "frac_of_nominal": achieved / NOMINAL_HBM_GBS},
         "e2e": {"value": aggregate_throughput(wl.N, world, r["e2e_ms"]), "unit": UNIT,
                 "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"]},
-        "gpu_launches": block_kernels(wl) * args.steps,
+        "step_ms_min_median_max": r["step_ms"],
+        "step_ms_stat": "mean of the K per-step CUDA-event times",
+        "gpu_launches": r["launches"],
         "clocks": r["clocks"],
     }
 
@@ -548,75 +523,158 @@ def gate_up_roofline(wl, touched, gate_up_ms, peaks):
         obj.update({"bound": "tensor", "achieved": achieved,
                     "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
                     "frac": achieved / peaks["bf16_tflops_sustained"], "traffic": None,
-                    "peak_kind": "sustained bf16"})
+                    "peak_kind": "sustained bf16", "peak_nominal": NOMINAL_BF16_TFLOPS,
+                    "frac_of_nominal": achieved / NOMINAL_BF16_TFLOPS})
     else:
         achieved = nbytes / sec / 1e9
         obj.update({"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"],
                     "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
-                    "traffic": gate_up_traffic(touched)})
+                    "traffic": gate_up_traffic(touched), "peak_nominal": NOMINAL_HBM_GBS,
+                    "frac_of_nominal": achieved / NOMINAL_HBM_GBS})
     obj.update({"peak_source": peaks["source"], "touched_experts": touched})
     return obj
 
 
 # ------------------------------------------------------------ oracle arm
-def oracle_sample(wl, n_experts=8, router=("sigmoid", "top2_sum")):
-    """Time the CPU reference on a bounded sample of the workload.
+ROUTE_SAMPLE_TOKENS = 2048   # tokens routed, sorted and combined per sample
+FFN_SAMPLE_ROWS = 240        # expert-MLP rows per sample
+FFN_SAMPLE_EXPERTS = 8       # at most this many experts' weights drawn per sample
+SUBSET_TOKENS = 256          # the single-threaded subset
+SUBSET_FFN_ROWS = 24
 
-    Route, dispatch and combine run on the whole batch; the expert MLP runs on
-    the rows of the first `n_experts` experts that received rows and its time
-    is scaled by (all slots / sampled slots).  Returns tokens/s and details.
-    """
+
+def _router_codes(router):
     import oracle
-    import synth
-    from synth.workloads import host_inputs, host_expert
+    return ({"sigmoid": oracle.SCORE_SIGMOID, "softmax": oracle.SCORE_SOFTMAX}[router[0]],
+            {"top2_sum": oracle.GROUP_TOP2_SUM, "max": oracle.GROUP_MAX}[router[1]])
+
+
+def _oracle_step(wl, inp, n_tok, n_rows, router):
+    """One bounded pass of the CPU reference over the first `n_tok` tokens of
+    the batch: route, sort + gather and combine run on all of them; the
+    expert MLP runs on up to `n_rows` of their sorted rows, taken from the
+    least-, median- and most-loaded experts they touch and, while those hold
+    too few rows, the next most-loaded ones (the cost of a row does not
+    depend on its expert).
+    Returns the measured seconds of each stage, each scaled to the whole
+    batch (route, sort and combine by N / n_tok, the MLP by N*K / n_rows),
+    and what was sampled."""
+    import oracle
+    from synth.workloads import host_expert
+
+    score, group = _router_codes(router)
+    x = np.ascontiguousarray(inp["x"][:n_tok])
+    xe = np.ascontiguousarray(inp["x_e"][:n_tok])
+    raw = {}
+    t0 = time.perf_counter()
+    idx, w, _ = oracle.route(x, inp["W"], inp["bias"], wl.G, wl.TG, wl.K, wl.route_scale,
+                             wl.norm, score=score, group=group)
+    raw["route"] = time.perf_counter() - t0
+    t0 = time.perf_counter()
+    counts, offsets, perm, pos = oracle.dispatch(idx, wl.E)
+    xs = oracle.gather(xe, perm, wl.K)
+    raw["dispatch"] = time.perf_counter() - t0
+    touched = [int(e) for e in np.argsort(counts, kind="stable") if counts[e] > 0]
+    # the least-, median- and most-loaded experts, then the next most-loaded
+    # ones (at most FFN_SAMPLE_EXPERTS) while their rows fall short of n_rows
+    picks = list(dict.fromkeys([touched[0], touched[len(touched) // 2], touched[-1]]))
+    for e in reversed(touched):
+        if len(picks) >= FFN_SAMPLE_EXPERTS or int(counts[picks].sum()) >= n_rows:
+            break
+        if e not in picks:
+            picks.append(e)
+    # an equal share each, the lighter experts' shortfall taken by the heavier
+    spans, left = [], min(n_rows, int(counts[picks].sum()))
+    for i, e in enumerate(picks):
+        take = min(int(counts[e]), left // (len(picks) - i))
+        spans.append((e, int(offsets[e]), int(offsets[e]) + take))
+        left -= take
+    weights = {e: host_expert(wl, e) for e in picks}  # inputs, not timed
+    ys = np.zeros_like(xs)
+    done = 0
+    t0 = time.perf_counter()
+    for e, a, b in spans:
+        ys[a:b] = oracle.expert_ffn(xs[a:b], *weights[e], wl.act, wl.beta, wl.lbeta)
+        done += b - a
+    raw["ffn"] = time.perf_counter() - t0
+    t0 = time.perf_counter()
+    oracle.combine(ys, pos, w, wl.K)
+    raw["combine"] = time.perf_counter() - t0
+    scale_tok = wl.N / n_tok
+    scaled_s = {"route": raw["route"] * scale_tok, "dispatch": raw["dispatch"] * scale_tok,
+                "ffn": raw["ffn"] * wl.N * wl.K / max(done, 1),
+                "combine": raw["combine"] * scale_tok}
+    what = (f"route, sort+gather and combine of the first {n_tok} of {wl.N} tokens (time x "
+            f"{scale_tok:g}); expert MLP on {done} of their sorted rows from experts "
+            f"{[(e, b - a) for e, a, b in spans]} ((expert, rows): least-, median-, most-loaded, "
+            f"then the next most-loaded; "
+            f"time x {wl.N * wl.K}/{done} slots)")
+    return scaled_s, raw, what
+
+
+def oracle_sample(wl, router=("sigmoid", "top2_sum")):
+    """The CPU reference on all host cores over a bounded sample of one step
+    (_oracle_step with ROUTE_SAMPLE_TOKENS tokens and FFN_SAMPLE_ROWS MLP
+    rows), extrapolated to the whole batch.  Returns tokens/s, the cores
+    used, the per-stage seconds (extrapolated and as measured) and the
+    sample's description."""
+    import oracle
+    from synth.workloads import host_inputs
 
     oracle.set_threads(os.cpu_count() or 1)
     cores = oracle.max_threads()
-    inp = host_inputs(wl)
-    t = {}
-    t0 = time.perf_counter()
-    idx, w, _ = oracle.route(inp["x"], inp["W"], inp["bias"], wl.G, wl.TG, wl.K,
-                             wl.route_scale, wl.norm,
-                             score={"sigmoid": oracle.SCORE_SIGMOID,
-                                    "softmax": oracle.SCORE_SOFTMAX}[router[0]],
-                             group={"top2_sum": oracle.GROUP_TOP2_SUM,
-                                    "max": oracle.GROUP_MAX}[router[1]])
-    t["route"] = time.perf_counter() - t0
-    t0 = time.perf_counter()
-    counts, offsets, perm, pos = oracle.dispatch(idx, wl.E)
-    xs = oracle.gather(inp["x_e"], perm, wl.K)
-    t["dispatch"] = time.perf_counter() - t0
-    experts = [e for e in range(wl.E) if counts[e] > 0][:n_experts]
-    weights = {e: host_expert(wl, e) for e in experts}  # inputs, not timed
-    ys = np.zeros_like(xs)
-    t0 = time.perf_counter()
-    done = 0
-    for e in experts:
-        a, b = int(offsets[e]), int(offsets[e + 1])
-        ys[a:b] = oracle.expert_ffn(xs[a:b], *weights[e], wl.act, wl.beta, wl.lbeta)
-        done += b - a
-    t_ffn_sample = time.perf_counter() - t0
-    S = wl.N * wl.K
-    t["ffn"] = t_ffn_sample * S / max(done, 1)
-    t0 = time.perf_counter()
-    oracle.combine(ys, pos, w, wl.K)
-    t["combine"] = time.perf_counter() - t0
-    total = sum(t.values())
-    return {
-        "value": wl.N / total, "cores": cores, "seconds": t,
-        "sample": (f"route+dispatch+combine on all {wl.N} tokens; expert MLP on the {done} "
-                   f"rows of {len(experts)} experts, time scaled by {S}/{done} slots"),
-    }
+    n_tok = min(wl.N, ROUTE_SAMPLE_TOKENS)
+    inp = host_inputs(wl, n_tokens=n_tok)
+    sc, raw, what = _oracle_step(wl, inp, n_tok, FFN_SAMPLE_ROWS, router)
+    total = sum(sc.values())
+    return {"value": wl.N / total, "cores": cores, "seconds": sc, "sample_seconds": raw,
+            "sample": what}
 
 
-def oracle_sample_block(wl, n_experts=8, n_tokens=4, router=("sigmoid", "top2_sum")):
+def oracle_subset_single(wl, router=("sigmoid", "top2_sum")):
+    """The single-threaded CPU reference on the first SUBSET_TOKENS tokens
+    (route, sort, combine on all of them; the expert MLP on SUBSET_FFN_ROWS
+    of their rows, scaled to their slots): tokens/s of that subset, labelled
+    as such and not extrapolated to the batch."""
+    import oracle
+    from synth.workloads import host_inputs, scaled
+
+    n_tok = min(wl.N, SUBSET_TOKENS)
+    sub = scaled(wl, N=n_tok)
+    inp = host_inputs(wl, n_tokens=n_tok)
+    oracle.set_threads(1)
+    try:
+        sc, raw, what = _oracle_step(sub, inp, n_tok, SUBSET_FFN_ROWS, router)
+    finally:
+        oracle.set_threads(os.cpu_count() or 1)
+    return {"value": n_tok / sum(sc.values()), "cores": 1, "tokens": n_tok, "seconds": sc,
+            "sample": "subset: " + what}
+
+
+def cpu_baseline_obj(cb, subset=None):
+    """The line's cpu_baseline object: the all-core sample as the value, its
+    per-stage seconds, and the single-threaded subset beside it."""
+    obj = {"value": cb["value"], "unit": UNIT, "cores": cb["cores"], "kind": "oracle",
+           "sample": cb["sample"], "extrapolated": True,
+           "stage_seconds": {k: round(v, 6) for k, v in cb["seconds"].items()}}
+    if "sample_seconds" in cb:
+        obj["sample_stage_seconds"] = {k: round(v, 6) for k, v in cb["sample_seconds"].items()}
+    if subset is not None:
+        obj["single_thread_subset"] = {
+            "value": subset["value"], "unit": UNIT, "cores": 1, "tokens": subset["tokens"],
+            "stage_seconds": {k: round(v, 6) for k, v in subset["seconds"].items()},
+            "sample": subset["sample"]}
+    return obj
+
+
+def oracle_sample_block(wl, n_tokens=4, router=("sigmoid", "top2_sum")):
     """The CPU reference on a bounded sample of a whole-block step: the routed
     layer as oracle_sample; the latent projections and the norm on all
     tokens; the shared experts on `n_tokens` tokens, scaled to all."""
     import oracle
     from synth.workloads import host_block, host_inputs
 
-    r = oracle_sample(wl, n_experts, router)
+    r = oracle_sample(wl, router)
     hb = host_block(wl)
     x = host_inputs(wl)["x"]
     t = dict(r["seconds"])
@@ -640,22 +698,32 @@ def oracle_sample_block(wl, n_experts=8, n_tokens=4, router=("sigmoid", "top2_su
 
 
 def run_reference(args, rank, world):
+    """The reference arm: the CPU reference (oracle/) as it stands, timed on
+    the host cores, each step one bounded sample of the workload (the same
+    sample as the cpu_baseline leg), W untimed sample steps first.  The
+    figure is extrapolated from the sample and says so."""
     if rank != 0:
         return
     wl = workload_of(args)
+    from synth.workloads import BLOCKS
+    block = args.workload in BLOCKS
+    rt = (args.score_func, args.group_score)
+
+    def one():
+        return oracle_sample_block(wl, router=rt) if block else oracle_sample(wl, router=rt)
+
     for _ in range(args.warmup):
-        pass  # the reference has nothing to warm up; steps are timed below
+        one()
     vals = []
     t_start = time.perf_counter()
     res = None
-    from synth.workloads import BLOCKS
-    block = args.workload in BLOCKS
     for _ in range(args.steps):
-        rt = (args.score_func, args.group_score)
-        res = oracle_sample_block(wl, router=rt) if block else oracle_sample(wl, router=rt)
+        res = one()
         vals.append(res["value"])
     wall = time.perf_counter() - t_start
     v = statistics.mean(vals)
+    cb = cpu_baseline_obj(res)
+    cb["value"] = v
     line = {
         "impl": "reference", "metric": BLOCK_METRIC if block else METRIC, "value": v,
         "unit": UNIT, "n_gpus": args.gpus,
@@ -664,8 +732,8 @@ def run_reference(args, rank, world):
         "data": "synthetic", "config": {"workload": wl.name, "N": wl.N, "d_r": wl.d_r,
                                         "d_e": wl.d_e, "E": wl.E, "K": wl.K, "F": wl.F,
                                         "router": f"{args.score_func}/{args.group_score}"},
-        "cpu_baseline": {"value": v, "unit": UNIT, "cores": res["cores"], "kind": "oracle",
-                         "sample": res["sample"]},
+        "extrapolated": True,
+        "cpu_baseline": cb,
         "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
         "wall_s": wall,
     }
@@ -692,9 +760,8 @@ def main():
         wl, r = run_block(args, rank, world, local_rank)
         line = block_line(args, wl, r, world)
         if rank == 0 and world == 1 and not args.no_cpu_baseline:
-            cb = oracle_sample_block(wl, router=(args.score_func, args.group_score))
-            line["cpu_baseline"] = {"value": cb["value"], "unit": UNIT, "cores": cb["cores"],
-                                    "kind": "oracle", "sample": cb["sample"]}
+            line["cpu_baseline"] = cpu_baseline_obj(
+                oracle_sample_block(wl, router=(args.score_func, args.group_score)))
         if world > 1:
             import torch.distributed as dist
             dist.barrier()
@@ -725,16 +792,20 @@ def main():
                          "per-step events"},
         "roofline": gate_up_roofline(wl, r["touched"], r["gate_up_ms"], peaks),
         "stages_ms": r["stage_ms"],
+        "stages_pass": "a second pass of K steps with a CUDA event after every stage",
         "step_ms_min_median_max": r["step_ms"],
+        "step_ms_stat": "mean of the K per-step CUDA-event times",
+        "routing": {"touched_experts": r["touched"], "max_rows_per_expert": r["counts_max"],
+                    "top10pct_expert_share": r["top10_share"]},
         "e2e": {"value": aggregate_throughput(wl.N, world, r["e2e_ms"]), "unit": UNIT,
                 "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"]},
-        "gpu_launches": kernels_per_step(wl) * args.steps,
+        "gpu_launches": r["launches"],
         "clocks": r["clocks"],
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cb = oracle_sample(wl, router=(args.score_func, args.group_score))
-        line["cpu_baseline"] = {"value": cb["value"], "unit": UNIT, "cores": cb["cores"],
-                                "kind": "oracle", "sample": cb["sample"]}
+        line["cpu_baseline"] = cpu_baseline_obj(
+            oracle_sample(wl, router=(args.score_func, args.group_score)),
+            oracle_subset_single(wl, router=(args.score_func, args.group_score)))
     if world > 1:
         import torch.distributed as dist
         dist.barrier()

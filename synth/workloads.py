@@ -13,7 +13,9 @@ Recipe (seed 0 unless stated):
   w1   [E, F, d_e] bf16 ~ N(0, 0.02)      tensor id 4
   w3   [E, F, d_e] bf16 ~ N(0, 0.02)      tensor id 5
   w2   [E, d_e, F] bf16 ~ N(0, 0.02)      tensor id 6
-  x_e  [N, d_e]  bf16  ~ N(0, 1)          tensor id 7 (latent workload only; else x_e = x)
+  x_e  [N, d_e]  bf16  = bf16(x . P^T)    latent workload only (else x_e = x): the
+                                           down-projected x, P [d_e, d_r] fp32 ~
+                                           N(0, 1/d_r), tensor id 7, so x_e ~ N(0, 1)
 
 The whole-block workload (routed layer inside KimiSparseMoeBlock) adds:
   down_proj [d_e, d_r] bf16 ~ N(0, 0.02)          tensor id 9
@@ -121,20 +123,33 @@ def skew_bias() -> np.ndarray:
     return np.asarray(vals, dtype=np.float32)
 
 
-def host_inputs(wl: Workload, rank: int = 0) -> dict:
-    """Router-side inputs and x_e on the host (expert weights: ``host_expert``)."""
+def latent_x_e(wl: Workload, x: np.ndarray) -> np.ndarray:
+    """x_e = bf16(x . P^T) for the latent workload: the routed experts see a
+    down projection of the router's input (the workload's "down-projected
+    x"); the projection P [d_e, d_r] is synthetic, fp32 ~ N(0, 1/d_r) with
+    tensor id 7, so x_e ~ N(0, 1).  Input preparation, not the layer: the dot
+    products are taken in double, rounded to fp32 and then to bf16 (nearest
+    even).  x: bf16 bit patterns [n, d_r]; returns bf16 bit patterns."""
+    from . import bf16_bits_to_f32, host_normal_f32
+    P = host_normal_f32(wl.seed, TID_XE, (wl.d_e, wl.d_r), 1.0 / np.sqrt(wl.d_r))
+    xf = bf16_bits_to_f32(x).astype(np.float64)
+    y = (xf @ P.astype(np.float64).T).astype(np.float32)
+    return _bf16_bits_rne(y).reshape(x.shape[0], wl.d_e)
+
+
+def host_inputs(wl: Workload, rank: int = 0, n_tokens: int | None = None) -> dict:
+    """Router-side inputs and x_e on the host (expert weights: ``host_expert``).
+    n_tokens: only the first n_tokens rows of the rank's batch."""
     from . import host_normal_bf16, host_normal_f32, host_uniform_f32
-    x = host_normal_bf16(wl.seed, TID_X, (wl.N, wl.d_r), SIGMA_X, start=rank * wl.N * wl.d_r)
+    n = wl.N if n_tokens is None else min(int(n_tokens), wl.N)
+    x = host_normal_bf16(wl.seed, TID_X, (n, wl.d_r), SIGMA_X, start=rank * wl.N * wl.d_r)
     W = host_normal_f32(wl.seed, TID_W, (wl.E, wl.d_r), SIGMA_W)
     if wl.skew:
         b = skew_bias()
         assert b.shape == (wl.E,)
     else:
         b = host_uniform_f32(wl.seed, TID_BIAS, (wl.E,), BIAS_LO, BIAS_HI)
-    if wl.latent:
-        xe = host_normal_bf16(wl.seed, TID_XE, (wl.N, wl.d_e), SIGMA_X, start=rank * wl.N * wl.d_e)
-    else:
-        xe = x
+    xe = latent_x_e(wl, x) if wl.latent else x
     return {"x": x, "W": W, "bias": b, "x_e": xe}
 
 
@@ -173,8 +188,11 @@ def dev_inputs(wl: Workload, rank: int = 0, device="cuda", experts: bool = True)
         b = dev_uniform_f32(torch.empty((wl.E,), dtype=f32, device=device), wl.seed, TID_BIAS,
                             BIAS_LO, BIAS_HI)
     if wl.latent:
-        xe = dev_normal_bf16(torch.empty((wl.N, wl.d_e), dtype=bf, device=device), wl.seed,
-                             TID_XE, SIGMA_X, start=rank * wl.N * wl.d_e)
+        # the down projection is computed once on the host (from the host
+        # twin's identical x) and uploaded, so both sides see the same bits
+        from . import host_normal_bf16
+        xh = host_normal_bf16(wl.seed, TID_X, (wl.N, wl.d_r), SIGMA_X, start=rank * wl.N * wl.d_r)
+        xe = torch.from_numpy(latent_x_e(wl, xh).view(np.int16)).to(device).view(bf)
     else:
         xe = x
     out = {"x": x, "W": W, "bias": b, "x_e": xe}

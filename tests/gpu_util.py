@@ -48,3 +48,50 @@ def random_topk(N: int, K: int, E: int, rng, skew: float = 0.0) -> np.ndarray:
         return np.argsort(-keys, axis=1)[:, :K].astype(np.int32)
     keys = rng.random((N, E))
     return np.argsort(keys, axis=1)[:, :K].astype(np.int32)
+
+
+def oracle_layer_tokens(wl, xe_rows: np.ndarray, idx: np.ndarray, w: np.ndarray,
+                        workers: int | None = None) -> np.ndarray:
+    """The reference layer output of a few tokens: out[i] = combine over k of
+    expert_ffn(idx[i, k]) on xe_rows[i], weighted by w[i, k] -- the per-token
+    loop of moe_infer.  Tokens are grouped by expert so that each expert's
+    weights are drawn once; experts run in a thread pool (the reference's C
+    calls release the GIL), each call single-threaded.  Bit-identical to the
+    same loop run serially: every row's arithmetic is independent."""
+    import os
+    from concurrent.futures import ThreadPoolExecutor
+
+    import oracle
+    from synth.workloads import host_expert
+
+    n, K = idx.shape
+    by_e: dict[int, list[tuple[int, int]]] = {}
+    for i in range(n):
+        for k in range(K):
+            by_e.setdefault(int(idx[i, k]), []).append((i, k))
+    ys = np.zeros((n, K, xe_rows.shape[1]), np.uint16)
+
+    def run(e):
+        oracle.set_threads(1)  # this thread's OpenMP team (the generator's too)
+        slots = by_e[e]
+        w1, w3, w2 = host_expert(wl, e)
+        rows = np.ascontiguousarray(xe_rows[[i for i, _ in slots]])
+        y = oracle.expert_ffn(rows, w1, w3, w2, wl.act, wl.beta, wl.lbeta)
+        for (i, k), r in zip(slots, y):
+            ys[i, k] = r
+
+    with ThreadPoolExecutor(max_workers=workers or os.cpu_count() or 1) as ex:
+        list(ex.map(run, sorted(by_e)))
+    out = np.zeros((n, xe_rows.shape[1]), np.uint16)
+    for i in range(n):
+        out[i] = oracle.combine(ys[i], np.arange(K, dtype=np.int32),
+                                np.ascontiguousarray(w[i:i + 1]), K)[0]
+    return out
+
+
+def ulp_stats(got_bits: np.ndarray, ref_bits: np.ndarray) -> dict:
+    """Fraction of outputs within 0, 1 and 2 bf16 ulp of the reference, and the
+    largest distance."""
+    u = ulp_diff(got_bits, ref_bits)
+    return {"n": int(u.size), "eq": float((u == 0).mean()), "le1": float((u <= 1).mean()),
+            "le2": float((u <= 2).mean()), "max": int(u.max()) if u.size else 0}

@@ -17,8 +17,8 @@ import pytest
 import oracle
 import synth
 from synth.workloads import WORKLOADS, host_inputs, host_expert, scaled
-from tests.gpu_util import (MARGIN, REL_L2_OUT, W_REL, dev_bf16, host_bf16, random_topk, rel_l2,
-                            ulp_diff)
+from tests.gpu_util import (MARGIN, REL_L2_OUT, W_REL, dev_bf16, host_bf16, oracle_layer_tokens,
+                            random_topk, rel_l2, ulp_diff, ulp_stats)
 
 pytestmark = pytest.mark.gpu
 
@@ -269,9 +269,8 @@ def _expert_case(moe, wl, counts, sample_experts, rows_per_expert=48, seed=5):
         y_r = oracle.expert_ffn(xs_rows, w1, w3, w2, wl.act, wl.beta, wl.lbeta)
         y_g = host_bf16(y_d[torch.from_numpy(rows).cuda()])
         err = rel_l2(y_g, y_r)
-        u = ulp_diff(y_g, y_r)
-        print(f"expert {e}: rows {len(rows)}/{n} rel_l2 {err:.2e} max_ulp {u.max()} "
-              f"frac>1ulp {(u > 1).mean():.2e}")
+        print(f"expert {wl.name} {e}: rows {len(rows)}/{n} rel_l2 {err:.2e} "
+              f"ulp {ulp_stats(y_g, y_r)}")
         assert err <= REL_L2_OUT
         worst = max(worst, err)
     return worst
@@ -320,11 +319,14 @@ def _forward(moe, wl, dev):
 
 @pytest.mark.parametrize("name", ALL)
 def test_forward_end_to_end(moe, name):
+    """The whole layer against the reference's per-token loop (the reference's
+    own routing), on every token of the small batches and on 128 sampled
+    tokens (first, last and 126 random) of the larger ones."""
     wl = WORKLOADS[name]
     dev = synth.workloads.dev_inputs(wl)
     out_g, idx_g, w_g = _forward(moe, wl, dev)
     inp = host_inputs(wl)
-    n_tok = wl.N if wl.N <= 64 else 12
+    n_tok = wl.N if wl.N <= 128 else 128
     toks = np.arange(wl.N) if n_tok == wl.N else np.unique(
         np.concatenate([[0, wl.N - 1], np.random.default_rng(7).choice(wl.N, n_tok - 2, False)]))
     x = np.ascontiguousarray(inp["x"][toks])
@@ -333,20 +335,10 @@ def test_forward_end_to_end(moe, name):
                                       wl.route_scale, wl.norm)
     _check_routing(idx_g[toks], w_g[toks], idx_r, w_r, margin)
     keep = margin > MARGIN
-    cache = {}
-    out_r = np.zeros((len(toks), wl.d_e), np.uint16)
-    for i in range(len(toks)):
-        ys = []
-        for k in range(wl.K):
-            e = int(idx_r[i, k])
-            if e not in cache:
-                cache[e] = host_expert(wl, e)
-            w1, w3, w2 = cache[e]
-            ys.append(oracle.expert_ffn(xe[i:i + 1], w1, w3, w2, wl.act, wl.beta, wl.lbeta)[0])
-        out_r[i] = oracle.combine(np.stack(ys), np.arange(wl.K, dtype=np.int32),
-                                  np.ascontiguousarray(w_r[i:i + 1]), wl.K)[0]
+    out_r = oracle_layer_tokens(wl, xe, idx_r, w_r)
     err = rel_l2(out_g[toks][keep], out_r[keep])
-    print(f"{name}: {keep.sum()}/{len(toks)} tokens, rel_l2 {err:.2e}")
+    st = ulp_stats(out_g[toks][keep], out_r[keep])
+    print(f"forward {name}: {keep.sum()}/{len(toks)} tokens, rel_l2 {err:.2e}, ulp {st}")
     assert err <= REL_L2_OUT
 
 

@@ -79,3 +79,28 @@ def test_device_twin_bit_identical():
         du = synth.dev_uniform_f32(torch.empty(n, dtype=torch.float32, device="cuda"), 7, 3,
                                    -0.01, 0.01, start=start)
         assert np.array_equal(du.cpu().numpy().view(np.uint32), hu.view(np.uint32))
+
+
+def test_latent_x_e_is_the_down_projection_of_x():
+    """The latent workload's x_e is bf16(x . P^T) with P [d_e, d_r] drawn with
+    tensor id 7 and sigma 1/sqrt(d_r): entries checked against the exact
+    rational dot product (rounded to fp32, then to bf16), and the whole
+    tensor is about N(0, 1)."""
+    from fractions import Fraction
+    wl = WORKLOADS["k3_latent_decode"]
+    inp = host_inputs(wl)
+    x, xe = inp["x"], inp["x_e"]
+    assert xe.shape == (wl.N, wl.d_e) and xe.dtype == np.uint16
+    P = synth.host_normal_f32(wl.seed, synth.TID_XE, (wl.d_e, wl.d_r), 1.0 / np.sqrt(wl.d_r))
+    xf = synth.bf16_bits_to_f32(x)
+    for t, j in [(0, 0), (3, 17), (63, 2047), (40, 1000)]:
+        exact = sum(Fraction(float(a)) * Fraction(float(b)) for a, b in zip(xf[t], P[j]))
+        f32 = np.float32(float(exact))
+        want = int(np.asarray([f32]).view(np.uint32)[0])
+        want = (want + 0x7FFF + ((want >> 16) & 1)) >> 16
+        assert int(xe[t, j]) == want, (t, j)
+    v = synth.bf16_bits_to_f32(xe).astype(np.float64)
+    assert abs(v.mean()) < 0.02 and abs(v.std() - 1.0) < 0.03
+    # the first rows alone are the first rows of the whole batch
+    part = host_inputs(wl, n_tokens=5)
+    assert np.array_equal(part["x_e"], xe[:5]) and np.array_equal(part["x"], x[:5])
