@@ -232,9 +232,25 @@ MOE_API size_t moe_combine_workspace_size(void);
 /* Unpermute and combine:
  *   out[t, :] = bf16( sum_{k=0..K-1} fp32(y[pos[t*K+k], :]) * topk_w[t, k] )
  * with every product rounded to fp32 and the sum taken in k order in fp32.
- * y: [S, d_e] bf16; pos: [S] int32; topk_w: [N, K] fp32; out: [N, d_e] bf16. */
+ * y: [S, d_e] bf16; pos: [S] int32; topk_w: [N, K] fp32; out: [N, d_e] bf16.
+ * pos == NULL: y is already in slot order (the page's new_x, as
+ * moe_expert_ffn_to_slots writes it), so row t*K+k is read for slot (t, k). */
 MOE_API int moe_combine(const moe_bf16* y, const int32_t* pos, const float* topk_w, int64_t N,
                         int K, int d_e, moe_bf16* out, void* ws, size_t ws_bytes, void* stream);
+
+/* moe_expert_ffn with the scatter inside the w2 kernel ("Kimi K3 · Add shared
+ * output", moe-forward excerpt: new_x[idxs] = outs): the output row of sorted
+ * row j is stored at row perm[j] of y_slots, so y_slots is the MLP output in
+ * slot order (token t's K rows are rows t*K .. t*K+K-1) and moe_combine reads
+ * it with pos == NULL.  perm: [S] int32 as moe_dispatch writes it (a
+ * permutation of 0 .. S-1; an entry outside it is recorded as
+ * MOE_ERR_DEVICE_BOUNDS and its row is not stored).  y_slots: [S, d_e] bf16.
+ * Arithmetic, arguments and workspace otherwise as moe_expert_ffn. */
+MOE_API int moe_expert_ffn_to_slots(const moe_bf16* xs, const int32_t* offsets,
+                                    const int32_t* perm, int E, int64_t S, int d_e, int F,
+                                    const moe_bf16* w1, const moe_bf16* w3, const moe_bf16* w2,
+                                    const moe_act_cfg* act, moe_bf16* y_slots, void* ws,
+                                    size_t ws_bytes, void* stream);
 
 /* moe_expert_ffn with the gather inside the w1/w3 kernel: row j of segment
  * e is x_e[perm[j] / K] (perm and offsets as moe_dispatch writes them), read
@@ -458,6 +474,21 @@ MOE_API const char* moe_strerror(int code);
  * the number of libmoe kernels that region enqueued.  Not part of the pages'
  * method: bookkeeping for measurement. */
 MOE_API uint64_t moe_launch_count(void);
+
+/* Diagnostics hook for the kernels' bounded waits (not part of the pages'
+ * method).  Every mbarrier wait in the tensor-core kernels gives up after a
+ * time limit, records MOE_ERR_DEVICE_TIMEOUT in the status word and stops the
+ * kernel cleanly (its other roles stop, its tensor memory is freed), so a
+ * broken protocol cannot hang the GPU.  With on != 0 the grouped expert GEMM
+ * kernels launched afterwards (moe_expert_ffn, moe_forward and every entry
+ * point built on them) make that path run: before issuing any copy, each
+ * CTA's producer waits on a barrier that nothing arrives on, with a 1 ms
+ * limit; the wait runs out, the call's status word reads
+ * MOE_ERR_DEVICE_TIMEOUT and its outputs are left unwritten.  on = 0 (the
+ * default) restores normal operation; the CUDA context stays usable.
+ * Process-wide and read at launch: not for use while other threads launch
+ * libmoe kernels.  Returns the previous setting. */
+MOE_API int moe_set_wait_probe(int on);
 
 #ifdef __cplusplus
 }

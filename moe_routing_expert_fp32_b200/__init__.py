@@ -150,7 +150,8 @@ EXPORTS = ("moe_route_workspace_size", "moe_route", "moe_route_from_logits",
            "moe_linear_workspace_size", "moe_linear", "moe_rms_norm", "moe_block_workspace_size",
            "moe_block_forward", "moe_shared_experts_workspace_size", "moe_shared_experts",
            "moe_ep_expert_ffn_workspace_size", "moe_ep_expert_ffn", "moe_expert_ffn_gathered",
-           "moe_ep_dispatch_rows", "moe_ep_combine_rows", "moe_launch_count")
+           "moe_ep_dispatch_rows", "moe_ep_combine_rows", "moe_launch_count",
+           "moe_set_wait_probe", "moe_expert_ffn_to_slots")
 
 
 def lib() -> ctypes.CDLL:
@@ -199,6 +200,9 @@ def lib() -> ctypes.CDLL:
         "moe_ep_dispatch_rows": ([vp, i64, i32, i32, vp, vp, i32, pr, vp, sz, vp], i32),
         "moe_ep_combine_rows": ([pr, vp, vp, i32, vp, i64, i32, i32, vp, vp, sz, vp], i32),
         "moe_launch_count": ([], ctypes.c_uint64),
+        "moe_set_wait_probe": ([i32], i32),
+        "moe_expert_ffn_to_slots": ([vp, vp, vp, i32, i64, i32, i32, vp, vp, vp, ac, vp, vp, sz,
+                                     vp], i32),
     }
     for name, (args, res) in sig.items():
         fn = getattr(L, name)
@@ -211,6 +215,12 @@ def lib() -> ctypes.CDLL:
 def launch_count() -> int:
     """Kernels libmoe has launched in this process so far (moe_launch_count)."""
     return int(lib().moe_launch_count())
+
+
+def set_wait_probe(on: bool) -> bool:
+    """Diagnostics: make the grouped expert GEMM's bounded wait run out (see
+    moe_set_wait_probe in include/moe.h).  Returns the previous setting."""
+    return bool(lib().moe_set_wait_probe(1 if on else 0))
 
 
 # ----------------------------------------------------------------- helpers
@@ -375,12 +385,37 @@ def expert_ffn(xs, offsets, w1, w3, w2, act: ActConfig, ws=None, y=None):
     return y
 
 
+def expert_ffn_to_slots(xs, offsets, perm, w1, w3, w2, act: ActConfig, ws=None, y=None):
+    """moe_expert_ffn writing output row j to row perm[j] (slot order)."""
+    torch = _torch()
+    S, d_e = xs.shape
+    E, F, _ = w1.shape
+    _need(xs, torch.bfloat16, name="xs")
+    _need(offsets, torch.int32, (E + 1,), "offsets")
+    _need(perm, torch.int32, (S,), "perm")
+    _need(w1, torch.bfloat16, (E, F, d_e), "w1")
+    _need(w3, torch.bfloat16, (E, F, d_e), "w3")
+    _need(w2, torch.bfloat16, (E, d_e, F), "w2")
+    dev = xs.device
+    need = lib().moe_expert_ffn_workspace_size(S, d_e, E, F)
+    ws = workspace(need, dev) if ws is None else ws
+    y = torch.empty((S, d_e), dtype=torch.bfloat16, device=dev) if y is None else y
+    a = act._c()
+    _check("moe_expert_ffn_to_slots",
+           lib().moe_expert_ffn_to_slots(_ptr(xs), _ptr(offsets), _ptr(perm), E, S, d_e, F,
+                                         _ptr(w1), _ptr(w3), _ptr(w2), ctypes.byref(a), _ptr(y),
+                                         _ptr(ws), ws.numel(), _stream()))
+    return y
+
+
 def combine(y, pos, topk_w, ws=None):
+    """pos None: y is in slot order (moe_expert_ffn_to_slots)."""
     torch = _torch()
     N, K = topk_w.shape
     d_e = y.shape[1]
     _need(y, torch.bfloat16, (N * K, d_e), "y")
-    _need(pos, torch.int32, (N * K,), "pos")
+    if pos is not None:
+        _need(pos, torch.int32, (N * K,), "pos")
     _need(topk_w, torch.float32, name="topk_w")
     ws = workspace(256, y.device) if ws is None else ws
     out = torch.empty((N, d_e), dtype=torch.bfloat16, device=y.device)

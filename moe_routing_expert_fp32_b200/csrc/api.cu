@@ -3,6 +3,8 @@
 // kernels of router.cu, dispatch.cu, expert_gemm.cu and combine.cu.
 #include <math.h>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include <atomic>
 #include <mutex>
 
@@ -45,6 +47,16 @@ using namespace moe;
 namespace {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// An NVTX range around the host-side enqueue of one stage ("moe.route",
+// "moe.dispatch", ...): a profiler that records NVTX (Nsight Systems) shows
+// each stage's kernels under its name; without one the calls cost nothing.
+struct Range {
+  explicit Range(const char* name) { nvtxRangePushA(name); }
+  ~Range() { nvtxRangePop(); }
+  Range(const Range&) = delete;
+  Range& operator=(const Range&) = delete;
+};
 
 int check_device() {
   const DevInfo* d = dev_info();
@@ -95,8 +107,14 @@ int route_impl(const __nv_bfloat16* x, int64_t N, int d_r, const float* W, const
                const moe_route_cfg& cfg, int32_t* idx, float* w, uint8_t* scratch,
                DeviceStatus* st, cudaStream_t s) {
   const int E = cfg.num_experts;
-  if (launch_gate(x, N, d_r, W, E, scratch, st, s) != cudaSuccess) return MOE_ERR_CUDA;
-  if (launch_select(route_logits_of(scratch), N, bias, cfg, idx, w, st, s) != cudaSuccess)
+  // split-K partials of the gate GEMM (decode batches) are summed by the
+  // selection kernel itself, so no reduce kernel runs between them
+  int splits = 1;
+  const double* part = route_fused_partials(scratch, N, E, d_r, &splits);
+  if (launch_gate(x, N, d_r, W, E, scratch, st, s, part == nullptr) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  if (launch_select(route_logits_of(scratch), N, bias, cfg, idx, w, st, s, part, splits) !=
+      cudaSuccess)
     return MOE_ERR_CUDA;
   return MOE_OK;
 }
@@ -274,6 +292,32 @@ int moe_expert_ffn(const moe_bf16* xs, const int32_t* offsets, int E, int64_t S,
                         nullptr);
 }
 
+// The expert MLP writing each output row to its slot (the scatter inside the
+// w2 kernel's epilogue): y_slots[perm[j]] = the MLP of sorted row j.
+int moe_expert_ffn_to_slots(const moe_bf16* xs, const int32_t* offsets, const int32_t* perm,
+                            int E, int64_t S, int d_e, int F, const moe_bf16* w1,
+                            const moe_bf16* w3, const moe_bf16* w2, const moe_act_cfg* act,
+                            moe_bf16* y_slots, void* ws, size_t ws_bytes, void* stream) {
+  int rc = check_expert_shape(S, d_e, E, F);
+  if (rc) return rc;
+  if ((rc = check_act(act))) return rc;
+  if (!offsets || !w1 || !w3 || !w2) return MOE_ERR_INVALID_ARG;
+  if (S > 0 && (!xs || !perm || !y_slots)) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(w1) || !aligned16(w3) || !aligned16(w2)) return MOE_ERR_ALIGNMENT;
+  if (S > 0 && (!aligned16(xs) || !aligned16(y_slots))) return MOE_ERR_ALIGNMENT;
+  if ((rc = check_ws(ws, ws_bytes, moe_expert_ffn_workspace_size(S, d_e, E, F)))) return rc;
+  if ((rc = check_device())) return rc;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if ((rc = reset_status(ws, s))) return rc;
+  if (S == 0) return MOE_OK;
+  return expert_ffn_run(reinterpret_cast<const __nv_bfloat16*>(xs), offsets, E, S, d_e, F,
+                        reinterpret_cast<const __nv_bfloat16*>(w1),
+                        reinterpret_cast<const __nv_bfloat16*>(w3),
+                        reinterpret_cast<const __nv_bfloat16*>(w2), *act,
+                        reinterpret_cast<__nv_bfloat16*>(y_slots), body_of(ws), status_of(ws), s,
+                        nullptr, nullptr, nullptr, 0, perm);
+}
+
 // The expert MLP reading its token rows straight from x_e through perm (the
 // gather inside the w1/w3 kernel): no S x d_e copy of the tokens.
 int moe_expert_ffn_gathered(const moe_bf16* x_e, int64_t N, int K, const int32_t* perm,
@@ -352,7 +396,8 @@ int moe_combine(const moe_bf16* y, const int32_t* pos, const float* topk_w, int6
   if (N < 0 || K < 1 || d_e <= 0) return MOE_ERR_INVALID_ARG;
   if (K > 16) return MOE_ERR_UNSUPPORTED;
   if (d_e % 8 != 0) return MOE_ERR_UNSUPPORTED;
-  if (N > 0 && (!y || !pos || !topk_w || !out)) return MOE_ERR_INVALID_ARG;
+  // pos == NULL: y is in slot order (moe_expert_ffn_to_slots)
+  if (N > 0 && (!y || !topk_w || !out)) return MOE_ERR_INVALID_ARG;
   if (N > 0 && (!aligned16(y) || !aligned16(out))) return MOE_ERR_ALIGNMENT;
   int rc;
   if ((rc = check_ws(ws, ws_bytes, kStatusBytes))) return rc;
@@ -444,6 +489,10 @@ int moe_ep_combine_rows(const moe_peer_rows* peers, const int32_t* pos, const in
 
 // ------------------------------------------------------------ whole layer
 namespace {
+// Whether moe_forward scatters y into slot order in the w2 epilogue (and
+// combines contiguous rows) or keeps y sorted (and combines through pos).
+constexpr bool kForwardSlotOrder = false;
+
 struct ForwardLayout {
   size_t stage;                    // shared scratch of the stages
   size_t idx, w, counts, offsets, perm, pos, xs, y, total;
@@ -520,25 +569,42 @@ int moe_forward(const moe_bf16* x_r, const moe_bf16* x_e, int64_t N, int d_r, in
   auto rec = [&](void* ev) {
     return ev ? cudaEventRecord(static_cast<cudaEvent_t>(ev), s) == cudaSuccess : true;
   };
-  if ((rc = route_impl(reinterpret_cast<const __nv_bfloat16*>(x_r), N, d_r, W, bias, *cfg, idx, w,
-                       stage, st, s)))
-    return rc;
+  const Range layer("moe.forward");
+  {
+    const Range r("moe.route");
+    if ((rc = route_impl(reinterpret_cast<const __nv_bfloat16*>(x_r), N, d_r, W, bias, *cfg, idx,
+                         w, stage, st, s)))
+      return rc;
+  }
   if (events && !rec(events->after_route)) return MOE_ERR_CUDA;
-  if (launch_dispatch(idx, N, K, E, reinterpret_cast<const __nv_bfloat16*>(x_e), d_e, counts,
-                      offsets, perm, pos, xs, reinterpret_cast<int32_t*>(stage), st,
-                      s) != cudaSuccess)
-    return MOE_ERR_CUDA;
+  {
+    const Range r("moe.dispatch");
+    if (launch_dispatch(idx, N, K, E, reinterpret_cast<const __nv_bfloat16*>(x_e), d_e, counts,
+                        offsets, perm, pos, xs, reinterpret_cast<int32_t*>(stage), st,
+                        s) != cudaSuccess)
+      return MOE_ERR_CUDA;
+  }
   if (events && !rec(events->after_dispatch)) return MOE_ERR_CUDA;
-  if ((rc = expert_ffn_run(xs, offsets, E, N * K, d_e, F,
-                           reinterpret_cast<const __nv_bfloat16*>(w1),
-                           reinterpret_cast<const __nv_bfloat16*>(w3),
-                           reinterpret_cast<const __nv_bfloat16*>(w2), *act, y, stage, st, s,
-                           events ? static_cast<cudaEvent_t>(events->after_gate_up) : nullptr)))
-    return rc;
+  // with kForwardSlotOrder the w2 epilogue writes y in slot order (row
+  // perm[j] for sorted row j) and the combine reads each token's K rows
+  // contiguously; otherwise y stays sorted and the combine reads it via pos
+  {
+    const Range r("moe.expert_ffn");
+    if ((rc = expert_ffn_run(xs, offsets, E, N * K, d_e, F,
+                             reinterpret_cast<const __nv_bfloat16*>(w1),
+                             reinterpret_cast<const __nv_bfloat16*>(w3),
+                             reinterpret_cast<const __nv_bfloat16*>(w2), *act, y, stage, st, s,
+                             events ? static_cast<cudaEvent_t>(events->after_gate_up) : nullptr,
+                             nullptr, nullptr, 0, kForwardSlotOrder ? perm : nullptr)))
+      return rc;
+  }
   if (events && !rec(events->after_down)) return MOE_ERR_CUDA;
-  if (launch_combine(y, pos, w, N, K, d_e, N * K, reinterpret_cast<__nv_bfloat16*>(out), st, s) !=
-      cudaSuccess)
-    return MOE_ERR_CUDA;
+  {
+    const Range r("moe.combine");
+    if (launch_combine(y, kForwardSlotOrder ? nullptr : pos, w, N, K, d_e, N * K,
+                       reinterpret_cast<__nv_bfloat16*>(out), st, s) != cudaSuccess)
+      return MOE_ERR_CUDA;
+  }
   if (events && !rec(events->after_combine)) return MOE_ERR_CUDA;
   return MOE_OK;
 }
@@ -740,10 +806,15 @@ int moe_block_forward(const moe_bf16* x, int64_t N, const moe_block_dims* dims,
   __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(out);
   float* part = L.part_bytes ? reinterpret_cast<float*>(base + L.part) : nullptr;
 
+  const Range block("moe.block_forward");
   if (launch_dense_tiles(N, tiles, s) != cudaSuccess) return MOE_ERR_CUDA;
   // gate on the full-width input
-  if ((rc = route_impl(xr, N, d_r, wt->gate_weight, wt->gate_bias, *cfg, idx, w, stage, st, s)))
-    return rc;
+  {
+    const Range r("moe.route");
+    if ((rc = route_impl(xr, N, d_r, wt->gate_weight, wt->gate_bias, *cfg, idx, w, stage, st,
+                         s)))
+      return rc;
+  }
   // shared experts on the full-width input (their output is the residual of
   // the last step)
   if (shared && (rc = shared_ffn_run(xr, N, d_r, dims->F_shared, cbf(wt->shared_w1),

@@ -2,9 +2,12 @@
 //
 // Follows "Kimi K3 · Add shared output", moe-forward excerpt (moe_infer):
 // new_x[idxs] = outs, then new_x.view(N, K, d).type(fp32).mul_(w).sum(dim=1)
-// .type(bf16).  The scatter into new_x is not materialised: token t reads its
-// K rows straight from y through pos[t*K + k].  Products are rounded to fp32
-// (__fmul_rn) and summed in k order (__fadd_rn), then rounded once to bf16.
+// .type(bf16).  Token t's K rows come either straight from the sorted y
+// through pos[t*K + k] (the scatter into new_x is not materialised), or, when
+// the expert MLP's last GEMM has already written y in slot order (new_x
+// itself), from rows t*K .. t*K+K-1 (pos == nullptr).  Products are rounded
+// to fp32 (__fmul_rn) and summed in k order (__fadd_rn), then rounded once to
+// bf16.
 #include "moe_internal.cuh"
 
 namespace moe {
@@ -35,7 +38,7 @@ __global__ void __launch_bounds__(32 * kWarps) k_combine(const __nv_bfloat16* __
     int my_p = -1;
     float my_w = 0.f;
     if (lane < K) {
-      my_p = pos[t * K + lane];
+      my_p = pos ? pos[t * K + lane] : (int)(t * K + lane);
       my_w = w[t * K + lane];
       if (my_p < 0 || my_p >= S) {
         record_error(st, MOE_ERR_DEVICE_BOUNDS, 40);
@@ -172,7 +175,7 @@ __global__ void __launch_bounds__(32 * kWarps) k_combine_rms_norm(
     int my_p = -1;
     float my_w = 0.f;
     if (lane < K) {
-      my_p = pos[t * K + lane];
+      my_p = pos ? pos[t * K + lane] : (int)(t * K + lane);
       my_w = w[t * K + lane];
       if (my_p < 0 || my_p >= S) {
         record_error(st, MOE_ERR_DEVICE_BOUNDS, 41);

@@ -47,7 +47,10 @@
 #include <cuda.h>
 #include <math.h>
 
+#include <atomic>
+
 #include "moe_internal.cuh"
+#include "sm100.cuh"
 
 namespace moe {
 namespace {
@@ -60,7 +63,6 @@ constexpr int kBoxRows = 16;   // token rows per small TMA box
 constexpr int kBigBoxRows = 64;  // token rows per large TMA box (prefill variant)
 constexpr int kGateUpRows = 64;  // d_ff rows per gate_up unit (w1 + w3 = 128 A rows)
 constexpr int kXchgBytes = 8192;  // gate_up epilogue exchange: 2 pairs x 2 bufs x 2 x 32x8 fp32
-constexpr uint64_t kTimeoutNs = 2000000000ull;
 
 enum Mode { kGateUp = 0, kDown = 1 };
 
@@ -83,80 +85,21 @@ struct Cfg {
 };
 
 // ------------------------------------------------------------ PTX wrappers
-__device__ __forceinline__ uint32_t smem_u32(const void* p) {
-  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-__device__ __forceinline__ uint64_t gtimer() {
-  uint64_t t;
-  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-  return t;
-}
-__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
-}
-__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
-               "r"(bytes)
-               : "memory");
-}
-__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
-}
-__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-// Waits for the phase of parity `parity` to complete; false if it did not
-// within kTimeoutNs or another role gave up first.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
-                                          volatile int* abort_flag) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = gtimer();
-  for (uint32_t i = 1;; ++i) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((i & 63) == 0) {
-      if (*abort_flag) return false;
-      if (gtimer() - t0 > kTimeoutNs) return false;
-    }
-  }
-}
-__device__ __forceinline__ void tma_load_2d(const CUtensorMap* map, uint64_t* bar, void* dst,
-                                            int c0, int c1) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1)
-      : "memory");
-}
-__device__ __forceinline__ void tma_load_3d(const CUtensorMap* map, uint64_t* bar, void* dst,
-                                            int c0, int c1, int c2) {
-  asm volatile(
-      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(smem_u32(dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2)
-      : "memory");
-}
-__device__ __forceinline__ uint64_t l2_evict_first_policy() {
-  uint64_t p;
-  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
-  return p;
-}
-__device__ __forceinline__ void tma_load_3d_hint(const CUtensorMap* map, uint64_t* bar, void* dst,
-                                                 int c0, int c1, int c2, uint64_t policy) {
-  asm volatile(
-      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
-      " [%0], [%1, {%3, %4, %5}], [%2], %6;" ::"r"(smem_u32(dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2),
-      "l"(policy)
-      : "memory");
-}
+// (the shared ones are in sm100.cuh)
+using sm100::gtimer;
+using sm100::l2_evict_first_policy;
+using sm100::mbar_arrive;
+using sm100::mbar_arrive_expect_tx;
+using sm100::mbar_init;
+using sm100::mbar_try_wait;
+using sm100::mbar_wait;
+using sm100::smem_u32;
+using sm100::tc_fence_after;
+using sm100::tc_fence_before;
+using sm100::tma_load_2d;
+using sm100::tma_load_3d;
+using sm100::tma_load_3d_hint;
+using sm100::umma_commit;
 
 // Four rows r0..r3 (any order, any rows) of a 2-D map whose box is 64 columns
 // x 1 row, written to dst as consecutive 128-byte rows with the map's swizzle.
@@ -172,19 +115,9 @@ __device__ __forceinline__ void tma_gather4(const CUtensorMap* map, uint64_t* ba
 
 // Programmatic dependent launch: the dependent kernel waits here until the
 // preceding kernel's memory is visible; a primary lets dependents launch.
-__device__ __forceinline__ void grid_dep_wait() {
-  asm volatile("griddepcontrol.wait;" ::: "memory");
-}
-__device__ __forceinline__ void grid_dep_launch() {
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-}
+__device__ __forceinline__ void grid_dep_wait() { pdl_wait(); }
+__device__ __forceinline__ void grid_dep_launch() { pdl_trigger(); }
 
-__device__ __forceinline__ void tc_fence_before() {
-  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-}
-__device__ __forceinline__ void tc_fence_after() {
-  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-}
 __device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
                                           uint32_t idesc, uint32_t accumulate) {
   asm volatile(
@@ -193,24 +126,10 @@ __device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t a_desc, uint
       "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
       "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate));
 }
-__device__ __forceinline__ void umma_commit(uint64_t* bar) {
-  asm volatile(
-      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-          smem_u32(bar))
-      : "memory");
-}
 // 32 lanes x 16 consecutive fp32 columns; waits for the load before returning.
 __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float* v) {
   uint32_t r[16];
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
-      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];\n\t"
-      "tcgen05.wait::ld.sync.aligned;"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
-        "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
-      : "r"(taddr)
-      : "memory");
+  sm100::tmem_ld16(taddr, r);
 #pragma unroll
   for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
 }
@@ -218,18 +137,27 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float* v) {
 // Shared-memory matrix descriptor: K-major operand, 128-byte swizzle, rows of
 // 128 bytes, 8-row groups 1024 bytes apart (tile base 1024-byte aligned).
 __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
-  uint64_t d = 0;
-  d |= (uint64_t)((saddr & 0x3FFFFu) >> 4);  // start address
-  d |= (uint64_t)1 << 16;                     // leading byte offset (unused here)
-  d |= (uint64_t)(1024 >> 4) << 32;           // stride byte offset
-  d |= (uint64_t)1 << 46;                     // descriptor version
-  d |= (uint64_t)2 << 61;                     // 128-byte swizzle
-  return d;
+  return sm100::smem_desc(saddr, 1024, 2);
 }
 // Instruction descriptor: bf16 x bf16 -> fp32, both K-major, M = 128.
 __device__ __forceinline__ uint32_t idesc_bf16(int n) {
   return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) |
          ((uint32_t)(BM >> 4) << 24);
+}
+
+// Diagnostics hook (moe_set_wait_probe): with `probe` set, the producer first
+// waits on a barrier that nothing arrives on, with a 1 ms limit, before it
+// issues any copy; the wait runs out and the kernel takes its abort path (the
+// error recorded, the other roles stopped, TMEM freed).  Returns true when the
+// kernel must stop.
+constexpr uint64_t kProbeLimitNs = 1000000ull;
+__device__ __forceinline__ bool probe_abort(int probe, uint64_t* never, volatile int* abort_flag,
+                                            DeviceStatus* st, int detail) {
+  if (!probe) return false;
+  if (mbar_wait(never, 0, abort_flag, kProbeLimitNs)) return false;  // nothing arrives on it
+  record_error(st, MOE_ERR_DEVICE_TIMEOUT, detail);
+  *abort_flag = 1;
+  return true;
 }
 
 __device__ __forceinline__ float bf16r(float x) {
@@ -275,7 +203,10 @@ __device__ __forceinline__ float situ_mul(float g, float u, float beta, float lb
 // group is transposed by shuffles so that lane i holds tokens 2i and 2i+1 of
 // the group's 8 features.  Every lane of the warp must call it.
 __device__ __forceinline__ void store_down_t8(const float* v, __nv_bfloat16* out, int64_t tok0,
-                                              int ntok, int M_rows, int m8, bool live, int lane) {
+                                              int ntok, int M_rows, int m8, bool live, int lane,
+                                              const int32_t* rowmap = nullptr,
+                                              int64_t map_rows = 0,
+                                              DeviceStatus* st = nullptr) {
   uint32_t a[8];
 #pragma unroll
   for (int t = 0; t < 8; ++t) {
@@ -303,8 +234,21 @@ __device__ __forceinline__ void store_down_t8(const float* v, __nv_bfloat16* out
   lo.z = __byte_perm(a[4], a[5], 0x5410); hi.z = __byte_perm(a[4], a[5], 0x7632);
   lo.w = __byte_perm(a[6], a[7], 0x5410); hi.w = __byte_perm(a[6], a[7], 0x7632);
   if (live) {
-    if (2 * i < ntok) *reinterpret_cast<uint4*>(out + (tok0 + 2 * i) * M_rows + m8) = lo;
-    if (2 * i + 1 < ntok) *reinterpret_cast<uint4*>(out + (tok0 + 2 * i + 1) * M_rows + m8) = hi;
+    // row r of the token tile goes to output row r, or to rowmap[r] (the
+    // slot-order scatter: sorted row j is written where slot perm[j] lives)
+    int64_t r0 = tok0 + 2 * i, r1 = r0 + 1;
+    if (rowmap) {
+      r0 = 2 * i < ntok ? rowmap[r0] : -1;
+      r1 = 2 * i + 1 < ntok ? rowmap[r1] : -1;
+      if ((2 * i < ntok && (r0 < 0 || r0 >= map_rows)) ||
+          (2 * i + 1 < ntok && (r1 < 0 || r1 >= map_rows))) {
+        record_error(st, MOE_ERR_DEVICE_BOUNDS, 140);
+        if (r0 >= map_rows) r0 = -1;
+        if (r1 >= map_rows) r1 = -1;
+      }
+    }
+    if (2 * i < ntok && r0 >= 0) *reinterpret_cast<uint4*>(out + r0 * M_rows + m8) = lo;
+    if (2 * i + 1 < ntok && r1 >= 0) *reinterpret_cast<uint4*>(out + r1 * M_rows + m8) = hi;
   }
 }
 
@@ -376,7 +320,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                   __nv_bfloat16* __restrict__ out, const __nv_bfloat16* __restrict__ res,
                   int act_kind, float beta, float lbeta, DeviceStatus* st, int pdl,
                   const int32_t* __restrict__ gperm, int gk, int gn, int ksplit,
-                  float* __restrict__ part, int emod) {
+                  float* __restrict__ part, int emod, int probe,
+                  const int32_t* __restrict__ yrow) {
   using C = Cfg<NTMAX, STAGES, UM, KSUB>;
   constexpr int KS = BK * KSUB;  // K columns per stage
   constexpr bool kDecode = NTMAX <= 32;
@@ -387,7 +332,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* empty = full + STAGES;
   uint64_t* tfull = empty + STAGES;
   uint64_t* tempty = tfull + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + 2);
+  uint64_t* never = tempty + 2;  // the diagnostics hook's barrier (nothing arrives on it)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(never + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   float* xchg = reinterpret_cast<float*>(smem + STAGES * C::kStageBytes + 256);
 
@@ -411,15 +357,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&tfull[b], 1);
       mbar_init(&tempty[b], 128);
     }
+    mbar_init(never, 1);
     *abort_flag = 0;
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    sm100::mbar_init_fence();
   }
-  if (warp == 1) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
-                     smem_u32(tmem_slot)),
-                 "r"(C::kTmemCols));
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
-  }
+  if (warp == 1) sm100::tmem_alloc(tmem_slot, C::kTmemCols);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -441,6 +383,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
+      if (lane == 0) ok = !probe_abort(probe, never, abort_flag, st, 190 + MODE);
+      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
       for (int64_t u = blockIdx.x; u < total_units && ok; u += gridDim.x) {
         const Unit w = decode_unit(u / ksplit, RB, NTMAX, tile_start, offsets, E, emod);
         const int ks = (int)(u % ksplit);
@@ -506,7 +450,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint64_t wpol = kDecode ? l2_evict_first_policy() : 0;
       int stage = 0;
       uint32_t phase = 0;
-      bool ok = true;
+      bool ok = !probe_abort(probe, never, abort_flag, st, 190 + MODE);
       // With programmatic dependent launch the token rows (written by the
       // preceding kernel) may be read only after grid_dep_wait(); the weight
       // tiles of the first ring of stages are fetched before it.
@@ -722,7 +666,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_ld16(taddr + c0, v);
           int lim = w.nrows - c0 < 16 ? w.nrows - c0 : 16;
           if (!res) {
-            store_down_t8(v, out, w.row0 + c0, lim, M_rows, m & ~7, lim_m != 0, lane);
+            store_down_t8(v, out, w.row0 + c0, lim, M_rows, m & ~7, lim_m != 0, lane, yrow,
+                          yrow ? (int64_t)offsets[E] : 0, st);
             continue;
           }
           lim = lim < lim_m ? lim : lim_m;
@@ -740,8 +685,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 1) {
     __syncwarp();
     tc_fence_after();
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
-                 "r"(C::kTmemCols));
+    sm100::tmem_dealloc(tmem_base, C::kTmemCols);
   }
 }
 
@@ -818,19 +762,29 @@ __device__ __forceinline__ uint32_t idesc_bf16_m256(int n) {
 }
 
 constexpr int kPairNt = 256;     // token rows per tile (N, split 128 + 128)
-constexpr int kPairStages = 6;   // (A 16 KB + B half 16 KB) per stage
 
+// PUM weight blocks of 256 rows (128 per CTA) per unit, all against the same
+// token tile.  PUM = 1: 6 stages of (A 16 KB + B half 16 KB) per CTA, two
+// TMEM accumulator buffers (the epilogue of one unit overlaps the MMAs of the
+// next).  PUM = 2: 4 stages of (A 2 x 16 KB + B half 16 KB): each token byte
+// brought from L2 feeds twice the MMAs; the two 256-column accumulators fill
+// TMEM, so there is one buffer, and the next unit's first-block MMAs run on
+// held stages while the epilogue drains the second accumulator.
+template <int PUM>
 struct PairCfg {
-  static constexpr int kABytes = BM * BK * 2;
+  static constexpr int kStages = PUM == 1 ? 6 : 4;
+  static constexpr int kABlockBytes = BM * BK * 2;
+  static constexpr int kABytes = PUM * kABlockBytes;
   static constexpr int kBBytes = (kPairNt / 2) * BK * 2;
   static constexpr int kStageBytes = kABytes + kBBytes;
   static constexpr int kBufCols = kPairNt;
   static constexpr int kTmemCols = 2 * kPairNt;
-  static constexpr size_t kSmem = (size_t)kPairStages * kStageBytes + 1024 + 256 + kXchgBytes;
+  static constexpr size_t kSmem = (size_t)kStages * kStageBytes + 1024 + 256 + kXchgBytes;
   static_assert(kSmem <= 227 * 1024, "shared memory");
+  static_assert(PUM == 1 || PUM == 2, "one or two weight blocks per unit");
 };
 
-template <int MODE>
+template <int MODE, int PUM>
 __global__ void __launch_bounds__(kThreads, 1)
     k_expert_gemm_pair(const __grid_constant__ CUtensorMap tmA0,
                        const __grid_constant__ CUtensorMap tmA1,
@@ -839,9 +793,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                        const int32_t* __restrict__ offsets, const int32_t* __restrict__ tile_start,
                        int E, int M_rows, int Kdim, __nv_bfloat16* __restrict__ out,
                        const __nv_bfloat16* __restrict__ res, int act_kind, float beta,
-                       float lbeta, DeviceStatus* st, int pdl, int emod) {
-  using C = PairCfg;
-  constexpr int STAGES = kPairStages;
+                       float lbeta, DeviceStatus* st, int pdl, int emod, int probe,
+                       const int32_t* __restrict__ yrow) {
+  using C = PairCfg<PUM>;
+  constexpr int STAGES = C::kStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -849,7 +804,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* empty = full + STAGES;
   uint64_t* tfull = empty + STAGES;
   uint64_t* tempty = tfull + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + 2);
+  uint64_t* never = tempty + 2;  // the diagnostics hook's barrier (nothing arrives on it)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(never + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   float* xchg = reinterpret_cast<float*>(smem + STAGES * C::kStageBytes + 256);
 
@@ -857,12 +813,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t rank = cluster_rank();  // 0: issues the MMAs for the pair
   const bool leader = rank == 0;
   const int pair_id = blockIdx.x >> 1, npairs = gridDim.x >> 1;
-  // rows of the output per CTA: 64 d_ff rows (gate_up) or 128 d rows (down)
+  // rows of the output per CTA and weight block: 64 d_ff rows (gate_up) or
+  // 128 d rows (down); a block is 2 * blk_rows rows of the pair, a unit PUM
+  // blocks
   const int blk_rows = (MODE == kGateUp) ? kGateUpRows : BM;
-  const int unit_rows = 2 * blk_rows;
+  const int unit_rows = PUM * 2 * blk_rows;
   const int RB = (M_rows + unit_rows - 1) / unit_rows;
   const int KB = Kdim / BK;
   const int64_t total_units = (int64_t)tile_start[E] * RB;
+  // TMEM accumulators: PUM = 1, tfull/tempty[i] guard buffer i (units
+  // alternate); PUM = 2, they guard the accumulator of block i (one buffer)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -873,8 +833,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&tfull[b], 1);
       mbar_init(&tempty[b], 256);
     }
+    mbar_init(never, 1);
     *abort_flag = 0;
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    sm100::mbar_init_fence();
   }
   if (warp == 1) {
     asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
@@ -893,7 +854,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
-      bool ok = true;
+      bool ok = !probe_abort(probe, never, abort_flag, st, 290 + MODE);
       bool dep_pending = pdl != 0;  // see the single-CTA kernel
       for (int64_t u = pair_id; u < total_units && ok; u += npairs) {
         const Unit w = decode_unit(u, RB, kPairNt, tile_start, offsets, E, emod);
@@ -903,14 +864,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int brows = big ? kBigBoxRows : kBoxRows;
         const int nb = (half + brows - 1) / brows;
         const uint32_t cta_bytes = C::kABytes + nb * brows * BK * 2;
-        const int ra = w.rb * unit_rows + rank * blk_rows;
         const int tb = w.row0 + rank * half;
         auto load_a = [&](int kb, uint8_t* sA, int st_idx) {
-          if (MODE == kGateUp) {
-            tma_load_3d_pair(&tmA0, &full[st_idx], sA, kb * BK, ra, w.e);
-            tma_load_3d_pair(&tmA1, &full[st_idx], sA + kGateUpRows * BK * 2, kb * BK, ra, w.e);
-          } else {
-            tma_load_3d_pair(&tmA0, &full[st_idx], sA, kb * BK, ra, w.e);
+#pragma unroll
+          for (int a = 0; a < PUM; ++a) {
+            const int ra = w.rb * unit_rows + a * 2 * blk_rows + rank * blk_rows;
+            uint8_t* dA = sA + a * C::kABlockBytes;
+            if (MODE == kGateUp) {
+              tma_load_3d_pair(&tmA0, &full[st_idx], dA, kb * BK, ra, w.e);
+              tma_load_3d_pair(&tmA1, &full[st_idx], dA + kGateUpRows * BK * 2, kb * BK, ra, w.e);
+            } else {
+              tma_load_3d_pair(&tmA0, &full[st_idx], dA, kb * BK, ra, w.e);
+            }
           }
         };
         auto load_b = [&](int kb, uint8_t* sB, int st_idx) {
@@ -960,24 +925,79 @@ __global__ void __launch_bounds__(kThreads, 1)
         const Unit w = decode_unit(u, RB, kPairNt, tile_start, offsets, E, emod);
         const int n = ((w.nrows + 15) / 16) * 16;
         const uint32_t idesc = idesc_bf16_m256(n);
-        const int buf = local & 1;
-        const uint32_t tphase = (local >> 1) & 1;
-        if (!mbar_wait(&tempty[buf], tphase ^ 1, abort_flag)) { ok = false; break; }
-        tc_fence_after();
-        const uint32_t d0 = tmem_base + buf * C::kBufCols;
-        for (int kb = 0; kb < KB; ++kb) {
-          if (!mbar_wait(&full[stage], phase, abort_flag)) { ok = false; break; }
-          tc_fence_after();
-          const uint32_t a0 = smem_u32(smem + stage * C::kStageBytes);
-          const uint32_t b0 = a0 + C::kABytes;
+        // the MMAs of weight block a on stage st (k-block kb)
+        auto mma_block = [&](int a, int st, int kb, uint32_t d) {
+          const uint32_t a0 = smem_u32(smem + st * C::kStageBytes) + a * C::kABlockBytes;
+          const uint32_t b0 = smem_u32(smem + st * C::kStageBytes) + C::kABytes;
 #pragma unroll
           for (int k = 0; k < BK / UK; ++k)
-            umma_bf16_pair(d0, sw128_desc(a0 + k * UK * 2), sw128_desc(b0 + k * UK * 2), idesc,
+            umma_bf16_pair(d, sw128_desc(a0 + k * UK * 2), sw128_desc(b0 + k * UK * 2), idesc,
                            (kb | k) != 0);
-          umma_commit_pair(&empty[stage]);
-          if (++stage == STAGES) { stage = 0; phase ^= 1; }
+        };
+        if constexpr (PUM == 1) {
+          const int buf = local & 1;
+          const uint32_t tphase = (local >> 1) & 1;
+          if (!mbar_wait(&tempty[buf], tphase ^ 1, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t d0 = tmem_base + buf * C::kBufCols;
+          for (int kb = 0; kb < KB; ++kb) {
+            if (!mbar_wait(&full[stage], phase, abort_flag)) { ok = false; break; }
+            tc_fence_after();
+            mma_block(0, stage, kb, d0);
+            umma_commit_pair(&empty[stage]);
+            if (++stage == STAGES) { stage = 0; phase ^= 1; }
+          }
+          if (ok) umma_commit_pair(&tfull[buf]);
+        } else {
+          // block 0's accumulator must be drained before the unit starts;
+          // block 1's may still be draining: its MMAs wait on held stages
+          // (kept out of the ring until both blocks have used them)
+          const uint32_t tpar = (local & 1) ^ 1;
+          if (!mbar_wait(&tempty[0], tpar, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          int held_st[STAGES], held_kb[STAGES];
+          int held = 0;
+          bool b1_free = false;
+          auto flush_held = [&]() {
+            for (int i = 0; i < held; ++i) {
+              mma_block(1, held_st[i], held_kb[i], tmem_base + C::kBufCols);
+              umma_commit_pair(&empty[held_st[i]]);
+            }
+            held = 0;
+          };
+          for (int kb = 0; kb < KB; ++kb) {
+            if (!b1_free && held == STAGES) {  // the ring is all held: wait for block 1
+              if (!mbar_wait(&tempty[1], tpar, abort_flag)) { ok = false; break; }
+              tc_fence_after();
+              b1_free = true;
+              flush_held();
+            }
+            if (!mbar_wait(&full[stage], phase, abort_flag)) { ok = false; break; }
+            tc_fence_after();
+            mma_block(0, stage, kb, tmem_base);
+            if (kb == KB - 1) umma_commit_pair(&tfull[0]);  // block 0 is complete
+            if (!b1_free && mbar_try_wait(&tempty[1], tpar)) {
+              tc_fence_after();
+              b1_free = true;
+              flush_held();
+            }
+            if (b1_free) {
+              mma_block(1, stage, kb, tmem_base + C::kBufCols);
+              umma_commit_pair(&empty[stage]);
+            } else {
+              held_st[held] = stage;
+              held_kb[held] = kb;
+              ++held;
+            }
+            if (++stage == STAGES) { stage = 0; phase ^= 1; }
+          }
+          if (ok && !b1_free) {
+            if (!mbar_wait(&tempty[1], tpar, abort_flag)) { ok = false; break; }
+            tc_fence_after();
+            flush_held();
+          }
+          if (ok) umma_commit_pair(&tfull[1]);
         }
-        if (ok) umma_commit_pair(&tfull[buf]);
       }
       if (!ok) {
         record_error(st, MOE_ERR_DEVICE_TIMEOUT, 210 + MODE);
@@ -992,18 +1012,21 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tempty_leader0 = peer_addr(smem_u32(&tempty[0]), 0);
     int local = 0;
     uint32_t xbuf = 0;
-    for (int64_t u = pair_id; u < total_units; u += npairs, ++local) {
+    bool stop = false;
+    for (int64_t u = pair_id; u < total_units && !stop; u += npairs, ++local) {
       const Unit w = decode_unit(u, RB, kPairNt, tile_start, offsets, E, emod);
-      const int buf = local & 1;
-      const uint32_t tphase = (local >> 1) & 1;
+      for (int a = 0; a < PUM; ++a) {
+      const int buf = PUM == 1 ? (local & 1) : a;
+      const uint32_t tphase = PUM == 1 ? ((local >> 1) & 1) : (local & 1);
       if (!mbar_wait(&tfull[buf], tphase, abort_flag)) {
         if (lane == 0) record_error(st, MOE_ERR_DEVICE_TIMEOUT, 220 + MODE);
         *abort_flag = 1;
+        stop = true;
         break;
       }
       tc_fence_after();
       const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + buf * C::kBufCols;
-      const int r0 = w.rb * unit_rows + rank * blk_rows;
+      const int r0 = w.rb * unit_rows + a * 2 * blk_rows + rank * blk_rows;
       if (MODE == kGateUp) {
         const int pair = quarter & 1;
         const bool is_g = quarter < 2;
@@ -1042,7 +1065,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_ld16(taddr + c0, v);
           int lim = w.nrows - c0 < 16 ? w.nrows - c0 : 16;
           if (!res) {
-            store_down_t8(v, out, w.row0 + c0, lim, M_rows, m & ~7, lim_m != 0, lane);
+            store_down_t8(v, out, w.row0 + c0, lim, M_rows, m & ~7, lim_m != 0, lane, yrow,
+                          yrow ? (int64_t)offsets[E] : 0, st);
             continue;
           }
           lim = lim < lim_m ? lim : lim_m;
@@ -1052,8 +1076,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       tc_fence_before();
-      // release the buffer to the even CTA's MMA issuer
+      // release the buffer (or the block's accumulator) to the even CTA's
+      // MMA issuer
       mbar_arrive_remote(tempty_leader0 + buf * (uint32_t)sizeof(uint64_t));
+      }  // weight blocks
     }
   }
   __syncthreads();
@@ -1154,6 +1180,10 @@ bool make_map_2d(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// The diagnostics hook's switch (moe_set_wait_probe), read at every launch.
+std::atomic<int> g_wait_probe{0};
+int wait_probe() { return g_wait_probe.load(std::memory_order_relaxed); }
+
 template <int MODE, int NTMAX, int STAGES, int UM, int KSUB>
 cudaError_t launch_gemm(const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorMap& b,
                         const CUtensorMap& b64, const int32_t* offsets, const int32_t* tile_start,
@@ -1161,7 +1191,7 @@ cudaError_t launch_gemm(const CUtensorMap& a0, const CUtensorMap& a1, const CUte
                         const __nv_bfloat16* res, const moe_act_cfg& act, DeviceStatus* st,
                         cudaStream_t s, bool pdl_ok, const int32_t* gperm = nullptr,
                         int gk = 1, int gn = 0, int ksplit = 1, float* part = nullptr,
-                        int emod = 0) {
+                        int emod = 0, const int32_t* yrow = nullptr) {
   using C = Cfg<NTMAX, STAGES, UM, KSUB>;
   static std::once_flag once[kMaxDevices];
   static cudaError_t set_up[kMaxDevices];
@@ -1189,8 +1219,14 @@ cudaError_t launch_gemm(const CUtensorMap& a0, const CUtensorMap& a1, const CUte
   return counted(cudaLaunchKernelEx(&cfg, k_expert_gemm<MODE, NTMAX, STAGES, UM, KSUB>, a0, a1, b, b64,
                             offsets, tile_start, E, M_rows, Kdim, out, res, (int)act.kind,
                             act.beta, act.linear_beta, st, pdl, gperm, gk, gn, ksplit, part,
-                            emod > 0 ? emod : E));
+                            emod > 0 ? emod : E, wait_probe(), yrow));
 }
+
+// Weight blocks per CTA-pair unit (1 or 2; see PairCfg).
+#ifndef MOE_PAIR_BLOCKS
+#define MOE_PAIR_BLOCKS 1
+#endif
+constexpr int kPairBlocks = MOE_PAIR_BLOCKS;
 
 // Launches the CTA-pair kernel on as many pairs as can be resident at once.
 template <int MODE>
@@ -1199,8 +1235,9 @@ cudaError_t launch_gemm_pair(const CUtensorMap& a0, const CUtensorMap& a1, const
                              const int32_t* tile_start, int E, int M_rows, int Kdim,
                              __nv_bfloat16* out, const __nv_bfloat16* res,
                              const moe_act_cfg& act, DeviceStatus* st, cudaStream_t s,
-                             bool pdl_ok, int emod = 0) {
-  using C = PairCfg;
+                             bool pdl_ok, int emod = 0, const int32_t* yrow = nullptr) {
+  using C = PairCfg<kPairBlocks>;
+  constexpr auto kernel = k_expert_gemm_pair<MODE, kPairBlocks>;
   static std::once_flag once[kMaxDevices];
   static cudaError_t set_up[kMaxDevices];
   static int grid_of[kMaxDevices] = {0};
@@ -1220,14 +1257,13 @@ cudaError_t launch_gemm_pair(const CUtensorMap& a0, const CUtensorMap& a1, const
   const int pdl = (MODE == kDown && pdl_ok) ? 1 : 0;
   // kernel attribute and the number of resident pairs, once per device
   const cudaError_t e0 = once_per_device(once, set_up, [&](int dev) {
-    cudaError_t e = cudaFuncSetAttribute(k_expert_gemm_pair<MODE>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)C::kSmem);
     if (e != cudaSuccess) return e;
     int pairs = 0;
     cudaLaunchConfig_t q = cfg;
     q.gridDim = dim3(dev_info()->sm_count & ~1, 1, 1);
-    e = cudaOccupancyMaxActiveClusters(&pairs, k_expert_gemm_pair<MODE>, &q);
+    e = cudaOccupancyMaxActiveClusters(&pairs, kernel, &q);
     if (e != cudaSuccess || pairs < 1) pairs = dev_info()->sm_count / 2;
     if (pairs > dev_info()->sm_count / 2) pairs = dev_info()->sm_count / 2;
     grid_of[dev] = 2 * pairs;
@@ -1238,9 +1274,9 @@ cudaError_t launch_gemm_pair(const CUtensorMap& a0, const CUtensorMap& a1, const
   cudaGetDevice(&dev);
   cfg.gridDim = dim3(grid_of[dev], 1, 1);
   cfg.numAttrs = pdl ? 2 : 1;
-  return counted(cudaLaunchKernelEx(&cfg, k_expert_gemm_pair<MODE>, a0, a1, b, b64, offsets, tile_start,
+  return counted(cudaLaunchKernelEx(&cfg, kernel, a0, a1, b, b64, offsets, tile_start,
                             E, M_rows, Kdim, out, res, (int)act.kind, act.beta, act.linear_beta,
-                            st, pdl, emod > 0 ? emod : E));
+                            st, pdl, emod > 0 ? emod : E, wait_probe(), yrow));
 }
 
 // Variant choice from shapes only (no host round trip), by the average rows
@@ -1265,19 +1301,19 @@ cudaError_t launch_variant(Variant v, const CUtensorMap& a0, const CUtensorMap& 
                            const int32_t* tile_start, int E, int M_rows, int Kdim,
                            __nv_bfloat16* out, const __nv_bfloat16* res, const moe_act_cfg& act,
                            DeviceStatus* st, cudaStream_t s, bool pdl_ok = true,
-                           int emod = 0) {
+                           int emod = 0, const int32_t* yrow = nullptr) {
   switch (v) {
     case kVarDecode:
       return launch_gemm<MODE, kNtDecode, kStagesDecode, kUmDecode, kKsubDecode>(
           a0, a1, b, b64, offsets, tile_start, E, M_rows, Kdim, out, res, act, st, s, pdl_ok,
-          nullptr, 1, 0, 1, nullptr, emod);
+          nullptr, 1, 0, 1, nullptr, emod, yrow);
     case kVarMid:
       return launch_gemm<MODE, kNtMid, kStagesMid, kUmMid, kKsubMid>(
           a0, a1, b, b64, offsets, tile_start, E, M_rows, Kdim, out, res, act, st, s, pdl_ok,
-          nullptr, 1, 0, 1, nullptr, emod);
+          nullptr, 1, 0, 1, nullptr, emod, yrow);
     default:
       return launch_gemm_pair<MODE>(a0, a1, b, b64, offsets, tile_start, E, M_rows, Kdim, out,
-                                    res, act, st, s, pdl_ok, emod);
+                                    res, act, st, s, pdl_ok, emod, yrow);
   }
 }
 
@@ -1294,7 +1330,8 @@ int expert_ffn_run(const __nv_bfloat16* xs, const int32_t* offsets, int E, int64
                    int F, const __nv_bfloat16* w1, const __nv_bfloat16* w3,
                    const __nv_bfloat16* w2, const moe_act_cfg& act, __nv_bfloat16* y,
                    void* scratch, DeviceStatus* st, cudaStream_t s, cudaEvent_t after_gate_up,
-                   const __nv_bfloat16* residual, const GatherSrc* gather, int n_weights) {
+                   const __nv_bfloat16* residual, const GatherSrc* gather, int n_weights,
+                   const int32_t* y_rows) {
   // segments s use weights s % n_weights (n_weights = E for the layer)
   const int emod = n_weights > 0 ? n_weights : E;
   int32_t* tile_start = static_cast<int32_t*>(scratch);
@@ -1334,7 +1371,7 @@ int expert_ffn_run(const __nv_bfloat16* xs, const int32_t* offsets, int E, int64
   if (rc != cudaSuccess) return MOE_ERR_CUDA;
   if (after_gate_up && cudaEventRecord(after_gate_up, s) != cudaSuccess) return MOE_ERR_CUDA;
   rc = launch_variant<kDown>(var, mw2, mw2, mh, mh64, offsets, tile_start, E, d_e, F, y, residual,
-                             act, st, s, true, emod);
+                             act, st, s, true, emod, y_rows);
   return rc == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
@@ -1512,3 +1549,7 @@ int shared_ffn_run(const __nv_bfloat16* x, int64_t M, int d, int F, const __nv_b
 }
 
 }  // namespace moe
+
+extern "C" int moe_set_wait_probe(int on) {
+  return moe::g_wait_probe.exchange(on ? 1 : 0);
+}

@@ -87,9 +87,14 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
 // router.cu
 int route_splits(int64_t N, int E, int d_r);
 size_t route_partial_bytes(int64_t N, int E, int d_r);
-// gate GEMM into the router scratch; the fp32 logits [N, E] are at its start
+// gate GEMM into the router scratch; the fp32 logits [N, E] are at its start.
+// reduce = false leaves split-K partials unsummed (route_fused_partials says
+// where they are; the selection sums them).
 cudaError_t launch_gate(const __nv_bfloat16* x, int64_t N, int d_r, const float* W, int E,
-                        void* scratch, DeviceStatus* st, cudaStream_t s);
+                        void* scratch, DeviceStatus* st, cudaStream_t s, bool reduce = true);
+// the gate GEMM's double partials [splits, N, E] when the fp32 path splits
+// over d_r (*splits set), else nullptr (*splits = 1)
+const double* route_fused_partials(void* scratch, int64_t N, int E, int d_r, int* splits);
 
 // router_i8.cu: the same GEMM on the int8 tensor cores (exact digit products),
 // used when the batch fills enough 128x96 tiles
@@ -98,9 +103,11 @@ size_t gate_i8_scratch_bytes(int64_t N, int E, int d_r);
 cudaError_t launch_gate_i8(const __nv_bfloat16* x, int64_t N, int d_r, const float* W, int E,
                            void* scratch, DeviceStatus* st, cudaStream_t s);
 float* route_logits_of(void* scratch);
+// part (optional): take the logits as the sum of the gate GEMM's split
+// partials instead of reading `logits`
 cudaError_t launch_select(const float* logits, int64_t N, const float* bias,
                           const moe_route_cfg& cfg, int32_t* idx, float* w, DeviceStatus* st,
-                          cudaStream_t s);
+                          cudaStream_t s, const double* part = nullptr, int splits = 1);
 
 // dispatch.cu
 int dispatch_chunks(int64_t S);
@@ -131,13 +138,15 @@ bool expert_gather_fusable(int64_t S, int E);
 // residual (optional, [S, d_e] bf16): y = bf16(bf16(x.w2^T) + residual);
 // gather (optional): xs is not read, the rows come from gather->x_e;
 // n_weights: E segments (offsets[E+1]) use weights s % n_weights of the
-// stacked w1/w3/w2 ([n_weights, ...]); 0 means n_weights = E
+// stacked w1/w3/w2 ([n_weights, ...]); 0 means n_weights = E;
+// y_rows (optional, [S]): sorted row j of the output is stored at row
+// y_rows[j] of y (the slot-order scatter; not with a residual)
 int expert_ffn_run(const __nv_bfloat16* xs, const int32_t* offsets, int E, int64_t S, int d_e,
                    int F, const __nv_bfloat16* w1, const __nv_bfloat16* w3,
                    const __nv_bfloat16* w2, const moe_act_cfg& act, __nv_bfloat16* y,
                    void* scratch, DeviceStatus* st, cudaStream_t s, cudaEvent_t after_gate_up,
                    const __nv_bfloat16* residual = nullptr, const GatherSrc* gather = nullptr,
-                   int n_weights = 0);
+                   int n_weights = 0, const int32_t* y_rows = nullptr);
 // Dense layers on the same kernels (one expert, every row): `tiles` is 8 int32
 // of device memory written by launch_dense_tiles(M) before use.
 constexpr size_t kDenseTilesBytes = 256;
@@ -163,7 +172,8 @@ int shared_ffn_run(const __nv_bfloat16* x, int64_t M, int d, int F, const __nv_b
                    const int32_t* tiles, DeviceStatus* st, cudaStream_t s, float* part);
 
 // combine.cu
-// residual (optional, [N, d_e]): out = bf16(bf16(sum) + residual)
+// residual (optional, [N, d_e]): out = bf16(bf16(sum) + residual);
+// pos == nullptr: y is in slot order (token t's K rows at t*K .. t*K+K-1)
 cudaError_t launch_combine(const __nv_bfloat16* y, const int32_t* pos, const float* w, int64_t N,
                            int K, int d_e, int64_t S, __nv_bfloat16* out, DeviceStatus* st,
                            cudaStream_t s, const __nv_bfloat16* residual = nullptr);

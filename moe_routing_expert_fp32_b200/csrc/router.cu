@@ -26,17 +26,19 @@ namespace moe {
 namespace {
 
 constexpr int GT = 64;    // tokens per tile
-constexpr int GE = 64;    // experts per tile
+constexpr int GE = 128;   // experts per tile
 constexpr int GK = 32;    // k per chunk = length of every fp32 FMA chain
-constexpr int GEP = GE + 2;  // padded row of the transposed W tile (8-byte aligned)
+constexpr int GEP = GE + 4;  // padded row of the transposed W tile (16-byte aligned)
 constexpr float kNegInf = -INFINITY;
 
-// logits (or split-K partials) of a 64-token x 64-expert tile.  Thread
-// (tx = lane, ty = warp) owns tokens ty*8..ty*8+7 and experts tx*2, tx*2+1;
-// the token values are warp-uniform (broadcast loads).  Each 32-wide k chunk
-// is accumulated in fp32 (FMA) and then added to a double accumulator, so no
-// fp32 rounding chain is longer than 32 terms.  Chunks are staged global ->
-// registers -> shared memory one chunk ahead (double buffer).
+// logits (or split-K partials) of a 64-token x 128-expert tile.  Thread
+// (tx = lane, ty = warp) owns tokens ty*8..ty*8+7 and experts tx*4..tx*4+3:
+// per k it reads the 8 token values as one warp-uniform (broadcast) 16-byte
+// load of bf16 and its 4 weights as one 16-byte load, for 32 FMAs.  Each
+// 32-wide k chunk is accumulated in fp32 (FMA, k ascending) and then added
+// to a double accumulator, so no fp32 rounding chain is longer than 32
+// terms.  Chunks are staged global -> registers -> shared memory one chunk
+// ahead (double buffer).
 __global__ void __launch_bounds__(256, 2) k_gate_partial(const __nv_bfloat16* __restrict__ x,
                                                          int64_t N, int d,
                                                          const float* __restrict__ W, int E,
@@ -45,7 +47,7 @@ __global__ void __launch_bounds__(256, 2) k_gate_partial(const __nv_bfloat16* __
                                                          double* __restrict__ part) {
   pdl_wait();
   pdl_trigger();
-  __shared__ __align__(16) float xs[2][GK][GT];
+  __shared__ __align__(16) __nv_bfloat16 xs[2][GK][GT];
   __shared__ __align__(16) float wsm[2][GK][GEP];
   const int tid = threadIdx.x;
   const int tx = tid & 31, ty = tid >> 5;
@@ -56,16 +58,16 @@ __global__ void __launch_bounds__(256, 2) k_gate_partial(const __nv_bfloat16* __
   const int kc1 = min(nk, kc0 + cps);
 
   // global -> register staging of one chunk: x 64 tokens x 32 k (one 16-byte
-  // vector per thread), W 64 experts x 32 k (two float4 per thread)
+  // vector of 8 bf16 per thread), W 128 experts x 32 k (four float4 per thread)
   const int xtok = tid >> 2, xkk = (tid & 3) * 8;
   uint4 xr = make_uint4(0, 0, 0, 0);
-  float4 wr[2];
+  float4 wr[4];
   auto load_chunk = [&](int kc) {
     const int k0 = kc * GK;
     xr = make_uint4(0, 0, 0, 0);
     if (t0 + xtok < N) xr = *reinterpret_cast<const uint4*>(x + (t0 + xtok) * d + k0 + xkk);
 #pragma unroll
-    for (int r = 0; r < 2; ++r) {
+    for (int r = 0; r < 4; ++r) {
       const int i = tid + 256 * r;
       const int ex = i >> 3, kq = (i & 7) * 4;
       wr[r] = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -76,9 +78,9 @@ __global__ void __launch_bounds__(256, 2) k_gate_partial(const __nv_bfloat16* __
   auto store_chunk = [&](int b) {
     const __nv_bfloat16* h = reinterpret_cast<const __nv_bfloat16*>(&xr);
 #pragma unroll
-    for (int j = 0; j < 8; ++j) xs[b][xkk + j][xtok] = __bfloat162float(h[j]);
+    for (int j = 0; j < 8; ++j) xs[b][xkk + j][xtok] = h[j];
 #pragma unroll
-    for (int r = 0; r < 2; ++r) {
+    for (int r = 0; r < 4; ++r) {
       const int i = tid + 256 * r;
       const int ex = i >> 3, kq = (i & 7) * 4;
       wsm[b][kq + 0][ex] = wr[r].x;
@@ -88,9 +90,11 @@ __global__ void __launch_bounds__(256, 2) k_gate_partial(const __nv_bfloat16* __
     }
   };
 
-  double acc[8][2];
+  double acc[8][4];
 #pragma unroll
-  for (int i = 0; i < 8; ++i) acc[i][0] = acc[i][1] = 0.0;
+  for (int i = 0; i < 8; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) acc[i][j] = 0.0;
 
   int buf = 0;
   if (kc0 < kc1) {
@@ -101,26 +105,30 @@ __global__ void __launch_bounds__(256, 2) k_gate_partial(const __nv_bfloat16* __
   for (int kc = kc0; kc < kc1; ++kc) {
     const bool more = kc + 1 < kc1;
     if (more) load_chunk(kc + 1);
-    float blk[8][2];
+    float blk[8][4];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) blk[i][0] = blk[i][1] = 0.f;
+    for (int i = 0; i < 8; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) blk[i][j] = 0.f;
 #pragma unroll 8
     for (int k = 0; k < GK; ++k) {
-      const float4 a0 = *reinterpret_cast<const float4*>(&xs[buf][k][ty * 8]);
-      const float4 a1 = *reinterpret_cast<const float4*>(&xs[buf][k][ty * 8 + 4]);
-      const float2 b = *reinterpret_cast<const float2*>(&wsm[buf][k][tx * 2]);
-      const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+      const uint4 a = *reinterpret_cast<const uint4*>(&xs[buf][k][ty * 8]);
+      const float4 b = *reinterpret_cast<const float4*>(&wsm[buf][k][tx * 4]);
+      // bf16 -> fp32 is exact: the 16 bits become the high half of the word
+      const float av[8] = {__uint_as_float(a.x << 16), __uint_as_float(a.x & 0xFFFF0000u),
+                           __uint_as_float(a.y << 16), __uint_as_float(a.y & 0xFFFF0000u),
+                           __uint_as_float(a.z << 16), __uint_as_float(a.z & 0xFFFF0000u),
+                           __uint_as_float(a.w << 16), __uint_as_float(a.w & 0xFFFF0000u)};
+      const float bv[4] = {b.x, b.y, b.z, b.w};
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        blk[i][0] = fmaf(av[i], b.x, blk[i][0]);
-        blk[i][1] = fmaf(av[i], b.y, blk[i][1]);
-      }
+      for (int i = 0; i < 8; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) blk[i][j] = fmaf(av[i], bv[j], blk[i][j]);
     }
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      acc[i][0] += (double)blk[i][0];
-      acc[i][1] += (double)blk[i][1];
-    }
+    for (int i = 0; i < 8; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) acc[i][j] += (double)blk[i][j];
     if (more) store_chunk(buf ^ 1);
     __syncthreads();
     buf ^= 1;
@@ -130,8 +138,8 @@ __global__ void __launch_bounds__(256, 2) k_gate_partial(const __nv_bfloat16* __
     const int64_t t = t0 + ty * 8 + i;
     if (t >= N) continue;
 #pragma unroll
-    for (int j = 0; j < 2; ++j) {
-      const int e = e0 + tx * 2 + j;
+    for (int j = 0; j < 4; ++j) {
+      const int e = e0 + tx * 4 + j;
       if (e >= E) continue;
       if (splits == 1) logits[t * E + e] = (float)acc[i][j];
       else part[((int64_t)blockIdx.z * N + t) * E + e] = acc[i][j];
@@ -274,6 +282,160 @@ __global__ void __launch_bounds__(32 * kSelWarps) k_select(
   }
 }
 
+// Small batches: one block per token, one thread per expert (blockDim = E
+// rounded up to 32).  The logits come either from `logits` or, when the gate
+// GEMM ran split over d_r, straight from its double partials (summed in split
+// order and rounded once, exactly as k_reduce_partials does), so no reduce
+// kernel runs.  The score of each expert is computed by its own thread; the
+// top-K is taken per warp (32 experts each) and the per-warp candidates are
+// merged by warp 0, under the same total order (value desc, index asc) as
+// k_select, so the result is identical to it.
+constexpr int kMaxSelWarps = 32;  // E <= 1024
+constexpr int64_t kBlockSelectMaxN = 1024;  // batches up to this size: a block per token
+__global__ void __launch_bounds__(1024) k_select_block(
+    const float* __restrict__ logits, const double* __restrict__ part, int splits, int64_t N,
+    int E, const float* __restrict__ bias, int G, int TG, int K, int norm, float route_scale,
+    int score_func, int group_mode, int32_t* __restrict__ idx_out, float* __restrict__ w_out,
+    DeviceStatus* st) {
+  pdl_wait();
+  pdl_trigger();
+  __shared__ float s_s[1024];
+  __shared__ float s_c[1024];
+  __shared__ double s_x[1024];
+  __shared__ float cand_v[kMaxSelWarps][16];
+  __shared__ int cand_i[kMaxSelWarps][16];
+  __shared__ float s_red[kMaxSelWarps];
+  __shared__ float s_gs[32];
+  __shared__ unsigned s_kept;
+  __shared__ double s_sum;
+  const int e = threadIdx.x, lane = e & 31, warp = e >> 5;
+  const int nw = blockDim.x >> 5;
+  const int64_t t = blockIdx.x;
+  const bool live = e < E;
+  float L = 0.f;
+  if (live) {
+    if (part) {
+      double a = 0.0;
+      for (int z = 0; z < splits; ++z) a += part[((int64_t)z * N + t) * E + e];
+      L = (float)a;
+    } else {
+      L = logits[t * E + e];
+    }
+  }
+  float sv = 0.f;
+  if (score_func == MOE_SCORE_SOFTMAX) {
+    // block maximum, exp(L - max) in double, the normaliser summed by one
+    // thread in expert order, quotient rounded once (as k_select)
+    float mx = live ? L : -INFINITY;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+    if (lane == 0) s_red[warp] = mx;
+    __syncthreads();
+    mx = s_red[0];
+    for (int i = 1; i < nw; ++i) mx = fmaxf(mx, s_red[i]);
+    if (live) s_x[e] = exp((double)L - (double)mx);
+    __syncthreads();
+    if (e == 0) {
+      double sum = 0.0;
+      for (int i = 0; i < E; ++i) sum += s_x[i];
+      s_sum = sum;
+    }
+    __syncthreads();
+    if (live) sv = (float)(s_x[e] / s_sum);
+  } else if (live) {
+    sv = (float)__drcp_rn(1.0 + exp(-(double)L));
+  }
+  float cv = live ? (bias ? __fadd_rn(sv, bias[e]) : sv) : kNegInf;
+  if (live) {
+    s_s[e] = sv;
+    s_c[e] = cv;
+  }
+  __syncthreads();
+  if (G > 1) {
+    const int gsz = E / G;
+    if (e < G) {
+      float a = kNegInf, b = kNegInf;
+      for (int i = 0; i < gsz; ++i) {
+        const float v = s_c[e * gsz + i];
+        if (v > a) { b = a; a = v; }
+        else if (v > b) { b = v; }
+      }
+      s_gs[e] = group_mode == MOE_GROUP_MAX ? a : __fadd_rn(a, b);
+    }
+    __syncthreads();
+    if (warp == 0) {
+      const float gs = lane < G ? s_gs[lane] : kNegInf;
+      bool kept = false;
+      for (int r = 0; r < TG; ++r) {
+        float v = (lane < G && !kept) ? gs : kNegInf;
+        int i = (lane < G && !kept) ? lane : 0x7fffffff;
+        warp_best(v, i);
+        if (lane == i) kept = true;
+      }
+      const unsigned m = __ballot_sync(0xffffffffu, kept);
+      if (lane == 0) s_kept = m;
+    }
+    __syncthreads();
+    if (live && !((s_kept >> (e / gsz)) & 1u)) cv = kNegInf;
+  }
+  // per-warp top-K of (cv, e), then the merge by warp 0
+  {
+    float v = cv;
+    const int my = live ? e : 0x7fffffff;
+    bool taken = false;
+    for (int k = 0; k < K; ++k) {
+      float bv = taken ? kNegInf : v;
+      int bi = taken ? 0x7fffffff : my;
+      warp_best(bv, bi);
+      if (bi == my) taken = true;
+      if (lane == 0) {
+        cand_v[warp][k] = bv;
+        cand_i[warp][k] = bi;
+      }
+    }
+  }
+  __syncthreads();
+  if (warp == 0) {
+    const int nc = nw * K;  // candidates, lane l holds c = l, l + 32, ...
+    unsigned chosen = 0;
+    int my_e = 0;
+    for (int k = 0; k < K; ++k) {
+      float bv = kNegInf;
+      int bi = 0x7fffffff;
+      for (int j = 0, c = lane; c < nc; ++j, c += 32) {
+        if ((chosen >> j) & 1u) continue;
+        const float cvv = cand_v[c / K][c % K];
+        const int ci = cand_i[c / K][c % K];
+        if (ranks_before(cvv, ci, bv, bi)) { bv = cvv; bi = ci; }
+      }
+      const int src_bi = bi;
+      warp_best(bv, bi);
+      if (bi == 0x7fffffff) {  // cannot happen for a validated config
+        record_error(st, MOE_ERR_DEVICE_BOUNDS, 2);
+        bi = 0;
+      }
+      // the lane whose scan produced the winner marks that candidate taken
+      if (src_bi == bi) {
+        for (int j = 0, c = lane; c < nc; ++j, c += 32)
+          if (!((chosen >> j) & 1u) && cand_i[c / K][c % K] == bi) { chosen |= 1u << j; break; }
+      }
+      if (lane == k) my_e = bi;
+    }
+    float wk = (lane < K) ? s_s[my_e] : 0.f;
+    if (K > 1 && norm) {
+      float den = __shfl_sync(0xffffffffu, wk, 0);
+      for (int k = 1; k < K; ++k) den = __fadd_rn(den, __shfl_sync(0xffffffffu, wk, k));
+      den = __fadd_rn(den, 1e-20f);
+      wk = __fdiv_rn(wk, den);
+    }
+    wk = __fmul_rn(wk, route_scale);
+    if (lane < K) {
+      idx_out[t * K + lane] = my_e;
+      w_out[t * K + lane] = wk;
+    }
+  }
+}
+
 }  // namespace
 
 int route_splits(int64_t N, int E, int d_r) {
@@ -283,7 +445,7 @@ int route_splits(int64_t N, int E, int d_r) {
   int64_t want = (296 + tiles - 1) / tiles;  // about two CTAs per SM
   int64_t maxs = nk / 4 > 0 ? nk / 4 : 1;    // at least 4 chunks per split
   if (want > maxs) want = maxs;
-  if (want > 32) want = 32;
+  if (want > 64) want = 64;
   if (want < 1) want = 1;
   const int cps = (int)((nk + want - 1) / want);
   return (nk + cps - 1) / cps;
@@ -305,8 +467,17 @@ static double* route_part_of(void* scratch, int64_t N, int E) {
                                    align_up(sizeof(float) * (size_t)N * (size_t)E, 256));
 }
 
+const double* route_fused_partials(void* scratch, int64_t N, int E, int d_r, int* splits) {
+  *splits = 1;
+  if (gate_i8_applies(N, E, d_r)) return nullptr;
+  const int sp = route_splits(N, E, d_r);
+  if (sp <= 1) return nullptr;
+  *splits = sp;
+  return route_part_of(scratch, N, E);
+}
+
 cudaError_t launch_gate(const __nv_bfloat16* x, int64_t N, int d_r, const float* W, int E,
-                        void* scratch, DeviceStatus* st, cudaStream_t s) {
+                        void* scratch, DeviceStatus* st, cudaStream_t s, bool reduce) {
   if (gate_i8_applies(N, E, d_r)) return launch_gate_i8(x, N, d_r, W, E, scratch, st, s);
   const int splits = route_splits(N, E, d_r);
   const int nk = d_r / GK;
@@ -317,7 +488,7 @@ cudaError_t launch_gate(const __nv_bfloat16* x, int64_t N, int d_r, const float*
   cudaError_t e = launch_pdl(k_gate_partial, grid, dim3(256), 0, s, x, N, d_r, W, E, cps, splits,
                              logits, part);
   if (e != cudaSuccess) return e;
-  if (splits > 1) {
+  if (splits > 1 && reduce) {
     const int64_t ne = N * (int64_t)E;
     int64_t blocks = (ne + 255) / 256;
     const int64_t cap = (int64_t)dev_info()->sm_count * 16;
@@ -331,8 +502,15 @@ cudaError_t launch_gate(const __nv_bfloat16* x, int64_t N, int d_r, const float*
 
 cudaError_t launch_select(const float* logits, int64_t N, const float* bias,
                           const moe_route_cfg& cfg, int32_t* idx, float* w, DeviceStatus* st,
-                          cudaStream_t s) {
+                          cudaStream_t s, const double* part, int splits) {
   const int E = cfg.num_experts;
+  if (part || N <= kBlockSelectMaxN) {
+    const int threads = (E + 31) / 32 * 32;
+    return launch_pdl(k_select_block, dim3((unsigned)N), dim3(threads), 0, s, logits, part,
+                      splits, N, E, bias, cfg.n_group, cfg.topk_group, cfg.top_k,
+                      cfg.norm_topk_prob, cfg.route_scale, cfg.score_func, cfg.group_score, idx,
+                      w, st);
+  }
   const bool softmax = cfg.score_func == MOE_SCORE_SOFTMAX;
   const size_t smem = sizeof(float) * 2 * E * kSelWarps + (softmax ? sizeof(double) * E * kSelWarps : 0);
   if (softmax && smem > 48 * 1024) {

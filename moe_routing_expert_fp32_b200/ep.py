@@ -186,6 +186,30 @@ def exchange_forward_p2p(x_r, x_e, steps: P2PSteps, num_experts: int, group=None
     return out, idx, w
 
 
+class GrowingBuffer:
+    """A buffer of at least `rows` rows kept from one step to the next: it is
+    (re)allocated only when a step needs more rows than it holds, rounded up
+    to a power of two.  With symmetric memory the allocation is collective;
+    every rank asks for the same row count (the largest receive count, from
+    the all-gathered counts), so every rank reallocates at the same steps."""
+
+    def __init__(self, alloc):
+        self._alloc = alloc
+        self.rows = 0
+        self.obj = None
+
+    def get(self, rows: int):
+        if rows > self.rows:
+            self.rows = 1 << max(0, int(rows) - 1).bit_length()
+            self.obj = None  # the old buffer goes before the new one is made
+            self.obj = self._alloc(self.rows)
+        return self.obj, self.rows
+
+
+# symmetric row buffers of ep_forward_p2p, one per (group, device, width)
+_P2P_BUFFERS: dict = {}
+
+
 def ep_forward_p2p(x_r, W, bias, cfg, w1_local, w3_local, w2_local, act, x_e=None, group=None):
     """The routed layer with this rank's experts (w1_local, w3_local
     [E_local, F, d_e], w2_local [E_local, d_e, F]), the rows moved through
@@ -194,6 +218,8 @@ def ep_forward_p2p(x_r, W, bias, cfg, w1_local, w3_local, w2_local, act, x_e=Non
     same size on every rank: the largest receive count), the experts write
     their outputs to the other half, and moe_ep_combine_rows loads them back.
     The barriers are a stream synchronisation and a process-group barrier.
+    The buffer is kept for the next step (GrowingBuffer) and grows only when a
+    step receives more rows than it holds.
     Returns (out [N, d_e] bf16, topk_idx, topk_w)."""
     import torch
     import torch.distributed as dist
@@ -206,20 +232,26 @@ def ep_forward_p2p(x_r, W, bias, cfg, w1_local, w3_local, w2_local, act, x_e=Non
     rank = dist.get_rank(group)
     E = cfg.num_experts
     x_e = x_r if x_e is None else x_e
-    held = []  # the symmetric buffer lives until the step returns
 
     def _dispatch(idx, xe):
         counts, offsets, _, pos, _ = dispatch(idx, xe, E, gather=False)
         return counts, offsets, pos
 
+    def _alloc(d_e, device):
+        def make(rows):
+            buf = symm.empty(2 * rows, d_e, dtype=torch.bfloat16, device=device)
+            return buf, symm.rendezvous(buf, group)
+        return make
+
     def _buffers(cap, d_e, like):
-        buf = symm.empty(2 * cap, d_e, dtype=torch.bfloat16, device=like.device)
-        handle = symm.rendezvous(buf, group)
-        held.append((buf, handle))
+        key = (group.group_name, like.device.index, d_e)
+        if key not in _P2P_BUFFERS:
+            _P2P_BUFFERS[key] = GrowingBuffer(_alloc(d_e, like.device))
+        (buf, handle), rows = _P2P_BUFFERS[key].get(cap)
         offset = buf.data_ptr() - handle.buffer_ptrs[rank]
         xr_at = [handle.buffer_ptrs[q] + offset for q in range(P)]
-        y_at = [a + cap * d_e * buf.element_size() for a in xr_at]
-        return buf[:cap], buf[cap:], xr_at, y_at
+        y_at = [a + rows * d_e * buf.element_size() for a in xr_at]
+        return buf[:cap], buf[rows:rows + cap], xr_at, y_at
 
     def _send(xe, pos, offsets, xr_at, first_row, cap):
         ep_dispatch_rows(xe, pos, offsets, E, peer_rows(xr_at, first_row, [cap] * P), cfg.top_k)

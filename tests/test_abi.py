@@ -359,3 +359,35 @@ def test_dispatch_without_the_copy_needs_no_rows(L):
                           None) == -3
 
 
+
+
+def test_expert_ffn_to_slots_validation(L):
+    """moe_expert_ffn_to_slots rejects bad arguments on the host (fake
+    pointers, nothing reaches a device): it needs perm whenever there are
+    rows, the expert MLP's shape limits and 16-byte aligned rows."""
+    import moe_routing_expert_fp32_b200 as m
+    p = ctypes.c_void_p(256)
+    a = m.ActConfig("silu")._c()
+    ws = ctypes.c_void_p(1 << 20)
+    big = 1 << 30
+    # perm missing with rows present
+    assert L.moe_expert_ffn_to_slots(p, p, None, 8, 64, 256, 128, p, p, p, ctypes.byref(a), p, ws,
+                                     big, None) == -1
+    # d_e not a multiple of 128
+    assert L.moe_expert_ffn_to_slots(p, p, p, 8, 64, 200, 128, p, p, p, ctypes.byref(a), p, ws,
+                                     big, None) == -2
+    # y_slots not 16-byte aligned
+    assert L.moe_expert_ffn_to_slots(p, p, p, 8, 64, 256, 128, p, p, p, ctypes.byref(a),
+                                     ctypes.c_void_p(264), ws, big, None) == -3
+    # workspace too small
+    assert L.moe_expert_ffn_to_slots(p, p, p, 8, 64, 256, 128, p, p, p, ctypes.byref(a), p, ws,
+                                     8, None) == -4
+
+
+def test_wait_probe_switch_round_trips(L):
+    """moe_set_wait_probe returns the previous setting; it launches nothing."""
+    before = L.moe_launch_count()
+    prev = L.moe_set_wait_probe(1)
+    assert L.moe_set_wait_probe(prev) == 1
+    assert L.moe_set_wait_probe(prev) == prev
+    assert L.moe_launch_count() == before

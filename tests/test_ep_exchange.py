@@ -242,3 +242,19 @@ def test_exchange_forward_p2p_equals_one_rank(world, E):
         assert p.exitcode == 0
     assert sorted(r[0] for r in res) == list(range(world))
     assert all(r[1] for r in res), res
+
+
+def test_growing_buffer_reallocates_only_when_needed():
+    """The peer-memory step's row buffer is kept across steps and grows to
+    the next power of two only when a step needs more rows; the same row
+    counts give the same decisions on every rank."""
+    from moe_routing_expert_fp32_b200.ep import GrowingBuffer
+    made = []
+    g = GrowingBuffer(lambda rows: made.append(rows) or f"buf{rows}")
+    assert g.get(100) == ("buf128", 128)
+    assert g.get(128) == ("buf128", 128) and g.get(1) == ("buf128", 128)
+    assert g.get(129) == ("buf256", 256)
+    assert g.get(200) == ("buf256", 256)
+    assert made == [128, 256]
+    h = GrowingBuffer(lambda rows: rows)
+    assert h.get(1) == (1, 1) and h.get(3) == (4, 4)

@@ -9,8 +9,10 @@ Bars:
   * moe_rms_norm and the fused combine + RMSNorm: bit-exact (both sides take
     the mean in double and round once from double), allowing a handful of
     one-ulp flips where the two sum orders straddle a rounding midpoint;
-  * moe_block_forward: routing as moe_route; output relative L2 <= 2e-2 over
-    tokens whose biased-score margin exceeds 1e-5.
+  * moe_block_forward: routing as moe_route; over the tokens whose
+    biased-score margin exceeds 1e-5, output relative L2 <= 2e-2 and the
+    per-row and per-element bars of the layer output (tests/gpu_util.py);
+    the shared experts' MLP meets the expert MLP's bars.
 """
 import numpy as np
 import pytest
@@ -18,7 +20,8 @@ import pytest
 import oracle
 import synth
 from synth.workloads import BLOCKS, host_block, host_expert, host_inputs, scaled
-from tests.gpu_util import MARGIN, REL_L2_OUT, dev_bf16, host_bf16, rel_l2, ulp_diff
+from tests.gpu_util import (MARGIN, REL_L2_OUT, check_bf16_outputs, dev_bf16, host_bf16, rel_l2,
+                            ulp_diff)
 
 pytestmark = pytest.mark.gpu
 
@@ -152,9 +155,10 @@ def _check_block(wl, out_g, idx_g, toks, norm=True, shared=True):
     assert keep.mean() > 0.5
     for i in np.nonzero(keep)[0]:
         assert set(idx_g[toks[i]].tolist()) == set(idx_r[i].tolist())
-    err = rel_l2(out_g[toks][keep], out_r[keep])
-    print(f"{wl.name}: {keep.sum()}/{len(toks)} tokens, rel_l2 {err:.2e}")
-    assert err <= REL_L2_OUT
+    print(f"{wl.name}: {keep.sum()}/{len(toks)} tokens")
+    check_bf16_outputs(out_g[toks][keep], out_r[keep],
+                       long_dots=max(wl.d_r, wl.d_e, wl.F, wl.F_shared) > 512,
+                       what=f"block {wl.name}", layer=True, ulp_bars=False)
 
 
 @pytest.mark.parametrize("norm,shared", [(True, True), (False, True), (True, False)])
@@ -174,7 +178,7 @@ def test_block_not_latent_with_shared(moe):
 def test_block_k3_decode(moe):
     wl = BLOCKS["k3_block_decode"]
     out_g, idx_g, _ = _run_block(moe, wl)
-    toks = np.array([0, 5, 17, 31, 40, 63])
+    toks = np.array([0, 3, 5, 9, 17, 22, 28, 31, 36, 40, 44, 49, 53, 58, 61, 63])
     _check_block(wl, out_g, idx_g, toks)
 
 
@@ -231,9 +235,8 @@ def test_shared_experts(moe, M, d, F, act):
     rows = np.arange(M) if M <= 100 else np.array([0, 1, 255, 256, M - 1])
     y_r = oracle.expert_ffn(np.ascontiguousarray(x[rows]), w1, w3, w2, a.kind, a.beta,
                             a.linear_beta)
-    err = rel_l2(y_g[rows], y_r)
-    print(f"M={M} d={d} F={F}: rel_l2 {err:.2e}")
-    assert err <= REL_L2_OUT
+    print(f"M={M} d={d} F={F}")
+    check_bf16_outputs(y_g[rows], y_r, long_dots=max(d, F) > 512, what=f"shared M={M}")
     z_g = host_bf16(moe.shared_experts(dev_bf16(x), dev_bf16(w1), dev_bf16(w3), dev_bf16(w2), a,
                                        residual=dev_bf16(res)))
     assert np.array_equal(z_g, oracle.add(y_g, res))

@@ -8,7 +8,10 @@ moe_ep_expert_ffn on what it received with its own slice of the expert
 weights; the outputs go back to their sources in the same slices and each
 source combines them.  The result must match the single-GPU layer
 (moe_forward) on the same tokens: same routing, outputs within 1e-3 relative
-L2 (the rows meet the same MMAs in the same k order; tile shapes may differ).
+L2 (the rows meet the same MMAs in the same k order; tile shapes may differ);
+and sampled tokens of every rank must meet the reference (the CPU oracle's
+expert MLP and combine, fed with the GPU's routing) under the layer's output
+bars.
 A real multi-GPU run of this exchange (NCCL all-to-all over NVLink) needs
 more than one GPU; its host logic is tested with gloo on CPU.
 """
@@ -16,8 +19,8 @@ import numpy as np
 import pytest
 
 import synth
-from synth.workloads import WORKLOADS, scaled
-from tests.gpu_util import host_bf16, rel_l2
+from synth.workloads import WORKLOADS, host_inputs, scaled
+from tests.gpu_util import check_bf16_outputs, host_bf16, oracle_layer_tokens, rel_l2
 
 pytestmark = pytest.mark.gpu
 
@@ -64,12 +67,33 @@ def test_ep_emulated_equals_one_gpu(moe, name, P, N):
             y_back[p][r["offs"][lo]:r["offs"][hi]] = yq[o:o + n]
             o += n
         assert o == recv.shape[0]
+    outs = []
     for p, r in enumerate(ranks):
         out = moe.combine(y_back[p], r["pos"], r["w"])
+        outs.append(out)
         got, ref = host_bf16(out), host_bf16(r["ref"])
         err = rel_l2(got, ref)
         print(f"{name} rank {p}/{P}: rel_l2 {err:.2e}, bit-exact {np.mean(got == ref):.4f}")
         assert err <= 1e-3
+    _check_against_reference(wl, P, outs, ranks)
+
+
+def _check_against_reference(wl, P, outs, ranks, per_rank=16):
+    """Sampled tokens of every emulated rank against the reference's
+    per-token loop (its expert MLP and combine), fed with the routing the
+    GPU computed for them, so that only the expert-parallel step is judged."""
+    xe, idx, w, got = [], [], [], []
+    for p, r in enumerate(ranks):
+        n = wl.N
+        toks = np.arange(n) if n <= per_rank else np.unique(
+            np.concatenate([[0, n - 1], np.random.default_rng(p).choice(n, per_rank - 2, False)]))
+        xe.append(host_inputs(wl, rank=p)["x_e"][toks])
+        idx.append(r["idx"].cpu().numpy()[toks])
+        w.append(r["w"].cpu().numpy()[toks])
+        got.append(host_bf16(outs[p])[toks])
+    ref = oracle_layer_tokens(wl, np.concatenate(xe), np.concatenate(idx), np.concatenate(w))
+    check_bf16_outputs(np.concatenate(got), ref, long_dots=max(wl.d_e, wl.F) > 512,
+                       what=f"expert-parallel {wl.name} P={P}", layer=True)
 
 
 def test_ep_expert_ffn_reports_inconsistent_counts(moe):
@@ -115,7 +139,8 @@ def test_ep_peer_rows_emulated(moe, name, P, N):
         for a, b2 in ((counts, counts2), (offs, offs2), (perm, perm2), (pos, pos2)):
             assert torch.equal(a, b2)
         ref = moe.forward(d["x"], W, b, cfg, w1, w3, w2, act, x_e=d["x_e"] if wl.latent else None)
-        ranks.append(dict(x_e=x_e, w=w, counts=counts, offs=offs, pos=pos, xs=xs, ref=ref))
+        ranks.append(dict(x_e=x_e, idx=idx, w=w, counts=counts, offs=offs, pos=pos, xs=xs,
+                          ref=ref))
     all_counts = torch.stack([r["counts"] for r in ranks]).cpu().numpy()
     plans = [p2p_plan(all_counts, p, P) for p in range(P)]
     cap = [max(1, plans[q][2]) for q in range(P)]
@@ -138,10 +163,12 @@ def test_ep_peer_rows_emulated(moe, name, P, N):
         assert bool((xr[q][cap[q]] == 7.0).all()), "guard row overwritten"
         rc = torch.from_numpy(plans[q][1]).cuda()
         moe.ep_expert_ffn(xr[q][:R], rc, w1[lo:hi], w3[lo:hi], w2[lo:hi], act, y=yb[q][:R])
+    outs = []
     for p, r in enumerate(ranks):
         table = moe.peer_rows(yb, plans[p][0], cap)
         ws = moe.workspace(256)
         out = moe.ep_combine_rows(table, r["pos"], r["offs"], wl.E, r["w"], wl.d_e, ws=ws)
+        outs.append(out)
         assert moe.get_status(ws) == 0
         # the same outputs brought home in sorted order, then moe_combine
         home = torch.empty_like(r["xs"])
@@ -154,6 +181,7 @@ def test_ep_peer_rows_emulated(moe, name, P, N):
         err = rel_l2(got, ref)
         print(f"{name} rank {p}/{P} (peer rows): rel_l2 {err:.2e}")
         assert err <= 1e-3
+    _check_against_reference(wl, P, outs, ranks)
 
 
 def test_ep_peer_rows_out_of_capacity_is_reported(moe):
