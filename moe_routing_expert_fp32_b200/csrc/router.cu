@@ -26,19 +26,17 @@ namespace moe {
 namespace {
 
 constexpr int GT = 64;    // tokens per tile
-constexpr int GE = 128;   // experts per tile
+constexpr int GE = 64;    // experts per tile
 constexpr int GK = 32;    // k per chunk = length of every fp32 FMA chain
-constexpr int GEP = GE + 4;  // padded row of the transposed W tile (16-byte aligned)
+constexpr int GEP = GE + 2;  // padded row of the transposed W tile (8-byte aligned)
 constexpr float kNegInf = -INFINITY;
 
-// logits (or split-K partials) of a 64-token x 128-expert tile.  Thread
-// (tx = lane, ty = warp) owns tokens ty*8..ty*8+7 and experts tx*4..tx*4+3:
-// per k it reads the 8 token values as one warp-uniform (broadcast) 16-byte
-// load of bf16 and its 4 weights as one 16-byte load, for 32 FMAs.  Each
-// 32-wide k chunk is accumulated in fp32 (FMA, k ascending) and then added
-// to a double accumulator, so no fp32 rounding chain is longer than 32
-// terms.  Chunks are staged global -> registers -> shared memory one chunk
-// ahead (double buffer).
+// logits (or split-K partials) of a 64-token x 64-expert tile.  Thread
+// (tx = lane, ty = warp) owns tokens ty*8..ty*8+7 and experts tx*2, tx*2+1;
+// the token values are warp-uniform (broadcast loads).  Each 32-wide k chunk
+// is accumulated in fp32 (FMA) and then added to a double accumulator, so no
+// fp32 rounding chain is longer than 32 terms.  Chunks are staged global ->
+// registers -> shared memory one chunk ahead (double buffer).
 __global__ void __launch_bounds__(256, 2) k_gate_partial(const __nv_bfloat16* __restrict__ x,
                                                          int64_t N, int d,
                                                          const float* __restrict__ W, int E,
@@ -47,7 +45,7 @@ __global__ void __launch_bounds__(256, 2) k_gate_partial(const __nv_bfloat16* __
                                                          double* __restrict__ part) {
   pdl_wait();
   pdl_trigger();
-  __shared__ __align__(16) __nv_bfloat16 xs[2][GK][GT];
+  __shared__ __align__(16) float xs[2][GK][GT];
   __shared__ __align__(16) float wsm[2][GK][GEP];
   const int tid = threadIdx.x;
   const int tx = tid & 31, ty = tid >> 5;
@@ -58,16 +56,16 @@ __global__ void __launch_bounds__(256, 2) k_gate_partial(const __nv_bfloat16* __
   const int kc1 = min(nk, kc0 + cps);
 
   // global -> register staging of one chunk: x 64 tokens x 32 k (one 16-byte
-  // vector of 8 bf16 per thread), W 128 experts x 32 k (four float4 per thread)
+  // vector per thread), W 64 experts x 32 k (two float4 per thread)
   const int xtok = tid >> 2, xkk = (tid & 3) * 8;
   uint4 xr = make_uint4(0, 0, 0, 0);
-  float4 wr[4];
+  float4 wr[2];
   auto load_chunk = [&](int kc) {
     const int k0 = kc * GK;
     xr = make_uint4(0, 0, 0, 0);
     if (t0 + xtok < N) xr = *reinterpret_cast<const uint4*>(x + (t0 + xtok) * d + k0 + xkk);
 #pragma unroll
-    for (int r = 0; r < 4; ++r) {
+    for (int r = 0; r < 2; ++r) {
       const int i = tid + 256 * r;
       const int ex = i >> 3, kq = (i & 7) * 4;
       wr[r] = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -78,9 +76,9 @@ __global__ void __launch_bounds__(256, 2) k_gate_partial(const __nv_bfloat16* __
   auto store_chunk = [&](int b) {
     const __nv_bfloat16* h = reinterpret_cast<const __nv_bfloat16*>(&xr);
 #pragma unroll
-    for (int j = 0; j < 8; ++j) xs[b][xkk + j][xtok] = h[j];
+    for (int j = 0; j < 8; ++j) xs[b][xkk + j][xtok] = __bfloat162float(h[j]);
 #pragma unroll
-    for (int r = 0; r < 4; ++r) {
+    for (int r = 0; r < 2; ++r) {
       const int i = tid + 256 * r;
       const int ex = i >> 3, kq = (i & 7) * 4;
       wsm[b][kq + 0][ex] = wr[r].x;
@@ -90,11 +88,9 @@ __global__ void __launch_bounds__(256, 2) k_gate_partial(const __nv_bfloat16* __
     }
   };
 
-  double acc[8][4];
+  double acc[8][2];
 #pragma unroll
-  for (int i = 0; i < 8; ++i)
-#pragma unroll
-    for (int j = 0; j < 4; ++j) acc[i][j] = 0.0;
+  for (int i = 0; i < 8; ++i) acc[i][0] = acc[i][1] = 0.0;
 
   int buf = 0;
   if (kc0 < kc1) {
@@ -105,30 +101,26 @@ __global__ void __launch_bounds__(256, 2) k_gate_partial(const __nv_bfloat16* __
   for (int kc = kc0; kc < kc1; ++kc) {
     const bool more = kc + 1 < kc1;
     if (more) load_chunk(kc + 1);
-    float blk[8][4];
+    float blk[8][2];
 #pragma unroll
-    for (int i = 0; i < 8; ++i)
-#pragma unroll
-      for (int j = 0; j < 4; ++j) blk[i][j] = 0.f;
+    for (int i = 0; i < 8; ++i) blk[i][0] = blk[i][1] = 0.f;
 #pragma unroll 8
     for (int k = 0; k < GK; ++k) {
-      const uint4 a = *reinterpret_cast<const uint4*>(&xs[buf][k][ty * 8]);
-      const float4 b = *reinterpret_cast<const float4*>(&wsm[buf][k][tx * 4]);
-      // bf16 -> fp32 is exact: the 16 bits become the high half of the word
-      const float av[8] = {__uint_as_float(a.x << 16), __uint_as_float(a.x & 0xFFFF0000u),
-                           __uint_as_float(a.y << 16), __uint_as_float(a.y & 0xFFFF0000u),
-                           __uint_as_float(a.z << 16), __uint_as_float(a.z & 0xFFFF0000u),
-                           __uint_as_float(a.w << 16), __uint_as_float(a.w & 0xFFFF0000u)};
-      const float bv[4] = {b.x, b.y, b.z, b.w};
+      const float4 a0 = *reinterpret_cast<const float4*>(&xs[buf][k][ty * 8]);
+      const float4 a1 = *reinterpret_cast<const float4*>(&xs[buf][k][ty * 8 + 4]);
+      const float2 b = *reinterpret_cast<const float2*>(&wsm[buf][k][tx * 2]);
+      const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
 #pragma unroll
-      for (int i = 0; i < 8; ++i)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) blk[i][j] = fmaf(av[i], bv[j], blk[i][j]);
+      for (int i = 0; i < 8; ++i) {
+        blk[i][0] = fmaf(av[i], b.x, blk[i][0]);
+        blk[i][1] = fmaf(av[i], b.y, blk[i][1]);
+      }
     }
 #pragma unroll
-    for (int i = 0; i < 8; ++i)
-#pragma unroll
-      for (int j = 0; j < 4; ++j) acc[i][j] += (double)blk[i][j];
+    for (int i = 0; i < 8; ++i) {
+      acc[i][0] += (double)blk[i][0];
+      acc[i][1] += (double)blk[i][1];
+    }
     if (more) store_chunk(buf ^ 1);
     __syncthreads();
     buf ^= 1;
@@ -138,8 +130,8 @@ __global__ void __launch_bounds__(256, 2) k_gate_partial(const __nv_bfloat16* __
     const int64_t t = t0 + ty * 8 + i;
     if (t >= N) continue;
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int e = e0 + tx * 4 + j;
+    for (int j = 0; j < 2; ++j) {
+      const int e = e0 + tx * 2 + j;
       if (e >= E) continue;
       if (splits == 1) logits[t * E + e] = (float)acc[i][j];
       else part[((int64_t)blockIdx.z * N + t) * E + e] = acc[i][j];
@@ -316,6 +308,7 @@ __global__ void __launch_bounds__(1024) k_select_block(
   if (live) {
     if (part) {
       double a = 0.0;
+#pragma unroll 8
       for (int z = 0; z < splits; ++z) a += part[((int64_t)z * N + t) * E + e];
       L = (float)a;
     } else {
@@ -445,7 +438,7 @@ int route_splits(int64_t N, int E, int d_r) {
   int64_t want = (296 + tiles - 1) / tiles;  // about two CTAs per SM
   int64_t maxs = nk / 4 > 0 ? nk / 4 : 1;    // at least 4 chunks per split
   if (want > maxs) want = maxs;
-  if (want > 64) want = 64;
+  if (want > 32) want = 32;
   if (want < 1) want = 1;
   const int cps = (int)((nk + want - 1) / want);
   return (nk + cps - 1) / cps;

@@ -17,14 +17,9 @@
 //   * pairs with i + k > 4 are dropped; with the digit truncation the logit
 //     error stays below ~2e-8 for unit-variance x and 0.02-scale W, far below
 //     one fp32 ulp of a logit of size 1.
-// Kernels: k_slice_rows cuts W's rows into digit planes in memory (W is small
-// and read by every token tile); k_row_sig takes each token row's scale;
-// k_gate_i8 is persistent over (token tile, expert tile) pairs: TMA brings W's
-// digit planes and the token tile as bf16, eight slicer warps cut the tile's
-// digits into shared memory (so x's digit planes never exist in global
-// memory), and one thread issues the 13 int8 products per k-block
-// (tcgen05.mma kind::i8) into five int32 TMEM accumulators (one per s); the
-// epilogue recombines them in double and rounds once to fp32.
+// k_slice_* cut the rows; k_gate_i8 runs the 13 int8 products per k-block
+// with tcgen05.mma kind::i8 into five int32 TMEM accumulators (one per s) and
+// recombines them in double in its epilogue, rounding once to fp32.
 #include <cuda.h>
 #include <math.h>
 
@@ -42,9 +37,13 @@ constexpr int INT = 96;          // tokens per tile (MMA N)
 constexpr int IKB = 64;          // K bytes per stage (64-byte swizzle rows)
 constexpr int IUK = 32;          // K per tcgen05.mma kind::i8
 constexpr int ISTAGES = 3;
+constexpr int kThreadsI8 = 192;
 
-constexpr int kAStageBytes = PS * IM * IKB;   // 32 KB: W's digit planes
-constexpr int kBStageBytes = PS * INT * IKB;  // 24 KB: the token tile's digit planes
+constexpr int kAStageBytes = PS * IM * IKB;   // 32 KB
+constexpr int kBStageBytes = PS * INT * IKB;  // 24 KB
+constexpr int kStageBytesI8 = kAStageBytes + kBStageBytes;
+constexpr size_t kSmemI8 = (size_t)ISTAGES * kStageBytesI8 + 1024 + 256;
+static_assert(kSmemI8 <= 227 * 1024, "shared memory");
 static_assert(NACC * INT <= 512, "TMEM columns");
 
 // ------------------------------------------------------------------ slicing
@@ -86,6 +85,19 @@ struct Vec<float> {
     b[0] = r.x; b[1] = r.y; b[2] = r.z; b[3] = r.w;
   }
 };
+template <>
+struct Vec<__nv_bfloat16> {
+  static constexpr int n = 8;
+  __device__ static void bits(const uint4 r, uint32_t* b) {
+    const uint32_t w[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      b[2 * i] = w[i] << 16;
+      b[2 * i + 1] = w[i] & 0xFFFF0000u;
+    }
+  }
+};
+
 constexpr int kSliceThreads = 256;
 
 // The largest |v| of one 16-byte vector, as the bits of an fp32 (|v| bits
@@ -186,6 +198,19 @@ __device__ __forceinline__ void planes4_bf16(uint32_t a, uint32_t b, const RowSc
   }
 }
 
+template <>
+__device__ __forceinline__ void store_digits<__nv_bfloat16>(const uint4 r, const RowScale& sc,
+                                                            int8_t* __restrict__ out,
+                                                            int64_t plane, int64_t row, int d,
+                                                            int j) {
+  uint32_t P0[PS], P1[PS];
+  planes4_bf16(r.x, r.y, sc, P0);
+  planes4_bf16(r.z, r.w, sc, P1);
+#pragma unroll
+  for (int p = 0; p < PS; ++p)
+    *reinterpret_cast<uint2*>(out + p * plane + row * d + j) = make_uint2(P0[p], P1[p]);
+}
+
 // One block per row: row maximum -> scale, then the 4 digits of every element
 // (d % 8 == 0).  out: [PS][rows][d] int8.  With R > 0 (rows of at most
 // R * 256 vectors) every thread keeps its R vectors in registers, so the row
@@ -242,50 +267,28 @@ __global__ void __launch_bounds__(kSliceThreads) k_slice_rows(const T* __restric
 
 // Launch with the smallest register tile that holds a row.
 template <typename T>
-cudaError_t launch_slice_rows(const T* v, int64_t rows, int d, int8_t* out, int* sig,
-                              cudaStream_t s) {
+void launch_slice_rows(const T* v, int64_t rows, int d, int8_t* out, int* sig, cudaStream_t s) {
   const int steps = (d + kSliceThreads * Vec<T>::n - 1) / (kSliceThreads * Vec<T>::n);
   const dim3 g((unsigned)rows), b(kSliceThreads);
-  if (steps <= 1) return launch_pdl(k_slice_rows<T, 1>, g, b, 0, s, v, rows, d, out, sig);
-  if (steps <= 2) return launch_pdl(k_slice_rows<T, 2>, g, b, 0, s, v, rows, d, out, sig);
-  if (steps <= 4) return launch_pdl(k_slice_rows<T, 4>, g, b, 0, s, v, rows, d, out, sig);
-  if (steps <= 8) return launch_pdl(k_slice_rows<T, 8>, g, b, 0, s, v, rows, d, out, sig);
-  return launch_pdl(k_slice_rows<T, 0>, g, b, 0, s, v, rows, d, out, sig);
+  if (steps <= 1) k_slice_rows<T, 1><<<g, b, 0, s>>>(v, rows, d, out, sig);
+  else if (steps <= 2) k_slice_rows<T, 2><<<g, b, 0, s>>>(v, rows, d, out, sig);
+  else if (steps <= 4) k_slice_rows<T, 4><<<g, b, 0, s>>>(v, rows, d, out, sig);
+  else if (steps <= 8) k_slice_rows<T, 8><<<g, b, 0, s>>>(v, rows, d, out, sig);
+  else k_slice_rows<T, 0><<<g, b, 0, s>>>(v, rows, d, out, sig);
+  (void)counted(cudaPeekAtLastError());
 }
 
-// Row scale of every token: one warp per row reads it once (16-byte vectors,
-// bf16 maxima in pairs) and writes sig with max|x| < 2^sig (0 for a zero
-// row), exactly as k_slice_rows computes it.
-constexpr int kSigWarps = 8;
-__global__ void __launch_bounds__(32 * kSigWarps) k_row_sig(const __nv_bfloat16* __restrict__ x,
-                                                           int64_t rows, int d,
-                                                           int* __restrict__ sig_out) {
-  pdl_wait();
-  pdl_trigger();
-  const int lane = threadIdx.x & 31;
-  const int64_t row = (int64_t)blockIdx.x * kSigWarps + (threadIdx.x >> 5);
-  if (row >= rows) return;
-  const uint4* src = reinterpret_cast<const uint4*>(x + row * d);
-  const int nv = d / 8;
-  uint32_t mx = 0;
-  int j = lane;
-  for (; j + 96 < nv; j += 128) {  // four loads in flight per lane
-    const uint4 a = src[j], b = src[j + 32], c = src[j + 64], e = src[j + 96];
-    mx = max(mx, max(max(vec_absmax<__nv_bfloat16>(a), vec_absmax<__nv_bfloat16>(b)),
-                     max(vec_absmax<__nv_bfloat16>(c), vec_absmax<__nv_bfloat16>(e))));
-  }
-  for (; j < nv; j += 32) mx = max(mx, vec_absmax<__nv_bfloat16>(src[j]));
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-  if (lane == 0) sig_out[row] = row_sig(__uint_as_float(mx));
-}
+// -------------------------------------------------------------- PTX helpers
+// (the shared ones are in sm100.cuh)
+using sm100::mbar_arrive_expect_tx;
+using sm100::mbar_init;
+using sm100::mbar_wait;
+using sm100::smem_u32;
+using sm100::tc_fence_after;
+using sm100::tc_fence_before;
+using sm100::tma_load_3d;
+using sm100::umma_commit;
 
-// ------------------------------------------------------------ the GEMM
-// s8 x s8 -> s32, both K-major, M = 128.
-__device__ __forceinline__ uint32_t idesc_i8(int n) {
-  return (2u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) |
-         ((uint32_t)(IM >> 4) << 24);
-}
 __device__ __forceinline__ void umma_i8(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc,
                                         uint32_t acc) {
   asm volatile(
@@ -294,238 +297,139 @@ __device__ __forceinline__ void umma_i8(uint32_t d, uint64_t a, uint64_t b, uint
       "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(d),
       "l"(a), "l"(b), "r"(idesc), "r"(acc));
 }
-// K-major int8 operand in the 64-byte swizzle: rows of 64 bytes, 8-row groups
-// 512 bytes apart.
+// 32 lanes x 16 consecutive int32 TMEM columns
+__device__ __forceinline__ void tld16(uint32_t taddr, int32_t* v) {
+  uint32_t r[16];
+  sm100::tmem_ld16(taddr, r);
+#pragma unroll
+  for (int i = 0; i < 16; ++i) v[i] = (int32_t)r[i];
+}
+// K-major operand in 64-byte swizzle: rows of 64 bytes, 8-row groups 512 B apart.
 __device__ __forceinline__ uint64_t sw64_desc(uint32_t saddr) {
   return sm100::smem_desc(saddr, 512, 4);
 }
-// Byte offset of columns 8c .. 8c+7 of row r in a 64-byte-swizzled plane:
-// 16-byte unit g of a row sits at unit g ^ ((r >> 1) & 3) (the swizzle
-// repeats every 8 rows = 512 bytes).
-__device__ __forceinline__ uint32_t sw64_off(int r, int c) {
-  return (uint32_t)r * IKB + ((((uint32_t)c >> 1) ^ (((uint32_t)r >> 1) & 3u)) << 4) +
-         ((uint32_t)c & 1u) * 8u;
+// s8 x s8 -> s32, both K-major, M = 128.
+__device__ __forceinline__ uint32_t idesc_i8(int n) {
+  return (2u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) |
+         ((uint32_t)(IM >> 4) << 24);
 }
 
-// Persistent over tiles u = blockIdx.x, +gridDim.x, ...: token tile u / ET,
-// expert tile u % ET (the expert tiles of one token tile run side by side, so
-// its rows are read from L2 after the first).  Roles:
-//   warp 0        TMA: W digit planes (4 x 128 rows x 64 B) and the token
-//                 tile (96 rows x 64 bf16, zero rows past N) per k-block,
-//                 both on tma_full[stage];
-//   warp 1        TMEM owner; one thread issues the MMAs of a k-block once
-//                 the slicers have filled it (full[stage]) and frees the
-//                 stage by a commit to empty[stage];
-//   warps 2-5     epilogue: the five accumulators of a tile -> logits;
-//   warps 6-13    slicers: the token tile's digits into the stage's B planes
-//                 (each thread: rows r, r+32, r+64, one 16-byte column chunk).
-// One TMEM buffer (5 x 96 of 512 columns): the next tile's MMAs wait for the
-// epilogue (tfull / tempty).  Every wait is bounded; a wait that runs out
-// records MOE_ERR_DEVICE_TIMEOUT and the roles stop; the producer then waits
-// (bounded) for the copies it issued, and TMEM is freed before the CTA exits.
-constexpr int kSliceWarpsI8 = 8;
-constexpr int kThreadsI8 = 32 * (6 + kSliceWarpsI8);
-constexpr int kXStageRaw = INT * IKB * 2;  // the token tile as bf16, 128-byte rows
-constexpr int kStageBytesI8 = kAStageBytes + kBStageBytes + kXStageRaw;
-constexpr size_t kSmemI8 = (size_t)ISTAGES * kStageBytesI8 + 1024 + 256;
-static_assert(kSmemI8 <= 227 * 1024, "shared memory");
-static_assert(kStageBytesI8 % 1024 == 0, "stage alignment");
-static_assert(kSliceWarpsI8 * 32 * 3 == INT * 8, "slicer threads: 3 row chunks each");
-
+// One 128-expert x 96-token tile per CTA.  Warp 0: TMA producer; warp 1: MMA
+// issuer and TMEM owner; warps 2-5: epilogue.
 __global__ void __launch_bounds__(kThreadsI8, 1)
     k_gate_i8(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
               const int* __restrict__ sig_w, const int* __restrict__ sig_x, int64_t N, int E,
               int d, float* __restrict__ logits, DeviceStatus* st) {
-  using namespace sm100;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* tma_full = reinterpret_cast<uint64_t*>(smem + ISTAGES * kStageBytesI8);
-  uint64_t* full = tma_full + ISTAGES;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + ISTAGES * kStageBytesI8);
   uint64_t* empty = full + ISTAGES;
   uint64_t* tfull = empty + ISTAGES;
-  uint64_t* tempty = tfull + 1;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + 1);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tfull + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int ET = (E + IM - 1) / IM;
-  const int64_t tiles = (int64_t)ET * ((N + INT - 1) / INT);
+  const int e0 = blockIdx.x * IM;
+  const int64_t t0 = (int64_t)blockIdx.y * INT;
   const int KB = d / IKB;
-  // W's digit planes and the row scales come from the two kernels before
-  pdl_wait();
-  pdl_trigger();
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < ISTAGES; ++s) {
-      mbar_init(&tma_full[s], 1);
-      mbar_init(&full[s], kSliceWarpsI8);
+      mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
     mbar_init(tfull, 1);
-    mbar_init(tempty, 128);
     *abort_flag = 0;
-    mbar_init_fence();
+    sm100::mbar_init_fence();
   }
-  if (warp == 1) tmem_alloc(tmem_slot, 512);
+  if (warp == 1) {
+    sm100::tmem_alloc(tmem_slot, 512);
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
   if (warp == 0) {
-    // ------------------------------------------------------------ producer
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
-      int64_t issued = 0;
-      bool ok = true;
-      for (int64_t u = blockIdx.x; u < tiles && ok; u += gridDim.x) {
-        const int e0 = (int)(u % ET) * IM;
-        const int t0 = (int)(u / ET) * INT;
-        for (int kb = 0; kb < KB; ++kb) {
-          if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag)) { ok = false; break; }
-          uint8_t* sA = smem + stage * kStageBytesI8;
-          uint8_t* sRaw = sA + kAStageBytes + kBStageBytes;
-          mbar_arrive_expect_tx(&tma_full[stage], kAStageBytes + kXStageRaw);
-#pragma unroll
-          for (int p = 0; p < PS; ++p)
-            tma_load_3d(&tmW, &tma_full[stage], sA + p * IM * IKB, kb * IKB, e0, p);
-          tma_load_2d(&tmX, &tma_full[stage], sRaw, kb * IKB, t0);
-          ++issued;
-          if (++stage == ISTAGES) { stage = 0; phase ^= 1; }
+      for (int kb = 0; kb < KB; ++kb) {
+        if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag)) {
+          record_error(st, MOE_ERR_DEVICE_TIMEOUT, 300);
+          *abort_flag = 1;
+          break;
         }
+        uint8_t* sA = smem + stage * kStageBytesI8;
+        uint8_t* sB = sA + kAStageBytes;
+        mbar_arrive_expect_tx(&full[stage], kStageBytesI8);
+#pragma unroll
+        for (int p = 0; p < PS; ++p) {
+          tma_load_3d(&tmW, &full[stage], sA + p * IM * IKB, kb * IKB, e0, p);
+          tma_load_3d(&tmX, &full[stage], sB + p * INT * IKB, kb * IKB, (int)t0, p);
+        }
+        if (++stage == ISTAGES) { stage = 0; phase ^= 1; }
       }
-      if (!ok) {
-        record_error(st, MOE_ERR_DEVICE_TIMEOUT, 300);
-        *abort_flag = 1;
-      }
-      // no copy of this CTA may still be in flight when it exits
-      volatile int never = 0;
-      for (int64_t k = issued - 1; k >= 0 && k >= issued - ISTAGES; --k)
-        if (!mbar_wait(&tma_full[k % ISTAGES], (uint32_t)((k / ISTAGES) & 1), &never))
-          record_error(st, MOE_ERR_DEVICE_TIMEOUT, 301);
     }
   } else if (warp == 1) {
-    // ---------------------------------------------------------- MMA issuer
     if (lane == 0) {
       const uint32_t idesc = idesc_i8(INT);
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
-      int local = 0;
-      for (int64_t u = blockIdx.x; u < tiles && ok; u += gridDim.x, ++local) {
-        if (!mbar_wait(tempty, (local & 1) ^ 1, abort_flag)) { ok = false; break; }
+      for (int kb = 0; kb < KB; ++kb) {
+        if (!mbar_wait(&full[stage], phase, abort_flag)) { ok = false; break; }
         tc_fence_after();
-        for (int kb = 0; kb < KB; ++kb) {
-          if (!mbar_wait(&full[stage], phase, abort_flag)) { ok = false; break; }
-          tc_fence_after();
-          const uint32_t a0 = smem_u32(smem + stage * kStageBytesI8);
-          const uint32_t b0 = a0 + kAStageBytes;
-          // digit pairs (i of x, k of W), grouped by s = i + k
+        const uint32_t a0 = smem_u32(smem + stage * kStageBytesI8);
+        const uint32_t b0 = a0 + kAStageBytes;
+        // digit pairs (i of x, k of W), grouped by s = i + k
 #pragma unroll
-          for (int s = 0; s <= SMAX; ++s) {
-            bool first = kb == 0;
+        for (int s = 0; s <= SMAX; ++s) {
+          bool first = kb == 0;
 #pragma unroll
-            for (int i = 0; i < PS; ++i) {
-              const int k = s - i;
-              if (k < 0 || k >= PS) continue;
+          for (int i = 0; i < PS; ++i) {
+            const int k = s - i;
+            if (k < 0 || k >= PS) continue;
 #pragma unroll
-              for (int h = 0; h < IKB / IUK; ++h) {
-                umma_i8(tmem + s * INT, sw64_desc(a0 + k * IM * IKB + h * IUK),
-                        sw64_desc(b0 + i * INT * IKB + h * IUK), idesc, first ? 0u : 1u);
-                first = false;
-              }
+            for (int h = 0; h < IKB / IUK; ++h) {
+              umma_i8(tmem + s * INT, sw64_desc(a0 + k * IM * IKB + h * IUK),
+                      sw64_desc(b0 + i * INT * IKB + h * IUK), idesc, first ? 0u : 1u);
+              first = false;
             }
           }
-          umma_commit(&empty[stage]);
-          if (++stage == ISTAGES) { stage = 0; phase ^= 1; }
         }
-        if (ok) umma_commit(tfull);
+        umma_commit(&empty[stage]);
+        if (++stage == ISTAGES) { stage = 0; phase ^= 1; }
       }
-      if (!ok) {
+      if (ok) umma_commit(tfull);
+      else {
         record_error(st, MOE_ERR_DEVICE_TIMEOUT, 310);
         *abort_flag = 1;
       }
     }
-  } else if (warp < 6) {
-    // ------------------------------------------------------------ epilogue
-    const int quarter = warp & 3;  // TMEM lanes 32 * quarter .. + 31
-    const int el = quarter * 32 + lane;
-    int local = 0;
-    for (int64_t u = blockIdx.x; u < tiles; u += gridDim.x, ++local) {
-      const int e = (int)(u % ET) * IM + el;
-      const int64_t t0 = (u / ET) * INT;
-      if (!mbar_wait(tfull, local & 1, abort_flag)) {
-        if (lane == 0) record_error(st, MOE_ERR_DEVICE_TIMEOUT, 320);
-        *abort_flag = 1;
-        break;
-      }
+  } else {
+    const int quarter = warp & 3;
+    const int e = e0 + quarter * 32 + lane;
+    if (mbar_wait(tfull, 0, abort_flag)) {
       tc_fence_after();
       const uint32_t taddr = tmem + ((uint32_t)(quarter * 32) << 16);
       const int sw = e < E ? sig_w[e] : 0;
       for (int c0 = 0; c0 < INT; c0 += 16) {
-        // v = sum_s 2^(-7s) S_s by Horner from s = NACC - 1 down (exact in
-        // double: every step is a power-of-two scaling and a 31-bit add)
-        double v[16];
-        uint32_t a[16];
-        tmem_ld16(taddr + (NACC - 1) * INT + c0, a);
+        int32_t acc[NACC][16];
 #pragma unroll
-        for (int j = 0; j < 16; ++j) v[j] = (double)(int32_t)a[j];
-#pragma unroll
-        for (int s = NACC - 2; s >= 0; --s) {
-          tmem_ld16(taddr + s * INT + c0, a);
-#pragma unroll
-          for (int j = 0; j < 16; ++j) v[j] = v[j] * 0x1p-7 + (double)(int32_t)a[j];
-        }
+        for (int s = 0; s < NACC; ++s) tld16(taddr + s * INT + c0, acc[s]);
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
           const int64_t t = t0 + c0 + j;
-          if (t < N && e < E) logits[t * E + e] = (float)ldexp(v[j], sig_x[t] + sw - 14);
+          if (t >= N || e >= E) continue;
+          double v = 0.0;
+#pragma unroll
+          for (int s = NACC - 1; s >= 0; --s) v = v * 0x1p-7 + (double)acc[s][j];
+          logits[t * E + e] = (float)ldexp(v, sig_x[t] + sw - 14);
         }
       }
-      tc_fence_before();
-      mbar_arrive(tempty);
-    }
-  } else {
-    // ------------------------------------------------------------- slicers
-    const int ts = threadIdx.x - 192;  // 0 .. 255
-    const int c = ts & 7;              // 16-byte chunk of the 128-byte bf16 row
-    const int r0 = ts >> 3;            // rows r0, r0 + 32, r0 + 64
-    int stage = 0;
-    uint32_t phase = 0;
-    bool ok = true;
-    for (int64_t u = blockIdx.x; u < tiles && ok; u += gridDim.x) {
-      const int64_t t0 = (u / ET) * INT;
-      RowScale sc[3];
-#pragma unroll
-      for (int j = 0; j < 3; ++j) {
-        const int64_t t = t0 + r0 + 32 * j;
-        sc[j] = row_scale(t < N ? sig_x[t] : 0);
-      }
-      for (int kb = 0; kb < KB; ++kb) {
-        if (!mbar_wait(&tma_full[stage], phase, abort_flag)) { ok = false; break; }
-        uint8_t* sB = smem + stage * kStageBytesI8 + kAStageBytes;
-        const uint8_t* sRaw = sB + kBStageBytes;
-#pragma unroll
-        for (int j = 0; j < 3; ++j) {
-          const int r = r0 + 32 * j;
-          const uint4 v = *reinterpret_cast<const uint4*>(sRaw + r * (IKB * 2) + c * 16);
-          uint32_t P0[PS], P1[PS];
-          planes4_bf16(v.x, v.y, sc[j], P0);
-          planes4_bf16(v.z, v.w, sc[j], P1);
-          const uint32_t off = sw64_off(r, c);
-#pragma unroll
-          for (int p = 0; p < PS; ++p)
-            *reinterpret_cast<uint2*>(sB + p * INT * IKB + off) = make_uint2(P0[p], P1[p]);
-        }
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&full[stage]);
-        if (++stage == ISTAGES) { stage = 0; phase ^= 1; }
-      }
-    }
-    if (!ok) {
-      if (lane == 0) record_error(st, MOE_ERR_DEVICE_TIMEOUT, 330);
+    } else {
+      if (lane == 0) record_error(st, MOE_ERR_DEVICE_TIMEOUT, 320);
       *abort_flag = 1;
     }
   }
@@ -534,7 +438,7 @@ __global__ void __launch_bounds__(kThreadsI8, 1)
   if (warp == 1) {
     __syncwarp();
     tc_fence_after();
-    tmem_dealloc(tmem, 512);
+    sm100::tmem_dealloc(tmem, 512);
   }
 }
 
@@ -569,23 +473,8 @@ bool map_planes(CUtensorMap* m, const void* base, uint64_t d, uint64_t rows, uin
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// x [rows][d] bf16, box 64 columns x box_rows, no swizzle (128-byte rows);
-// rows past the end read as zero
-bool map_rows_bf16(CUtensorMap* m, const void* base, uint64_t d, uint64_t rows,
-                   uint32_t box_rows) {
-  EncodeTiledFnI8 fn = encode_i8();
-  if (!fn) return false;
-  cuuint64_t dims[2] = {d, rows};
-  cuuint64_t strides[1] = {d * 2};
-  cuuint32_t box[2] = {(cuuint32_t)IKB, box_rows};
-  cuuint32_t es[2] = {1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
-            es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 struct I8Layout {
-  size_t logits, wd, ws, xs, total;
+  size_t logits, wd, ws, xd, xs, total;
 };
 
 I8Layout i8_layout(int64_t N, int E, int d) {
@@ -594,6 +483,7 @@ I8Layout i8_layout(int64_t N, int E, int d) {
   L.logits = o; o += align_up(sizeof(float) * (size_t)N * E, 256);
   L.wd = o; o += align_up((size_t)PS * E * d, 256);
   L.ws = o; o += align_up(sizeof(int) * (size_t)E, 256);
+  L.xd = o; o += align_up((size_t)PS * N * d, 256);
   L.xs = o; o += align_up(sizeof(int) * (size_t)N, 256);
   L.total = o;
   return L;
@@ -615,9 +505,12 @@ cudaError_t launch_gate_i8(const __nv_bfloat16* x, int64_t N, int d_r, const flo
   float* logits = reinterpret_cast<float*>(base + L.logits);
   int8_t* wd = reinterpret_cast<int8_t*>(base + L.wd);
   int* wsig = reinterpret_cast<int*>(base + L.ws);
+  int8_t* xd = reinterpret_cast<int8_t*>(base + L.xd);
   int* xsig = reinterpret_cast<int*>(base + L.xs);
+  launch_slice_rows(W, E, d_r, wd, wsig, s);
+  launch_slice_rows(x, N, d_r, xd, xsig, s);
   CUtensorMap mw, mx;
-  if (!map_planes(&mw, wd, d_r, E, IM) || !map_rows_bf16(&mx, x, d_r, N, INT))
+  if (!map_planes(&mw, wd, d_r, E, IM) || !map_planes(&mx, xd, d_r, N, INT))
     return cudaErrorInvalidValue;
   static std::once_flag once[kMaxDevices];
   static cudaError_t set_up[kMaxDevices];
@@ -626,15 +519,9 @@ cudaError_t launch_gate_i8(const __nv_bfloat16* x, int64_t N, int d_r, const flo
                                 (int)kSmemI8);
   });
   if (e0 != cudaSuccess) return e0;
-  cudaError_t e = launch_slice_rows(W, E, d_r, wd, wsig, s);
-  if (e != cudaSuccess) return e;
-  e = launch_pdl(k_row_sig, dim3((unsigned)((N + kSigWarps - 1) / kSigWarps)),
-                 dim3(32 * kSigWarps), 0, s, x, N, d_r, xsig);
-  if (e != cudaSuccess) return e;
-  const int64_t tiles = (int64_t)((E + IM - 1) / IM) * ((N + INT - 1) / INT);
-  const int64_t grid = tiles < dev_info()->sm_count ? tiles : dev_info()->sm_count;
-  return launch_pdl(k_gate_i8, dim3((unsigned)grid), dim3(kThreadsI8), kSmemI8, s, mw, mx,
-                    (const int*)wsig, (const int*)xsig, N, E, d_r, logits, st);
+  dim3 grid((E + IM - 1) / IM, (unsigned)((N + INT - 1) / INT), 1);
+  k_gate_i8<<<grid, kThreadsI8, kSmemI8, s>>>(mw, mx, wsig, xsig, N, E, d_r, logits, st);
+  return counted(cudaGetLastError(), 3);  // the two slicers and the GEMM
 }
 
 }  // namespace moe
