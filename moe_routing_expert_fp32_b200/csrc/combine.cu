@@ -91,6 +91,94 @@ __global__ void __launch_bounds__(32 * kWarps) k_combine(const __nv_bfloat16* __
   }
 }
 
+// The same combine with every lane issuing the loads of all KK = K rows of
+// its 16-byte column before it sums any of them, so each warp has K loads in
+// flight instead of one.  Row k of token t is pos[t*K + k] (the sorted y), or
+// t*K + k when pos is NULL (y in slot order, as moe_expert_ffn_to_slots
+// writes it).  Rows are skipped and reported exactly as in k_combine, and the
+// arithmetic is k_combine's (products rounded to fp32, summed in k order), so
+// the result is the same bits.  KK is 4, 8 or 16.
+template <int KK>
+__global__ void __launch_bounds__(32 * kWarps) k_combine_rows(
+    const __nv_bfloat16* __restrict__ y, const int32_t* __restrict__ pos,
+    const float* __restrict__ w, int64_t N, int d, int64_t S, __nv_bfloat16* __restrict__ out,
+    const __nv_bfloat16* __restrict__ res, DeviceStatus* st) {
+  pdl_wait();
+  pdl_trigger();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nv = d / 8;
+  const int nch = (nv + 31) / 32;
+  const int64_t items = N * nch;
+  for (int64_t it = (int64_t)blockIdx.x * kWarps + warp; it < items;
+       it += (int64_t)gridDim.x * kWarps) {
+    const int64_t t = it / nch;
+    const int v = (int)(it - t * nch) * 32 + lane;
+    // the K rows and weights go to every lane before any lane leaves the item
+    int my_p = -1;
+    float my_w = 0.f;
+    if (lane < KK) {
+      my_p = pos ? pos[t * KK + lane] : (int)(t * KK + lane);
+      my_w = w[t * KK + lane];
+      if (my_p < 0 || my_p >= S) {
+        record_error(st, MOE_ERR_DEVICE_BOUNDS, 41);
+        my_p = -1;
+      }
+    }
+    int rk[KK];
+    float wks[KK];
+#pragma unroll
+    for (int k = 0; k < KK; ++k) {
+      rk[k] = __shfl_sync(0xffffffffu, my_p, k);
+      wks[k] = __shfl_sync(0xffffffffu, my_w, k);
+    }
+    if (v >= nv) continue;
+    uint4 raw[KK];
+#pragma unroll
+    for (int k = 0; k < KK; ++k)
+      raw[k] = rk[k] >= 0 ? reinterpret_cast<const uint4*>(y + (int64_t)rk[k] * d)[v]
+                          : make_uint4(0, 0, 0, 0);
+    float acc[8];
+    bool have = false;
+#pragma unroll
+    for (int k = 0; k < KK; ++k) {
+      if (rk[k] < 0) continue;
+      const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&raw[k]);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float2 f = __bfloat1622float2(h2[j]);
+        const float p0 = __fmul_rn(f.x, wks[k]), p1 = __fmul_rn(f.y, wks[k]);
+        if (have) {
+          acc[2 * j] = __fadd_rn(acc[2 * j], p0);
+          acc[2 * j + 1] = __fadd_rn(acc[2 * j + 1], p1);
+        } else {
+          acc[2 * j] = p0;
+          acc[2 * j + 1] = p1;
+        }
+      }
+      have = true;
+    }
+    if (!have) {
+#pragma unroll
+      for (int j = 0; j < 8; ++j) acc[j] = 0.f;
+    }
+    if (res) {
+      const uint4 rr = reinterpret_cast<const uint4*>(res + t * d)[v];
+      const __nv_bfloat162* r2 = reinterpret_cast<const __nv_bfloat162*>(&rr);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float2 f = __bfloat1622float2(r2[j]);
+        acc[2 * j] = __fadd_rn(__bfloat162float(__float2bfloat16_rn(acc[2 * j])), f.x);
+        acc[2 * j + 1] = __fadd_rn(__bfloat162float(__float2bfloat16_rn(acc[2 * j + 1])), f.y);
+      }
+    }
+    uint4 o;
+    __nv_bfloat162* o2 = reinterpret_cast<__nv_bfloat162*>(&o);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) o2[j] = __floats2bfloat162_rn(acc[2 * j], acc[2 * j + 1]);
+    reinterpret_cast<uint4*>(out + t * d)[v] = o;
+  }
+}
+
 // ------------------------------------------------------------------ RMSNorm
 // routed_expert_norm of the latent block, read as an RMSNorm: per row
 // r = 1/sqrt(mean(x^2) + eps) in double, n = bf16(x*r) (one rounding from
@@ -242,6 +330,14 @@ cudaError_t launch_combine(const __nv_bfloat16* y, const int32_t* pos, const flo
   int64_t blocks = (items + kWarps - 1) / kWarps;
   const int64_t cap = (int64_t)dev_info()->sm_count * 16;
   if (blocks > cap) blocks = cap;
+  if (K == 4 || K == 8 || K == 16) {  // all K loads of a column in flight together
+    const dim3 g((unsigned)blocks), b(32 * kWarps);
+    if (K == 4)
+      return launch_pdl(k_combine_rows<4>, g, b, 0, s, y, pos, w, N, d_e, S, out, residual, st);
+    if (K == 8)
+      return launch_pdl(k_combine_rows<8>, g, b, 0, s, y, pos, w, N, d_e, S, out, residual, st);
+    return launch_pdl(k_combine_rows<16>, g, b, 0, s, y, pos, w, N, d_e, S, out, residual, st);
+  }
   return launch_pdl(k_combine, dim3((unsigned)blocks), dim3(32 * kWarps), 0, s, y, pos, w, N, K,
                     d_e, S, out, residual, st);
 }
