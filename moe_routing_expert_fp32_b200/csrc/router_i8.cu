@@ -521,7 +521,7 @@ cudaError_t launch_gate_i8(const __nv_bfloat16* x, int64_t N, int d_r, const flo
   if (e0 != cudaSuccess) return e0;
   dim3 grid((E + IM - 1) / IM, (unsigned)((N + INT - 1) / INT), 1);
   k_gate_i8<<<grid, kThreadsI8, kSmemI8, s>>>(mw, mx, wsig, xsig, N, E, d_r, logits, st);
-  return counted(cudaGetLastError(), 3);  // the two slicers and the GEMM
+  return counted(cudaGetLastError());  // the GEMM (each slicer launch was counted above)
 }
 
 }  // namespace moe

@@ -48,3 +48,23 @@ def test_launch_count_of_forward_is_stable():
     torch.cuda.synchronize()
     # route (gate GEMM + selection), dispatch (4), tile list, two expert GEMMs, combine
     assert deltas[0] == deltas[1] == deltas[2] and 10 <= deltas[0] <= 13
+
+
+def test_launch_count_of_route_on_both_gate_paths():
+    """moe_route launches: the fp32 gate GEMM and the selection for a decode
+    batch (the split-K partials are summed by the selection, no reduce
+    kernel); the two slicers, the int8 gate GEMM and the selection once the
+    batch fills the int8 tiles (here 25 tiles of 128 experts x 96 tokens)."""
+    import torch
+    import moe_routing_expert_fp32_b200 as moe
+    for (N, E, d, want) in [(128, 256, 7168, 2), (2400, 128, 64, 4)]:
+        x = synth.dev_normal_bf16(torch.empty((N, d), dtype=torch.bfloat16, device="cuda"), 1, 1,
+                                  1.0)
+        W = synth.dev_normal_f32(torch.empty((E, d), dtype=torch.float32, device="cuda"), 1, 2,
+                                 0.02)
+        cfg = moe.RouteConfig(E, 1, 1, 8, 1.0, True)
+        moe.route(x, W, None, cfg)  # kernel attributes set up
+        n0 = moe.launch_count()
+        moe.route(x, W, None, cfg)
+        assert moe.launch_count() - n0 == want, (N, E, d)
+    torch.cuda.synchronize()
