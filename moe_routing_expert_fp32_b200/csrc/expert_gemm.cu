@@ -197,22 +197,30 @@ __device__ __forceinline__ float situ_mul(float g, float u, float beta, float lb
 // offsets[s+1]) uses weights s % emod: emod = E for the layer, E_local for
 // rows received from several ranks, grouped by (source rank, local expert).
 
+// bf16 of (lo, hi) in one word, lo in the low half.
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
+__device__ __forceinline__ float bf16_lo(uint32_t p) { return __uint_as_float(p << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t p) { return __uint_as_float(p & 0xffff0000u); }
+
 // Stores one 16-token chunk of a down-projection accumulator (lane l holds
 // feature m = m8 + (l & 7) of its 8-lane group, v[j] = token c0 + j) as
 // out[token][feature] with 16-byte stores: the 8 x 16 block of each 8-lane
 // group is transposed by shuffles so that lane i holds tokens 2i and 2i+1 of
 // the group's 8 features.  Every lane of the warp must call it.
-__device__ __forceinline__ void store_down_t8(const float* v, __nv_bfloat16* out, int64_t tok0,
-                                              int ntok, int M_rows, int m8, bool live, int lane,
-                                              const int32_t* rowmap = nullptr,
-                                              int64_t map_rows = 0,
-                                              DeviceStatus* st = nullptr) {
+// (store_down_t8_packed takes the chunk already rounded: p[t] = bf16 of
+// tokens 2t, 2t+1.)
+__device__ __forceinline__ void store_down_t8_packed(const uint32_t* p, __nv_bfloat16* out,
+                                                     int64_t tok0, int ntok, int M_rows, int m8,
+                                                     bool live, int lane,
+                                                     const int32_t* rowmap = nullptr,
+                                                     int64_t map_rows = 0,
+                                                     DeviceStatus* st = nullptr) {
   uint32_t a[8];
 #pragma unroll
-  for (int t = 0; t < 8; ++t) {
-    const __nv_bfloat162 h = __floats2bfloat162_rn(v[2 * t], v[2 * t + 1]);
-    a[t] = *reinterpret_cast<const uint32_t*>(&h);
-  }
+  for (int t = 0; t < 8; ++t) a[t] = p[t];
   const int i = lane & 7;
 #pragma unroll
   for (int s = 1; s < 8; s <<= 1) {
@@ -250,6 +258,16 @@ __device__ __forceinline__ void store_down_t8(const float* v, __nv_bfloat16* out
     if (2 * i < ntok && r0 >= 0) *reinterpret_cast<uint4*>(out + r0 * M_rows + m8) = lo;
     if (2 * i + 1 < ntok && r1 >= 0) *reinterpret_cast<uint4*>(out + r1 * M_rows + m8) = hi;
   }
+}
+__device__ __forceinline__ void store_down_t8(const float* v, __nv_bfloat16* out, int64_t tok0,
+                                              int ntok, int M_rows, int m8, bool live, int lane,
+                                              const int32_t* rowmap = nullptr,
+                                              int64_t map_rows = 0,
+                                              DeviceStatus* st = nullptr) {
+  uint32_t p[8];
+#pragma unroll
+  for (int t = 0; t < 8; ++t) p[t] = pack_bf16x2(v[2 * t], v[2 * t + 1]);
+  store_down_t8_packed(p, out, tok0, ntok, M_rows, m8, live, lane, rowmap, map_rows, st);
 }
 
 
@@ -762,14 +780,31 @@ __device__ __forceinline__ uint32_t idesc_bf16_m256(int n) {
 }
 
 constexpr int kPairNt = 256;     // token rows per tile (N, split 128 + 128)
+// Epilogue warps of the CTA-pair kernel: kPairSlices warps per TMEM lane
+// quarter, each copying kPairNt / kPairSlices columns of an accumulator to
+// registers.  With two weight blocks per unit the accumulators fill TMEM and
+// the next unit's MMAs wait for this copy, so it is split over 16 warps; with
+// the 64 TMA / MMA threads that is 576 per CTA (96 registers a thread).
+#ifndef MOE_PAIR_SLICES
+#define MOE_PAIR_SLICES 4
+#endif
+constexpr int kPairSlices = MOE_PAIR_SLICES;
+constexpr int kPairThreads = 64 + 4 * 32 * kPairSlices;  // TMA, MMA, 4 x kPairSlices epilogue
+static_assert(kPairNt % (32 * kPairSlices) == 0, "whole 32-column TMEM loads per slice");
+// gate_up exchange through shared memory: per slice, quarter pair, parity and
+// g/u, one 16-byte word per lane
+constexpr int kPairXchgWords = 32 * 4;  // 32-bit words per entry
 
 // PUM weight blocks of 256 rows (128 per CTA) per unit, all against the same
 // token tile.  PUM = 1: 6 stages of (A 16 KB + B half 16 KB) per CTA, two
 // TMEM accumulator buffers (the epilogue of one unit overlaps the MMAs of the
 // next).  PUM = 2: 4 stages of (A 2 x 16 KB + B half 16 KB): each token byte
-// brought from L2 feeds twice the MMAs; the two 256-column accumulators fill
-// TMEM, so there is one buffer, and the next unit's first-block MMAs run on
-// held stages while the epilogue drains the second accumulator.
+// brought from L2 feeds twice the MMAs, a quarter fewer bytes per MMA, which
+// is what bounds the one-block form (its TMA issue runs flat out while the
+// MMAs wait for data).  The two 256-column accumulators fill TMEM, so there
+// is one buffer: the epilogue copies each accumulator to registers and hands
+// it back before it computes and stores, and the next unit's first-block MMAs
+// run on held stages while the second accumulator is copied.
 template <int PUM>
 struct PairCfg {
   static constexpr int kStages = PUM == 1 ? 6 : 4;
@@ -779,13 +814,14 @@ struct PairCfg {
   static constexpr int kStageBytes = kABytes + kBBytes;
   static constexpr int kBufCols = kPairNt;
   static constexpr int kTmemCols = 2 * kPairNt;
-  static constexpr size_t kSmem = (size_t)kStages * kStageBytes + 1024 + 256 + kXchgBytes;
+  static constexpr int kXchg = kPairSlices * 2 * 2 * 2 * kPairXchgWords * 4;
+  static constexpr size_t kSmem = (size_t)kStages * kStageBytes + 1024 + 256 + kXchg;
   static_assert(kSmem <= 227 * 1024, "shared memory");
   static_assert(PUM == 1 || PUM == 2, "one or two weight blocks per unit");
 };
 
 template <int MODE, int PUM>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kPairThreads, 1)
     k_expert_gemm_pair(const __grid_constant__ CUtensorMap tmA0,
                        const __grid_constant__ CUtensorMap tmA1,
                        const __grid_constant__ CUtensorMap tmB,
@@ -831,7 +867,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&tfull[b], 1);
-      mbar_init(&tempty[b], 256);
+      mbar_init(&tempty[b], 2 * (kPairThreads - 64));  // every epilogue thread of the pair
     }
     mbar_init(never, 1);
     *abort_flag = 0;
@@ -1006,7 +1042,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ------------------------------------------------------ epilogue (both CTAs)
-    const int quarter = warp & 3;
+    // Each warp copies its share of an accumulator (the TMEM lanes of its
+    // quarter, the columns of its slice) to registers, rounded to bf16 in
+    // pairs as every output of the kernel is rounded first, and hands the
+    // accumulator back at once: the MMAs of the next unit then wait only for
+    // the copy, and the exchange, activation and stores overlap them.  (The
+    // residual form keeps fp32 to the end and drains in place.)
+    constexpr int kSliceCols = kPairNt / kPairSlices;
+    constexpr int kChunks = kSliceCols / 16;
+    const int quarter = warp & 3;       // TMEM lanes 32 * quarter .. + 31
+    const int slice = (warp - 2) >> 2;  // TMEM columns col0 .. col0 + kSliceCols - 1
+    const int col0 = slice * kSliceCols;
     const bool has_lb = !(lbeta == 0.0f || lbeta != lbeta);
     const float b_eff = (beta == 0.0f || beta != beta) ? 1.0f : beta;
     const uint32_t tempty_leader0 = peer_addr(smem_u32(&tempty[0]), 0);
@@ -1015,71 +1061,121 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool stop = false;
     for (int64_t u = pair_id; u < total_units && !stop; u += npairs, ++local) {
       const Unit w = decode_unit(u, RB, kPairNt, tile_start, offsets, E, emod);
+      if (MODE == kDown && res) {
+        for (int a = 0; a < PUM; ++a) {
+          const int buf = PUM == 1 ? (local & 1) : a;
+          const uint32_t tphase = PUM == 1 ? ((local >> 1) & 1) : (local & 1);
+          if (!mbar_wait(&tfull[buf], tphase, abort_flag)) {
+            if (lane == 0) record_error(st, MOE_ERR_DEVICE_TIMEOUT, 220 + MODE);
+            *abort_flag = 1;
+            stop = true;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + buf * C::kBufCols;
+          const int m = w.rb * unit_rows + a * 2 * blk_rows + rank * blk_rows + quarter * 32 + lane;
+          __nv_bfloat16* col = out + m;
+          const int lim_m = m < M_rows ? 16 : 0;
+          for (int c0 = col0; c0 < w.nrows && c0 < col0 + kSliceCols; c0 += 16) {
+            float v[16];
+            tmem_ld16(taddr + c0, v);
+            int lim = w.nrows - c0 < 16 ? w.nrows - c0 : 16;
+            lim = lim < lim_m ? lim : lim_m;
+#pragma unroll
+            for (int j = 0; j < 16; ++j)
+              if (j < lim)
+                col[(int64_t)(w.row0 + c0 + j) * M_rows] =
+                    down_out(v[j], res, w.row0 + c0 + j, M_rows, m);
+          }
+          tc_fence_before();
+          mbar_arrive_remote(tempty_leader0 + buf * (uint32_t)sizeof(uint64_t));
+        }
+        continue;
+      }
+      // pk[a][8 * ci + t]: block a, chunk ci (columns col0 + 16 ci ..), tokens
+      // 2t and 2t + 1 of the chunk
+      uint32_t pk[PUM][kSliceCols / 2];
+#pragma unroll
       for (int a = 0; a < PUM; ++a) {
-      const int buf = PUM == 1 ? (local & 1) : a;
-      const uint32_t tphase = PUM == 1 ? ((local >> 1) & 1) : (local & 1);
-      if (!mbar_wait(&tfull[buf], tphase, abort_flag)) {
-        if (lane == 0) record_error(st, MOE_ERR_DEVICE_TIMEOUT, 220 + MODE);
-        *abort_flag = 1;
-        stop = true;
-        break;
-      }
-      tc_fence_after();
-      const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + buf * C::kBufCols;
-      const int r0 = w.rb * unit_rows + a * 2 * blk_rows + rank * blk_rows;
-      if (MODE == kGateUp) {
-        const int pair = quarter & 1;
-        const bool is_g = quarter < 2;
-        const int f = r0 + pair * 32 + lane;
-        const bool live = f < M_rows;
-        for (int c0 = 0; c0 < w.nrows; c0 += 16, ++xbuf) {
-          float v[16];
-          tmem_ld16(taddr + c0, v);
-          float* xg = xchg + ((pair * 2 + (xbuf & 1)) * 2 + 0) * 256;
-          float* xu = xchg + ((pair * 2 + (xbuf & 1)) * 2 + 1) * 256;
-          float4* mine = reinterpret_cast<float4*>((is_g ? xg : xu) + lane * 8);
-          const float* give = is_g ? v + 8 : v;
-          mine[0] = make_float4(give[0], give[1], give[2], give[3]);
-          mine[1] = make_float4(give[4], give[5], give[6], give[7]);
-          asm volatile("bar.sync %0, 64;" ::"r"(1 + pair) : "memory");
-          const float4* theirs = reinterpret_cast<const float4*>((is_g ? xu : xg) + lane * 8);
-          const float4 t0 = theirs[0], t1 = theirs[1];
-          const float other[8] = {t0.x, t0.y, t0.z, t0.w, t1.x, t1.y, t1.z, t1.w};
-          const int cbase = c0 + (is_g ? 0 : 8);
-          float hv[8];
-#pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            const float g = is_g ? v[j] : other[j];
-            const float uu = is_g ? other[j] : v[8 + j];
-            hv[j] = act_kind == MOE_ACT_SITU ? situ_mul(g, uu, b_eff, lbeta, has_lb)
-                                             : silu_mul(g, uu);
-          }
-          store_h_t8(hv, out, w.row0 + cbase, w.nrows - cbase, M_rows, f & ~7, live, lane);
+        const int buf = PUM == 1 ? (local & 1) : a;
+        const uint32_t tphase = PUM == 1 ? ((local >> 1) & 1) : (local & 1);
+        if (!mbar_wait(&tfull[buf], tphase, abort_flag)) {
+          if (lane == 0) record_error(st, MOE_ERR_DEVICE_TIMEOUT, 220 + MODE);
+          *abort_flag = 1;
+          stop = true;
+          break;
         }
-      } else {
-        const int m = r0 + quarter * 32 + lane;
-        __nv_bfloat16* col = out + m;
-        const int lim_m = m < M_rows ? 16 : 0;
-        for (int c0 = 0; c0 < w.nrows; c0 += 16) {
-          float v[16];
-          tmem_ld16(taddr + c0, v);
-          int lim = w.nrows - c0 < 16 ? w.nrows - c0 : 16;
-          if (!res) {
-            store_down_t8(v, out, w.row0 + c0, lim, M_rows, m & ~7, lim_m != 0, lane, yrow,
-                          yrow ? (int64_t)offsets[E] : 0, st);
-            continue;
-          }
-          lim = lim < lim_m ? lim : lim_m;
+        tc_fence_after();
+        const uint32_t taddr =
+            tmem_base + ((uint32_t)(quarter * 32) << 16) + buf * C::kBufCols + col0;
+        if (col0 < w.nrows) {
 #pragma unroll
-          for (int j = 0; j < 16; ++j)
-            if (j < lim) col[(int64_t)(w.row0 + c0 + j) * M_rows] = down_out(v[j], res, w.row0 + c0 + j, M_rows, m);
+          for (int q = 0; q < kSliceCols / 32; ++q) {
+            uint32_t r[32];
+            sm100::tmem_ld32(taddr + 32 * q, r);
+#pragma unroll
+            for (int t = 0; t < 16; ++t)
+              pk[a][16 * q + t] =
+                  pack_bf16x2(__uint_as_float(r[2 * t]), __uint_as_float(r[2 * t + 1]));
+          }
+        }
+        tc_fence_before();
+        // the accumulator (buffer, or block) goes back to the even CTA's MMA issuer
+        mbar_arrive_remote(tempty_leader0 + buf * (uint32_t)sizeof(uint64_t));
+      }
+      if (stop) break;
+#pragma unroll
+      for (int a = 0; a < PUM; ++a) {
+        const int r0 = w.rb * unit_rows + a * 2 * blk_rows + rank * blk_rows;
+        if (MODE == kGateUp) {
+          // lanes 0-63 of the block hold g (w1 rows), 64-127 u (w3 rows) of the
+          // same 64 features: quarters q and q + 2 swap half of each chunk, so
+          // the g quarter forms h for the chunk's first 8 tokens, the u quarter
+          // for the last 8
+          const int pair = quarter & 1;
+          const bool is_g = quarter < 2;
+          const int f = r0 + pair * 32 + lane;
+          const bool live = f < M_rows;
+#pragma unroll
+          for (int ci = 0; ci < kChunks; ++ci) {
+            const int c0 = col0 + 16 * ci;
+            if (c0 >= w.nrows) break;
+            const uint32_t* p = &pk[a][8 * ci];
+            const int xe = ((slice * 2 + pair) * 2 + (xbuf & 1)) * 2;
+            uint4* xg = reinterpret_cast<uint4*>(xchg + (xe + 0) * kPairXchgWords);
+            uint4* xu = reinterpret_cast<uint4*>(xchg + (xe + 1) * kPairXchgWords);
+            (is_g ? xg : xu)[lane] =
+                is_g ? make_uint4(p[4], p[5], p[6], p[7]) : make_uint4(p[0], p[1], p[2], p[3]);
+            asm volatile("bar.sync %0, 64;" ::"r"(1 + pair + 2 * slice) : "memory");
+            const uint4 th = (is_g ? xu : xg)[lane];
+            const uint32_t other[4] = {th.x, th.y, th.z, th.w};
+            const int cbase = c0 + (is_g ? 0 : 8);
+            float hv[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              const uint32_t own = is_g ? p[j >> 1] : p[4 + (j >> 1)];
+              const float mv = (j & 1) ? bf16_hi(own) : bf16_lo(own);
+              const float ov = (j & 1) ? bf16_hi(other[j >> 1]) : bf16_lo(other[j >> 1]);
+              const float g = is_g ? mv : ov;
+              const float uu = is_g ? ov : mv;
+              hv[j] = act_kind == MOE_ACT_SITU ? situ_mul(g, uu, b_eff, lbeta, has_lb)
+                                               : silu_mul(g, uu);
+            }
+            store_h_t8(hv, out, w.row0 + cbase, w.nrows - cbase, M_rows, f & ~7, live, lane);
+            ++xbuf;
+          }
+        } else {
+          const int m = r0 + quarter * 32 + lane;
+#pragma unroll
+          for (int ci = 0; ci < kChunks; ++ci) {
+            const int c0 = col0 + 16 * ci;
+            if (c0 >= w.nrows) break;
+            const int lim = w.nrows - c0 < 16 ? w.nrows - c0 : 16;
+            store_down_t8_packed(&pk[a][8 * ci], out, w.row0 + c0, lim, M_rows, m & ~7,
+                                 m < M_rows, lane, yrow, yrow ? (int64_t)offsets[E] : 0, st);
+          }
         }
       }
-      tc_fence_before();
-      // release the buffer (or the block's accumulator) to the even CTA's
-      // MMA issuer
-      mbar_arrive_remote(tempty_leader0 + buf * (uint32_t)sizeof(uint64_t));
-      }  // weight blocks
     }
   }
   __syncthreads();
@@ -1224,7 +1320,7 @@ cudaError_t launch_gemm(const CUtensorMap& a0, const CUtensorMap& a1, const CUte
 
 // Weight blocks per CTA-pair unit (1 or 2; see PairCfg).
 #ifndef MOE_PAIR_BLOCKS
-#define MOE_PAIR_BLOCKS 1
+#define MOE_PAIR_BLOCKS 2
 #endif
 constexpr int kPairBlocks = MOE_PAIR_BLOCKS;
 
@@ -1238,6 +1334,7 @@ cudaError_t launch_gemm_pair(const CUtensorMap& a0, const CUtensorMap& a1, const
                              bool pdl_ok, int emod = 0, const int32_t* yrow = nullptr) {
   using C = PairCfg<kPairBlocks>;
   constexpr auto kernel = k_expert_gemm_pair<MODE, kPairBlocks>;
+  static_assert(kPairSlices >= 1 && 1 + 2 * kPairSlices <= 15, "named barriers 1 .. 2 * slices");
   static std::once_flag once[kMaxDevices];
   static cudaError_t set_up[kMaxDevices];
   static int grid_of[kMaxDevices] = {0};
@@ -1249,7 +1346,7 @@ cudaError_t launch_gemm_pair(const CUtensorMap& a0, const CUtensorMap& a1, const
   attr[0].val.clusterDim.z = 1;
   attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[1].val.programmaticStreamSerializationAllowed = 1;
-  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.blockDim = dim3(kPairThreads, 1, 1);
   cfg.dynamicSmemBytes = C::kSmem;
   cfg.stream = s;
   cfg.attrs = attr;
