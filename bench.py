@@ -478,20 +478,31 @@ def block_line(args, wl, r, world):
     }
 
 
-def gate_up_traffic(touched):
-    """DRAM bytes of one gate_up launch from the committed ncu capture of a
-    smaller case, scaled by touched experts; None once the kernel source has
-    changed since the capture."""
+def gate_up_traffic(workload, touched, bound, path=None):
+    # workload: the bench's Workload (name and sizes must match a same-workload record)
+    """DRAM bytes of one gate_up launch from a committed ncu capture: for an
+    HBM-bound launch the decode-shaped capture scaled by touched experts, for a
+    tensor-bound one the capture of the same workload; None when there is no
+    such record or the kernel source has changed since it was taken."""
     import hashlib
-    path = os.path.join(ROOT, "profiles", "expert_gemm_traffic.json")
+    path = path or os.path.join(ROOT, "profiles", "expert_gemm_traffic.json")
     if not os.path.exists(path):
         return None
     with open(path) as f:
-        rec = json.load(f)
-    with open(os.path.join(ROOT, rec["source"]), "rb") as f:
-        if hashlib.sha256(f.read()).hexdigest() != rec["source_sha256"]:
-            return None
-    return (rec["dram_bytes_read"] + rec["dram_bytes_write"]) * touched / rec["touched_experts"]
+        records = json.load(f)["records"]
+    for rec in records:
+        if bound == "hbm" and rec["scaling"] == "touched":
+            scale = touched / rec["touched_experts"]
+        elif bound == "tensor" and rec["scaling"] == "same-workload" and \
+                (rec["workload"], rec["N"], rec["E"]) == (workload.name, workload.N, workload.E):
+            scale = 1.0
+        else:
+            continue
+        with open(os.path.join(ROOT, rec["source"]), "rb") as f:
+            if hashlib.sha256(f.read()).hexdigest() != rec["source_sha256"]:
+                return None
+        return (rec["dram_bytes_read"] + rec["dram_bytes_write"]) * scale
+    return None
 
 
 def gate_up_bytes(wl, touched):
@@ -510,9 +521,8 @@ def gate_up_roofline(wl, touched, gate_up_ms, peaks):
     """The roofline object of the w1/w3 kernel.  Its bound is the one with the
     longer ideal time: the algorithmic bytes at the measured copy bandwidth,
     or the algorithmic flops at the sustained bf16 peak (the kernel runs for
-    milliseconds inside a long step).  DRAM traffic is reported for the HBM
-    case only; it comes from the decode-shaped capture, which does not
-    describe a tensor-bound launch."""
+    milliseconds inside a long step).  DRAM traffic comes from the committed
+    captures (gate_up_traffic)."""
     nbytes, flops = gate_up_bytes(wl, touched), gate_up_flops(wl)
     t_hbm = nbytes / (peaks["hbm_gbs"] * 1e9)
     t_tensor = flops / (peaks["bf16_tflops_sustained"] * 1e12)
@@ -522,14 +532,16 @@ def gate_up_roofline(wl, touched, gate_up_ms, peaks):
         achieved = flops / sec / 1e12
         obj.update({"bound": "tensor", "achieved": achieved,
                     "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
-                    "frac": achieved / peaks["bf16_tflops_sustained"], "traffic": None,
+                    "frac": achieved / peaks["bf16_tflops_sustained"],
+                    "traffic": gate_up_traffic(wl, touched, "tensor"),
                     "peak_kind": "sustained bf16", "peak_nominal": NOMINAL_BF16_TFLOPS,
                     "frac_of_nominal": achieved / NOMINAL_BF16_TFLOPS})
     else:
         achieved = nbytes / sec / 1e9
         obj.update({"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"],
                     "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
-                    "traffic": gate_up_traffic(touched), "peak_nominal": NOMINAL_HBM_GBS,
+                    "traffic": gate_up_traffic(wl, touched, "hbm"),
+                    "peak_nominal": NOMINAL_HBM_GBS,
                     "frac_of_nominal": achieved / NOMINAL_HBM_GBS})
     obj.update({"peak_source": peaks["source"], "touched_experts": touched})
     return obj

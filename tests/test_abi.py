@@ -299,10 +299,39 @@ def test_bench_roofline_picks_the_binding_peak():
     assert pre["bound"] == "hbm"
     skew = WORKLOADS["k2_skew"]
     sk = bench.gate_up_roofline(skew, 364, 8.8, peaks)
-    assert sk["bound"] == "tensor" and sk["unit"] == "TFLOP/s" and sk["traffic"] is None
+    assert sk["bound"] == "tensor" and sk["unit"] == "TFLOP/s"
+    assert sk["traffic"] is None or sk["traffic"] > 0
     flops = 4 * skew.N * skew.K * skew.F * skew.d_e
     assert abs(sk["achieved"] - flops / 8.8e-3 / 1e12) < 1e-9
     assert abs(sk["frac"] - sk["achieved"] / 1374.1) < 1e-12
+
+
+def test_bench_traffic_records(tmp_path):
+    """gate_up_traffic: an HBM-bound launch scales the decode-shaped record by
+    touched experts; a tensor-bound one takes only the record of the same
+    workload and sizes; a record whose kernel source hash no longer matches
+    gives None."""
+    import hashlib, json, bench
+    from synth.workloads import WORKLOADS, scaled
+    src = "bench.py"
+    with open(os.path.join(bench.ROOT, src), "rb") as f:
+        sha = hashlib.sha256(f.read()).hexdigest()
+    skew = WORKLOADS["k2_skew"]
+    recs = [{"workload": "dsv32_decode", "source": src, "source_sha256": sha,
+             "touched_experts": 10, "dram_bytes_read": 1000, "dram_bytes_write": 24,
+             "scaling": "touched"},
+            {"workload": "k2_skew", "N": skew.N, "E": skew.E, "source": src,
+             "source_sha256": sha, "touched_experts": 364, "dram_bytes_read": 5000,
+             "dram_bytes_write": 7, "scaling": "same-workload"}]
+    p = tmp_path / "t.json"
+    p.write_text(json.dumps({"records": recs}))
+    assert bench.gate_up_traffic(WORKLOADS["dsv32_decode"], 30, "hbm", str(p)) == 3 * 1024
+    assert bench.gate_up_traffic(skew, 364, "tensor", str(p)) == 5007
+    assert bench.gate_up_traffic(scaled(skew, N=8192), 300, "tensor", str(p)) is None
+    assert bench.gate_up_traffic(WORKLOADS["k2_prefill"], 384, "tensor", str(p)) is None
+    recs[1]["source_sha256"] = "0" * 64
+    p.write_text(json.dumps({"records": recs}))
+    assert bench.gate_up_traffic(skew, 364, "tensor", str(p)) is None
 
 
 def test_ep_rows_validation(L):
