@@ -311,11 +311,15 @@ struct Unit {
   int e, row0, nrows, rb;
 };
 
+// Unit u is weight block u % RB of the tile at position u / RB of the tile
+// list; order (may be null) maps that position to a tile index.
 __device__ __forceinline__ Unit decode_unit(int64_t u, int RB, int nt, const int32_t* tile_start,
-                                            const int32_t* offsets, int E, int emod) {
+                                            const int32_t* offsets, int E, int emod,
+                                            const int32_t* order = nullptr) {
   Unit r;
-  const int tt = (int)(u / RB);
-  r.rb = (int)(u - (int64_t)tt * RB);
+  const int tp = (int)(u / RB);
+  r.rb = (int)(u - (int64_t)tp * RB);
+  const int tt = order ? order[tp] : tp;
   int lo = 0, hi = E - 1;
   while (lo < hi) {  // largest e with tile_start[e] <= tt
     const int mid = (lo + hi + 1) >> 1;
@@ -780,6 +784,12 @@ __device__ __forceinline__ uint32_t idesc_bf16_m256(int n) {
 }
 
 constexpr int kPairNt = 256;     // token rows per tile (N, split 128 + 128)
+// Tile order of the CTA-pair kernels: 1 spreads the one-tile experts among
+// the tiles of larger ones (k_tiles' order), 0 keeps expert order.
+#ifndef MOE_PAIR_INTERLEAVE
+#define MOE_PAIR_INTERLEAVE 1
+#endif
+constexpr bool kPairInterleave = MOE_PAIR_INTERLEAVE != 0;
 // Epilogue warps of the CTA-pair kernel: kPairSlices warps per TMEM lane
 // quarter, each copying kPairNt / kPairSlices columns of an accumulator to
 // registers.  With two weight blocks per unit the accumulators fill TMEM and
@@ -830,7 +840,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
                        int E, int M_rows, int Kdim, __nv_bfloat16* __restrict__ out,
                        const __nv_bfloat16* __restrict__ res, int act_kind, float beta,
                        float lbeta, DeviceStatus* st, int pdl, int emod, int probe,
-                       const int32_t* __restrict__ yrow) {
+                       const int32_t* __restrict__ yrow, const int32_t* __restrict__ order) {
   using C = PairCfg<PUM>;
   constexpr int STAGES = C::kStages;
   extern __shared__ uint8_t smem_raw[];
@@ -893,7 +903,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
       bool ok = !probe_abort(probe, never, abort_flag, st, 290 + MODE);
       bool dep_pending = pdl != 0;  // see the single-CTA kernel
       for (int64_t u = pair_id; u < total_units && ok; u += npairs) {
-        const Unit w = decode_unit(u, RB, kPairNt, tile_start, offsets, E, emod);
+        const Unit w = decode_unit(u, RB, kPairNt, tile_start, offsets, E, emod, order);
         const int n = ((w.nrows + 15) / 16) * 16;
         const int half = n / 2;  // token rows this CTA contributes
         const bool big = half > 2 * kBoxRows;
@@ -958,7 +968,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
       int local = 0;
       bool ok = true;
       for (int64_t u = pair_id; u < total_units && ok; u += npairs, ++local) {
-        const Unit w = decode_unit(u, RB, kPairNt, tile_start, offsets, E, emod);
+        const Unit w = decode_unit(u, RB, kPairNt, tile_start, offsets, E, emod, order);
         const int n = ((w.nrows + 15) / 16) * 16;
         const uint32_t idesc = idesc_bf16_m256(n);
         // the MMAs of weight block a on stage st (k-block kb)
@@ -1060,7 +1070,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
     uint32_t xbuf = 0;
     bool stop = false;
     for (int64_t u = pair_id; u < total_units && !stop; u += npairs, ++local) {
-      const Unit w = decode_unit(u, RB, kPairNt, tile_start, offsets, E, emod);
+      const Unit w = decode_unit(u, RB, kPairNt, tile_start, offsets, E, emod, order);
       if (MODE == kDown && res) {
         for (int a = 0; a < PUM; ++a) {
           const int buf = PUM == 1 ? (local & 1) : a;
@@ -1188,33 +1198,21 @@ __global__ void __launch_bounds__(kPairThreads, 1)
   }
 }
 
-// Token tiles per expert and their prefix: tile_start[e] = sum_{e'<e}
-// ceil(n_e'/nt), tile_start[E] = total.  Inconsistent offsets are recorded
-// and give the expert no tile, so the GEMM never reads outside xs.
-__global__ void __launch_bounds__(1024) k_tiles(const int32_t* __restrict__ offsets, int E,
-                                                int64_t S, int nt, int32_t* __restrict__ tile_start,
-                                                DeviceStatus* st) {
-  pdl_wait();
-  pdl_trigger();
-  __shared__ int32_t warp_tot[32];
-  const int e = threadIdx.x, lane = e & 31, warp = e >> 5;
-  int32_t n = 0;
-  if (e < E) {
-    const int32_t a = offsets[e], b = offsets[e + 1];
-    const bool bad = a < 0 || b < a || b > S || (e == 0 && a != 0) || (e == E - 1 && b != S);
-    if (bad) record_error(st, MOE_ERR_DEVICE_BOUNDS, 30);
-    else n = (b - a + nt - 1) / nt;
-  }
-  int32_t v = n;
+// Exclusive prefix of v over the block (<= 1024 threads); *total gets the sum.
+__device__ __forceinline__ int32_t block_excl_scan(int32_t v, int32_t* warp_tot, int32_t* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int32_t x = v;
 #pragma unroll
   for (int off = 1; off < 32; off <<= 1) {
-    const int32_t o = __shfl_up_sync(0xffffffffu, v, off);
-    if (lane >= off) v += o;
+    const int32_t o = __shfl_up_sync(0xffffffffu, x, off);
+    if (lane >= off) x += o;
   }
-  if (lane == 31) warp_tot[warp] = v;
+  __syncthreads();  // warp_tot is free (an earlier scan has read it)
+  if (lane == 31) warp_tot[warp] = x;
   __syncthreads();
   if (warp == 0) {
-    int32_t w = warp_tot[lane];
+    const int nw = (blockDim.x + 31) >> 5;
+    int32_t w = lane < nw ? warp_tot[lane] : 0;
 #pragma unroll
     for (int off = 1; off < 32; off <<= 1) {
       const int32_t o = __shfl_up_sync(0xffffffffu, w, off);
@@ -1223,10 +1221,63 @@ __global__ void __launch_bounds__(1024) k_tiles(const int32_t* __restrict__ offs
     warp_tot[lane] = w;
   }
   __syncthreads();
-  const int32_t excl = v - n + (warp > 0 ? warp_tot[warp - 1] : 0);
+  *total = warp_tot[31];
+  return x - v + (warp > 0 ? warp_tot[warp - 1] : 0);
+}
+
+// Token tiles per expert and their prefix: tile_start[e] = sum_{e'<e}
+// ceil(n_e'/nt), tile_start[E] = total.  Inconsistent offsets are recorded
+// and give the expert no tile, so the GEMM never reads outside xs.
+//
+// order (may be null) receives the order in which the CTA-pair kernels take
+// the tiles.  An expert with one tile streams its weights from HBM for that
+// tile alone; the weights of an expert with several are read from HBM once and
+// reused from L2.  In expert order the one-tile experts come in runs: while
+// the pairs work on such a run the kernel waits on HBM, and in a run of a
+// large expert's tiles on the tensor cores.  The order spreads the P one-tile
+// tiles evenly among the R others, each group keeping its own order (the two
+// are merged by the keys (2j+1)/2P and (2i+1)/2R, a tie going to the reused
+// tile), so that at any time a share of the pairs streams weights while the
+// rest compute.
+__global__ void __launch_bounds__(1024) k_tiles(const int32_t* __restrict__ offsets, int E,
+                                                int64_t S, int nt, int32_t* __restrict__ tile_start,
+                                                int32_t* __restrict__ order, DeviceStatus* st) {
+  pdl_wait();
+  pdl_trigger();
+  __shared__ int32_t warp_tot[32];
+  const int e = threadIdx.x;
+  int32_t n = 0;
+  if (e < E) {
+    const int32_t a = offsets[e], b = offsets[e + 1];
+    const bool bad = a < 0 || b < a || b > S || (e == 0 && a != 0) || (e == E - 1 && b != S);
+    if (bad) record_error(st, MOE_ERR_DEVICE_BOUNDS, 30);
+    else n = (b - a + nt - 1) / nt;
+  }
+  int32_t T = 0, P = 0;
+  const int32_t excl = block_excl_scan(n, warp_tot, &T);
   if (e < E) {
     tile_start[e] = excl;
     if (e == E - 1) tile_start[E] = excl + n;
+  }
+  if (!order) return;
+  const int32_t j = block_excl_scan(n == 1 ? 1 : 0, warp_tot, &P);  // one-tile rank
+  const int64_t R = (int64_t)T - P;
+  if (n == 1) {
+    // j + #{i < R : (2i+1) P <= (2j+1) R}
+    const int64_t num = (2 * (int64_t)j + 1) * R - P;
+    int64_t c = num < 0 ? 0 : num / (2 * (int64_t)P) + 1;
+    c = c < R ? c : R;
+    order[j + c] = excl;
+  } else {
+    const int32_t i0 = excl - j;  // reused tiles before this expert's
+    for (int32_t t = 0; t < n; ++t) {
+      // i + #{j < P : (2j+1) R < (2i+1) P}
+      const int64_t i = i0 + t;
+      const int64_t num = (2 * i + 1) * P - 1 - R;
+      int64_t c = num < 0 ? 0 : num / (2 * R) + 1;
+      c = c < P ? c : P;
+      order[i + c] = excl + t;
+    }
   }
 }
 
@@ -1331,7 +1382,8 @@ cudaError_t launch_gemm_pair(const CUtensorMap& a0, const CUtensorMap& a1, const
                              const int32_t* tile_start, int E, int M_rows, int Kdim,
                              __nv_bfloat16* out, const __nv_bfloat16* res,
                              const moe_act_cfg& act, DeviceStatus* st, cudaStream_t s,
-                             bool pdl_ok, int emod = 0, const int32_t* yrow = nullptr) {
+                             bool pdl_ok, int emod = 0, const int32_t* yrow = nullptr,
+                             const int32_t* order = nullptr) {
   using C = PairCfg<kPairBlocks>;
   constexpr auto kernel = k_expert_gemm_pair<MODE, kPairBlocks>;
   static_assert(kPairSlices >= 1 && 1 + 2 * kPairSlices <= 15, "named barriers 1 .. 2 * slices");
@@ -1373,7 +1425,7 @@ cudaError_t launch_gemm_pair(const CUtensorMap& a0, const CUtensorMap& a1, const
   cfg.numAttrs = pdl ? 2 : 1;
   return counted(cudaLaunchKernelEx(&cfg, kernel, a0, a1, b, b64, offsets, tile_start,
                             E, M_rows, Kdim, out, res, (int)act.kind, act.beta, act.linear_beta,
-                            st, pdl, emod > 0 ? emod : E, wait_probe(), yrow));
+                            st, pdl, emod > 0 ? emod : E, wait_probe(), yrow, order));
 }
 
 // Variant choice from shapes only (no host round trip), by the average rows
@@ -1398,7 +1450,8 @@ cudaError_t launch_variant(Variant v, const CUtensorMap& a0, const CUtensorMap& 
                            const int32_t* tile_start, int E, int M_rows, int Kdim,
                            __nv_bfloat16* out, const __nv_bfloat16* res, const moe_act_cfg& act,
                            DeviceStatus* st, cudaStream_t s, bool pdl_ok = true,
-                           int emod = 0, const int32_t* yrow = nullptr) {
+                           int emod = 0, const int32_t* yrow = nullptr,
+                           const int32_t* order = nullptr) {
   switch (v) {
     case kVarDecode:
       return launch_gemm<MODE, kNtDecode, kStagesDecode, kUmDecode, kKsubDecode>(
@@ -1410,14 +1463,19 @@ cudaError_t launch_variant(Variant v, const CUtensorMap& a0, const CUtensorMap& 
           nullptr, 1, 0, 1, nullptr, emod, yrow);
     default:
       return launch_gemm_pair<MODE>(a0, a1, b, b64, offsets, tile_start, E, M_rows, Kdim, out,
-                                    res, act, st, s, pdl_ok, emod, yrow);
+                                    res, act, st, s, pdl_ok, emod, yrow, order);
   }
 }
 
 }  // namespace
 
+// Scratch of the expert MLP: tile_start (E + 1), the CTA-pair tile order (one
+// entry per tile: at most S / 256 + E), then h [S, F] bf16.
+static size_t order_entries(int64_t S, int E) { return (size_t)(S / kPairNt) + (size_t)E + 1; }
+
 size_t expert_scratch_bytes(int64_t S, int E, int F) {
   return align_up(sizeof(int32_t) * (size_t)(E + 1), 256) +
+         align_up(sizeof(int32_t) * order_entries(S, E), 256) +
          align_up(sizeof(__nv_bfloat16) * (size_t)S * (size_t)F, 256);
 }
 
@@ -1432,8 +1490,10 @@ int expert_ffn_run(const __nv_bfloat16* xs, const int32_t* offsets, int E, int64
   // segments s use weights s % n_weights (n_weights = E for the layer)
   const int emod = n_weights > 0 ? n_weights : E;
   int32_t* tile_start = static_cast<int32_t*>(scratch);
-  __nv_bfloat16* h = reinterpret_cast<__nv_bfloat16*>(
-      static_cast<uint8_t*>(scratch) + align_up(sizeof(int32_t) * (size_t)(E + 1), 256));
+  uint8_t* p = static_cast<uint8_t*>(scratch) + align_up(sizeof(int32_t) * (size_t)(E + 1), 256);
+  int32_t* order = reinterpret_cast<int32_t*>(p);
+  p += align_up(sizeof(int32_t) * order_entries(S, E), 256);
+  __nv_bfloat16* h = reinterpret_cast<__nv_bfloat16*>(p);
   CUtensorMap mw1, mw3, mw2, mxs, mh, mxs64, mh64;
   if (!make_map_3d(&mw1, w1, d_e, F, emod, kGateUpRows) ||
       !make_map_3d(&mw3, w3, d_e, F, emod, kGateUpRows) ||
@@ -1445,7 +1505,8 @@ int expert_ffn_run(const __nv_bfloat16* xs, const int32_t* offsets, int E, int64
     return MOE_ERR_CUDA;
   const Variant var = pick_variant(S, E);
   const int nt = var == kVarDecode ? kNtDecode : (var == kVarMid ? kNtMid : kPairNt);
-  if (launch_pdl(k_tiles, dim3(1), dim3(1024), 0, s, offsets, E, S, nt, tile_start, st) !=
+  if (var != kVarLarge || !kPairInterleave) order = nullptr;
+  if (launch_pdl(k_tiles, dim3(1), dim3(1024), 0, s, offsets, E, S, nt, tile_start, order, st) !=
       cudaSuccess)
     return MOE_ERR_CUDA;
   cudaError_t rc;
@@ -1463,12 +1524,12 @@ int expert_ffn_run(const __nv_bfloat16* xs, const int32_t* offsets, int E, int64
                    false, gather->perm, gather->K, (int)gather->N, 1, nullptr, emod);
   } else {
     rc = launch_variant<kGateUp>(var, mw1, mw3, mxs, mxs64, offsets, tile_start, E, F, d_e, h,
-                                 nullptr, act, st, s, true, emod);
+                                 nullptr, act, st, s, true, emod, nullptr, order);
   }
   if (rc != cudaSuccess) return MOE_ERR_CUDA;
   if (after_gate_up && cudaEventRecord(after_gate_up, s) != cudaSuccess) return MOE_ERR_CUDA;
   rc = launch_variant<kDown>(var, mw2, mw2, mh, mh64, offsets, tile_start, E, d_e, F, y, residual,
-                             act, st, s, true, emod, y_rows);
+                             act, st, s, true, emod, y_rows, order);
   return rc == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
