@@ -1239,6 +1239,8 @@ __device__ __forceinline__ int32_t block_excl_scan(int32_t v, int32_t* warp_tot,
 // are merged by the keys (2j+1)/2P and (2i+1)/2R, a tie going to the reused
 // tile), so that at any time a share of the pairs streams weights while the
 // rest compute.
+constexpr int kMaxTileExperts = 1024;  // k_tiles: one thread per expert
+
 __global__ void __launch_bounds__(1024) k_tiles(const int32_t* __restrict__ offsets, int E,
                                                 int64_t S, int nt, int32_t* __restrict__ tile_start,
                                                 int32_t* __restrict__ order, DeviceStatus* st) {
@@ -1262,22 +1264,39 @@ __global__ void __launch_bounds__(1024) k_tiles(const int32_t* __restrict__ offs
   if (!order) return;
   const int32_t j = block_excl_scan(n == 1 ? 1 : 0, warp_tot, &P);  // one-tile rank
   const int64_t R = (int64_t)T - P;
-  if (n == 1) {
-    // j + #{i < R : (2i+1) P <= (2j+1) R}
-    const int64_t num = (2 * (int64_t)j + 1) * R - P;
-    int64_t c = num < 0 ? 0 : num / (2 * (int64_t)P) + 1;
-    c = c < R ? c : R;
-    order[j + c] = excl;
-  } else {
-    const int32_t i0 = excl - j;  // reused tiles before this expert's
-    for (int32_t t = 0; t < n; ++t) {
-      // i + #{j < P : (2j+1) R < (2i+1) P}
-      const int64_t i = i0 + t;
+  // Each tile is placed by one thread: the tile's expert by binary search of
+  // the tile prefix, then its rank in its group and the count of the other
+  // group's tiles before it under the merge.
+  __shared__ int32_t s_start[kMaxTileExperts + 1], s_one[kMaxTileExperts + 1];
+  if (e < E) {
+    s_start[e] = excl;
+    s_one[e] = (n == 1) ? -1 - j : j;  // one-tile experts: -1 - rank; others: one-tile count before
+  }
+  if (e == 0) s_start[E] = T;
+  __syncthreads();
+  for (int32_t t = e; t < T; t += blockDim.x) {
+    int lo = 0, hi = E - 1;
+    while (lo < hi) {  // largest expert whose tiles start at or before t
+      const int mid = (lo + hi + 1) >> 1;
+      if (s_start[mid] <= t) lo = mid;
+      else hi = mid - 1;
+    }
+    const int32_t q = s_one[lo];
+    int64_t pos;
+    if (q < 0) {
+      // one-tile rank jj: jj + #{i < R : (2i+1) P <= (2jj+1) R}
+      const int64_t jj = -1 - q;
+      const int64_t num = (2 * jj + 1) * R - P;
+      int64_t c = num < 0 ? 0 : num / (2 * (int64_t)P) + 1;
+      pos = jj + (c < R ? c : R);
+    } else {
+      // reused rank i: i + #{jj < P : (2jj+1) R < (2i+1) P}
+      const int64_t i = t - q;
       const int64_t num = (2 * i + 1) * P - 1 - R;
       int64_t c = num < 0 ? 0 : num / (2 * R) + 1;
-      c = c < P ? c : P;
-      order[i + c] = excl + t;
+      pos = i + (c < P ? c : P);
     }
+    order[pos] = t;
   }
 }
 
