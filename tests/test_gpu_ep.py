@@ -81,7 +81,7 @@ def test_ep_emulated_equals_one_gpu(moe, name, P, N):
 def _check_against_reference(wl, P, outs, ranks, per_rank=16):
     """Sampled tokens of every emulated rank against the reference's
     per-token loop (its expert MLP and combine), fed with the routing the
-    GPU computed for them, so that only the expert-parallel step is judged."""
+    GPU computed for them, so that only the expert-parallel step is checked."""
     xe, idx, w, got = [], [], [], []
     for p, r in enumerate(ranks):
         n = wl.N
