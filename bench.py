@@ -63,6 +63,9 @@ def parse():
     p.add_argument("--workload", default=DEFAULT_WORKLOAD)
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--no-cpu-baseline", action="store_true")
+    # time replays of one moe_forward captured in a CUDA graph (the routed
+    # layer only; the stage breakdown and the end-to-end pass stay eager)
+    p.add_argument("--graph", action="store_true")
     # profiling cases: the same workload with fewer tokens / experts
     p.add_argument("--tokens", type=int, default=None)
     p.add_argument("--experts", type=int, default=None)
@@ -270,6 +273,27 @@ def run_ours(args, rank, world, local_rank):
             import torch.distributed as dist
             dist.barrier()
 
+    # with --graph the timed steps replay one captured moe_forward (the same
+    # kernels and arguments; the library counts launches at capture, so the
+    # timed region's count is the graph's kernels times the steps)
+    graph, per_graph = None, 0
+    if args.graph:
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            step()
+        torch.cuda.current_stream().wait_stream(side)
+        torch.cuda.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        c0 = moe.launch_count()
+        with torch.cuda.graph(graph):
+            step()
+        per_graph = moe.launch_count() - c0
+        for _ in range(max(args.warmup, 3)):
+            flush.zero_()
+            graph.replay()
+        torch.cuda.synchronize()
+
     # timed region: K steps, one start/end event pair around each moe_forward
     ev0 = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
            for _ in range(args.steps)]
@@ -281,12 +305,16 @@ def run_ours(args, rank, world, local_rank):
         for i in range(args.steps):
             flush.zero_()
             ev0[i][0].record()
-            step()
+            if graph is not None:
+                graph.replay()
+            else:
+                step()
             ev0[i][1].record()
         torch.cuda.synchronize()
         barrier()
         wall = time.perf_counter() - t0
-        launches = moe.launch_count() - n0
+        launches = moe.launch_count() - n0 + per_graph * args.steps
+    del graph
     per_step = [a.elapsed_time(b) for a, b in ev0]
     ms = statistics.mean(per_step)
 
@@ -801,7 +829,8 @@ def main():
                    "router": f"{args.score_func}/{args.group_score}",
                    "global_batch": world * wl.N, "parallelism": f"dp{world}",
                    "l2": "expert weights > L2, plus a 256 MB write between steps outside the "
-                         "per-step events"},
+                         "per-step events",
+                   "launch": "CUDA graph replay" if args.graph else "eager"},
         "roofline": gate_up_roofline(wl, r["touched"], r["gate_up_ms"], peaks),
         "stages_ms": r["stage_ms"],
         "stages_pass": "a second pass of K steps with a CUDA event after every stage",
