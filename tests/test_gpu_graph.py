@@ -71,3 +71,55 @@ def test_forward_graph_replay_matches_eager(moe, name):
     assert torch.equal(out.view(torch.int16), ref2.view(torch.int16))
     assert not torch.equal(ref2.view(torch.int16), ref.view(torch.int16))
     print(f"{name}: {captured} kernels in the graph")
+
+
+@pytest.mark.parametrize("name", ["tiny_block", "k3_block_decode"])
+def test_block_graph_replay_matches_eager(moe, name):
+    """The whole MoE block (latent projections, norm, shared experts, split-K
+    dense layers) captured and replayed."""
+    import torch
+    import synth
+    from synth.workloads import BLOCKS
+    wl = BLOCKS[name]
+    dev = dev_inputs(wl)
+    blk = synth.workloads.dev_block(wl)
+    W = moe.BlockWeights(
+        gate_weight=dev["W"], gate_bias=dev["bias"], w1=dev["w1"], w3=dev["w3"], w2=dev["w2"],
+        down_proj=blk["down_proj"], norm_weight=blk["norm_w"], up_proj=blk["up_proj"],
+        shared_w1=None if blk["shared"] is None else blk["shared"][0],
+        shared_w3=None if blk["shared"] is None else blk["shared"][1],
+        shared_w2=None if blk["shared"] is None else blk["shared"][2])
+    cfg = moe.RouteConfig(wl.E, wl.G, wl.TG, wl.K, wl.route_scale, wl.norm)
+    act = moe.ActConfig(wl.act, wl.beta, wl.lbeta)
+    x = dev["x"].clone()
+    ref = moe.block_forward(x, W, cfg, act, norm_eps=wl.norm_eps).clone()
+    torch.cuda.synchronize()
+    ws = moe.workspace(moe.lib().moe_block_workspace_size(
+        wl.N, *_block_args(moe, wl, W, cfg)))
+    out = torch.empty_like(ref)
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        moe.block_forward(x, W, cfg, act, norm_eps=wl.norm_eps, ws=ws, out=out)
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        moe.block_forward(x, W, cfg, act, norm_eps=wl.norm_eps, ws=ws, out=out)
+    out.zero_()
+    g.replay()
+    torch.cuda.synchronize()
+    assert moe.get_status(ws) == 0
+    assert torch.equal(out.view(torch.int16), ref.view(torch.int16))
+    x.copy_(-dev["x"])
+    g.replay()
+    ref2 = moe.block_forward(-dev["x"], W, cfg, act, norm_eps=wl.norm_eps)
+    torch.cuda.synchronize()
+    assert torch.equal(out.view(torch.int16), ref2.view(torch.int16))
+
+
+def _block_args(moe, wl, W, cfg):
+    import ctypes
+    F_sh = 0 if W.shared_w1 is None else W.shared_w1.shape[0]
+    dims = moe._BlockDims(wl.d_r, wl.d_e, wl.F, F_sh, float(wl.norm_eps))
+    return ctypes.byref(dims), ctypes.byref(W._c()), ctypes.byref(cfg._c())
