@@ -430,13 +430,17 @@ def test_expert_ffn_large_tiles_ragged(moe, counts):
     _expert_case(moe, wl, np.array(counts), list(range(5)), rows_per_expert=96)
 
 
-def test_expert_ffn_pair_tile_order_all_rows(moe):
+@pytest.mark.parametrize("act", ["silu", "situ"])
+def test_expert_ffn_pair_tile_order_all_rows(moe, act):
     """The CTA-pair variant takes the tiles of one-tile experts (1 to 256 rows)
     spread among the tiles of larger ones; with 8 one-tile experts (1, 2, 3,
     17, 40, 64, 255 and 256 rows), an empty one and three of 3-4 tiles, every
     output row is checked against the oracle: a tile taken twice or never
-    would leave rows wrong."""
-    wl = scaled(WORKLOADS["tiny"], E=12, d_e=256, F=384)
+    would leave rows wrong.  SiTU takes the same epilogue with its own
+    activation."""
+    wl = scaled(WORKLOADS["tiny"], E=12, d_e=256, F=384, act=act,
+                beta=4.0 if act == "situ" else WORKLOADS["tiny"].beta,
+                lbeta=8.0 if act == "situ" else WORKLOADS["tiny"].lbeta)
     counts = np.array([700, 3, 40, 256, 1, 0, 900, 17, 255, 64, 520, 2])
     assert counts.sum() > 128 * wl.E  # the 256-row tile variant
     _expert_case(moe, wl, counts, list(range(12)), rows_per_expert=10 ** 6)
