@@ -378,6 +378,32 @@ def test_forward_end_to_end(moe, name):
                        what=f"layer {name}", layer=True)
 
 
+@pytest.mark.parametrize("N", [512, 9216])
+def test_forward_max_experts_and_top_k(moe, N):
+    """The largest expert count and top-k the ABI accepts (E = 1024, K = 16)
+    through the whole layer: 512 tokens take the decode kernels (8 rows per
+    expert), 9216 tokens the CTA-pair kernels (144 rows per expert, one-tile
+    experts spread among larger ones); both take the int8 gate.  128 sampled
+    tokens against the reference's per-token loop."""
+    wl = scaled(WORKLOADS["tiny"], N=N, E=1024, K=16, name=f"e1024_k16_n{N}")
+    assert (N * wl.K) / wl.E > 128 or N == 512
+    dev = synth.workloads.dev_inputs(wl)
+    out_g, idx_g, w_g = _forward(moe, wl, dev)
+    inp = host_inputs(wl)
+    toks = np.unique(np.concatenate(
+        [[0, N - 1], np.random.default_rng(11).choice(N, 126, False)]))
+    x = np.ascontiguousarray(inp["x"][toks])
+    xe = np.ascontiguousarray(inp["x_e"][toks])
+    idx_r, w_r, margin = oracle.route(x, inp["W"], inp["bias"], wl.G, wl.TG, wl.K,
+                                      wl.route_scale, wl.norm)
+    _check_routing(idx_g[toks], w_g[toks], idx_r, w_r, margin)
+    keep = margin > MARGIN
+    out_r = oracle_layer_tokens(wl, xe, idx_r, w_r)
+    print(f"forward E=1024 K=16 N={N}: {keep.sum()}/{len(toks)} tokens")
+    check_bf16_outputs(out_g[toks][keep], out_r[keep], long_dots=False,
+                       what=f"layer E=1024 K=16 N={N}", layer=True)
+
+
 def test_forward_tiny_matches_reference_moe_infer_exactly_where_routing_agrees(moe):
     """At the tiny size the whole batch goes through the reference's sorted
     moe_infer; compare every token with margin > 1e-5."""
