@@ -967,18 +967,23 @@ __global__ void __launch_bounds__(kPairThreads, 1)
       uint32_t phase = 0;
       int local = 0;
       bool ok = true;
+      const uint64_t desc_base = sw128_desc(smem_u32(smem));
       for (int64_t u = pair_id; u < total_units && ok; u += npairs, ++local) {
         const Unit w = decode_unit(u, RB, kPairNt, tile_start, offsets, E, emod, order);
         const int n = ((w.nrows + 15) / 16) * 16;
         const uint32_t idesc = idesc_bf16_m256(n);
         // the MMAs of weight block a on stage st (k-block kb)
+        // descriptors: the shared-memory base's, plus each operand's byte
+        // offset / 16 (the start-address field; no carry at these offsets)
         auto mma_block = [&](int a, int st, int kb, uint32_t d) {
-          const uint32_t a0 = smem_u32(smem + st * C::kStageBytes) + a * C::kABlockBytes;
-          const uint32_t b0 = smem_u32(smem + st * C::kStageBytes) + C::kABytes;
+          const uint64_t so = (uint64_t)(st * (C::kStageBytes >> 4));
+          const uint64_t da = desc_base + so + (uint64_t)(a * (C::kABlockBytes >> 4));
+          const uint64_t db = desc_base + so + (uint64_t)(C::kABytes >> 4);
+          umma_bf16_pair(d, da, db, idesc, kb != 0);
 #pragma unroll
-          for (int k = 0; k < BK / UK; ++k)
-            umma_bf16_pair(d, sw128_desc(a0 + k * UK * 2), sw128_desc(b0 + k * UK * 2), idesc,
-                           (kb | k) != 0);
+          for (int k = 1; k < BK / UK; ++k)
+            umma_bf16_pair(d, da + (uint64_t)(k * UK * 2 / 16), db + (uint64_t)(k * UK * 2 / 16),
+                           idesc, 1u);
         };
         if constexpr (PUM == 1) {
           const int buf = local & 1;
