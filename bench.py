@@ -506,13 +506,23 @@ def block_line(args, wl, r, world):
     }
 
 
+def source_sha256(source):
+    """sha256 of a record's kernel source: one path, or the bytes of several
+    (the kernel file and the headers it includes) in the listed order."""
+    import hashlib
+    h = hashlib.sha256()
+    for rel in ([source] if isinstance(source, str) else source):
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
 def gate_up_traffic(workload, touched, bound, path=None):
     # workload: the bench's Workload (name and sizes must match a same-workload record)
     """DRAM bytes of one gate_up launch from a committed ncu capture: for an
     HBM-bound launch the decode-shaped capture scaled by touched experts, for a
     tensor-bound one the capture of the same workload; None when there is no
     such record or the kernel source has changed since it was taken."""
-    import hashlib
     path = path or os.path.join(ROOT, "profiles", "expert_gemm_traffic.json")
     if not os.path.exists(path):
         return None
@@ -526,9 +536,8 @@ def gate_up_traffic(workload, touched, bound, path=None):
             scale = 1.0
         else:
             continue
-        with open(os.path.join(ROOT, rec["source"]), "rb") as f:
-            if hashlib.sha256(f.read()).hexdigest() != rec["source_sha256"]:
-                return None
+        if source_sha256(rec["source"]) != rec["source_sha256"]:
+            return None
         return (rec["dram_bytes_read"] + rec["dram_bytes_write"]) * scale
     return None
 

@@ -332,6 +332,15 @@ def test_bench_traffic_records(tmp_path):
     recs[1]["source_sha256"] = "0" * 64
     p.write_text(json.dumps({"records": recs}))
     assert bench.gate_up_traffic(skew, 364, "tensor", str(p)) is None
+    # several source files: the hash covers all of them, in order
+    two = [src, "__graft_entry__.py"]
+    recs[1]["source"] = two
+    recs[1]["source_sha256"] = bench.source_sha256(two)
+    p.write_text(json.dumps({"records": recs}))
+    assert bench.gate_up_traffic(skew, 364, "tensor", str(p)) == 5007
+    recs[1]["source"] = two[::-1]
+    p.write_text(json.dumps({"records": recs}))
+    assert bench.gate_up_traffic(skew, 364, "tensor", str(p)) is None
 
 
 def test_ep_rows_validation(L):
