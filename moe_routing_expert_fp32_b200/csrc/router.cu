@@ -91,6 +91,8 @@ __global__ void __launch_bounds__(256, 2) k_gate_partial(const __nv_bfloat16* __
   double acc[8][2];
 #pragma unroll
   for (int i = 0; i < 8; ++i) acc[i][0] = acc[i][1] = 0.0;
+  // fp32 chains as packed pairs: p2[p][j] holds tokens 2p and 2p + 1 of
+  // expert j; fma.rn.f32x2 rounds each half as fmaf does
 
   int buf = 0;
   if (kc0 < kc1) {
@@ -101,25 +103,31 @@ __global__ void __launch_bounds__(256, 2) k_gate_partial(const __nv_bfloat16* __
   for (int kc = kc0; kc < kc1; ++kc) {
     const bool more = kc + 1 < kc1;
     if (more) load_chunk(kc + 1);
-    float blk[8][2];
+    uint64_t p2[4][2];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) blk[i][0] = blk[i][1] = 0.f;
+    for (int q = 0; q < 4; ++q) p2[q][0] = p2[q][1] = 0ull;
 #pragma unroll 8
     for (int k = 0; k < GK; ++k) {
-      const float4 a0 = *reinterpret_cast<const float4*>(&xs[buf][k][ty * 8]);
-      const float4 a1 = *reinterpret_cast<const float4*>(&xs[buf][k][ty * 8 + 4]);
+      const ulonglong2 a0 = *reinterpret_cast<const ulonglong2*>(&xs[buf][k][ty * 8]);
+      const ulonglong2 a1 = *reinterpret_cast<const ulonglong2*>(&xs[buf][k][ty * 8 + 4]);
       const float2 b = *reinterpret_cast<const float2*>(&wsm[buf][k][tx * 2]);
-      const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+      const uint64_t av[4] = {a0.x, a0.y, a1.x, a1.y};
+      uint64_t bb[2];
+      asm("mov.b64 %0, {%1, %1};" : "=l"(bb[0]) : "r"(__float_as_uint(b.x)));
+      asm("mov.b64 %0, {%1, %1};" : "=l"(bb[1]) : "r"(__float_as_uint(b.y)));
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        blk[i][0] = fmaf(av[i], b.x, blk[i][0]);
-        blk[i][1] = fmaf(av[i], b.y, blk[i][1]);
+      for (int q = 0; q < 4; ++q) {
+        asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(p2[q][0]) : "l"(av[q]), "l"(bb[0]));
+        asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(p2[q][1]) : "l"(av[q]), "l"(bb[1]));
       }
     }
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      acc[i][0] += (double)blk[i][0];
-      acc[i][1] += (double)blk[i][1];
+    for (int q = 0; q < 4; ++q) {
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        acc[2 * q][j] += (double)__uint_as_float((uint32_t)p2[q][j]);
+        acc[2 * q + 1][j] += (double)__uint_as_float((uint32_t)(p2[q][j] >> 32));
+      }
     }
     if (more) store_chunk(buf ^ 1);
     __syncthreads();
@@ -278,10 +286,14 @@ __global__ void __launch_bounds__(32 * kSelWarps) k_select(
 // rounded up to 32).  The logits come either from `logits` or, when the gate
 // GEMM ran split over d_r, straight from its double partials (summed in split
 // order and rounded once, exactly as k_reduce_partials does), so no reduce
-// kernel runs.  The score of each expert is computed by its own thread; the
-// top-K is taken per warp (32 experts each) and the per-warp candidates are
-// merged by warp 0, under the same total order (value desc, index asc) as
-// k_select, so the result is identical to it.
+// kernel runs.  The score of each expert is computed by its own thread.  Every
+// "best of" step is a rank under the total order of k_select (value desc,
+// index asc), computed by each candidate in parallel instead of rounds of
+// warp arg-max: an expert's rank in its group gives the group's top-2 (or
+// maximum), a group's rank among the groups decides whether it is kept, an
+// expert's rank in its warp makes the warp's top-K candidates, and a
+// candidate's rank among all candidates its place in the token's list.  The
+// order is strict, so every rank is unique and the result is k_select's.
 constexpr int kMaxSelWarps = 32;  // E <= 1024
 constexpr int64_t kBlockSelectMaxN = 1024;  // batches up to this size: a block per token
 __global__ void __launch_bounds__(1024) k_select_block(
@@ -294,12 +306,13 @@ __global__ void __launch_bounds__(1024) k_select_block(
   __shared__ float s_s[1024];
   __shared__ float s_c[1024];
   __shared__ double s_x[1024];
-  __shared__ float cand_v[kMaxSelWarps][16];
-  __shared__ int cand_i[kMaxSelWarps][16];
+  __shared__ float cand_v[kMaxSelWarps * 16];
+  __shared__ int cand_i[kMaxSelWarps * 16];
   __shared__ float s_red[kMaxSelWarps];
-  __shared__ float s_gs[32];
+  __shared__ float s_g1[32], s_g2[32], s_gs[32];
   __shared__ unsigned s_kept;
   __shared__ double s_sum;
+  __shared__ int sel_i[16];
   const int e = threadIdx.x, lane = e & 31, warp = e >> 5;
   const int nw = blockDim.x >> 5;
   const int64_t t = blockIdx.x;
@@ -307,9 +320,18 @@ __global__ void __launch_bounds__(1024) k_select_block(
   float L = 0.f;
   if (live) {
     if (part) {
+      // all partial loads in flight before the sums (summed in split order)
+      const double* p = part + t * E + e;
+      const int64_t zs = N * (int64_t)E;
       double a = 0.0;
-#pragma unroll 8
-      for (int z = 0; z < splits; ++z) a += part[((int64_t)z * N + t) * E + e];
+      for (int z0 = 0; z0 < splits; z0 += 16) {
+        double v[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) v[j] = z0 + j < splits ? p[(int64_t)(z0 + j) * zs] : 0.0;
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+          if (z0 + j < splits) a += v[j];
+      }
       L = (float)a;
     } else {
       L = logits[t * E + e];
@@ -338,83 +360,90 @@ __global__ void __launch_bounds__(1024) k_select_block(
   } else if (live) {
     sv = (float)__drcp_rn(1.0 + exp(-(double)L));
   }
+  const int my = live ? e : 0x7fffffff;
   float cv = live ? (bias ? __fadd_rn(sv, bias[e]) : sv) : kNegInf;
   if (live) {
     s_s[e] = sv;
     s_c[e] = cv;
   }
+  if (e < 32) s_g2[e] = kNegInf;  // a group of one expert has no second
   __syncthreads();
   if (G > 1) {
+    // the expert's rank in its group: rank 0 is the group's maximum, rank 1
+    // its second (equal values count twice, as in a top-2)
     const int gsz = E / G;
-    if (e < G) {
-      float a = kNegInf, b = kNegInf;
-      for (int i = 0; i < gsz; ++i) {
-        const float v = s_c[e * gsz + i];
-        if (v > a) { b = a; a = v; }
-        else if (v > b) { b = v; }
-      }
-      s_gs[e] = group_mode == MOE_GROUP_MAX ? a : __fadd_rn(a, b);
+    if (live) {
+      const int g = e / gsz, b0 = g * gsz;
+      int r = 0;
+      for (int j = 0; j < gsz; ++j) r += ranks_before(s_c[b0 + j], b0 + j, cv, e) ? 1 : 0;
+      if (r == 0) s_g1[g] = cv;
+      if (r == 1) s_g2[g] = cv;
     }
     __syncthreads();
+    if (e < G) s_gs[e] = group_mode == MOE_GROUP_MAX ? s_g1[e] : __fadd_rn(s_g1[e], s_g2[e]);
+    __syncthreads();
+    // a group is kept when fewer than TG groups rank before it
     if (warp == 0) {
-      const float gs = lane < G ? s_gs[lane] : kNegInf;
       bool kept = false;
-      for (int r = 0; r < TG; ++r) {
-        float v = (lane < G && !kept) ? gs : kNegInf;
-        int i = (lane < G && !kept) ? lane : 0x7fffffff;
-        warp_best(v, i);
-        if (lane == i) kept = true;
+      if (lane < G) {
+        const float gs = s_gs[lane];
+        int r = 0;
+        for (int h = 0; h < G; ++h) r += ranks_before(s_gs[h], h, gs, lane) ? 1 : 0;
+        kept = r < TG;
       }
       const unsigned m = __ballot_sync(0xffffffffu, kept);
       if (lane == 0) s_kept = m;
     }
     __syncthreads();
     if (live && !((s_kept >> (e / gsz)) & 1u)) cv = kNegInf;
+    if (live) s_c[e] = cv;
+    __syncthreads();
   }
-  // per-warp top-K of (cv, e), then the merge by warp 0
-  {
-    float v = cv;
-    const int my = live ? e : 0x7fffffff;
-    bool taken = false;
-    for (int k = 0; k < K; ++k) {
-      float bv = taken ? kNegInf : v;
-      int bi = taken ? 0x7fffffff : my;
-      warp_best(bv, bi);
-      if (bi == my) taken = true;
-      if (lane == 0) {
-        cand_v[warp][k] = bv;
-        cand_i[warp][k] = bi;
+  // the warp's top-K: its experts of rank < K in the warp (live experts only;
+  // a warp with fewer than K live experts offers them all)
+  const int w0 = warp * 32;
+  const int nlive_w = E - w0 < 32 ? (E - w0 > 0 ? E - w0 : 0) : 32;
+  const int kw = nlive_w < K ? nlive_w : K;
+  if (live) {
+    int r = 0;
+    for (int j = 0; j < nlive_w; ++j) r += ranks_before(s_c[w0 + j], w0 + j, cv, my) ? 1 : 0;
+    if (r < kw) {
+      cand_v[warp * K + r] = cv;
+      cand_i[warp * K + r] = e;
+    }
+  }
+  __syncthreads();
+  // each candidate's rank among all candidates: rank k is the token's k-th
+  // expert.  A warp's candidates are stored best first, so the ones ranking
+  // before a given candidate are a prefix: its length by binary search.
+  const int nc = nw * K;
+  if (e < nc) {
+    const int cw = e / K, own = e - cw * K;
+    const int cw0 = cw * 32;
+    const int cnl = E - cw0 < 32 ? (E - cw0 > 0 ? E - cw0 : 0) : 32;
+    if (own < (cnl < K ? cnl : K)) {
+      const float v = cand_v[e];
+      const int i = cand_i[e];
+      int r = own;
+      for (int w = 0; w < nw; ++w) {
+        if (w == cw) continue;
+        const int wl = E - w * 32 < 32 ? (E - w * 32 > 0 ? E - w * 32 : 0) : 32;
+        int lo = 0, hi = wl < K ? wl : K;  // first entry not ranking before (v, i)
+        while (lo < hi) {
+          const int mid = (lo + hi) >> 1;
+          if (ranks_before(cand_v[w * K + mid], cand_i[w * K + mid], v, i)) lo = mid + 1;
+          else hi = mid;
+        }
+        r += lo;
       }
+      if (r < K) sel_i[r] = i;
     }
   }
   __syncthreads();
   if (warp == 0) {
-    const int nc = nw * K;  // candidates, lane l holds c = l, l + 32, ...
-    unsigned chosen = 0;
-    int my_e = 0;
-    for (int k = 0; k < K; ++k) {
-      float bv = kNegInf;
-      int bi = 0x7fffffff;
-      for (int j = 0, c = lane; c < nc; ++j, c += 32) {
-        if ((chosen >> j) & 1u) continue;
-        const float cvv = cand_v[c / K][c % K];
-        const int ci = cand_i[c / K][c % K];
-        if (ranks_before(cvv, ci, bv, bi)) { bv = cvv; bi = ci; }
-      }
-      const int src_bi = bi;
-      warp_best(bv, bi);
-      if (bi == 0x7fffffff) {  // cannot happen for a validated config
-        record_error(st, MOE_ERR_DEVICE_BOUNDS, 2);
-        bi = 0;
-      }
-      // the lane whose scan produced the winner marks that candidate taken
-      if (src_bi == bi) {
-        for (int j = 0, c = lane; c < nc; ++j, c += 32)
-          if (!((chosen >> j) & 1u) && cand_i[c / K][c % K] == bi) { chosen |= 1u << j; break; }
-      }
-      if (lane == k) my_e = bi;
-    }
-    float wk = (lane < K) ? s_s[my_e] : 0.f;
+    const int my_e = lane < K ? sel_i[lane] : 0;
+    if (lane < K && (my_e < 0 || my_e >= E)) record_error(st, MOE_ERR_DEVICE_BOUNDS, 2);
+    float wk = (lane < K && my_e >= 0 && my_e < E) ? s_s[my_e] : 0.f;
     if (K > 1 && norm) {
       float den = __shfl_sync(0xffffffffu, wk, 0);
       for (int k = 1; k < K; ++k) den = __fadd_rn(den, __shfl_sync(0xffffffffu, wk, k));
