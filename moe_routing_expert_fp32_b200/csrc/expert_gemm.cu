@@ -723,7 +723,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 //             for both CTAs' bytes; both CTAs' TMA loads credit it;
 //   empty[s]  (both CTAs) the MMA commit is multicast to both;
 //   tfull[b]  (both CTAs) the MMA commit is multicast to both;
-//   tempty[b] (even CTA) 256 arrivals: the epilogue threads of both CTAs.
+//   tempty[b] (even CTA) one arrival per epilogue warp of both CTAs, by an
+//             elected lane after the warp's TMEM loads and a warp sync.
 // Cluster barriers after set-up and before freeing TMEM; every mbarrier wait
 // is bounded as in the single-CTA kernel.
 constexpr uint32_t kPeerBitMask = 0xFEFFFFFFu;  // clears the pair-rank bit of a cluster address
@@ -877,7 +878,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&tfull[b], 1);
-      mbar_init(&tempty[b], 2 * (kPairThreads - 64));  // every epilogue thread of the pair
+      mbar_init(&tempty[b], 2 * (kPairThreads - 64) / 32);  // every epilogue warp of the pair
     }
     mbar_init(never, 1);
     *abort_flag = 0;
@@ -1000,52 +1001,21 @@ __global__ void __launch_bounds__(kPairThreads, 1)
           }
           if (ok) umma_commit_pair(&tfull[buf]);
         } else {
-          // block 0's accumulator must be drained before the unit starts;
-          // block 1's may still be draining: its MMAs wait on held stages
-          // (kept out of the ring until both blocks have used them)
+          // both accumulators must have been copied out by the epilogue
+          // before the unit starts (block 1's copy follows block 0's by ~1 k
+          // cycles); the loop then issues both blocks' MMAs on every stage
           const uint32_t tpar = (local & 1) ^ 1;
           if (!mbar_wait(&tempty[0], tpar, abort_flag)) { ok = false; break; }
+          if (!mbar_wait(&tempty[1], tpar, abort_flag)) { ok = false; break; }
           tc_fence_after();
-          int held_st[STAGES], held_kb[STAGES];
-          int held = 0;
-          bool b1_free = false;
-          auto flush_held = [&]() {
-            for (int i = 0; i < held; ++i) {
-              mma_block(1, held_st[i], held_kb[i], tmem_base + C::kBufCols);
-              umma_commit_pair(&empty[held_st[i]]);
-            }
-            held = 0;
-          };
           for (int kb = 0; kb < KB; ++kb) {
-            if (!b1_free && held == STAGES) {  // the ring is all held: wait for block 1
-              if (!mbar_wait(&tempty[1], tpar, abort_flag)) { ok = false; break; }
-              tc_fence_after();
-              b1_free = true;
-              flush_held();
-            }
             if (!mbar_wait(&full[stage], phase, abort_flag)) { ok = false; break; }
             tc_fence_after();
             mma_block(0, stage, kb, tmem_base);
             if (kb == KB - 1) umma_commit_pair(&tfull[0]);  // block 0 is complete
-            if (!b1_free && mbar_try_wait(&tempty[1], tpar)) {
-              tc_fence_after();
-              b1_free = true;
-              flush_held();
-            }
-            if (b1_free) {
-              mma_block(1, stage, kb, tmem_base + C::kBufCols);
-              umma_commit_pair(&empty[stage]);
-            } else {
-              held_st[held] = stage;
-              held_kb[held] = kb;
-              ++held;
-            }
+            mma_block(1, stage, kb, tmem_base + C::kBufCols);
+            umma_commit_pair(&empty[stage]);
             if (++stage == STAGES) { stage = 0; phase ^= 1; }
-          }
-          if (ok && !b1_free) {
-            if (!mbar_wait(&tempty[1], tpar, abort_flag)) { ok = false; break; }
-            tc_fence_after();
-            flush_held();
           }
           if (ok) umma_commit_pair(&tfull[1]);
         }
@@ -1080,7 +1050,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
         for (int a = 0; a < PUM; ++a) {
           const int buf = PUM == 1 ? (local & 1) : a;
           const uint32_t tphase = PUM == 1 ? ((local >> 1) & 1) : (local & 1);
-          if (!mbar_wait(&tfull[buf], tphase, abort_flag)) {
+          if (!__all_sync(0xffffffffu, mbar_wait(&tfull[buf], tphase, abort_flag))) {
             if (lane == 0) record_error(st, MOE_ERR_DEVICE_TIMEOUT, 220 + MODE);
             *abort_flag = 1;
             stop = true;
@@ -1103,7 +1073,8 @@ __global__ void __launch_bounds__(kPairThreads, 1)
                     down_out(v[j], res, w.row0 + c0 + j, M_rows, m);
           }
           tc_fence_before();
-          mbar_arrive_remote(tempty_leader0 + buf * (uint32_t)sizeof(uint64_t));
+          __syncwarp();
+          if (lane == 0) mbar_arrive_remote(tempty_leader0 + buf * (uint32_t)sizeof(uint64_t));
         }
         continue;
       }
@@ -1114,7 +1085,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
       for (int a = 0; a < PUM; ++a) {
         const int buf = PUM == 1 ? (local & 1) : a;
         const uint32_t tphase = PUM == 1 ? ((local >> 1) & 1) : (local & 1);
-        if (!mbar_wait(&tfull[buf], tphase, abort_flag)) {
+        if (!__all_sync(0xffffffffu, mbar_wait(&tfull[buf], tphase, abort_flag))) {
           if (lane == 0) record_error(st, MOE_ERR_DEVICE_TIMEOUT, 220 + MODE);
           *abort_flag = 1;
           stop = true;
@@ -1135,8 +1106,11 @@ __global__ void __launch_bounds__(kPairThreads, 1)
           }
         }
         tc_fence_before();
-        // the accumulator (buffer, or block) goes back to the even CTA's MMA issuer
-        mbar_arrive_remote(tempty_leader0 + buf * (uint32_t)sizeof(uint64_t));
+        __syncwarp();
+        // the accumulator (buffer, or block) goes back to the even CTA's MMA
+        // issuer: one arrival per warp (1024 single-thread arrivals on one
+        // barrier word cost ~8-20 k cycles per unit)
+        if (lane == 0) mbar_arrive_remote(tempty_leader0 + buf * (uint32_t)sizeof(uint64_t));
       }
       if (stop) break;
 #pragma unroll
