@@ -1108,8 +1108,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
         tc_fence_before();
         __syncwarp();
         // the accumulator (buffer, or block) goes back to the even CTA's MMA
-        // issuer: one arrival per warp (1024 single-thread arrivals on one
-        // barrier word cost ~8-20 k cycles per unit)
+        // issuer: one arrival per warp, after the warp's loads and a warp sync
         if (lane == 0) mbar_arrive_remote(tempty_leader0 + buf * (uint32_t)sizeof(uint64_t));
       }
       if (stop) break;
