@@ -36,7 +36,8 @@
 //     weight row is read 256 contiguous bytes at a time, loaded with an L2
 //     evict-first hint since each is read once), mid (NTMAX 128, two A blocks
 //     and accumulators per unit, 4 stages) and large (a CTA pair running
-//     256x256x16 cta_group::2 MMAs, 6 stages; see k_expert_gemm_pair).
+//     256x256x16 cta_group::2 MMAs on two weight blocks per token tile, 4
+//     stages; see k_expert_gemm_pair).
 //   * the page's rounding points: g, u rounded to bf16; SiLU output rounded to
 //     bf16 before the product; SiTU evaluated in fp32; h and y rounded to bf16.
 //   * unit u -> (token tile, weight-row block), row block fastest: CTAs that
