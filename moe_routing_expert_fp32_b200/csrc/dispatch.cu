@@ -14,6 +14,9 @@
 //   k_scatter one warp per chunk again: every block takes the exclusive scan
 //             of counts (block 0 stores it as offsets), then the slots are
 //             ranked in slot order within the chunk -> pos[slot], perm[pos].
+// Small sorts (at most 4096 slots and 256 experts, decode batches) run the
+// same three passes in one block instead: k_sort_small, 32 warps, warp w the
+// w-th of 32 contiguous chunks, its counts in shared memory.
 // Then k_gather copies every token row once from HBM and writes it to its K
 // sorted positions (token-major, so x_e is read once, not K times).  Without
 // xs (the expert MLP gathering its rows itself) k_gather is skipped.
@@ -203,6 +206,102 @@ __global__ void __launch_bounds__(32 * kWarps) k_scatter(const int32_t* __restri
   }
 }
 
+// The stable counting sort of k_hist + k_scan + k_scatter in one block of 32
+// warps for S <= kSmallSortMaxS slots and E <= kSmallSortMaxE experts: warp w
+// takes the w-th of 32 contiguous chunks of slots, counts them per expert
+// (pass 1), every expert's thread turns the warps' counts into their
+// exclusive prefix and the expert totals into offsets (pass 2), and each warp
+// ranks its slots in slot order (pass 3).  The ranks are those of the
+// three-kernel sort: pos and perm are unique for a stable sort.
+constexpr int kSmallSortMaxS = 4096;
+constexpr int kSmallSortMaxE = 256;
+constexpr int kSmallSortRounds = kSmallSortMaxS / (32 * 32);  // slots per lane
+
+__global__ void __launch_bounds__(1024) k_sort_small(const int32_t* __restrict__ idx, int S, int E,
+                                                     int32_t* __restrict__ counts,
+                                                     int32_t* __restrict__ offsets,
+                                                     int32_t* __restrict__ perm,
+                                                     int32_t* __restrict__ pos,
+                                                     DeviceStatus* st) {
+  pdl_wait();
+  pdl_trigger();
+  __shared__ int32_t cnt[32][kSmallSortMaxE];
+  __shared__ int32_t warp_tot[32];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int CH = (S + 31) / 32;
+  const int beg = warp * CH;
+  const int end = beg + CH < S ? beg + CH : S;
+  for (int e = lane; e < E; e += 32) cnt[warp][e] = 0;
+  __syncwarp();
+  // pass 1: this warp's counts; the slot indices stay in registers
+  int ev[kSmallSortRounds];
+#pragma unroll
+  for (int i = 0; i < kSmallSortRounds; ++i) {
+    const int slot = beg + 32 * i + lane;
+    int e = slot < end ? idx[slot] : -1;
+    if (slot < end && (e < 0 || e >= E)) {
+      record_error(st, MOE_ERR_DEVICE_BOUNDS, 10);
+      e = -1;
+    }
+    ev[i] = e;
+  }
+#pragma unroll
+  for (int i = 0; i < kSmallSortRounds; ++i) {
+    const unsigned peers = __match_any_sync(0xffffffffu, ev[i]);
+    if (ev[i] >= 0 && lane == __ffs(peers) - 1) cnt[warp][ev[i]] += __popc(peers);
+    __syncwarp();
+  }
+  __syncthreads();
+  // pass 2: thread e, expert e: the warps' exclusive prefix, the total, then
+  // the exclusive scan of the totals over the experts
+  const int e = threadIdx.x;
+  int32_t tot = 0;
+  if (e < E) {
+    for (int w = 0; w < 32; ++w) {
+      const int32_t t = cnt[w][e];
+      cnt[w][e] = tot;
+      tot += t;
+    }
+    counts[e] = tot;
+  }
+  int32_t v = tot;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int32_t u = __shfl_up_sync(0xffffffffu, v, o);
+    if (lane >= o) v += u;
+  }
+  if (lane == 31) warp_tot[warp] = v;
+  __syncthreads();
+  int32_t off = v - tot;
+  for (int i = 0; i < warp; ++i) off += warp_tot[i];
+  if (e < E) {
+    offsets[e] = off;
+    for (int w = 0; w < 32; ++w) cnt[w][e] += off;
+    if (e == E - 1) offsets[E] = off + tot;
+  }
+  __syncthreads();
+  // pass 3: ranks in slot order, as k_scatter
+  const unsigned lt = lanemask_lt();
+#pragma unroll
+  for (int i = 0; i < kSmallSortRounds; ++i) {
+    const int slot = beg + 32 * i + lane;
+    const int ee = ev[i];
+    const unsigned peers = __match_any_sync(0xffffffffu, ee);
+    if (slot < end) {
+      if (ee >= 0) {
+        const int32_t p = cnt[warp][ee] + __popc(peers & lt);
+        pos[slot] = p;
+        perm[p] = slot;
+      } else {
+        pos[slot] = -1;
+      }
+    }
+    __syncwarp();
+    if (ee >= 0 && lane == __ffs(peers) - 1) cnt[warp][ee] += __popc(peers);
+    __syncwarp();
+  }
+}
+
 // One warp per (token, chunk of 256 columns): each lane reads one 16-byte
 // vector of the token's row once and writes it to the K sorted positions
 // pos[t*K + k] (token-major, so x_e is read once, not K times).  The next
@@ -317,18 +416,24 @@ cudaError_t launch_dispatch(const int32_t* idx, int64_t N, int K, int E, const _
                             int32_t* pos, __nv_bfloat16* xs, int32_t* scratch, DeviceStatus* st,
                             cudaStream_t s) {
   const int64_t S = N * K;
-  const int CH = dispatch_chunk_len(S);
-  const int nchunks = dispatch_chunks(S);
-  const size_t smem = sizeof(int32_t) * (size_t)E * kWarps;
-  const unsigned blocks = (unsigned)((nchunks + kWarps - 1) / kWarps);
   cudaError_t e;
-  if ((e = launch_pdl(k_hist, dim3(blocks), dim3(32 * kWarps), smem, s, idx, S, E, CH, nchunks,
-                      scratch, st)) != cudaSuccess ||
-      (e = launch_pdl(k_scan, dim3((unsigned)((E + 31) / 32)), dim3(1024), 0, s, scratch,
-                      nchunks, E, counts)) != cudaSuccess ||
-      (e = launch_pdl(k_scatter, dim3(blocks), dim3(32 * kWarps), smem + sizeof(int32_t) * E, s,
-                      idx, S, E, CH, nchunks, scratch, counts, offsets, perm, pos)) != cudaSuccess)
-    return e;
+  if (S >= 1 && S <= kSmallSortMaxS && E <= kSmallSortMaxE) {
+    if ((e = launch_pdl(k_sort_small, dim3(1), dim3(1024), 0, s, idx, (int)S, E, counts, offsets,
+                        perm, pos, st)) != cudaSuccess)
+      return e;
+  } else {
+    const int CH = dispatch_chunk_len(S);
+    const int nchunks = dispatch_chunks(S);
+    const size_t smem = sizeof(int32_t) * (size_t)E * kWarps;
+    const unsigned blocks = (unsigned)((nchunks + kWarps - 1) / kWarps);
+    if ((e = launch_pdl(k_hist, dim3(blocks), dim3(32 * kWarps), smem, s, idx, S, E, CH, nchunks,
+                        scratch, st)) != cudaSuccess ||
+        (e = launch_pdl(k_scan, dim3((unsigned)((E + 31) / 32)), dim3(1024), 0, s, scratch,
+                        nchunks, E, counts)) != cudaSuccess ||
+        (e = launch_pdl(k_scatter, dim3(blocks), dim3(32 * kWarps), smem + sizeof(int32_t) * E, s,
+                        idx, S, E, CH, nchunks, scratch, counts, offsets, perm, pos)) != cudaSuccess)
+      return e;
+  }
   if (!xs) return cudaSuccess;
   int64_t gb = (N * ((d_e / 8 + 31) / 32) + 7) / 8;
   const int64_t cap = (int64_t)dev_info()->sm_count * 16;

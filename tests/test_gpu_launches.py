@@ -1,7 +1,8 @@
 """moe_launch_count counts the kernels the library actually launched: one per
-combine, four per dispatch that copies rows (histogram, scan, scatter,
-gather), three per sort-only dispatch, and the same number for every
-repetition of one moe_forward."""
+combine; for a dispatch that copies rows four (histogram, scan, scatter,
+gather), or two for a small one (the one-block sort, gather); three or one
+per sort-only dispatch; and the same number for every repetition of one
+moe_forward."""
 import numpy as np
 import pytest
 
@@ -11,10 +12,13 @@ from tests.gpu_util import dev_bf16, random_topk
 pytestmark = pytest.mark.gpu
 
 
-def test_launch_count_per_entry_point():
+@pytest.mark.parametrize("N,E,want", [(300, 40, (2, 1, 1)),      # 1200 slots: the one-block sort
+                                      (300, 300, (4, 3, 1)),     # more than 256 experts
+                                      (2000, 40, (4, 3, 1))])    # more than 4096 slots
+def test_launch_count_per_entry_point(N, E, want):
     import torch
     import moe_routing_expert_fp32_b200 as moe
-    N, K, E, d = 300, 4, 40, 256
+    K, d = 4, 256
     idx = torch.from_numpy(random_topk(N, K, E, np.random.default_rng(5))).cuda()
     x = dev_bf16(synth.host_normal_bf16(3, 1, (N, d), 1.0))
     moe.dispatch(idx, x, E)  # first call: kernel attributes set up
@@ -27,7 +31,7 @@ def test_launch_count_per_entry_point():
     moe.combine(xs, pos, w)
     n3 = moe.launch_count()
     torch.cuda.synchronize()
-    assert (n1 - n0, n2 - n1, n3 - n2) == (4, 3, 1)
+    assert (n1 - n0, n2 - n1, n3 - n2) == want
 
 
 def test_launch_count_of_forward_is_stable():
@@ -46,8 +50,9 @@ def test_launch_count_of_forward_is_stable():
                     ws=ws)
         deltas.append(moe.launch_count() - n0)
     torch.cuda.synchronize()
-    # route (gate GEMM + selection), dispatch (4), tile list, two expert GEMMs, combine
-    assert deltas[0] == deltas[1] == deltas[2] and 10 <= deltas[0] <= 13
+    # route (gate GEMM + selection), dispatch (one-block sort + gather at
+    # 256 slots), tile list, two expert GEMMs, combine
+    assert deltas[0] == deltas[1] == deltas[2] and 8 <= deltas[0] <= 13
 
 
 def test_launch_count_of_route_on_both_gate_paths():
