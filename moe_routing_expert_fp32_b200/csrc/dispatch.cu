@@ -14,9 +14,9 @@
 //   k_scatter one warp per chunk again: every block takes the exclusive scan
 //             of counts (block 0 stores it as offsets), then the slots are
 //             ranked in slot order within the chunk -> pos[slot], perm[pos].
-// Small sorts (at most 4096 slots and 256 experts, decode batches) run the
-// same three passes in one block instead: k_sort_small, 32 warps, warp w the
-// w-th of 32 contiguous chunks, its counts in shared memory.
+// Small sorts (at most 4096 slots, at most 1024 experts: decode batches) run
+// the same three passes in one block instead: k_sort_small, 32 warps, warp w
+// the w-th of 32 contiguous chunks, its counts in shared memory.
 // Then k_gather copies every token row once from HBM and writes it to its K
 // sorted positions (token-major, so x_e is read once, not K times).  Without
 // xs (the expert MLP gathering its rows itself) k_gather is skipped.
@@ -212,9 +212,10 @@ __global__ void __launch_bounds__(32 * kWarps) k_scatter(const int32_t* __restri
 // (pass 1), every expert's thread turns the warps' counts into their
 // exclusive prefix and the expert totals into offsets (pass 2), and each warp
 // ranks its slots in slot order (pass 3).  The ranks are those of the
-// three-kernel sort: pos and perm are unique for a stable sort.
+// three-kernel sort: pos and perm are unique for a stable sort.  The counts
+// are 16-bit (at most 4096 slots), 32 x E of them in dynamic shared memory.
 constexpr int kSmallSortMaxS = 4096;
-constexpr int kSmallSortMaxE = 256;
+constexpr int kSmallSortMaxE = 1024;
 constexpr int kSmallSortRounds = kSmallSortMaxS / (32 * 32);  // slots per lane
 
 __global__ void __launch_bounds__(1024) k_sort_small(const int32_t* __restrict__ idx, int S, int E,
@@ -225,13 +226,14 @@ __global__ void __launch_bounds__(1024) k_sort_small(const int32_t* __restrict__
                                                      DeviceStatus* st) {
   pdl_wait();
   pdl_trigger();
-  __shared__ int32_t cnt[32][kSmallSortMaxE];
+  extern __shared__ int16_t cnt_raw[];  // [32][E]
   __shared__ int32_t warp_tot[32];
+  auto cnt = [&](int w, int e) -> int16_t& { return cnt_raw[w * E + e]; };
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int CH = (S + 31) / 32;
   const int beg = warp * CH;
   const int end = beg + CH < S ? beg + CH : S;
-  for (int e = lane; e < E; e += 32) cnt[warp][e] = 0;
+  for (int e = lane; e < E; e += 32) cnt(warp, e) = 0;
   __syncwarp();
   // pass 1: this warp's counts; the slot indices stay in registers
   int ev[kSmallSortRounds];
@@ -248,7 +250,8 @@ __global__ void __launch_bounds__(1024) k_sort_small(const int32_t* __restrict__
 #pragma unroll
   for (int i = 0; i < kSmallSortRounds; ++i) {
     const unsigned peers = __match_any_sync(0xffffffffu, ev[i]);
-    if (ev[i] >= 0 && lane == __ffs(peers) - 1) cnt[warp][ev[i]] += __popc(peers);
+    if (ev[i] >= 0 && lane == __ffs(peers) - 1)
+      cnt(warp, ev[i]) = (int16_t)(cnt(warp, ev[i]) + __popc(peers));
     __syncwarp();
   }
   __syncthreads();
@@ -258,8 +261,8 @@ __global__ void __launch_bounds__(1024) k_sort_small(const int32_t* __restrict__
   int32_t tot = 0;
   if (e < E) {
     for (int w = 0; w < 32; ++w) {
-      const int32_t t = cnt[w][e];
-      cnt[w][e] = tot;
+      const int32_t t = cnt(w, e);
+      cnt(w, e) = (int16_t)tot;
       tot += t;
     }
     counts[e] = tot;
@@ -276,7 +279,7 @@ __global__ void __launch_bounds__(1024) k_sort_small(const int32_t* __restrict__
   for (int i = 0; i < warp; ++i) off += warp_tot[i];
   if (e < E) {
     offsets[e] = off;
-    for (int w = 0; w < 32; ++w) cnt[w][e] += off;
+    for (int w = 0; w < 32; ++w) cnt(w, e) = (int16_t)(cnt(w, e) + off);
     if (e == E - 1) offsets[E] = off + tot;
   }
   __syncthreads();
@@ -289,7 +292,7 @@ __global__ void __launch_bounds__(1024) k_sort_small(const int32_t* __restrict__
     const unsigned peers = __match_any_sync(0xffffffffu, ee);
     if (slot < end) {
       if (ee >= 0) {
-        const int32_t p = cnt[warp][ee] + __popc(peers & lt);
+        const int32_t p = cnt(warp, ee) + __popc(peers & lt);
         pos[slot] = p;
         perm[p] = slot;
       } else {
@@ -297,7 +300,8 @@ __global__ void __launch_bounds__(1024) k_sort_small(const int32_t* __restrict__
       }
     }
     __syncwarp();
-    if (ee >= 0 && lane == __ffs(peers) - 1) cnt[warp][ee] += __popc(peers);
+    if (ee >= 0 && lane == __ffs(peers) - 1)
+      cnt(warp, ee) = (int16_t)(cnt(warp, ee) + __popc(peers));
     __syncwarp();
   }
 }
@@ -418,8 +422,16 @@ cudaError_t launch_dispatch(const int32_t* idx, int64_t N, int K, int E, const _
   const int64_t S = N * K;
   cudaError_t e;
   if (S >= 1 && S <= kSmallSortMaxS && E <= kSmallSortMaxE) {
-    if ((e = launch_pdl(k_sort_small, dim3(1), dim3(1024), 0, s, idx, (int)S, E, counts, offsets,
-                        perm, pos, st)) != cudaSuccess)
+    static std::once_flag once[kMaxDevices];
+    static cudaError_t set_up[kMaxDevices];
+    if ((e = once_per_device(once, set_up, [](int) {
+           return cudaFuncSetAttribute(k_sort_small, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)(sizeof(int16_t) * 32 * kSmallSortMaxE));
+         })) != cudaSuccess)
+      return e;
+    const size_t smem = sizeof(int16_t) * 32 * (size_t)E;
+    if ((e = launch_pdl(k_sort_small, dim3(1), dim3(1024), smem, s, idx, (int)S, E, counts,
+                        offsets, perm, pos, st)) != cudaSuccess)
       return e;
   } else {
     const int CH = dispatch_chunk_len(S);

@@ -13,7 +13,7 @@ pytestmark = pytest.mark.gpu
 
 
 @pytest.mark.parametrize("N,E,want", [(300, 40, (2, 1, 1)),      # 1200 slots: the one-block sort
-                                      (300, 300, (4, 3, 1)),     # more than 256 experts
+                                      (300, 1000, (2, 1, 1)),    # up to 1024 experts: the same
                                       (2000, 40, (4, 3, 1))])    # more than 4096 slots
 def test_launch_count_per_entry_point(N, E, want):
     import torch

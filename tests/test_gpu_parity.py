@@ -196,11 +196,11 @@ def test_dispatch(moe, name):
 
 # (40000, 8, 64): 320 000 slots make 313 chunks of 1024, more than the 256
 # that the scan keeps in registers, so its looping form runs.  Up to 4096
-# slots and 256 experts the one-block sort runs: (1024, 4, 256) is its
-# largest case, (4097, 1, 256) and (1, 8, 384) just outside it
+# slots the one-block sort runs: (1024, 4, 1024) is its largest case,
+# (4097, 1, 256) just outside it
 @pytest.mark.parametrize("N,K,E", [(1, 8, 384), (1000, 1, 16), (333, 3, 7), (5000, 16, 1024),
-                                   (40000, 8, 64), (1024, 4, 256), (4097, 1, 256), (512, 1, 1),
-                                   (1, 1, 1)])
+                                   (40000, 8, 64), (1024, 4, 256), (1024, 4, 1024),
+                                   (4097, 1, 256), (512, 1, 1), (1, 1, 1)])
 def test_dispatch_edge_shapes(moe, N, K, E):
     rng = np.random.default_rng(N + K + E)
     _dispatch_case(moe, N, K, E, 128, random_topk(N, K, E, rng, skew=1.5))
